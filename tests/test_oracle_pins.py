@@ -1,0 +1,431 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: values the
+pages print (fixtures under tests/golden/, each with its citation), closed
+forms, invariants, library routines that compute the same special case
+(torch fp64 CPU ops, numpy), brute force on tiny inputs, and finite
+differences of the oracle's own loss.  No GPU is needed.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from deep_cnn_image_b200 import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+# ---------------------------------------------------------------- Philox
+def test_philox_known_answers():
+    for row in _golden("philox4x32_10_kat.txt"):
+        ctr = [int(v, 16) for v in row[0:4]]
+        key = [int(v, 16) for v in row[4:6]]
+        want = [int(v, 16) for v in row[6:10]]
+        assert oracle.philox4x32_10(ctr, key) == want
+
+
+def test_dropout_keep_rate_and_independence():
+    # [S] 3.4 "Dropout": each hidden output is zeroed with probability 0.5.
+    m = oracle.dropout_mask(1234, 6, 0, 128, 4096).astype(np.float64)
+    n = m.size
+    rate = m.mean()
+    assert abs(rate - 0.5) < 4 * math.sqrt(0.25 / n)
+    # different layer / step / seed give different (uncorrelated) masks
+    for other in (oracle.dropout_mask(1234, 7, 0, 128, 4096), oracle.dropout_mask(1234, 6, 1, 128, 4096),
+                  oracle.dropout_mask(99, 6, 0, 128, 4096)):
+        agree = (m == other).mean()
+        assert abs(agree - 0.5) < 4 * math.sqrt(0.25 / n)
+    # per-unit rates over the batch are binomial(128, 1/2)
+    col = m.mean(axis=0)
+    assert abs(col.std() - math.sqrt(0.25 / 128)) < 0.01
+
+
+# ---------------------------------------------------------------- counts
+def test_shapes_and_counts_match_the_pages():
+    g = {r[0]: int(r[1]) for r in _golden("alexnet_counts.txt")}
+    net = oracle.alexnet(grouped=True)
+    ms = oracle.map_sizes(net)
+    assert ms[0][1] == g["conv1_out_side"] and ms[0][2] == g["pool1_out_side"]
+    assert ms[1][2] == g["pool2_out_side"] and ms[4][2] == g["pool5_out_side"]
+    assert [m[1] for m in ms] == [55, 27, 13, 13, 13]
+    assert ms[4][2] ** 2 * 256 == g["fc6_inputs"]
+    neurons = oracle.neuron_counts(net)
+    assert neurons[1:] == [g["neurons_conv2"], g["neurons_conv3"], g["neurons_conv4"],
+                           g["neurons_conv5"], g["neurons_fc6"], g["neurons_fc7"], g["neurons_fc8"]]
+    # the printed first-layer count is garbled on the pages; the stride math gives 55*55*96
+    assert neurons[0] == 55 * 55 * 96
+    assert abs(sum(neurons) - g["neurons_total_approx"]) / g["neurons_total_approx"] < 0.02
+    n_params = oracle.param_count(net)
+    assert n_params == 60965224
+    assert abs(n_params - g["params_total_approx"]) / g["params_total_approx"] < 0.02
+    lay = oracle.param_layout(net)
+    for l, key in ((5, "fc6_params_approx"), (6, "fc7_params_approx"), (7, "fc8_params_approx")):
+        assert abs(lay[l][1] - g[key]) / g[key] < 0.01
+    macs = oracle.forward_macs(net)
+    assert macs == 724406816
+    assert 0.5 * g["forward_macs_approx"] < macs < 1.5 * g["forward_macs_approx"]
+    assert oracle.param_count(oracle.alexnet(grouped=False)) == 62378344
+    assert synthetic.param_count(True) == n_params and synthetic.param_count(False) == 62378344
+
+
+# ---------------------------------------------------------------- conv
+def _brute_conv(x, w, b, stride, pad, groups):
+    B, H, W, C = x.shape
+    Co, K = w.shape[0], w.shape[1]
+    Cg, Og = C // groups, Co // groups
+    Ho, Wo = (H + 2 * pad - K) // stride + 1, (W + 2 * pad - K) // stride + 1
+    y = np.zeros((B, Ho, Wo, Co))
+    for n in range(B):
+        for i in range(Ho):
+            for j in range(Wo):
+                for o in range(Co):
+                    s = b[o]
+                    g = o // Og
+                    for p in range(K):
+                        for q in range(K):
+                            ih, iw = i * stride - pad + p, j * stride - pad + q
+                            if 0 <= ih < H and 0 <= iw < W:
+                                for c in range(Cg):
+                                    s += x[n, ih, iw, g * Cg + c] * w[o, p, q, c]
+                    y[n, i, j, o] = s
+    return y
+
+
+@pytest.mark.parametrize("stride,pad,groups,K", [(1, 1, 1, 3), (1, 2, 2, 5), (4, 0, 1, 5), (2, 1, 2, 3)])
+def test_conv_forward_brute_force(stride, pad, groups, K):
+    r = np.random.default_rng(7)
+    x = r.standard_normal((2, 9, 9, 4))
+    w = r.standard_normal((6, K, K, 4 // groups))
+    b = r.standard_normal(6)
+    want = _brute_conv(x, w, b, stride, pad, groups)
+    got = oracle.conv_fwd(x, w, b, stride, pad, groups)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("stride,pad,groups,K", [(1, 1, 1, 3), (1, 2, 2, 5), (4, 0, 1, 11), (1, 1, 2, 3)])
+def test_conv_forward_backward_vs_torch(stride, pad, groups, K):
+    r = np.random.default_rng(11)
+    H = 23 if K == 11 else 10
+    x = r.standard_normal((3, H, H, 8))
+    w = r.standard_normal((12, K, K, 8 // groups))
+    b = r.standard_normal(12)
+    xt = torch.tensor(x.transpose(0, 3, 1, 2), requires_grad=True)
+    wt = torch.tensor(w.transpose(0, 3, 1, 2), requires_grad=True)
+    bt = torch.tensor(b, requires_grad=True)
+    yt = F.conv2d(xt, wt, bt, stride=stride, padding=pad, groups=groups)
+    y = oracle.conv_fwd(x, w, b, stride, pad, groups)
+    np.testing.assert_allclose(y, yt.detach().numpy().transpose(0, 2, 3, 1), rtol=1e-10, atol=1e-10)
+    dy = r.standard_normal(y.shape)
+    yt.backward(torch.tensor(dy.transpose(0, 3, 1, 2)))
+    dx, dw, db = oracle.conv_bwd(x, w, dy, stride, pad, groups)
+    np.testing.assert_allclose(dx, xt.grad.numpy().transpose(0, 2, 3, 1), rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(dw, wt.grad.numpy().transpose(0, 2, 3, 1), rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(db, bt.grad.numpy(), rtol=1e-10, atol=1e-10)
+    # the sampled forms compute the same sums
+    idx = r.choice(y.size, 50, replace=False)
+    np.testing.assert_allclose(oracle.conv_fwd_sampled(x, w, b, stride, pad, groups, idx), y.ravel()[idx],
+                               rtol=1e-12, atol=1e-12)
+    widx = r.choice(w.size, 50, replace=False)
+    np.testing.assert_allclose(oracle.conv_wgrad_sampled(x, dy, 12, K, stride, pad, groups, widx),
+                               dw.ravel()[widx], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- LRN
+def test_lrn_isolated_channel_closed_form():
+    # [S] 3.4 "Local Response Normalization": a kernel that fires alone in its
+    # neighbourhood is divided by (k + alpha a^2)^beta ~ k^beta.
+    a = np.zeros((1, 96))
+    a[0, 40] = 3.0
+    b = oracle.lrn_fwd(a)
+    assert b[0, 40] == pytest.approx(3.0 / (2.0 + 1e-4 * 9.0) ** 0.75, rel=1e-14)
+    assert np.count_nonzero(b) == 1
+    small = oracle.lrn_fwd(np.full((1, 8), 1e-6))
+    np.testing.assert_allclose(small, 1e-6 / 2.0 ** 0.75, rtol=1e-12)
+
+
+def test_lrn_forward_backward_vs_torch():
+    # torch's local_response_norm divides alpha by the window size n; the
+    # pages' formula does not, so the library call gets alpha * n.
+    r = np.random.default_rng(3)
+    a = np.abs(r.standard_normal((2, 5, 5, 96))) * 30.0
+    at = torch.tensor(a.transpose(0, 3, 1, 2), requires_grad=True)
+    bt = F.local_response_norm(at, size=5, alpha=5 * 1e-4, beta=0.75, k=2.0)
+    b = oracle.lrn_fwd(a)
+    np.testing.assert_allclose(b, bt.detach().numpy().transpose(0, 2, 3, 1), rtol=1e-12)
+    g = r.standard_normal(a.shape)
+    bt.backward(torch.tensor(g.transpose(0, 3, 1, 2)))
+    da = oracle.lrn_bwd(a, g)
+    np.testing.assert_allclose(da, at.grad.numpy().transpose(0, 2, 3, 1), rtol=1e-10, atol=1e-12)
+
+
+def test_lrn_window_edges():
+    # the window is clipped to [0, N-1]: channel 0 sees channels 0..2 only
+    a = np.arange(1.0, 9.0).reshape(1, 8) * 10.0
+    b = oracle.lrn_fwd(a)
+    s0 = 2.0 + 1e-4 * (10.0 ** 2 + 20.0 ** 2 + 30.0 ** 2)
+    s7 = 2.0 + 1e-4 * (60.0 ** 2 + 70.0 ** 2 + 80.0 ** 2)
+    assert b[0, 0] == pytest.approx(10.0 / s0 ** 0.75, rel=1e-14)
+    assert b[0, 7] == pytest.approx(80.0 / s7 ** 0.75, rel=1e-14)
+
+
+# ---------------------------------------------------------------- pooling
+def test_maxpool_invariants_and_torch():
+    r = np.random.default_rng(5)
+    x = r.standard_normal((2, 55, 55, 16))
+    y, am = oracle.maxpool_fwd(x)
+    assert y.shape == (2, 27, 27, 16)
+    yt = F.max_pool2d(torch.tensor(x.transpose(0, 3, 1, 2)), 3, 2)
+    np.testing.assert_array_equal(y, yt.numpy().transpose(0, 2, 3, 1))
+    # the argmax points at the maximum, which is >= every window element
+    for (b, i, j, c) in [(0, 0, 0, 0), (1, 26, 26, 15), (0, 13, 7, 3), (1, 4, 20, 9)]:
+        win = x[b, 2 * i:2 * i + 3, 2 * j:2 * j + 3, c]
+        a = am[b, i, j, c]
+        assert win[a // 3, a % 3] == y[b, i, j, c] == win.max()
+
+
+def test_maxpool_ties_pick_first_in_row_major_order():
+    x = np.zeros((1, 3, 3, 2))
+    x[0, 0, 2, 0] = 5.0
+    x[0, 2, 1, 0] = 5.0
+    y, am = oracle.maxpool_fwd(x)
+    assert am[0, 0, 0, 0] == 2 and y[0, 0, 0, 0] == 5.0
+    assert am[0, 0, 0, 1] == 0  # all zeros: the first element
+
+
+def test_maxpool_backward_vs_torch():
+    r = np.random.default_rng(6)
+    x = r.standard_normal((2, 13, 13, 8))
+    y, am = oracle.maxpool_fwd(x)
+    g = r.standard_normal(y.shape)
+    xt = torch.tensor(x.transpose(0, 3, 1, 2), requires_grad=True)
+    F.max_pool2d(xt, 3, 2).backward(torch.tensor(g.transpose(0, 3, 1, 2)))
+    dx = oracle.maxpool_bwd(g, am, 13, 13)
+    np.testing.assert_allclose(dx, xt.grad.numpy().transpose(0, 2, 3, 1), rtol=1e-14, atol=1e-14)
+
+
+def test_nonoverlapping_pool_shapes():
+    # [S] 3.4 "Overlapping Pooling": z = 2, s = 2 halves 55 to 27 as well
+    y, _ = oracle.maxpool_fwd(np.zeros((1, 55, 55, 1)), z=2, s=2)
+    assert y.shape[1] == 27
+
+
+# ---------------------------------------------------------------- FC, softmax
+def test_fc_vs_numpy():
+    r = np.random.default_rng(8)
+    x, w, b = r.standard_normal((5, 33)), r.standard_normal((7, 33)), r.standard_normal(7)
+    np.testing.assert_allclose(oracle.fc_fwd(x, w, b), x @ w.T + b, rtol=1e-12)
+    dz = r.standard_normal((5, 7))
+    dx, dw, db = oracle.fc_bwd(x, w, dz)
+    np.testing.assert_allclose(dx, dz @ w, rtol=1e-12)
+    np.testing.assert_allclose(dw, dz.T @ x, rtol=1e-12)
+    np.testing.assert_allclose(db, dz.sum(0), rtol=1e-12)
+
+
+def test_softmax_worked_example_ratio():
+    rows = {r[0]: r[1:] for r in _golden("softmax_worked_example.txt")}
+    ia, za = int(rows["index_a"][0]), float(rows["index_a"][1])
+    ib, zb = int(rows["index_b"][0]), float(rows["index_b"][1])
+    ratio = float(rows["ratio_exp_0p8"][0])
+    r = np.random.default_rng(9)
+    z = r.uniform(0.0, 2.0, (3, 1000))
+    z[:, ia], z[:, ib] = za, zb
+    _, p, _ = oracle.softmax_ce(z)
+    np.testing.assert_allclose(p[:, ia] / p[:, ib], ratio, rtol=1e-12)
+    np.testing.assert_allclose(p.sum(1), 1.0, rtol=1e-14)
+    assert (p.argmax(1) == ia).all()
+
+
+def test_cross_entropy_uniform_and_torch():
+    loss, p, _ = oracle.softmax_ce(np.full((4, 1000), 0.37), np.array([0, 5, 999, 3]))
+    assert loss == pytest.approx(math.log(1000.0), rel=1e-14)
+    r = np.random.default_rng(10)
+    z = r.standard_normal((6, 1000)) * 3
+    y = r.integers(0, 1000, 6)
+    zt = torch.tensor(z, requires_grad=True)
+    lt = F.cross_entropy(zt, torch.tensor(y))
+    lt.backward()
+    loss, p, dz = oracle.softmax_ce(z, y)
+    assert loss == pytest.approx(lt.item(), rel=1e-12)
+    np.testing.assert_allclose(dz, zt.grad.numpy(), rtol=1e-10, atol=1e-15)
+
+
+# ---------------------------------------------------------------- SGD
+def test_sgd_hand_worked_steps():
+    w, v = np.array([1.0]), np.array([0.0])
+    for row in _golden("sgd_three_steps.txt"):
+        g = np.array([float(row[1])])
+        w, v = oracle.sgd(w, v, g, 0.01)
+        assert w[0] == pytest.approx(float(row[2]), rel=1e-13, abs=1e-15)
+        assert v[0] == pytest.approx(float(row[3]), rel=1e-13, abs=1e-15)
+
+
+def test_sgd_constant_gradient_closed_form():
+    # With a constant gradient the update is the affine map
+    # [w; v] <- A [w; v] + c, A = [[1 - wd lr, m], [-wd lr, m]], c = [-lr g, -lr g];
+    # n steps equal the matrix power form.
+    lr, m, wd, g = 0.05, 0.9, 5e-4, 0.3
+    A = np.array([[1 - wd * lr, m], [-wd * lr, m]])
+    c = np.array([-lr * g, -lr * g])
+    s = np.array([0.7, 0.0])
+    w, v = np.array([0.7]), np.array([0.0])
+    n = 40
+    for _ in range(n):
+        w, v = oracle.sgd(w, v, np.array([g]), lr, m, wd)
+    An = np.linalg.matrix_power(A, n)
+    want = An @ s + np.linalg.solve(np.eye(2) - A, (np.eye(2) - An) @ c)
+    np.testing.assert_allclose([w[0], v[0]], want, rtol=1e-11)
+
+
+# ---------------------------------------------------------------- gradients
+def test_train_step_gradients_finite_difference():
+    """fp64 central differences of the oracle's own loss on the shrunken net
+    (same op sequence, fixed dropout masks) pin every backward formula."""
+    net = oracle.small_net()
+    n = oracle.param_count(net)
+    r = np.random.default_rng(12)
+    params = r.standard_normal(n) * 0.2
+    lay = oracle.param_layout(net)
+    for (wo, wl, bo, bl) in lay:
+        params[bo:bo + bl] = r.uniform(0.05, 0.3, bl)
+    x = r.standard_normal((3, 67, 67, 3))
+    y = np.array([1, 7, 3], np.int32)
+    seed, step = 77, 5
+    loss, _, _, grads, _ = oracle.train_step(net, params, np.zeros(n), x, y, lr=0.0, seed=seed,
+                                             step=step)
+    assert loss == pytest.approx(oracle.loss(net, params, x, y, seed, step), rel=1e-14)
+    h = 1e-6
+    bad = 0
+    checked = 0
+    for (wo, wl, bo, bl) in lay:
+        for idx in list(r.choice(wl, min(12, wl), replace=False) + wo) + list(
+                r.choice(bl, min(4, bl), replace=False) + bo):
+            p1 = params.copy()
+            p1[idx] += h
+            p2 = params.copy()
+            p2[idx] -= h
+            fd = (oracle.loss(net, p1, x, y, seed, step) - oracle.loss(net, p2, x, y, seed, step)) / (2 * h)
+            checked += 1
+            if abs(fd - grads[idx]) > 1e-6 * max(1.0, abs(fd)) + 1e-8:
+                bad += 1
+    # a component may straddle a ReLU kink or a pooling switch; allow none to a couple
+    assert bad <= 2, (bad, checked)
+
+
+def test_dropout_gradient_follows_mask():
+    """Units dropped in FC6 get exactly zero gradient in FC6's weights' rows
+    for every image where they are dropped: with batch 1 the whole row is 0."""
+    net = oracle.small_net()
+    n = oracle.param_count(net)
+    r = np.random.default_rng(13)
+    params = r.standard_normal(n) * 0.2
+    lay = oracle.param_layout(net)
+    for (wo, wl, bo, bl) in lay:
+        params[bo:bo + bl] = 0.5
+    x = r.standard_normal((1, 67, 67, 3))
+    _, _, _, grads, _ = oracle.train_step(net, params, np.zeros(n), x, np.array([2], np.int32),
+                                          lr=0.0, seed=5, step=3)
+    keep = oracle.dropout_mask(5, 6, 3, 1, 16)[0]
+    wo, wl, bo, bl = lay[5]
+    gw = grads[wo:wo + wl].reshape(16, -1)
+    for j in range(16):
+        if not keep[j]:
+            assert np.all(gw[j] == 0.0) and grads[bo + j] == 0.0
+    assert keep.sum() not in (0, 16)
+
+
+def test_inference_scales_by_half():
+    """[S] 3.4 "Dropout", test time: FC6/FC7 outputs multiplied by 0.5; with
+    dropout disabled the same net (no scaling) differs exactly by that."""
+    net = oracle.small_net()
+    n = oracle.param_count(net)
+    r = np.random.default_rng(14)
+    params = r.standard_normal(n) * 0.2
+    x = r.standard_normal((2, 67, 67, 3))
+    f6 = oracle.forward_probe(net, params, x, oracle.PROBE_FC + 0, mode=1)
+    net.dropout_on = 0
+    f6_nodrop = oracle.forward_probe(net, params, x, oracle.PROBE_FC + 0, mode=1)
+    np.testing.assert_allclose(f6, 0.5 * f6_nodrop, rtol=1e-15)
+
+
+# ---------------------------------------------------------------- augmentation
+def test_augmentation_draw_support_is_2048_combinations():
+    # [P2] "Training/regularization interactions": 2048 position/mirror
+    # combinations per 256x256 image; offsets 0..31 on each axis x 2 mirrors.
+    seen = set()
+    alphas = []
+    for img in range(20000):
+        oy, ox, fl, a = oracle.aug_draws(42, img, 0)
+        assert 0 <= oy < 32 and 0 <= ox < 32 and fl in (0, 1)
+        seen.add((oy, ox, fl))
+        alphas.append(a)
+    assert len(seen) == 2048
+    al = np.array(alphas)
+    # [S] 3.4 "Data Augmentation" Form 2: alpha_i ~ N(0, 0.1^2)
+    assert np.all(np.abs(al.mean(0)) < 4 * 0.1 / math.sqrt(len(al)))
+    np.testing.assert_allclose(al.std(0), 0.1, rtol=0.03)
+
+
+def test_augmentation_crop_and_constant_colour_shift():
+    src = synthetic.source_images(1, 3)
+    mean = synthetic.mean_image(src).astype(np.float64)
+    vec, val = synthetic.pca(2)
+    out = oracle.augment(src, mean, vec, val, seed=9, step=4)
+    assert out.shape == (3, 227, 227, 3)
+    assert np.all(out[:, 224:, :, :] == 0) and np.all(out[:, :, 224:, :] == 0)
+    for b in range(3):
+        oy, ox, fl, a = oracle.aug_draws(9, b, 4)
+        crop = src[b, oy:oy + 224, ox:ox + 224].astype(np.float64) - mean[oy:oy + 224, ox:ox + 224]
+        if fl:
+            crop = crop[:, ::-1]
+        shift = out[b, :224, :224] - crop
+        # one colour offset for every pixel of the image, along the PCA basis
+        np.testing.assert_allclose(shift, np.broadcast_to(shift[0, 0], shift.shape), atol=1e-9)
+        coeff = np.linalg.solve(vec.astype(np.float64), shift[0, 0])
+        np.testing.assert_allclose(coeff, a * val.astype(np.float64), rtol=1e-9, atol=1e-12)
+
+
+def test_tencrop_patches_and_dominant_class():
+    src = synthetic.source_images(3, 2)
+    mean = synthetic.mean_image(src).astype(np.float64)
+    crops = oracle.tencrop_inputs(src, mean).reshape(2, 10, 227, 227, 3)
+    s0 = src[1].astype(np.float64) - mean
+    np.testing.assert_array_equal(crops[1, 0, :224, :224], s0[:224, :224])          # top-left
+    np.testing.assert_array_equal(crops[1, 1, :224, :224], s0[:224, 32:])           # top-right
+    np.testing.assert_array_equal(crops[1, 3, :224, :224], s0[32:, 32:])            # bottom-right
+    np.testing.assert_array_equal(crops[1, 4, :224, :224], s0[16:240, 16:240])      # centre
+    np.testing.assert_array_equal(crops[1, 5, :224, :224], s0[:224, :224][:, ::-1])  # reflected TL
+    # a network whose FC8 bias strongly favours class 417 puts it first everywhere
+    net = oracle.alexnet()
+    n = oracle.param_count(net)
+    params = np.zeros(n)
+    lay = oracle.param_layout(net)
+    bo = lay[7][2]
+    params[bo + 417] = 10.0
+    params[bo + 3] = 9.0
+    probs, top5 = oracle.tencrop(net, params, src[:1], mean)
+    assert top5[0, 0] == 417 and top5[0, 1] == 3
+    # the remaining classes tie exactly: ties go to the lower index
+    assert list(top5[0, 2:]) == [0, 1, 2]
+    np.testing.assert_allclose(probs.sum(1), 1.0, rtol=1e-12)
+
+
+def test_topk_against_numpy_sort():
+    r = np.random.default_rng(15)
+    p = r.random((5, 1000))
+    idx = oracle.topk(p, 5)
+    np.testing.assert_array_equal(idx, np.argsort(-p, axis=1, kind="stable")[:, :5])
