@@ -1,0 +1,305 @@
+#!/usr/bin/env python
+"""Benchmark: one AlexNet bf16 training step (forward, backward, SGD update)
+of the grouped network on a batch of 128 synthetic 227x227x3 images per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  For N > 1 launch one process per GPU with
+torch.distributed.run; each rank trains its own replica on its own batch
+(no gradient exchange is built), so the scaling is weak and `value` is the
+images of all ranks divided by the slowest rank's device time.
+
+Timing: W untimed steps; then K steps, each bracketed by CUDA events on the
+library's stream, with a 256 MB buffer written between steps (outside the
+events) so no step starts with the previous step's data in the 126 MB L2;
+barrier + synchronize on both sides; max over ranks.  `e2e` times the same
+steps through the public call with the batch copied from pinned host memory
+and the loss copied back inside the timed region.
+
+`--impl reference` times the CPU oracle (the plain fp64 C implementation
+under oracle/) as it stands on the host cores: each step is a training step
+on one image of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "images/sec, AlexNet bf16 train step, batch 128, 1×B200; % of bf16 tensor roofline"
+UNIT = "images/s"
+WORKLOAD = "AlexNet (grouped conv2/4/5) bf16 training step: forward + backward + SGD-momentum, " \
+           "227x227x3 NHWC inputs ~N(0,1), labels U[0,1000)"
+# Per-image FLOPs of one training step (2 x multiply-adds of the forward
+# convolutions and FC layers, their data gradients except conv1's, and their
+# weight gradients), from the layer shapes of the network.
+FWD_MACS_PER_IMAGE = 724406816
+CONV1_MACS_PER_IMAGE = 55 * 55 * 96 * 363
+
+
+def step_flops_per_image():
+    return 2.0 * (3 * FWD_MACS_PER_IMAGE - CONV1_MACS_PER_IMAGE)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_baseline_oracle(images_per_step, steps):
+    """Time the oracle's training step (fp64 C loops, OpenMP over the batch)
+    on the host cores; returns (images/s, cores, seconds)."""
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    os.environ["OMP_NUM_THREADS"] = str(cores)
+    import numpy as np
+
+    import oracle
+    from deep_cnn_image_b200 import synthetic
+    net = oracle.alexnet(grouped=True)
+    n = oracle.param_count(net)
+    params = synthetic.params(1).astype(np.float64)
+    vel = np.zeros(n)
+    x = synthetic.images(2, images_per_step).astype(np.float64)
+    y = synthetic.labels(3, images_per_step)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        _, params, vel, _, _ = oracle.train_step(net, params, vel, x, y, lr=0.01, seed=1, step=i)
+    dt = time.perf_counter() - t0
+    return images_per_step * steps / dt, cores, dt
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    # the oracle trains on one image per step: the same network, input shape
+    # and update; warm-up steps are run and not timed
+    cpu_baseline_oracle(1, args.warmup) if args.warmup > 0 else None
+    value, cores, dt = cpu_baseline_oracle(1, args.steps)
+    sample = "%d training steps on 1 image each (the batch-128 workload's per-image work)" % args.steps
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 1, "images_per_step": 1},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    from deep_cnn_image_b200 import alexnet as ax
+    from deep_cnn_image_b200 import synthetic
+
+    B = args.batch
+    net = ax.AlexNet(batch_max=B, seed=1234 + rank)
+    x_host, _ = synthetic.to_bf16(synthetic.images(100 + rank, B))
+    y_np = synthetic.labels(200 + rank, B)
+    x = x_host.cuda()
+    y = torch.from_numpy(y_np).cuda()
+    loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        net.train_step(x, y, B, 0.01, loss)
+    barrier()
+
+    # ---- device-timed steps (inputs resident in HBM)
+    net.stats_enable(True)
+    sampler = ClockSampler(local) if rank == 0 else None
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    t_wall = time.perf_counter()
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        net.train_step(x, y, B, 0.01, loss)
+        e1.record(stream)
+    barrier()
+    t_wall = time.perf_counter() - t_wall
+    clocks = sampler.stop() if sampler else None
+    stats = net.stats_read()
+    net.stats_enable(False)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
+    assert net.get_status() == ax.OK, "device status after the timed steps"
+    loss_val = float(loss.item())
+
+    # ---- end to end through the public call, host buffers
+    x_pin = x_host.pin_memory()
+    y_pin = torch.from_numpy(y_np).pin_memory()
+    loss_pin = torch.zeros(1, dtype=torch.float32).pin_memory()
+    evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    barrier()
+    for e0, e1 in evs2:
+        flush.zero_()
+        e0.record(stream)
+        x.copy_(x_pin, non_blocking=True)
+        y.copy_(y_pin, non_blocking=True)
+        net.train_step(x, y, B, 0.01, loss)
+        loss_pin.copy_(loss, non_blocking=True)
+        e1.record(stream)
+    barrier()
+    ms_e2e = sum(e0.elapsed_time(e1) for e0, e1 in evs2)
+
+    t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max, ms_e2e_max = t.tolist()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks = load_peaks()
+    images = world * B * args.steps
+    value = images / (ms_max / 1e3)
+    step_ms = ms_max / args.steps
+    step_tflops = step_flops_per_image() * B / (step_ms / 1e3) / 1e12
+    gemm_tflops = stats["gemm_flops"] / (stats["gemm_ms"] / 1e3) / 1e12 if stats["gemm_ms"] else None
+    peak = peaks["bf16_tflops_sustained"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": world * B, "batch_per_gpu": B,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "256 MB buffer written between timed steps"},
+        "roofline": {
+            "kernel": "tcgen05 GEMM (all conv/FC forward, data- and weight-gradient launches)",
+            "bound": "tensor", "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s",
+            "frac": gemm_tflops / peak if gemm_tflops else None, "traffic": None,
+            "peak_source": peaks["source"] + " bf16_tflops_sustained",
+            "gemm_launches_per_step": stats["gemm_launches"] / args.steps,
+            "gemm_ms_per_step": stats["gemm_ms"] / args.steps,
+        },
+        "step_roofline": {"achieved": step_tflops, "peak": peak, "unit": "TFLOP/s",
+                          "frac": step_tflops / peak,
+                          "flops_per_image": step_flops_per_image()},
+        "e2e": {"value": images / (ms_e2e_max / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": x_pin.numel() * 2 + y_pin.numel() * 4,
+                "d2h_bytes_per_step": 4},
+        "gpu_launches": stats["launches"],
+        "clocks": clocks,
+        "loss_last": loss_val,
+        "wall_s_timed": t_wall,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, cores, dt = cpu_baseline_oracle(args.cpu_images, 1)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": "one training step of the oracle on %d images "
+                                          "(fp64 C loops), %.1f s" % (args.cpu_images, dt)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--batch", type=int, default=128)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-images", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,286 @@
+"""ctypes binding of libalexnet.so (include/alexnet.h, include/alexnet_ops.h).
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels.  Tensors are torch tensors (their data pointers are passed); streams
+default to torch's current CUDA stream.  Importing this module loads the
+library and raises if it is missing: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_float, c_int, c_int64, c_size_t, c_uint32, c_uint64, c_void_p
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libalexnet.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_LABEL_RANGE = range(6)
+FP32, BF16 = 0, 1
+TRAIN, INFERENCE = 0, 1
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT",
+                5: "LABEL_RANGE"}
+
+
+class Config(ctypes.Structure):
+    """alexnet_config."""
+    _fields_ = [
+        ("batch_max", c_int), ("dtype", c_int), ("grouped", c_int), ("seed", c_uint64),
+        ("momentum", c_float), ("weight_decay", c_float), ("dropout_p", c_float),
+        ("lrn_k", c_float), ("lrn_alpha", c_float), ("lrn_beta", c_float), ("lrn_n", c_int),
+        ("lrn_on", c_int), ("pool_size", c_int), ("dropout_on", c_int), ("keep_grads", c_int),
+    ]
+
+
+class Stats(ctypes.Structure):
+    """alexnet_stats."""
+    _fields_ = [("launches", ctypes.c_int64), ("gemm_launches", ctypes.c_int64),
+                ("gemm_flops", ctypes.c_double), ("gemm_ms", ctypes.c_double)]
+
+
+class AlexNetError(RuntimeError):
+    def __init__(self, status, msg=""):
+        super().__init__("alexnet status %s: %s" % (STATUS_NAMES.get(status, status), msg))
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libalexnet.so is not built (python -m deep_cnn_image_b200.build)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, st, i, sz = c_void_p, c_int, c_int, c_size_t
+    cfgp = POINTER(Config)
+    sig = {
+        "alexnet_default_config": (None, [cfgp]),
+        "alexnet_param_count": (c_int64, [cfgp]),
+        "alexnet_workspace_bytes": (sz, [cfgp]),
+        "alexnet_create": (st, [cfgp, vp, sz, vp, POINTER(vp)]),
+        "alexnet_forward": (st, [vp, vp, i, i, vp, vp, vp]),
+        "alexnet_train_step": (st, [vp, vp, vp, i, c_float, vp, vp]),
+        "alexnet_augment": (st, [vp, vp, i, vp, vp, vp, vp, vp]),
+        "alexnet_tencrop": (st, [vp, vp, i, vp, vp, vp, vp]),
+        "alexnet_params_bytes": (sz, [vp]),
+        "alexnet_get_params": (st, [vp, vp, sz, vp]),
+        "alexnet_set_params": (st, [vp, vp, sz, vp]),
+        "alexnet_get_grads": (st, [vp, vp, sz, vp]),
+        "alexnet_get_status": (st, [vp]),
+        "alexnet_last_error": (ctypes.c_char_p, [vp]),
+        "alexnet_destroy": (st, [vp]),
+        "alexnet_op_conv_fwd": (st, [vp, i, i, i, i, vp, vp, i, i, i, i, i, vp, vp, sz, vp]),
+        "alexnet_op_conv1_fwd": (st, [vp, i, vp, vp, vp, vp, sz, vp]),
+        "alexnet_op_conv_dgrad": (st, [vp, i, i, i, i, vp, i, i, i, i, vp, vp, vp, sz, vp]),
+        "alexnet_op_conv_wgrad": (st, [vp, i, i, i, i, vp, i, i, i, i, i, vp, vp, sz, vp]),
+        "alexnet_op_conv1_wgrad": (st, [vp, i, vp, i, vp, vp, sz, vp]),
+        "alexnet_op_fc_fwd": (st, [vp, i, i, vp, i, i, vp, vp, sz, vp]),
+        "alexnet_op_fc_dgrad": (st, [vp, i, i, vp, i, i, vp, vp, sz, vp]),
+        "alexnet_op_fc_wgrad": (st, [vp, vp, i, i, i, vp, vp, sz, vp]),
+        "alexnet_op_lrn_fwd": (st, [vp, c_int64, i, c_float, c_float, c_float, vp, vp]),
+        "alexnet_op_lrn_bwd": (st, [vp, vp, c_int64, i, c_float, c_float, c_float, vp, vp]),
+        "alexnet_op_pool_fwd": (st, [vp, i, i, i, i, i, i, vp, vp, vp]),
+        "alexnet_op_pool_bwd": (st, [vp, vp, vp, i, i, i, i, i, i, i, vp, vp]),
+        "alexnet_op_softmax_ce": (st, [vp, vp, i, i, vp, vp, vp, vp, sz, vp]),
+        "alexnet_op_dropout_mask": (st, [c_uint64, c_uint32, c_uint32, c_float, i, i, vp, vp, sz,
+                                         vp]),
+        "alexnet_op_philox": (st, [vp, vp, i, vp, vp]),
+        "alexnet_debug_copy": (st, [vp, i, vp, sz, vp]),
+        "alexnet_stats_enable": (st, [vp, i]),
+        "alexnet_stats_read": (st, [vp, POINTER(Stats)]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L, sorted(sig)
+
+
+lib, EXPORTED = _load()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def check(status, handle=None):
+    if status != OK:
+        msg = lib.alexnet_last_error(handle)
+        raise AlexNetError(status, msg.decode() if msg else "")
+    return status
+
+
+def default_config(**overrides) -> Config:
+    c = Config()
+    lib.alexnet_default_config(ctypes.byref(c))
+    for k, v in overrides.items():
+        setattr(c, k, v)
+    return c
+
+
+def param_count(cfg: Config) -> int:
+    return lib.alexnet_param_count(ctypes.byref(cfg))
+
+
+def workspace_bytes(cfg: Config) -> int:
+    return lib.alexnet_workspace_bytes(ctypes.byref(cfg))
+
+
+class AlexNet:
+    """Owns a handle; the workspace is a torch uint8 CUDA tensor it keeps alive."""
+
+    def __init__(self, cfg: Config | None = None, stream=None, **overrides):
+        import torch
+        self.cfg = cfg if cfg is not None else default_config(**overrides)
+        nbytes = workspace_bytes(self.cfg)
+        if nbytes == 0:
+            raise AlexNetError(ERR_INVALID_ARG, "invalid config")
+        self.workspace = torch.empty(nbytes + 256, dtype=torch.uint8, device="cuda")
+        base = self.workspace.data_ptr()
+        aligned = (base + 255) & ~255
+        h = c_void_p()
+        check(lib.alexnet_create(ctypes.byref(self.cfg), aligned, nbytes, _stream(stream),
+                                 ctypes.byref(h)))
+        self.h = h
+
+    def close(self):
+        if getattr(self, "h", None):
+            lib.alexnet_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        self.close()
+
+    # -- the C calls, same names ------------------------------------------
+    def forward(self, x, B, mode, logits, probs=None, stream=None):
+        return check(lib.alexnet_forward(self.h, _ptr(x), B, mode, _ptr(logits), _ptr(probs),
+                                         _stream(stream)), self.h)
+
+    def train_step(self, x, labels, B, lr, loss=None, stream=None):
+        return check(lib.alexnet_train_step(self.h, _ptr(x), _ptr(labels), B, lr, _ptr(loss),
+                                            _stream(stream)), self.h)
+
+    def augment(self, src, B, mean, pca_vec, pca_val, x_out, stream=None):
+        return check(lib.alexnet_augment(self.h, _ptr(src), B, _ptr(mean), _ptr(pca_vec),
+                                         _ptr(pca_val), _ptr(x_out), _stream(stream)), self.h)
+
+    def tencrop(self, src, B, mean, probs_avg, top5, stream=None):
+        return check(lib.alexnet_tencrop(self.h, _ptr(src), B, _ptr(mean), _ptr(probs_avg),
+                                         _ptr(top5), _stream(stream)), self.h)
+
+    def params_bytes(self):
+        return lib.alexnet_params_bytes(self.h)
+
+    def get_params(self, dst, stream=None):
+        return check(lib.alexnet_get_params(self.h, _ptr(dst), dst.numel() * dst.element_size(),
+                                            _stream(stream)), self.h)
+
+    def set_params(self, src, stream=None):
+        return check(lib.alexnet_set_params(self.h, _ptr(src), src.numel() * src.element_size(),
+                                            _stream(stream)), self.h)
+
+    def get_grads(self, dst, stream=None):
+        return check(lib.alexnet_get_grads(self.h, _ptr(dst), dst.numel(), _stream(stream)), self.h)
+
+    def get_status(self):
+        return lib.alexnet_get_status(self.h)
+
+    def stats_enable(self, enable=True):
+        return check(lib.alexnet_stats_enable(self.h, 1 if enable else 0), self.h)
+
+    def stats_read(self):
+        st_ = Stats()
+        check(lib.alexnet_stats_read(self.h, ctypes.byref(st_)), self.h)
+        return {"launches": st_.launches, "gemm_launches": st_.gemm_launches,
+                "gemm_flops": st_.gemm_flops, "gemm_ms": st_.gemm_ms}
+
+    def debug_copy(self, which, dst, stream=None):
+        return check(lib.alexnet_debug_copy(self.h, which, _ptr(dst), dst.numel() * dst.element_size(),
+                                            _stream(stream)), self.h)
+
+
+# -- single-op entry points (alexnet_ops.h), same names ------------------------
+def _op(name, *args):
+    return check(getattr(lib, name)(*args))
+
+
+def op_conv_fwd(x, B, H, W, Cin, w, bias, Cout, K, pad, groups, relu, y, ws, stream=None):
+    return _op("alexnet_op_conv_fwd", _ptr(x), B, H, W, Cin, _ptr(w), _ptr(bias), Cout, K, pad,
+               groups, relu, _ptr(y), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def op_conv1_fwd(x, B, w, bias, y, ws, stream=None):
+    return _op("alexnet_op_conv1_fwd", _ptr(x), B, _ptr(w), _ptr(bias), _ptr(y), _ptr(ws),
+               ws.numel(), _stream(stream))
+
+
+def op_conv_dgrad(dy, B, H, W, Cin, w, Cout, K, pad, groups, mask, dx, ws, stream=None):
+    return _op("alexnet_op_conv_dgrad", _ptr(dy), B, H, W, Cin, _ptr(w), Cout, K, pad, groups,
+               _ptr(mask), _ptr(dx), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def op_conv_wgrad(x, B, H, W, Cin, dy, Cout, K, pad, groups, splits, dw, ws, stream=None):
+    return _op("alexnet_op_conv_wgrad", _ptr(x), B, H, W, Cin, _ptr(dy), Cout, K, pad, groups,
+               splits, _ptr(dw), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def op_conv1_wgrad(x, B, dy, splits, dw, ws, stream=None):
+    return _op("alexnet_op_conv1_wgrad", _ptr(x), B, _ptr(dy), splits, _ptr(dw), _ptr(ws),
+               ws.numel(), _stream(stream))
+
+
+def op_fc_fwd(x, B, In, w, Out, splits, y, ws, stream=None):
+    return _op("alexnet_op_fc_fwd", _ptr(x), B, In, _ptr(w), Out, splits, _ptr(y), _ptr(ws),
+               ws.numel(), _stream(stream))
+
+
+def op_fc_dgrad(dz, B, Out, w, In, splits, dx, ws, stream=None):
+    return _op("alexnet_op_fc_dgrad", _ptr(dz), B, Out, _ptr(w), In, splits, _ptr(dx), _ptr(ws),
+               ws.numel(), _stream(stream))
+
+
+def op_fc_wgrad(dz, x, B, Out, In, dw, ws, stream=None):
+    return _op("alexnet_op_fc_wgrad", _ptr(dz), _ptr(x), B, Out, In, _ptr(dw), _ptr(ws),
+               ws.numel(), _stream(stream))
+
+
+def op_lrn_fwd(a, P, C, k, alpha, beta, b, stream=None):
+    return _op("alexnet_op_lrn_fwd", _ptr(a), P, C, k, alpha, beta, _ptr(b), _stream(stream))
+
+
+def op_lrn_bwd(a, g, P, C, k, alpha, beta, da, stream=None):
+    return _op("alexnet_op_lrn_bwd", _ptr(a), _ptr(g), P, C, k, alpha, beta, _ptr(da),
+               _stream(stream))
+
+
+def op_pool_fwd(x, B, H, W, C, z, st, y, argmax, stream=None):
+    return _op("alexnet_op_pool_fwd", _ptr(x), B, H, W, C, z, st, _ptr(y), _ptr(argmax),
+               _stream(stream))
+
+
+def op_pool_bwd(dy, argmax, pooled, B, H, W, C, z, st, relu_mask, dx, stream=None):
+    return _op("alexnet_op_pool_bwd", _ptr(dy), _ptr(argmax), _ptr(pooled), B, H, W, C, z, st,
+               relu_mask, _ptr(dx), _stream(stream))
+
+
+def op_softmax_ce(logits, labels, B, N, probs, dlogits, loss, ws, stream=None):
+    return _op("alexnet_op_softmax_ce", _ptr(logits), _ptr(labels), B, N, _ptr(probs),
+               _ptr(dlogits), _ptr(loss), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def op_dropout_mask(seed, layer, step, p, rows, cols, keep, ws, stream=None):
+    return _op("alexnet_op_dropout_mask", seed, layer, step, p, rows, cols, _ptr(keep), _ptr(ws),
+               ws.numel(), _stream(stream))
+
+
+def op_philox(ctr, key, n, out, stream=None):
+    return _op("alexnet_op_philox", _ptr(ctr), _ptr(key), n, _ptr(out), _stream(stream))

@@ -1,0 +1,90 @@
+// gemm.h -- host-side description of one tensor-core GEMM launch.
+//
+// Every convolution (forward, data gradient, weight gradient) and every
+// fully-connected product of the network is one launch of the same
+// tcgen05 kernel, described by a GemmDesc.  D[M x N] (+)= A[M x K] * B[N x K]^T
+// accumulates in fp32 tensor memory; K is walked in 64-element blocks.
+//
+// Operand sources:
+//   A_TMA_K / A_TMA_MN : A read by TMA from a dense bf16 matrix that is
+//                        K-contiguous (rows = M) or M-contiguous (rows = K).
+//   A_GATHER_K         : implicit im2col of an NHWC bf16 map: row m is an
+//                        output pixel, its K entries are the (kh, kw, cin)
+//                        taps of one group (stride-1 convolution).
+//   A_GATHER_MN        : the transpose of that matrix (rows are output
+//                        pixels = the reduction, columns the conv taps), for
+//                        weight gradients.
+//   B_TMA_K / B_TMA_MN : B read by TMA, K-contiguous (rows = N) or
+//                        N-contiguous (rows = K).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace alx {
+
+enum ASrc : int { A_TMA_K = 0, A_TMA_MN = 1, A_GATHER_K = 2, A_GATHER_MN = 3 };
+enum BSrc : int { B_TMA_K = 0, B_TMA_MN = 1 };
+enum Epi : int {
+  EPI_BF16 = 0,       // out_bf16[row, col] = act(acc + bias[col])
+  EPI_BF16_MASK = 1,  // out_bf16[row, col] = acc if mask[row, col] > 0 else 0
+  EPI_F32 = 2,        // out_f32[split][group][row, col] = acc
+  EPI_F32_T = 3,      // out_f32[split][group][col, row] = acc
+};
+
+struct GatherDesc {
+  const __nv_bfloat16* src;  // NHWC map [B, H, W, C]
+  int H, W, C;               // C = channels per pixel (row length in elements)
+  int cg_off;                // channel offset of group g is g * cg_off
+  int Cg8;                   // channels per group / 8
+  int KW, pad;               // kernel width, zero padding (stride 1)
+  int Ho, Wo;                // output map size
+  int Kc;                    // number of 8-channel tap chunks = KH * KW * Cg8
+  int Mpix;                  // B * Ho * Wo
+};
+
+struct GemmArgs {
+  int M, N;           // output extent (rows, columns) of one group
+  int Kblocks;        // 64-wide blocks of the reduction
+  int kb_per_split;   // blocks per split-K slice
+  int splits, groups;
+  int m_tiles, n_tiles;
+  int a_goff, b_goff;  // per-group coordinate offsets of the TMA operands (in M / N)
+  GatherDesc g;
+  // epilogue
+  int epi;
+  int relu;
+  void* out;
+  long long ld_out;        // elements between rows (cols for EPI_F32_T)
+  long long split_stride;  // elements between split-K slices
+  long long group_stride;  // elements between groups (F32 modes)
+  int col_goff;            // column offset per group (BF16 modes)
+  const float* bias;       // nullable, indexed by col + g * col_goff
+  const __nv_bfloat16* mask;
+  long long ld_mask;
+  int* status;
+};
+
+struct GemmDesc {
+  int asrc, bsrc, bn;
+  CUtensorMap tmA, tmB;
+  GemmArgs args;
+  int grid;
+  int smem;
+  int stages;
+};
+
+// Build a 2-D bf16 tensor map with 128-byte swizzle: `inner` contiguous
+// elements per row, `outer` rows `row_bytes` apart, box of box_inner x
+// box_outer elements.  Returns false if the driver rejects it.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+
+// Fill grid/smem/stages of a descriptor whose asrc/bsrc/bn/args are set.
+// Returns false for an unsupported combination.
+bool gemm_finalize(GemmDesc* d, int num_sms);
+
+cudaError_t gemm_launch(const GemmDesc& d, cudaStream_t stream);
+
+}  // namespace alx

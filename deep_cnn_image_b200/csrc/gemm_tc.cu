@@ -1,0 +1,527 @@
+// gemm_tc.cu -- the one tensor-core GEMM kernel behind every convolution and
+// fully-connected product of the network (forward, data and weight gradients).
+//
+// Design (sm_100a):
+//   * persistent: one 320-thread CTA per SM walks a static list of output
+//     tiles (128 x BN), split-K slices and groups;
+//   * warp roles: warps 0-3 epilogue (TMEM -> registers -> global),
+//     warps 4-7 implicit-im2col gather producers (cp.async, 16 B per
+//     thread per row chunk, zero-fill for padding), warp 8 TMA producer,
+//     warp 9 MMA issuer (one thread) and TMEM owner;
+//   * operands staged in a ring of shared-memory stages laid out in the
+//     128-byte-swizzled canonical form that both TMA and tcgen05.mma use;
+//     full/empty mbarriers between producers and the MMA thread;
+//   * two fp32 accumulators in tensor memory so the epilogue of tile i
+//     overlaps the main loop of tile i+1.
+// The operation itself is the plain sum D = sum_k A[m,k] B[n,k]: the
+// convolution as an implicit GEMM over the (kh, kw, cin) taps
+// ("ImageNet Classification with Deep Convolutional Neural Networks",
+// summary page, 3.4 "Overall Architecture"; "AlexNet and Deep CNNs",
+// "Time complexity of one forward pass").
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+
+#include "gemm.h"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace alx {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int NUM_THREADS = 320;
+constexpr int A_TILE_BYTES = BM * BK * 2;
+constexpr int MN_BLOCK_BYTES = 64 * 128;  // 64 K-rows x 64 MN elements (bf16)
+
+__host__ __device__ constexpr int tmem_cols_for(int bn) {
+  return 2 * bn <= 32 ? 32 : (2 * bn <= 64 ? 64 : (2 * bn <= 128 ? 128 : (2 * bn <= 256 ? 256 : 512)));
+}
+
+__device__ __forceinline__ void cp_async_wait_dyn(int n) {
+  switch (n) {
+    case 0: cp_async_wait<0>(); break;
+    case 1: cp_async_wait<1>(); break;
+    case 2: cp_async_wait<2>(); break;
+    case 3: cp_async_wait<3>(); break;
+    case 4: cp_async_wait<4>(); break;
+    case 5: cp_async_wait<5>(); break;
+    case 6: cp_async_wait<6>(); break;
+    default: cp_async_wait<7>(); break;
+  }
+}
+
+struct TileCoord {
+  int m_t, n_t, sp, g;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const GemmArgs& a, int t) {
+  TileCoord c;
+  c.n_t = t % a.n_tiles;
+  t /= a.n_tiles;
+  c.m_t = t % a.m_tiles;
+  t /= a.m_tiles;
+  c.sp = t % a.splits;
+  c.g = t / a.splits;
+  return c;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int BN>
+__device__ __forceinline__ void epilogue_store(const GemmArgs& a, const TileCoord& tc, int row,
+                                               int col0, const float (&v)[16]) {
+  if (row >= a.M) return;
+  const int g = tc.g;
+  if (a.epi == EPI_BF16 || a.epi == EPI_BF16_MASK) {
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int col = col0 + 8 * h;
+      if (col >= a.N) continue;
+      float f[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] = v[8 * h + i];
+      const long long cg = static_cast<long long>(g) * a.col_goff + col;
+      if (a.epi == EPI_BF16) {
+        if (a.bias) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] += a.bias[cg + i];
+        }
+        if (a.relu) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) f[i] = f[i] > 0.f ? f[i] : 0.f;
+        }
+      } else {
+        const uint4 mv = *reinterpret_cast<const uint4*>(a.mask + row * a.ld_mask + cg);
+        const __nv_bfloat16* mb = reinterpret_cast<const __nv_bfloat16*>(&mv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = __bfloat162float(mb[i]) > 0.f ? f[i] : 0.f;
+      }
+      uint4 o;
+      o.x = pack_bf16x2(f[0], f[1]);
+      o.y = pack_bf16x2(f[2], f[3]);
+      o.z = pack_bf16x2(f[4], f[5]);
+      o.w = pack_bf16x2(f[6], f[7]);
+      *reinterpret_cast<uint4*>(out + row * a.ld_out + cg) = o;
+    }
+  } else if (a.epi == EPI_F32) {
+    float* out = reinterpret_cast<float*>(a.out) + tc.sp * a.split_stride + g * a.group_stride +
+                 row * a.ld_out;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = col0 + 4 * q;
+      if (col < a.N)
+        *reinterpret_cast<float4*>(out + col) =
+            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+  } else {  // EPI_F32_T
+    float* out = reinterpret_cast<float*>(a.out) + tc.sp * a.split_stride + g * a.group_stride;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int col = col0 + i;
+      if (col < a.N) out[col * a.ld_out + row] = v[i];
+    }
+  }
+}
+
+template <int BN, int ASRC, int BSRC>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ GemmArgs args, int stages) {
+  constexpr int B_TILE_BYTES = BN * BK * 2;
+  constexpr int TMEM_COLS = tmem_cols_for(BN);
+  constexpr bool A_GATHER = (ASRC == A_GATHER_K || ASRC == A_GATHER_MN);
+  constexpr int A_MN = (ASRC == A_TMA_MN || ASRC == A_GATHER_MN) ? 1 : 0;
+  constexpr int B_MN = (BSRC == B_TMA_MN) ? 1 : 0;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + stages * A_TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * (A_TILE_BYTES + B_TILE_BYTES));
+  const uint32_t bar_full = smem_u32(bars);
+  const uint32_t bar_empty = bar_full + 8 * stages;
+  const uint32_t bar_acc_full = bar_full + 16 * stages;
+  const uint32_t bar_acc_empty = bar_acc_full + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * stages + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(bar_full + 8 * s, (A_GATHER ? 128 : 0) + 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_acc_full + 8 * i, 1);
+      mbar_init(bar_acc_empty + 8 * i, 128);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int total_tiles = args.m_tiles * args.n_tiles * args.splits * args.groups;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      if (ASRC == A_TMA_K || ASRC == A_TMA_MN) tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const TileCoord tc = decode_tile(args, t);
+        const int kb0 = tc.sp * args.kb_per_split;
+        const int kb1 = min(args.Kblocks, kb0 + args.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % stages;
+          const uint32_t ph = (it / stages) & 1;
+          if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, args.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar_full + 8 * s;
+          mbar_arrive_expect_tx(fb, B_TILE_BYTES + (A_GATHER ? 0 : A_TILE_BYTES));
+          const uint32_t dB = sB + s * B_TILE_BYTES;
+          const int n0 = tc.g * args.b_goff + tc.n_t * BN;
+          if (BSRC == B_TMA_K) {
+            tma_load_2d(dB, &tmB, kb * BK, n0, fb);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_2d(dB + j * MN_BLOCK_BYTES, &tmB, n0 + j * 64, kb * BK, fb);
+          }
+          const uint32_t dA = sA + s * A_TILE_BYTES;
+          const int m0 = tc.g * args.a_goff + tc.m_t * BM;
+          if (ASRC == A_TMA_K) {
+            tma_load_2d(dA, &tmA, kb * BK, m0, fb);
+          } else if (ASRC == A_TMA_MN) {
+            tma_load_2d(dA, &tmA, m0, kb * BK, fb);
+            tma_load_2d(dA + MN_BLOCK_BYTES, &tmA, m0 + 64, kb * BK, fb);
+          }
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tcount) {
+        const TileCoord tc = decode_tile(args, t);
+        const int kb0 = tc.sp * args.kb_per_split;
+        const int kb1 = min(args.Kblocks, kb0 + args.kb_per_split);
+        const int acc = tcount & 1;
+        const uint32_t aph = (tcount >> 1) & 1;
+        if (!mbar_wait(bar_acc_empty + 8 * acc, aph ^ 1, args.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * (TMEM_COLS / 2);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % stages;
+          const uint32_t ph = (it / stages) & 1;
+          if (!mbar_wait(bar_full + 8 * s, ph, args.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = sA + s * A_TILE_BYTES;
+          const uint32_t b0 = sB + s * B_TILE_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(a0 + k * 2048, MN_BLOCK_BYTES, 1024)
+                                     : smem_desc_sw128(a0 + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, MN_BLOCK_BYTES, 1024)
+                                     : smem_desc_sw128(b0 + k * 32, 16, 1024);
+            tc_mma_f16(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(bar_empty + 8 * s);
+        }
+        if (!ok) break;
+        tc_commit(bar_acc_full + 8 * acc);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ gather producers
+    if (A_GATHER) {
+      const int t = threadIdx.x - 128;
+      const int c = t & 7;
+      const GatherDesc& G = args.g;
+      const int lag = stages - 1;
+      uint32_t it = 0;
+      bool ok = true;
+      const int HoWo = G.Ho * G.Wo;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const TileCoord tc = decode_tile(args, tile);
+        const int kb0 = tc.sp * args.kb_per_split;
+        const int kb1 = min(args.Kblocks, kb0 + args.kb_per_split);
+        if (ASRC == A_GATHER_K) {
+          // rows rg + 16 j of the tile are output pixels; chunk c of each k-block
+          const int rg = t >> 3;
+          int pbase[8], poh[8], pow_[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int m = tc.m_t * BM + rg + 16 * j;
+            if (m < G.Mpix) {
+              const int b = m / HoWo;
+              const int rem = m - b * HoWo;
+              poh[j] = rem / G.Wo;
+              pow_[j] = rem - poh[j] * G.Wo;
+              pbase[j] = b * G.H;
+            } else {
+              poh[j] = -(1 << 20);
+              pow_[j] = 0;
+              pbase[j] = 0;
+            }
+          }
+          const __nv_bfloat16* gsrc = G.src + tc.g * G.cg_off;
+          for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % stages;
+            const uint32_t ph = (it / stages) & 1;
+            if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, args.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const int kc = kb * 8 + c;
+            const bool kvalid = kc < G.Kc;
+            const int tap = kvalid ? kc / G.Cg8 : 0;
+            const int cin8 = kc - tap * G.Cg8;
+            const int kh = tap / G.KW;
+            const int kw = tap - kh * G.KW;
+            const int dh = kh - G.pad, dw = kw - G.pad;
+            const __nv_bfloat16* base = gsrc + cin8 * 8;
+            const uint32_t dst0 = sA + s * A_TILE_BYTES;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int r = rg + 16 * j;
+              const int ih = poh[j] + dh, iw = pow_[j] + dw;
+              const bool okp = kvalid && ih >= 0 && ih < G.H && iw >= 0 && iw < G.W;
+              const __nv_bfloat16* src =
+                  okp ? base + (static_cast<long long>(pbase[j] + ih) * G.W + iw) * G.C : G.src;
+              cp_async_16(dst0 + r * 128 + ((c ^ (r & 7)) << 4), src, okp ? 16u : 0u);
+            }
+            cp_async_commit();
+            if (static_cast<int>(it) >= lag) {
+              cp_async_wait_dyn(lag);
+              fence_proxy_async_smem();
+              mbar_arrive(bar_full + 8 * ((it - lag) % stages));
+            }
+          }
+        } else {
+          // A_GATHER_MN: rows are output pixels (the reduction), the two
+          // 64-wide column blocks are conv-tap chunks of this M tile
+          const int q = t >> 3;
+          bool kval[2];
+          int dh[2], dw[2];
+          const __nv_bfloat16* cbase[2];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int kc = tc.m_t * 16 + j * 8 + c;
+            kval[j] = kc < G.Kc;
+            const int tap = kval[j] ? kc / G.Cg8 : 0;
+            const int cin8 = kc - tap * G.Cg8;
+            const int kh = tap / G.KW;
+            const int kw = tap - kh * G.KW;
+            dh[j] = kh - G.pad;
+            dw[j] = kw - G.pad;
+            cbase[j] = G.src + tc.g * G.cg_off + cin8 * 8;
+          }
+          for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % stages;
+            const uint32_t ph = (it / stages) & 1;
+            if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, args.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            const uint32_t dst0 = sA + s * A_TILE_BYTES;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int r = q + 16 * i;
+              const int m = kb * BK + r;
+              int b = 0, oh = -(1 << 20), ow = 0;
+              if (m < G.Mpix) {
+                b = m / HoWo;
+                const int rem = m - b * HoWo;
+                oh = rem / G.Wo;
+                ow = rem - oh * G.Wo;
+              }
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const int ih = oh + dh[j], iw = ow + dw[j];
+                const bool okp = kval[j] && ih >= 0 && ih < G.H && iw >= 0 && iw < G.W;
+                const __nv_bfloat16* src =
+                    okp ? cbase[j] + (static_cast<long long>(b * G.H + ih) * G.W + iw) * G.C : G.src;
+                cp_async_16(dst0 + j * MN_BLOCK_BYTES + r * 128 + ((c ^ (r & 7)) << 4), src,
+                            okp ? 16u : 0u);
+              }
+            }
+            cp_async_commit();
+            if (static_cast<int>(it) >= lag) {
+              cp_async_wait_dyn(lag);
+              fence_proxy_async_smem();
+              mbar_arrive(bar_full + 8 * ((it - lag) % stages));
+            }
+          }
+        }
+      }
+      // drain: the last `lag` stages
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      if (ok) {
+        const uint32_t first = it > static_cast<uint32_t>(lag) ? it - lag : 0;
+        for (uint32_t i = first; i < it; ++i) mbar_arrive(bar_full + 8 * (i % stages));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    uint32_t tcount = 0;
+    const int row_in_tile = warp * 32 + lane;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tcount) {
+      const TileCoord tc = decode_tile(args, t);
+      const int acc = tcount & 1;
+      const uint32_t aph = (tcount >> 1) & 1;
+      if (!mbar_wait(bar_acc_full + 8 * acc, aph, args.status, abort_flag)) break;
+      tc_fence_after();
+      const int row = tc.m_t * BM + row_in_tile;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + acc * (TMEM_COLS / 2);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + c0, v);
+        epilogue_store<BN>(args, tc, row, tc.n_t * BN + c0, v);
+      }
+      tc_fence_before();
+      mbar_arrive(bar_acc_empty + 8 * acc);
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    // give bulk copies already in flight time to land before the CTA exits
+    for (int i = 0; i < 1000; ++i) __nanosleep(1000);
+  }
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, GemmArgs, int);
+
+template <int BN, int ASRC, int BSRC>
+void* kernel_ptr() {
+  return reinterpret_cast<void*>(&gemm_kernel<BN, ASRC, BSRC>);
+}
+
+struct KernelEntry {
+  int bn, asrc, bsrc;
+  void* fn;
+  bool attr_set;
+};
+
+#define ALX_K(BN_, A_, B_) {BN_, A_, B_, kernel_ptr<BN_, A_, B_>(), false}
+KernelEntry g_kernels[] = {
+    ALX_K(48, A_GATHER_K, B_TMA_K),    ALX_K(64, A_GATHER_K, B_TMA_K),
+    ALX_K(96, A_GATHER_K, B_TMA_K),    ALX_K(128, A_GATHER_K, B_TMA_K),
+    ALX_K(192, A_GATHER_K, B_TMA_K),   ALX_K(256, A_GATHER_K, B_TMA_K),
+    ALX_K(64, A_GATHER_MN, B_TMA_MN),  ALX_K(128, A_GATHER_MN, B_TMA_MN),
+    ALX_K(192, A_GATHER_MN, B_TMA_MN), ALX_K(256, A_GATHER_MN, B_TMA_MN),
+    ALX_K(64, A_TMA_K, B_TMA_K),       ALX_K(128, A_TMA_K, B_TMA_K),
+    ALX_K(256, A_TMA_K, B_TMA_K),      ALX_K(64, A_TMA_K, B_TMA_MN),
+    ALX_K(128, A_TMA_K, B_TMA_MN),     ALX_K(256, A_TMA_K, B_TMA_MN),
+    ALX_K(64, A_TMA_MN, B_TMA_MN),     ALX_K(128, A_TMA_MN, B_TMA_MN),
+    ALX_K(256, A_TMA_MN, B_TMA_MN),
+};
+#undef ALX_K
+
+KernelEntry* find_kernel(int bn, int asrc, int bsrc) {
+  for (auto& k : g_kernels)
+    if (k.bn == bn && k.asrc == asrc && k.bsrc == bsrc) return &k;
+  return nullptr;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  if (!g_encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (row_bytes & 15) || inner == 0 || outer == 0)
+    return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool gemm_finalize(GemmDesc* d, int num_sms) {
+  KernelEntry* k = find_kernel(d->bn, d->asrc, d->bsrc);
+  if (!k) return false;
+  GemmArgs& a = d->args;
+  if (a.M <= 0 || a.N <= 0 || a.Kblocks <= 0 || a.groups <= 0) return false;
+  if (a.N % 8) return false;
+  if (d->bsrc == B_TMA_MN && d->bn % 64) return false;
+  a.m_tiles = (a.M + BM - 1) / BM;
+  a.n_tiles = (a.N + d->bn - 1) / d->bn;
+  if (a.kb_per_split <= 0 || a.kb_per_split > a.Kblocks) a.kb_per_split = a.Kblocks;
+  a.splits = (a.Kblocks + a.kb_per_split - 1) / a.kb_per_split;
+  const int stage_bytes = A_TILE_BYTES + d->bn * BK * 2;
+  const int budget = 227 * 1024 - 1024 - 256;
+  int stages = budget / stage_bytes;
+  if (stages > 8) stages = 8;
+  if (stages < 3) return false;
+  d->stages = stages;
+  d->smem = stages * stage_bytes + 1024 + 256;
+  const long long tiles = 1LL * a.m_tiles * a.n_tiles * a.splits * a.groups;
+  d->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+  return true;
+}
+
+cudaError_t gemm_launch(const GemmDesc& d, cudaStream_t stream) {
+  KernelEntry* k = find_kernel(d.bn, d.asrc, d.bsrc);
+  if (!k) return cudaErrorInvalidValue;
+  if (!k->attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k->fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         227 * 1024);
+    if (e != cudaSuccess) return e;
+    k->attr_set = true;
+  }
+  void* params[] = {const_cast<CUtensorMap*>(&d.tmA), const_cast<CUtensorMap*>(&d.tmB),
+                    const_cast<GemmArgs*>(&d.args), const_cast<int*>(&d.stages)};
+  count_launch();
+  return cudaLaunchKernel(k->fn, dim3(d.grid), dim3(NUM_THREADS), params, d.smem, stream);
+}
+
+}  // namespace alx

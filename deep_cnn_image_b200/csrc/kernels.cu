@@ -1,0 +1,1046 @@
+// kernels.cu -- the memory-bound kernels of the AlexNet training step.
+//
+// Pages cited:
+//   [S] "ImageNet Classification with Deep Convolutional Neural Networks",
+//       paper-graph-ui summary page, section 3.4 subsections.
+//   [W] "AlexNet and Deep CNNs" (fermi.ai wiki page).
+// Layout: NHWC bf16 activations, channels fastest; each thread moves one
+// 16-byte chunk (8 channels) so every load and store is a full vector.
+#include <cuda_bf16.h>
+
+#include <atomic>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace alx {
+
+namespace {
+
+constexpr int kMaxGrid = 148 * 16;
+
+inline int grid_for(long long n, int block) {
+  long long g = (n + block - 1) / block;
+  if (g > kMaxGrid) g = kMaxGrid;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  return u;
+}
+__device__ __forceinline__ float2 ld_bf16x2(const bf16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+
+// ------------------------------------------------------------------ hparams
+__global__ void k_write_hparams(HParams* hp, HParams v) { *hp = v; }
+
+// ------------------------------------------------------------------ s2d
+__global__ void k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs, int B) {
+  const long long n = 1LL * B * 57 * 57 * 6;
+  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
+       t += 1LL * gridDim.x * blockDim.x) {
+    const int chunk = static_cast<int>(t % 6);
+    long long pix = t / 6;
+    const int j = static_cast<int>(pix % 57);
+    const int i = static_cast<int>((pix / 57) % 57);
+    const int b = static_cast<int>(pix / (57 * 57));
+    float f[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int ch = chunk * 8 + q;
+      const int dy = ch / 12, dx = (ch / 3) % 4, c = ch % 3;
+      const int y = 4 * i + dy, xx = 4 * j + dx;
+      f[q] = (y < 227 && xx < 227)
+                 ? __bfloat162float(x[((static_cast<long long>(b) * 227 + y) * 227 + xx) * 3 + c])
+                 : 0.f;
+    }
+    *reinterpret_cast<uint4*>(xs + pix * 48 + chunk * 8) = pack8(f);
+  }
+}
+
+// ------------------------------------------------------------------ LRN
+// [S] 3.4 "Local Response Normalization": b_i = a_i / (k + alpha * sum_{|j-i|<=2} a_j^2)^beta
+// with the window clipped to the layer's channels (n = 5).
+__global__ void k_lrn_fwd(const bf16* __restrict__ a, bf16* __restrict__ b, long long P, int C,
+                          float k, float alpha, float beta) {
+  const int chunks = C >> 3;
+  const long long n = P * chunks;
+  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
+       t += 1LL * gridDim.x * blockDim.x) {
+    const long long p = t / chunks;
+    const int c0 = static_cast<int>(t - p * chunks) * 8;
+    const bf16* ap = a + p * C;
+    float v[12];
+    {
+      float f[8];
+      unpack8(*reinterpret_cast<const uint4*>(ap + c0), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[2 + i] = f[i];
+    }
+    if (c0 > 0) {
+      const float2 lo = ld_bf16x2(ap + c0 - 2);
+      v[0] = lo.x;
+      v[1] = lo.y;
+    } else {
+      v[0] = v[1] = 0.f;
+    }
+    if (c0 + 8 < C) {
+      const float2 hi = ld_bf16x2(ap + c0 + 8);
+      v[10] = hi.x;
+      v[11] = hi.y;
+    } else {
+      v[10] = v[11] = 0.f;
+    }
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 5; ++j) sum += v[i + j] * v[i + j];
+      const float s = k + alpha * sum;
+      o[i] = v[i + 2] * powf(s, -beta);
+    }
+    *reinterpret_cast<uint4*>(b + p * C + c0) = pack8(o);
+  }
+}
+
+// Backward: da_j = g_j s_j^-beta - 2 alpha beta a_j sum_{|i-j|<=2} g_i a_i s_i^(-beta-1),
+// then times relu'(a_j) (a is the ReLU output, so a_j > 0 <=> the unit was active).
+__global__ void k_lrn_bwd(const bf16* __restrict__ a, const bf16* __restrict__ g,
+                          bf16* __restrict__ da, long long P, int C, float k, float alpha,
+                          float beta) {
+  const int chunks = C >> 3;
+  const long long n = P * chunks;
+  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
+       t += 1LL * gridDim.x * blockDim.x) {
+    const long long p = t / chunks;
+    const int c0 = static_cast<int>(t - p * chunks) * 8;
+    const bf16* ap = a + p * C;
+    const bf16* gp = g + p * C;
+    float av[16];  // channels c0-4 .. c0+11
+    float gv[12];  // channels c0-2 .. c0+9
+#pragma unroll
+    for (int i = 0; i < 16; ++i) av[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 12; ++i) gv[i] = 0.f;
+    {
+      float f[8];
+      unpack8(*reinterpret_cast<const uint4*>(ap + c0), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) av[4 + i] = f[i];
+      unpack8(*reinterpret_cast<const uint4*>(gp + c0), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) gv[2 + i] = f[i];
+    }
+    if (c0 > 0) {
+      const float2 a0 = ld_bf16x2(ap + c0 - 4), a1 = ld_bf16x2(ap + c0 - 2);
+      av[0] = a0.x; av[1] = a0.y; av[2] = a1.x; av[3] = a1.y;
+      const float2 g1 = ld_bf16x2(gp + c0 - 2);
+      gv[0] = g1.x; gv[1] = g1.y;
+    }
+    if (c0 + 8 < C) {
+      const float2 a0 = ld_bf16x2(ap + c0 + 8), a1 = ld_bf16x2(ap + c0 + 10);
+      av[12] = a0.x; av[13] = a0.y; av[14] = a1.x; av[15] = a1.y;
+      const float2 g1 = ld_bf16x2(gp + c0 + 8);
+      gv[10] = g1.x; gv[11] = g1.y;
+    }
+    // s_i and t_i = g_i a_i s_i^(-beta-1) for channels c0-2 .. c0+9 (index i+2 in av)
+    float sp[12], tt[12];
+#pragma unroll
+    for (int i = 0; i < 12; ++i) {
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 5; ++j) sum += av[i + j] * av[i + j];
+      const float s = k + alpha * sum;
+      const float sb = powf(s, -beta);
+      sp[i] = sb;
+      tt[i] = gv[i] * av[i + 2] * (sb / s);
+    }
+    float o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float cross = 0.f;
+#pragma unroll
+      for (int q = 0; q < 5; ++q) cross += tt[j + q];
+      const float aj = av[j + 4];
+      const float d = gv[j + 2] * sp[j + 2] - 2.f * alpha * beta * aj * cross;
+      o[j] = aj > 0.f ? d : 0.f;
+    }
+    *reinterpret_cast<uint4*>(da + p * C + c0) = pack8(o);
+  }
+}
+
+__global__ void k_lrn_fwd_f32(const float* __restrict__ a, float* __restrict__ b, long long P,
+                              int C, float k, float alpha, float beta) {
+  const long long n = P * C;
+  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
+       t += 1LL * gridDim.x * blockDim.x) {
+    const long long p = t / C;
+    const int c = static_cast<int>(t - p * C);
+    const float* ap = a + p * C;
+    float sum = 0.f;
+    for (int j = max(0, c - 2); j <= min(C - 1, c + 2); ++j) sum += ap[j] * ap[j];
+    b[t] = ap[c] * powf(k + alpha * sum, -beta);
+  }
+}
+
+// ------------------------------------------------------------------ pooling
+// [S] 3.4 "Overlapping Pooling": max over z x z windows at stride st, no padding.
+__global__ void k_pool_fwd(const bf16* __restrict__ x, bf16* __restrict__ y,
+                           uint8_t* __restrict__ am, int B, int H, int W, int C, int z, int st) {
+  const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
+  const int chunks = C >> 3;
+  const long long n = 1LL * B * Ho * Wo * chunks;
+  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
+       t += 1LL * gridDim.x * blockDim.x) {
+    const int c0 = static_cast<int>(t % chunks) * 8;
+    const long long pix = t / chunks;
+    const int ow = static_cast<int>(pix % Wo);
+    const int oh = static_cast<int>((pix / Wo) % Ho);
+    const int b = static_cast<int>(pix / (1LL * Wo * Ho));
+    float best[8];
+    int arg[8];
+    for (int dy = 0; dy < z; ++dy)
+      for (int dx = 0; dx < z; ++dx) {
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4*>(
+                    x + ((1LL * b * H + oh * st + dy) * W + ow * st + dx) * C + c0),
+                f);
+        const int off = dy * z + dx;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (off == 0 || f[i] > best[i]) {
+            best[i] = f[i];
+            arg[i] = off;
+          }
+        }
+      }
+    *reinterpret_cast<uint4*>(y + pix * C + c0) = pack8(best);
+    uint2 packed;
+    packed.x = arg[0] | (arg[1] << 8) | (arg[2] << 16) | (arg[3] << 24);
+    packed.y = arg[4] | (arg[5] << 8) | (arg[6] << 16) | (arg[7] << 24);
+    *reinterpret_cast<uint2*>(am + pix * C + c0) = packed;
+  }
+}
+
+__global__ void k_pool_bwd(const bf16* __restrict__ dy, const uint8_t* __restrict__ am,
+                           const bf16* __restrict__ pooled, bf16* __restrict__ dx, int B, int H,
+                           int W, int C, int z, int st, int relu_mask) {
+  const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
+  const int chunks = C >> 3;
+  const long long n = 1LL * B * H * W * chunks;
+  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
+       t += 1LL * gridDim.x * blockDim.x) {
+    const int c0 = static_cast<int>(t % chunks) * 8;
+    const long long pix = t / chunks;
+    const int iw = static_cast<int>(pix % W);
+    const int ih = static_cast<int>((pix / W) % H);
+    const int b = static_cast<int>(pix / (1LL * W * H));
+    const int oh_lo = ih < z ? 0 : (ih - z + st) / st;
+    const int oh_hi = min(Ho - 1, ih / st);
+    const int ow_lo = iw < z ? 0 : (iw - z + st) / st;
+    const int ow_hi = min(Wo - 1, iw / st);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int oh = oh_lo; oh <= oh_hi; ++oh)
+      for (int ow = ow_lo; ow <= ow_hi; ++ow) {
+        const long long o = ((1LL * b * Ho + oh) * Wo + ow) * C + c0;
+        const int off = (ih - oh * st) * z + (iw - ow * st);
+        const uint2 a2 = *reinterpret_cast<const uint2*>(am + o);
+        float g[8];
+        unpack8(*reinterpret_cast<const uint4*>(dy + o), g);
+        float pv[8];
+        if (relu_mask) unpack8(*reinterpret_cast<const uint4*>(pooled + o), pv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t word = i < 4 ? a2.x : a2.y;
+          const int ai = (word >> (8 * (i & 3))) & 0xFF;
+          const bool take = ai == off && (!relu_mask || pv[i] > 0.f);
+          if (take) acc[i] += g[i];
+        }
+      }
+    *reinterpret_cast<uint4*>(dx + pix * C + c0) = pack8(acc);
+  }
+}
+
+__global__ void k_pool_fwd_f32(const float* __restrict__ x, float* __restrict__ y, int B, int H,
+                               int W, int C, int z, int st) {
+  const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
+  const long long n = 1LL * B * Ho * Wo * C;
+  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
+       t += 1LL * gridDim.x * blockDim.x) {
+    const int c = static_cast<int>(t % C);
+    const long long pix = t / C;
+    const int ow = static_cast<int>(pix % Wo);
+    const int oh = static_cast<int>((pix / Wo) % Ho);
+    const int b = static_cast<int>(pix / (1LL * Wo * Ho));
+    float best = 0.f;
+    for (int dy = 0; dy < z; ++dy)
+      for (int dx = 0; dx < z; ++dx) {
+        const float v = x[((1LL * b * H + oh * st + dy) * W + ow * st + dx) * C + c];
+        if ((dy == 0 && dx == 0) || v > best) best = v;
+      }
+    y[t] = best;
+  }
+}
+
+// ------------------------------------------------------------------ FC epilogues
+// Dropout ([S] 3.4 "Dropout"): element e = row*cols + col of FC layer `layer`
+// is kept iff word (e & 3) of Philox4x32-10((e >> 2, layer, step, 0),
+// (seed_lo, seed_hi)) >= drop_thresh; kept units are not rescaled at
+// training time; at inference every unit is multiplied by 1 - p.
+__device__ __forceinline__ U4 dropout_words(const HParams& hp, long long e4, int layer) {
+  U4 c{static_cast<uint32_t>(e4), static_cast<uint32_t>(layer), hp.step, 0u};
+  return philox4x32_10(c, hp.seed_lo, hp.seed_hi);
+}
+
+__global__ void k_fc_finalize(const float* __restrict__ part, int S, int rows, int cols,
+                              const float* __restrict__ bias, int relu, int dropout_mode,
+                              int layer, const HParams* __restrict__ hpp, bf16* out_bf16,
+                              float* out_f32) {
+  const HParams hp = *hpp;
+  const long long n4 = 1LL * rows * cols / 4;
+  const long long plane = 1LL * rows * cols;
+  for (long long q = blockIdx.x * 1LL * blockDim.x + threadIdx.x; q < n4;
+       q += 1LL * gridDim.x * blockDim.x) {
+    const long long e = q * 4;
+    const int col = static_cast<int>(e % cols);
+    float4 acc = *reinterpret_cast<const float4*>(part + e);
+    for (int s = 1; s < S; ++s) {
+      const float4 p = *reinterpret_cast<const float4*>(part + s * plane + e);
+      acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+    }
+    float v[4] = {acc.x, acc.y, acc.z, acc.w};
+    if (bias) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] += bias[col + i];
+    }
+    if (relu) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = v[i] > 0.f ? v[i] : 0.f;
+    }
+    if (dropout_mode == 1) {
+      const U4 w = dropout_words(hp, q, layer);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = u4_word(w, i) >= hp.drop_thresh ? v[i] : 0.f;
+    } else if (dropout_mode == 2) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] *= (1.f - hp.dropout_p);
+    }
+    if (out_bf16) {
+      uint2 u;
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
+      u.x = *reinterpret_cast<uint32_t*>(&h0);
+      u.y = *reinterpret_cast<uint32_t*>(&h1);
+      *reinterpret_cast<uint2*>(out_bf16 + e) = u;
+    } else {
+      *reinterpret_cast<float4*>(out_f32 + e) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+  }
+}
+
+__global__ void k_dropout_mask(const HParams* __restrict__ hpp, int layer, int rows, int cols,
+                               uint8_t* keep) {
+  const HParams hp = *hpp;
+  const long long n4 = 1LL * rows * cols / 4;
+  for (long long q = blockIdx.x * 1LL * blockDim.x + threadIdx.x; q < n4;
+       q += 1LL * gridDim.x * blockDim.x) {
+    const U4 w = dropout_words(hp, q, layer);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) keep[q * 4 + i] = u4_word(w, i) >= hp.drop_thresh ? 1 : 0;
+  }
+}
+
+__global__ void k_dgrad_finalize(const float* __restrict__ part, int S, int rows, int cols,
+                                 const bf16* __restrict__ mask, bf16* __restrict__ out) {
+  const long long n8 = 1LL * rows * cols / 8;
+  const long long plane = 1LL * rows * cols;
+  for (long long q = blockIdx.x * 1LL * blockDim.x + threadIdx.x; q < n8;
+       q += 1LL * gridDim.x * blockDim.x) {
+    const long long e = q * 8;
+    float v[8];
+    {
+      const float4 a = *reinterpret_cast<const float4*>(part + e);
+      const float4 b = *reinterpret_cast<const float4*>(part + e + 4);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+    for (int s = 1; s < S; ++s) {
+      const float4 a = *reinterpret_cast<const float4*>(part + s * plane + e);
+      const float4 b = *reinterpret_cast<const float4*>(part + s * plane + e + 4);
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+    if (mask) {
+      float m[8];
+      unpack8(*reinterpret_cast<const uint4*>(mask + e), m);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = m[i] > 0.f ? v[i] : 0.f;
+    }
+    *reinterpret_cast<uint4*>(out + e) = pack8(v);
+  }
+}
+
+// ------------------------------------------------------------------ softmax + CE
+// [S] 3.4 "Training Procedure Details", "Objective function": the mean over
+// the batch of -log softmax(z)_label; dlogits = (p - onehot) / B.
+__global__ void k_softmax_ce(const float* __restrict__ logits, const int32_t* __restrict__ labels,
+                             int B, int N, float* probs, bf16* dlogits, float* loss_rows,
+                             int* status) {
+  __shared__ float red[32];
+  const int b = blockIdx.x;
+  const float* z = logits + 1LL * b * N;
+  const int tid = threadIdx.x, nw = blockDim.x >> 5;
+  float m = -INFINITY;
+  for (int j = tid; j < N; j += blockDim.x) m = fmaxf(m, z[j]);
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((tid & 31) == 0) red[tid >> 5] = m;
+  __syncthreads();
+  if (tid < 32) {
+    float v = tid < nw ? red[tid] : -INFINITY;
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (tid == 0) red[0] = v;
+  }
+  __syncthreads();
+  m = red[0];
+  __syncthreads();
+  float sum = 0.f;
+  for (int j = tid; j < N; j += blockDim.x) sum += expf(z[j] - m);
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if ((tid & 31) == 0) red[tid >> 5] = sum;
+  __syncthreads();
+  if (tid < 32) {
+    float v = tid < nw ? red[tid] : 0.f;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (tid == 0) red[0] = v;
+  }
+  __syncthreads();
+  sum = red[0];
+  int y = -1;
+  if (labels) {
+    y = labels[b];
+    if (y < 0 || y >= N) {
+      if (tid == 0) atomicOr(status, STATUS_LABEL_RANGE);
+      y = -1;
+    }
+  }
+  const float inv = 1.f / sum;
+  const float invB = 1.f / static_cast<float>(B);
+  for (int j = tid; j < N; j += blockDim.x) {
+    const float p = expf(z[j] - m) * inv;
+    if (probs) probs[1LL * b * N + j] = p;
+    if (dlogits) dlogits[1LL * b * N + j] = __float2bfloat16_rn((p - (j == y ? 1.f : 0.f)) * invB);
+  }
+  if (tid == 0 && loss_rows) loss_rows[b] = y >= 0 ? -((z[y] - m) - logf(sum)) : 0.f;
+}
+
+__global__ void k_loss_mean(const float* __restrict__ rows, int B, float* out1, float* out2) {
+  __shared__ float red[256];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < B; i += blockDim.x) s += rows[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const float v = red[0] / static_cast<float>(B);
+    if (out1) *out1 = v;
+    if (out2) *out2 = v;
+  }
+}
+
+// ------------------------------------------------------------------ bias gradients
+constexpr int kColsumRows = 256;
+
+__global__ void k_colsum_partial(const bf16* __restrict__ m, long long rows, int cols,
+                                 float* __restrict__ partial) {
+  const int chunk = blockIdx.x;
+  const int col = blockIdx.y * blockDim.x + threadIdx.x;
+  if (col >= cols) return;
+  const long long r0 = 1LL * chunk * kColsumRows;
+  const long long r1 = min(rows, r0 + kColsumRows);
+  float s = 0.f;
+  for (long long r = r0; r < r1; ++r) s += __bfloat162float(m[r * cols + col]);
+  partial[1LL * chunk * cols + col] = s;
+}
+
+// ------------------------------------------------------------------ SGD
+// [S] 3.4 "Training Procedure Details", update rule; [W] listing TRAIN_STEP:
+// v <- momentum v - wd lr w - lr g ; w <- w + v, for every parameter.
+__device__ __forceinline__ void sgd_one(float& w, float& v, float g, const HParams& hp) {
+  const float vn = hp.momentum * v - hp.weight_decay * hp.lr * w - hp.lr * g;
+  v = vn;
+  w = w + vn;
+}
+
+struct ConvIdx {
+  long long fwd, dg, part_inner;
+  int g, co;
+};
+
+// canonical p = ((o*K + kh)*K + kw)*Cg + ci
+__device__ __forceinline__ ConvIdx conv_index(const ConvMap& m, long long p) {
+  const int ci = static_cast<int>(p % m.Cg);
+  long long t = p / m.Cg;
+  const int kw = static_cast<int>(t % m.K);
+  t /= m.K;
+  const int kh = static_cast<int>(t % m.K);
+  const int o = static_cast<int>(t / m.K);
+  const int Og = m.Cout / m.groups;
+  ConvIdx r;
+  r.g = o / Og;
+  r.co = o - r.g * Og;
+  if (m.s2d) {
+    const int kg = ((kh >> 2) * 3 + (kw >> 2)) * 48 + ((kh & 3) * 4 + (kw & 3)) * 3 + ci;
+    r.fwd = 1LL * o * 432 + kg;
+    r.part_inner = kg;
+    r.dg = -1;
+  } else {
+    r.fwd = p;
+    r.part_inner = (1LL * kh * m.K + kw) * m.Cg + ci;
+    r.dg = (((1LL * r.g * m.Cg + ci) * m.K + (m.K - 1 - kh)) * m.K + (m.K - 1 - kw)) * Og + r.co;
+  }
+  return r;
+}
+
+__global__ void k_sgd_conv(float* __restrict__ w, float* __restrict__ v,
+                           const float* __restrict__ part, int S, ConvMap m, bf16* fwd, bf16* dg,
+                           float* grads_out, const HParams* __restrict__ hpp) {
+  const HParams hp = *hpp;
+  const long long n = 1LL * m.Cout * m.K * m.K * m.Cg;
+  const int Og = m.Cout / m.groups;
+  const long long Kg = m.s2d ? 432 : 1LL * m.K * m.K * m.Cg;
+  const long long split_stride = 1LL * m.groups * Og * Kg;
+  for (long long p = blockIdx.x * 1LL * blockDim.x + threadIdx.x; p < n;
+       p += 1LL * gridDim.x * blockDim.x) {
+    const ConvIdx ix = conv_index(m, p);
+    const long long base = (1LL * ix.g * Og + ix.co) * Kg + ix.part_inner;
+    float g = 0.f;
+    for (int s = 0; s < S; ++s) g += part[s * split_stride + base];
+    float wv = w[p], vv = v[p];
+    sgd_one(wv, vv, g, hp);
+    w[p] = wv;
+    v[p] = vv;
+    const bf16 hb = __float2bfloat16_rn(wv);
+    fwd[ix.fwd] = hb;
+    if (dg) dg[ix.dg] = hb;
+    if (grads_out) grads_out[p] = g;
+  }
+}
+
+__global__ void k_conv_shadows(const float* __restrict__ w, ConvMap m, bf16* fwd, bf16* dg) {
+  const long long n = 1LL * m.Cout * m.K * m.K * m.Cg;
+  for (long long p = blockIdx.x * 1LL * blockDim.x + threadIdx.x; p < n;
+       p += 1LL * gridDim.x * blockDim.x) {
+    const ConvIdx ix = conv_index(m, p);
+    const bf16 hb = __float2bfloat16_rn(w[p]);
+    fwd[ix.fwd] = hb;
+    if (dg) dg[ix.dg] = hb;
+  }
+}
+
+__global__ void k_sgd_dense(float* __restrict__ w, float* __restrict__ v,
+                            const float* __restrict__ g, long long n, bf16* shadow,
+                            float* grads_out, const HParams* __restrict__ hpp) {
+  const HParams hp = *hpp;
+  const long long n4 = n / 4;
+  for (long long q = blockIdx.x * 1LL * blockDim.x + threadIdx.x; q < n4;
+       q += 1LL * gridDim.x * blockDim.x) {
+    float4 wv = reinterpret_cast<float4*>(w)[q];
+    float4 vv = reinterpret_cast<float4*>(v)[q];
+    const float4 gv = reinterpret_cast<const float4*>(g)[q];
+    sgd_one(wv.x, vv.x, gv.x, hp);
+    sgd_one(wv.y, vv.y, gv.y, hp);
+    sgd_one(wv.z, vv.z, gv.z, hp);
+    sgd_one(wv.w, vv.w, gv.w, hp);
+    reinterpret_cast<float4*>(w)[q] = wv;
+    reinterpret_cast<float4*>(v)[q] = vv;
+    if (shadow) {
+      uint2 u;
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(wv.x, wv.y);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(wv.z, wv.w);
+      u.x = *reinterpret_cast<uint32_t*>(&h0);
+      u.y = *reinterpret_cast<uint32_t*>(&h1);
+      reinterpret_cast<uint2*>(shadow)[q] = u;
+    }
+    if (grads_out) reinterpret_cast<float4*>(grads_out)[q] = gv;
+  }
+}
+
+__global__ void k_sgd_bias(float* __restrict__ b, float* __restrict__ v,
+                           const float* __restrict__ partial, int chunks, int n, float* grads_out,
+                           const HParams* __restrict__ hpp) {
+  const HParams hp = *hpp;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    float g = 0.f;
+    for (int c = 0; c < chunks; ++c) g += partial[1LL * c * n + i];
+    float wv = b[i], vv = v[i];
+    sgd_one(wv, vv, g, hp);
+    b[i] = wv;
+    v[i] = vv;
+    if (grads_out) grads_out[i] = g;
+  }
+}
+
+__global__ void k_f32_to_bf16(const float* __restrict__ w, bf16* __restrict__ out, long long n) {
+  for (long long i = blockIdx.x * 1LL * blockDim.x + threadIdx.x; i < n;
+       i += 1LL * gridDim.x * blockDim.x)
+    out[i] = __float2bfloat16_rn(w[i]);
+}
+
+__global__ void k_f32_from_bf16(const bf16* __restrict__ in, float* __restrict__ out, long long n) {
+  for (long long i = blockIdx.x * 1LL * blockDim.x + threadIdx.x; i < n;
+       i += 1LL * gridDim.x * blockDim.x)
+    out[i] = __bfloat162float(in[i]);
+}
+
+// ------------------------------------------------------------------ init
+// [S] 3.4 "Training Procedure Details", weight initialisation: zero-mean
+// Gaussian with standard deviation 0.01.  Normals from Box-Muller on Philox
+// words: Philox((q, tag, 0xC0, 0), seed) gives elements 4q .. 4q+3.
+__global__ void k_init_normal(float* __restrict__ w, long long n, float stdv, uint32_t k0,
+                              uint32_t k1, uint32_t tag) {
+  const long long n4 = (n + 3) / 4;
+  for (long long q = blockIdx.x * 1LL * blockDim.x + threadIdx.x; q < n4;
+       q += 1LL * gridDim.x * blockDim.x) {
+    const U4 r = philox4x32_10(U4{static_cast<uint32_t>(q), tag, 0xC0u, 0u}, k0, k1);
+    const float r1 = sqrtf(-2.f * logf(word_unit(r.x)));
+    const float r2 = sqrtf(-2.f * logf(word_unit(r.z)));
+    float s1, c1, s2, c2;
+    sincospif(2.f * word_unit(r.y), &s1, &c1);
+    sincospif(2.f * word_unit(r.w), &s2, &c2);
+    const float z[4] = {r1 * c1, r1 * s1, r2 * c2, r2 * s2};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (q * 4 + i < n) w[q * 4 + i] = stdv * z[i];
+  }
+}
+
+__global__ void k_fill(float* __restrict__ w, long long n, float value) {
+  for (long long i = blockIdx.x * 1LL * blockDim.x + threadIdx.x; i < n;
+       i += 1LL * gridDim.x * blockDim.x)
+    w[i] = value;
+}
+
+// ------------------------------------------------------------------ augmentation
+// [S] 3.4 "Data Augmentation": Form 1, a 224x224 patch at offset (oy, ox) in
+// 0..31 with an optional horizontal reflection; Form 2, the same colour
+// offset [p1 p2 p3][a1 l1, a2 l2, a3 l3]^T added to every pixel of the image,
+// a_i ~ N(0, 0.1^2).  Per-pixel mean subtracted first ([S] 3.2).  Draws for
+// image i at step t: word 0 of Philox((i, 0xA0, t, 0)) -> bits 0-4 oy,
+// bits 5-9 ox, bit 10 reflection; Philox((i, 0xA1, t, 0)) -> Box-Muller
+// pairs (words 0, 1 -> a1, a2; words 2, 3 -> a3 from the cosine branch).
+struct AugDraw {
+  int oy, ox, flip;
+  float add[3];
+};
+
+__device__ __forceinline__ AugDraw aug_draw(const HParams& hp, uint32_t img, const float* pv,
+                                            const float* pl) {
+  AugDraw d;
+  const U4 r0 = philox4x32_10(U4{img, 0xA0u, hp.step, 0u}, hp.seed_lo, hp.seed_hi);
+  d.oy = static_cast<int>(r0.x & 31u);
+  d.ox = static_cast<int>((r0.x >> 5) & 31u);
+  d.flip = static_cast<int>((r0.x >> 10) & 1u);
+  const U4 r1 = philox4x32_10(U4{img, 0xA1u, hp.step, 0u}, hp.seed_lo, hp.seed_hi);
+  const float m1 = sqrtf(-2.f * logf(word_unit(r1.x)));
+  const float m2 = sqrtf(-2.f * logf(word_unit(r1.z)));
+  float s1, c1, s2, c2;
+  sincospif(2.f * word_unit(r1.y), &s1, &c1);
+  sincospif(2.f * word_unit(r1.w), &s2, &c2);
+  const float a[3] = {0.1f * m1 * c1, 0.1f * m1 * s1, 0.1f * m2 * c2};
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) s += pv[c * 3 + i] * (a[i] * pl[i]);
+    d.add[c] = s;
+  }
+  return d;
+}
+
+__global__ void k_augment(const uint8_t* __restrict__ src, int B, const float* __restrict__ mean,
+                          const float* __restrict__ pca_vec, const float* __restrict__ pca_val,
+                          const HParams* __restrict__ hpp, bf16* __restrict__ out) {
+  const HParams hp = *hpp;
+  __shared__ AugDraw d;
+  __shared__ float pv[9], pl[3];
+  // one block per (image, output row)
+  for (long long job = blockIdx.x; job < 1LL * B * 227; job += gridDim.x) {
+    const int b = static_cast<int>(job / 227);
+    const int y = static_cast<int>(job % 227);
+    __syncthreads();
+    if (threadIdx.x < 9) pv[threadIdx.x] = pca_vec[threadIdx.x];
+    if (threadIdx.x < 3) pl[threadIdx.x] = pca_val[threadIdx.x];
+    __syncthreads();
+    if (threadIdx.x == 0) d = aug_draw(hp, static_cast<uint32_t>(b), pv, pl);
+    __syncthreads();
+    bf16* orow = out + (1LL * b * 227 + y) * 227 * 3;
+    for (int e = threadIdx.x; e < 227 * 3; e += blockDim.x) {
+      const int x = e / 3, c = e - x * 3;
+      float v = 0.f;
+      if (y < 224 && x < 224) {
+        const int sy = d.oy + y;
+        const int sx = d.flip ? d.ox + 223 - x : d.ox + x;
+        const long long si = (1LL * sy * 256 + sx) * 3 + c;
+        v = static_cast<float>(src[1LL * b * 256 * 256 * 3 + si]) - mean[si] + d.add[c];
+      }
+      orow[e] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+// [S] 3.4 "Data Augmentation", test time: four corner patches and the centre
+// patch, then their reflections (order TL, TR, BL, BR, centre, reflected x5).
+__constant__ int kTenOy[5] = {0, 0, 32, 32, 16};
+__constant__ int kTenOx[5] = {0, 32, 0, 32, 16};
+
+__global__ void k_tencrop_inputs(const uint8_t* __restrict__ src, int B,
+                                 const float* __restrict__ mean, bf16* __restrict__ out) {
+  for (long long job = blockIdx.x; job < 1LL * B * 10 * 227; job += gridDim.x) {
+    const int img = static_cast<int>(job / 227);
+    const int y = static_cast<int>(job % 227);
+    const int b = img / 10, p = img % 10;
+    const int oy = kTenOy[p % 5], ox = kTenOx[p % 5], flip = p >= 5;
+    bf16* orow = out + (1LL * img * 227 + y) * 227 * 3;
+    for (int e = threadIdx.x; e < 227 * 3; e += blockDim.x) {
+      const int x = e / 3, c = e - x * 3;
+      float v = 0.f;
+      if (y < 224 && x < 224) {
+        const int sy = oy + y;
+        const int sx = flip ? ox + 223 - x : ox + x;
+        const long long si = (1LL * sy * 256 + sx) * 3 + c;
+        v = static_cast<float>(src[1LL * b * 256 * 256 * 3 + si]) - mean[si];
+      }
+      orow[e] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+// Average of the ten softmax outputs, then top-5 by descending probability,
+// ties to the lower class index.
+__global__ void k_tencrop_reduce(const float* __restrict__ probs10, int B, int N,
+                                 float* __restrict__ avg, int32_t* __restrict__ top5) {
+  extern __shared__ float sp[];
+  __shared__ float bv[32];
+  __shared__ int bi[32];
+  const int b = blockIdx.x;
+  for (int j = threadIdx.x; j < N; j += blockDim.x) {
+    float s = 0.f;
+    for (int p = 0; p < 10; ++p) s += probs10[(1LL * b * 10 + p) * N + j];
+    s = s / 10.f;
+    sp[j] = s;
+    avg[1LL * b * N + j] = s;
+  }
+  __syncthreads();
+  const int nw = blockDim.x >> 5;
+  for (int k = 0; k < 5; ++k) {
+    float best = -INFINITY;
+    int idx = 0x7fffffff;
+    for (int j = threadIdx.x; j < N; j += blockDim.x) {
+      const float v = sp[j];
+      if (v > best || (v == best && j < idx)) {
+        best = v;
+        idx = j;
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, idx, o);
+      if (ov > best || (ov == best && oi < idx)) {
+        best = ov;
+        idx = oi;
+      }
+    }
+    if ((threadIdx.x & 31) == 0) {
+      bv[threadIdx.x >> 5] = best;
+      bi[threadIdx.x >> 5] = idx;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float b0 = bv[0];
+      int i0 = bi[0];
+      for (int w = 1; w < nw; ++w)
+        if (bv[w] > b0 || (bv[w] == b0 && bi[w] < i0)) {
+          b0 = bv[w];
+          i0 = bi[w];
+        }
+      top5[b * 5 + k] = i0;
+      sp[i0] = -INFINITY;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ fp32 path
+// wt[g][t][co] with t = (kh*K + kw)*Cg + ci, co within the group.
+__global__ void k_conv_wt_f32(const float* __restrict__ w, float* __restrict__ wt, int Cout, int K,
+                              int Cg, int groups) {
+  const long long n = 1LL * Cout * K * K * Cg;
+  const int Og = Cout / groups;
+  const long long T = 1LL * K * K * Cg;
+  for (long long p = blockIdx.x * 1LL * blockDim.x + threadIdx.x; p < n;
+       p += 1LL * gridDim.x * blockDim.x) {
+    const long long t = p % T;
+    const int o = static_cast<int>(p / T);
+    const int g = o / Og, co = o - g * Og;
+    wt[(1LL * g * T + t) * Og + co] = w[p];
+  }
+}
+
+__global__ void k_conv_fwd_f32(const float* __restrict__ x, const float* __restrict__ wt,
+                               const float* __restrict__ bias, float* __restrict__ y, int B, int H,
+                               int W, int Cin, int Cout, int K, int stride, int pad, int groups,
+                               int Ho, int Wo) {
+  const int Og = Cout / groups, Cg = Cin / groups;
+  const int g = blockIdx.z;
+  const int co = blockIdx.y * blockDim.x + threadIdx.x;
+  const long long T = 1LL * K * K * Cg;
+  for (long long pix = blockIdx.x; pix < 1LL * B * Ho * Wo; pix += gridDim.x) {
+    if (co >= Og) continue;
+    const int ow = static_cast<int>(pix % Wo);
+    const int oh = static_cast<int>((pix / Wo) % Ho);
+    const int b = static_cast<int>(pix / (1LL * Wo * Ho));
+    float acc = bias[g * Og + co];
+    for (int kh = 0; kh < K; ++kh) {
+      const int ih = oh * stride - pad + kh;
+      if (ih < 0 || ih >= H) continue;
+      for (int kw = 0; kw < K; ++kw) {
+        const int iw = ow * stride - pad + kw;
+        if (iw < 0 || iw >= W) continue;
+        const float* xp = x + ((1LL * b * H + ih) * W + iw) * Cin + g * Cg;
+        const float* wp = wt + (1LL * g * T + (1LL * kh * K + kw) * Cg) * Og + co;
+        for (int ci = 0; ci < Cg; ++ci) acc = fmaf(__ldg(xp + ci), wp[1LL * ci * Og], acc);
+      }
+    }
+    y[pix * Cout + g * Og + co] = acc > 0.f ? acc : 0.f;
+  }
+}
+
+__global__ void k_fc_fwd_f32(const float* __restrict__ x, const float* __restrict__ w,
+                             const float* __restrict__ bias, float* __restrict__ y, int B, int In,
+                             int Out, int relu, float scale) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = 1LL * gridDim.x * (blockDim.x >> 5);
+  for (long long job = blockIdx.x * 1LL * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       job < 1LL * B * Out; job += warps) {
+    const int b = static_cast<int>(job / Out), o = static_cast<int>(job % Out);
+    const float* xr = x + 1LL * b * In;
+    const float* wr = w + 1LL * o * In;
+    float s = 0.f;
+    for (int i = lane; i < In; i += 32) s = fmaf(xr[i], wr[i], s);
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) {
+      float v = s + bias[o];
+      if (relu) v = v > 0.f ? v : 0.f;
+      y[job] = v * scale;
+    }
+  }
+}
+
+}  // namespace
+
+// ================================================================== launchers
+namespace {
+std::atomic<int64_t> g_launches{0};
+}
+int64_t launch_counter() { return g_launches.load(); }
+void count_launch() { g_launches.fetch_add(1); }
+
+void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s) {
+  k_write_hparams<<<1, 1, 0, s>>>(hp, v);
+  count_launch();
+}
+
+void launch_s2d(const bf16* x, bf16* xs, int B, cudaStream_t s) {
+  k_s2d<<<grid_for(1LL * B * 57 * 57 * 6, 256), 256, 0, s>>>(x, xs, B);
+  count_launch();
+}
+void launch_lrn_fwd(const bf16* a, bf16* b, long long P, int C, int, float k, float alpha,
+                    float beta, cudaStream_t s) {
+  k_lrn_fwd<<<grid_for(P * (C / 8), 256), 256, 0, s>>>(a, b, P, C, k, alpha, beta);
+  count_launch();
+}
+void launch_lrn_bwd(const bf16* a, const bf16* g, bf16* da, long long P, int C, int, float k,
+                    float alpha, float beta, cudaStream_t s) {
+  k_lrn_bwd<<<grid_for(P * (C / 8), 256), 256, 0, s>>>(a, g, da, P, C, k, alpha, beta);
+  count_launch();
+}
+void launch_lrn_fwd_f32(const float* a, float* b, long long P, int C, int, float k, float alpha,
+                        float beta, cudaStream_t s) {
+  k_lrn_fwd_f32<<<grid_for(P * C, 256), 256, 0, s>>>(a, b, P, C, k, alpha, beta);
+  count_launch();
+}
+void launch_pool_fwd(const bf16* x, bf16* y, uint8_t* am, int B, int H, int W, int C, int z,
+                     int st, cudaStream_t s) {
+  const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
+  k_pool_fwd<<<grid_for(1LL * B * Ho * Wo * (C / 8), 256), 256, 0, s>>>(x, y, am, B, H, W, C, z,
+                                                                        st);
+  count_launch();
+}
+void launch_pool_bwd(const bf16* dy, const uint8_t* am, const bf16* pooled, bf16* dx, int B,
+                     int H, int W, int C, int z, int st, int relu_mask, cudaStream_t s) {
+  k_pool_bwd<<<grid_for(1LL * B * H * W * (C / 8), 256), 256, 0, s>>>(dy, am, pooled, dx, B, H,
+                                                                     W, C, z, st, relu_mask);
+  count_launch();
+}
+void launch_pool_fwd_f32(const float* x, float* y, int B, int H, int W, int C, int z, int st,
+                         cudaStream_t s) {
+  const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
+  k_pool_fwd_f32<<<grid_for(1LL * B * Ho * Wo * C, 256), 256, 0, s>>>(x, y, B, H, W, C, z, st);
+  count_launch();
+}
+void launch_fc_finalize(const float* part, int S, int rows, int cols, const float* bias,
+                        int relu, int dropout_mode, int layer, const HParams* hp, bf16* out_bf16,
+                        float* out_f32, cudaStream_t s) {
+  k_fc_finalize<<<grid_for(1LL * rows * cols / 4, 256), 256, 0, s>>>(
+      part, S, rows, cols, bias, relu, dropout_mode, layer, hp, out_bf16, out_f32);
+  count_launch();
+}
+void launch_dgrad_finalize(const float* part, int S, int rows, int cols, const bf16* mask,
+                           bf16* out, cudaStream_t s) {
+  k_dgrad_finalize<<<grid_for(1LL * rows * cols / 8, 256), 256, 0, s>>>(part, S, rows, cols,
+                                                                       mask, out);
+  count_launch();
+}
+void launch_dropout_mask(const HParams* hp, int layer, int rows, int cols, uint8_t* keep,
+                         cudaStream_t s) {
+  k_dropout_mask<<<grid_for(1LL * rows * cols / 4, 256), 256, 0, s>>>(hp, layer, rows, cols,
+                                                                     keep);
+  count_launch();
+}
+void launch_softmax_ce(const float* logits, const int32_t* labels, int B, int N, float* probs,
+                       bf16* dlogits, float* loss_rows, int* status, cudaStream_t s) {
+  k_softmax_ce<<<B, 256, 0, s>>>(logits, labels, B, N, probs, dlogits, loss_rows, status);
+  count_launch();
+}
+void launch_loss_mean(const float* loss_rows, int B, float* out1, float* out2, cudaStream_t s) {
+  k_loss_mean<<<1, 256, 0, s>>>(loss_rows, B, out1, out2);
+  count_launch();
+}
+int colsum_chunks(long long rows) { return static_cast<int>((rows + kColsumRows - 1) / kColsumRows); }
+void launch_colsum_partial(const bf16* m, long long rows, int cols, float* partial,
+                           cudaStream_t s) {
+  dim3 grid(colsum_chunks(rows), (cols + 127) / 128);
+  k_colsum_partial<<<grid, 128, 0, s>>>(m, rows, cols, partial);
+  count_launch();
+}
+void launch_sgd_conv(float* w, float* v, const float* part, int S, const ConvMap& m, bf16* fwd,
+                     bf16* dg, float* grads_out, const HParams* hp, cudaStream_t s) {
+  const long long n = 1LL * m.Cout * m.K * m.K * m.Cg;
+  k_sgd_conv<<<grid_for(n, 256), 256, 0, s>>>(w, v, part, S, m, fwd, dg, grads_out, hp);
+  count_launch();
+}
+void launch_sgd_dense(float* w, float* v, const float* g, long long n, bf16* shadow,
+                      float* grads_out, const HParams* hp, cudaStream_t s) {
+  k_sgd_dense<<<grid_for(n / 4, 256), 256, 0, s>>>(w, v, g, n, shadow, grads_out, hp);
+  count_launch();
+}
+void launch_sgd_bias(float* b, float* v, const float* partial, int chunks, int n, float* grads_out,
+                     const HParams* hp, cudaStream_t s) {
+  k_sgd_bias<<<grid_for(n, 256), 256, 0, s>>>(b, v, partial, chunks, n, grads_out, hp);
+  count_launch();
+}
+void launch_conv_shadows(const float* w, const ConvMap& m, bf16* fwd, bf16* dg, cudaStream_t s) {
+  const long long n = 1LL * m.Cout * m.K * m.K * m.Cg;
+  k_conv_shadows<<<grid_for(n, 256), 256, 0, s>>>(w, m, fwd, dg);
+  count_launch();
+}
+void launch_f32_to_bf16(const float* w, bf16* out, long long n, cudaStream_t s) {
+  k_f32_to_bf16<<<grid_for(n, 256), 256, 0, s>>>(w, out, n);
+  count_launch();
+}
+void launch_f32_from_bf16(const bf16* in, float* out, long long n, cudaStream_t s) {
+  k_f32_from_bf16<<<grid_for(n, 256), 256, 0, s>>>(in, out, n);
+  count_launch();
+}
+void launch_init_normal(float* w, long long n, float stdv, uint64_t seed, uint32_t tag,
+                        cudaStream_t s) {
+  k_init_normal<<<grid_for((n + 3) / 4, 256), 256, 0, s>>>(
+      w, n, stdv, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), tag);
+  count_launch();
+}
+void launch_fill(float* w, long long n, float value, cudaStream_t s) {
+  k_fill<<<grid_for(n, 256), 256, 0, s>>>(w, n, value);
+  count_launch();
+}
+void launch_augment(const uint8_t* src, int B, const float* mean, const float* pca_vec,
+                    const float* pca_val, const HParams* hp, bf16* out, cudaStream_t s) {
+  k_augment<<<grid_for(1LL * B * 227 * 256, 256), 256, 0, s>>>(src, B, mean, pca_vec, pca_val,
+                                                                hp, out);
+  count_launch();
+}
+void launch_tencrop_inputs(const uint8_t* src, int B, const float* mean, bf16* out,
+                           cudaStream_t s) {
+  k_tencrop_inputs<<<grid_for(1LL * B * 10 * 227 * 256, 256), 256, 0, s>>>(src, B, mean, out);
+  count_launch();
+}
+void launch_tencrop_reduce(const float* probs10, int B, int N, float* probs_avg, int32_t* top5,
+                           cudaStream_t s) {
+  k_tencrop_reduce<<<B, 256, N * sizeof(float), s>>>(probs10, B, N, probs_avg, top5);
+  count_launch();
+}
+void launch_conv_wt_f32(const float* w, float* wt, int Cout, int K, int Cg, int groups,
+                        cudaStream_t s) {
+  k_conv_wt_f32<<<grid_for(1LL * Cout * K * K * Cg, 256), 256, 0, s>>>(w, wt, Cout, K, Cg,
+                                                                       groups);
+  count_launch();
+}
+void launch_conv_fwd_f32(const float* x, const float* wt, const float* bias, float* y, int B,
+                         int H, int W, int Cin, int Cout, int K, int stride, int pad, int groups,
+                         int Ho, int Wo, cudaStream_t s) {
+  const int Og = Cout / groups;
+  long long pix = 1LL * B * Ho * Wo;
+  dim3 grid(static_cast<unsigned>(pix < 65535 * 4 ? pix : 65535 * 4), (Og + 127) / 128, groups);
+  k_conv_fwd_f32<<<grid, 128, 0, s>>>(x, wt, bias, y, B, H, W, Cin, Cout, K, stride, pad, groups,
+                                      Ho, Wo);
+  count_launch();
+}
+void launch_fc_fwd_f32(const float* x, const float* w, const float* bias, float* y, int B, int In,
+                       int Out, int relu, float scale, cudaStream_t s) {
+  k_fc_fwd_f32<<<grid_for(1LL * B * Out * 32, 256), 256, 0, s>>>(x, w, bias, y, B, In, Out, relu,
+                                                                 scale);
+  count_launch();
+}
+
+}  // namespace alx
+
+namespace alx {
+namespace {
+__global__ void k_philox_raw(const uint32_t* __restrict__ ctr, const uint32_t* __restrict__ key,
+                             int n, uint32_t* __restrict__ out) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const U4 r = philox4x32_10(U4{ctr[4 * i], ctr[4 * i + 1], ctr[4 * i + 2], ctr[4 * i + 3]},
+                               key[2 * i], key[2 * i + 1]);
+    out[4 * i] = r.x;
+    out[4 * i + 1] = r.y;
+    out[4 * i + 2] = r.z;
+    out[4 * i + 3] = r.w;
+  }
+}
+}  // namespace
+void launch_philox_raw(const uint32_t* ctr, const uint32_t* key, int n, uint32_t* out,
+                       cudaStream_t s) {
+  k_philox_raw<<<grid_for(n, 256), 256, 0, s>>>(ctr, key, n, out);
+  count_launch();
+}
+}  // namespace alx

@@ -1,0 +1,1149 @@
+// net.cu -- the host side of libalexnet.so: handle, workspace layout,
+// per-batch GEMM plans and the order of launches of a forward pass and of a
+// training step.  All device memory is the caller's workspace; nothing here
+// allocates device memory.
+//
+// Pages cited:
+//   [S] "ImageNet Classification with Deep Convolutional Neural Networks",
+//       paper-graph-ui summary page (section 3.4 subsections).
+//   [W] "AlexNet and Deep CNNs" (fermi.ai wiki page), listings
+//       ALEXNET_FORWARD and TRAIN_STEP.
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "alexnet.h"
+#include "alexnet_ops.h"
+#include "gemm.h"
+#include "kernels.h"
+
+using namespace alx;
+
+namespace {
+
+constexpr int kClasses = 1000;
+
+// Bump allocator over the caller's workspace (base == nullptr: size only).
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t n) {
+    off = (off + 255) & ~static_cast<size_t>(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+};
+
+struct ConvL {
+  int Cin, Cout, K, stride, pad, groups;
+  int H, Ho;    // input / output side
+  int lrn, pool;
+  int P;        // side after pooling (or Ho)
+  // GEMM view (conv1 is the 3x3 stride-1 convolution of its 57x57x48
+  // space-to-depth input)
+  int gH, gC, gK, gpad, gCg;
+  int Og() const { return Cout / groups; }
+  int Kdim() const { return gK * gK * gCg; }
+};
+
+struct FcL {
+  int In, Out;
+};
+
+struct Plan {
+  GemmDesc cf[5], cd[5], cw[5], ff[3], fd[3], fw[3];
+  double conv_flops[5], fc_flops[3];  // algorithmic FLOPs of one pass of each layer
+  bool ok = false;
+};
+
+int pick_bn(int n) {
+  if (n <= 256 && (n == 48 || n == 64 || n == 96 || n == 128 || n == 192 || n == 256)) return n;
+  if (n % 192 == 0) return 192;
+  if (n % 256 == 0) return 256;
+  if (n % 128 == 0) return 128;
+  return 0;
+}
+int pick_bn_mn(int n) {
+  if (n <= 64) return 64;
+  if (n <= 128) return 128;
+  if (n == 192 || n % 192 == 0) return 192;
+  if (n <= 256 || n % 256 == 0) return 256;
+  return 128;
+}
+int pick_kbps(long long tiles, int kblocks, int num_sms, int min_blocks) {
+  long long s = (2LL * num_sms + tiles - 1) / tiles;
+  const long long smax = kblocks / min_blocks > 0 ? kblocks / min_blocks : 1;
+  if (s > smax) s = smax;
+  if (s < 1) s = 1;
+  return static_cast<int>((kblocks + s - 1) / s);
+}
+
+}  // namespace
+
+struct alexnet {
+  alexnet_config cfg;
+  int num_sms = 148;
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  std::string err;
+  cudaStream_t last_stream = nullptr;
+  uint64_t step = 0;
+
+  ConvL conv[5];
+  FcL fc[3];
+  size_t w_off[8], w_len[8], b_off[8], b_len[8];
+  size_t n_params = 0;
+
+  // device buffers
+  float* params = nullptr;  // [n_params] then vel [n_params] contiguous
+  float* vel = nullptr;
+  float* grads = nullptr;
+  bf16* wf[8] = {};  // forward GEMM operands
+  bf16* wd[5] = {};  // data-gradient operands (conv2..conv5)
+  HParams* hp = nullptr;
+  int* status = nullptr;
+  float* loss_dev = nullptr;
+  float* loss_rows = nullptr;
+  bf16* xin = nullptr;  // staged inputs (ten-crop patches)
+  bf16* xs = nullptr;
+  bf16* a[5] = {};
+  bf16* lo[5] = {};
+  bf16* p[5] = {};
+  uint8_t* am[5] = {};
+  bf16* f6 = nullptr;
+  bf16* f7 = nullptr;
+  float* logits = nullptr;
+  float* probs = nullptr;
+  bf16* dlogits = nullptr;
+  bf16* d7 = nullptr;
+  bf16* d6 = nullptr;
+  bf16* dp5 = nullptr;
+  bf16* da[5] = {};
+  bf16* dp[5] = {};
+  bf16* dl[5] = {};
+  float* scratch = nullptr;
+  size_t scratch_floats = 0;
+  float* cpart = nullptr;
+  size_t cpart_floats = 0;
+  // fp32 path
+  float* fa = nullptr;
+  float* fb = nullptr;
+  float* fwt = nullptr;
+  size_t f_act = 0;
+
+  HParams hp_host;
+  std::map<int, Plan> plans;
+
+  // launch accounting (alexnet_stats_*)
+  bool stats_on = false;
+  int64_t launch_base = 0;
+  int64_t gemm_launches = 0;
+  double gemm_flops = 0.0;
+  std::vector<cudaEvent_t> ev;
+  size_t ev_used = 0;
+  cudaStream_t stats_stream = nullptr;
+
+  const bf16* conv_input(int l) const {
+    if (l == 0) return xs;
+    const int q = l - 1;
+    if (conv[q].pool) return p[q];
+    if (conv[q].lrn) return lo[q];
+    return a[q];
+  }
+};
+
+namespace {
+
+std::string g_create_error;
+
+bool set_err(alexnet* h, const char* msg) {
+  if (h) h->err = msg;
+  return false;
+}
+
+alexnet_status cuda_status(alexnet* h, cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return ALEXNET_OK;
+  char buf[256];
+  snprintf(buf, sizeof(buf), "%s: %s", where, cudaGetErrorString(e));
+  if (h) h->err = buf;
+  return ALEXNET_ERR_CUDA;
+}
+
+bool valid_config(const alexnet_config* c) {
+  if (!c) return false;
+  if (c->batch_max < 1 || c->batch_max > 4096) return false;
+  if (c->dtype != ALEXNET_FP32 && c->dtype != ALEXNET_BF16) return false;
+  if (c->grouped != 0 && c->grouped != 1) return false;
+  if (c->lrn_n != 5) return false;
+  if (c->pool_size != 2 && c->pool_size != 3) return false;
+  if (!(c->dropout_p >= 0.f && c->dropout_p < 1.f)) return false;
+  if (!(c->lrn_k > 0.f)) return false;
+  return true;
+}
+
+void build_geometry(alexnet* h) {
+  const alexnet_config& c = h->cfg;
+  const int g = c.grouped ? 2 : 1;
+  const int cin[5] = {3, 96, 256, 384, 384};
+  const int cout[5] = {96, 256, 384, 384, 256};
+  const int ks[5] = {11, 5, 3, 3, 3};
+  const int st[5] = {4, 1, 1, 1, 1};
+  const int pd[5] = {0, 2, 1, 1, 1};
+  const int gr[5] = {1, g, 1, g, g};
+  const int lrn[5] = {c.lrn_on, c.lrn_on, 0, 0, 0};
+  const int pool[5] = {1, 1, 0, 0, 1};
+  int H = 227;
+  size_t off = 0;
+  for (int l = 0; l < 5; ++l) {
+    ConvL& L = h->conv[l];
+    L.Cin = cin[l];
+    L.Cout = cout[l];
+    L.K = ks[l];
+    L.stride = st[l];
+    L.pad = pd[l];
+    L.groups = gr[l];
+    L.H = H;
+    L.Ho = (H + 2 * L.pad - L.K) / L.stride + 1;
+    L.lrn = lrn[l];
+    L.pool = pool[l];
+    L.P = L.pool ? (L.Ho - c.pool_size) / 2 + 1 : L.Ho;
+    if (l == 0) {
+      L.gH = 57;
+      L.gC = 48;
+      L.gK = 3;
+      L.gpad = 0;
+      L.gCg = 48;
+    } else {
+      L.gH = H;
+      L.gC = L.Cin;
+      L.gK = L.K;
+      L.gpad = L.pad;
+      L.gCg = L.Cin / L.groups;
+    }
+    h->w_off[l] = off;
+    h->w_len[l] = static_cast<size_t>(L.Cout) * L.K * L.K * (L.Cin / L.groups);
+    off += h->w_len[l];
+    h->b_off[l] = off;
+    h->b_len[l] = L.Cout;
+    off += h->b_len[l];
+    H = L.P;
+  }
+  int in = H * H * h->conv[4].Cout;
+  const int outs[3] = {4096, 4096, kClasses};
+  for (int f = 0; f < 3; ++f) {
+    h->fc[f].In = in;
+    h->fc[f].Out = outs[f];
+    h->w_off[5 + f] = off;
+    h->w_len[5 + f] = static_cast<size_t>(in) * outs[f];
+    off += h->w_len[5 + f];
+    h->b_off[5 + f] = off;
+    h->b_len[5 + f] = outs[f];
+    off += h->b_len[5 + f];
+    in = outs[f];
+  }
+  h->n_params = off;
+}
+
+// ---------------------------------------------------------------- GEMM descs
+// When sizing the workspace no tensor map is encoded (no device is needed).
+bool g_dry_tmaps = false;
+
+bool tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+          uint32_t box_inner, uint32_t box_outer) {
+  if (g_dry_tmaps) {
+    memset(m, 0, sizeof(*m));
+    return true;
+  }
+  return make_tmap_bf16(m, base, inner, outer, row_bytes, box_inner, box_outer);
+}
+
+GatherDesc gather_fwd(const ConvL& L, const bf16* src, int B) {
+  GatherDesc g;
+  g.src = src;
+  g.H = L.gH;
+  g.W = L.gH;
+  g.C = L.gC;
+  g.cg_off = L.gCg;
+  g.Cg8 = L.gCg / 8;
+  g.KW = L.gK;
+  g.pad = L.gpad;
+  g.Ho = L.Ho;
+  g.Wo = L.Ho;
+  g.Kc = L.gK * L.gK * L.gCg / 8;
+  g.Mpix = B * L.Ho * L.Ho;
+  return g;
+}
+
+bool desc_conv_fwd(GemmDesc* d, const ConvL& L, const bf16* in, const bf16* w, const float* bias,
+                   bf16* out, int B, int num_sms, int* status) {
+  memset(d, 0, sizeof(*d));
+  d->asrc = A_GATHER_K;
+  d->bsrc = B_TMA_K;
+  d->bn = pick_bn(L.Og());
+  if (!d->bn) return false;
+  GemmArgs& a = d->args;
+  a.g = gather_fwd(L, in, B);
+  a.M = a.g.Mpix;
+  a.N = L.Og();
+  a.Kblocks = (a.g.Kc + 7) / 8;
+  a.groups = L.groups;
+  a.b_goff = L.Og();
+  a.epi = EPI_BF16;
+  a.relu = 1;
+  a.out = out;
+  a.ld_out = L.Cout;
+  a.col_goff = L.Og();
+  a.bias = bias;
+  a.status = status;
+  if (!tmap(&d->tmB, w, L.Kdim(), L.Cout, static_cast<uint64_t>(L.Kdim()) * 2, 64,
+                      d->bn))
+    return false;
+  d->tmA = d->tmB;
+  return gemm_finalize(d, num_sms);
+}
+
+// Data gradient of a stride-1 conv as a forward conv of dY with the flipped,
+// transposed kernel and padding K-1-pad.
+bool desc_conv_dgrad(GemmDesc* d, const ConvL& L, const bf16* dy, const bf16* wdg,
+                     const bf16* mask, bf16* out, int B, int num_sms, int* status) {
+  memset(d, 0, sizeof(*d));
+  const int Cg = L.Cin / L.groups, Og = L.Og();
+  d->asrc = A_GATHER_K;
+  d->bsrc = B_TMA_K;
+  d->bn = pick_bn(Cg);
+  if (!d->bn || L.stride != 1) return false;
+  GemmArgs& a = d->args;
+  GatherDesc& g = a.g;
+  g.src = dy;
+  g.H = L.Ho;
+  g.W = L.Ho;
+  g.C = L.Cout;
+  g.cg_off = Og;
+  g.Cg8 = Og / 8;
+  g.KW = L.K;
+  g.pad = L.K - 1 - L.pad;
+  g.Ho = L.H;
+  g.Wo = L.H;
+  g.Kc = L.K * L.K * Og / 8;
+  g.Mpix = B * L.H * L.H;
+  a.M = g.Mpix;
+  a.N = Cg;
+  a.Kblocks = (g.Kc + 7) / 8;
+  a.groups = L.groups;
+  a.b_goff = Cg;
+  a.epi = mask ? EPI_BF16_MASK : EPI_BF16;
+  a.out = out;
+  a.ld_out = L.Cin;
+  a.col_goff = Cg;
+  a.mask = mask;
+  a.ld_mask = L.Cin;
+  a.status = status;
+  const int Kd = L.K * L.K * Og;
+  if (!tmap(&d->tmB, wdg, Kd, L.Cin, static_cast<uint64_t>(Kd) * 2, 64, d->bn))
+    return false;
+  d->tmA = d->tmB;
+  return gemm_finalize(d, num_sms);
+}
+
+bool desc_conv_wgrad(GemmDesc* d, const ConvL& L, const bf16* in, const bf16* dy, float* part,
+                     int B, int splits, int num_sms, int* status) {
+  memset(d, 0, sizeof(*d));
+  const int Og = L.Og();
+  d->asrc = A_GATHER_MN;
+  d->bsrc = B_TMA_MN;
+  d->bn = pick_bn_mn(Og);
+  GemmArgs& a = d->args;
+  a.g = gather_fwd(L, in, B);
+  a.M = L.Kdim();
+  a.N = Og;
+  a.Kblocks = (a.g.Mpix + 63) / 64;
+  a.groups = L.groups;
+  a.b_goff = Og;
+  const long long tiles = 1LL * ((a.M + 127) / 128) * ((a.N + d->bn - 1) / d->bn) * a.groups;
+  a.kb_per_split = splits > 0 ? (a.Kblocks + splits - 1) / splits
+                              : pick_kbps(tiles, a.Kblocks, num_sms, 8);
+  a.epi = EPI_F32_T;
+  a.out = part;
+  a.ld_out = a.M;
+  a.group_stride = 1LL * Og * a.M;
+  a.split_stride = 1LL * L.groups * Og * a.M;
+  a.status = status;
+  if (!tmap(&d->tmB, dy, L.Cout, a.g.Mpix, static_cast<uint64_t>(L.Cout) * 2, 64, 64))
+    return false;
+  d->tmA = d->tmB;
+  return gemm_finalize(d, num_sms);
+}
+
+bool desc_fc_fwd(GemmDesc* d, const FcL& F, const bf16* x, const bf16* w, float* part, int B,
+                 int splits, int num_sms, int* status) {
+  memset(d, 0, sizeof(*d));
+  d->asrc = A_TMA_K;
+  d->bsrc = B_TMA_K;
+  d->bn = 128;
+  GemmArgs& a = d->args;
+  a.M = B;
+  a.N = F.Out;
+  a.Kblocks = (F.In + 63) / 64;
+  a.groups = 1;
+  const long long tiles = 1LL * ((B + 127) / 128) * ((F.Out + 127) / 128);
+  a.kb_per_split = splits > 0 ? (a.Kblocks + splits - 1) / splits
+                              : pick_kbps(tiles, a.Kblocks, num_sms / 2, 4);
+  a.epi = EPI_F32;
+  a.out = part;
+  a.ld_out = F.Out;
+  a.split_stride = 1LL * B * F.Out;
+  a.status = status;
+  if (!tmap(&d->tmA, x, F.In, B, static_cast<uint64_t>(F.In) * 2, 64, 128)) return false;
+  if (!tmap(&d->tmB, w, F.In, F.Out, static_cast<uint64_t>(F.In) * 2, 64, 128))
+    return false;
+  return gemm_finalize(d, num_sms);
+}
+
+bool desc_fc_dgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* w, float* part, int B,
+                   int splits, int num_sms, int* status) {
+  memset(d, 0, sizeof(*d));
+  d->asrc = A_TMA_K;
+  d->bsrc = B_TMA_MN;
+  d->bn = F.In % 256 == 0 ? 256 : 128;
+  GemmArgs& a = d->args;
+  a.M = B;
+  a.N = F.In;
+  a.Kblocks = (F.Out + 63) / 64;
+  a.groups = 1;
+  const long long tiles = 1LL * ((B + 127) / 128) * ((F.In + d->bn - 1) / d->bn);
+  a.kb_per_split = splits > 0 ? (a.Kblocks + splits - 1) / splits
+                              : pick_kbps(tiles, a.Kblocks, num_sms / 2, 4);
+  a.epi = EPI_F32;
+  a.out = part;
+  a.ld_out = F.In;
+  a.split_stride = 1LL * B * F.In;
+  a.status = status;
+  if (!tmap(&d->tmA, dz, F.Out, B, static_cast<uint64_t>(F.Out) * 2, 64, 128))
+    return false;
+  if (!tmap(&d->tmB, w, F.In, F.Out, static_cast<uint64_t>(F.In) * 2, 64, 64))
+    return false;
+  return gemm_finalize(d, num_sms);
+}
+
+bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, float* out, int B,
+                   int num_sms, int* status) {
+  memset(d, 0, sizeof(*d));
+  d->asrc = A_TMA_MN;
+  d->bsrc = B_TMA_MN;
+  d->bn = F.In % 256 == 0 ? 256 : 128;
+  GemmArgs& a = d->args;
+  a.M = F.Out;
+  a.N = F.In;
+  a.Kblocks = (B + 63) / 64;
+  a.groups = 1;
+  a.kb_per_split = a.Kblocks;
+  a.epi = EPI_F32;
+  a.out = out;
+  a.ld_out = F.In;
+  a.split_stride = 0;
+  a.status = status;
+  if (!tmap(&d->tmA, dz, F.Out, B, static_cast<uint64_t>(F.Out) * 2, 64, 64))
+    return false;
+  if (!tmap(&d->tmB, x, F.In, B, static_cast<uint64_t>(F.In) * 2, 64, 64)) return false;
+  return gemm_finalize(d, num_sms);
+}
+
+size_t desc_f32_need(const GemmDesc& d) {
+  const GemmArgs& a = d.args;
+  if (a.epi == EPI_F32_T) return static_cast<size_t>(a.splits) * a.split_stride;
+  if (a.epi == EPI_F32)
+    return a.split_stride ? static_cast<size_t>(a.splits) * a.split_stride
+                          : static_cast<size_t>(a.M) * a.ld_out;
+  return 0;
+}
+
+bool build_plan(alexnet* h, int B, Plan* P) {
+  const int ns = h->num_sms;
+  for (int l = 0; l < 5; ++l) {
+    const ConvL& L = h->conv[l];
+    if (!desc_conv_fwd(&P->cf[l], L, h->conv_input(l), h->wf[l], h->params + h->b_off[l], h->a[l],
+                       B, ns, h->status))
+      return set_err(h, "conv forward plan");
+    if (l > 0) {
+      const bf16* mask = (!h->conv[l - 1].pool) ? h->a[l - 1] : nullptr;
+      bf16* out = mask ? h->da[l - 1] : h->dp[l - 1];
+      if (!desc_conv_dgrad(&P->cd[l], L, h->da[l], h->wd[l], mask, out, B, ns, h->status))
+        return set_err(h, "conv data-gradient plan");
+    }
+    if (!desc_conv_wgrad(&P->cw[l], L, h->conv_input(l), h->da[l], h->scratch, B, 0, ns,
+                         h->status))
+      return set_err(h, "conv weight-gradient plan");
+  }
+  for (int l = 0; l < 5; ++l) {
+    const ConvL& L = h->conv[l];
+    P->conv_flops[l] = 2.0 * B * L.Ho * L.Ho * L.Cout * L.K * L.K * (L.Cin / L.groups);
+  }
+  for (int f = 0; f < 3; ++f) P->fc_flops[f] = 2.0 * B * h->fc[f].In * h->fc[f].Out;
+  const bf16* fin[3] = {h->p[4], h->f6, h->f7};
+  const bf16* dz[3] = {h->d6, h->d7, h->dlogits};
+  for (int f = 0; f < 3; ++f) {
+    if (!desc_fc_fwd(&P->ff[f], h->fc[f], fin[f], h->wf[5 + f], h->scratch, B, 0, ns, h->status))
+      return set_err(h, "fc forward plan");
+    if (!desc_fc_dgrad(&P->fd[f], h->fc[f], dz[f], h->wf[5 + f], h->scratch, B, 0, ns, h->status))
+      return set_err(h, "fc data-gradient plan");
+    if (!desc_fc_wgrad(&P->fw[f], h->fc[f], dz[f], fin[f], h->scratch, B, ns, h->status))
+      return set_err(h, "fc weight-gradient plan");
+  }
+  if (h->scratch) {
+    const GemmDesc* all[] = {&P->cw[0], &P->cw[1], &P->cw[2], &P->cw[3], &P->cw[4],
+                             &P->ff[0], &P->ff[1], &P->ff[2], &P->fd[0], &P->fd[1],
+                             &P->fd[2], &P->fw[0], &P->fw[1], &P->fw[2]};
+    for (const GemmDesc* d : all)
+      if (desc_f32_need(*d) > h->scratch_floats) return set_err(h, "scratch too small for plan");
+  }
+  P->ok = true;
+  return true;
+}
+
+// Carve every buffer of the handle out of the workspace (or size it).
+size_t carve(alexnet* h, void* base) {
+  Carver c(base);
+  const alexnet_config& cfg = h->cfg;
+  const int B = cfg.batch_max;
+  const size_t n = h->n_params;
+  float* pv = c.take<float>(2 * n);
+  h->params = pv;
+  h->vel = pv ? pv + n : nullptr;
+  h->grads = cfg.keep_grads ? c.take<float>(n) : nullptr;
+  h->hp = c.take<HParams>(1);
+  h->status = c.take<int>(4);
+  h->loss_dev = c.take<float>(4);
+  h->loss_rows = c.take<float>(B > 16 ? B : 16);
+  h->logits = c.take<float>(static_cast<size_t>(B) * kClasses);
+  h->probs = c.take<float>(static_cast<size_t>(B) * kClasses);
+  if (cfg.dtype == ALEXNET_FP32) {
+    size_t mx = 0;
+    for (int l = 0; l < 5; ++l) {
+      const ConvL& L = h->conv[l];
+      const size_t e = static_cast<size_t>(B) * L.Ho * L.Ho * L.Cout;
+      if (e > mx) mx = e;
+    }
+    const size_t xin = static_cast<size_t>(B) * 227 * 227 * 3;
+    if (xin > mx) mx = xin;
+    h->f_act = mx;
+    h->fa = c.take<float>(mx);
+    h->fb = c.take<float>(mx);
+    size_t wmax = 0;
+    for (int l = 0; l < 5; ++l) wmax = h->w_len[l] > wmax ? h->w_len[l] : wmax;
+    h->fwt = c.take<float>(wmax);
+    return c.off;
+  }
+  for (int l = 0; l < 5; ++l) {
+    const ConvL& L = h->conv[l];
+    h->wf[l] = c.take<bf16>(static_cast<size_t>(L.Cout) * L.Kdim());
+    if (l > 0) h->wd[l] = c.take<bf16>(h->w_len[l]);
+  }
+  for (int f = 0; f < 3; ++f) h->wf[5 + f] = c.take<bf16>(h->w_len[5 + f]);
+  h->xin = c.take<bf16>(static_cast<size_t>(B) * 227 * 227 * 3);
+  h->xs = c.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 48);
+  for (int l = 0; l < 5; ++l) {
+    const ConvL& L = h->conv[l];
+    const size_t e = static_cast<size_t>(B) * L.Ho * L.Ho * L.Cout;
+    const size_t ep = static_cast<size_t>(B) * L.P * L.P * L.Cout;
+    h->a[l] = c.take<bf16>(e);
+    h->da[l] = c.take<bf16>(e);
+    if (L.lrn) {
+      h->lo[l] = c.take<bf16>(e);
+      h->dl[l] = c.take<bf16>(e);
+    }
+    if (L.pool) {
+      h->p[l] = c.take<bf16>(ep);
+      h->am[l] = c.take<uint8_t>(ep);
+      h->dp[l] = c.take<bf16>(ep);
+    }
+  }
+  h->dp5 = h->dp[4];
+  h->f6 = c.take<bf16>(static_cast<size_t>(B) * 4096);
+  h->f7 = c.take<bf16>(static_cast<size_t>(B) * 4096);
+  h->dlogits = c.take<bf16>(static_cast<size_t>(B) * kClasses);
+  h->d7 = c.take<bf16>(static_cast<size_t>(B) * 4096);
+  h->d6 = c.take<bf16>(static_cast<size_t>(B) * 4096);
+  // column-sum partials for bias gradients: max over layers of chunks x cols
+  size_t cp = static_cast<size_t>(colsum_chunks(B)) * 4096;
+  for (int l = 0; l < 5; ++l) {
+    const ConvL& L = h->conv[l];
+    const size_t e = static_cast<size_t>(colsum_chunks(1LL * B * L.Ho * L.Ho)) * L.Cout;
+    if (e > cp) cp = e;
+  }
+  h->cpart_floats = cp;
+  h->cpart = c.take<float>(cp);
+  // fp32 scratch: split-K partials and FC weight gradients, sized by the
+  // plans at batch_max (smaller batches never need more)
+  {
+    alexnet tmp;
+    tmp.cfg = h->cfg;
+    tmp.num_sms = h->num_sms;
+    build_geometry(&tmp);
+    Plan P;
+    g_dry_tmaps = true;
+    const bool ok = build_plan(&tmp, B, &P);
+    g_dry_tmaps = false;
+    size_t need = 1;
+    if (ok) {
+      const GemmDesc* all[] = {&P.cw[0], &P.cw[1], &P.cw[2], &P.cw[3], &P.cw[4],
+                               &P.ff[0], &P.ff[1], &P.ff[2], &P.fd[0], &P.fd[1],
+                               &P.fd[2], &P.fw[0], &P.fw[1], &P.fw[2]};
+      for (const GemmDesc* d : all) need = desc_f32_need(*d) > need ? desc_f32_need(*d) : need;
+    }
+    h->scratch_floats = need;
+    h->scratch = c.take<float>(need);
+  }
+  return c.off;
+}
+
+void write_hp(alexnet* h, float lr, cudaStream_t s) {
+  h->hp_host.lr = lr;
+  h->hp_host.momentum = h->cfg.momentum;
+  h->hp_host.weight_decay = h->cfg.weight_decay;
+  h->hp_host.dropout_p = h->cfg.dropout_p;
+  h->hp_host.step = static_cast<uint32_t>(h->step);
+  h->hp_host.seed_lo = static_cast<uint32_t>(h->cfg.seed);
+  h->hp_host.seed_hi = static_cast<uint32_t>(h->cfg.seed >> 32);
+  const double t = static_cast<double>(h->cfg.dropout_p) * 4294967296.0 + 0.5;
+  h->hp_host.drop_thresh = t >= 4294967295.0 ? 0xFFFFFFFFu : static_cast<uint32_t>(t);
+  launch_write_hparams(h->hp, h->hp_host, s);
+}
+
+ConvMap conv_map(const alexnet* h, int l) {
+  const ConvL& L = h->conv[l];
+  ConvMap m;
+  m.Cout = L.Cout;
+  m.K = L.K;
+  m.Cg = L.Cin / L.groups;
+  m.groups = L.groups;
+  m.s2d = l == 0 ? 1 : 0;
+  return m;
+}
+
+void refresh_shadows(alexnet* h, cudaStream_t s) {
+  if (h->cfg.dtype != ALEXNET_BF16) return;
+  for (int l = 0; l < 5; ++l)
+    launch_conv_shadows(h->params + h->w_off[l], conv_map(h, l), h->wf[l], h->wd[l], s);
+  for (int f = 5; f < 8; ++f) launch_f32_to_bf16(h->params + h->w_off[f], h->wf[f], h->w_len[f], s);
+}
+
+Plan* get_plan(alexnet* h, int B) {
+  auto it = h->plans.find(B);
+  if (it != h->plans.end()) return &it->second;
+  Plan P;
+  if (!build_plan(h, B, &P)) return nullptr;
+  auto r = h->plans.emplace(B, P);
+  return &r.first->second;
+}
+
+#define ALX_TRY(expr, where)                                                 \
+  do {                                                                       \
+    cudaError_t e_ = (expr);                                                 \
+    if (e_ != cudaSuccess) return cuda_status(h, e_, where);                 \
+  } while (0)
+
+cudaError_t run_gemm(alexnet* h, const GemmDesc& d, double flops, cudaStream_t s) {
+  if (!h->stats_on) return gemm_launch(d, s);
+  if (h->ev_used + 2 > h->ev.size()) {
+    for (int i = 0; i < 2; ++i) {
+      cudaEvent_t e;
+      cudaError_t r = cudaEventCreate(&e);
+      if (r != cudaSuccess) return r;
+      h->ev.push_back(e);
+    }
+  }
+  cudaEvent_t e0 = h->ev[h->ev_used], e1 = h->ev[h->ev_used + 1];
+  h->ev_used += 2;
+  h->stats_stream = s;
+  cudaEventRecord(e0, s);
+  cudaError_t r = gemm_launch(d, s);
+  cudaEventRecord(e1, s);
+  h->gemm_launches += 1;
+  h->gemm_flops += flops;
+  return r;
+}
+
+alexnet_status forward_bf16(alexnet* h, const bf16* x, int B, int dropout_mode, float* logits,
+                            cudaStream_t s, Plan* P) {
+  launch_s2d(x, h->xs, B, s);
+  for (int l = 0; l < 5; ++l) {
+    const ConvL& L = h->conv[l];
+    ALX_TRY(run_gemm(h, P->cf[l], P->conv_flops[l], s), "conv forward launch");
+    const bf16* cur = h->a[l];
+    if (L.lrn) {
+      launch_lrn_fwd(h->a[l], h->lo[l], 1LL * B * L.Ho * L.Ho, L.Cout, h->cfg.lrn_n, h->cfg.lrn_k,
+                     h->cfg.lrn_alpha, h->cfg.lrn_beta, s);
+      cur = h->lo[l];
+    }
+    if (L.pool)
+      launch_pool_fwd(cur, h->p[l], h->am[l], B, L.Ho, L.Ho, L.Cout, h->cfg.pool_size, 2, s);
+  }
+  bf16* fout[2] = {h->f6, h->f7};
+  for (int f = 0; f < 3; ++f) {
+    ALX_TRY(run_gemm(h, P->ff[f], P->fc_flops[f], s), "fc forward launch");
+    const float* bias = h->params + h->b_off[5 + f];
+    if (f < 2)
+      launch_fc_finalize(h->scratch, P->ff[f].args.splits, B, h->fc[f].Out, bias, 1, dropout_mode,
+                         6 + f, h->hp, fout[f], nullptr, s);
+    else
+      launch_fc_finalize(h->scratch, P->ff[f].args.splits, B, h->fc[f].Out, bias, 0, 0, 8, h->hp,
+                         nullptr, logits, s);
+  }
+  return cuda_status(h, cudaGetLastError(), "forward");
+}
+
+alexnet_status forward_f32(alexnet* h, const float* x, int B, float* logits, cudaStream_t s) {
+  const float* cur = x;
+  float* bufs[2] = {h->fa, h->fb};
+  int which = 0;
+  for (int l = 0; l < 5; ++l) {
+    const ConvL& L = h->conv[l];
+    launch_conv_wt_f32(h->params + h->w_off[l], h->fwt, L.Cout, L.K, L.Cin / L.groups, L.groups, s);
+    float* y = bufs[which];
+    launch_conv_fwd_f32(cur, h->fwt, h->params + h->b_off[l], y, B, L.H, L.H, L.Cin, L.Cout, L.K,
+                        L.stride, L.pad, L.groups, L.Ho, L.Ho, s);
+    which ^= 1;
+    cur = y;
+    if (L.lrn) {
+      float* z = bufs[which];
+      launch_lrn_fwd_f32(cur, z, 1LL * B * L.Ho * L.Ho, L.Cout, 5, h->cfg.lrn_k, h->cfg.lrn_alpha,
+                         h->cfg.lrn_beta, s);
+      which ^= 1;
+      cur = z;
+    }
+    if (L.pool) {
+      float* z = bufs[which];
+      launch_pool_fwd_f32(cur, z, B, L.Ho, L.Ho, L.Cout, h->cfg.pool_size, 2, s);
+      which ^= 1;
+      cur = z;
+    }
+  }
+  const float scale = h->cfg.dropout_on ? 1.f - h->cfg.dropout_p : 1.f;
+  for (int f = 0; f < 3; ++f) {
+    float* y = f < 2 ? bufs[which] : logits;
+    launch_fc_fwd_f32(cur, h->params + h->w_off[5 + f], h->params + h->b_off[5 + f], y, B,
+                      h->fc[f].In, h->fc[f].Out, f < 2 ? 1 : 0, f < 2 ? scale : 1.f, s);
+    if (f < 2) {
+      which ^= 1;
+      cur = y;
+    }
+  }
+  return cuda_status(h, cudaGetLastError(), "forward fp32");
+}
+
+alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int B, float* loss,
+                          cudaStream_t s, Plan* P) {
+  const alexnet_config& cfg = h->cfg;
+  alexnet_status st = forward_bf16(h, x, B, cfg.dropout_on ? 1 : 0, h->logits, s, P);
+  if (st != ALEXNET_OK) return st;
+  launch_softmax_ce(h->logits, labels, B, kClasses, nullptr, h->dlogits, h->loss_rows, h->status,
+                    s);
+  launch_loss_mean(h->loss_rows, B, h->loss_dev, loss, s);
+  float* gr = h->grads;
+  auto gptr = [&](size_t off) { return gr ? gr + off : nullptr; };
+  // FC8, FC7, FC6: data gradient (old weights), then weight gradient + SGD
+  const bf16* dz[3] = {h->d6, h->d7, h->dlogits};
+  bf16* dxo[3] = {h->dp5, h->d6, h->d7};
+  const bf16* mask[3] = {nullptr, h->f6, h->f7};
+  for (int f = 2; f >= 0; --f) {
+    const FcL& F = h->fc[f];
+    ALX_TRY(run_gemm(h, P->fd[f], P->fc_flops[f], s), "fc dgrad launch");
+    launch_dgrad_finalize(h->scratch, P->fd[f].args.splits, B, F.In, mask[f], dxo[f], s);
+    ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s), "fc wgrad launch");
+    launch_sgd_dense(h->params + h->w_off[5 + f], h->vel + h->w_off[5 + f], h->scratch,
+                     h->w_len[5 + f], h->wf[5 + f], gptr(h->w_off[5 + f]), h->hp, s);
+    launch_colsum_partial(dz[f], B, F.Out, h->cpart, s);
+    launch_sgd_bias(h->params + h->b_off[5 + f], h->vel + h->b_off[5 + f], h->cpart,
+                    colsum_chunks(B), F.Out, gptr(h->b_off[5 + f]), h->hp, s);
+  }
+  // pool5 backward straight into conv5's pre-activation gradient
+  {
+    const ConvL& L = h->conv[4];
+    launch_pool_bwd(h->dp5, h->am[4], h->p[4], h->da[4], B, L.Ho, L.Ho, L.Cout, cfg.pool_size, 2,
+                    1, s);
+  }
+  for (int l = 4; l >= 0; --l) {
+    const ConvL& L = h->conv[l];
+    if (l > 0) {
+      ALX_TRY(run_gemm(h, P->cd[l], P->conv_flops[l], s), "conv dgrad launch");
+      const ConvL& Q = h->conv[l - 1];
+      if (Q.pool) {
+        // dp[l-1] = d(pooled map) -> through the pool (and LRN) to da[l-1]
+        if (Q.lrn) {
+          launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->dl[l - 1], B, Q.Ho, Q.Ho,
+                          Q.Cout, cfg.pool_size, 2, 0, s);
+        } else {
+          launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->da[l - 1], B, Q.Ho, Q.Ho,
+                          Q.Cout, cfg.pool_size, 2, 1, s);
+        }
+      }
+    }
+    ALX_TRY(run_gemm(h, P->cw[l], P->conv_flops[l], s), "conv wgrad launch");
+    launch_sgd_conv(h->params + h->w_off[l], h->vel + h->w_off[l], h->scratch,
+                    P->cw[l].args.splits, conv_map(h, l), h->wf[l], h->wd[l], gptr(h->w_off[l]),
+                    h->hp, s);
+    const long long rows = 1LL * B * L.Ho * L.Ho;
+    launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart, s);
+    launch_sgd_bias(h->params + h->b_off[l], h->vel + h->b_off[l], h->cpart, colsum_chunks(rows),
+                    L.Cout, gptr(h->b_off[l]), h->hp, s);
+    if (l > 0) {
+      const ConvL& Q = h->conv[l - 1];
+      if (Q.pool && Q.lrn)
+        launch_lrn_bwd(h->a[l - 1], h->dl[l - 1], h->da[l - 1], 1LL * B * Q.Ho * Q.Ho, Q.Cout,
+                       cfg.lrn_n, cfg.lrn_k, cfg.lrn_alpha, cfg.lrn_beta, s);
+    }
+  }
+  return cuda_status(h, cudaGetLastError(), "train step");
+}
+
+}  // namespace
+
+// ======================================================================
+// C ABI
+// ======================================================================
+extern "C" {
+
+void alexnet_default_config(alexnet_config* c) {
+  if (!c) return;
+  memset(c, 0, sizeof(*c));
+  c->batch_max = 128;
+  c->dtype = ALEXNET_BF16;
+  c->grouped = 1;
+  c->seed = 0x5EEDULL;
+  c->momentum = 0.9f;
+  c->weight_decay = 5e-4f;
+  c->dropout_p = 0.5f;
+  c->lrn_k = 2.f;
+  c->lrn_alpha = 1e-4f;
+  c->lrn_beta = 0.75f;
+  c->lrn_n = 5;
+  c->lrn_on = 1;
+  c->pool_size = 3;
+  c->dropout_on = 1;
+  c->keep_grads = 0;
+}
+
+int64_t alexnet_param_count(const alexnet_config* cfg) {
+  if (!valid_config(cfg)) return -1;
+  alexnet tmp;
+  tmp.cfg = *cfg;
+  build_geometry(&tmp);
+  return static_cast<int64_t>(tmp.n_params);
+}
+
+size_t alexnet_workspace_bytes(const alexnet_config* cfg) {
+  if (!valid_config(cfg)) return 0;
+  alexnet tmp;
+  tmp.cfg = *cfg;
+  build_geometry(&tmp);
+  return carve(&tmp, nullptr) + 256;
+}
+
+alexnet_status alexnet_create(const alexnet_config* cfg, void* workspace, size_t bytes,
+                              void* stream, alexnet_t** out) {
+  if (!out) return ALEXNET_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!valid_config(cfg)) {
+    g_create_error = "invalid config";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255)) {
+    g_create_error = "workspace must be a 256-byte aligned device pointer";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  const size_t need = alexnet_workspace_bytes(cfg);
+  if (bytes < need) {
+    g_create_error = "workspace too small";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  alexnet* h = new alexnet();
+  h->cfg = *cfg;
+  h->ws = static_cast<char*>(workspace);
+  h->ws_bytes = bytes;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  build_geometry(h);
+  carve(h, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  // initial parameters ([S] 3.4 "Training Procedure Details")
+  const int bias_one[8] = {0, 1, 0, 1, 1, 1, 1, 0};
+  for (int l = 0; l < 8; ++l) {
+    launch_init_normal(h->params + h->w_off[l], h->w_len[l], 0.01f, cfg->seed,
+                       static_cast<uint32_t>(l), s);
+    launch_fill(h->params + h->b_off[l], h->b_len[l], bias_one[l] ? 1.f : 0.f, s);
+  }
+  launch_fill(h->vel, h->n_params, 0.f, s);
+  cudaError_t e = cudaMemsetAsync(h->status, 0, sizeof(int), s);
+  if (e == cudaSuccess && h->cfg.dtype == ALEXNET_BF16 && h->wf[0])
+    e = cudaMemsetAsync(h->wf[0], 0, sizeof(bf16) * 96 * 432, s);
+  refresh_shadows(h, s);
+  write_hp(h, 0.f, s);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    g_create_error = std::string("create: ") + cudaGetErrorString(e);
+    delete h;
+    return ALEXNET_ERR_CUDA;
+  }
+  *out = h;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_forward(alexnet_t* h, const void* x, int B, alexnet_mode mode,
+                               float* logits, float* probs, void* stream) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  if (!x || !logits || B < 1 || B > h->cfg.batch_max ||
+      (mode != ALEXNET_TRAIN && mode != ALEXNET_INFERENCE)) {
+    h->err = "forward: invalid argument";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  alexnet_status st;
+  if (h->cfg.dtype == ALEXNET_FP32) {
+    if (mode == ALEXNET_TRAIN && h->cfg.dropout_on) {
+      h->err = "forward: the fp32 path serves inference only";
+      return ALEXNET_ERR_UNSUPPORTED;
+    }
+    st = forward_f32(h, static_cast<const float*>(x), B, logits, s);
+  } else {
+    Plan* P = get_plan(h, B);
+    if (!P) return ALEXNET_ERR_CUDA;
+    write_hp(h, 0.f, s);
+    const int dm = !h->cfg.dropout_on ? 0 : (mode == ALEXNET_TRAIN ? 1 : 2);
+    st = forward_bf16(h, static_cast<const bf16*>(x), B, dm, logits, s, P);
+  }
+  if (st != ALEXNET_OK) return st;
+  if (probs)
+    launch_softmax_ce(logits, nullptr, B, kClasses, probs, nullptr, nullptr, h->status, s);
+  if (logits != h->logits)
+    cudaMemcpyAsync(h->logits, logits, sizeof(float) * B * kClasses, cudaMemcpyDeviceToDevice, s);
+  return cuda_status(h, cudaGetLastError(), "forward");
+}
+
+alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* labels, int B,
+                                  float lr, float* loss, void* stream) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  if (!x || !labels || B < 1 || B > h->cfg.batch_max || !(lr >= 0.f)) {
+    h->err = "train_step: invalid argument";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  if (h->cfg.dtype != ALEXNET_BF16) {
+    h->err = "train_step: training runs on the bf16 path only";
+    return ALEXNET_ERR_UNSUPPORTED;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  Plan* P = get_plan(h, B);
+  if (!P) return ALEXNET_ERR_CUDA;
+  write_hp(h, lr, s);
+  const alexnet_status st = train_bf16(h, static_cast<const bf16*>(x), labels, B, loss, s, P);
+  if (st == ALEXNET_OK) h->step += 1;
+  return st;
+}
+
+alexnet_status alexnet_augment(alexnet_t* h, const uint8_t* src, int B, const float* mean,
+                               const float* pca_vec, const float* pca_val, void* x_out,
+                               void* stream) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  if (!src || !mean || !pca_vec || !pca_val || !x_out || B < 1) {
+    h->err = "augment: invalid argument";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  write_hp(h, h->hp_host.lr, s);
+  launch_augment(src, B, mean, pca_vec, pca_val, h->hp, static_cast<bf16*>(x_out), s);
+  return cuda_status(h, cudaGetLastError(), "augment");
+}
+
+alexnet_status alexnet_tencrop(alexnet_t* h, const uint8_t* src, int B, const float* mean,
+                               float* probs_avg, int32_t* top5, void* stream) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  if (!src || !mean || !probs_avg || !top5 || B < 1) {
+    h->err = "tencrop: invalid argument";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  if (h->cfg.dtype != ALEXNET_BF16) {
+    h->err = "tencrop: bf16 handles only";
+    return ALEXNET_ERR_UNSUPPORTED;
+  }
+  const int chunk = h->cfg.batch_max / 10;
+  if (chunk < 1) {
+    h->err = "tencrop: batch_max must be >= 10";
+    return ALEXNET_ERR_UNSUPPORTED;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  write_hp(h, 0.f, s);
+  for (int b0 = 0; b0 < B; b0 += chunk) {
+    const int nb = B - b0 < chunk ? B - b0 : chunk;
+    Plan* P = get_plan(h, nb * 10);
+    if (!P) return ALEXNET_ERR_CUDA;
+    launch_tencrop_inputs(src + static_cast<size_t>(b0) * 256 * 256 * 3, nb, mean, h->xin, s);
+    alexnet_status st = forward_bf16(h, h->xin, nb * 10, h->cfg.dropout_on ? 2 : 0, h->logits, s, P);
+    if (st != ALEXNET_OK) return st;
+    launch_softmax_ce(h->logits, nullptr, nb * 10, kClasses, h->probs, nullptr, nullptr, h->status,
+                      s);
+    launch_tencrop_reduce(h->probs, nb, kClasses, probs_avg + static_cast<size_t>(b0) * kClasses,
+                          top5 + static_cast<size_t>(b0) * 5, s);
+  }
+  return cuda_status(h, cudaGetLastError(), "tencrop");
+}
+
+size_t alexnet_params_bytes(const alexnet_t* h) {
+  return h ? 8 * h->n_params + 8 : 0;
+}
+
+alexnet_status alexnet_get_params(alexnet_t* h, void* dst, size_t bytes, void* stream) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  if (!dst || bytes < alexnet_params_bytes(h)) {
+    h->err = "get_params: invalid argument";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  ALX_TRY(cudaMemcpyAsync(dst, h->params, 8 * h->n_params, cudaMemcpyDefault, s), "get_params");
+  ALX_TRY(cudaMemcpyAsync(static_cast<char*>(dst) + 8 * h->n_params, &h->step, 8,
+                          cudaMemcpyDefault, s),
+          "get_params");
+  ALX_TRY(cudaStreamSynchronize(s), "get_params");
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_set_params(alexnet_t* h, const void* src, size_t bytes, void* stream) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  if (!src || bytes < alexnet_params_bytes(h)) {
+    h->err = "set_params: invalid argument";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  ALX_TRY(cudaMemcpyAsync(h->params, src, 8 * h->n_params, cudaMemcpyDefault, s), "set_params");
+  uint64_t step = 0;
+  ALX_TRY(cudaMemcpyAsync(&step, static_cast<const char*>(src) + 8 * h->n_params, 8,
+                          cudaMemcpyDefault, s),
+          "set_params");
+  ALX_TRY(cudaStreamSynchronize(s), "set_params");
+  h->step = step;
+  refresh_shadows(h, s);
+  return cuda_status(h, cudaGetLastError(), "set_params");
+}
+
+alexnet_status alexnet_get_grads(alexnet_t* h, float* dst, size_t n, void* stream) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  if (!h->grads) {
+    h->err = "get_grads: handle was created without keep_grads";
+    return ALEXNET_ERR_UNSUPPORTED;
+  }
+  if (!dst || n < h->n_params) {
+    h->err = "get_grads: invalid argument";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ALX_TRY(cudaMemcpyAsync(dst, h->grads, 4 * h->n_params, cudaMemcpyDefault, s), "get_grads");
+  ALX_TRY(cudaStreamSynchronize(s), "get_grads");
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_get_status(alexnet_t* h) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(h->last_stream);
+  if (e != cudaSuccess) return cuda_status(h, e, "get_status");
+  int st = 0;
+  e = cudaMemcpy(&st, h->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_status(h, e, "get_status");
+  if (st & STATUS_TIMEOUT) {
+    h->err = "a device wait ran out of time";
+    return ALEXNET_ERR_TIMEOUT;
+  }
+  if (st & STATUS_LABEL_RANGE) {
+    h->err = "a label was outside [0, 1000)";
+    return ALEXNET_ERR_LABEL_RANGE;
+  }
+  return ALEXNET_OK;
+}
+
+const char* alexnet_last_error(const alexnet_t* h) {
+  return h ? h->err.c_str() : g_create_error.c_str();
+}
+
+alexnet_status alexnet_destroy(alexnet_t* h) {
+  if (h)
+    for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+  delete h;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_stats_enable(alexnet_t* h, int enable) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  h->stats_on = enable != 0;
+  h->launch_base = launch_counter();
+  h->gemm_launches = 0;
+  h->gemm_flops = 0.0;
+  h->ev_used = 0;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_stats_read(alexnet_t* h, alexnet_stats* out) {
+  if (!h || !out) return ALEXNET_ERR_INVALID_ARG;
+  double ms = 0.0;
+  if (h->ev_used) {
+    ALX_TRY(cudaStreamSynchronize(h->stats_stream), "stats_read");
+    for (size_t i = 0; i + 1 < h->ev_used; i += 2) {
+      float t = 0.f;
+      ALX_TRY(cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]), "stats_read");
+      ms += t;
+    }
+  }
+  const int64_t now = launch_counter();
+  out->launches = now - h->launch_base;
+  out->gemm_launches = h->gemm_launches;
+  out->gemm_flops = h->gemm_flops;
+  out->gemm_ms = ms;
+  h->launch_base = now;
+  h->gemm_launches = 0;
+  h->gemm_flops = 0.0;
+  h->ev_used = 0;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst, size_t bytes, void* stream) {
+  if (!h || !dst) return ALEXNET_ERR_INVALID_ARG;
+  if (h->cfg.dtype != ALEXNET_BF16) return ALEXNET_ERR_UNSUPPORTED;
+  const int B = h->cfg.batch_max;
+  const void* src = nullptr;
+  size_t n = 0;
+  if (which >= 0 && which < 5) {
+    const ConvL& L = h->conv[which];
+    src = h->a[which];
+    n = 2ull * B * L.Ho * L.Ho * L.Cout;
+  } else if ((which == 10 || which == 11) && h->lo[which - 10]) {
+    const ConvL& L = h->conv[which - 10];
+    src = h->lo[which - 10];
+    n = 2ull * B * L.Ho * L.Ho * L.Cout;
+  } else if ((which == 20 || which == 21 || which == 24) && h->p[which - 20]) {
+    const ConvL& L = h->conv[which - 20];
+    src = h->p[which - 20];
+    n = 2ull * B * L.P * L.P * L.Cout;
+  } else if (which == 30 || which == 31) {
+    src = which == 30 ? h->f6 : h->f7;
+    n = 2ull * B * 4096;
+  } else if (which == 40) {
+    src = h->logits;
+    n = 4ull * B * kClasses;
+  } else {
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ALX_TRY(cudaMemcpyAsync(dst, src, bytes < n ? bytes : n, cudaMemcpyDefault, s), "debug_copy");
+  return ALEXNET_OK;
+}
+
+}  // extern "C"

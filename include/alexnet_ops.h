@@ -1,0 +1,144 @@
+/*
+ * alexnet_ops.h -- single-operation entry points of libalexnet.so.
+ *
+ * Each call runs exactly one stage of the network's hot path (the same
+ * kernels alexnet_train_step launches) on caller-provided tensors, so that a
+ * test can feed the oracle the very inputs the kernel saw.  All pointers are
+ * device pointers owned by the caller; `ws` is caller-owned device scratch
+ * of `ws_bytes` (a call returns ALEXNET_ERR_INVALID_ARG if it is too small);
+ * `stream` is a cudaStream_t as void*.  Calls are asynchronous.  Layouts are
+ * NHWC with channels fastest; channel counts must be multiples of 8.
+ * Pages cited as in alexnet.h ([S], [W]).
+ */
+#ifndef ALEXNET_OPS_H_
+#define ALEXNET_OPS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "alexnet.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Stride-1 convolution with zero padding, bias and ReLU ([S] 3.4 "Overall
+ * Architecture"), on the tensor cores:
+ *   y[b,oh,ow,o] = relu(bias[o] + sum x[b,oh-pad+kh,ow-pad+kw,g*Cg+ci] w[o,kh,kw,ci])
+ * x bf16 [B,H,W,Cin]; w bf16 [Cout][K][K][Cin/groups]; bias fp32 [Cout]
+ * (nullable); y bf16 [B,Ho,Wo,Cout].  relu 0/1.  Output channels per group
+ * must be one of 48, 64, 96, 128, 192, 256 or split into 192/128/256 tiles. */
+ALEXNET_API alexnet_status alexnet_op_conv_fwd(const void* x, int B, int H, int W, int Cin, const void* w,
+                                   const float* bias, int Cout, int K, int pad, int groups,
+                                   int relu, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* conv1 of the network: 11x11, stride 4, no padding, on a [B,227,227,3]
+ * input (computed as a 3x3 stride-1 convolution of its 4x4 space-to-depth
+ * form).  w bf16 [96][11][11][3]; y bf16 [B,55,55,96] = relu(conv + bias). */
+ALEXNET_API alexnet_status alexnet_op_conv1_fwd(const void* x, int B, const void* w, const float* bias,
+                                    void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Data gradient of a stride-1 convolution:
+ *   dx[b,ih,iw,c] = sum_{o,kh,kw} dy[b,ih+pad-kh,iw+pad-kw,o] w[o,kh,kw,c-g*Cg]
+ * (o in c's group), then zeroed where mask[b,ih,iw,c] <= 0 if mask != NULL
+ * (mask = the ReLU output that fed this convolution).  dy bf16 [B,H',W',Cout];
+ * dx bf16 [B,H,W,Cin] (H' = H for the layers here). */
+ALEXNET_API alexnet_status alexnet_op_conv_dgrad(const void* dy, int B, int H, int W, int Cin,
+                                     const void* w, int Cout, int K, int pad, int groups,
+                                     const void* mask, void* dx, void* ws, size_t ws_bytes,
+                                     void* stream);
+
+/* Weight gradient of a stride-1 convolution (fp32 out, canonical layout):
+ *   dw[o,kh,kw,ci] = sum_{b,oh,ow} dy[b,oh,ow,o] x[b,oh-pad+kh,ow-pad+kw,g*Cg+ci]
+ * split into `splits` K-slices (0 = automatic) summed in a fixed order. */
+ALEXNET_API alexnet_status alexnet_op_conv_wgrad(const void* x, int B, int H, int W, int Cin,
+                                     const void* dy, int Cout, int K, int pad, int groups,
+                                     int splits, float* dw, void* ws, size_t ws_bytes,
+                                     void* stream);
+
+/* conv1 weight gradient on a [B,227,227,3] input: dw fp32 [96][11][11][3]. */
+ALEXNET_API alexnet_status alexnet_op_conv1_wgrad(const void* x, int B, const void* dy, int splits,
+                                      float* dw, void* ws, size_t ws_bytes, void* stream);
+
+/* Fully-connected products (fp32 out, no bias):
+ *   fwd:   y[b,o]  = sum_i x[b,i] w[o,i]      x bf16 [B,In], w bf16 [Out,In]
+ *   dgrad: dx[b,i] = sum_o dz[b,o] w[o,i]     dz bf16 [B,Out]
+ *   wgrad: dw[o,i] = sum_b dz[b,o] x[b,i]
+ * In and Out must be multiples of 8. */
+ALEXNET_API alexnet_status alexnet_op_fc_fwd(const void* x, int B, int In, const void* w, int Out,
+                                 int splits, float* y, void* ws, size_t ws_bytes, void* stream);
+ALEXNET_API alexnet_status alexnet_op_fc_dgrad(const void* dz, int B, int Out, const void* w, int In,
+                                   int splits, float* dx, void* ws, size_t ws_bytes,
+                                   void* stream);
+ALEXNET_API alexnet_status alexnet_op_fc_wgrad(const void* dz, const void* x, int B, int Out, int In,
+                                   float* dw, void* ws, size_t ws_bytes, void* stream);
+
+/* LRN over channels ([S] 3.4 "Local Response Normalization", n = 5):
+ * b = a / (k + alpha * sum_{|j-i|<=2} a_j^2)^beta; bwd gives
+ * da = relu'(a) * (dLRN/da)^T g.  a, b, g, da bf16 [P, C]. */
+ALEXNET_API alexnet_status alexnet_op_lrn_fwd(const void* a, int64_t P, int C, float k, float alpha,
+                                  float beta, void* b, void* stream);
+ALEXNET_API alexnet_status alexnet_op_lrn_bwd(const void* a, const void* g, int64_t P, int C, float k,
+                                  float alpha, float beta, void* da, void* stream);
+
+/* Max pool z x z, stride st, no padding ([S] 3.4 "Overlapping Pooling"):
+ * y bf16 [B,Ho,Wo,C] and argmax uint8 (window offset dy*z+dx of the first
+ * maximum in row-major order).  bwd routes dy to the argmax of every window
+ * (overlaps add); relu_mask zeroes windows whose pooled value is <= 0. */
+ALEXNET_API alexnet_status alexnet_op_pool_fwd(const void* x, int B, int H, int W, int C, int z, int st,
+                                   void* y, uint8_t* argmax, void* stream);
+ALEXNET_API alexnet_status alexnet_op_pool_bwd(const void* dy, const uint8_t* argmax, const void* pooled,
+                                   int B, int H, int W, int C, int z, int st, int relu_mask,
+                                   void* dx, void* stream);
+
+/* Softmax + cross-entropy over N classes: probs fp32 [B,N] (nullable),
+ * dlogits bf16 [B,N] = (p - onehot)/B (nullable), loss fp32 scalar (mean).
+ * labels device int32 [B] (nullable: no loss, no dlogits). */
+ALEXNET_API alexnet_status alexnet_op_softmax_ce(const float* logits, const int32_t* labels, int B, int N,
+                                     float* probs, void* dlogits, float* loss, void* ws,
+                                     size_t ws_bytes, void* stream);
+
+/* Dropout keep mask (uint8 0/1, [rows, cols]) of FC `layer` (6 or 7) at
+ * `step` with key `seed` and drop probability p ([S] 3.4 "Dropout"): kept
+ * iff word (e & 3) of Philox4x32-10((e >> 2, layer, step, 0), seed) >=
+ * round(p * 2^32), e = row*cols + col. */
+ALEXNET_API alexnet_status alexnet_op_dropout_mask(uint64_t seed, uint32_t layer, uint32_t step, float p,
+                                       int rows, int cols, uint8_t* keep, void* ws,
+                                       size_t ws_bytes, void* stream);
+
+/* Raw Philox4x32-10 blocks on the device: for i < n, out[4i..4i+3] =
+ * Philox(ctr[4i..4i+3], key[2i..2i+1]).  ctr, key, out device uint32. */
+ALEXNET_API alexnet_status alexnet_op_philox(const uint32_t* ctr, const uint32_t* key, int n, uint32_t* out,
+                                 void* stream);
+
+/* One internal tensor of the handle's last forward (debug / parity):
+ * which = 0..4 conv l+1 output after ReLU, 10/11 LRN1/LRN2 output,
+ * 20/21/24 pool1/pool2/pool5 output, 30/31 FC6/FC7 output after dropout,
+ * 40 logits.  Copies min(bytes, tensor bytes) to dst (host or device). */
+ALEXNET_API alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst, size_t bytes,
+                                  void* stream);
+
+/* Launch accounting and GEMM timing of a handle's calls.  While enabled,
+ * every tensor-core GEMM launch is bracketed by CUDA events on the call's
+ * stream.  alexnet_stats_read synchronises that stream, fills *out with the
+ * totals since the previous read (or since enabling) and resets them.
+ *   launches:      kernels this library launched
+ *   gemm_launches: of which tensor-core GEMMs
+ *   gemm_flops:    algorithmic FLOPs of those GEMMs (2 x multiply-adds of
+ *                  the network's own layer shapes, padding not counted)
+ *   gemm_ms:       summed device time of those GEMM launches */
+typedef struct {
+  int64_t launches;
+  int64_t gemm_launches;
+  double gemm_flops;
+  double gemm_ms;
+} alexnet_stats;
+
+ALEXNET_API alexnet_status alexnet_stats_enable(alexnet_t* h, int enable);
+ALEXNET_API alexnet_status alexnet_stats_read(alexnet_t* h, alexnet_stats* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ALEXNET_OPS_H_ */

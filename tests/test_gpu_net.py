@@ -1,0 +1,316 @@
+"""End-to-end parity of the C-ABI network calls against the CPU oracle.
+
+Both sides get the same seeded inputs and the same parameters: the oracle
+takes the bf16-rounded weights the GPU computes with (and the fp32 biases) and
+keeps every activation in fp64.  Bounds: rel-L2 <= 2e-2 on the bf16 path
+(logits and every parameter gradient), <= 1e-4 on the fp32 path; dropout
+masks, crop offsets and reflections bit-exact; top-5 bit-exact on the GPU's
+own averaged probabilities and, end to end, wherever the oracle's margin
+between neighbouring ranks is clear of the measured error."""
+import numpy as np
+import pytest
+
+import oracle
+from deep_cnn_image_b200 import synthetic
+from tests._gpu import TOL_BF16, TOL_FP32, bf16_round, dev, host, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ax():
+    from deep_cnn_image_b200 import alexnet
+    return alexnet
+
+
+def _blob(params, n, step=0):
+    import torch
+    blob = np.zeros(2 * n + 2, dtype=np.float32)
+    blob[:n] = params
+    blob[2 * n:].view(np.uint64)[0] = step
+    return torch.from_numpy(blob)
+
+
+def _oracle_params(params, net):
+    """Weights rounded to bf16 (what the tensor cores read), biases as is."""
+    p = params.astype(np.float64).copy()
+    for (wo, wl, bo, bl) in oracle.param_layout(net):
+        p[wo:wo + wl] = bf16_round(params[wo:wo + wl])
+    return p
+
+
+def _make(ax, **cfg):
+    net = ax.AlexNet(**cfg)
+    return net
+
+
+def test_init_distribution(ax):
+    import torch
+    net = _make(ax, batch_max=2, seed=77)
+    blob = torch.zeros(net.params_bytes() // 4, dtype=torch.float32)
+    net.get_params(blob)
+    n = ax.param_count(net.cfg)
+    p = blob.numpy()[:n]
+    lay = oracle.param_layout(oracle.alexnet())
+    bias_one = [False, True, False, True, True, True, True, False]
+    allw = np.concatenate([p[wo:wo + wl] for (wo, wl, bo, bl) in lay])
+    assert abs(allw.mean()) < 1e-5 and abs(allw.std() - 0.01) < 1e-4
+    for l, (wo, wl, bo, bl) in enumerate(lay):
+        assert np.all(p[bo:bo + bl] == (1.0 if bias_one[l] else 0.0))
+        w = p[wo:wo + wl]
+        assert abs(w.std() - 0.01) < 0.01 * 6 / np.sqrt(wl) + 2e-4
+    assert np.all(blob.numpy()[n:2 * n] == 0)
+
+
+def test_forward_inference_matches_oracle(ax):
+    import torch
+    B = 3
+    net = _make(ax, batch_max=4)
+    n = ax.param_count(net.cfg)
+    params = synthetic.params(11)
+    net.set_params(_blob(params, n))
+    x = synthetic.images(12, B)
+    xt, xr = synthetic.to_bf16(x)
+    logits = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+    probs = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+    net.forward(xt.cuda(), B, ax.INFERENCE, logits, probs)
+    onet = oracle.alexnet()
+    op = _oracle_params(params, onet)
+    wl, wp = oracle.forward(onet, op, xr, mode=1)
+    # the conv1 map as a first diagnostic
+    a1 = torch.empty((4, 55, 55, 96), dtype=torch.bfloat16, device="cuda")
+    net.debug_copy(0, a1)
+    a1_want = oracle.forward_probe(onet, op, xr, oracle.PROBE_RELU + 0).reshape(B, 55, 55, 96)
+    assert rel_l2(host(a1)[:B], a1_want) < TOL_BF16
+    err = rel_l2(host(logits), wl)
+    assert err < TOL_BF16, err
+    assert rel_l2(host(probs), wp) < TOL_BF16
+    np.testing.assert_allclose(host(probs).sum(1), 1.0, rtol=1e-5)
+
+
+def test_fp32_path_matches_oracle(ax):
+    """Batch 1, fp32, ungrouped, inference (FC6/FC7 outputs x 0.5)."""
+    import torch
+    net = _make(ax, batch_max=1, dtype=ax.FP32, grouped=0)
+    n = ax.param_count(net.cfg)
+    params = synthetic.params(21, grouped=False)
+    net.set_params(_blob(params, n))
+    x = synthetic.images(22, 1)
+    logits = torch.empty((1, 1000), dtype=torch.float32, device="cuda")
+    probs = torch.empty((1, 1000), dtype=torch.float32, device="cuda")
+    net.forward(dev(x), 1, ax.INFERENCE, logits, probs)
+    wl, wp = oracle.forward(oracle.alexnet(grouped=False), params.astype(np.float64),
+                            x.astype(np.float64), mode=1)
+    err = rel_l2(host(logits), wl)
+    assert err < TOL_FP32, err
+    assert rel_l2(host(probs), wp) < TOL_FP32
+
+
+def _train_compare(ax, B, seed, grouped=True, lr=0.01):
+    import torch
+    net = _make(ax, batch_max=B, keep_grads=1, grouped=int(grouped), seed=seed)
+    n = ax.param_count(net.cfg)
+    params = synthetic.params(seed + 1, grouped=grouped)
+    step = 5
+    net.set_params(_blob(params, n, step))
+    x = synthetic.images(seed + 2, B)
+    y = synthetic.labels(seed + 3, B)
+    xt, xr = synthetic.to_bf16(x)
+    loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+    net.train_step(xt.cuda(), dev(y), B, lr, loss)
+    assert net.get_status() == ax.OK
+    grads = torch.zeros(n, dtype=torch.float32)
+    net.get_grads(grads)
+    blob = torch.zeros(net.params_bytes() // 4, dtype=torch.float32)
+    net.get_params(blob)
+    onet = oracle.alexnet(grouped=grouped)
+    op = _oracle_params(params, onet)
+    wloss, _, _, wg, _ = oracle.train_step(onet, op, np.zeros(n), xr, y, lr=lr,
+                                           seed=net.cfg.seed, step=step)
+    return net, host(loss)[0], grads.numpy(), blob.numpy(), wloss, wg, params, n, xr, y
+
+
+def test_train_step_matches_oracle(ax):
+    net, loss, g, blob, wloss, wg, params, n, xr, y = _train_compare(ax, 2, 100)
+    assert abs(loss - wloss) / wloss < 1e-2
+    names = ["conv1", "conv2", "conv3", "conv4", "conv5", "fc6", "fc7", "fc8"]
+    for l, (wo, wl, bo, bl) in enumerate(oracle.param_layout(oracle.alexnet())):
+        ew = rel_l2(g[wo:wo + wl], wg[wo:wo + wl])
+        eb = rel_l2(g[bo:bo + bl], wg[bo:bo + bl])
+        assert ew < TOL_BF16, (names[l], "W", ew)
+        assert eb < TOL_BF16, (names[l], "b", eb)
+    # the update: v = 0.9*0 - wd*lr*w - lr*g applied to the fp32 masters
+    w_new, v_new = oracle.sgd(params.astype(np.float64), np.zeros(n), wg, 0.01)
+    assert rel_l2(blob[n:2 * n], v_new) < TOL_BF16
+    assert rel_l2(blob[:n], w_new) < 1e-4
+    assert blob[2 * n:].view(np.uint64)[0] == 6
+
+
+def test_train_step_batch8_matches_oracle(ax):
+    net, loss, g, blob, wloss, wg, params, n, xr, y = _train_compare(ax, 8, 200)
+    assert abs(loss - wloss) / wloss < 1e-2
+    assert rel_l2(g, wg) < TOL_BF16
+    for l, (wo, wl, bo, bl) in enumerate(oracle.param_layout(oracle.alexnet())):
+        assert rel_l2(g[wo:wo + wl], wg[wo:wo + wl]) < TOL_BF16, l
+
+
+def test_dropout_masks_end_to_end(ax):
+    """After a training-mode forward, every unit the oracle's mask drops is
+    exactly zero in the GPU's FC6/FC7 outputs; kept units with a clearly
+    positive pre-activation are non-zero."""
+    import torch
+    B = 2
+    net = _make(ax, batch_max=B, seed=4242)
+    n = ax.param_count(net.cfg)
+    params = synthetic.params(3)
+    net.set_params(_blob(params, n, 9))
+    x = synthetic.images(4, B)
+    xt, xr = synthetic.to_bf16(x)
+    logits = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+    net.forward(xt.cuda(), B, ax.TRAIN, logits)
+    onet = oracle.alexnet()
+    op = _oracle_params(params, onet)
+    for which, layer in ((30, 6), (31, 7)):
+        f = torch.empty((B, 4096), dtype=torch.bfloat16, device="cuda")
+        net.debug_copy(which, f)
+        got = host(f)
+        keep = oracle.dropout_mask(4242, layer, 9, B, 4096)
+        assert np.all(got[keep == 0] == 0)
+        want = oracle.forward_probe(onet, op, xr, which, mode=0, seed=4242, step=9).reshape(B, 4096)
+        clear = (keep == 1) & (want > 0.05)
+        assert clear.sum() > 100 and np.all(got[clear] > 0)
+
+
+def test_full_batch_forward_sampled(ax):
+    """Batch 128 (the benchmark's batch): logits of sampled images against
+    the oracle run on those images alone (inference mode: images are
+    independent)."""
+    import torch
+    B = 128
+    net = _make(ax, batch_max=B)
+    n = ax.param_count(net.cfg)
+    params = synthetic.params(31)
+    net.set_params(_blob(params, n))
+    x = synthetic.images(32, B)
+    xt, xr = synthetic.to_bf16(x)
+    logits = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+    net.forward(xt.cuda(), B, ax.INFERENCE, logits)
+    got = host(logits)
+    assert np.all(np.isfinite(got))
+    onet = oracle.alexnet()
+    op = _oracle_params(params, onet)
+    idx = [0, 77, 127]
+    wl, _ = oracle.forward(onet, op, xr[idx], mode=1)
+    assert rel_l2(got[idx], wl) < TOL_BF16
+
+
+def test_full_batch_train_step_properties(ax):
+    """Batch 128: the loss at the pages' initialisation is close to ln(1000),
+    every gradient is finite, and two identical handles give bit-identical
+    results (the step is deterministic)."""
+    import torch
+    B = 128
+    outs = []
+    for _ in range(2):
+        net = _make(ax, batch_max=B, keep_grads=1, seed=5)
+        x = synthetic.images(6, B)
+        y = synthetic.labels(7, B)
+        xt, _ = synthetic.to_bf16(x)
+        loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+        net.train_step(xt.cuda(), dev(y), B, 0.01, loss)
+        assert net.get_status() == ax.OK
+        g = torch.zeros(ax.param_count(net.cfg), dtype=torch.float32)
+        net.get_grads(g)
+        outs.append((host(loss)[0], g.numpy().copy()))
+        net.close()
+    assert abs(outs[0][0] - np.log(1000.0)) < 0.05
+    assert np.all(np.isfinite(outs[0][1]))
+    assert outs[0][0] == outs[1][0]
+    np.testing.assert_array_equal(outs[0][1], outs[1][1])
+
+
+def test_resume_is_bit_identical(ax):
+    """k steps, get_params, a new handle, set_params, the remaining steps ==
+    the same number of steps straight through."""
+    import torch
+    B, N, k = 4, 3, 1
+    xs = [synthetic.to_bf16(synthetic.images(50 + i, B))[0].cuda() for i in range(N)]
+    ys = [dev(synthetic.labels(60 + i, B)) for i in range(N)]
+    a = _make(ax, batch_max=B, seed=9)
+    for i in range(N):
+        a.train_step(xs[i], ys[i], B, 0.01)
+    pa = torch.zeros(a.params_bytes() // 4, dtype=torch.float32)
+    a.get_params(pa)
+    b = _make(ax, batch_max=B, seed=9)
+    for i in range(k):
+        b.train_step(xs[i], ys[i], B, 0.01)
+    mid = torch.zeros(b.params_bytes() // 4, dtype=torch.float32)
+    b.get_params(mid)
+    b.close()
+    c = _make(ax, batch_max=B, seed=9)
+    c.set_params(mid)
+    for i in range(k, N):
+        c.train_step(xs[i], ys[i], B, 0.01)
+    pc = torch.zeros(c.params_bytes() // 4, dtype=torch.float32)
+    c.get_params(pc)
+    np.testing.assert_array_equal(pa.numpy(), pc.numpy())
+
+
+def test_label_out_of_range_sets_status(ax):
+    import torch
+    B = 2
+    net = _make(ax, batch_max=B)
+    xt, _ = synthetic.to_bf16(synthetic.images(1, B))
+    y = dev(np.array([3, 1000], dtype=np.int32))
+    net.train_step(xt.cuda(), y, B, 0.01)
+    assert net.get_status() == ax.ERR_LABEL_RANGE
+
+
+def test_augmentation_matches_oracle(ax):
+    import torch
+    B = 6
+    net = _make(ax, batch_max=8, seed=314)
+    n = ax.param_count(net.cfg)
+    net.set_params(_blob(synthetic.params(1), n, 17))
+    src = synthetic.source_images(8, B)
+    mean = synthetic.mean_image(src)
+    vec, val = synthetic.pca(9)
+    out = torch.empty((B, 227, 227, 3), dtype=torch.bfloat16, device="cuda")
+    net.augment(dev(src), B, dev(mean), dev(vec), dev(val), out)
+    want = oracle.augment(src, mean.astype(np.float64), vec.astype(np.float64),
+                          val.astype(np.float64), seed=314, step=17)
+    got = host(out)
+    # exact crop offsets and reflections: every element within bf16 rounding
+    assert np.all(np.abs(got - want) <= np.abs(want) * 2 ** -8 + 1e-6)
+    assert rel_l2(got, want) < 4e-3
+
+
+def test_tencrop_matches_oracle(ax):
+    import torch
+    B = 2
+    net = _make(ax, batch_max=20)
+    n = ax.param_count(net.cfg)
+    params = synthetic.params(41)
+    # a strong class signal so that the ranking is well separated
+    lay = oracle.param_layout(oracle.alexnet())
+    bo = lay[7][2]
+    params[bo:bo + 1000] = np.linspace(0, 3, 1000, dtype=np.float32)[::-1]
+    net.set_params(_blob(params, n))
+    src = synthetic.source_images(42, B)
+    mean = synthetic.mean_image(src)
+    probs = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+    top5 = torch.empty((B, 5), dtype=torch.int32, device="cuda")
+    net.tencrop(dev(src), B, dev(mean), probs, top5)
+    onet = oracle.alexnet()
+    wp, wt = oracle.tencrop(onet, _oracle_params(params, onet), src, mean.astype(np.float64))
+    gp = host(probs)
+    assert rel_l2(gp, wp) < TOL_BF16
+    # top-5 exact on the GPU's own averaged probabilities
+    np.testing.assert_array_equal(host(top5), oracle.topk(gp, 5))
+    # and against the oracle's ranking where its margins are clear
+    err = np.abs(gp - wp).max()
+    for b in range(B):
+        srt = np.sort(wp[b])[::-1]
+        for k in range(5):
+            if srt[k] - srt[k + 1] > 4 * err and (k == 0 or srt[k - 1] - srt[k] > 4 * err):
+                assert host(top5)[b, k] == wt[b, k]
