@@ -1138,6 +1138,24 @@ alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst, size_t byt
   } else if (which == 40) {
     src = h->logits;
     n = 4ull * B * kClasses;
+  } else if (which >= 50 && which < 55) {
+    const ConvL& L = h->conv[which - 50];
+    src = h->da[which - 50];
+    n = 2ull * B * L.Ho * L.Ho * L.Cout;
+  } else if (which >= 60 && which < 65 && h->dp[which - 60]) {
+    const ConvL& L = h->conv[which - 60];
+    src = h->dp[which - 60];
+    n = 2ull * B * L.P * L.P * L.Cout;
+  } else if (which >= 70 && which < 75 && h->dl[which - 70]) {
+    const ConvL& L = h->conv[which - 70];
+    src = h->dl[which - 70];
+    n = 2ull * B * L.Ho * L.Ho * L.Cout;
+  } else if (which == 80) {
+    src = h->dlogits;
+    n = 2ull * B * kClasses;
+  } else if (which == 81 || which == 82) {
+    src = which == 81 ? h->d7 : h->d6;
+    n = 2ull * B * 4096;
   } else {
     return ALEXNET_ERR_INVALID_ARG;
   }

@@ -114,7 +114,10 @@ ALEXNET_API alexnet_status alexnet_op_philox(const uint32_t* ctr, const uint32_t
 /* One internal tensor of the handle's last forward (debug / parity):
  * which = 0..4 conv l+1 output after ReLU, 10/11 LRN1/LRN2 output,
  * 20/21/24 pool1/pool2/pool5 output, 30/31 FC6/FC7 output after dropout,
- * 40 logits.  Copies min(bytes, tensor bytes) to dst (host or device). */
+ * 40 logits (fp32); gradients of the last training step (bf16):
+ * 50+l dL/d(pre-activation of conv l+1), 60+l dL/d(pooled map after conv
+ * l+1), 70+l dL/d(LRN output of conv l+1), 80 dL/dlogits, 81/82 dL/d(FC7/FC6
+ * pre-activation).  Copies min(bytes, tensor bytes) to dst (host or device). */
 ALEXNET_API alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst, size_t bytes,
                                   void* stream);
 

@@ -124,6 +124,8 @@ def lib():
             "oracle_train_step": (c_double, [netp, dp, dp, dp, i32p, c_int, c_double, c_double,
                                              c_double, c_uint64, c_uint32, dp, dp]),
             "oracle_loss": (c_double, [netp, dp, dp, i32p, c_int, c_uint64, c_uint32]),
+            "oracle_train_probe": (None, [netp, dp, dp, i32p, c_int, c_uint64, c_uint32, c_int,
+                                          dp]),
             "oracle_aug_draws": (None, [c_uint64, c_uint32, c_uint32, i32p, dp]),
             "oracle_augment": (None, [u8p, c_int, dp, dp, dp, c_uint64, c_uint32, dp]),
             "oracle_tencrop_inputs": (None, [u8p, c_int, dp, dp]),
@@ -427,6 +429,33 @@ def train_step(net, params, velocity, x, labels, lr=0.01, momentum=0.9, wd=5e-4,
                                    momentum, wd, seed, step, _p(grads, c_double),
                                    _p(logits, c_double))
     return loss, params, velocity, grads, logits
+
+
+GPROBE_DZ, GPROBE_DPOOL, GPROBE_DLRN, GPROBE_DLOGITS, GPROBE_DZ7, GPROBE_DZ6 = 50, 60, 70, 80, 81, 82
+
+
+def gprobe_size(net, which):
+    """Elements per image of the gradient train_probe returns for `which`."""
+    ms = map_sizes(net)
+    if 50 <= which < 60 or 70 <= which < 80:
+        l = which % 10
+        return ms[l][1] ** 2 * net.conv_c[l]
+    if 60 <= which < 70:
+        l = which - 60
+        return ms[l][2] ** 2 * net.conv_c[l]
+    return {80: net.fc_n[2], 81: net.fc_n[1], 82: net.fc_n[0]}[which]
+
+
+def train_probe(net, params, x, labels, which, seed=0, step=0):
+    """One intermediate gradient of a training step (see oracle_train_probe), flat."""
+    params, pp = _d(params)
+    x, xp = _d(x)
+    labels = np.ascontiguousarray(labels, dtype=np.int32)
+    B = x.shape[0]
+    out = np.zeros(B * gprobe_size(net, which))
+    lib().oracle_train_probe(ctypes.byref(net), pp, xp, _p(labels, ctypes.c_int32), B, seed, step,
+                             which, _p(out, c_double))
+    return out
 
 
 def loss(net, params, x, labels, seed=0, step=0):

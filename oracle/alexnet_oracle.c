@@ -733,10 +733,44 @@ ORACLE_API void oracle_forward_probe(const oracle_net* net, const double* params
  * velocity are updated in place; grads (nullable) receives dL/dparams at the
  * pre-update weights; logits (nullable) receives the forward logits.
  * Returns the loss. */
+static double train_step_probe(const oracle_net* net, double* params, double* velocity,
+                               const double* x, const int32_t* labels, int B, double lr,
+                               double momentum, double wd, uint64_t seed, uint32_t step,
+                               double* grads, double* logits, int probe, double* probe_out);
+
 ORACLE_API double oracle_train_step(const oracle_net* net, double* params, double* velocity,
                                     const double* x, const int32_t* labels, int B, double lr,
                                     double momentum, double wd, uint64_t seed, uint32_t step,
                                     double* grads, double* logits) {
+  return train_step_probe(net, params, velocity, x, labels, B, lr, momentum, wd, seed, step,
+                          grads, logits, -1, NULL);
+}
+
+/* Intermediate gradients of a training step (no update is kept):
+ *   50+l  dL/d(pre-activation of conv l)      60+l dL/d(pooled map of conv l)
+ *   70+l  dL/d(LRN output of conv l)          80 dL/dlogits, 81/82 dL/d(FC7/FC6
+ *   pre-activation) */
+ORACLE_API void oracle_train_probe(const oracle_net* net, const double* params, const double* x,
+                                   const int32_t* labels, int B, uint64_t seed, uint32_t step,
+                                   int which, double* out) {
+  oracle_shapes s;
+  net_shapes(net, &s);
+  double* p = dalloc(s.n_params);
+  double* v = dalloc(s.n_params);
+  memcpy(p, params, sizeof(double) * (size_t)s.n_params);
+  train_step_probe(net, p, v, x, labels, B, 0.0, 0.0, 0.0, seed, step, NULL, NULL, which, out);
+  free(p);
+  free(v);
+}
+
+static void probe_copy(int probe, int which, const double* src, int64_t n, double* out) {
+  if (probe == which && out) memcpy(out, src, sizeof(double) * (size_t)n);
+}
+
+static double train_step_probe(const oracle_net* net, double* params, double* velocity,
+                               const double* x, const int32_t* labels, int B, double lr,
+                               double momentum, double wd, uint64_t seed, uint32_t step,
+                               double* grads, double* logits, int probe, double* probe_out) {
   fwd_cache c;
   net_forward(net, params, x, B, 0, seed, step, &c);
   const oracle_shapes* s = &c.s;
@@ -745,6 +779,7 @@ ORACLE_API double oracle_train_step(const oracle_net* net, double* params, doubl
   double* g = dalloc(s->n_params);
   double* dz = dalloc((int64_t)B * N);
   const double loss = oracle_softmax_ce(c.logits, labels, B, N, NULL, dz);
+  probe_copy(probe, 80, dz, (int64_t)B * N, probe_out);
 
   /* FC8, FC7, FC6 */
   double* dcur = dz;
@@ -765,6 +800,7 @@ ORACLE_API double oracle_train_step(const oracle_net* net, double* params, doubl
         dcur[e] = d;
       }
       oracle_relu_bwd(c.fc_relu[f - 1], dcur, n);
+      probe_copy(probe, 80 + (3 - f), dcur, n, probe_out);
     }
   }
   /* conv5 ... conv1: dcur is dL/d(pooled or last map of layer l) */
@@ -773,18 +809,21 @@ ORACLE_API double oracle_train_step(const oracle_net* net, double* params, doubl
     const int64_t n = (int64_t)B * O * O * Co;
     if (net->pool_after[l]) {
       double* d = dalloc(n);
+      probe_copy(probe, 60 + l, dcur, (int64_t)B * s->pool_out[l] * s->pool_out[l] * Co, probe_out);
       oracle_maxpool_bwd(dcur, c.argmax[l], B, O, O, Co, net->pool_z, net->pool_s, d);
       free(dcur);
       dcur = d;
     }
     if (net->lrn_after[l]) {
       double* d = dalloc(n);
+      probe_copy(probe, 70 + l, dcur, n, probe_out);
       oracle_lrn_bwd(c.relu_out[l], dcur, (int64_t)B * O * O, Co, net->lrn_n, net->lrn_k,
                      net->lrn_alpha, net->lrn_beta, d);
       free(dcur);
       dcur = d;
     }
     oracle_relu_bwd(c.relu_out[l], dcur, n);
+    probe_copy(probe, 50 + l, dcur, n, probe_out);
     const int H = s->hw[l];
     const int Ci = l == 0 ? net->in_c : net->conv_c[l - 1];
     double* dx = l > 0 ? dalloc((int64_t)B * H * H * Ci) : NULL;
