@@ -40,19 +40,6 @@ __host__ __device__ constexpr int tmem_cols_for(int bn) {
   return 2 * bn <= 32 ? 32 : (2 * bn <= 64 ? 64 : (2 * bn <= 128 ? 128 : (2 * bn <= 256 ? 256 : 512)));
 }
 
-__device__ __forceinline__ void cp_async_wait_dyn(int n) {
-  switch (n) {
-    case 0: cp_async_wait<0>(); break;
-    case 1: cp_async_wait<1>(); break;
-    case 2: cp_async_wait<2>(); break;
-    case 3: cp_async_wait<3>(); break;
-    case 4: cp_async_wait<4>(); break;
-    case 5: cp_async_wait<5>(); break;
-    case 6: cp_async_wait<6>(); break;
-    default: cp_async_wait<7>(); break;
-  }
-}
-
 struct TileCoord {
   int m_t, n_t, sp, g;
 };
@@ -120,12 +107,39 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, const TileCoor
         *reinterpret_cast<float4*>(out + col) =
             make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
-  } else {  // EPI_F32_T
+  } else if (a.epi == EPI_F32_T) {
     float* out = reinterpret_cast<float*>(a.out) + tc.sp * a.split_stride + g * a.group_stride;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int col = col0 + i;
       if (col < a.N) out[col * a.ld_out + row] = v[i];
+    }
+  } else {  // EPI_SGD: [S] 3.4 "Training Procedure Details" update rule
+    const float lr = a.hp->lr, mom = a.hp->momentum, wd = a.hp->weight_decay;
+    const long long base = static_cast<long long>(row) * a.ld_out;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = col0 + 4 * q;
+      if (col >= a.N) continue;
+      float4 w4 = *reinterpret_cast<const float4*>(a.sgd_w + base + col);
+      float4 v4 = *reinterpret_cast<const float4*>(a.sgd_v + base + col);
+      float* wp = reinterpret_cast<float*>(&w4);
+      float* vp = reinterpret_cast<float*>(&v4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float vn = mom * vp[i] - wd * lr * wp[i] - lr * v[4 * q + i];
+        vp[i] = vn;
+        wp[i] = wp[i] + vn;
+      }
+      *reinterpret_cast<float4*>(a.sgd_w + base + col) = w4;
+      *reinterpret_cast<float4*>(a.sgd_v + base + col) = v4;
+      uint2 h;
+      h.x = pack_bf16x2(wp[0], wp[1]);
+      h.y = pack_bf16x2(wp[2], wp[3]);
+      *reinterpret_cast<uint2*>(a.sgd_shadow + base + col) = h;
+      if (a.sgd_grads)
+        *reinterpret_cast<float4*>(a.sgd_grads + base + col) =
+            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
   }
 }
@@ -264,7 +278,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int t = threadIdx.x - 128;
       const int c = t & 7;
       const GatherDesc& G = args.g;
-      const int lag = stages - 1;
       uint32_t it = 0;
       bool ok = true;
       const int HoWo = G.Ho * G.Wo;
@@ -317,12 +330,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   okp ? base + (static_cast<long long>(pbase[j] + ih) * G.W + iw) * G.C : G.src;
               cp_async_16(dst0 + r * 128 + ((c ^ (r & 7)) << 4), src, okp ? 16u : 0u);
             }
-            cp_async_commit();
-            if (static_cast<int>(it) >= lag) {
-              cp_async_wait_dyn(lag);
-              fence_proxy_async_smem();
-              mbar_arrive(bar_full + 8 * ((it - lag) % stages));
-            }
+            // the stage counts as full once these copies have landed
+            cp_async_arrive(bar_full + 8 * s);
+            mbar_arrive(bar_full + 8 * s);
           }
         } else {
           // A_GATHER_MN: rows are output pixels (the reduction), the two
@@ -372,22 +382,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             okp ? 16u : 0u);
               }
             }
-            cp_async_commit();
-            if (static_cast<int>(it) >= lag) {
-              cp_async_wait_dyn(lag);
-              fence_proxy_async_smem();
-              mbar_arrive(bar_full + 8 * ((it - lag) % stages));
-            }
+            cp_async_arrive(bar_full + 8 * s);
+            mbar_arrive(bar_full + 8 * s);
           }
         }
       }
-      // drain: the last `lag` stages
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      if (ok) {
-        const uint32_t first = it > static_cast<uint32_t>(lag) ? it - lag : 0;
-        for (uint32_t i = first; i < it; ++i) mbar_arrive(bar_full + 8 * (i % stages));
-      }
+      // no copy may still be landing in shared memory when the CTA exits
+      cp_async_wait_all();
     }
   } else {
     // ------------------------------------------------------------ epilogue

@@ -51,11 +51,10 @@ __global__ void k_write_hparams(HParams* hp, HParams v) { *hp = v; }
 
 // ------------------------------------------------------------------ s2d
 __global__ void k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs, int B) {
-  const long long n = 1LL * B * 57 * 57 * 6;
-  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
-       t += 1LL * gridDim.x * blockDim.x) {
+  const uint32_t n = static_cast<uint32_t>(B) * 57 * 57 * 6;
+  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
     const int chunk = static_cast<int>(t % 6);
-    long long pix = t / 6;
+    const uint32_t pix = t / 6;
     const int j = static_cast<int>(pix % 57);
     const int i = static_cast<int>((pix / 57) % 57);
     const int b = static_cast<int>(pix / (57 * 57));
@@ -69,7 +68,7 @@ __global__ void k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs, int B) 
                  ? __bfloat162float(x[((static_cast<long long>(b) * 227 + y) * 227 + xx) * 3 + c])
                  : 0.f;
     }
-    *reinterpret_cast<uint4*>(xs + pix * 48 + chunk * 8) = pack8(f);
+    *reinterpret_cast<uint4*>(xs + static_cast<size_t>(pix) * 48 + chunk * 8) = pack8(f);
   }
 }
 
@@ -78,13 +77,12 @@ __global__ void k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs, int B) 
 // with the window clipped to the layer's channels (n = 5).
 __global__ void k_lrn_fwd(const bf16* __restrict__ a, bf16* __restrict__ b, long long P, int C,
                           float k, float alpha, float beta) {
-  const int chunks = C >> 3;
-  const long long n = P * chunks;
-  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
-       t += 1LL * gridDim.x * blockDim.x) {
-    const long long p = t / chunks;
+  const uint32_t chunks = static_cast<uint32_t>(C) >> 3;
+  const uint32_t n = static_cast<uint32_t>(P) * chunks;
+  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
+    const uint32_t p = t / chunks;
     const int c0 = static_cast<int>(t - p * chunks) * 8;
-    const bf16* ap = a + p * C;
+    const bf16* ap = a + static_cast<size_t>(p) * C;
     float v[12];
     {
       float f[8];
@@ -113,9 +111,9 @@ __global__ void k_lrn_fwd(const bf16* __restrict__ a, bf16* __restrict__ b, long
 #pragma unroll
       for (int j = 0; j < 5; ++j) sum += v[i + j] * v[i + j];
       const float s = k + alpha * sum;
-      o[i] = v[i + 2] * powf(s, -beta);
+      o[i] = v[i + 2] * __powf(s, -beta);
     }
-    *reinterpret_cast<uint4*>(b + p * C + c0) = pack8(o);
+    *reinterpret_cast<uint4*>(b + static_cast<size_t>(p) * C + c0) = pack8(o);
   }
 }
 
@@ -124,14 +122,13 @@ __global__ void k_lrn_fwd(const bf16* __restrict__ a, bf16* __restrict__ b, long
 __global__ void k_lrn_bwd(const bf16* __restrict__ a, const bf16* __restrict__ g,
                           bf16* __restrict__ da, long long P, int C, float k, float alpha,
                           float beta) {
-  const int chunks = C >> 3;
-  const long long n = P * chunks;
-  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
-       t += 1LL * gridDim.x * blockDim.x) {
-    const long long p = t / chunks;
+  const uint32_t chunks = static_cast<uint32_t>(C) >> 3;
+  const uint32_t n = static_cast<uint32_t>(P) * chunks;
+  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
+    const uint32_t p = t / chunks;
     const int c0 = static_cast<int>(t - p * chunks) * 8;
-    const bf16* ap = a + p * C;
-    const bf16* gp = g + p * C;
+    const bf16* ap = a + static_cast<size_t>(p) * C;
+    const bf16* gp = g + static_cast<size_t>(p) * C;
     float av[16];  // channels c0-4 .. c0+11
     float gv[12];  // channels c0-2 .. c0+9
 #pragma unroll
@@ -167,7 +164,7 @@ __global__ void k_lrn_bwd(const bf16* __restrict__ a, const bf16* __restrict__ g
 #pragma unroll
       for (int j = 0; j < 5; ++j) sum += av[i + j] * av[i + j];
       const float s = k + alpha * sum;
-      const float sb = powf(s, -beta);
+      const float sb = __powf(s, -beta);
       sp[i] = sb;
       tt[i] = gv[i] * av[i + 2] * (sb / s);
     }
@@ -181,7 +178,7 @@ __global__ void k_lrn_bwd(const bf16* __restrict__ a, const bf16* __restrict__ g
       const float d = gv[j + 2] * sp[j + 2] - 2.f * alpha * beta * aj * cross;
       o[j] = aj > 0.f ? d : 0.f;
     }
-    *reinterpret_cast<uint4*>(da + p * C + c0) = pack8(o);
+    *reinterpret_cast<uint4*>(da + static_cast<size_t>(p) * C + c0) = pack8(o);
   }
 }
 
@@ -203,24 +200,23 @@ __global__ void k_lrn_fwd_f32(const float* __restrict__ a, float* __restrict__ b
 // [S] 3.4 "Overlapping Pooling": max over z x z windows at stride st, no padding.
 __global__ void k_pool_fwd(const bf16* __restrict__ x, bf16* __restrict__ y,
                            uint8_t* __restrict__ am, int B, int H, int W, int C, int z, int st) {
-  const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
-  const int chunks = C >> 3;
-  const long long n = 1LL * B * Ho * Wo * chunks;
-  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
-       t += 1LL * gridDim.x * blockDim.x) {
-    const int c0 = static_cast<int>(t % chunks) * 8;
-    const long long pix = t / chunks;
-    const int ow = static_cast<int>(pix % Wo);
-    const int oh = static_cast<int>((pix / Wo) % Ho);
-    const int b = static_cast<int>(pix / (1LL * Wo * Ho));
+  const uint32_t Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
+  const uint32_t chunks = static_cast<uint32_t>(C) >> 3;
+  const uint32_t n = static_cast<uint32_t>(B) * Ho * Wo * chunks;
+  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
+    const uint32_t pix = t / chunks;
+    const int c0 = static_cast<int>(t - pix * chunks) * 8;
+    const uint32_t ow = pix % Wo;
+    const uint32_t q = pix / Wo;
+    const uint32_t oh = q % Ho;
+    const uint32_t b = q / Ho;
     float best[8];
     int arg[8];
+    const bf16* xb = x + (static_cast<size_t>(b * H + oh * st) * W + ow * st) * C + c0;
     for (int dy = 0; dy < z; ++dy)
       for (int dx = 0; dx < z; ++dx) {
         float f[8];
-        unpack8(*reinterpret_cast<const uint4*>(
-                    x + ((1LL * b * H + oh * st + dy) * W + ow * st + dx) * C + c0),
-                f);
+        unpack8(*reinterpret_cast<const uint4*>(xb + (static_cast<size_t>(dy) * W + dx) * C), f);
         const int off = dy * z + dx;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -230,11 +226,11 @@ __global__ void k_pool_fwd(const bf16* __restrict__ x, bf16* __restrict__ y,
           }
         }
       }
-    *reinterpret_cast<uint4*>(y + pix * C + c0) = pack8(best);
+    *reinterpret_cast<uint4*>(y + static_cast<size_t>(pix) * C + c0) = pack8(best);
     uint2 packed;
     packed.x = arg[0] | (arg[1] << 8) | (arg[2] << 16) | (arg[3] << 24);
     packed.y = arg[4] | (arg[5] << 8) | (arg[6] << 16) | (arg[7] << 24);
-    *reinterpret_cast<uint2*>(am + pix * C + c0) = packed;
+    *reinterpret_cast<uint2*>(am + static_cast<size_t>(pix) * C + c0) = packed;
   }
 }
 
@@ -242,15 +238,15 @@ __global__ void k_pool_bwd(const bf16* __restrict__ dy, const uint8_t* __restric
                            const bf16* __restrict__ pooled, bf16* __restrict__ dx, int B, int H,
                            int W, int C, int z, int st, int relu_mask) {
   const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
-  const int chunks = C >> 3;
-  const long long n = 1LL * B * H * W * chunks;
-  for (long long t = blockIdx.x * 1LL * blockDim.x + threadIdx.x; t < n;
-       t += 1LL * gridDim.x * blockDim.x) {
-    const int c0 = static_cast<int>(t % chunks) * 8;
-    const long long pix = t / chunks;
+  const uint32_t chunks = static_cast<uint32_t>(C) >> 3;
+  const uint32_t n = static_cast<uint32_t>(B) * H * W * chunks;
+  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
+    const uint32_t pix = t / chunks;
+    const int c0 = static_cast<int>(t - pix * chunks) * 8;
     const int iw = static_cast<int>(pix % W);
-    const int ih = static_cast<int>((pix / W) % H);
-    const int b = static_cast<int>(pix / (1LL * W * H));
+    const uint32_t q = pix / W;
+    const int ih = static_cast<int>(q % H);
+    const int b = static_cast<int>(q / H);
     const int oh_lo = ih < z ? 0 : (ih - z + st) / st;
     const int oh_hi = min(Ho - 1, ih / st);
     const int ow_lo = iw < z ? 0 : (iw - z + st) / st;
@@ -260,22 +256,26 @@ __global__ void k_pool_bwd(const bf16* __restrict__ dy, const uint8_t* __restric
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     for (int oh = oh_lo; oh <= oh_hi; ++oh)
       for (int ow = ow_lo; ow <= ow_hi; ++ow) {
-        const long long o = ((1LL * b * Ho + oh) * Wo + ow) * C + c0;
+        const size_t o = (static_cast<size_t>(b * Ho + oh) * Wo + ow) * C + c0;
         const int off = (ih - oh * st) * z + (iw - ow * st);
         const uint2 a2 = *reinterpret_cast<const uint2*>(am + o);
         float g[8];
         unpack8(*reinterpret_cast<const uint4*>(dy + o), g);
         float pv[8];
-        if (relu_mask) unpack8(*reinterpret_cast<const uint4*>(pooled + o), pv);
+        if (relu_mask) {
+          unpack8(*reinterpret_cast<const uint4*>(pooled + o), pv);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pv[i] = 1.f;
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint32_t word = i < 4 ? a2.x : a2.y;
           const int ai = (word >> (8 * (i & 3))) & 0xFF;
-          const bool take = ai == off && (!relu_mask || pv[i] > 0.f);
-          if (take) acc[i] += g[i];
+          if (ai == off && pv[i] > 0.f) acc[i] += g[i];
         }
       }
-    *reinterpret_cast<uint4*>(dx + pix * C + c0) = pack8(acc);
+    *reinterpret_cast<uint4*>(dx + static_cast<size_t>(pix) * C + c0) = pack8(acc);
   }
 }
 
@@ -320,7 +320,7 @@ __global__ void k_fc_finalize(const float* __restrict__ part, int S, int rows, i
   for (long long q = blockIdx.x * 1LL * blockDim.x + threadIdx.x; q < n4;
        q += 1LL * gridDim.x * blockDim.x) {
     const long long e = q * 4;
-    const int col = static_cast<int>(e % cols);
+    const int col = static_cast<int>(static_cast<uint32_t>(e) % static_cast<uint32_t>(cols));
     float4 acc = *reinterpret_cast<const float4*>(part + e);
     for (int s = 1; s < S; ++s) {
       const float4 p = *reinterpret_cast<const float4*>(part + s * plane + e);
@@ -498,9 +498,10 @@ struct ConvIdx {
 };
 
 // canonical p = ((o*K + kh)*K + kw)*Cg + ci
-__device__ __forceinline__ ConvIdx conv_index(const ConvMap& m, long long p) {
+__device__ __forceinline__ ConvIdx conv_index(const ConvMap& m, long long p64) {
+  const uint32_t p = static_cast<uint32_t>(p64);
   const int ci = static_cast<int>(p % m.Cg);
-  long long t = p / m.Cg;
+  uint32_t t = p / m.Cg;
   const int kw = static_cast<int>(t % m.K);
   t /= m.K;
   const int kh = static_cast<int>(t % m.K);
@@ -515,7 +516,7 @@ __device__ __forceinline__ ConvIdx conv_index(const ConvMap& m, long long p) {
     r.part_inner = kg;
     r.dg = -1;
   } else {
-    r.fwd = p;
+    r.fwd = p64;
     r.part_inner = (1LL * kh * m.K + kw) * m.Cg + ci;
     r.dg = (((1LL * r.g * m.Cg + ci) * m.K + (m.K - 1 - kh)) * m.K + (m.K - 1 - kw)) * Og + r.co;
   }
@@ -590,14 +591,20 @@ __global__ void k_sgd_bias(float* __restrict__ b, float* __restrict__ v,
                            const float* __restrict__ partial, int chunks, int n, float* grads_out,
                            const HParams* __restrict__ hpp) {
   const HParams hp = *hpp;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < n; i += warps) {
     float g = 0.f;
-    for (int c = 0; c < chunks; ++c) g += partial[1LL * c * n + i];
-    float wv = b[i], vv = v[i];
-    sgd_one(wv, vv, g, hp);
-    b[i] = wv;
-    v[i] = vv;
-    if (grads_out) grads_out[i] = g;
+    for (int c = lane; c < chunks; c += 32) g += partial[static_cast<size_t>(c) * n + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) g += __shfl_xor_sync(0xffffffffu, g, o);
+    if (lane == 0) {
+      float wv = b[i], vv = v[i];
+      sgd_one(wv, vv, g, hp);
+      b[i] = wv;
+      v[i] = vv;
+      if (grads_out) grads_out[i] = g;
+    }
   }
 }
 
@@ -957,7 +964,8 @@ void launch_sgd_dense(float* w, float* v, const float* g, long long n, bf16* sha
 }
 void launch_sgd_bias(float* b, float* v, const float* partial, int chunks, int n, float* grads_out,
                      const HParams* hp, cudaStream_t s) {
-  k_sgd_bias<<<grid_for(n, 256), 256, 0, s>>>(b, v, partial, chunks, n, grads_out, hp);
+  k_sgd_bias<<<grid_for(static_cast<long long>(n) * 32, 256), 256, 0, s>>>(b, v, partial, chunks,
+                                                                           n, grads_out, hp);
   count_launch();
 }
 void launch_conv_shadows(const float* w, const ConvMap& m, bf16* fwd, bf16* dg, cudaStream_t s) {

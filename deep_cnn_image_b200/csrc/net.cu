@@ -430,8 +430,11 @@ bool desc_fc_dgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* w, flo
   return gemm_finalize(d, num_sms);
 }
 
-bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, float* out, int B,
-                   int num_sms, int* status) {
+// FC weight gradient with the SGD update fused into the epilogue: the fp32
+// gradient never reaches memory (optionally kept in `grads` for checks).
+bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, float* w, float* v,
+                   bf16* shadow, float* grads, const HParams* hp, int B, int num_sms,
+                   int* status) {
   memset(d, 0, sizeof(*d));
   d->asrc = A_TMA_MN;
   d->bsrc = B_TMA_MN;
@@ -442,10 +445,13 @@ bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, flo
   a.Kblocks = (B + 63) / 64;
   a.groups = 1;
   a.kb_per_split = a.Kblocks;
-  a.epi = EPI_F32;
-  a.out = out;
+  a.epi = EPI_SGD;
   a.ld_out = F.In;
-  a.split_stride = 0;
+  a.sgd_w = w;
+  a.sgd_v = v;
+  a.sgd_shadow = shadow;
+  a.sgd_grads = grads;
+  a.hp = hp;
   a.status = status;
   if (!tmap(&d->tmA, dz, F.Out, B, static_cast<uint64_t>(F.Out) * 2, 64, 64))
     return false;
@@ -491,7 +497,10 @@ bool build_plan(alexnet* h, int B, Plan* P) {
       return set_err(h, "fc forward plan");
     if (!desc_fc_dgrad(&P->fd[f], h->fc[f], dz[f], h->wf[5 + f], h->scratch, B, 0, ns, h->status))
       return set_err(h, "fc data-gradient plan");
-    if (!desc_fc_wgrad(&P->fw[f], h->fc[f], dz[f], fin[f], h->scratch, B, ns, h->status))
+    const size_t wo = h->w_off[5 + f];
+    if (!desc_fc_wgrad(&P->fw[f], h->fc[f], dz[f], fin[f], h->params ? h->params + wo : nullptr,
+                       h->vel ? h->vel + wo : nullptr, h->wf[5 + f],
+                       h->grads ? h->grads + wo : nullptr, h->hp, B, ns, h->status))
       return set_err(h, "fc weight-gradient plan");
   }
   if (h->scratch) {
@@ -754,9 +763,7 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     const FcL& F = h->fc[f];
     ALX_TRY(run_gemm(h, P->fd[f], P->fc_flops[f], s), "fc dgrad launch");
     launch_dgrad_finalize(h->scratch, P->fd[f].args.splits, B, F.In, mask[f], dxo[f], s);
-    ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s), "fc wgrad launch");
-    launch_sgd_dense(h->params + h->w_off[5 + f], h->vel + h->w_off[5 + f], h->scratch,
-                     h->w_len[5 + f], h->wf[5 + f], gptr(h->w_off[5 + f]), h->hp, s);
+    ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s), "fc wgrad + SGD launch");
     launch_colsum_partial(dz[f], B, F.Out, h->cpart, s);
     launch_sgd_bias(h->params + h->b_off[5 + f], h->vel + h->b_off[5 + f], h->cpart,
                     colsum_chunks(B), F.Out, gptr(h->b_off[5 + f]), h->hp, s);
@@ -1156,6 +1163,10 @@ alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst, size_t byt
   } else if (which == 81 || which == 82) {
     src = which == 81 ? h->d7 : h->d6;
     n = 2ull * B * 4096;
+  } else if ((which == 90 || which == 91 || which == 94) && h->am[which - 90]) {
+    const ConvL& L = h->conv[which - 90];
+    src = h->am[which - 90];
+    n = 1ull * B * L.P * L.P * L.Cout;
   } else {
     return ALEXNET_ERR_INVALID_ARG;
   }

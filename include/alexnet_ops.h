@@ -117,7 +117,9 @@ ALEXNET_API alexnet_status alexnet_op_philox(const uint32_t* ctr, const uint32_t
  * 40 logits (fp32); gradients of the last training step (bf16):
  * 50+l dL/d(pre-activation of conv l+1), 60+l dL/d(pooled map after conv
  * l+1), 70+l dL/d(LRN output of conv l+1), 80 dL/dlogits, 81/82 dL/d(FC7/FC6
- * pre-activation).  Copies min(bytes, tensor bytes) to dst (host or device). */
+ * pre-activation); 90/91/94 the uint8 window choices (argmax) of the pools
+ * after conv1/conv2/conv5.  Copies min(bytes, tensor bytes) to dst (host or
+ * device). */
 ALEXNET_API alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst, size_t bytes,
                                   void* stream);
 

@@ -125,7 +125,12 @@ def lib():
                                              c_double, c_uint64, c_uint32, dp, dp]),
             "oracle_loss": (c_double, [netp, dp, dp, i32p, c_int, c_uint64, c_uint32]),
             "oracle_train_probe": (None, [netp, dp, dp, i32p, c_int, c_uint64, c_uint32, c_int,
-                                          dp]),
+                                          dp, u8p, u8p, u8p]),
+            "oracle_train_step_given": (c_double, [netp, dp, dp, dp, i32p, c_int, c_double,
+                                                   c_double, c_double, c_uint64, c_uint32, dp, dp,
+                                                   u8p, u8p, u8p]),
+            "oracle_maxpool_select": (None, [dp, u8p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                             dp]),
             "oracle_aug_draws": (None, [c_uint64, c_uint32, c_uint32, i32p, dp]),
             "oracle_augment": (None, [u8p, c_int, dp, dp, dp, c_uint64, c_uint32, dp]),
             "oracle_tencrop_inputs": (None, [u8p, c_int, dp, dp]),
@@ -414,9 +419,11 @@ def forward_probe(net, params, x, which, mode=1, seed=0, step=0):
 
 
 def train_step(net, params, velocity, x, labels, lr=0.01, momentum=0.9, wd=5e-4, seed=0,
-               step=0):
+               step=0, given_argmax=None):
     """One step of [W] TRAIN_STEP.  Returns (loss, new_params, new_velocity,
-    grads, logits)."""
+    grads, logits).  given_argmax: optional {0|1|4: uint8 map} of pool window
+    choices (for instance an implementation's own) used instead of the
+    oracle's."""
     params = np.array(params, dtype=np.float64, copy=True)
     velocity = np.array(velocity, dtype=np.float64, copy=True)
     x, xp = _d(x)
@@ -424,10 +431,11 @@ def train_step(net, params, velocity, x, labels, lr=0.01, momentum=0.9, wd=5e-4,
     B = x.shape[0]
     grads = np.zeros_like(params)
     logits = np.zeros((B, net.fc_n[2]))
-    loss = lib().oracle_train_step(ctypes.byref(net), _p(params, c_double),
-                                   _p(velocity, c_double), xp, _p(labels, ctypes.c_int32), B, lr,
-                                   momentum, wd, seed, step, _p(grads, c_double),
-                                   _p(logits, c_double))
+    keep, ptrs = _am_ptrs(given_argmax)
+    loss = lib().oracle_train_step_given(ctypes.byref(net), _p(params, c_double),
+                                         _p(velocity, c_double), xp, _p(labels, ctypes.c_int32),
+                                         B, lr, momentum, wd, seed, step, _p(grads, c_double),
+                                         _p(logits, c_double), *ptrs)
     return loss, params, velocity, grads, logits
 
 
@@ -446,16 +454,44 @@ def gprobe_size(net, which):
     return {80: net.fc_n[2], 81: net.fc_n[1], 82: net.fc_n[0]}[which]
 
 
-def train_probe(net, params, x, labels, which, seed=0, step=0):
-    """One intermediate gradient of a training step (see oracle_train_probe), flat."""
+def _am_ptrs(given):
+    """given: None or dict {0: am1, 1: am2, 4: am5} of uint8 window choices."""
+    given = given or {}
+    keep, ptrs = [], []
+    for l in (0, 1, 4):
+        a = given.get(l)
+        if a is None:
+            ptrs.append(None)
+        else:
+            a = np.ascontiguousarray(a, dtype=np.uint8)
+            keep.append(a)
+            ptrs.append(_p(a, c_uint8))
+    return keep, ptrs
+
+
+def train_probe(net, params, x, labels, which, seed=0, step=0, given_argmax=None):
+    """One intermediate gradient of a training step (see oracle_train_probe), flat.
+    given_argmax: optional {0|1|4: uint8 map} of pool window choices to use."""
     params, pp = _d(params)
     x, xp = _d(x)
     labels = np.ascontiguousarray(labels, dtype=np.int32)
     B = x.shape[0]
     out = np.zeros(B * gprobe_size(net, which))
+    keep, ptrs = _am_ptrs(given_argmax)
     lib().oracle_train_probe(ctypes.byref(net), pp, xp, _p(labels, ctypes.c_int32), B, seed, step,
-                             which, _p(out, c_double))
+                             which, _p(out, c_double), *ptrs)
     return out
+
+
+def maxpool_select(x, argmax, z=3, s=2):
+    """Pooled map taking the given window choice (argmax) in every window."""
+    x, xp = _d(x)
+    argmax = np.ascontiguousarray(argmax, dtype=np.uint8)
+    B, H, W, C = x.shape
+    Ho, Wo = (H - z) // s + 1, (W - z) // s + 1
+    y = np.zeros((B, Ho, Wo, C))
+    lib().oracle_maxpool_select(xp, _p(argmax, c_uint8), B, H, W, C, z, s, _p(y, c_double))
+    return y
 
 
 def loss(net, params, x, labels, seed=0, step=0):

@@ -353,6 +353,23 @@ ORACLE_API void oracle_maxpool_fwd(const double* x, int B, int H, int W, int C, 
         }
 }
 
+/* Pooling with the window choice given (argmax from elsewhere, e.g. the
+ * decision of an implementation that stores its maps in a lower precision):
+ * y = x at the named window offset. */
+ORACLE_API void oracle_maxpool_select(const double* x, const uint8_t* argmax, int B, int H, int W,
+                                      int C, int z, int s, double* y) {
+  const int Ho = oracle_pool_out_size(H, z, s), Wo = oracle_pool_out_size(W, z, s);
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int oh = 0; oh < Ho; ++oh)
+      for (int ow = 0; ow < Wo; ++ow)
+        for (int c = 0; c < C; ++c) {
+          const size_t o = (((size_t)b * Ho + oh) * Wo + ow) * C + c;
+          const int a = argmax[o];
+          y[o] = x[(((size_t)b * H + oh * s + a / z) * W + ow * s + a % z) * C + c];
+        }
+}
+
 /* The gradient of each window goes to the input element its argmax names;
  * overlapping windows add their contributions. */
 ORACLE_API void oracle_maxpool_bwd(const double* dy, const uint8_t* argmax, int B, int H, int W,
@@ -614,8 +631,20 @@ static void cache_free(fwd_cache* c) {
 }
 
 /* mode: 0 = training (dropout masks drawn), 1 = inference (x (1-p)). */
+static void net_forward_given(const oracle_net* net, const double* params, const double* x,
+                              int B, int mode, uint64_t seed, uint32_t step,
+                              const uint8_t* const* am_in, fwd_cache* c);
+
 static void net_forward(const oracle_net* net, const double* params, const double* x, int B,
                         int mode, uint64_t seed, uint32_t step, fwd_cache* c) {
+  net_forward_given(net, params, x, B, mode, seed, step, NULL, c);
+}
+
+/* am_in (nullable; entries nullable): window choices of the max-pools after
+ * conv l, used instead of the oracle's own argmax. */
+static void net_forward_given(const oracle_net* net, const double* params, const double* x,
+                              int B, int mode, uint64_t seed, uint32_t step,
+                              const uint8_t* const* am_in, fwd_cache* c) {
   memset(c, 0, sizeof(*c));
   net_shapes(net, &c->s);
   const oracle_shapes* s = &c->s;
@@ -642,8 +671,14 @@ static void net_forward(const oracle_net* net, const double* params, const doubl
       const int64_t np = (int64_t)B * P * P * Co;
       c->pool_out[l] = dalloc(np);
       c->argmax[l] = (uint8_t*)calloc((size_t)np, 1);
-      oracle_maxpool_fwd(cur, B, O, O, Co, net->pool_z, net->pool_s, c->pool_out[l],
-                         c->argmax[l]);
+      if (am_in && am_in[l]) {
+        memcpy(c->argmax[l], am_in[l], (size_t)np);
+        oracle_maxpool_select(cur, c->argmax[l], B, O, O, Co, net->pool_z, net->pool_s,
+                              c->pool_out[l]);
+      } else {
+        oracle_maxpool_fwd(cur, B, O, O, Co, net->pool_z, net->pool_s, c->pool_out[l],
+                           c->argmax[l]);
+      }
       cur = c->pool_out[l];
     }
     if (l < 4) {
@@ -736,14 +771,28 @@ ORACLE_API void oracle_forward_probe(const oracle_net* net, const double* params
 static double train_step_probe(const oracle_net* net, double* params, double* velocity,
                                const double* x, const int32_t* labels, int B, double lr,
                                double momentum, double wd, uint64_t seed, uint32_t step,
-                               double* grads, double* logits, int probe, double* probe_out);
+                               double* grads, double* logits, int probe, double* probe_out,
+                               const uint8_t* const* am_in);
 
 ORACLE_API double oracle_train_step(const oracle_net* net, double* params, double* velocity,
                                     const double* x, const int32_t* labels, int B, double lr,
                                     double momentum, double wd, uint64_t seed, uint32_t step,
                                     double* grads, double* logits) {
   return train_step_probe(net, params, velocity, x, labels, B, lr, momentum, wd, seed, step,
-                          grads, logits, -1, NULL);
+                          grads, logits, -1, NULL, NULL);
+}
+
+/* The same step with the max-pool window choices given (am1, am2, am5 for the
+ * pools after conv1, conv2, conv5; each nullable). */
+ORACLE_API double oracle_train_step_given(const oracle_net* net, double* params, double* velocity,
+                                          const double* x, const int32_t* labels, int B,
+                                          double lr, double momentum, double wd, uint64_t seed,
+                                          uint32_t step, double* grads, double* logits,
+                                          const uint8_t* am1, const uint8_t* am2,
+                                          const uint8_t* am5) {
+  const uint8_t* am_in[5] = {am1, am2, NULL, NULL, am5};
+  return train_step_probe(net, params, velocity, x, labels, B, lr, momentum, wd, seed, step,
+                          grads, logits, -1, NULL, am_in);
 }
 
 /* Intermediate gradients of a training step (no update is kept):
@@ -752,13 +801,16 @@ ORACLE_API double oracle_train_step(const oracle_net* net, double* params, doubl
  *   pre-activation) */
 ORACLE_API void oracle_train_probe(const oracle_net* net, const double* params, const double* x,
                                    const int32_t* labels, int B, uint64_t seed, uint32_t step,
-                                   int which, double* out) {
+                                   int which, double* out, const uint8_t* am1,
+                                   const uint8_t* am2, const uint8_t* am5) {
+  const uint8_t* am_in[5] = {am1, am2, NULL, NULL, am5};
   oracle_shapes s;
   net_shapes(net, &s);
   double* p = dalloc(s.n_params);
   double* v = dalloc(s.n_params);
   memcpy(p, params, sizeof(double) * (size_t)s.n_params);
-  train_step_probe(net, p, v, x, labels, B, 0.0, 0.0, 0.0, seed, step, NULL, NULL, which, out);
+  train_step_probe(net, p, v, x, labels, B, 0.0, 0.0, 0.0, seed, step, NULL, NULL, which, out,
+                   am_in);
   free(p);
   free(v);
 }
@@ -770,9 +822,10 @@ static void probe_copy(int probe, int which, const double* src, int64_t n, doubl
 static double train_step_probe(const oracle_net* net, double* params, double* velocity,
                                const double* x, const int32_t* labels, int B, double lr,
                                double momentum, double wd, uint64_t seed, uint32_t step,
-                               double* grads, double* logits, int probe, double* probe_out) {
+                               double* grads, double* logits, int probe, double* probe_out,
+                               const uint8_t* const* am_in) {
   fwd_cache c;
-  net_forward(net, params, x, B, 0, seed, step, &c);
+  net_forward_given(net, params, x, B, 0, seed, step, am_in, &c);
   const oracle_shapes* s = &c.s;
   const int N = net->fc_n[2];
   if (logits) memcpy(logits, c.logits, sizeof(double) * (size_t)B * N);

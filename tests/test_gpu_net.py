@@ -44,6 +44,40 @@ def _make(ax, **cfg):
     return net
 
 
+POOLS = ((0, oracle.PROBE_LRN + 0, 55, 96), (1, oracle.PROBE_LRN + 1, 27, 256),
+         (4, oracle.PROBE_RELU + 4, 13, 256))
+
+
+def _gpu_pool_choices(net, B):
+    """The GPU's own max-pool window choices of its last forward."""
+    import torch
+    out = {}
+    for l, _, side, C in POOLS:
+        P = (side - 3) // 2 + 1
+        t = torch.empty(B * P * P * C, dtype=torch.uint8, device="cuda")
+        net.debug_copy(90 + l, t)
+        torch.cuda.synchronize()
+        out[l] = t.cpu().numpy().reshape(B, P, P, C)
+    return out
+
+
+def _check_choices_valid(onet, op, xr, choices, seed, step):
+    """Each GPU window choice must be a maximum of the oracle's own map at
+    bf16 resolution (within 2 bf16 units of the window's maximum); returns the
+    fraction of windows where it is also the oracle's fp64 argmax."""
+    B = xr.shape[0]
+    same = []
+    for l, which, side, C in POOLS:
+        m = oracle.forward_probe(onet, op, xr, which, mode=0, seed=seed, step=step)
+        m = m.reshape(B, side, side, C)
+        _, own = oracle.maxpool_fwd(m)
+        sel = oracle.maxpool_select(m, choices[l])
+        mx = oracle.maxpool_fwd(m)[0]
+        assert np.all(sel >= mx - 2 * 2.0 ** -8 * np.abs(mx) - 1e-30), l
+        same.append(float((own == choices[l]).mean()))
+    return same
+
+
 def test_init_distribution(ax):
     import torch
     net = _make(ax, batch_max=2, seed=77)
@@ -107,6 +141,10 @@ def test_fp32_path_matches_oracle(ax):
 
 
 def _train_compare(ax, B, seed, grouped=True, lr=0.01):
+    """One GPU training step and the oracle's step on the same inputs.  The
+    max-pool window choices are a decision taken on rounded values: the
+    oracle takes the GPU's own choices after checking each one is a maximum
+    of its own map at bf16 resolution (identical inputs to that decision)."""
     import torch
     net = _make(ax, batch_max=B, keep_grads=1, grouped=int(grouped), seed=seed)
     n = ax.param_count(net.cfg)
@@ -125,8 +163,11 @@ def _train_compare(ax, B, seed, grouped=True, lr=0.01):
     net.get_params(blob)
     onet = oracle.alexnet(grouped=grouped)
     op = _oracle_params(params, onet)
+    choices = _gpu_pool_choices(net, B)
+    _check_choices_valid(onet, op, xr, choices, net.cfg.seed, step)
     wloss, _, _, wg, _ = oracle.train_step(onet, op, np.zeros(n), xr, y, lr=lr,
-                                           seed=net.cfg.seed, step=step)
+                                           seed=net.cfg.seed, step=step, given_argmax=choices)
+    net.choices = choices
     return net, host(loss)[0], grads.numpy(), blob.numpy(), wloss, wg, params, n, xr, y
 
 
@@ -164,7 +205,8 @@ def test_train_intermediate_gradients(ax):
         t = torch.empty(B * size, dtype=torch.bfloat16, device="cuda")
         net.debug_copy(which, t)
         got[which] = host(t)
-        want = oracle.train_probe(onet, op, xr, y, which, seed=seed, step=step)
+        want = oracle.train_probe(onet, op, xr, y, which, seed=seed, step=step,
+                                  given_argmax=net.choices)
         errs[which] = rel_l2(got[which], want)
     bad = {k: v for k, v in errs.items() if not v < TOL_BF16}
     assert not bad, (bad, errs)

@@ -326,6 +326,37 @@ def test_train_step_gradients_finite_difference():
     assert bad <= 2, (bad, checked)
 
 
+def test_given_pool_choices_reproduce_the_oracle_step():
+    """Passing the oracle's own pool window choices back in changes nothing;
+    maxpool_select with the argmax of maxpool_fwd gives the pooled map."""
+    r = np.random.default_rng(17)
+    x = r.standard_normal((2, 13, 13, 8))
+    y, am = oracle.maxpool_fwd(x)
+    np.testing.assert_array_equal(oracle.maxpool_select(x, am), y)
+    net = oracle.small_net()
+    n = oracle.param_count(net)
+    params = r.standard_normal(n) * 0.2
+    xi = r.standard_normal((2, 67, 67, 3))
+    lab = np.array([3, 4], np.int32)
+    own = {}
+    for l, which, side in ((0, oracle.PROBE_LRN + 0, 15), (1, oracle.PROBE_LRN + 1, 7),
+                           (4, oracle.PROBE_RELU + 4, 3)):
+        C = net.conv_c[l]
+        m = oracle.forward_probe(net, params, xi, which, mode=0, seed=2, step=1).reshape(2, side, side, C)
+        own[l] = oracle.maxpool_fwd(m)[1]
+    a = oracle.train_step(net, params, np.zeros(n), xi, lab, seed=2, step=1)
+    b = oracle.train_step(net, params, np.zeros(n), xi, lab, seed=2, step=1, given_argmax=own)
+    assert a[0] == b[0]
+    np.testing.assert_array_equal(a[3], b[3])
+    # a different (still in-window) choice changes the gradients below that pool
+    other = dict(own)
+    other[4] = (own[4] + 1) % 9
+    c = oracle.train_step(net, params, np.zeros(n), xi, lab, seed=2, step=1, given_argmax=other)
+    lay = oracle.param_layout(net)
+    wo, wl = lay[4][0], lay[4][1]
+    assert not np.allclose(c[3][wo:wo + wl], a[3][wo:wo + wl])
+
+
 def test_dropout_gradient_follows_mask():
     """Units dropped in FC6 get exactly zero gradient in FC6's weights' rows
     for every image where they are dropped: with batch 1 the whole row is 0."""
