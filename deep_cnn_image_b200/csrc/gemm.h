@@ -31,8 +31,8 @@ enum Epi : int {
   EPI_BF16_MASK = 1,  // out_bf16[row, col] = acc if mask[row, col] > 0 else 0
   EPI_F32 = 2,        // out_f32[split][group][row, col] = acc
   EPI_F32_T = 3,      // out_f32[split][group][col, row] = acc
-  EPI_SGD = 4,        // acc is dL/dw[row, col]: SGD update of w, v (fp32, ld_out apart)
-                      // and of the bf16 copy; grads[row, col] = acc if grads != nullptr
+  EPI_SGD = 4,        // acc[row, col] is dL/dw of parameter col * ld_out + row: SGD update
+                      // of w, v (fp32) and of the bf16 copy; grads[...] = acc if non-null
 };
 
 struct HParams;
@@ -94,6 +94,9 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
 // Fill grid/smem/stages of a descriptor whose asrc/bsrc/bn/args are set.
 // Returns false for an unsupported combination.
 bool gemm_finalize(GemmDesc* d, int num_sms);
+
+// Set the kernels' shared-memory attribute once (before any stream capture).
+cudaError_t gemm_prepare();
 
 cudaError_t gemm_launch(const GemmDesc& d, cudaStream_t stream);
 

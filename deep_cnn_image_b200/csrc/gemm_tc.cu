@@ -115,31 +115,30 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, const TileCoor
       if (col < a.N) out[col * a.ld_out + row] = v[i];
     }
   } else {  // EPI_SGD: [S] 3.4 "Training Procedure Details" update rule
+    // acc[row, col] is dL/dw for the parameter at col * ld_out + row: for a
+    // fixed column the 32 lanes of a warp touch 32 consecutive parameters.
     const float lr = a.hp->lr, mom = a.hp->momentum, wd = a.hp->weight_decay;
-    const long long base = static_cast<long long>(row) * a.ld_out;
+    float wv[16], vv[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int col = col0 + 4 * q;
-      if (col >= a.N) continue;
-      float4 w4 = *reinterpret_cast<const float4*>(a.sgd_w + base + col);
-      float4 v4 = *reinterpret_cast<const float4*>(a.sgd_v + base + col);
-      float* wp = reinterpret_cast<float*>(&w4);
-      float* vp = reinterpret_cast<float*>(&v4);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float vn = mom * vp[i] - wd * lr * wp[i] - lr * v[4 * q + i];
-        vp[i] = vn;
-        wp[i] = wp[i] + vn;
+    for (int i = 0; i < 16; ++i) {
+      const int col = col0 + i;
+      if (col < a.N) {
+        const long long idx = static_cast<long long>(col) * a.ld_out + row;
+        wv[i] = a.sgd_w[idx];
+        vv[i] = a.sgd_v[idx];
       }
-      *reinterpret_cast<float4*>(a.sgd_w + base + col) = w4;
-      *reinterpret_cast<float4*>(a.sgd_v + base + col) = v4;
-      uint2 h;
-      h.x = pack_bf16x2(wp[0], wp[1]);
-      h.y = pack_bf16x2(wp[2], wp[3]);
-      *reinterpret_cast<uint2*>(a.sgd_shadow + base + col) = h;
-      if (a.sgd_grads)
-        *reinterpret_cast<float4*>(a.sgd_grads + base + col) =
-            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int col = col0 + i;
+      if (col >= a.N) continue;
+      const long long idx = static_cast<long long>(col) * a.ld_out + row;
+      const float vn = mom * vv[i] - wd * lr * wv[i] - lr * v[i];
+      const float wn = wv[i] + vn;
+      a.sgd_w[idx] = wn;
+      a.sgd_v[idx] = vn;
+      a.sgd_shadow[idx] = __float2bfloat16_rn(wn);
+      if (a.sgd_grads) a.sgd_grads[idx] = v[i];
     }
   }
 }
@@ -508,6 +507,17 @@ bool gemm_finalize(GemmDesc* d, int num_sms) {
   const long long tiles = 1LL * a.m_tiles * a.n_tiles * a.splits * a.groups;
   d->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   return true;
+}
+
+cudaError_t gemm_prepare() {
+  for (auto& k : g_kernels) {
+    if (k.attr_set) continue;
+    cudaError_t e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         227 * 1024);
+    if (e != cudaSuccess) return e;
+    k.attr_set = true;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t gemm_launch(const GemmDesc& d, cudaStream_t stream) {

@@ -872,6 +872,7 @@ std::atomic<int64_t> g_launches{0};
 }
 int64_t launch_counter() { return g_launches.load(); }
 void count_launch() { g_launches.fetch_add(1); }
+void count_launch_n(int64_t n) { g_launches.fetch_add(n); }
 
 void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s) {
   k_write_hparams<<<1, 1, 0, s>>>(hp, v);

@@ -33,6 +33,7 @@ struct ConvMap {
 // Kernels launched by this library so far (all launchers and GEMMs).
 int64_t launch_counter();
 void count_launch();
+void count_launch_n(int64_t n);
 
 void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s);
 

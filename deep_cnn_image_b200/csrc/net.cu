@@ -139,6 +139,13 @@ struct alexnet {
   HParams hp_host;
   std::map<int, Plan> plans;
 
+  // CUDA graphs of the training step, one per batch size (see train_step)
+  int32_t* labels_buf = nullptr;
+  cudaStream_t cap_stream = nullptr;
+  std::map<int, cudaGraphExec_t> train_graphs;
+  std::map<int, int64_t> graph_kernels;  // kernels in each captured step
+  bool use_graphs = true;
+
   // launch accounting (alexnet_stats_*)
   bool stats_on = false;
   int64_t launch_base = 0;
@@ -431,17 +438,19 @@ bool desc_fc_dgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* w, flo
 }
 
 // FC weight gradient with the SGD update fused into the epilogue: the fp32
-// gradient never reaches memory (optionally kept in `grads` for checks).
+// gradient never reaches memory (optionally kept in `grads` for checks).  The
+// product is computed transposed, D[i, o] = sum_b x[b, i] dz[b, o], so that a
+// warp's lanes (rows) address consecutive weights w[o][i].
 bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, float* w, float* v,
                    bf16* shadow, float* grads, const HParams* hp, int B, int num_sms,
                    int* status) {
   memset(d, 0, sizeof(*d));
   d->asrc = A_TMA_MN;
   d->bsrc = B_TMA_MN;
-  d->bn = F.In % 256 == 0 ? 256 : 128;
+  d->bn = 256;
   GemmArgs& a = d->args;
-  a.M = F.Out;
-  a.N = F.In;
+  a.M = F.In;
+  a.N = F.Out;
   a.Kblocks = (B + 63) / 64;
   a.groups = 1;
   a.kb_per_split = a.Kblocks;
@@ -453,9 +462,8 @@ bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, flo
   a.sgd_grads = grads;
   a.hp = hp;
   a.status = status;
-  if (!tmap(&d->tmA, dz, F.Out, B, static_cast<uint64_t>(F.Out) * 2, 64, 64))
-    return false;
-  if (!tmap(&d->tmB, x, F.In, B, static_cast<uint64_t>(F.In) * 2, 64, 64)) return false;
+  if (!tmap(&d->tmA, x, F.In, B, static_cast<uint64_t>(F.In) * 2, 64, 64)) return false;
+  if (!tmap(&d->tmB, dz, F.Out, B, static_cast<uint64_t>(F.Out) * 2, 64, 64)) return false;
   return gemm_finalize(d, num_sms);
 }
 
@@ -528,6 +536,7 @@ size_t carve(alexnet* h, void* base) {
   h->status = c.take<int>(4);
   h->loss_dev = c.take<float>(4);
   h->loss_rows = c.take<float>(B > 16 ? B : 16);
+  h->labels_buf = c.take<int32_t>(B > 16 ? B : 16);
   h->logits = c.take<float>(static_cast<size_t>(B) * kClasses);
   h->probs = c.take<float>(static_cast<size_t>(B) * kClasses);
   if (cfg.dtype == ALEXNET_FP32) {
@@ -677,9 +686,10 @@ cudaError_t run_gemm(alexnet* h, const GemmDesc& d, double flops, cudaStream_t s
   return r;
 }
 
+// x == nullptr: the space-to-depth input xs is already in place.
 alexnet_status forward_bf16(alexnet* h, const bf16* x, int B, int dropout_mode, float* logits,
                             cudaStream_t s, Plan* P) {
-  launch_s2d(x, h->xs, B, s);
+  if (x) launch_s2d(x, h->xs, B, s);
   for (int l = 0; l < 5; ++l) {
     const ConvL& L = h->conv[l];
     ALX_TRY(run_gemm(h, P->cf[l], P->conv_flops[l], s), "conv forward launch");
@@ -749,6 +759,7 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
                           cudaStream_t s, Plan* P) {
   const alexnet_config& cfg = h->cfg;
   alexnet_status st = forward_bf16(h, x, B, cfg.dropout_on ? 1 : 0, h->logits, s, P);
+  // (x == nullptr: the caller converted the input already)
   if (st != ALEXNET_OK) return st;
   launch_softmax_ce(h->logits, labels, B, kClasses, nullptr, h->dlogits, h->loss_rows, h->status,
                     s);
@@ -879,6 +890,11 @@ alexnet_status alexnet_create(const alexnet_config* cfg, void* workspace, size_t
   carve(h, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->last_stream = s;
+  if (cudaError_t pe = gemm_prepare()) {
+    g_create_error = std::string("create: ") + cudaGetErrorString(pe);
+    delete h;
+    return ALEXNET_ERR_CUDA;
+  }
   // initial parameters ([S] 3.4 "Training Procedure Details")
   const int bias_one[8] = {0, 1, 0, 1, 1, 1, 1, 0};
   for (int l = 0; l < 8; ++l) {
@@ -949,10 +965,50 @@ alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* la
   h->last_stream = s;
   Plan* P = get_plan(h, B);
   if (!P) return ALEXNET_ERR_CUDA;
+  // Everything that depends on the call's arguments runs outside the graph:
+  // the hyper-parameters (lr, step), the input conversion, the labels copy
+  // and the loss copy.  The graph itself only touches the workspace.
   write_hp(h, lr, s);
-  const alexnet_status st = train_bf16(h, static_cast<const bf16*>(x), labels, B, loss, s, P);
-  if (st == ALEXNET_OK) h->step += 1;
-  return st;
+  launch_s2d(static_cast<const bf16*>(x), h->xs, B, s);
+  ALX_TRY(cudaMemcpyAsync(h->labels_buf, labels, sizeof(int32_t) * B, cudaMemcpyDeviceToDevice, s),
+          "train_step labels");
+  alexnet_status st = ALEXNET_OK;
+  if (h->use_graphs && !h->stats_on) {
+    auto it = h->train_graphs.find(B);
+    if (it == h->train_graphs.end()) {
+      if (!h->cap_stream)
+        ALX_TRY(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking), "capture stream");
+      ALX_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal),
+              "begin capture");
+      const int64_t c0 = launch_counter();
+      st = train_bf16(h, nullptr, h->labels_buf, B, nullptr, h->cap_stream, P);
+      // captured kernels are counted when a replay runs them, not now
+      h->graph_kernels[B] = launch_counter() - c0;
+      count_launch_n(-(launch_counter() - c0));
+      cudaGraph_t g = nullptr;
+      const cudaError_t ce = cudaStreamEndCapture(h->cap_stream, &g);
+      if (st != ALEXNET_OK) {
+        if (g) cudaGraphDestroy(g);
+        return st;
+      }
+      ALX_TRY(ce, "end capture");
+      cudaGraphExec_t ex = nullptr;
+      const cudaError_t ie = cudaGraphInstantiate(&ex, g, 0);
+      cudaGraphDestroy(g);
+      ALX_TRY(ie, "graph instantiate");
+      it = h->train_graphs.emplace(B, ex).first;
+    }
+    ALX_TRY(cudaGraphLaunch(it->second, s), "graph launch");
+    count_launch_n(h->graph_kernels[B]);
+  } else {
+    st = train_bf16(h, nullptr, h->labels_buf, B, nullptr, s, P);
+  }
+  if (st != ALEXNET_OK) return st;
+  if (loss)
+    ALX_TRY(cudaMemcpyAsync(loss, h->loss_dev, sizeof(float), cudaMemcpyDeviceToDevice, s),
+            "train_step loss");
+  h->step += 1;
+  return cuda_status(h, cudaGetLastError(), "train step");
 }
 
 alexnet_status alexnet_augment(alexnet_t* h, const uint8_t* src, int B, const float* mean,
@@ -1082,8 +1138,11 @@ const char* alexnet_last_error(const alexnet_t* h) {
 }
 
 alexnet_status alexnet_destroy(alexnet_t* h) {
-  if (h)
+  if (h) {
     for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+    for (auto& kv : h->train_graphs) cudaGraphExecDestroy(kv.second);
+    if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  }
   delete h;
   return ALEXNET_OK;
 }

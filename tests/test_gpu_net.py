@@ -64,7 +64,10 @@ def _gpu_pool_choices(net, B):
 def _check_choices_valid(onet, op, xr, choices, seed, step):
     """Each GPU window choice must be a maximum of the oracle's own map at
     bf16 resolution (within 2 bf16 units of the window's maximum); returns the
-    fraction of windows where it is also the oracle's fp64 argmax."""
+    fraction of windows where it is also the oracle's fp64 argmax.  Bound:
+    the GPU's stored map is within 1 bf16 unit of the oracle's (its inputs
+    were rounded once, its output once), so a valid choice is at most 2 units
+    (2 x 2^-7 relative) below the oracle's window maximum."""
     B = xr.shape[0]
     same = []
     for l, which, side, C in POOLS:
@@ -73,7 +76,8 @@ def _check_choices_valid(onet, op, xr, choices, seed, step):
         _, own = oracle.maxpool_fwd(m)
         sel = oracle.maxpool_select(m, choices[l])
         mx = oracle.maxpool_fwd(m)[0]
-        assert np.all(sel >= mx - 2 * 2.0 ** -8 * np.abs(mx) - 1e-30), l
+        deficit = (mx - sel) / np.maximum(np.abs(mx), 1e-30)
+        assert deficit.max() <= 2.0 ** -6, (l, float(deficit.max()))
         same.append(float((own == choices[l]).mean()))
     return same
 
