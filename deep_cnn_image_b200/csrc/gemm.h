@@ -24,7 +24,14 @@
 
 namespace alx {
 
-enum ASrc : int { A_TMA_K = 0, A_TMA_MN = 1, A_GATHER_K = 2, A_GATHER_MN = 3 };
+enum ASrc : int {
+  A_TMA_K = 0,
+  A_TMA_MN = 1,
+  A_GATHER_K = 2,
+  A_GATHER_MN = 3,
+  A_IM2COL_K = 4,   // conv operand by TMA im2col: rows = output pixels, 64 channels of one tap
+  A_IM2COL_MN = 5,  // its transpose for weight gradients: rows = pixels (the reduction)
+};
 enum BSrc : int { B_TMA_K = 0, B_TMA_MN = 1 };
 enum Epi : int {
   EPI_BF16 = 0,       // out_bf16[row, col] = act(acc + bias[col])
@@ -46,6 +53,7 @@ struct GatherDesc {
   int Ho, Wo;                // output map size
   int Kc;                    // number of 8-channel tap chunks = KH * KW * Cg8
   int Mpix;                  // B * Ho * Wo
+  int cpt;                   // im2col modes: 64-channel chunks per tap (K = taps * cpt * 64)
 };
 
 struct GemmArgs {
@@ -90,6 +98,12 @@ struct GemmDesc {
 // box_outer elements.  Returns false if the driver rejects it.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+
+// im2col tensor map over an NHWC bf16 tensor [N, H, W, C] for a stride-1
+// K x K convolution with zero padding `pad` (both sides): 64 channels per
+// pixel, `pixels` pixels per load, 128-byte swizzle.
+bool make_tmap_im2col(CUtensorMap* m, const void* base, int N, int H, int W, int C, int K,
+                      int pad, int pixels);
 
 // Fill grid/smem/stages of a descriptor whose asrc/bsrc/bn/args are set.
 // Returns false for an unsupported combination.

@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr int B_TILE_BYTES = BN * BK * 2;
   constexpr int TMEM_COLS = tmem_cols_for(BN);
   constexpr bool A_GATHER = (ASRC == A_GATHER_K || ASRC == A_GATHER_MN);
-  constexpr int A_MN = (ASRC == A_TMA_MN || ASRC == A_GATHER_MN) ? 1 : 0;
+  constexpr int A_MN = (ASRC == A_TMA_MN || ASRC == A_GATHER_MN || ASRC == A_IM2COL_MN) ? 1 : 0;
   constexpr int B_MN = (BSRC == B_TMA_MN) ? 1 : 0;
 
   extern __shared__ uint8_t smem_raw[];
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      if (ASRC == A_TMA_K || ASRC == A_TMA_MN) tma_prefetch_desc(&tmA);
+      if (!A_GATHER) tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
       uint32_t it = 0;
       bool ok = true;
@@ -204,6 +204,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const TileCoord tc = decode_tile(args, t);
         const int kb0 = tc.sp * args.kb_per_split;
         const int kb1 = min(args.Kblocks, kb0 + args.kb_per_split);
+        // im2col, K-major: the tile's first output pixel (n, oh, ow) -> the
+        // top-left input corner of its filter window
+        int iw0 = 0, ih0 = 0, in0 = 0;
+        if (ASRC == A_IM2COL_K) {
+          const GatherDesc& G = args.g;
+          const int m0 = tc.m_t * BM;
+          const int HoWo = G.Ho * G.Wo;
+          in0 = m0 / HoWo;
+          const int rem = m0 - in0 * HoWo;
+          ih0 = rem / G.Wo - G.pad;
+          iw0 = rem - (rem / G.Wo) * G.Wo - G.pad;
+        }
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % stages;
           const uint32_t ph = (it / stages) & 1;
@@ -228,6 +240,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else if (ASRC == A_TMA_MN) {
             tma_load_2d(dA, &tmA, m0, kb * BK, fb);
             tma_load_2d(dA + MN_BLOCK_BYTES, &tmA, m0 + 64, kb * BK, fb);
+          } else if (ASRC == A_IM2COL_K) {
+            // k-block kb = (tap, 64-channel chunk)
+            const GatherDesc& G = args.g;
+            const int tap = kb / G.cpt;
+            const int chunk = kb - tap * G.cpt;
+            const int kh = tap / G.KW, kw = tap - (tap / G.KW) * G.KW;
+            tma_load_im2col_4d(dA, &tmA, tc.g * G.cg_off + chunk * 64, iw0, ih0, in0,
+                               static_cast<uint16_t>(kw), static_cast<uint16_t>(kh), fb);
+          } else if (ASRC == A_IM2COL_MN) {
+            // k-block kb = 64 output pixels (the reduction); the tile's two
+            // 64-wide M blocks are (tap, 64-channel chunk) pairs
+            const GatherDesc& G = args.g;
+            const int p0 = kb * BK;
+            const int HoWo = G.Ho * G.Wo;
+            const int n = p0 / HoWo;
+            const int rem = p0 - n * HoWo;
+            const int oh = rem / G.Wo, ow = rem - (rem / G.Wo) * G.Wo;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              // blocks past the last tap (the M tail) load tap 0; their rows
+              // are never stored
+              const int mb = min(tc.m_t * 2 + j, G.Kc - 1) * (tc.m_t * 2 + j < G.Kc);
+              const int tap = mb / G.cpt;
+              const int chunk = mb - tap * G.cpt;
+              const int kh = tap / G.KW, kw = tap - (tap / G.KW) * G.KW;
+              tma_load_im2col_4d(dA + j * MN_BLOCK_BYTES, &tmA, tc.g * G.cg_off + chunk * 64,
+                                 ow - G.pad, oh - G.pad, n, static_cast<uint16_t>(kw),
+                                 static_cast<uint16_t>(kh), fb);
+            }
           }
         }
       }
@@ -449,6 +490,11 @@ KernelEntry g_kernels[] = {
     ALX_K(128, A_TMA_K, B_TMA_MN),     ALX_K(256, A_TMA_K, B_TMA_MN),
     ALX_K(64, A_TMA_MN, B_TMA_MN),     ALX_K(128, A_TMA_MN, B_TMA_MN),
     ALX_K(256, A_TMA_MN, B_TMA_MN),
+    ALX_K(48, A_IM2COL_K, B_TMA_K),    ALX_K(64, A_IM2COL_K, B_TMA_K),
+    ALX_K(96, A_IM2COL_K, B_TMA_K),    ALX_K(128, A_IM2COL_K, B_TMA_K),
+    ALX_K(192, A_IM2COL_K, B_TMA_K),   ALX_K(256, A_IM2COL_K, B_TMA_K),
+    ALX_K(64, A_IM2COL_MN, B_TMA_MN),  ALX_K(128, A_IM2COL_MN, B_TMA_MN),
+    ALX_K(192, A_IM2COL_MN, B_TMA_MN), ALX_K(256, A_IM2COL_MN, B_TMA_MN),
 };
 #undef ALX_K
 
@@ -483,6 +529,40 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
+PFN_cuTensorMapEncodeIm2col_v12000 g_encode_im2col = nullptr;
+}
+
+bool make_tmap_im2col(CUtensorMap* m, const void* base, int N, int H, int W, int C, int K,
+                      int pad, int pixels) {
+  if (!g_encode_im2col) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeIm2col", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    g_encode_im2col = reinterpret_cast<PFN_cuTensorMapEncodeIm2col_v12000>(fn);
+  }
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (C * 2) % 16 || N < 1 || H < 1 || W < 1)
+    return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(W),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(W) * C * 2,
+                           static_cast<cuuint64_t>(H) * W * C * 2};
+  // bounding box of the filter window's top-left corner, in (W, H) order:
+  // from -pad to (size - 1) + (pad - (K - 1))
+  int lower[2] = {-pad, -pad};
+  int upper[2] = {pad - (K - 1), pad - (K - 1)};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode_im2col(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+                               dims, strides, lower, upper, 64, static_cast<cuuint32_t>(pixels),
+                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 

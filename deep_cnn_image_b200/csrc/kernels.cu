@@ -51,10 +51,10 @@ __global__ void k_write_hparams(HParams* hp, HParams v) { *hp = v; }
 
 // ------------------------------------------------------------------ s2d
 __global__ void k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs, int B) {
-  const uint32_t n = static_cast<uint32_t>(B) * 57 * 57 * 6;
+  const uint32_t n = static_cast<uint32_t>(B) * 57 * 57 * 8;
   for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
-    const int chunk = static_cast<int>(t % 6);
-    const uint32_t pix = t / 6;
+    const int chunk = static_cast<int>(t % 8);
+    const uint32_t pix = t / 8;
     const int j = static_cast<int>(pix % 57);
     const int i = static_cast<int>((pix / 57) % 57);
     const int b = static_cast<int>(pix / (57 * 57));
@@ -64,11 +64,11 @@ __global__ void k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs, int B) 
       const int ch = chunk * 8 + q;
       const int dy = ch / 12, dx = (ch / 3) % 4, c = ch % 3;
       const int y = 4 * i + dy, xx = 4 * j + dx;
-      f[q] = (y < 227 && xx < 227)
+      f[q] = (ch < 48 && y < 227 && xx < 227)
                  ? __bfloat162float(x[((static_cast<long long>(b) * 227 + y) * 227 + xx) * 3 + c])
                  : 0.f;
     }
-    *reinterpret_cast<uint4*>(xs + static_cast<size_t>(pix) * 48 + chunk * 8) = pack8(f);
+    *reinterpret_cast<uint4*>(xs + static_cast<size_t>(pix) * 64 + chunk * 8) = pack8(f);
   }
 }
 
@@ -511,13 +511,13 @@ __device__ __forceinline__ ConvIdx conv_index(const ConvMap& m, long long p64) {
   r.g = o / Og;
   r.co = o - r.g * Og;
   if (m.s2d) {
-    const int kg = ((kh >> 2) * 3 + (kw >> 2)) * 48 + ((kh & 3) * 4 + (kw & 3)) * 3 + ci;
-    r.fwd = 1LL * o * 432 + kg;
+    const int kg = ((kh >> 2) * 3 + (kw >> 2)) * 64 + ((kh & 3) * 4 + (kw & 3)) * 3 + ci;
+    r.fwd = 1LL * o * 576 + kg;
     r.part_inner = kg;
     r.dg = -1;
   } else {
-    r.fwd = p64;
-    r.part_inner = (1LL * kh * m.K + kw) * m.Cg + ci;
+    r.part_inner = (1LL * kh * m.K + kw) * m.P + ci;
+    r.fwd = 1LL * o * m.K * m.K * m.P + r.part_inner;
     r.dg = (((1LL * r.g * m.Cg + ci) * m.K + (m.K - 1 - kh)) * m.K + (m.K - 1 - kw)) * Og + r.co;
   }
   return r;
@@ -529,7 +529,7 @@ __global__ void k_sgd_conv(float* __restrict__ w, float* __restrict__ v,
   const HParams hp = *hpp;
   const long long n = 1LL * m.Cout * m.K * m.K * m.Cg;
   const int Og = m.Cout / m.groups;
-  const long long Kg = m.s2d ? 432 : 1LL * m.K * m.K * m.Cg;
+  const long long Kg = m.s2d ? 576 : 1LL * m.K * m.K * m.P;
   const long long split_stride = 1LL * m.groups * Og * Kg;
   for (long long p = blockIdx.x * 1LL * blockDim.x + threadIdx.x; p < n;
        p += 1LL * gridDim.x * blockDim.x) {
@@ -880,7 +880,7 @@ void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s) {
 }
 
 void launch_s2d(const bf16* x, bf16* xs, int B, cudaStream_t s) {
-  k_s2d<<<grid_for(1LL * B * 57 * 57 * 6, 256), 256, 0, s>>>(x, xs, B);
+  k_s2d<<<grid_for(1LL * B * 57 * 57 * 8, 256), 256, 0, s>>>(x, xs, B);
   count_launch();
 }
 void launch_lrn_fwd(const bf16* a, bf16* b, long long P, int C, int, float k, float alpha,

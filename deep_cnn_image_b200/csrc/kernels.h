@@ -27,7 +27,9 @@ struct HParams {
 // Canonical conv weight [Cout][K][K][Cg] -> positions in the GEMM layouts.
 struct ConvMap {
   int Cout, K, Cg, groups;
-  int s2d;  // conv1: forward operand is the space-to-depth [Cout][3][3][48] form
+  int s2d;  // conv1: forward operand is the space-to-depth [Cout][3][3][64] form
+  int P;    // channels per tap in the forward operand and the weight-gradient
+            // partials (64 * ceil(Cg / 64); 64 for the space-to-depth form)
 };
 
 // Kernels launched by this library so far (all launchers and GEMMs).
@@ -37,8 +39,8 @@ void count_launch_n(int64_t n);
 
 void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s);
 
-// x [B,227,227,3] (bf16) -> xs [B,57,57,48]: xs[b,i,j,(dy*4+dx)*3+c] = x[b,4i+dy,4j+dx,c]
-// (zero beyond row/column 226).
+// x [B,227,227,3] (bf16) -> xs [B,57,57,64]: xs[b,i,j,(dy*4+dx)*3+c] = x[b,4i+dy,4j+dx,c]
+// (zero beyond row/column 226, and channels 48..63 zero).
 void launch_s2d(const bf16* x, bf16* xs, int B, cudaStream_t s);
 
 // LRN over the channel axis of a [P, C] map (C % 8 == 0).

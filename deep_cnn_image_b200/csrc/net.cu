@@ -16,6 +16,7 @@
 
 #include "alexnet.h"
 #include "alexnet_ops.h"
+#include "conv_desc.h"
 #include "gemm.h"
 #include "kernels.h"
 
@@ -48,7 +49,14 @@ struct ConvL {
   // space-to-depth input)
   int gH, gC, gK, gpad, gCg;
   int Og() const { return Cout / groups; }
-  int Kdim() const { return gK * gK * gCg; }
+  int Pch() const { return 64 * ((gCg + 63) / 64); }  // channels per tap, padded
+  int Kdim() const { return gK * gK * Pch(); }
+  // GEMM views: forward / weight gradient over the layer input, and the data
+  // gradient as a forward convolution of dY with the flipped kernel
+  ConvShape fwd(int B) const { return ConvShape{B, gH, gH, gC, gCg, Og(), groups, gK, gpad}; }
+  ConvShape dgrad(int B) const {
+    return ConvShape{B, Ho, Ho, Cout, Og(), Cin / groups, groups, K, K - 1 - pad};
+  }
 };
 
 struct FcL {
@@ -61,20 +69,6 @@ struct Plan {
   bool ok = false;
 };
 
-int pick_bn(int n) {
-  if (n <= 256 && (n == 48 || n == 64 || n == 96 || n == 128 || n == 192 || n == 256)) return n;
-  if (n % 192 == 0) return 192;
-  if (n % 256 == 0) return 256;
-  if (n % 128 == 0) return 128;
-  return 0;
-}
-int pick_bn_mn(int n) {
-  if (n <= 64) return 64;
-  if (n <= 128) return 128;
-  if (n == 192 || n % 192 == 0) return 192;
-  if (n <= 256 || n % 256 == 0) return 256;
-  return 128;
-}
 int pick_kbps(long long tiles, int kblocks, int num_sms, int min_blocks) {
   long long s = (2LL * num_sms + tiles - 1) / tiles;
   const long long smax = kblocks / min_blocks > 0 ? kblocks / min_blocks : 1;
@@ -146,13 +140,26 @@ struct alexnet {
   std::map<int, int64_t> graph_kernels;  // kernels in each captured step
   bool use_graphs = true;
 
-  // launch accounting (alexnet_stats_*)
+  // launch accounting (alexnet_stats_*): the GEMM events of one call; a
+  // captured graph owns the events recorded into it (as event-record nodes)
+  struct StepRec {
+    std::vector<cudaEvent_t> ev;  // start/stop pairs
+    size_t used = 0;
+    int64_t gemm_launches = 0;
+    double gemm_flops = 0.0;
+    void reset() {
+      used = 0;
+      gemm_launches = 0;
+      gemm_flops = 0.0;
+    }
+  };
   bool stats_on = false;
-  int64_t launch_base = 0;
-  int64_t gemm_launches = 0;
-  double gemm_flops = 0.0;
-  std::vector<cudaEvent_t> ev;
-  size_t ev_used = 0;
+  bool capturing = false;
+  StepRec direct_rec;
+  std::map<int, StepRec> graph_rec;
+  StepRec* rec = nullptr;       // where run_gemm records
+  StepRec* last_rec = nullptr;  // the most recent call's record
+  int64_t last_launches = 0;
   cudaStream_t stats_stream = nullptr;
 
   const bf16* conv_input(int l) const {
@@ -221,7 +228,7 @@ void build_geometry(alexnet* h) {
     L.P = L.pool ? (L.Ho - c.pool_size) / 2 + 1 : L.Ho;
     if (l == 0) {
       L.gH = 57;
-      L.gC = 48;
+      L.gC = 64;
       L.gK = 3;
       L.gpad = 0;
       L.gCg = 48;
@@ -267,123 +274,6 @@ bool tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint
     return true;
   }
   return make_tmap_bf16(m, base, inner, outer, row_bytes, box_inner, box_outer);
-}
-
-GatherDesc gather_fwd(const ConvL& L, const bf16* src, int B) {
-  GatherDesc g;
-  g.src = src;
-  g.H = L.gH;
-  g.W = L.gH;
-  g.C = L.gC;
-  g.cg_off = L.gCg;
-  g.Cg8 = L.gCg / 8;
-  g.KW = L.gK;
-  g.pad = L.gpad;
-  g.Ho = L.Ho;
-  g.Wo = L.Ho;
-  g.Kc = L.gK * L.gK * L.gCg / 8;
-  g.Mpix = B * L.Ho * L.Ho;
-  return g;
-}
-
-bool desc_conv_fwd(GemmDesc* d, const ConvL& L, const bf16* in, const bf16* w, const float* bias,
-                   bf16* out, int B, int num_sms, int* status) {
-  memset(d, 0, sizeof(*d));
-  d->asrc = A_GATHER_K;
-  d->bsrc = B_TMA_K;
-  d->bn = pick_bn(L.Og());
-  if (!d->bn) return false;
-  GemmArgs& a = d->args;
-  a.g = gather_fwd(L, in, B);
-  a.M = a.g.Mpix;
-  a.N = L.Og();
-  a.Kblocks = (a.g.Kc + 7) / 8;
-  a.groups = L.groups;
-  a.b_goff = L.Og();
-  a.epi = EPI_BF16;
-  a.relu = 1;
-  a.out = out;
-  a.ld_out = L.Cout;
-  a.col_goff = L.Og();
-  a.bias = bias;
-  a.status = status;
-  if (!tmap(&d->tmB, w, L.Kdim(), L.Cout, static_cast<uint64_t>(L.Kdim()) * 2, 64,
-                      d->bn))
-    return false;
-  d->tmA = d->tmB;
-  return gemm_finalize(d, num_sms);
-}
-
-// Data gradient of a stride-1 conv as a forward conv of dY with the flipped,
-// transposed kernel and padding K-1-pad.
-bool desc_conv_dgrad(GemmDesc* d, const ConvL& L, const bf16* dy, const bf16* wdg,
-                     const bf16* mask, bf16* out, int B, int num_sms, int* status) {
-  memset(d, 0, sizeof(*d));
-  const int Cg = L.Cin / L.groups, Og = L.Og();
-  d->asrc = A_GATHER_K;
-  d->bsrc = B_TMA_K;
-  d->bn = pick_bn(Cg);
-  if (!d->bn || L.stride != 1) return false;
-  GemmArgs& a = d->args;
-  GatherDesc& g = a.g;
-  g.src = dy;
-  g.H = L.Ho;
-  g.W = L.Ho;
-  g.C = L.Cout;
-  g.cg_off = Og;
-  g.Cg8 = Og / 8;
-  g.KW = L.K;
-  g.pad = L.K - 1 - L.pad;
-  g.Ho = L.H;
-  g.Wo = L.H;
-  g.Kc = L.K * L.K * Og / 8;
-  g.Mpix = B * L.H * L.H;
-  a.M = g.Mpix;
-  a.N = Cg;
-  a.Kblocks = (g.Kc + 7) / 8;
-  a.groups = L.groups;
-  a.b_goff = Cg;
-  a.epi = mask ? EPI_BF16_MASK : EPI_BF16;
-  a.out = out;
-  a.ld_out = L.Cin;
-  a.col_goff = Cg;
-  a.mask = mask;
-  a.ld_mask = L.Cin;
-  a.status = status;
-  const int Kd = L.K * L.K * Og;
-  if (!tmap(&d->tmB, wdg, Kd, L.Cin, static_cast<uint64_t>(Kd) * 2, 64, d->bn))
-    return false;
-  d->tmA = d->tmB;
-  return gemm_finalize(d, num_sms);
-}
-
-bool desc_conv_wgrad(GemmDesc* d, const ConvL& L, const bf16* in, const bf16* dy, float* part,
-                     int B, int splits, int num_sms, int* status) {
-  memset(d, 0, sizeof(*d));
-  const int Og = L.Og();
-  d->asrc = A_GATHER_MN;
-  d->bsrc = B_TMA_MN;
-  d->bn = pick_bn_mn(Og);
-  GemmArgs& a = d->args;
-  a.g = gather_fwd(L, in, B);
-  a.M = L.Kdim();
-  a.N = Og;
-  a.Kblocks = (a.g.Mpix + 63) / 64;
-  a.groups = L.groups;
-  a.b_goff = Og;
-  const long long tiles = 1LL * ((a.M + 127) / 128) * ((a.N + d->bn - 1) / d->bn) * a.groups;
-  a.kb_per_split = splits > 0 ? (a.Kblocks + splits - 1) / splits
-                              : pick_kbps(tiles, a.Kblocks, num_sms, 8);
-  a.epi = EPI_F32_T;
-  a.out = part;
-  a.ld_out = a.M;
-  a.group_stride = 1LL * Og * a.M;
-  a.split_stride = 1LL * L.groups * Og * a.M;
-  a.status = status;
-  if (!tmap(&d->tmB, dy, L.Cout, a.g.Mpix, static_cast<uint64_t>(L.Cout) * 2, 64, 64))
-    return false;
-  d->tmA = d->tmB;
-  return gemm_finalize(d, num_sms);
 }
 
 bool desc_fc_fwd(GemmDesc* d, const FcL& F, const bf16* x, const bf16* w, float* part, int B,
@@ -480,17 +370,18 @@ bool build_plan(alexnet* h, int B, Plan* P) {
   const int ns = h->num_sms;
   for (int l = 0; l < 5; ++l) {
     const ConvL& L = h->conv[l];
-    if (!desc_conv_fwd(&P->cf[l], L, h->conv_input(l), h->wf[l], h->params + h->b_off[l], h->a[l],
-                       B, ns, h->status))
+    if (!conv_desc_fwd(&P->cf[l], L.fwd(B), h->conv_input(l), h->wf[l], h->params + h->b_off[l], 1,
+                       nullptr, h->a[l], ns, h->status, g_dry_tmaps))
       return set_err(h, "conv forward plan");
     if (l > 0) {
       const bf16* mask = (!h->conv[l - 1].pool) ? h->a[l - 1] : nullptr;
       bf16* out = mask ? h->da[l - 1] : h->dp[l - 1];
-      if (!desc_conv_dgrad(&P->cd[l], L, h->da[l], h->wd[l], mask, out, B, ns, h->status))
+      if (!conv_desc_fwd(&P->cd[l], L.dgrad(B), h->da[l], h->wd[l], nullptr, 0, mask, out, ns,
+                         h->status, g_dry_tmaps))
         return set_err(h, "conv data-gradient plan");
     }
-    if (!desc_conv_wgrad(&P->cw[l], L, h->conv_input(l), h->da[l], h->scratch, B, 0, ns,
-                         h->status))
+    if (!conv_desc_wgrad(&P->cw[l], L.fwd(B), h->conv_input(l), h->da[l], h->scratch, 0, ns,
+                         h->status, g_dry_tmaps))
       return set_err(h, "conv weight-gradient plan");
   }
   for (int l = 0; l < 5; ++l) {
@@ -563,7 +454,7 @@ size_t carve(alexnet* h, void* base) {
   }
   for (int f = 0; f < 3; ++f) h->wf[5 + f] = c.take<bf16>(h->w_len[5 + f]);
   h->xin = c.take<bf16>(static_cast<size_t>(B) * 227 * 227 * 3);
-  h->xs = c.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 48);
+  h->xs = c.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 64);
   for (int l = 0; l < 5; ++l) {
     const ConvL& L = h->conv[l];
     const size_t e = static_cast<size_t>(B) * L.Ho * L.Ho * L.Cout;
@@ -640,6 +531,7 @@ ConvMap conv_map(const alexnet* h, int l) {
   m.Cg = L.Cin / L.groups;
   m.groups = L.groups;
   m.s2d = l == 0 ? 1 : 0;
+  m.P = L.Pch();
   return m;
 }
 
@@ -666,23 +558,23 @@ Plan* get_plan(alexnet* h, int B) {
   } while (0)
 
 cudaError_t run_gemm(alexnet* h, const GemmDesc& d, double flops, cudaStream_t s) {
-  if (!h->stats_on) return gemm_launch(d, s);
-  if (h->ev_used + 2 > h->ev.size()) {
-    for (int i = 0; i < 2; ++i) {
-      cudaEvent_t e;
-      cudaError_t r = cudaEventCreate(&e);
-      if (r != cudaSuccess) return r;
-      h->ev.push_back(e);
-    }
+  if (!h->stats_on || !h->rec) return gemm_launch(d, s);
+  alexnet::StepRec& R = *h->rec;
+  while (R.used + 2 > R.ev.size()) {
+    cudaEvent_t e;
+    cudaError_t r = cudaEventCreate(&e);
+    if (r != cudaSuccess) return r;
+    R.ev.push_back(e);
   }
-  cudaEvent_t e0 = h->ev[h->ev_used], e1 = h->ev[h->ev_used + 1];
-  h->ev_used += 2;
-  h->stats_stream = s;
-  cudaEventRecord(e0, s);
+  cudaEvent_t e0 = R.ev[R.used], e1 = R.ev[R.used + 1];
+  R.used += 2;
+  // inside a capture the records become event nodes of the graph
+  const unsigned flags = h->capturing ? cudaEventRecordExternal : cudaEventRecordDefault;
+  cudaEventRecordWithFlags(e0, s, flags);
   cudaError_t r = gemm_launch(d, s);
-  cudaEventRecord(e1, s);
-  h->gemm_launches += 1;
-  h->gemm_flops += flops;
+  cudaEventRecordWithFlags(e1, s, flags);
+  R.gemm_launches += 1;
+  R.gemm_flops += flops;
   return r;
 }
 
@@ -904,8 +796,8 @@ alexnet_status alexnet_create(const alexnet_config* cfg, void* workspace, size_t
   }
   launch_fill(h->vel, h->n_params, 0.f, s);
   cudaError_t e = cudaMemsetAsync(h->status, 0, sizeof(int), s);
-  if (e == cudaSuccess && h->cfg.dtype == ALEXNET_BF16 && h->wf[0])
-    e = cudaMemsetAsync(h->wf[0], 0, sizeof(bf16) * 96 * 432, s);
+  for (int l = 0; l < 5 && e == cudaSuccess && h->cfg.dtype == ALEXNET_BF16; ++l)
+    e = cudaMemsetAsync(h->wf[l], 0, sizeof(bf16) * h->conv[l].Cout * h->conv[l].Kdim(), s);
   refresh_shadows(h, s);
   write_hp(h, 0.f, s);
   if (e == cudaSuccess) e = cudaGetLastError();
@@ -938,9 +830,18 @@ alexnet_status alexnet_forward(alexnet_t* h, const void* x, int B, alexnet_mode 
   } else {
     Plan* P = get_plan(h, B);
     if (!P) return ALEXNET_ERR_CUDA;
+    const int64_t l0 = launch_counter();
     write_hp(h, 0.f, s);
     const int dm = !h->cfg.dropout_on ? 0 : (mode == ALEXNET_TRAIN ? 1 : 2);
+    h->direct_rec.reset();
+    h->rec = h->stats_on ? &h->direct_rec : nullptr;
     st = forward_bf16(h, static_cast<const bf16*>(x), B, dm, logits, s, P);
+    h->rec = nullptr;
+    if (h->stats_on) {
+      h->last_rec = &h->direct_rec;
+      h->last_launches = launch_counter() - l0;
+      h->stats_stream = s;
+    }
   }
   if (st != ALEXNET_OK) return st;
   if (probs)
@@ -973,17 +874,23 @@ alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* la
   ALX_TRY(cudaMemcpyAsync(h->labels_buf, labels, sizeof(int32_t) * B, cudaMemcpyDeviceToDevice, s),
           "train_step labels");
   alexnet_status st = ALEXNET_OK;
-  if (h->use_graphs && !h->stats_on) {
-    auto it = h->train_graphs.find(B);
+  const int64_t l0 = launch_counter();
+  if (h->use_graphs) {
+    const int key = 2 * B + (h->stats_on ? 1 : 0);
+    auto it = h->train_graphs.find(key);
     if (it == h->train_graphs.end()) {
       if (!h->cap_stream)
         ALX_TRY(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking), "capture stream");
       ALX_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal),
               "begin capture");
       const int64_t c0 = launch_counter();
+      h->rec = h->stats_on ? &h->graph_rec[key] : nullptr;
+      h->capturing = true;
       st = train_bf16(h, nullptr, h->labels_buf, B, nullptr, h->cap_stream, P);
+      h->capturing = false;
+      h->rec = nullptr;
       // captured kernels are counted when a replay runs them, not now
-      h->graph_kernels[B] = launch_counter() - c0;
+      h->graph_kernels[key] = launch_counter() - c0;
       count_launch_n(-(launch_counter() - c0));
       cudaGraph_t g = nullptr;
       const cudaError_t ce = cudaStreamEndCapture(h->cap_stream, &g);
@@ -996,12 +903,21 @@ alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* la
       const cudaError_t ie = cudaGraphInstantiate(&ex, g, 0);
       cudaGraphDestroy(g);
       ALX_TRY(ie, "graph instantiate");
-      it = h->train_graphs.emplace(B, ex).first;
+      it = h->train_graphs.emplace(key, ex).first;
     }
     ALX_TRY(cudaGraphLaunch(it->second, s), "graph launch");
-    count_launch_n(h->graph_kernels[B]);
+    count_launch_n(h->graph_kernels[key]);
+    if (h->stats_on) h->last_rec = &h->graph_rec[key];
   } else {
+    h->direct_rec.reset();
+    h->rec = h->stats_on ? &h->direct_rec : nullptr;
     st = train_bf16(h, nullptr, h->labels_buf, B, nullptr, s, P);
+    h->rec = nullptr;
+    if (h->stats_on) h->last_rec = &h->direct_rec;
+  }
+  if (h->stats_on) {
+    h->last_launches = launch_counter() - l0;
+    h->stats_stream = s;
   }
   if (st != ALEXNET_OK) return st;
   if (loss)
@@ -1139,7 +1055,9 @@ const char* alexnet_last_error(const alexnet_t* h) {
 
 alexnet_status alexnet_destroy(alexnet_t* h) {
   if (h) {
-    for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+    for (cudaEvent_t e : h->direct_rec.ev) cudaEventDestroy(e);
+    for (auto& kv : h->graph_rec)
+      for (cudaEvent_t e : kv.second.ev) cudaEventDestroy(e);
     for (auto& kv : h->train_graphs) cudaGraphExecDestroy(kv.second);
     if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   }
@@ -1150,33 +1068,27 @@ alexnet_status alexnet_destroy(alexnet_t* h) {
 alexnet_status alexnet_stats_enable(alexnet_t* h, int enable) {
   if (!h) return ALEXNET_ERR_INVALID_ARG;
   h->stats_on = enable != 0;
-  h->launch_base = launch_counter();
-  h->gemm_launches = 0;
-  h->gemm_flops = 0.0;
-  h->ev_used = 0;
+  h->last_rec = nullptr;
+  h->last_launches = 0;
   return ALEXNET_OK;
 }
 
 alexnet_status alexnet_stats_read(alexnet_t* h, alexnet_stats* out) {
   if (!h || !out) return ALEXNET_ERR_INVALID_ARG;
+  memset(out, 0, sizeof(*out));
+  if (!h->last_rec) return ALEXNET_OK;
+  ALX_TRY(cudaStreamSynchronize(h->stats_stream), "stats_read");
   double ms = 0.0;
-  if (h->ev_used) {
-    ALX_TRY(cudaStreamSynchronize(h->stats_stream), "stats_read");
-    for (size_t i = 0; i + 1 < h->ev_used; i += 2) {
-      float t = 0.f;
-      ALX_TRY(cudaEventElapsedTime(&t, h->ev[i], h->ev[i + 1]), "stats_read");
-      ms += t;
-    }
+  const alexnet::StepRec& R = *h->last_rec;
+  for (size_t i = 0; i + 1 < R.used; i += 2) {
+    float t = 0.f;
+    ALX_TRY(cudaEventElapsedTime(&t, R.ev[i], R.ev[i + 1]), "stats_read");
+    ms += t;
   }
-  const int64_t now = launch_counter();
-  out->launches = now - h->launch_base;
-  out->gemm_launches = h->gemm_launches;
-  out->gemm_flops = h->gemm_flops;
+  out->launches = h->last_launches;
+  out->gemm_launches = R.gemm_launches;
+  out->gemm_flops = R.gemm_flops;
   out->gemm_ms = ms;
-  h->launch_base = now;
-  h->gemm_launches = 0;
-  h->gemm_flops = 0.0;
-  h->ev_used = 0;
   return ALEXNET_OK;
 }
 

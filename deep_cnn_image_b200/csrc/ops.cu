@@ -5,6 +5,7 @@
 
 #include "alexnet.h"
 #include "alexnet_ops.h"
+#include "conv_desc.h"
 #include "gemm.h"
 #include "kernels.h"
 
@@ -40,115 +41,6 @@ struct Scratch {
 
 alexnet_status done(cudaError_t e) { return e == cudaSuccess ? ALEXNET_OK : ALEXNET_ERR_CUDA; }
 
-int pick_bn(int n) {
-  if (n == 48 || n == 64 || n == 96 || n == 128 || n == 192 || n == 256) return n;
-  if (n % 192 == 0) return 192;
-  if (n % 256 == 0) return 256;
-  if (n % 128 == 0) return 128;
-  return 0;
-}
-int pick_bn_mn(int n) {
-  if (n <= 64) return 64;
-  if (n <= 128) return 128;
-  if (n % 192 == 0) return 192;
-  if (n <= 256 || n % 256 == 0) return 256;
-  return 128;
-}
-
-struct ConvGeom {
-  int H, W, Cin, Cout, K, pad, groups, Ho, Wo;
-  int Cg() const { return Cin / groups; }
-  int Og() const { return Cout / groups; }
-};
-
-bool geom_ok(const ConvGeom& g) {
-  return g.H > 0 && g.W > 0 && g.Cin > 0 && g.Cout > 0 && g.K > 0 && g.pad >= 0 && g.groups > 0 &&
-         g.Cin % g.groups == 0 && g.Cout % g.groups == 0 && g.Cg() % 8 == 0 && g.Og() % 8 == 0 &&
-         g.Ho > 0 && g.Wo > 0;
-}
-
-GatherDesc gather_of(const ConvGeom& g, const void* x, int B) {
-  GatherDesc d;
-  d.src = static_cast<const bf16*>(x);
-  d.H = g.H;
-  d.W = g.W;
-  d.C = g.Cin;
-  d.cg_off = g.Cg();
-  d.Cg8 = g.Cg() / 8;
-  d.KW = g.K;
-  d.pad = g.pad;
-  d.Ho = g.Ho;
-  d.Wo = g.Wo;
-  d.Kc = g.K * g.K * g.Cg() / 8;
-  d.Mpix = B * g.Ho * g.Wo;
-  return d;
-}
-
-alexnet_status run_conv_fwd(const ConvGeom& g, const void* x, int B, const bf16* wgemm,
-                            const float* bias, int relu, void* y, int* status, cudaStream_t s) {
-  GemmDesc d;
-  memset(&d, 0, sizeof(d));
-  d.asrc = A_GATHER_K;
-  d.bsrc = B_TMA_K;
-  d.bn = pick_bn(g.Og());
-  if (!d.bn) return ALEXNET_ERR_UNSUPPORTED;
-  GemmArgs& a = d.args;
-  a.g = gather_of(g, x, B);
-  a.M = a.g.Mpix;
-  a.N = g.Og();
-  a.Kblocks = (a.g.Kc + 7) / 8;
-  a.groups = g.groups;
-  a.b_goff = g.Og();
-  a.epi = EPI_BF16;
-  a.relu = relu;
-  a.out = y;
-  a.ld_out = g.Cout;
-  a.col_goff = g.Og();
-  a.bias = bias;
-  a.status = status;
-  const int Kd = g.K * g.K * g.Cg();
-  if (!make_tmap_bf16(&d.tmB, wgemm, Kd, g.Cout, 2ull * Kd, 64, d.bn)) return ALEXNET_ERR_INVALID_ARG;
-  d.tmA = d.tmB;
-  if (!gemm_finalize(&d, num_sms())) return ALEXNET_ERR_UNSUPPORTED;
-  return done(gemm_launch(d, s));
-}
-
-alexnet_status run_conv_wgrad(const ConvGeom& g, const void* x, int B, const void* dy, int splits,
-                              float* part, int* S_out, int* status, cudaStream_t s) {
-  GemmDesc d;
-  memset(&d, 0, sizeof(d));
-  d.asrc = A_GATHER_MN;
-  d.bsrc = B_TMA_MN;
-  d.bn = pick_bn_mn(g.Og());
-  GemmArgs& a = d.args;
-  a.g = gather_of(g, x, B);
-  a.M = g.K * g.K * g.Cg();
-  a.N = g.Og();
-  a.Kblocks = (a.g.Mpix + 63) / 64;
-  a.groups = g.groups;
-  a.b_goff = g.Og();
-  if (splits <= 0) {
-    const long long tiles = 1LL * ((a.M + 127) / 128) * ((a.N + d.bn - 1) / d.bn) * a.groups;
-    long long sp = (2LL * num_sms() + tiles - 1) / tiles;
-    if (sp > a.Kblocks / 8) sp = a.Kblocks / 8;
-    splits = sp < 1 ? 1 : static_cast<int>(sp);
-  }
-  if (splits > a.Kblocks) splits = a.Kblocks;
-  a.kb_per_split = (a.Kblocks + splits - 1) / splits;
-  a.epi = EPI_F32_T;
-  a.out = part;
-  a.ld_out = a.M;
-  a.group_stride = 1LL * g.Og() * a.M;
-  a.split_stride = 1LL * g.groups * g.Og() * a.M;
-  a.status = status;
-  if (!make_tmap_bf16(&d.tmB, dy, g.Cout, a.g.Mpix, 2ull * g.Cout, 64, 64))
-    return ALEXNET_ERR_INVALID_ARG;
-  d.tmA = d.tmB;
-  if (!gemm_finalize(&d, num_sms())) return ALEXNET_ERR_UNSUPPORTED;
-  *S_out = d.args.splits;
-  return done(gemm_launch(d, s));
-}
-
 HParams zero_hp() {
   HParams hp;
   memset(&hp, 0, sizeof(hp));
@@ -163,7 +55,8 @@ alexnet_status reduce_wgrad(const ConvMap& m, const float* part, int S, float* d
   const size_t n = static_cast<size_t>(m.Cout) * m.K * m.K * m.Cg;
   float* w = sc.take<float>(n);
   float* v = sc.take<float>(n);
-  bf16* fwd = sc.take<bf16>(m.s2d ? static_cast<size_t>(m.Cout) * 432 : n);
+  bf16* fwd = sc.take<bf16>(m.s2d ? static_cast<size_t>(m.Cout) * 576
+                               : static_cast<size_t>(m.Cout) * m.K * m.K * m.P);
   bf16* dg = m.s2d ? nullptr : sc.take<bf16>(n);
   HParams* hp = sc.take<HParams>(1);
   if (!w || !v || !fwd || (!m.s2d && !dg) || !hp) return ALEXNET_ERR_INVALID_ARG;
@@ -181,14 +74,27 @@ extern "C" {
 alexnet_status alexnet_op_conv_fwd(const void* x, int B, int H, int W, int Cin, const void* w,
                                    const float* bias, int Cout, int K, int pad, int groups,
                                    int relu, void* y, void* ws, size_t ws_bytes, void* stream) {
-  ConvGeom g{H, W, Cin, Cout, K, pad, groups, H + 2 * pad - K + 1, W + 2 * pad - K + 1};
-  if (!x || !w || !y || B < 1 || !geom_ok(g)) return ALEXNET_ERR_INVALID_ARG;
+  if (!x || !w || !y || B < 1 || groups < 1 || Cin % groups || Cout % groups)
+    return ALEXNET_ERR_INVALID_ARG;
+  ConvShape cs{B, H, W, Cin, Cin / groups, Cout / groups, groups, K, pad};
+  if (cs.Cg % 8 || cs.Og % 8 || cs.Ho() < 1 || cs.Wo() < 1 || K < 1 || pad < 0)
+    return ALEXNET_ERR_INVALID_ARG;
   Scratch sc(ws, ws_bytes);
   int* status = sc.take<int>(1);
-  if (!status) return ALEXNET_ERR_INVALID_ARG;
+  const size_t n = static_cast<size_t>(Cout) * K * K * cs.Cg;
+  float* wf = sc.take<float>(n);
+  bf16* wg = sc.take<bf16>(static_cast<size_t>(Cout) * cs.Kdim());
+  if (!status || !wf || !wg) return ALEXNET_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaMemsetAsync(status, 0, 4, s);
-  return run_conv_fwd(g, x, B, static_cast<const bf16*>(w), bias, relu, y, status, s);
+  // canonical [Cout][K][K][Cg] -> the GEMM operand [Cout][K*K*P] (zero pads)
+  cudaMemsetAsync(wg, 0, 2 * static_cast<size_t>(Cout) * cs.Kdim(), s);
+  launch_f32_from_bf16(static_cast<const bf16*>(w), wf, n, s);
+  launch_conv_shadows(wf, ConvMap{Cout, K, cs.Cg, groups, 0, cs.P()}, wg, nullptr, s);
+  GemmDesc d;
+  if (!conv_desc_fwd(&d, cs, x, wg, bias, relu, nullptr, y, num_sms(), status))
+    return ALEXNET_ERR_UNSUPPORTED;
+  return done(gemm_launch(d, s));
 }
 
 alexnet_status alexnet_op_conv1_fwd(const void* x, int B, const void* w, const float* bias,
@@ -196,19 +102,21 @@ alexnet_status alexnet_op_conv1_fwd(const void* x, int B, const void* w, const f
   if (!x || !w || !y || B < 1) return ALEXNET_ERR_INVALID_ARG;
   Scratch sc(ws, ws_bytes);
   int* status = sc.take<int>(1);
-  bf16* xs = sc.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 48);
+  bf16* xs = sc.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 64);
   float* wf = sc.take<float>(96 * 363);
-  bf16* ws2 = sc.take<bf16>(96 * 432);
+  bf16* ws2 = sc.take<bf16>(96 * 576);
   if (!status || !xs || !wf || !ws2) return ALEXNET_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaMemsetAsync(status, 0, 4, s);
-  cudaMemsetAsync(ws2, 0, 2 * 96 * 432, s);
+  cudaMemsetAsync(ws2, 0, 2 * 96 * 576, s);
   launch_s2d(static_cast<const bf16*>(x), xs, B, s);
   launch_f32_from_bf16(static_cast<const bf16*>(w), wf, 96 * 363, s);
-  ConvMap m{96, 11, 3, 1, 1};
-  launch_conv_shadows(wf, m, ws2, nullptr, s);
-  ConvGeom g{57, 57, 48, 96, 3, 0, 1, 55, 55};
-  return run_conv_fwd(g, xs, B, ws2, bias, 1, y, status, s);
+  launch_conv_shadows(wf, ConvMap{96, 11, 3, 1, 1, 64}, ws2, nullptr, s);
+  GemmDesc d;
+  if (!conv_desc_fwd(&d, ConvShape{B, 57, 57, 64, 48, 96, 1, 3, 0}, xs, ws2, bias, 1, nullptr, y,
+                     num_sms(), status))
+    return ALEXNET_ERR_UNSUPPORTED;
+  return done(gemm_launch(d, s));
 }
 
 alexnet_status alexnet_op_conv_dgrad(const void* dy, int B, int H, int W, int Cin, const void* w,
@@ -216,68 +124,53 @@ alexnet_status alexnet_op_conv_dgrad(const void* dy, int B, int H, int W, int Ci
                                      void* dx, void* ws, size_t ws_bytes, void* stream) {
   // the forward conv maps [H,W,Cin] -> [Ho,Wo,Cout]; its data gradient is a
   // forward conv of dy with the flipped kernel and padding K-1-pad
-  ConvGeom fw{H, W, Cin, Cout, K, pad, groups, H + 2 * pad - K + 1, W + 2 * pad - K + 1};
-  if (!dy || !w || !dx || B < 1 || !geom_ok(fw)) return ALEXNET_ERR_INVALID_ARG;
-  ConvGeom g{fw.Ho, fw.Wo, Cout, Cin, K, K - 1 - pad, groups, H, W};
-  if (g.Ho != fw.Ho + 2 * g.pad - K + 1 || g.Wo != fw.Wo + 2 * g.pad - K + 1)
-    return ALEXNET_ERR_UNSUPPORTED;
+  if (!dy || !w || !dx || B < 1 || groups < 1 || Cin % groups || Cout % groups)
+    return ALEXNET_ERR_INVALID_ARG;
+  const int Cg = Cin / groups, Og = Cout / groups;
+  const int Ho = H + 2 * pad - K + 1, Wo = W + 2 * pad - K + 1;
+  if (Cg % 8 || Og % 8 || Ho < 1 || Wo < 1 || K < 1 || pad < 0) return ALEXNET_ERR_INVALID_ARG;
+  // the flipped operand keeps Og channels per tap unpadded
+  if (Og % 64 || Ho + 2 * (K - 1 - pad) - K + 1 != H) return ALEXNET_ERR_UNSUPPORTED;
   Scratch sc(ws, ws_bytes);
   int* status = sc.take<int>(1);
-  const size_t n = static_cast<size_t>(Cout) * K * K * (Cin / groups);
+  const size_t n = static_cast<size_t>(Cout) * K * K * Cg;
+  const ConvMap m{Cout, K, Cg, groups, 0, 64 * ((Cg + 63) / 64)};
   float* wf = sc.take<float>(n);
-  bf16* fwd = sc.take<bf16>(n);
+  bf16* fwd = sc.take<bf16>(static_cast<size_t>(Cout) * K * K * m.P);
   bf16* dg = sc.take<bf16>(n);
   if (!status || !wf || !fwd || !dg) return ALEXNET_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaMemsetAsync(status, 0, 4, s);
   launch_f32_from_bf16(static_cast<const bf16*>(w), wf, n, s);
-  ConvMap m{Cout, K, Cin / groups, groups, 0};
   launch_conv_shadows(wf, m, fwd, dg, s);
   GemmDesc d;
-  memset(&d, 0, sizeof(d));
-  d.asrc = A_GATHER_K;
-  d.bsrc = B_TMA_K;
-  d.bn = pick_bn(g.Og());
-  if (!d.bn) return ALEXNET_ERR_UNSUPPORTED;
-  GemmArgs& a = d.args;
-  a.g = gather_of(g, dy, B);
-  a.M = a.g.Mpix;
-  a.N = g.Og();
-  a.Kblocks = (a.g.Kc + 7) / 8;
-  a.groups = groups;
-  a.b_goff = g.Og();
-  a.epi = mask ? EPI_BF16_MASK : EPI_BF16;
-  a.out = dx;
-  a.ld_out = Cin;
-  a.col_goff = g.Og();
-  a.mask = static_cast<const bf16*>(mask);
-  a.ld_mask = Cin;
-  a.status = status;
-  const int Kd = K * K * g.Cg();
-  if (!make_tmap_bf16(&d.tmB, dg, Kd, Cin, 2ull * Kd, 64, d.bn)) return ALEXNET_ERR_INVALID_ARG;
-  d.tmA = d.tmB;
-  if (!gemm_finalize(&d, num_sms())) return ALEXNET_ERR_UNSUPPORTED;
+  if (!conv_desc_fwd(&d, ConvShape{B, Ho, Wo, Cout, Og, Cg, groups, K, K - 1 - pad}, dy, dg,
+                     nullptr, 0, mask, dx, num_sms(), status))
+    return ALEXNET_ERR_UNSUPPORTED;
   return done(gemm_launch(d, s));
 }
 
 alexnet_status alexnet_op_conv_wgrad(const void* x, int B, int H, int W, int Cin, const void* dy,
                                      int Cout, int K, int pad, int groups, int splits, float* dw,
                                      void* ws, size_t ws_bytes, void* stream) {
-  ConvGeom g{H, W, Cin, Cout, K, pad, groups, H + 2 * pad - K + 1, W + 2 * pad - K + 1};
-  if (!x || !dy || !dw || B < 1 || !geom_ok(g)) return ALEXNET_ERR_INVALID_ARG;
+  if (!x || !dy || !dw || B < 1 || groups < 1 || Cin % groups || Cout % groups)
+    return ALEXNET_ERR_INVALID_ARG;
+  ConvShape cs{B, H, W, Cin, Cin / groups, Cout / groups, groups, K, pad};
+  if (cs.Cg % 8 || cs.Og % 8 || cs.Ho() < 1 || cs.Wo() < 1 || K < 1 || pad < 0)
+    return ALEXNET_ERR_INVALID_ARG;
   Scratch sc(ws, ws_bytes);
   int* status = sc.take<int>(1);
-  const int Kb = (B * g.Ho * g.Wo + 63) / 64;
+  const int Kb = (B * cs.Ho() * cs.Wo() + 63) / 64;
   const int smax = splits > 0 ? (splits < Kb ? splits : Kb) : Kb;
-  float* part = sc.take<float>(static_cast<size_t>(smax) * Cout * K * K * g.Cg());
+  float* part = sc.take<float>(static_cast<size_t>(smax) * Cout * cs.Kdim());
   if (!status || !part) return ALEXNET_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaMemsetAsync(status, 0, 4, s);
-  int S = 0;
-  alexnet_status st = run_conv_wgrad(g, x, B, dy, splits, part, &S, status, s);
-  if (st != ALEXNET_OK) return st;
-  ConvMap m{Cout, K, g.Cg(), groups, 0};
-  return reduce_wgrad(m, part, S, dw, sc, s);
+  GemmDesc d;
+  if (!conv_desc_wgrad(&d, cs, x, dy, part, splits, num_sms(), status))
+    return ALEXNET_ERR_UNSUPPORTED;
+  if (cudaError_t e = gemm_launch(d, s)) return done(e);
+  return reduce_wgrad(ConvMap{Cout, K, cs.Cg, groups, 0, cs.P()}, part, d.args.splits, dw, sc, s);
 }
 
 alexnet_status alexnet_op_conv1_wgrad(const void* x, int B, const void* dy, int splits, float* dw,
@@ -285,20 +178,20 @@ alexnet_status alexnet_op_conv1_wgrad(const void* x, int B, const void* dy, int 
   if (!x || !dy || !dw || B < 1) return ALEXNET_ERR_INVALID_ARG;
   Scratch sc(ws, ws_bytes);
   int* status = sc.take<int>(1);
-  bf16* xs = sc.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 48);
+  bf16* xs = sc.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 64);
   const int Kb = (B * 55 * 55 + 63) / 64;
   const int smax = splits > 0 ? (splits < Kb ? splits : Kb) : Kb;
-  float* part = sc.take<float>(static_cast<size_t>(smax) * 96 * 432);
+  float* part = sc.take<float>(static_cast<size_t>(smax) * 96 * 576);
   if (!status || !xs || !part) return ALEXNET_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaMemsetAsync(status, 0, 4, s);
   launch_s2d(static_cast<const bf16*>(x), xs, B, s);
-  ConvGeom g{57, 57, 48, 96, 3, 0, 1, 55, 55};
-  int S = 0;
-  alexnet_status st = run_conv_wgrad(g, xs, B, dy, splits, part, &S, status, s);
-  if (st != ALEXNET_OK) return st;
-  ConvMap m{96, 11, 3, 1, 1};
-  return reduce_wgrad(m, part, S, dw, sc, s);
+  GemmDesc d;
+  if (!conv_desc_wgrad(&d, ConvShape{B, 57, 57, 64, 48, 96, 1, 3, 0}, xs, dy, part, splits,
+                       num_sms(), status))
+    return ALEXNET_ERR_UNSUPPORTED;
+  if (cudaError_t e = gemm_launch(d, s)) return done(e);
+  return reduce_wgrad(ConvMap{96, 11, 3, 1, 1, 64}, part, d.args.splits, dw, sc, s);
 }
 
 alexnet_status alexnet_op_fc_fwd(const void* x, int B, int In, const void* w, int Out, int splits,

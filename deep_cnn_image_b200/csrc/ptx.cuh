@@ -83,6 +83,21 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
       : "memory");
 }
 
+// im2col load of a 4-D NHWC tensor: pixelsPerColumn consecutive output
+// positions starting at (w, h, n) (top-left input corner of the filter window,
+// may be negative), each fetching the map's channelsPerPixel channels from
+// c at input position (w + off_w, h + off_h); out-of-range pixels are zero.
+__device__ __forceinline__ void tma_load_im2col_4d(uint32_t dst, const void* tmap, int c, int w,
+                                                   int h, int n, uint16_t off_w, uint16_t off_h,
+                                                   uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.im2col.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], {%7, %8};" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c), "r"(w), "r"(h), "r"(n),
+      "h"(off_w), "h"(off_h)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async
 // 16-byte global->shared copy; src_bytes = 0 writes 16 zero bytes.
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {

@@ -124,10 +124,11 @@ ALEXNET_API alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst
                                   void* stream);
 
 /* Launch accounting and GEMM timing of a handle's calls.  While enabled,
- * every tensor-core GEMM launch is bracketed by CUDA events on the call's
- * stream.  alexnet_stats_read synchronises that stream, fills *out with the
- * totals since the previous read (or since enabling) and resets them.
- *   launches:      kernels this library launched
+ * every tensor-core GEMM launch of alexnet_train_step / alexnet_forward is
+ * bracketed by CUDA events on the call's stream (inside a replayed CUDA graph
+ * as event nodes of that graph).  alexnet_stats_read synchronises that stream
+ * and fills *out for the most recent such call (zeros if none since enabling):
+ *   launches:      kernels this library launched for it
  *   gemm_launches: of which tensor-core GEMMs
  *   gemm_flops:    algorithmic FLOPs of those GEMMs (2 x multiply-adds of
  *                  the network's own layer shapes, padding not counted)
