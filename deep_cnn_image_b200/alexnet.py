@@ -70,6 +70,7 @@ def _load():
         "alexnet_op_conv_dgrad": (st, [vp, i, i, i, i, vp, i, i, i, i, vp, vp, vp, sz, vp]),
         "alexnet_op_conv_wgrad": (st, [vp, i, i, i, i, vp, i, i, i, i, i, vp, vp, sz, vp]),
         "alexnet_op_conv1_wgrad": (st, [vp, i, vp, i, vp, vp, sz, vp]),
+        "alexnet_op_conv_wgrad_noalloc": (st, [vp, i, i, i, i, vp, i, i, i, i, i, vp, vp]),
         "alexnet_op_fc_fwd": (st, [vp, i, i, vp, i, i, vp, vp, sz, vp]),
         "alexnet_op_fc_dgrad": (st, [vp, i, i, vp, i, i, vp, vp, sz, vp]),
         "alexnet_op_fc_wgrad": (st, [vp, vp, i, i, i, vp, vp, sz, vp]),
@@ -231,6 +232,13 @@ def op_conv_dgrad(dy, B, H, W, Cin, w, Cout, K, pad, groups, mask, dx, ws, strea
 def op_conv_wgrad(x, B, H, W, Cin, dy, Cout, K, pad, groups, splits, dw, ws, stream=None):
     return _op("alexnet_op_conv_wgrad", _ptr(x), B, H, W, Cin, _ptr(dy), Cout, K, pad, groups,
                splits, _ptr(dw), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def op_conv_wgrad_noalloc(x, B, H, W, Cin, dy, Cout, K, pad, groups, splits, dw, stream=None):
+    """alexnet_op_conv_wgrad without scratch: for callers that can neither pass
+    scratch memory nor let the library allocate (see alexnet_ops.h)."""
+    return _op("alexnet_op_conv_wgrad_noalloc", _ptr(x), B, H, W, Cin, _ptr(dy), Cout, K, pad,
+               groups, splits, _ptr(dw), _stream(stream))
 
 
 def op_conv1_wgrad(x, B, dy, splits, dw, ws, stream=None):

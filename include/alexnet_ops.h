@@ -56,6 +56,26 @@ ALEXNET_API alexnet_status alexnet_op_conv_wgrad(const void* x, int B, int H, in
                                      int splits, float* dw, void* ws, size_t ws_bytes,
                                      void* stream);
 
+/* The same weight gradient without caller scratch and without allocating:
+ * for callers that can neither pass this library scratch memory nor let it
+ * allocate device memory (for instance code running after a framework has
+ * reserved the whole device through its own allocator, or a service that
+ * forbids device allocation once it has started).  Arguments as in
+ * alexnet_op_conv_wgrad, minus ws/ws_bytes.  The split-K partial sums live
+ * in a 16 MiB array in this library's own device memory, which every GPU
+ * that loads the library holds until the process exits.  Its device address
+ * is looked up (cudaGetSymbolAddress) on the first call on each device, so
+ * that first call should come before any stream capture.  All calls share
+ * the array: calls whose work overlaps on the GPU race and must be ordered
+ * by the caller.  Returns ALEXNET_ERR_UNSUPPORTED when even one K-slice of
+ * partial sums (Cout * K * K * Cin/groups floats) exceeds the array; splits
+ * is reduced to what the array holds.  The pages have no counterpart: this
+ * is an integration convenience, not part of the method. */
+ALEXNET_API alexnet_status alexnet_op_conv_wgrad_noalloc(const void* x, int B, int H, int W,
+                                                         int Cin, const void* dy, int Cout, int K,
+                                                         int pad, int groups, int splits,
+                                                         float* dw, void* stream);
+
 /* conv1 weight gradient on a [B,227,227,3] input: dw fp32 [96][11][11][3]. */
 ALEXNET_API alexnet_status alexnet_op_conv1_wgrad(const void* x, int B, const void* dy, int splits,
                                       float* dw, void* ws, size_t ws_bytes, void* stream);
