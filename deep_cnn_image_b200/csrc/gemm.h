@@ -38,11 +38,7 @@ enum Epi : int {
   EPI_BF16_MASK = 1,  // out_bf16[row, col] = acc if mask[row, col] > 0 else 0
   EPI_F32 = 2,        // out_f32[split][group][row, col] = acc
   EPI_F32_T = 3,      // out_f32[split][group][col, row] = acc
-  EPI_SGD = 4,        // acc[row, col] is dL/dw of parameter col * ld_out + row: SGD update
-                      // of w, v (fp32) and of the bf16 copy; grads[...] = acc if non-null
 };
-
-struct HParams;
 
 struct GatherDesc {
   const __nv_bfloat16* src;  // NHWC map [B, H, W, C]
@@ -75,12 +71,6 @@ struct GemmArgs {
   const float* bias;       // nullable, indexed by col + g * col_goff
   const __nv_bfloat16* mask;
   long long ld_mask;
-  // EPI_SGD
-  float* sgd_w;
-  float* sgd_v;
-  __nv_bfloat16* sgd_shadow;
-  float* sgd_grads;
-  const HParams* hp;
   int* status;
 };
 

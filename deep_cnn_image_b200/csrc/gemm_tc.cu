@@ -107,38 +107,12 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, const TileCoor
         *reinterpret_cast<float4*>(out + col) =
             make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
-  } else if (a.epi == EPI_F32_T) {
+  } else {  // EPI_F32_T
     float* out = reinterpret_cast<float*>(a.out) + tc.sp * a.split_stride + g * a.group_stride;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int col = col0 + i;
       if (col < a.N) out[col * a.ld_out + row] = v[i];
-    }
-  } else {  // EPI_SGD: [S] 3.4 "Training Procedure Details" update rule
-    // acc[row, col] is dL/dw for the parameter at col * ld_out + row: for a
-    // fixed column the 32 lanes of a warp touch 32 consecutive parameters.
-    const float lr = a.hp->lr, mom = a.hp->momentum, wd = a.hp->weight_decay;
-    float wv[16], vv[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int col = col0 + i;
-      if (col < a.N) {
-        const long long idx = static_cast<long long>(col) * a.ld_out + row;
-        wv[i] = a.sgd_w[idx];
-        vv[i] = a.sgd_v[idx];
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int col = col0 + i;
-      if (col >= a.N) continue;
-      const long long idx = static_cast<long long>(col) * a.ld_out + row;
-      const float vn = mom * vv[i] - wd * lr * wv[i] - lr * v[i];
-      const float wn = wv[i] + vn;
-      a.sgd_w[idx] = wn;
-      a.sgd_v[idx] = vn;
-      a.sgd_shadow[idx] = __float2bfloat16_rn(wn);
-      if (a.sgd_grads) a.sgd_grads[idx] = v[i];
     }
   }
 }

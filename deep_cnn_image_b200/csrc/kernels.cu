@@ -75,43 +75,58 @@ __global__ void k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs, int B) 
 // ------------------------------------------------------------------ LRN
 // [S] 3.4 "Local Response Normalization": b_i = a_i / (k + alpha * sum_{|j-i|<=2} a_j^2)^beta
 // with the window clipped to the layer's channels (n = 5).
+// Each thread owns one 8-channel chunk; consecutive lanes own consecutive
+// chunks, so the channel halo comes from the neighbouring lanes (explicit
+// loads only at the warp's edges).
 __global__ void k_lrn_fwd(const bf16* __restrict__ a, bf16* __restrict__ b, long long P, int C,
                           float k, float alpha, float beta) {
   const uint32_t chunks = static_cast<uint32_t>(C) >> 3;
   const uint32_t n = static_cast<uint32_t>(P) * chunks;
-  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
-    const uint32_t p = t / chunks;
-    const int c0 = static_cast<int>(t - p * chunks) * 8;
+  const int lane = threadIdx.x & 31;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; __any_sync(0xffffffffu, t < n);
+       t += stride) {
+    const bool active = t < n;
+    const uint32_t p = active ? t / chunks : 0;
+    const int c0 = active ? static_cast<int>(t - p * chunks) * 8 : 0;
     const bf16* ap = a + static_cast<size_t>(p) * C;
+    float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (active) unpack8(*reinterpret_cast<const uint4*>(ap + c0), f);
     float v[12];
-    {
-      float f[8];
-      unpack8(*reinterpret_cast<const uint4*>(ap + c0), f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[2 + i] = f[i];
+    for (int i = 0; i < 8; ++i) v[2 + i] = f[i];
+    const float up6 = __shfl_up_sync(0xffffffffu, f[6], 1), up7 = __shfl_up_sync(0xffffffffu, f[7], 1);
+    const float dn0 = __shfl_down_sync(0xffffffffu, f[0], 1), dn1 = __shfl_down_sync(0xffffffffu, f[1], 1);
+    v[0] = v[1] = v[10] = v[11] = 0.f;
+    if (active && c0 > 0) {
+      if (lane > 0) {
+        v[0] = up6;
+        v[1] = up7;
+      } else {
+        const float2 lo = ld_bf16x2(ap + c0 - 2);
+        v[0] = lo.x;
+        v[1] = lo.y;
+      }
     }
-    if (c0 > 0) {
-      const float2 lo = ld_bf16x2(ap + c0 - 2);
-      v[0] = lo.x;
-      v[1] = lo.y;
-    } else {
-      v[0] = v[1] = 0.f;
+    if (active && c0 + 8 < C) {
+      if (lane < 31) {
+        v[10] = dn0;
+        v[11] = dn1;
+      } else {
+        const float2 hi = ld_bf16x2(ap + c0 + 8);
+        v[10] = hi.x;
+        v[11] = hi.y;
+      }
     }
-    if (c0 + 8 < C) {
-      const float2 hi = ld_bf16x2(ap + c0 + 8);
-      v[10] = hi.x;
-      v[11] = hi.y;
-    } else {
-      v[10] = v[11] = 0.f;
-    }
+    if (!active) continue;
     float o[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       float sum = 0.f;
 #pragma unroll
       for (int j = 0; j < 5; ++j) sum += v[i + j] * v[i + j];
-      const float s = k + alpha * sum;
-      o[i] = v[i + 2] * __powf(s, -beta);
+      const float sc = k + alpha * sum;
+      o[i] = v[i + 2] * __powf(sc, -beta);
     }
     *reinterpret_cast<uint4*>(b + static_cast<size_t>(p) * C + c0) = pack8(o);
   }
@@ -124,38 +139,70 @@ __global__ void k_lrn_bwd(const bf16* __restrict__ a, const bf16* __restrict__ g
                           float beta) {
   const uint32_t chunks = static_cast<uint32_t>(C) >> 3;
   const uint32_t n = static_cast<uint32_t>(P) * chunks;
-  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
-    const uint32_t p = t / chunks;
-    const int c0 = static_cast<int>(t - p * chunks) * 8;
+  const int lane = threadIdx.x & 31;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; __any_sync(0xffffffffu, t < n);
+       t += stride) {
+    const bool active = t < n;
+    const uint32_t p = active ? t / chunks : 0;
+    const int c0 = active ? static_cast<int>(t - p * chunks) * 8 : 0;
     const bf16* ap = a + static_cast<size_t>(p) * C;
     const bf16* gp = g + static_cast<size_t>(p) * C;
+    float fa[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float fg[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (active) {
+      unpack8(*reinterpret_cast<const uint4*>(ap + c0), fa);
+      unpack8(*reinterpret_cast<const uint4*>(gp + c0), fg);
+    }
     float av[16];  // channels c0-4 .. c0+11
     float gv[12];  // channels c0-2 .. c0+9
 #pragma unroll
     for (int i = 0; i < 16; ++i) av[i] = 0.f;
 #pragma unroll
     for (int i = 0; i < 12; ++i) gv[i] = 0.f;
-    {
-      float f[8];
-      unpack8(*reinterpret_cast<const uint4*>(ap + c0), f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) av[4 + i] = f[i];
-      unpack8(*reinterpret_cast<const uint4*>(gp + c0), f);
+    for (int i = 0; i < 8; ++i) {
+      av[4 + i] = fa[i];
+      gv[2 + i] = fg[i];
+    }
+    float ua[4], ug[2], da_[4], dg[2];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) gv[2 + i] = f[i];
+    for (int i = 0; i < 4; ++i) {
+      ua[i] = __shfl_up_sync(0xffffffffu, fa[4 + i], 1);
+      da_[i] = __shfl_down_sync(0xffffffffu, fa[i], 1);
     }
-    if (c0 > 0) {
-      const float2 a0 = ld_bf16x2(ap + c0 - 4), a1 = ld_bf16x2(ap + c0 - 2);
-      av[0] = a0.x; av[1] = a0.y; av[2] = a1.x; av[3] = a1.y;
-      const float2 g1 = ld_bf16x2(gp + c0 - 2);
-      gv[0] = g1.x; gv[1] = g1.y;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      ug[i] = __shfl_up_sync(0xffffffffu, fg[6 + i], 1);
+      dg[i] = __shfl_down_sync(0xffffffffu, fg[i], 1);
     }
-    if (c0 + 8 < C) {
-      const float2 a0 = ld_bf16x2(ap + c0 + 8), a1 = ld_bf16x2(ap + c0 + 10);
-      av[12] = a0.x; av[13] = a0.y; av[14] = a1.x; av[15] = a1.y;
-      const float2 g1 = ld_bf16x2(gp + c0 + 8);
-      gv[10] = g1.x; gv[11] = g1.y;
+    if (active && c0 > 0) {
+      if (lane > 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) av[i] = ua[i];
+        gv[0] = ug[0];
+        gv[1] = ug[1];
+      } else {
+        const float2 a0 = ld_bf16x2(ap + c0 - 4), a1 = ld_bf16x2(ap + c0 - 2);
+        av[0] = a0.x; av[1] = a0.y; av[2] = a1.x; av[3] = a1.y;
+        const float2 g1 = ld_bf16x2(gp + c0 - 2);
+        gv[0] = g1.x; gv[1] = g1.y;
+      }
     }
+    if (active && c0 + 8 < C) {
+      if (lane < 31) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) av[12 + i] = da_[i];
+        gv[10] = dg[0];
+        gv[11] = dg[1];
+      } else {
+        const float2 a0 = ld_bf16x2(ap + c0 + 8), a1 = ld_bf16x2(ap + c0 + 10);
+        av[12] = a0.x; av[13] = a0.y; av[14] = a1.x; av[15] = a1.y;
+        const float2 g1 = ld_bf16x2(gp + c0 + 8);
+        gv[10] = g1.x; gv[11] = g1.y;
+      }
+    }
+    if (!active) continue;
     // s_i and t_i = g_i a_i s_i^(-beta-1) for channels c0-2 .. c0+9 (index i+2 in av)
     float sp[12], tt[12];
 #pragma unroll
@@ -163,10 +210,10 @@ __global__ void k_lrn_bwd(const bf16* __restrict__ a, const bf16* __restrict__ g
       float sum = 0.f;
 #pragma unroll
       for (int j = 0; j < 5; ++j) sum += av[i + j] * av[i + j];
-      const float s = k + alpha * sum;
-      const float sb = __powf(s, -beta);
+      const float sc = k + alpha * sum;
+      const float sb = __powf(sc, -beta);
       sp[i] = sb;
-      tt[i] = gv[i] * av[i + 2] * (sb / s);
+      tt[i] = gv[i] * av[i + 2] * (sb / sc);
     }
     float o[8];
 #pragma unroll
@@ -198,8 +245,10 @@ __global__ void k_lrn_fwd_f32(const float* __restrict__ a, float* __restrict__ b
 
 // ------------------------------------------------------------------ pooling
 // [S] 3.4 "Overlapping Pooling": max over z x z windows at stride st, no padding.
+template <int Z>
 __global__ void k_pool_fwd(const bf16* __restrict__ x, bf16* __restrict__ y,
-                           uint8_t* __restrict__ am, int B, int H, int W, int C, int z, int st) {
+                           uint8_t* __restrict__ am, int B, int H, int W, int C, int st) {
+  constexpr int z = Z;
   const uint32_t Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
   const uint32_t chunks = static_cast<uint32_t>(C) >> 3;
   const uint32_t n = static_cast<uint32_t>(B) * Ho * Wo * chunks;
@@ -213,10 +262,16 @@ __global__ void k_pool_fwd(const bf16* __restrict__ x, bf16* __restrict__ y,
     float best[8];
     int arg[8];
     const bf16* xb = x + (static_cast<size_t>(b * H + oh * st) * W + ow * st) * C + c0;
+    uint4 win[Z * Z];
+#pragma unroll
+    for (int q = 0; q < Z * Z; ++q)
+      win[q] = *reinterpret_cast<const uint4*>(xb + (static_cast<size_t>(q / Z) * W + q % Z) * C);
+#pragma unroll
     for (int dy = 0; dy < z; ++dy)
+#pragma unroll
       for (int dx = 0; dx < z; ++dx) {
         float f[8];
-        unpack8(*reinterpret_cast<const uint4*>(xb + (static_cast<size_t>(dy) * W + dx) * C), f);
+        unpack8(win[dy * Z + dx], f);
         const int off = dy * z + dx;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -469,18 +524,51 @@ __global__ void k_loss_mean(const float* __restrict__ rows, int B, float* out1, 
 }
 
 // ------------------------------------------------------------------ bias gradients
-constexpr int kColsumRows = 256;
+constexpr int kColsumRows = 128;
 
+// Column sums of a bf16 [rows, cols] matrix (cols % 8 == 0) over chunks of
+// kColsumRows rows: thread (lane row rl, column group cg) sums 8 columns over
+// rows r0 + rl, r0 + rl + R, ...; the R lane rows are then added in order.
 __global__ void k_colsum_partial(const bf16* __restrict__ m, long long rows, int cols,
                                  float* __restrict__ partial) {
-  const int chunk = blockIdx.x;
-  const int col = blockIdx.y * blockDim.x + threadIdx.x;
-  if (col >= cols) return;
-  const long long r0 = 1LL * chunk * kColsumRows;
+  __shared__ float red[4096];
+  const int G = cols >> 3;
+  const long long r0 = 1LL * blockIdx.x * kColsumRows;
   const long long r1 = min(rows, r0 + kColsumRows);
-  float s = 0.f;
-  for (long long r = r0; r < r1; ++r) s += __bfloat162float(m[r * cols + col]);
-  partial[1LL * chunk * cols + col] = s;
+  const int t = threadIdx.x;
+  if (G > static_cast<int>(blockDim.x)) {
+    for (int cg = t; cg < G; cg += blockDim.x) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (long long r = r0; r < r1; ++r) {
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4*>(m + r * cols + cg * 8), f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += f[i];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) partial[1LL * blockIdx.x * cols + cg * 8 + i] = acc[i];
+    }
+    return;
+  }
+  const int R = blockDim.x / G;
+  const int cg = t % G, rl = t / G;
+  if (rl < R) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (long long r = r0 + rl; r < r1; r += R) {
+      float f[8];
+      unpack8(*reinterpret_cast<const uint4*>(m + r * cols + cg * 8), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += f[i];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[rl * cols + cg * 8 + i] = acc[i];
+  }
+  __syncthreads();
+  for (int c = t; c < cols; c += blockDim.x) {
+    float v = 0.f;
+    for (int q = 0; q < R; ++q) v += red[q * cols + c];
+    partial[1LL * blockIdx.x * cols + c] = v;
+  }
 }
 
 // ------------------------------------------------------------------ SGD
@@ -901,8 +989,11 @@ void launch_lrn_fwd_f32(const float* a, float* b, long long P, int C, int, float
 void launch_pool_fwd(const bf16* x, bf16* y, uint8_t* am, int B, int H, int W, int C, int z,
                      int st, cudaStream_t s) {
   const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
-  k_pool_fwd<<<grid_for(1LL * B * Ho * Wo * (C / 8), 256), 256, 0, s>>>(x, y, am, B, H, W, C, z,
-                                                                        st);
+  const int grid = grid_for(1LL * B * Ho * Wo * (C / 8), 256);
+  if (z == 3)
+    k_pool_fwd<3><<<grid, 256, 0, s>>>(x, y, am, B, H, W, C, st);
+  else
+    k_pool_fwd<2><<<grid, 256, 0, s>>>(x, y, am, B, H, W, C, st);
   count_launch();
 }
 void launch_pool_bwd(const bf16* dy, const uint8_t* am, const bf16* pooled, bf16* dx, int B,
@@ -948,8 +1039,7 @@ void launch_loss_mean(const float* loss_rows, int B, float* out1, float* out2, c
 int colsum_chunks(long long rows) { return static_cast<int>((rows + kColsumRows - 1) / kColsumRows); }
 void launch_colsum_partial(const bf16* m, long long rows, int cols, float* partial,
                            cudaStream_t s) {
-  dim3 grid(colsum_chunks(rows), (cols + 127) / 128);
-  k_colsum_partial<<<grid, 128, 0, s>>>(m, rows, cols, partial);
+  k_colsum_partial<<<colsum_chunks(rows), 256, 0, s>>>(m, rows, cols, partial);
   count_launch();
 }
 void launch_sgd_conv(float* w, float* v, const float* part, int S, const ConvMap& m, bf16* fwd,

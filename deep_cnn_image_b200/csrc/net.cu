@@ -327,33 +327,26 @@ bool desc_fc_dgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* w, flo
   return gemm_finalize(d, num_sms);
 }
 
-// FC weight gradient with the SGD update fused into the epilogue: the fp32
-// gradient never reaches memory (optionally kept in `grads` for checks).  The
-// product is computed transposed, D[i, o] = sum_b x[b, i] dz[b, o], so that a
-// warp's lanes (rows) address consecutive weights w[o][i].
-bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, float* w, float* v,
-                   bf16* shadow, float* grads, const HParams* hp, int B, int num_sms,
-                   int* status) {
+// FC weight gradient dW[o][i] = sum_b dz[b, o] x[b, i] (fp32, to scratch).
+bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, float* out, int B,
+                   int num_sms, int* status) {
   memset(d, 0, sizeof(*d));
   d->asrc = A_TMA_MN;
   d->bsrc = B_TMA_MN;
-  d->bn = 256;
+  d->bn = F.In % 256 == 0 ? 256 : 128;
   GemmArgs& a = d->args;
-  a.M = F.In;
-  a.N = F.Out;
+  a.M = F.Out;
+  a.N = F.In;
   a.Kblocks = (B + 63) / 64;
   a.groups = 1;
   a.kb_per_split = a.Kblocks;
-  a.epi = EPI_SGD;
+  a.epi = EPI_F32;
+  a.out = out;
   a.ld_out = F.In;
-  a.sgd_w = w;
-  a.sgd_v = v;
-  a.sgd_shadow = shadow;
-  a.sgd_grads = grads;
-  a.hp = hp;
+  a.split_stride = 0;
   a.status = status;
-  if (!tmap(&d->tmA, x, F.In, B, static_cast<uint64_t>(F.In) * 2, 64, 64)) return false;
-  if (!tmap(&d->tmB, dz, F.Out, B, static_cast<uint64_t>(F.Out) * 2, 64, 64)) return false;
+  if (!tmap(&d->tmA, dz, F.Out, B, static_cast<uint64_t>(F.Out) * 2, 64, 64)) return false;
+  if (!tmap(&d->tmB, x, F.In, B, static_cast<uint64_t>(F.In) * 2, 64, 64)) return false;
   return gemm_finalize(d, num_sms);
 }
 
@@ -396,10 +389,7 @@ bool build_plan(alexnet* h, int B, Plan* P) {
       return set_err(h, "fc forward plan");
     if (!desc_fc_dgrad(&P->fd[f], h->fc[f], dz[f], h->wf[5 + f], h->scratch, B, 0, ns, h->status))
       return set_err(h, "fc data-gradient plan");
-    const size_t wo = h->w_off[5 + f];
-    if (!desc_fc_wgrad(&P->fw[f], h->fc[f], dz[f], fin[f], h->params ? h->params + wo : nullptr,
-                       h->vel ? h->vel + wo : nullptr, h->wf[5 + f],
-                       h->grads ? h->grads + wo : nullptr, h->hp, B, ns, h->status))
+    if (!desc_fc_wgrad(&P->fw[f], h->fc[f], dz[f], fin[f], h->scratch, B, ns, h->status))
       return set_err(h, "fc weight-gradient plan");
   }
   if (h->scratch) {
@@ -666,7 +656,9 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     const FcL& F = h->fc[f];
     ALX_TRY(run_gemm(h, P->fd[f], P->fc_flops[f], s), "fc dgrad launch");
     launch_dgrad_finalize(h->scratch, P->fd[f].args.splits, B, F.In, mask[f], dxo[f], s);
-    ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s), "fc wgrad + SGD launch");
+    ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s), "fc wgrad launch");
+    launch_sgd_dense(h->params + h->w_off[5 + f], h->vel + h->w_off[5 + f], h->scratch,
+                     h->w_len[5 + f], h->wf[5 + f], gptr(h->w_off[5 + f]), h->hp, s);
     launch_colsum_partial(dz[f], B, F.Out, h->cpart, s);
     launch_sgd_bias(h->params + h->b_off[5 + f], h->vel + h->b_off[5 + f], h->cpart,
                     colsum_chunks(B), F.Out, gptr(h->b_off[5 + f]), h->hp, s);

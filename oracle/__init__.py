@@ -125,10 +125,10 @@ def lib():
                                              c_double, c_uint64, c_uint32, dp, dp]),
             "oracle_loss": (c_double, [netp, dp, dp, i32p, c_int, c_uint64, c_uint32]),
             "oracle_train_probe": (None, [netp, dp, dp, i32p, c_int, c_uint64, c_uint32, c_int,
-                                          dp, u8p, u8p, u8p]),
+                                          dp, u8p, u8p, u8p, POINTER(u8p)]),
             "oracle_train_step_given": (c_double, [netp, dp, dp, dp, i32p, c_int, c_double,
                                                    c_double, c_double, c_uint64, c_uint32, dp, dp,
-                                                   u8p, u8p, u8p]),
+                                                   u8p, u8p, u8p, POINTER(u8p)]),
             "oracle_maxpool_select": (None, [dp, u8p, c_int, c_int, c_int, c_int, c_int, c_int,
                                              dp]),
             "oracle_aug_draws": (None, [c_uint64, c_uint32, c_uint32, i32p, dp]),
@@ -419,11 +419,12 @@ def forward_probe(net, params, x, which, mode=1, seed=0, step=0):
 
 
 def train_step(net, params, velocity, x, labels, lr=0.01, momentum=0.9, wd=5e-4, seed=0,
-               step=0, given_argmax=None):
+               step=0, given_argmax=None, given_relu=None):
     """One step of [W] TRAIN_STEP.  Returns (loss, new_params, new_velocity,
     grads, logits).  given_argmax: optional {0|1|4: uint8 map} of pool window
     choices (for instance an implementation's own) used instead of the
-    oracle's."""
+    oracle's; given_relu: optional {0..4 conv, 5 FC6, 6 FC7: uint8 mask} of
+    ReLU sign decisions used instead of the oracle's own (z > 0)."""
     params = np.array(params, dtype=np.float64, copy=True)
     velocity = np.array(velocity, dtype=np.float64, copy=True)
     x, xp = _d(x)
@@ -432,10 +433,11 @@ def train_step(net, params, velocity, x, labels, lr=0.01, momentum=0.9, wd=5e-4,
     grads = np.zeros_like(params)
     logits = np.zeros((B, net.fc_n[2]))
     keep, ptrs = _am_ptrs(given_argmax)
+    keep2, relu = _relu_ptrs(given_relu)
     loss = lib().oracle_train_step_given(ctypes.byref(net), _p(params, c_double),
                                          _p(velocity, c_double), xp, _p(labels, ctypes.c_int32),
                                          B, lr, momentum, wd, seed, step, _p(grads, c_double),
-                                         _p(logits, c_double), *ptrs)
+                                         _p(logits, c_double), *ptrs, relu)
     return loss, params, velocity, grads, logits
 
 
@@ -469,17 +471,37 @@ def _am_ptrs(given):
     return keep, ptrs
 
 
-def train_probe(net, params, x, labels, which, seed=0, step=0, given_argmax=None):
+def _relu_ptrs(given):
+    """given: None or dict {0..4: conv mask, 5: FC6 mask, 6: FC7 mask} (uint8)."""
+    if not given:
+        return [], None
+    keep = []
+    arr = (POINTER(c_uint8) * 7)()
+    for i in range(7):
+        a = given.get(i)
+        if a is None:
+            arr[i] = None
+        else:
+            a = np.ascontiguousarray(a, dtype=np.uint8)
+            keep.append(a)
+            arr[i] = _p(a, c_uint8)
+    return keep, arr
+
+
+def train_probe(net, params, x, labels, which, seed=0, step=0, given_argmax=None,
+                given_relu=None):
     """One intermediate gradient of a training step (see oracle_train_probe), flat.
-    given_argmax: optional {0|1|4: uint8 map} of pool window choices to use."""
+    given_argmax: optional {0|1|4: uint8 map} of pool window choices to use;
+    given_relu: optional {0..4, 5, 6: uint8 mask} of ReLU sign decisions."""
     params, pp = _d(params)
     x, xp = _d(x)
     labels = np.ascontiguousarray(labels, dtype=np.int32)
     B = x.shape[0]
     out = np.zeros(B * gprobe_size(net, which))
     keep, ptrs = _am_ptrs(given_argmax)
+    keep2, relu = _relu_ptrs(given_relu)
     lib().oracle_train_probe(ctypes.byref(net), pp, xp, _p(labels, ctypes.c_int32), B, seed, step,
-                             which, _p(out, c_double), *ptrs)
+                             which, _p(out, c_double), *ptrs, relu)
     return out
 
 

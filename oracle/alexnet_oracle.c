@@ -610,6 +610,7 @@ typedef struct {
   double* fc_out[2];    /* after dropout / scaling */
   uint8_t* keep[2];
   double* logits;
+  const uint8_t* relu_given[7];  /* optional ReLU decisions: conv1..5, FC6, FC7 */
 } fwd_cache;
 
 static double* dalloc(int64_t n) { return (double*)calloc((size_t)(n > 0 ? n : 1), sizeof(double)); }
@@ -633,19 +634,43 @@ static void cache_free(fwd_cache* c) {
 /* mode: 0 = training (dropout masks drawn), 1 = inference (x (1-p)). */
 static void net_forward_given(const oracle_net* net, const double* params, const double* x,
                               int B, int mode, uint64_t seed, uint32_t step,
-                              const uint8_t* const* am_in, fwd_cache* c);
+                              const uint8_t* const* am_in, const uint8_t* const* relu_in,
+                              fwd_cache* c);
 
 static void net_forward(const oracle_net* net, const double* params, const double* x, int B,
                         int mode, uint64_t seed, uint32_t step, fwd_cache* c) {
-  net_forward_given(net, params, x, B, mode, seed, step, NULL, c);
+  net_forward_given(net, params, x, B, mode, seed, step, NULL, NULL, c);
+}
+
+/* ReLU with the sign decision optionally given: out = z where the unit is
+ * taken as active (given[e] != 0, or z > 0 when given is NULL), else 0. */
+static void relu_decided(double* z, int64_t n, const uint8_t* given) {
+  if (!given) {
+    oracle_relu(z, n);
+    return;
+  }
+  for (int64_t i = 0; i < n; ++i) z[i] = given[i] ? z[i] : 0.0;
+}
+
+/* The ReLU derivative with the same decision: d passes where active. */
+static void relu_bwd_decided(const double* y, double* d, int64_t n, const uint8_t* given) {
+  if (!given) {
+    oracle_relu_bwd(y, d, n);
+    return;
+  }
+  for (int64_t i = 0; i < n; ++i) d[i] = given[i] ? d[i] : 0.0;
 }
 
 /* am_in (nullable; entries nullable): window choices of the max-pools after
- * conv l, used instead of the oracle's own argmax. */
+ * conv l, used instead of the oracle's own argmax.  relu_in (nullable;
+ * entries nullable): ReLU sign decisions of conv1..conv5, FC6, FC7 used
+ * instead of the oracle's own (z > 0). */
 static void net_forward_given(const oracle_net* net, const double* params, const double* x,
                               int B, int mode, uint64_t seed, uint32_t step,
-                              const uint8_t* const* am_in, fwd_cache* c) {
+                              const uint8_t* const* am_in, const uint8_t* const* relu_in,
+                              fwd_cache* c) {
   memset(c, 0, sizeof(*c));
+  for (int i = 0; i < 7; ++i) c->relu_given[i] = relu_in ? relu_in[i] : NULL;
   net_shapes(net, &c->s);
   const oracle_shapes* s = &c->s;
   const double* in = x;
@@ -658,7 +683,7 @@ static void net_forward_given(const oracle_net* net, const double* params, const
     oracle_conv_fwd(in, B, H, H, C, params + s->w_off[l], params + s->b_off[l], Co,
                     net->conv_k[l], net->conv_s[l], net->conv_p[l], net->conv_g[l],
                     c->relu_out[l]);
-    oracle_relu(c->relu_out[l], n);
+    relu_decided(c->relu_out[l], n, c->relu_given[l]);
     const double* cur = c->relu_out[l];
     if (net->lrn_after[l]) {
       c->lrn_out[l] = dalloc(n);
@@ -698,7 +723,7 @@ static void net_forward_given(const oracle_net* net, const double* params, const
     double* z = dalloc((int64_t)B * Out);
     oracle_fc_fwd(c->fc_in[f], B, In, params + s->w_off[5 + f], params + s->b_off[5 + f], Out, z);
     if (f < 2) {
-      oracle_relu(z, (int64_t)B * Out);
+      relu_decided(z, (int64_t)B * Out, c->relu_given[5 + f]);
       c->fc_relu[f] = z;
       double* d = dalloc((int64_t)B * Out);
       c->keep[f] = (uint8_t*)calloc((size_t)B * Out, 1);
@@ -772,27 +797,28 @@ static double train_step_probe(const oracle_net* net, double* params, double* ve
                                const double* x, const int32_t* labels, int B, double lr,
                                double momentum, double wd, uint64_t seed, uint32_t step,
                                double* grads, double* logits, int probe, double* probe_out,
-                               const uint8_t* const* am_in);
+                               const uint8_t* const* am_in, const uint8_t* const* relu_in);
 
 ORACLE_API double oracle_train_step(const oracle_net* net, double* params, double* velocity,
                                     const double* x, const int32_t* labels, int B, double lr,
                                     double momentum, double wd, uint64_t seed, uint32_t step,
                                     double* grads, double* logits) {
   return train_step_probe(net, params, velocity, x, labels, B, lr, momentum, wd, seed, step,
-                          grads, logits, -1, NULL, NULL);
+                          grads, logits, -1, NULL, NULL, NULL);
 }
 
 /* The same step with the max-pool window choices given (am1, am2, am5 for the
- * pools after conv1, conv2, conv5; each nullable). */
+ * pools after conv1, conv2, conv5; each nullable) and the ReLU sign decisions
+ * given (relu7: 7 nullable masks for conv1..conv5, FC6, FC7; nullable). */
 ORACLE_API double oracle_train_step_given(const oracle_net* net, double* params, double* velocity,
                                           const double* x, const int32_t* labels, int B,
                                           double lr, double momentum, double wd, uint64_t seed,
                                           uint32_t step, double* grads, double* logits,
                                           const uint8_t* am1, const uint8_t* am2,
-                                          const uint8_t* am5) {
+                                          const uint8_t* am5, const uint8_t* const* relu7) {
   const uint8_t* am_in[5] = {am1, am2, NULL, NULL, am5};
   return train_step_probe(net, params, velocity, x, labels, B, lr, momentum, wd, seed, step,
-                          grads, logits, -1, NULL, am_in);
+                          grads, logits, -1, NULL, am_in, relu7);
 }
 
 /* Intermediate gradients of a training step (no update is kept):
@@ -802,7 +828,8 @@ ORACLE_API double oracle_train_step_given(const oracle_net* net, double* params,
 ORACLE_API void oracle_train_probe(const oracle_net* net, const double* params, const double* x,
                                    const int32_t* labels, int B, uint64_t seed, uint32_t step,
                                    int which, double* out, const uint8_t* am1,
-                                   const uint8_t* am2, const uint8_t* am5) {
+                                   const uint8_t* am2, const uint8_t* am5,
+                                   const uint8_t* const* relu7) {
   const uint8_t* am_in[5] = {am1, am2, NULL, NULL, am5};
   oracle_shapes s;
   net_shapes(net, &s);
@@ -810,7 +837,7 @@ ORACLE_API void oracle_train_probe(const oracle_net* net, const double* params, 
   double* v = dalloc(s.n_params);
   memcpy(p, params, sizeof(double) * (size_t)s.n_params);
   train_step_probe(net, p, v, x, labels, B, 0.0, 0.0, 0.0, seed, step, NULL, NULL, which, out,
-                   am_in);
+                   am_in, relu7);
   free(p);
   free(v);
 }
@@ -823,9 +850,9 @@ static double train_step_probe(const oracle_net* net, double* params, double* ve
                                const double* x, const int32_t* labels, int B, double lr,
                                double momentum, double wd, uint64_t seed, uint32_t step,
                                double* grads, double* logits, int probe, double* probe_out,
-                               const uint8_t* const* am_in) {
+                               const uint8_t* const* am_in, const uint8_t* const* relu_in) {
   fwd_cache c;
-  net_forward_given(net, params, x, B, 0, seed, step, am_in, &c);
+  net_forward_given(net, params, x, B, 0, seed, step, am_in, relu_in, &c);
   const oracle_shapes* s = &c.s;
   const int N = net->fc_n[2];
   if (logits) memcpy(logits, c.logits, sizeof(double) * (size_t)B * N);
@@ -852,7 +879,7 @@ static double train_step_probe(const oracle_net* net, double* params, double* ve
         if (net->dropout_on) d = c.keep[f - 1][e] ? d : 0.0;
         dcur[e] = d;
       }
-      oracle_relu_bwd(c.fc_relu[f - 1], dcur, n);
+      relu_bwd_decided(c.fc_relu[f - 1], dcur, n, c.relu_given[5 + f - 1]);
       probe_copy(probe, 80 + (3 - f), dcur, n, probe_out);
     }
   }
@@ -875,7 +902,7 @@ static double train_step_probe(const oracle_net* net, double* params, double* ve
       free(dcur);
       dcur = d;
     }
-    oracle_relu_bwd(c.relu_out[l], dcur, n);
+    relu_bwd_decided(c.relu_out[l], dcur, n, c.relu_given[l]);
     probe_copy(probe, 50 + l, dcur, n, probe_out);
     const int H = s->hw[l];
     const int Ci = l == 0 ? net->in_c : net->conv_c[l - 1];

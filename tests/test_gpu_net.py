@@ -61,6 +61,43 @@ def _gpu_pool_choices(net, B):
     return out
 
 
+CONV_MAPS = ((0, 55, 96), (1, 27, 256), (2, 13, 384), (3, 13, 384), (4, 13, 256))
+
+
+def _gpu_relu_decisions(net, B):
+    """The GPU's ReLU sign decisions of its last forward: unit active iff its
+    stored output is positive (conv1..conv5, then FC6, FC7 after dropout)."""
+    import torch
+    out = {}
+    for l, side, C in CONV_MAPS:
+        t = torch.empty(B * side * side * C, dtype=torch.bfloat16, device="cuda")
+        net.debug_copy(l, t)
+        out[l] = (host(t) > 0).astype(np.uint8)
+    for f in range(2):
+        t = torch.empty(B * 4096, dtype=torch.bfloat16, device="cuda")
+        net.debug_copy(30 + f, t)
+        out[5 + f] = (host(t) > 0).astype(np.uint8)
+    return out
+
+
+def _check_relu_valid(onet, op, xr, relu, seed, step):
+    """Where the GPU's sign decision differs from the oracle's, the unit sits
+    at the ReLU's kink: the active side's value is within 5% of the layer's
+    RMS activation.  Returns the fraction of units decided differently."""
+    flips = []
+    for l in range(7):
+        which = oracle.PROBE_RELU + l if l < 5 else oracle.PROBE_FC + (l - 5)
+        a = oracle.forward_probe(onet, op, xr, which, mode=0, seed=seed, step=step)
+        mine = (a > 0)
+        theirs = relu[l].ravel().astype(bool)
+        diff = mine != theirs
+        rms = np.sqrt(np.mean(a * a))
+        # oracle active but GPU not: the oracle's value is small
+        assert np.all(a[diff & mine] <= 0.05 * rms), l
+        flips.append(float(diff.mean()))
+    return flips
+
+
 def _check_choices_valid(net, onet, op, xr, choices, seed, step):
     """The GPU's window choices are exactly the first maxima of the GPU's own
     pooled-from map (bit-exact on identical inputs), and that map matches the
@@ -146,9 +183,10 @@ def test_fp32_path_matches_oracle(ax):
 
 def _train_compare(ax, B, seed, grouped=True, lr=0.01):
     """One GPU training step and the oracle's step on the same inputs.  The
-    max-pool window choices are a decision taken on rounded values: the
-    oracle takes the GPU's own choices after checking each one is a maximum
-    of its own map at bf16 resolution (identical inputs to that decision)."""
+    max-pool window choices and the ReLU sign decisions are decisions taken on
+    rounded values: the oracle takes the GPU's own, after checking that each
+    pool choice is the first maximum of the GPU's own map and that every
+    differing sign decision sits at the ReLU's kink."""
     import torch
     net = _make(ax, batch_max=B, keep_grads=1, grouped=int(grouped), seed=seed)
     n = ax.param_count(net.cfg)
@@ -169,9 +207,13 @@ def _train_compare(ax, B, seed, grouped=True, lr=0.01):
     op = _oracle_params(params, onet)
     choices = _gpu_pool_choices(net, B)
     _check_choices_valid(net, onet, op, xr, choices, net.cfg.seed, step)
+    relu = _gpu_relu_decisions(net, B)
+    _check_relu_valid(onet, op, xr, relu, net.cfg.seed, step)
     wloss, _, _, wg, _ = oracle.train_step(onet, op, np.zeros(n), xr, y, lr=lr,
-                                           seed=net.cfg.seed, step=step, given_argmax=choices)
+                                           seed=net.cfg.seed, step=step, given_argmax=choices,
+                                           given_relu=relu)
     net.choices = choices
+    net.relu = relu
     return net, host(loss)[0], grads.numpy(), blob.numpy(), wloss, wg, params, n, xr, y
 
 
@@ -210,7 +252,7 @@ def test_train_intermediate_gradients(ax):
         net.debug_copy(which, t)
         got[which] = host(t)
         want = oracle.train_probe(onet, op, xr, y, which, seed=seed, step=step,
-                                  given_argmax=net.choices)
+                                  given_argmax=net.choices, given_relu=net.relu)
         errs[which] = rel_l2(got[which], want)
     bad = {k: v for k, v in errs.items() if not v < TOL_BF16}
     assert not bad, (bad, errs)

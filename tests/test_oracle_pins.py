@@ -357,6 +357,37 @@ def test_given_pool_choices_reproduce_the_oracle_step():
     assert not np.allclose(c[3][wo:wo + wl], a[3][wo:wo + wl])
 
 
+def test_given_relu_decisions_reproduce_the_oracle_step():
+    """Passing the oracle's own ReLU sign decisions back in changes nothing;
+    flipping one unit's decision changes the gradients."""
+    r = np.random.default_rng(19)
+    net = oracle.small_net()
+    n = oracle.param_count(net)
+    params = r.standard_normal(n) * 0.2
+    xi = r.standard_normal((2, 67, 67, 3))
+    lab = np.array([1, 6], np.int32)
+    own = {}
+    for l in range(5):
+        a = oracle.forward_probe(net, params, xi, oracle.PROBE_RELU + l, mode=0, seed=3, step=2)
+        own[l] = (a > 0).astype(np.uint8)
+    for f in range(2):
+        # FC outputs after dropout: a dropped unit's decision does not matter
+        a = oracle.forward_probe(net, params, xi, oracle.PROBE_FC + f, mode=0, seed=3, step=2)
+        own[5 + f] = (a > 0).astype(np.uint8)
+    a = oracle.train_step(net, params, np.zeros(n), xi, lab, seed=3, step=2)
+    b = oracle.train_step(net, params, np.zeros(n), xi, lab, seed=3, step=2, given_relu=own)
+    assert a[0] == b[0]
+    np.testing.assert_array_equal(a[3], b[3])
+    flipped = dict(own)
+    m = own[2].copy()
+    i = int(np.flatnonzero(m)[0])
+    m[i] = 0
+    flipped[2] = m
+    c = oracle.train_step(net, params, np.zeros(n), xi, lab, seed=3, step=2, given_relu=flipped)
+    lay = oracle.param_layout(net)
+    assert not np.array_equal(c[3][lay[2][0]:lay[2][0] + lay[2][1]], a[3][lay[2][0]:lay[2][0] + lay[2][1]])
+
+
 def test_dropout_gradient_follows_mask():
     """Units dropped in FC6 get exactly zero gradient in FC6's weights' rows
     for every image where they are dropped: with batch 1 the whole row is 0."""
