@@ -9,7 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from ctypes import POINTER, c_float, c_int, c_int64, c_size_t, c_uint32, c_uint64, c_void_p
+from ctypes import POINTER, byref, c_float, c_int, c_int64, c_size_t, c_uint32, c_uint64, c_void_p
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libalexnet.so")
@@ -78,11 +78,17 @@ def _load():
         "alexnet_op_lrn_bwd": (st, [vp, vp, c_int64, i, c_float, c_float, c_float, vp, vp]),
         "alexnet_op_pool_fwd": (st, [vp, i, i, i, i, i, i, vp, vp, vp]),
         "alexnet_op_pool_bwd": (st, [vp, vp, vp, i, i, i, i, i, i, i, vp, vp]),
+        "alexnet_op_lrn_pool_fwd": (st, [vp, i, i, i, i, i, c_float, c_float, c_float, vp, vp, vp,
+                                         vp]),
+        "alexnet_op_pool_lrn_bwd": (st, [vp, vp, vp, i, i, i, i, i, c_float, c_float, c_float, vp,
+                                         vp, vp]),
         "alexnet_op_softmax_ce": (st, [vp, vp, i, i, vp, vp, vp, vp, sz, vp]),
         "alexnet_op_dropout_mask": (st, [c_uint64, c_uint32, c_uint32, c_float, i, i, vp, vp, sz,
                                          vp]),
         "alexnet_op_philox": (st, [vp, vp, i, vp, vp]),
         "alexnet_debug_copy": (st, [vp, i, vp, sz, vp]),
+        "alexnet_debug_keep": (st, [vp, i]),
+        "alexnet_conv_algo": (st, [vp, i, i, i, POINTER(c_int)]),
         "alexnet_stats_enable": (st, [vp, i]),
         "alexnet_stats_read": (st, [vp, POINTER(Stats)]),
     }
@@ -204,6 +210,18 @@ class AlexNet:
         return {"launches": st_.launches, "gemm_launches": st_.gemm_launches,
                 "gemm_flops": st_.gemm_flops, "gemm_ms": st_.gemm_ms}
 
+    def conv_algo(self, batch, layer, pass_):
+        """1 if convolution `layer` runs the shifted-box kernel for this batch
+        size in pass 0 (forward), 1 (data gradient) or 2 (weight gradient)."""
+        v = c_int(-1)
+        check(lib.alexnet_conv_algo(self.h, batch, layer, pass_, byref(v)))
+        return v.value
+
+    def debug_keep(self, keep=True):
+        """Also store the normalised maps and their gradients (debug_copy
+        10/11, 70/71) in later calls."""
+        return check(lib.alexnet_debug_keep(self.h, 1 if keep else 0))
+
     def debug_copy(self, which, dst, stream=None):
         return check(lib.alexnet_debug_copy(self.h, which, _ptr(dst), dst.numel() * dst.element_size(),
                                             _stream(stream)), self.h)
@@ -278,6 +296,16 @@ def op_pool_fwd(x, B, H, W, C, z, st, y, argmax, stream=None):
 def op_pool_bwd(dy, argmax, pooled, B, H, W, C, z, st, relu_mask, dx, stream=None):
     return _op("alexnet_op_pool_bwd", _ptr(dy), _ptr(argmax), _ptr(pooled), B, H, W, C, z, st,
                relu_mask, _ptr(dx), _stream(stream))
+
+
+def op_lrn_pool_fwd(a, B, H, W, C, z, k, alpha, beta, lo, y, argmax, stream=None):
+    return _op("alexnet_op_lrn_pool_fwd", _ptr(a), B, H, W, C, z, k, alpha, beta, _ptr(lo),
+               _ptr(y), _ptr(argmax), _stream(stream))
+
+
+def op_pool_lrn_bwd(dy, argmax, a, B, H, W, C, z, k, alpha, beta, dl, da, stream=None):
+    return _op("alexnet_op_pool_lrn_bwd", _ptr(dy), _ptr(argmax), _ptr(a), B, H, W, C, z, k,
+               alpha, beta, _ptr(dl), _ptr(da), _stream(stream))
 
 
 def op_softmax_ce(logits, labels, B, N, probs, dlogits, loss, ws, stream=None):

@@ -1,0 +1,670 @@
+// conv_box.cu -- the shifted-box convolution kernels (see conv_box.h).
+//
+// The operation is the stride-1 convolution of "ImageNet Classification
+// with Deep Convolutional Neural Networks" (summary page, 3.4 "Overall
+// Architecture"; "AlexNet and Deep CNNs", "Time complexity of one forward
+// pass"): a sum over the (kh, kw, cin) taps, here ordered chunk by chunk of
+// 64 input channels, tap by tap within a chunk.
+//
+// Both kernels are persistent (one 192-thread CTA per SM): warps 0-3 drain
+// tensor memory (epilogue), warp 4 issues TMA loads, warp 5 issues tcgen05
+// MMAs and owns the tensor memory.  Every mbarrier wait is bounded; on
+// expiry the kernel records a timeout in the status word and winds down.
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
+#include "conv_box.h"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace alx {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kSmemBudget = 227 * 1024;
+constexpr int kBarBytes = 1024;  // mbarriers, tmem slot, abort flag
+
+__host__ __device__ constexpr int pow2_cols(int n) {
+  return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : (n <= 256 ? 256 : 512)));
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Zero the operand rings once: rows of a stage that no box ever writes are
+// read by the MMA (for positions that are dropped) and must hold finite
+// values.
+__device__ __forceinline__ void zero_smem(uint8_t* p, int bytes) {
+  for (int i = threadIdx.x * 16; i < bytes; i += kThreads * 16)
+    *reinterpret_cast<uint4*>(p + i) = make_uint4(0, 0, 0, 0);
+}
+
+// ---------------------------------------------------------------- forward
+// Tile t = ((g * B + b) * tiles_img + ti) * n_tiles + n_t: output rows
+// ti * To_h .. of image b, output channels n_t * BN .. of group g.
+template <int BN, int NSUB>
+__global__ void __launch_bounds__(kThreads, 1)
+    conv_box_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                 const __grid_constant__ BoxArgs a, int stA, int stB, int a_bytes) {
+  constexpr int B_BYTES = BN * 128;
+  constexpr int ACC_BUFS = (2 * NSUB * BN <= 512) ? 2 : 1;
+  constexpr int TMEM_COLS = pow2_cols(ACC_BUFS * NSUB * BN);
+  constexpr uint32_t IDESC = idesc_bf16(128, BN, 0, 0);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + stA * a_bytes;
+  uint8_t* barp = smem + stA * a_bytes + stB * B_BYTES;
+  const uint32_t a_full = smem_u32(barp);
+  const uint32_t a_empty = a_full + 8 * stA;
+  const uint32_t b_full = a_empty + 8 * stA;
+  const uint32_t b_empty = b_full + 8 * stB;
+  const uint32_t acc_full = b_empty + 8 * stB;
+  const uint32_t acc_empty = acc_full + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barp + 8 * (2 * stA + 2 * stB + 4));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  zero_smem(smem, stA * a_bytes);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stA; ++s) {
+      mbar_init(a_full + 8 * s, 1);
+      mbar_init(a_empty + 8 * s, 1);
+    }
+    for (int s = 0; s < stB; ++s) {
+      mbar_init(b_full + 8 * s, 1);
+      mbar_init(b_empty + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full + 8 * i, 1);
+      mbar_init(acc_empty + 8 * i, 128);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  fence_proxy_async_smem();
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int total = a.n_tiles * a.tiles_img * a.B * a.groups;
+  const int taps = a.K * a.K;
+  const uint32_t box_bytes = static_cast<uint32_t>(a.Hb) * a.Wb * 128;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmW);
+      uint32_t ia = 0, ib = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int q = t;
+        const int n_t = q % a.n_tiles;
+        q /= a.n_tiles;
+        const int ti = q % a.tiles_img;
+        q /= a.tiles_img;
+        const int b = q % a.B;
+        const int g = q / a.B;
+        const int oh0 = ti * a.To_h;
+        for (int ch = 0; ch < a.cpt && ok; ++ch, ++ia) {
+          const int s = ia % stA;
+          if (!mbar_wait(a_empty + 8 * s, ((ia / stA) & 1) ^ 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(a_full + 8 * s, box_bytes);
+          tma_load_4d(sA + s * a_bytes, &tmX, g * a.cg_off + ch * 64, -a.pad, oh0 - a.pad, b,
+                      a_full + 8 * s);
+          for (int tap = 0; tap < taps; ++tap, ++ib) {
+            const int sb = ib % stB;
+            if (!mbar_wait(b_empty + 8 * sb, ((ib / stB) & 1) ^ 1, a.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(b_full + 8 * sb, B_BYTES);
+            tma_load_2d(sB + sb * B_BYTES, &tmW, (tap * a.cpt + ch) * 64, g * a.Og + n_t * BN,
+                        b_full + 8 * sb);
+          }
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      uint32_t ia = 0, ib = 0, tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tcount) {
+        const int acc = ACC_BUFS == 2 ? (tcount & 1) : 0;
+        const uint32_t aph = ACC_BUFS == 2 ? ((tcount >> 1) & 1) : (tcount & 1);
+        if (!mbar_wait(acc_empty + 8 * acc, aph ^ 1, a.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t dbase = tmem_base + acc * NSUB * BN;
+        for (int ch = 0; ch < a.cpt && ok; ++ch, ++ia) {
+          const int s = ia % stA;
+          if (!mbar_wait(a_full + 8 * s, (ia / stA) & 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t abox = sA + s * a_bytes;
+          for (int tap = 0; tap < taps; ++tap, ++ib) {
+            const int sb = ib % stB;
+            if (!mbar_wait(b_full + 8 * sb, (ib / stB) & 1, a.status, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int kh = tap / a.K, kw = tap - (tap / a.K) * a.K;
+            const uint32_t shift = static_cast<uint32_t>(kh * a.Wb + kw) * 128;
+            const uint32_t bt = sB + sb * B_BYTES;
+#pragma unroll
+            for (int sub = 0; sub < NSUB; ++sub) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t ad = smem_desc_sw128(abox + sub * 128 * 128 + shift + k * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(bt + k * 32, 16, 1024);
+                tc_mma_f16(dbase + sub * BN, ad, bd, IDESC, (ch | tap | k) != 0 ? 1u : 0u);
+              }
+            }
+            tc_commit(b_empty + 8 * sb);
+          }
+          if (!ok) break;
+          tc_commit(a_empty + 8 * s);
+        }
+        if (!ok) break;
+        tc_commit(acc_full + 8 * acc);
+      }
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------------- epilogue
+    uint32_t tcount = 0;
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tcount) {
+      int q = t;
+      const int n_t = q % a.n_tiles;
+      q /= a.n_tiles;
+      const int ti = q % a.tiles_img;
+      q /= a.tiles_img;
+      const int b = q % a.B;
+      const int g = q / a.B;
+      const int oh0 = ti * a.To_h;
+      const int acc = ACC_BUFS == 2 ? (tcount & 1) : 0;
+      const uint32_t aph = ACC_BUFS == 2 ? ((tcount >> 1) & 1) : (tcount & 1);
+      if (!mbar_wait(acc_full + 8 * acc, aph, a.status, abort_flag)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int sub = 0; sub < NSUB; ++sub) {
+        const int m = sub * 128 + warp * 32 + lane;
+        const int r = m / a.Wb;
+        const int col = m - r * a.Wb;
+        const int oh = oh0 + r;
+        const bool valid = r < a.To_h && oh < a.Ho && col < a.Wo;
+        const long long row = (static_cast<long long>(b) * a.Ho + oh) * a.Wo + col;
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
+                            acc * NSUB * BN + sub * BN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(tb + c0, v);
+          if (!valid) continue;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int n = n_t * BN + c0 + 8 * h;
+            if (n >= a.Og) continue;
+            const long long cg = static_cast<long long>(g) * a.col_goff + n;
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = v[8 * h + i];
+            if (a.epi == EPI_BF16) {
+              if (a.bias) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] += a.bias[cg + i];
+              }
+              if (a.relu) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = f[i] > 0.f ? f[i] : 0.f;
+              }
+            } else {
+              const uint4 mv = *reinterpret_cast<const uint4*>(a.mask + row * a.ld_mask + cg);
+              const __nv_bfloat16* mb = reinterpret_cast<const __nv_bfloat16*>(&mv);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) f[i] = __bfloat162float(mb[i]) > 0.f ? f[i] : 0.f;
+            }
+            uint4 o;
+            o.x = pack2(f[0], f[1]);
+            o.y = pack2(f[2], f[3]);
+            o.z = pack2(f[4], f[5]);
+            o.w = pack2(f[6], f[7]);
+            *reinterpret_cast<uint4*>(out + row * a.ld_out + cg) = o;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty + 8 * acc);
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    for (int i = 0; i < 1000; ++i) __nanosleep(1000);
+  }
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- weight gradient
+// Item i = ((((split * groups + g) * cpt + ch) * n_tiles + n_t) * tsets + ts):
+// tap pairs [ts * npairs / tsets, (ts + 1) * npairs / tsets) of input chunk
+// ch, output channels n_t * BN .., over the position tiles of one split.
+// Pair q covers taps 2q and 2q + 1; for an odd tap count the last pair's
+// second half re-reads the box one row further on and is dropped.
+template <int BN, int NPAIR>
+__global__ void __launch_bounds__(kThreads, 1)
+    conv_box_wgrad(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                   const __grid_constant__ BoxArgs a, int stages, int x_bytes) {
+  constexpr int NB = (BN + 63) / 64;  // 64-channel blocks of dY per stage
+  constexpr int TMEM_COLS = pow2_cols(NPAIR * BN);
+  constexpr uint32_t IDESC = idesc_bf16(128, BN, 1, 1);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int y_block = a.rows_pad * 128;
+  const int stage_bytes = x_bytes + NB * y_block;
+  const uint32_t s0 = smem_u32(smem);
+  uint8_t* barp = smem + stages * stage_bytes;
+  const uint32_t full = smem_u32(barp);
+  const uint32_t empty = full + 8 * stages;
+  const uint32_t acc_full = empty + 8 * stages;
+  const uint32_t acc_empty = acc_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barp + 8 * (2 * stages + 2));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // dY rows past a tile's To_h * Wb positions stay zero: they are the tail
+  // of the 16-row K steps and multiply box rows of other positions
+  zero_smem(smem, stages * stage_bytes);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full + 8 * s, 1);
+      mbar_init(empty + 8 * s, 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 128);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  fence_proxy_async_smem();
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int items = a.tsets * a.n_tiles * a.cpt * a.groups * a.splits;
+  const int ptiles = a.B * a.tiles_img;
+  const int taps = a.K * a.K;
+  const uint32_t x_box = static_cast<uint32_t>(a.Hb) * a.Wb * 128;
+  const uint32_t y_box = static_cast<uint32_t>(a.To_h) * a.Wb * 128;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmY);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; i < items && ok; i += gridDim.x) {
+        int q = i / a.tsets;
+        const int n_t = q % a.n_tiles;
+        q /= a.n_tiles;
+        const int ch = q % a.cpt;
+        q /= a.cpt;
+        const int g = q % a.groups;
+        const int sp = q / a.groups;
+        const int p0 = sp * a.tiles_per_split;
+        const int p1 = min(ptiles, p0 + a.tiles_per_split);
+        for (int p = p0; p < p1; ++p, ++it) {
+          const int b = p / a.tiles_img;
+          const int oh0 = (p - b * a.tiles_img) * a.To_h;
+          const int s = it % stages;
+          if (!mbar_wait(empty + 8 * s, ((it / stages) & 1) ^ 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = s0 + s * stage_bytes;
+          mbar_arrive_expect_tx(full + 8 * s, x_box + NB * y_box);
+          tma_load_4d(st, &tmX, g * a.cg_off + ch * 64, -a.pad, oh0 - a.pad, b, full + 8 * s);
+#pragma unroll
+          for (int j = 0; j < NB; ++j)
+            tma_load_4d(st + x_bytes + j * y_block, &tmY, g * a.Og + n_t * BN + 64 * j, 0, oh0, b,
+                        full + 8 * s);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      uint32_t it = 0, icount = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; i < items && ok; i += gridDim.x, ++icount) {
+        const int ts = i % a.tsets;
+        const int q0 = ts * a.npairs / a.tsets;
+        const int nq = (ts + 1) * a.npairs / a.tsets - q0;
+        int q = i / a.tsets;
+        q /= a.n_tiles;
+        q /= a.cpt;
+        const int sp = q / a.groups;
+        const int p0 = sp * a.tiles_per_split;
+        const int p1 = min(ptiles, p0 + a.tiles_per_split);
+        if (!mbar_wait(acc_empty, (icount & 1) ^ 1, a.status, abort_flag)) break;
+        tc_fence_after();
+        for (int p = p0; p < p1; ++p, ++it) {
+          const int s = it % stages;
+          if (!mbar_wait(full + 8 * s, (it / stages) & 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = s0 + s * stage_bytes;
+#pragma unroll 1
+          for (int j = 0; j < nq; ++j) {
+            const int ta = 2 * (q0 + j);
+            const int tb = ta + 1;
+            const int sa = (ta / a.K) * a.Wb + ta % a.K;
+            const int sb = tb < taps ? (tb / a.K) * a.Wb + tb % a.K : sa + 1;
+            const uint32_t lbo = static_cast<uint32_t>(sb - sa) * 128;
+            for (int k = 0; k < a.rows_pad / 16; ++k) {
+              const uint64_t ad = smem_desc_sw128(st + sa * 128 + k * 2048, lbo, 1024);
+              const uint64_t bd = smem_desc_sw128(st + x_bytes + k * 2048, y_block, 1024);
+              tc_mma_f16(tmem_base + j * BN, ad, bd, IDESC, (p > p0 || k > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(empty + 8 * s);
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+      }
+    }
+  } else if (warp < 4) {
+    uint32_t icount = 0;
+    for (int i = blockIdx.x; i < items; i += gridDim.x, ++icount) {
+      const int ts = i % a.tsets;
+      const int q0 = ts * a.npairs / a.tsets;
+      const int nq = (ts + 1) * a.npairs / a.tsets - q0;
+      int q = i / a.tsets;
+      const int n_t = q % a.n_tiles;
+      q /= a.n_tiles;
+      const int ch = q % a.cpt;
+      q /= a.cpt;
+      const int g = q % a.groups;
+      const int sp = q / a.groups;
+      if (!mbar_wait(acc_full, icount & 1, a.status, abort_flag)) break;
+      tc_fence_after();
+      const int m = warp * 32 + lane;  // row of D: half m / 64 of the pair, channel m % 64
+      const int c = ch * 64 + (m & 63);
+      float* base = a.part + sp * a.split_stride + g * a.group_stride;
+#pragma unroll 1
+      for (int j = 0; j < NPAIR; ++j) {
+        if (j >= nq) break;
+        const int tap = 2 * (q0 + j) + (m >> 6);
+        const bool valid = tap < taps;
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + j * BN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          float v[16];
+          tmem_ld16(tb + c0, v);
+          if (!valid) continue;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int o = n_t * BN + c0 + e;
+            if (o < a.Og) base[static_cast<long long>(o) * taps * a.P + tap * a.P + c] = v[e];
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty);
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    for (int i = 0; i < 1000; ++i) __nanosleep(1000);
+  }
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- kernel table
+struct Entry {
+  int kind, bn, nsub;
+  void* fn;
+  bool attr;
+};
+template <int BN, int NSUB>
+void* fwd_ptr() {
+  return reinterpret_cast<void*>(&conv_box_fwd<BN, NSUB>);
+}
+template <int BN, int NPAIR>
+void* wgrad_ptr() {
+  return reinterpret_cast<void*>(&conv_box_wgrad<BN, NPAIR>);
+}
+Entry g_entries[] = {
+    {0, 48, 2, fwd_ptr<48, 2>(), false},    {0, 96, 2, fwd_ptr<96, 2>(), false},
+    {0, 128, 2, fwd_ptr<128, 2>(), false},  {0, 192, 2, fwd_ptr<192, 2>(), false},
+    {0, 256, 2, fwd_ptr<256, 2>(), false},  {0, 64, 2, fwd_ptr<64, 2>(), false},
+    {1, 64, 8, wgrad_ptr<64, 8>(), false},  {1, 128, 4, wgrad_ptr<128, 4>(), false},
+    {1, 192, 2, wgrad_ptr<192, 2>(), false}, {1, 256, 2, wgrad_ptr<256, 2>(), false},
+};
+
+Entry* find_entry(int kind, int bn, int nsub) {
+  for (auto& e : g_entries)
+    if (e.kind == kind && e.bn == bn && e.nsub == nsub) return &e;
+  return nullptr;
+}
+
+int fwd_bn(int og) {
+  if (og == 48 || og == 64 || og == 96 || og == 192) return og;
+  if (og % 128 == 0) return 128;
+  if (og % 192 == 0) return 192;
+  if (og <= 256 && og % 16 == 0) return og <= 64 ? 64 : (og <= 128 ? 128 : 256);
+  return 0;
+}
+
+}  // namespace
+
+bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
+                  const float* bias, int relu, const void* mask, void* y, int num_sms,
+                  int* status, bool dry) {
+  memset(d, 0, sizeof(*d));
+  if (cs.Cg % 8 || cs.Og % 8 || cs.C % 8 || cs.Ho() < 1 || cs.Wo() < 1) return false;
+  const int bn = fwd_bn(cs.Og);
+  if (!bn || !find_entry(0, bn, 2)) return false;
+  BoxArgs& a = d->args;
+  a.B = cs.B;
+  a.Ho = cs.Ho();
+  a.Wo = cs.Wo();
+  a.K = cs.K;
+  a.pad = cs.pad;
+  a.Wb = a.Wo + cs.K - 1;
+  if (a.Wb > 256) return false;
+  const int nsub = 2;
+  a.To_h = (nsub * 128) / a.Wb;
+  if (a.To_h < 1) return false;
+  if (a.To_h > a.Ho) a.To_h = a.Ho;
+  // rows the MMAs read: the last sub-tile's 128 rows at the largest shift
+  const int rows = nsub * 128 + (cs.K - 1) * (a.Wb + 1);
+  a.Hb = (rows + a.Wb - 1) / a.Wb;
+  if (a.Hb > 256) return false;
+  a.tiles_img = (a.Ho + a.To_h - 1) / a.To_h;
+  a.cpt = cs.P() / 64;
+  a.cg_off = cs.Cg;
+  a.groups = cs.groups;
+  a.Og = cs.Og;
+  a.n_tiles = (cs.Og + bn - 1) / bn;
+  a.epi = mask ? EPI_BF16_MASK : EPI_BF16;
+  a.relu = relu;
+  a.out = y;
+  a.ld_out = static_cast<long long>(cs.groups) * cs.Og;
+  a.col_goff = cs.Og;
+  a.bias = bias;
+  a.mask = static_cast<const __nv_bfloat16*>(mask);
+  a.ld_mask = a.ld_out;
+  a.status = status;
+  d->kind = 0;
+  d->bn = bn;
+  d->nsub = nsub;
+  d->a_bytes = ((a.Hb * a.Wb * 128) + 1023) / 1024 * 1024;
+  d->b_bytes = bn * 128;
+  d->stages_a = 2;
+  const int left = kSmemBudget - 1024 - kBarBytes - 2 * d->a_bytes;
+  d->stages_b = left / d->b_bytes;
+  if (d->stages_b > 8) d->stages_b = 8;
+  if (d->stages_b < 2) return false;
+  d->smem = 1024 + kBarBytes + 2 * d->a_bytes + d->stages_b * d->b_bytes;
+  const long long tiles = 1LL * a.n_tiles * a.tiles_img * a.B * a.groups;
+  d->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+  if (!dry) {
+    if (!make_tmap_bf16_4d(&d->tmX, x, cs.C, cs.W, cs.H, cs.B, 64, a.Wb, a.Hb)) return false;
+    const int Kd = cs.Kdim();
+    if (!make_tmap_bf16(&d->tmW, w, Kd, static_cast<uint64_t>(cs.groups) * cs.Og,
+                        static_cast<uint64_t>(Kd) * 2, 64, bn))
+      return false;
+  }
+  return true;
+}
+
+bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* dy,
+                    float* part, int splits, int num_sms, int* status, bool dry) {
+  memset(d, 0, sizeof(*d));
+  if (cs.Cg % 8 || cs.Og % 8 || cs.C % 8 || cs.Ho() < 1 || cs.Wo() < 1) return false;
+  BoxArgs& a = d->args;
+  a.B = cs.B;
+  a.Ho = cs.Ho();
+  a.Wo = cs.Wo();
+  a.K = cs.K;
+  a.pad = cs.pad;
+  a.Wb = a.Wo + cs.K - 1;
+  if (a.Wb > 128) return false;
+  // position tiles of at most 128 positions (8 K steps)
+  a.To_h = 128 / a.Wb;
+  if (a.To_h > a.Ho) a.To_h = a.Ho;
+  a.rows_pad = (a.To_h * a.Wb + 15) / 16 * 16;
+  const int taps = cs.K * cs.K;
+  // rows read: the largest second-half shift plus one (the dropped half of an
+  // odd last pair) plus the K rows
+  const int rows = (cs.K - 1) * (a.Wb + 1) + 1 + a.rows_pad;
+  a.Hb = (rows + a.Wb - 1) / a.Wb;
+  if (a.Hb > 256) return false;
+  a.tiles_img = (a.Ho + a.To_h - 1) / a.To_h;
+  a.cpt = cs.P() / 64;
+  a.cg_off = cs.Cg;
+  a.groups = cs.groups;
+  a.Og = cs.Og;
+  a.npairs = (taps + 1) / 2;
+  a.P = cs.P();
+  // output-channel tile (N, a multiple of 64: the dY operand is MN-major in
+  // 64-channel blocks) and pairs per item within the 512 tensor-memory columns
+  int bn;
+  if (cs.Og <= 64)
+    bn = 64;
+  else if (cs.Og == 192)
+    bn = 192;
+  else if (cs.Og <= 128 || cs.Og % 128 == 0)
+    bn = 128;
+  else
+    bn = 256;
+  const int npair = 512 / bn > 8 ? 8 : 512 / bn;
+  if (!find_entry(1, bn, npair)) return false;
+  a.tsets = (a.npairs + npair - 1) / npair;
+  a.n_tiles = (cs.Og + bn - 1) / bn;
+  const int ptiles = a.B * a.tiles_img;
+  const long long base_items = 1LL * a.tsets * a.n_tiles * a.cpt * a.groups;
+  if (splits <= 0) {
+    long long s = (2LL * num_sms + base_items - 1) / base_items;
+    if (s > ptiles / 4) s = ptiles / 4;
+    splits = s < 1 ? 1 : static_cast<int>(s);
+  }
+  if (splits > ptiles) splits = ptiles;
+  a.tiles_per_split = (ptiles + splits - 1) / splits;
+  a.splits = (ptiles + a.tiles_per_split - 1) / a.tiles_per_split;
+  a.group_stride = static_cast<long long>(cs.Og) * taps * a.P;
+  a.split_stride = a.group_stride * cs.groups;
+  a.part = part;
+  a.status = status;
+  d->kind = 1;
+  d->bn = bn;
+  d->nsub = npair;
+  d->a_bytes = ((a.Hb * a.Wb * 128) + 1023) / 1024 * 1024;
+  d->b_bytes = ((bn + 63) / 64) * a.rows_pad * 128;
+  const int stage = d->a_bytes + d->b_bytes;
+  int st = (kSmemBudget - 1024 - kBarBytes) / stage;
+  if (st > 6) st = 6;
+  if (st < 2) return false;
+  d->stages_a = st;
+  d->smem = 1024 + kBarBytes + st * stage;
+  const long long items = base_items * a.splits;
+  d->grid = static_cast<int>(items < num_sms ? items : num_sms);
+  if (!dry) {
+    if (!make_tmap_bf16_4d(&d->tmX, x, cs.C, cs.W, cs.H, cs.B, 64, a.Wb, a.Hb)) return false;
+    if (!make_tmap_bf16_4d(&d->tmW, dy, cs.groups * cs.Og, a.Wo, a.Ho, cs.B, 64, a.Wb, a.To_h))
+      return false;
+  }
+  return true;
+}
+
+cudaError_t box_prepare() {
+  for (auto& e : g_entries) {
+    if (e.attr) continue;
+    cudaError_t r =
+        cudaFuncSetAttribute(e.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
+    if (r != cudaSuccess) return r;
+    e.attr = true;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t box_launch(const BoxDesc& d, cudaStream_t stream) {
+  Entry* e = find_entry(d.kind, d.bn, d.nsub);
+  if (!e) return cudaErrorInvalidValue;
+  if (!e->attr) {
+    cudaError_t r =
+        cudaFuncSetAttribute(e->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
+    if (r != cudaSuccess) return r;
+    e->attr = true;
+  }
+  count_launch();
+  if (d.kind == 0) {
+    void* params[] = {const_cast<CUtensorMap*>(&d.tmX), const_cast<CUtensorMap*>(&d.tmW),
+                      const_cast<BoxArgs*>(&d.args), const_cast<int*>(&d.stages_a),
+                      const_cast<int*>(&d.stages_b), const_cast<int*>(&d.a_bytes)};
+    return cudaLaunchKernel(e->fn, dim3(d.grid), dim3(kThreads), params, d.smem, stream);
+  }
+  void* params[] = {const_cast<CUtensorMap*>(&d.tmX), const_cast<CUtensorMap*>(&d.tmW),
+                    const_cast<BoxArgs*>(&d.args), const_cast<int*>(&d.stages_a),
+                    const_cast<int*>(&d.a_bytes)};
+  return cudaLaunchKernel(e->fn, dim3(d.grid), dim3(kThreads), params, d.smem, stream);
+}
+
+}  // namespace alx

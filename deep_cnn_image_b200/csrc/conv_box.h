@@ -1,0 +1,86 @@
+// conv_box.h -- stride-1 convolutions whose activation operand is one TMA
+// box per 64-channel chunk, reused by every filter tap.
+//
+// An output tile is To_h whole output rows of one image.  Its input box is
+// the (To_h + K - 1)-row, (Wo + K - 1)-pixel window of the zero-padded input
+// (TMA fills the padding), 64 channels, laid out as 128-byte rows: box row
+// r * Wb + c holds input pixel (oh0 - pad + r, c - pad).  Output position
+// m = r * Wb + c of the tile reads, for tap (kh, kw), box row
+// m + kh * Wb + kw: the tap's GEMM operand is the box itself, started
+// kh * Wb + kw rows further on.  tcgen05 matrix descriptors take such a
+// start address directly (the 128-byte swizzle follows the absolute shared
+// memory address), so a chunk is loaded once for all K * K taps instead of
+// once per tap as with im2col.  Positions c >= Wo of each row are computed
+// and dropped.
+//
+//   forward / data gradient: D[m, n] = sum_{tap, c} box[m + shift(tap), c] W[n][tap, c]
+//     M = positions (NSUB sub-tiles of 128), N = output channels, K-major.
+//   weight gradient: D[(tap, c), o] = sum_m box[m + shift(tap), c] dY[m, o]
+//     M = two taps x 64 channels (the two 64-row halves of the operand are the
+//     same box at the two taps' shifts), N = output channels, K = positions;
+//     both operands MN-major.  Partial sums per position split, reduced later.
+#pragma once
+#include "conv_shape.h"
+#include "gemm.h"
+
+namespace alx {
+
+struct BoxArgs {
+  int B, Ho, Wo;   // output map (forward) / dY map (weight gradient)
+  int K, pad;      // kernel size, zero padding of the input
+  int Wb;          // box width: Wo + K - 1
+  int To_h;        // output rows per tile
+  int Hb;          // input rows per box
+  int tiles_img;   // ceil(Ho / To_h)
+  int cpt;         // 64-channel chunks per tap
+  int cg_off;      // input channel offset of group g: g * cg_off
+  int groups;
+  int Og;          // output channels per group
+  int n_tiles;     // BN-wide tiles over Og
+  // forward epilogue (as GemmArgs)
+  int epi, relu;
+  void* out;
+  long long ld_out;
+  int col_goff;
+  const float* bias;
+  const __nv_bfloat16* mask;
+  long long ld_mask;
+  // weight gradient
+  int npairs;           // ceil(K * K / 2) tap pairs
+  int tsets;            // items the pairs are split over
+  int splits;           // position splits
+  int tiles_per_split;  // position tiles per split
+  int rows_pad;         // K rows (positions) per position tile, multiple of 16
+  int P;                // padded channels per tap in the partial sums
+  long long split_stride, group_stride;
+  float* part;
+  int* status;
+};
+
+struct BoxDesc {
+  int kind;  // 0: forward / data gradient, 1: weight gradient
+  int bn;
+  int nsub;  // forward: 128-row sub-tiles per tile; weight gradient: pairs per item
+  CUtensorMap tmX, tmW;  // weight gradient: tmW maps dY
+  BoxArgs args;
+  int grid, smem;
+  int stages_a, stages_b;  // weight gradient: stages_a only
+  int a_bytes, b_bytes;    // per-stage shared memory of each ring
+};
+
+// Forward (or data gradient as a forward convolution of dY): same meaning as
+// conv_desc_fwd.  False if the shape does not fit the kernel.
+bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
+                  const float* bias, int relu, const void* mask, void* y, int num_sms,
+                  int* status, bool dry = false);
+
+// Weight gradient into split partial sums, same layout as conv_desc_wgrad:
+// part[s][g][o][tap * P + c].  splits <= 0: automatic.  Returns the split
+// count used in d->args.splits.
+bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* dy,
+                    float* part, int splits, int num_sms, int* status, bool dry = false);
+
+cudaError_t box_prepare();
+cudaError_t box_launch(const BoxDesc& d, cudaStream_t stream);
+
+}  // namespace alx

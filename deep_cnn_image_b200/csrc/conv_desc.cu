@@ -111,4 +111,29 @@ bool conv_desc_wgrad(GemmDesc* d, const ConvShape& cs, const void* x, const void
   return gemm_finalize(d, num_sms);
 }
 
+size_t ConvPlan::f32_need() const {
+  if (box) return b.kind == 1 ? static_cast<size_t>(b.args.splits) * b.args.split_stride : 0;
+  const GemmArgs& a = g.args;
+  return a.epi == EPI_F32_T ? static_cast<size_t>(a.splits) * a.split_stride : 0;
+}
+
+bool conv_plan_fwd(ConvPlan* p, const ConvShape& cs, const void* x, const void* w,
+                   const float* bias, int relu, const void* mask, void* y, int num_sms,
+                   int* status, bool dry) {
+  p->box = box_desc_fwd(&p->b, cs, x, w, bias, relu, mask, y, num_sms, status, dry);
+  if (p->box) return true;
+  return conv_desc_fwd(&p->g, cs, x, w, bias, relu, mask, y, num_sms, status, dry);
+}
+
+bool conv_plan_wgrad(ConvPlan* p, const ConvShape& cs, const void* x, const void* dy,
+                     float* part, int splits, int num_sms, int* status, bool dry) {
+  p->box = box_desc_wgrad(&p->b, cs, x, dy, part, splits, num_sms, status, dry);
+  if (p->box) return true;
+  return conv_desc_wgrad(&p->g, cs, x, dy, part, splits, num_sms, status, dry);
+}
+
+cudaError_t conv_plan_launch(const ConvPlan& p, cudaStream_t s) {
+  return p.box ? box_launch(p.b, s) : gemm_launch(p.g, s);
+}
+
 }  // namespace alx

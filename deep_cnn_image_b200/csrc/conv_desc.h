@@ -7,22 +7,12 @@
 // channels (k = tap * P + c).  Channels Cg .. P-1 of a tap read either zeros
 // (beyond the tensor) or the next group's channels; their weights are zero.
 #pragma once
+#include "conv_box.h"
+#include "conv_shape.h"
 #include "gemm.h"
 
 namespace alx {
 
-struct ConvShape {
-  int B, H, W;   // input batch and spatial size (stride 1, output = H + 2 pad - K + 1)
-  int C;         // channels per input pixel (all groups)
-  int Cg;        // input channels per group
-  int Og;        // output channels per group
-  int groups;
-  int K, pad;
-  int Ho() const { return H + 2 * pad - K + 1; }
-  int Wo() const { return W + 2 * pad - K + 1; }
-  int P() const { return 64 * ((Cg + 63) / 64); }  // padded channels per tap
-  int Kdim() const { return K * K * P(); }
-};
 
 // Output channel tile for N output channels per group (0 if none fits).
 int conv_pick_bn(int n);
@@ -40,5 +30,23 @@ bool conv_desc_fwd(GemmDesc* d, const ConvShape& cs, const void* x, const void* 
 // of dy[p, g*Og + o] * im2col(x)[p, k], k over K*K*P.  splits <= 0: automatic.
 bool conv_desc_wgrad(GemmDesc* d, const ConvShape& cs, const void* x, const void* dy,
                      float* part, int splits, int num_sms, int* status, bool dry = false);
+
+// One convolution launch: the shifted-box kernel where the shape fits it,
+// else the im2col GEMM.
+struct ConvPlan {
+  bool box = false;
+  GemmDesc g;
+  BoxDesc b;
+  int splits() const { return box ? b.args.splits : g.args.splits; }
+  // fp32 scratch (elements) the launch writes: weight-gradient partials
+  size_t f32_need() const;
+};
+
+bool conv_plan_fwd(ConvPlan* p, const ConvShape& cs, const void* x, const void* w,
+                   const float* bias, int relu, const void* mask, void* y, int num_sms,
+                   int* status, bool dry = false);
+bool conv_plan_wgrad(ConvPlan* p, const ConvShape& cs, const void* x, const void* dy,
+                     float* part, int splits, int num_sms, int* status, bool dry = false);
+cudaError_t conv_plan_launch(const ConvPlan& p, cudaStream_t s);
 
 }  // namespace alx

@@ -8,10 +8,10 @@
 // Operand sources:
 //   A_TMA_K / A_TMA_MN : A read by TMA from a dense bf16 matrix that is
 //                        K-contiguous (rows = M) or M-contiguous (rows = K).
-//   A_GATHER_K         : implicit im2col of an NHWC bf16 map: row m is an
-//                        output pixel, its K entries are the (kh, kw, cin)
-//                        taps of one group (stride-1 convolution).
-//   A_GATHER_MN        : the transpose of that matrix (rows are output
+//   A_IM2COL_K         : implicit im2col of an NHWC bf16 map by TMA im2col
+//                        loads: row m is an output pixel, its K entries the
+//                        (kh, kw, cin) taps of one group (stride-1 conv).
+//   A_IM2COL_MN        : the transpose of that matrix (rows are output
 //                        pixels = the reduction, columns the conv taps), for
 //                        weight gradients.
 //   B_TMA_K / B_TMA_MN : B read by TMA, K-contiguous (rows = N) or
@@ -27,8 +27,6 @@ namespace alx {
 enum ASrc : int {
   A_TMA_K = 0,
   A_TMA_MN = 1,
-  A_GATHER_K = 2,
-  A_GATHER_MN = 3,
   A_IM2COL_K = 4,   // conv operand by TMA im2col: rows = output pixels, 64 channels of one tap
   A_IM2COL_MN = 5,  // its transpose for weight gradients: rows = pixels (the reduction)
 };
@@ -40,16 +38,14 @@ enum Epi : int {
   EPI_F32_T = 3,      // out_f32[split][group][col, row] = acc
 };
 
-struct GatherDesc {
-  const __nv_bfloat16* src;  // NHWC map [B, H, W, C]
+struct GatherDesc {           // im2col geometry of a stride-1 convolution
   int H, W, C;               // C = channels per pixel (row length in elements)
   int cg_off;                // channel offset of group g is g * cg_off
-  int Cg8;                   // channels per group / 8
   int KW, pad;               // kernel width, zero padding (stride 1)
   int Ho, Wo;                // output map size
-  int Kc;                    // number of 8-channel tap chunks = KH * KW * Cg8
+  int Kc;                    // number of (tap, 64-channel chunk) blocks
   int Mpix;                  // B * Ho * Wo
-  int cpt;                   // im2col modes: 64-channel chunks per tap (K = taps * cpt * 64)
+  int cpt;                   // 64-channel chunks per tap (K = taps * cpt * 64)
 };
 
 struct GemmArgs {
@@ -88,6 +84,12 @@ struct GemmDesc {
 // box_outer elements.  Returns false if the driver rejects it.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+
+// 4-D tiled tensor map over an NHWC bf16 tensor [N, H, W, C] (dimensions in
+// (C, W, H, N) order), box box_c x box_w x box_h x 1, 128-byte swizzle
+// (box_c * 2 <= 128).  Out-of-range box elements read as zero.
+bool make_tmap_bf16_4d(CUtensorMap* m, const void* base, int C, int W, int H, int N,
+                       uint32_t box_c, uint32_t box_w, uint32_t box_h);
 
 // im2col tensor map over an NHWC bf16 tensor [N, H, W, C] for a stride-1
 // K x K convolution with zero padding `pad` (both sides): 64 channels per

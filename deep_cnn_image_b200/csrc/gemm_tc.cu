@@ -4,10 +4,10 @@
 // Design (sm_100a):
 //   * persistent: one 320-thread CTA per SM walks a static list of output
 //     tiles (128 x BN), split-K slices and groups;
-//   * warp roles: warps 0-3 epilogue (TMEM -> registers -> global),
-//     warps 4-7 implicit-im2col gather producers (cp.async, 16 B per
-//     thread per row chunk, zero-fill for padding), warp 8 TMA producer,
-//     warp 9 MMA issuer (one thread) and TMEM owner;
+//   * warp roles: warps 0-7 epilogue (TMEM -> registers -> global; warps w
+//     and w + 4 share TMEM lane quarter w and split the 16-column chunks
+//     between them), warp 8 TMA producer, warp 9 MMA issuer (one thread)
+//     and TMEM owner;
 //   * operands staged in a ring of shared-memory stages laid out in the
 //     128-byte-swizzled canonical form that both TMA and tcgen05.mma use;
 //     full/empty mbarriers between producers and the MMA thread;
@@ -123,8 +123,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const __grid_constant__ GemmArgs args, int stages) {
   constexpr int B_TILE_BYTES = BN * BK * 2;
   constexpr int TMEM_COLS = tmem_cols_for(BN);
-  constexpr bool A_GATHER = (ASRC == A_GATHER_K || ASRC == A_GATHER_MN);
-  constexpr int A_MN = (ASRC == A_TMA_MN || ASRC == A_GATHER_MN || ASRC == A_IM2COL_MN) ? 1 : 0;
+  constexpr int A_MN = (ASRC == A_TMA_MN || ASRC == A_IM2COL_MN) ? 1 : 0;
   constexpr int B_MN = (BSRC == B_TMA_MN) ? 1 : 0;
 
   extern __shared__ uint8_t smem_raw[];
@@ -145,12 +144,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
-      mbar_init(bar_full + 8 * s, (A_GATHER ? 128 : 0) + 1);
+      mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar_acc_full + 8 * i, 1);
-      mbar_init(bar_acc_empty + 8 * i, 128);
+      mbar_init(bar_acc_empty + 8 * i, 256);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -170,7 +169,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      if (!A_GATHER) tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
       uint32_t it = 0;
       bool ok = true;
@@ -198,7 +197,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           const uint32_t fb = bar_full + 8 * s;
-          mbar_arrive_expect_tx(fb, B_TILE_BYTES + (A_GATHER ? 0 : A_TILE_BYTES));
+          mbar_arrive_expect_tx(fb, B_TILE_BYTES + A_TILE_BYTES);
           const uint32_t dB = sB + s * B_TILE_BYTES;
           const int n0 = tc.g * args.b_goff + tc.n_t * BN;
           if (BSRC == B_TMA_K) {
@@ -286,128 +285,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_commit(bar_acc_full + 8 * acc);
       }
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ gather producers
-    if (A_GATHER) {
-      const int t = threadIdx.x - 128;
-      const int c = t & 7;
-      const GatherDesc& G = args.g;
-      uint32_t it = 0;
-      bool ok = true;
-      const int HoWo = G.Ho * G.Wo;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const TileCoord tc = decode_tile(args, tile);
-        const int kb0 = tc.sp * args.kb_per_split;
-        const int kb1 = min(args.Kblocks, kb0 + args.kb_per_split);
-        if (ASRC == A_GATHER_K) {
-          // rows rg + 16 j of the tile are output pixels; chunk c of each k-block
-          const int rg = t >> 3;
-          int pbase[8], poh[8], pow_[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int m = tc.m_t * BM + rg + 16 * j;
-            if (m < G.Mpix) {
-              const int b = m / HoWo;
-              const int rem = m - b * HoWo;
-              poh[j] = rem / G.Wo;
-              pow_[j] = rem - poh[j] * G.Wo;
-              pbase[j] = b * G.H;
-            } else {
-              poh[j] = -(1 << 20);
-              pow_[j] = 0;
-              pbase[j] = 0;
-            }
-          }
-          const __nv_bfloat16* gsrc = G.src + tc.g * G.cg_off;
-          for (int kb = kb0; kb < kb1; ++kb, ++it) {
-            const int s = it % stages;
-            const uint32_t ph = (it / stages) & 1;
-            if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, args.status, abort_flag)) {
-              ok = false;
-              break;
-            }
-            const int kc = kb * 8 + c;
-            const bool kvalid = kc < G.Kc;
-            const int tap = kvalid ? kc / G.Cg8 : 0;
-            const int cin8 = kc - tap * G.Cg8;
-            const int kh = tap / G.KW;
-            const int kw = tap - kh * G.KW;
-            const int dh = kh - G.pad, dw = kw - G.pad;
-            const __nv_bfloat16* base = gsrc + cin8 * 8;
-            const uint32_t dst0 = sA + s * A_TILE_BYTES;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int r = rg + 16 * j;
-              const int ih = poh[j] + dh, iw = pow_[j] + dw;
-              const bool okp = kvalid && ih >= 0 && ih < G.H && iw >= 0 && iw < G.W;
-              const __nv_bfloat16* src =
-                  okp ? base + (static_cast<long long>(pbase[j] + ih) * G.W + iw) * G.C : G.src;
-              cp_async_16(dst0 + r * 128 + ((c ^ (r & 7)) << 4), src, okp ? 16u : 0u);
-            }
-            // the stage counts as full once these copies have landed
-            cp_async_arrive(bar_full + 8 * s);
-            mbar_arrive(bar_full + 8 * s);
-          }
-        } else {
-          // A_GATHER_MN: rows are output pixels (the reduction), the two
-          // 64-wide column blocks are conv-tap chunks of this M tile
-          const int q = t >> 3;
-          bool kval[2];
-          int dh[2], dw[2];
-          const __nv_bfloat16* cbase[2];
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int kc = tc.m_t * 16 + j * 8 + c;
-            kval[j] = kc < G.Kc;
-            const int tap = kval[j] ? kc / G.Cg8 : 0;
-            const int cin8 = kc - tap * G.Cg8;
-            const int kh = tap / G.KW;
-            const int kw = tap - kh * G.KW;
-            dh[j] = kh - G.pad;
-            dw[j] = kw - G.pad;
-            cbase[j] = G.src + tc.g * G.cg_off + cin8 * 8;
-          }
-          for (int kb = kb0; kb < kb1; ++kb, ++it) {
-            const int s = it % stages;
-            const uint32_t ph = (it / stages) & 1;
-            if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, args.status, abort_flag)) {
-              ok = false;
-              break;
-            }
-            const uint32_t dst0 = sA + s * A_TILE_BYTES;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int r = q + 16 * i;
-              const int m = kb * BK + r;
-              int b = 0, oh = -(1 << 20), ow = 0;
-              if (m < G.Mpix) {
-                b = m / HoWo;
-                const int rem = m - b * HoWo;
-                oh = rem / G.Wo;
-                ow = rem - oh * G.Wo;
-              }
-#pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                const int ih = oh + dh[j], iw = ow + dw[j];
-                const bool okp = kval[j] && ih >= 0 && ih < G.H && iw >= 0 && iw < G.W;
-                const __nv_bfloat16* src =
-                    okp ? cbase[j] + (static_cast<long long>(b * G.H + ih) * G.W + iw) * G.C : G.src;
-                cp_async_16(dst0 + j * MN_BLOCK_BYTES + r * 128 + ((c ^ (r & 7)) << 4), src,
-                            okp ? 16u : 0u);
-              }
-            }
-            cp_async_arrive(bar_full + 8 * s);
-            mbar_arrive(bar_full + 8 * s);
-          }
-        }
-      }
-      // no copy may still be landing in shared memory when the CTA exits
-      cp_async_wait_all();
-    }
   } else {
     // ------------------------------------------------------------ epilogue
     uint32_t tcount = 0;
-    const int row_in_tile = warp * 32 + lane;
+    const int quarter = warp & 3;
+    const int half = warp >> 2;
+    const int row_in_tile = quarter * 32 + lane;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tcount) {
       const TileCoord tc = decode_tile(args, t);
       const int acc = tcount & 1;
@@ -416,9 +299,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int row = tc.m_t * BM + row_in_tile;
       const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + acc * (TMEM_COLS / 2);
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * (TMEM_COLS / 2);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
+      for (int c0 = 16 * half; c0 < BN; c0 += 32) {
         float v[16];
         tmem_ld16(tbase + c0, v);
         epilogue_store<BN>(args, tc, row, tc.n_t * BN + c0, v);
@@ -454,11 +337,6 @@ struct KernelEntry {
 
 #define ALX_K(BN_, A_, B_) {BN_, A_, B_, kernel_ptr<BN_, A_, B_>(), false}
 KernelEntry g_kernels[] = {
-    ALX_K(48, A_GATHER_K, B_TMA_K),    ALX_K(64, A_GATHER_K, B_TMA_K),
-    ALX_K(96, A_GATHER_K, B_TMA_K),    ALX_K(128, A_GATHER_K, B_TMA_K),
-    ALX_K(192, A_GATHER_K, B_TMA_K),   ALX_K(256, A_GATHER_K, B_TMA_K),
-    ALX_K(64, A_GATHER_MN, B_TMA_MN),  ALX_K(128, A_GATHER_MN, B_TMA_MN),
-    ALX_K(192, A_GATHER_MN, B_TMA_MN), ALX_K(256, A_GATHER_MN, B_TMA_MN),
     ALX_K(64, A_TMA_K, B_TMA_K),       ALX_K(128, A_TMA_K, B_TMA_K),
     ALX_K(256, A_TMA_K, B_TMA_K),      ALX_K(64, A_TMA_K, B_TMA_MN),
     ALX_K(128, A_TMA_K, B_TMA_MN),     ALX_K(256, A_TMA_K, B_TMA_MN),
@@ -480,19 +358,23 @@ KernelEntry* find_kernel(int bn, int asrc, int bsrc) {
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+bool load_encode() {
+  if (g_encode) return true;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return false;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return true;
+}
+
 }  // namespace
 
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
-  if (!g_encode) {
-    cudaDriverEntryPointQueryResult q;
-    void* fn = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !fn)
-      return false;
-    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  }
+  if (!load_encode()) return false;
   if ((reinterpret_cast<uintptr_t>(base) & 15) || (row_bytes & 15) || inner == 0 || outer == 0)
     return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -500,6 +382,25 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16_4d(CUtensorMap* m, const void* base, int C, int W, int H, int N,
+                       uint32_t box_c, uint32_t box_w, uint32_t box_h) {
+  if (!load_encode()) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (C * 2) % 16 || C < 1 || W < 1 || H < 1 ||
+      N < 1 || box_c * 2 > 128 || box_w > 256 || box_h > 256)
+    return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(W),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * 2, static_cast<cuuint64_t>(W) * C * 2,
+                           static_cast<cuuint64_t>(H) * W * C * 2};
+  cuuint32_t box[4] = {box_c, box_w, box_h, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

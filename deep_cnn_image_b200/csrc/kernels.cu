@@ -334,6 +334,261 @@ __global__ void k_pool_bwd(const bf16* __restrict__ dy, const uint8_t* __restric
   }
 }
 
+// ------------------------------------------------------------------ LRN + pool
+// Response normalisation followed by overlapping max-pooling ("ImageNet
+// Classification with Deep Convolutional Neural Networks", 3.4 "Local
+// Response Normalization" and "Overlapping Pooling"; the two follow the first
+// and second convolutions in that order), fused: a block normalises the input
+// rows under kPoolTileRows output rows of one image and one 32-channel slab
+// into shared memory (rounded to bf16, the value a separate normalisation
+// kernel would store), then pools them.  The normalised map reaches global
+// memory only when `lo` is given.  Arithmetic and tie rule are those of
+// k_lrn_fwd and k_pool_fwd.
+constexpr int kPoolTileRows = 4;
+constexpr int kSlab = 32;  // channels per block
+
+template <int Z>
+__global__ void __launch_bounds__(256) k_lrn_pool_fwd(const bf16* __restrict__ a,
+                                                      bf16* __restrict__ lo,
+                                                      bf16* __restrict__ y,
+                                                      uint8_t* __restrict__ am, int H, int W,
+                                                      int C, float k, float alpha, float beta) {
+  extern __shared__ __align__(16) uint4 lds[];  // [rows][W][4 chunks]
+  const int Ho = (H - Z) / 2 + 1, Wo = (W - Z) / 2 + 1;
+  const int oh0 = blockIdx.x * kPoolTileRows;
+  const int oh1 = min(Ho, oh0 + kPoolTileRows);
+  const int b = blockIdx.y;
+  const int cs = blockIdx.z * kSlab;
+  const int r0 = 2 * oh0;
+  // rows this block normalises: those its windows read; the last tile also
+  // takes the rows below the last window so that `lo` is complete
+  const int r1 = oh1 == Ho ? H : 2 * (oh1 - 1) + Z;
+  // rows whose normalised values this block writes to `lo` (each row once)
+  const int own1 = oh1 == Ho ? H : 2 * oh1;
+  const int units1 = (r1 - r0) * W * 4;
+  for (int u = threadIdx.x; u < units1; u += blockDim.x) {
+    const int j = u & 3;
+    const int x = (u >> 2) % W;
+    const int r = (u >> 2) / W;
+    const int c0 = cs + j * 8;
+    const bf16* ap = a + ((static_cast<size_t>(b) * H + r0 + r) * W + x) * C + c0;
+    float v[12];
+    float f[8];
+    unpack8(*reinterpret_cast<const uint4*>(ap), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[2 + i] = f[i];
+    v[0] = v[1] = v[10] = v[11] = 0.f;
+    if (c0 > 0) {
+      const float2 l2 = ld_bf16x2(ap - 2);
+      v[0] = l2.x;
+      v[1] = l2.y;
+    }
+    if (c0 + 8 < C) {
+      const float2 h2 = ld_bf16x2(ap + 8);
+      v[10] = h2.x;
+      v[11] = h2.y;
+    }
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float sum = 0.f;
+#pragma unroll
+      for (int q = 0; q < 5; ++q) sum += v[i + q] * v[i + q];
+      const float sc = k + alpha * sum;
+      o[i] = v[i + 2] * __powf(sc, -beta);
+    }
+    const uint4 packed = pack8(o);
+    lds[(r * W + x) * 4 + j] = packed;
+    if (lo && r0 + r < own1)
+      *reinterpret_cast<uint4*>(lo + ((static_cast<size_t>(b) * H + r0 + r) * W + x) * C + c0) =
+          packed;
+  }
+  __syncthreads();
+  const int units2 = (oh1 - oh0) * Wo * 4;
+  for (int u = threadIdx.x; u < units2; u += blockDim.x) {
+    const int j = u & 3;
+    const int ow = (u >> 2) % Wo;
+    const int oh = oh0 + (u >> 2) / Wo;
+    // two channels per 32-bit word: values compared as bf16 pairs, the
+    // window offset of each half's first maximum kept in the matching half
+    uint32_t best[4], arg[4];
+#pragma unroll
+    for (int dy = 0; dy < Z; ++dy)
+#pragma unroll
+      for (int dx = 0; dx < Z; ++dx) {
+        const uint4 w = lds[((2 * oh + dy - r0) * W + 2 * ow + dx) * 4 + j];
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t off = static_cast<uint32_t>(dy * Z + dx) * 0x00010001u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (dy == 0 && dx == 0) {
+            best[q] = wv[q];
+            arg[q] = 0;
+          } else {
+            const uint32_t gt =
+                __hgt2_mask(*reinterpret_cast<const __nv_bfloat162*>(&wv[q]),
+                            *reinterpret_cast<const __nv_bfloat162*>(&best[q]));
+            best[q] = (best[q] & ~gt) | (wv[q] & gt);
+            arg[q] = (arg[q] & ~gt) | (off & gt);
+          }
+        }
+      }
+    const size_t o = ((static_cast<size_t>(b) * Ho + oh) * Wo + ow) * C + cs + j * 8;
+    *reinterpret_cast<uint4*>(y + o) = make_uint4(best[0], best[1], best[2], best[3]);
+    uint2 packed;  // one byte per channel: halves (lo, hi) of words 0..3
+    packed.x = __byte_perm(arg[0], arg[1], 0x6420);
+    packed.y = __byte_perm(arg[2], arg[3], 0x6420);
+    *reinterpret_cast<uint2*>(am + o) = packed;
+  }
+}
+
+// Gradient arriving at input pixel (ih, iw), channels c .. c+7, through the
+// stride-2 max-pool: the sum, in ascending window order, of the pooled
+// gradients of the windows whose recorded choice is this pixel.  A pixel
+// lies in at most two windows per axis, (i >> 1) - 1 and i >> 1; all four
+// candidates are loaded at once.
+__device__ __forceinline__ void pool_grad8(const bf16* __restrict__ dy,
+                                           const uint8_t* __restrict__ am, int b, int ih, int iw,
+                                           int c, int C, int Ho, int Wo, int z, float (&g)[8]) {
+  uint4 gv[4];
+  uint2 av[4];
+  const int oh_a = (ih >> 1) - 1, ow_a = (iw >> 1) - 1;
+  const uint32_t base = static_cast<uint32_t>((b * Ho + oh_a) * Wo + ow_a) * C + c;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int oh = oh_a + (q >> 1);
+    const int ow = ow_a + (q & 1);
+    const bool ok =
+        oh >= 0 && oh < Ho && ow >= 0 && ow < Wo && ih - 2 * oh < z && iw - 2 * ow < z;
+    gv[q] = make_uint4(0, 0, 0, 0);
+    av[q] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);  // no window offset is 255
+    if (ok) {
+      const uint32_t o = base + static_cast<uint32_t>(((q >> 1) * Wo + (q & 1)) * C);
+      gv[q] = *reinterpret_cast<const uint4*>(dy + o);
+      av[q] = *reinterpret_cast<const uint2*>(am + o);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) g[i] = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int oh = oh_a + (q >> 1);
+    const int ow = ow_a + (q & 1);
+    const uint32_t rep = static_cast<uint32_t>((ih - 2 * oh) * z + (iw - 2 * ow)) * 0x01010101u;
+    const uint32_t m0 = __vcmpeq4(av[q].x, rep), m1 = __vcmpeq4(av[q].y, rep);
+    float f[8];
+    unpack8(gv[q], f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t m = i < 4 ? m0 : m1;
+      if ((m >> (8 * (i & 3))) & 1u) g[i] += f[i];
+    }
+  }
+}
+
+// Backward of normalisation + pooling, fused: the pooled gradient is routed
+// to the chosen pixels and pushed through the normalisation (and the ReLU
+// below it, by the stored conv output a > 0) in one pass; `dl` (the
+// normalised map's gradient) is written only when given.  A block owns
+// `np` whole pixels (all C channels, one 8-channel unit per thread), so the
+// channel window never leaves the block: a and the cross terms
+// t_i = g_i a_i s_i^(-beta-1) go through shared memory.  Arithmetic as
+// k_lrn_bwd.
+__global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ dy,
+                                                      const uint8_t* __restrict__ am,
+                                                      const bf16* __restrict__ a,
+                                                      bf16* __restrict__ dl,
+                                                      bf16* __restrict__ da, int npix,
+                                                      int np, int H, int W, int C, int z,
+                                                      float k, float alpha, float beta) {
+  // a_s[p][4 + c] and t_s[p][4 + c], four zeros at each end of a row; every
+  // access is a 16-byte vector (a unit touches channels c0-4 .. c0+11)
+  extern __shared__ float4 fsm4[];
+  const int ld4 = (C + 8) >> 2;  // row length in float4
+  float4* a_s = fsm4;
+  float4* t_s = fsm4 + np * ld4;
+  const int Ho = (H - z) / 2 + 1, Wo = (W - z) / 2 + 1;
+  const int CH = C >> 3;
+  const int up = threadIdx.x / CH;
+  const int uj = threadIdx.x - up * CH;
+  const int pix = blockIdx.x * np + up;
+  const bool mine = up < np;
+  const bool live = mine && pix < npix;
+  float g[8], av[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) g[i] = av[i] = 0.f;
+  if (live) {
+    const int q = pix / W;
+    const int iw = pix - q * W;
+    const int b = q / H;
+    const int ih = q - b * H;
+    unpack8(*reinterpret_cast<const uint4*>(a + static_cast<size_t>(pix) * C + uj * 8), av);
+    pool_grad8(dy, am, b, ih, iw, uj * 8, C, Ho, Wo, z, g);
+  }
+  if (mine) {
+    float4* ar = a_s + up * ld4 + 1 + uj * 2;
+    ar[0] = make_float4(av[0], av[1], av[2], av[3]);
+    ar[1] = make_float4(av[4], av[5], av[6], av[7]);
+    if (uj == 0) ar[-1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (uj == CH - 1) ar[2] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+  float first[8];
+  if (mine) {
+    const float4* ar = a_s + up * ld4 + uj * 2;  // channels c0-4 .. c0+11
+    float w[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 x = ar[q];
+      w[4 * q] = x.x;
+      w[4 * q + 1] = x.y;
+      w[4 * q + 2] = x.z;
+      w[4 * q + 3] = x.w;
+    }
+    float tv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float sum = 0.f;
+#pragma unroll
+      for (int q = 2; q <= 6; ++q) sum += w[i + q] * w[i + q];
+      const float sc = k + alpha * sum;
+      const float sb = __powf(sc, -beta);
+      first[i] = g[i] * sb;
+      tv[i] = g[i] * av[i] * __fdividef(sb, sc);
+    }
+    float4* tr = t_s + up * ld4 + 1 + uj * 2;
+    tr[0] = make_float4(tv[0], tv[1], tv[2], tv[3]);
+    tr[1] = make_float4(tv[4], tv[5], tv[6], tv[7]);
+    if (uj == 0) tr[-1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (uj == CH - 1) tr[2] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+  if (!live) return;
+  const float4* tr = t_s + up * ld4 + uj * 2;  // channels c0-4 .. c0+11
+  float w[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 x = tr[q];
+    w[4 * q] = x.x;
+    w[4 * q + 1] = x.y;
+    w[4 * q + 2] = x.z;
+    w[4 * q + 3] = x.w;
+  }
+  float o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float cross = 0.f;
+#pragma unroll
+    for (int q = 2; q <= 6; ++q) cross += w[i + q];
+    const float aj = av[i];
+    const float d = first[i] - 2.f * alpha * beta * aj * cross;
+    o[i] = aj > 0.f ? d : 0.f;
+  }
+  const size_t e = static_cast<size_t>(pix) * C + uj * 8;
+  *reinterpret_cast<uint4*>(da + e) = pack8(o);
+  if (dl) *reinterpret_cast<uint4*>(dl + e) = pack8(g);
+}
+
 __global__ void k_pool_fwd_f32(const float* __restrict__ x, float* __restrict__ y, int B, int H,
                                int W, int C, int z, int st) {
   const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
@@ -524,50 +779,70 @@ __global__ void k_loss_mean(const float* __restrict__ rows, int B, float* out1, 
 }
 
 // ------------------------------------------------------------------ bias gradients
-constexpr int kColsumRows = 128;
+constexpr int kColsumRows = 128;  // minimum rows per chunk
+constexpr int kColsumMaxChunks = 512;
+
+// Rows per chunk: at least kColsumRows, a multiple of it, and no more than
+// kColsumMaxChunks chunks (the bias update sums the chunks).
+__host__ __device__ inline long long colsum_rows(long long rows) {
+  long long per = (rows + kColsumMaxChunks - 1) / kColsumMaxChunks;
+  per = (per + kColsumRows - 1) / kColsumRows * kColsumRows;
+  return per < kColsumRows ? kColsumRows : per;
+}
 
 // Column sums of a bf16 [rows, cols] matrix (cols % 8 == 0) over chunks of
-// kColsumRows rows: thread (lane row rl, column group cg) sums 8 columns over
-// rows r0 + rl, r0 + rl + R, ...; the R lane rows are then added in order.
-__global__ void k_colsum_partial(const bf16* __restrict__ m, long long rows, int cols,
-                                 float* __restrict__ partial) {
-  __shared__ float red[4096];
+// colsum_rows(rows) rows.  Block (chunk, column block) covers Gb groups of 8
+// columns; thread (lane row rl, group cg) sums its 8 columns over rows
+// r0 + rl, r0 + rl + R, ... (four loads in flight), then the R lane rows are
+// added in order.  Fixed order throughout: the sums are reproducible.
+__device__ __forceinline__ int colsum_gb(int G) { return G <= 64 ? G : 16; }
+
+__global__ void __launch_bounds__(256) k_colsum_partial(const bf16* __restrict__ m,
+                                                        long long rows, int cols,
+                                                        float* __restrict__ partial) {
+  __shared__ float red[2048];
   const int G = cols >> 3;
-  const long long r0 = 1LL * blockIdx.x * kColsumRows;
-  const long long r1 = min(rows, r0 + kColsumRows);
+  const int Gb = colsum_gb(G);
+  const int R = 256 / Gb;
+  const int g0 = blockIdx.y * Gb;
+  const int gn = min(Gb, G - g0);
+  const long long per = colsum_rows(rows);
+  const long long r0 = 1LL * blockIdx.x * per;
+  const long long r1 = min(rows, r0 + per);
   const int t = threadIdx.x;
-  if (G > static_cast<int>(blockDim.x)) {
-    for (int cg = t; cg < G; cg += blockDim.x) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (long long r = r0; r < r1; ++r) {
+  const int cg = t % Gb, rl = t / Gb;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (rl < R && cg < gn) {
+    const bf16* base = m + (g0 + cg) * 8;
+    long long r = r0 + rl;
+    for (; r + 3LL * R < r1; r += 4LL * R) {
+      uint4 u[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) u[q] = *reinterpret_cast<const uint4*>(base + (r + q * R) * cols);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
         float f[8];
-        unpack8(*reinterpret_cast<const uint4*>(m + r * cols + cg * 8), f);
+        unpack8(u[q], f);
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] += f[i];
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) partial[1LL * blockIdx.x * cols + cg * 8 + i] = acc[i];
     }
-    return;
-  }
-  const int R = blockDim.x / G;
-  const int cg = t % G, rl = t / G;
-  if (rl < R) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (long long r = r0 + rl; r < r1; r += R) {
+    for (; r < r1; r += R) {
       float f[8];
-      unpack8(*reinterpret_cast<const uint4*>(m + r * cols + cg * 8), f);
+      unpack8(*reinterpret_cast<const uint4*>(base + r * cols), f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += f[i];
     }
+  }
+  if (rl < R) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) red[rl * cols + cg * 8 + i] = acc[i];
+    for (int i = 0; i < 8; ++i) red[rl * Gb * 8 + cg * 8 + i] = acc[i];
   }
   __syncthreads();
-  for (int c = t; c < cols; c += blockDim.x) {
+  for (int c = t; c < gn * 8; c += blockDim.x) {
     float v = 0.f;
-    for (int q = 0; q < R; ++q) v += red[q * cols + c];
-    partial[1LL * blockIdx.x * cols + c] = v;
+    for (int q = 0; q < R; ++q) v += red[q * Gb * 8 + c];
+    partial[1LL * blockIdx.x * cols + g0 * 8 + c] = v;
   }
 }
 
@@ -1002,6 +1277,37 @@ void launch_pool_bwd(const bf16* dy, const uint8_t* am, const bf16* pooled, bf16
                                                                      W, C, z, st, relu_mask);
   count_launch();
 }
+bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, int H, int W,
+                         int C, int z, float k, float alpha, float beta, cudaStream_t s) {
+  if (C % kSlab || (z != 2 && z != 3) || H < z || W < z) return false;
+  const int Ho = (H - z) / 2 + 1;
+  // rows a tile normalises: 2T - 2 + z for an inner tile; the last tile also
+  // takes the rows below its last window, at most 2T + 2 in all
+  const int rows = 2 * kPoolTileRows + 2;
+  const size_t smem = static_cast<size_t>(rows) * W * kSlab * 2;
+  if (smem > 48 * 1024) return false;
+  const dim3 grid((Ho + kPoolTileRows - 1) / kPoolTileRows, B, C / kSlab);
+  if (z == 3)
+    k_lrn_pool_fwd<3><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+  else
+    k_lrn_pool_fwd<2><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+  count_launch();
+  return true;
+}
+bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
+                         int B, int H, int W, int C, int z, float k, float alpha, float beta,
+                         cudaStream_t s) {
+  if (C % kSlab || C > 2048 || (z != 2 && z != 3) || H < z || W < z) return false;
+  const int np = 256 / (C / 8);  // whole pixels per block, one 8-channel unit per thread
+  const long long npix = 1LL * B * H * W;
+  if (npix * C >= (1LL << 31)) return false;  // 32-bit element offsets
+  const size_t smem = static_cast<size_t>(np) * 2 * (C + 8) * sizeof(float);
+  if (np < 1 || smem > 48 * 1024) return false;
+  k_pool_lrn_bwd<<<static_cast<unsigned>((npix + np - 1) / np), 256, smem, s>>>(
+      dy, am, a, dl, da, static_cast<int>(npix), np, H, W, C, z, k, alpha, beta);
+  count_launch();
+  return true;
+}
 void launch_pool_fwd_f32(const float* x, float* y, int B, int H, int W, int C, int z, int st,
                          cudaStream_t s) {
   const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
@@ -1036,10 +1342,16 @@ void launch_loss_mean(const float* loss_rows, int B, float* out1, float* out2, c
   k_loss_mean<<<1, 256, 0, s>>>(loss_rows, B, out1, out2);
   count_launch();
 }
-int colsum_chunks(long long rows) { return static_cast<int>((rows + kColsumRows - 1) / kColsumRows); }
+int colsum_chunks(long long rows) {
+  const long long per = colsum_rows(rows);
+  return static_cast<int>((rows + per - 1) / per);
+}
 void launch_colsum_partial(const bf16* m, long long rows, int cols, float* partial,
                            cudaStream_t s) {
-  k_colsum_partial<<<colsum_chunks(rows), 256, 0, s>>>(m, rows, cols, partial);
+  const int G = cols / 8;
+  const int Gb = G <= 64 ? G : 16;
+  k_colsum_partial<<<dim3(colsum_chunks(rows), (G + Gb - 1) / Gb), 256, 0, s>>>(m, rows, cols,
+                                                                             partial);
   count_launch();
 }
 void launch_sgd_conv(float* w, float* v, const float* part, int S, const ConvMap& m, bf16* fwd,

@@ -59,6 +59,16 @@ void launch_pool_fwd(const bf16* x, bf16* y, uint8_t* am, int B, int H, int W, i
 // relu_mask: also zero where the pooled value (= the selected input) is <= 0.
 void launch_pool_bwd(const bf16* dy, const uint8_t* am, const bf16* pooled, bf16* dx, int B,
                      int H, int W, int C, int z, int st, int relu_mask, cudaStream_t s);
+// Fused normalisation (n = 5) + stride-2 max-pool forward; lo (the
+// normalised map) is written only when non-null.  False if C % 32 != 0,
+// z not in {2, 3}, or the row tile does not fit in shared memory.
+bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, int H, int W,
+                         int C, int z, float k, float alpha, float beta, cudaStream_t s);
+// Fused stride-2 max-pool backward + normalisation backward + ReLU mask
+// (a > 0) into da; dl (the normalised map's gradient) written when non-null.
+bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
+                         int B, int H, int W, int C, int z, float k, float alpha, float beta,
+                         cudaStream_t s);
 void launch_pool_fwd_f32(const float* x, float* y, int B, int H, int W, int C, int z, int st,
                          cudaStream_t s);
 

@@ -64,7 +64,8 @@ struct FcL {
 };
 
 struct Plan {
-  GemmDesc cf[5], cd[5], cw[5], ff[3], fd[3], fw[3];
+  ConvPlan cf[5], cd[5], cw[5];
+  GemmDesc ff[3], fd[3], fw[3];
   double conv_flops[5], fc_flops[3];  // algorithmic FLOPs of one pass of each layer
   bool ok = false;
 };
@@ -154,6 +155,9 @@ struct alexnet {
     }
   };
   bool stats_on = false;
+  // also store the normalised maps (lo) and their gradients (dl), which the
+  // fused normalisation + pooling kernels otherwise keep on chip
+  bool keep = false;
   bool capturing = false;
   StepRec direct_rec;
   std::map<int, StepRec> graph_rec;
@@ -363,17 +367,17 @@ bool build_plan(alexnet* h, int B, Plan* P) {
   const int ns = h->num_sms;
   for (int l = 0; l < 5; ++l) {
     const ConvL& L = h->conv[l];
-    if (!conv_desc_fwd(&P->cf[l], L.fwd(B), h->conv_input(l), h->wf[l], h->params + h->b_off[l], 1,
+    if (!conv_plan_fwd(&P->cf[l], L.fwd(B), h->conv_input(l), h->wf[l], h->params + h->b_off[l], 1,
                        nullptr, h->a[l], ns, h->status, g_dry_tmaps))
       return set_err(h, "conv forward plan");
     if (l > 0) {
       const bf16* mask = (!h->conv[l - 1].pool) ? h->a[l - 1] : nullptr;
       bf16* out = mask ? h->da[l - 1] : h->dp[l - 1];
-      if (!conv_desc_fwd(&P->cd[l], L.dgrad(B), h->da[l], h->wd[l], nullptr, 0, mask, out, ns,
+      if (!conv_plan_fwd(&P->cd[l], L.dgrad(B), h->da[l], h->wd[l], nullptr, 0, mask, out, ns,
                          h->status, g_dry_tmaps))
         return set_err(h, "conv data-gradient plan");
     }
-    if (!conv_desc_wgrad(&P->cw[l], L.fwd(B), h->conv_input(l), h->da[l], h->scratch, 0, ns,
+    if (!conv_plan_wgrad(&P->cw[l], L.fwd(B), h->conv_input(l), h->da[l], h->scratch, 0, ns,
                          h->status, g_dry_tmaps))
       return set_err(h, "conv weight-gradient plan");
   }
@@ -393,11 +397,13 @@ bool build_plan(alexnet* h, int B, Plan* P) {
       return set_err(h, "fc weight-gradient plan");
   }
   if (h->scratch) {
-    const GemmDesc* all[] = {&P->cw[0], &P->cw[1], &P->cw[2], &P->cw[3], &P->cw[4],
-                             &P->ff[0], &P->ff[1], &P->ff[2], &P->fd[0], &P->fd[1],
+    const GemmDesc* all[] = {&P->ff[0], &P->ff[1], &P->ff[2], &P->fd[0], &P->fd[1],
                              &P->fd[2], &P->fw[0], &P->fw[1], &P->fw[2]};
     for (const GemmDesc* d : all)
       if (desc_f32_need(*d) > h->scratch_floats) return set_err(h, "scratch too small for plan");
+    for (int l = 0; l < 5; ++l)
+      if (P->cw[l].f32_need() > h->scratch_floats)
+        return set_err(h, "scratch too small for plan");
   }
   P->ok = true;
   return true;
@@ -489,10 +495,10 @@ size_t carve(alexnet* h, void* base) {
     g_dry_tmaps = false;
     size_t need = 1;
     if (ok) {
-      const GemmDesc* all[] = {&P.cw[0], &P.cw[1], &P.cw[2], &P.cw[3], &P.cw[4],
-                               &P.ff[0], &P.ff[1], &P.ff[2], &P.fd[0], &P.fd[1],
+      const GemmDesc* all[] = {&P.ff[0], &P.ff[1], &P.ff[2], &P.fd[0], &P.fd[1],
                                &P.fd[2], &P.fw[0], &P.fw[1], &P.fw[2]};
       for (const GemmDesc* d : all) need = desc_f32_need(*d) > need ? desc_f32_need(*d) : need;
+      for (int l = 0; l < 5; ++l) need = P.cw[l].f32_need() > need ? P.cw[l].f32_need() : need;
     }
     h->scratch_floats = need;
     h->scratch = c.take<float>(need);
@@ -547,8 +553,12 @@ Plan* get_plan(alexnet* h, int B) {
     if (e_ != cudaSuccess) return cuda_status(h, e_, where);                 \
   } while (0)
 
-cudaError_t run_gemm(alexnet* h, const GemmDesc& d, double flops, cudaStream_t s) {
-  if (!h->stats_on || !h->rec) return gemm_launch(d, s);
+cudaError_t launch_any(const GemmDesc& d, cudaStream_t s) { return gemm_launch(d, s); }
+cudaError_t launch_any(const ConvPlan& d, cudaStream_t s) { return conv_plan_launch(d, s); }
+
+template <typename D>
+cudaError_t run_gemm(alexnet* h, const D& d, double flops, cudaStream_t s) {
+  if (!h->stats_on || !h->rec) return launch_any(d, s);
   alexnet::StepRec& R = *h->rec;
   while (R.used + 2 > R.ev.size()) {
     cudaEvent_t e;
@@ -561,7 +571,7 @@ cudaError_t run_gemm(alexnet* h, const GemmDesc& d, double flops, cudaStream_t s
   // inside a capture the records become event nodes of the graph
   const unsigned flags = h->capturing ? cudaEventRecordExternal : cudaEventRecordDefault;
   cudaEventRecordWithFlags(e0, s, flags);
-  cudaError_t r = gemm_launch(d, s);
+  cudaError_t r = launch_any(d, s);
   cudaEventRecordWithFlags(e1, s, flags);
   R.gemm_launches += 1;
   R.gemm_flops += flops;
@@ -575,6 +585,11 @@ alexnet_status forward_bf16(alexnet* h, const bf16* x, int B, int dropout_mode, 
   for (int l = 0; l < 5; ++l) {
     const ConvL& L = h->conv[l];
     ALX_TRY(run_gemm(h, P->cf[l], P->conv_flops[l], s), "conv forward launch");
+    if (L.lrn && L.pool &&
+        launch_lrn_pool_fwd(h->a[l], h->keep ? h->lo[l] : nullptr, h->p[l], h->am[l], B, L.Ho,
+                            L.Ho, L.Cout, h->cfg.pool_size, h->cfg.lrn_k, h->cfg.lrn_alpha,
+                            h->cfg.lrn_beta, s))
+      continue;
     const bf16* cur = h->a[l];
     if (L.lrn) {
       launch_lrn_fwd(h->a[l], h->lo[l], 1LL * B * L.Ho * L.Ho, L.Cout, h->cfg.lrn_n, h->cfg.lrn_k,
@@ -669,6 +684,7 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     launch_pool_bwd(h->dp5, h->am[4], h->p[4], h->da[4], B, L.Ho, L.Ho, L.Cout, cfg.pool_size, 2,
                     1, s);
   }
+  bool fused_bwd[5] = {false, false, false, false, false};
   for (int l = 4; l >= 0; --l) {
     const ConvL& L = h->conv[l];
     if (l > 0) {
@@ -677,8 +693,15 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
       if (Q.pool) {
         // dp[l-1] = d(pooled map) -> through the pool (and LRN) to da[l-1]
         if (Q.lrn) {
-          launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->dl[l - 1], B, Q.Ho, Q.Ho,
-                          Q.Cout, cfg.pool_size, 2, 0, s);
+          // pool + normalisation + ReLU backward in one pass when the shape
+          // allows it, else pool backward now and normalisation below
+          fused_bwd[l - 1] = launch_pool_lrn_bwd(
+              h->dp[l - 1], h->am[l - 1], h->a[l - 1], h->keep ? h->dl[l - 1] : nullptr,
+              h->da[l - 1], B, Q.Ho, Q.Ho, Q.Cout, cfg.pool_size, cfg.lrn_k, cfg.lrn_alpha,
+              cfg.lrn_beta, s);
+          if (!fused_bwd[l - 1])
+            launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->dl[l - 1], B, Q.Ho, Q.Ho,
+                            Q.Cout, cfg.pool_size, 2, 0, s);
         } else {
           launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->da[l - 1], B, Q.Ho, Q.Ho,
                           Q.Cout, cfg.pool_size, 2, 1, s);
@@ -687,7 +710,7 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     }
     ALX_TRY(run_gemm(h, P->cw[l], P->conv_flops[l], s), "conv wgrad launch");
     launch_sgd_conv(h->params + h->w_off[l], h->vel + h->w_off[l], h->scratch,
-                    P->cw[l].args.splits, conv_map(h, l), h->wf[l], h->wd[l], gptr(h->w_off[l]),
+                    P->cw[l].splits(), conv_map(h, l), h->wf[l], h->wd[l], gptr(h->w_off[l]),
                     h->hp, s);
     const long long rows = 1LL * B * L.Ho * L.Ho;
     launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart, s);
@@ -695,7 +718,7 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
                     L.Cout, gptr(h->b_off[l]), h->hp, s);
     if (l > 0) {
       const ConvL& Q = h->conv[l - 1];
-      if (Q.pool && Q.lrn)
+      if (Q.pool && Q.lrn && !fused_bwd[l - 1])
         launch_lrn_bwd(h->a[l - 1], h->dl[l - 1], h->da[l - 1], 1LL * B * Q.Ho * Q.Ho, Q.Cout,
                        cfg.lrn_n, cfg.lrn_k, cfg.lrn_alpha, cfg.lrn_beta, s);
     }
@@ -774,7 +797,9 @@ alexnet_status alexnet_create(const alexnet_config* cfg, void* workspace, size_t
   carve(h, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->last_stream = s;
-  if (cudaError_t pe = gemm_prepare()) {
+  cudaError_t pe = box_prepare();
+  if (pe == cudaSuccess) pe = gemm_prepare();
+  if (pe != cudaSuccess) {
     g_create_error = std::string("create: ") + cudaGetErrorString(pe);
     delete h;
     return ALEXNET_ERR_CUDA;
@@ -868,7 +893,7 @@ alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* la
   alexnet_status st = ALEXNET_OK;
   const int64_t l0 = launch_counter();
   if (h->use_graphs) {
-    const int key = 2 * B + (h->stats_on ? 1 : 0);
+    const int key = 4 * B + (h->keep ? 2 : 0) + (h->stats_on ? 1 : 0);
     auto it = h->train_graphs.find(key);
     if (it == h->train_graphs.end()) {
       if (!h->cap_stream)
@@ -1062,6 +1087,23 @@ alexnet_status alexnet_stats_enable(alexnet_t* h, int enable) {
   h->stats_on = enable != 0;
   h->last_rec = nullptr;
   h->last_launches = 0;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_conv_algo(alexnet_t* h, int batch, int layer, int pass, int* algo) {
+  if (!h || !algo || layer < 0 || layer > 4 || pass < 0 || pass > 2 || (pass == 1 && layer == 0) ||
+      batch < 1 || batch > h->cfg.batch_max || h->cfg.dtype != ALEXNET_BF16)
+    return ALEXNET_ERR_INVALID_ARG;
+  Plan* P = get_plan(h, batch);
+  if (!P) return ALEXNET_ERR_UNSUPPORTED;
+  const ConvPlan& c = pass == 0 ? P->cf[layer] : (pass == 1 ? P->cd[layer] : P->cw[layer]);
+  *algo = c.box ? 1 : 0;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_debug_keep(alexnet_t* h, int keep) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  h->keep = keep != 0;
   return ALEXNET_OK;
 }
 

@@ -91,10 +91,10 @@ alexnet_status alexnet_op_conv_fwd(const void* x, int B, int H, int W, int Cin, 
   cudaMemsetAsync(wg, 0, 2 * static_cast<size_t>(Cout) * cs.Kdim(), s);
   launch_f32_from_bf16(static_cast<const bf16*>(w), wf, n, s);
   launch_conv_shadows(wf, ConvMap{Cout, K, cs.Cg, groups, 0, cs.P()}, wg, nullptr, s);
-  GemmDesc d;
-  if (!conv_desc_fwd(&d, cs, x, wg, bias, relu, nullptr, y, num_sms(), status))
+  ConvPlan d;
+  if (!conv_plan_fwd(&d, cs, x, wg, bias, relu, nullptr, y, num_sms(), status))
     return ALEXNET_ERR_UNSUPPORTED;
-  return done(gemm_launch(d, s));
+  return done(conv_plan_launch(d, s));
 }
 
 alexnet_status alexnet_op_conv1_fwd(const void* x, int B, const void* w, const float* bias,
@@ -112,11 +112,11 @@ alexnet_status alexnet_op_conv1_fwd(const void* x, int B, const void* w, const f
   launch_s2d(static_cast<const bf16*>(x), xs, B, s);
   launch_f32_from_bf16(static_cast<const bf16*>(w), wf, 96 * 363, s);
   launch_conv_shadows(wf, ConvMap{96, 11, 3, 1, 1, 64}, ws2, nullptr, s);
-  GemmDesc d;
-  if (!conv_desc_fwd(&d, ConvShape{B, 57, 57, 64, 48, 96, 1, 3, 0}, xs, ws2, bias, 1, nullptr, y,
+  ConvPlan d;
+  if (!conv_plan_fwd(&d, ConvShape{B, 57, 57, 64, 48, 96, 1, 3, 0}, xs, ws2, bias, 1, nullptr, y,
                      num_sms(), status))
     return ALEXNET_ERR_UNSUPPORTED;
-  return done(gemm_launch(d, s));
+  return done(conv_plan_launch(d, s));
 }
 
 alexnet_status alexnet_op_conv_dgrad(const void* dy, int B, int H, int W, int Cin, const void* w,
@@ -143,11 +143,11 @@ alexnet_status alexnet_op_conv_dgrad(const void* dy, int B, int H, int W, int Ci
   cudaMemsetAsync(status, 0, 4, s);
   launch_f32_from_bf16(static_cast<const bf16*>(w), wf, n, s);
   launch_conv_shadows(wf, m, fwd, dg, s);
-  GemmDesc d;
-  if (!conv_desc_fwd(&d, ConvShape{B, Ho, Wo, Cout, Og, Cg, groups, K, K - 1 - pad}, dy, dg,
+  ConvPlan d;
+  if (!conv_plan_fwd(&d, ConvShape{B, Ho, Wo, Cout, Og, Cg, groups, K, K - 1 - pad}, dy, dg,
                      nullptr, 0, mask, dx, num_sms(), status))
     return ALEXNET_ERR_UNSUPPORTED;
-  return done(gemm_launch(d, s));
+  return done(conv_plan_launch(d, s));
 }
 
 alexnet_status alexnet_op_conv_wgrad(const void* x, int B, int H, int W, int Cin, const void* dy,
@@ -160,17 +160,17 @@ alexnet_status alexnet_op_conv_wgrad(const void* x, int B, int H, int W, int Cin
     return ALEXNET_ERR_INVALID_ARG;
   Scratch sc(ws, ws_bytes);
   int* status = sc.take<int>(1);
-  const int Kb = (B * cs.Ho() * cs.Wo() + 63) / 64;
-  const int smax = splits > 0 ? (splits < Kb ? splits : Kb) : Kb;
-  float* part = sc.take<float>(static_cast<size_t>(smax) * Cout * cs.Kdim());
+  ConvPlan d;
+  if (!conv_plan_wgrad(&d, cs, x, dy, nullptr, splits, num_sms(), status, true))
+    return ALEXNET_ERR_UNSUPPORTED;
+  float* part = sc.take<float>(d.f32_need());
   if (!status || !part) return ALEXNET_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaMemsetAsync(status, 0, 4, s);
-  GemmDesc d;
-  if (!conv_desc_wgrad(&d, cs, x, dy, part, splits, num_sms(), status))
+  if (!conv_plan_wgrad(&d, cs, x, dy, part, splits, num_sms(), status))
     return ALEXNET_ERR_UNSUPPORTED;
-  if (cudaError_t e = gemm_launch(d, s)) return done(e);
-  return reduce_wgrad(ConvMap{Cout, K, cs.Cg, groups, 0, cs.P()}, part, d.args.splits, dw, sc, s);
+  if (cudaError_t e = conv_plan_launch(d, s)) return done(e);
+  return reduce_wgrad(ConvMap{Cout, K, cs.Cg, groups, 0, cs.P()}, part, d.splits(), dw, sc, s);
 }
 
 alexnet_status alexnet_op_conv1_wgrad(const void* x, int B, const void* dy, int splits, float* dw,
@@ -179,19 +179,19 @@ alexnet_status alexnet_op_conv1_wgrad(const void* x, int B, const void* dy, int 
   Scratch sc(ws, ws_bytes);
   int* status = sc.take<int>(1);
   bf16* xs = sc.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 64);
-  const int Kb = (B * 55 * 55 + 63) / 64;
-  const int smax = splits > 0 ? (splits < Kb ? splits : Kb) : Kb;
-  float* part = sc.take<float>(static_cast<size_t>(smax) * 96 * 576);
+  const ConvShape cs{B, 57, 57, 64, 48, 96, 1, 3, 0};
+  ConvPlan d;
+  if (!conv_plan_wgrad(&d, cs, xs, dy, nullptr, splits, num_sms(), status, true))
+    return ALEXNET_ERR_UNSUPPORTED;
+  float* part = sc.take<float>(d.f32_need());
   if (!status || !xs || !part) return ALEXNET_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaMemsetAsync(status, 0, 4, s);
   launch_s2d(static_cast<const bf16*>(x), xs, B, s);
-  GemmDesc d;
-  if (!conv_desc_wgrad(&d, ConvShape{B, 57, 57, 64, 48, 96, 1, 3, 0}, xs, dy, part, splits,
-                       num_sms(), status))
+  if (!conv_plan_wgrad(&d, cs, xs, dy, part, splits, num_sms(), status))
     return ALEXNET_ERR_UNSUPPORTED;
-  if (cudaError_t e = gemm_launch(d, s)) return done(e);
-  return reduce_wgrad(ConvMap{96, 11, 3, 1, 1, 64}, part, d.args.splits, dw, sc, s);
+  if (cudaError_t e = conv_plan_launch(d, s)) return done(e);
+  return reduce_wgrad(ConvMap{96, 11, 3, 1, 1, 64}, part, d.splits(), dw, sc, s);
 }
 
 alexnet_status alexnet_op_fc_fwd(const void* x, int B, int In, const void* w, int Out, int splits,
@@ -342,6 +342,31 @@ alexnet_status alexnet_op_pool_bwd(const void* dy, const uint8_t* argmax, const 
   launch_pool_bwd(static_cast<const bf16*>(dy), argmax, static_cast<const bf16*>(pooled),
                   static_cast<bf16*>(dx), B, H, W, C, z, st, relu_mask,
                   static_cast<cudaStream_t>(stream));
+  return done(cudaGetLastError());
+}
+
+alexnet_status alexnet_op_lrn_pool_fwd(const void* a, int B, int H, int W, int C, int z, float k,
+                                       float alpha, float beta, void* lo, void* y,
+                                       uint8_t* argmax, void* stream) {
+  if (!a || !y || !argmax || B < 1 || C < 32 || C % 32 || (z != 2 && z != 3) || H < z || W < z)
+    return ALEXNET_ERR_INVALID_ARG;
+  if (!launch_lrn_pool_fwd(static_cast<const bf16*>(a), static_cast<bf16*>(lo),
+                           static_cast<bf16*>(y), argmax, B, H, W, C, z, k, alpha, beta,
+                           static_cast<cudaStream_t>(stream)))
+    return ALEXNET_ERR_UNSUPPORTED;
+  return done(cudaGetLastError());
+}
+
+alexnet_status alexnet_op_pool_lrn_bwd(const void* dy, const uint8_t* argmax, const void* a, int B,
+                                       int H, int W, int C, int z, float k, float alpha,
+                                       float beta, void* dl, void* da, void* stream) {
+  if (!dy || !argmax || !a || !da || B < 1 || C < 32 || C % 32 || (z != 2 && z != 3) || H < z ||
+      W < z)
+    return ALEXNET_ERR_INVALID_ARG;
+  if (!launch_pool_lrn_bwd(static_cast<const bf16*>(dy), argmax, static_cast<const bf16*>(a),
+                           static_cast<bf16*>(dl), static_cast<bf16*>(da), B, H, W, C, z, k, alpha,
+                           beta, static_cast<cudaStream_t>(stream)))
+    return ALEXNET_ERR_UNSUPPORTED;
   return done(cudaGetLastError());
 }
 

@@ -83,6 +83,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
       : "memory");
 }
 
+// 4-D tiled load of one box (x innermost); coordinates may be negative or
+// past the end, where the box reads zeros.  x * element size must be a
+// multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int x, int y, int z,
+                                            int w, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+      : "memory");
+}
+
 // im2col load of a 4-D NHWC tensor: pixelsPerColumn consecutive output
 // positions starting at (w, h, n) (top-left input corner of the filter window,
 // may be negative), each fetching the map's channelsPerPixel channels from
@@ -96,30 +108,6 @@ __device__ __forceinline__ void tma_load_im2col_4d(uint32_t dst, const void* tma
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c), "r"(w), "r"(h), "r"(n),
       "h"(off_w), "h"(off_h)
       : "memory");
-}
-
-// ---------------------------------------------------------------- cp.async
-// 16-byte global->shared copy; src_bytes = 0 writes 16 zero bytes.
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-// Arrive on `bar` once every cp.async this thread issued so far has landed
-// (the pending count is raised by one first, so a regular arrive must follow
-// for the thread's arrival to count).
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05

@@ -111,6 +111,31 @@ ALEXNET_API alexnet_status alexnet_op_pool_bwd(const void* dy, const uint8_t* ar
                                    int B, int H, int W, int C, int z, int st, int relu_mask,
                                    void* dx, void* stream);
 
+/* Normalisation (n = 5) then stride-2 max-pooling, fused ([S] 3.4 "Local
+ * Response Normalization" and "Overlapping Pooling"; pooling follows the
+ * normalisation after conv1 and conv2): a bf16 [B,H,W,C] (post-ReLU conv
+ * output), y bf16 [B,Ho,Wo,C] and argmax uint8 [B,Ho,Wo,C] as
+ * alexnet_op_pool_fwd produces them from alexnet_op_lrn_fwd's output
+ * (bit-identical); lo (nullable) receives that normalised map [B,H,W,C].
+ * Ho = (H - z)/2 + 1.  C % 32 == 0, z in {2, 3}, W small enough that
+ * 10 rows x W x 32 bf16 channels fit in 48 KB (W <= 76); else
+ * ALEXNET_ERR_INVALID_ARG / ALEXNET_ERR_UNSUPPORTED. */
+ALEXNET_API alexnet_status alexnet_op_lrn_pool_fwd(const void* a, int B, int H, int W, int C,
+                                                   int z, float k, float alpha, float beta,
+                                                   void* lo, void* y, uint8_t* argmax,
+                                                   void* stream);
+
+/* Backward of alexnet_op_lrn_pool_fwd and of the ReLU below it, fused: dy
+ * bf16 [B,Ho,Wo,C] pooled-map gradient, argmax from the forward, a the
+ * forward's input; da bf16 [B,H,W,C] = ReLU'(a) * LRN-backward(a,
+ * pool-backward(dy, argmax)); dl (nullable) receives the pool-backward
+ * result (the normalised map's gradient).  Same shape rules as the
+ * forward, and C <= 2048. */
+ALEXNET_API alexnet_status alexnet_op_pool_lrn_bwd(const void* dy, const uint8_t* argmax,
+                                                   const void* a, int B, int H, int W, int C,
+                                                   int z, float k, float alpha, float beta,
+                                                   void* dl, void* da, void* stream);
+
 /* Softmax + cross-entropy over N classes: probs fp32 [B,N] (nullable),
  * dlogits bf16 [B,N] = (p - onehot)/B (nullable), loss fp32 scalar (mean).
  * labels device int32 [B] (nullable: no loss, no dlogits). */
@@ -139,7 +164,22 @@ ALEXNET_API alexnet_status alexnet_op_philox(const uint32_t* ctr, const uint32_t
  * l+1), 70+l dL/d(LRN output of conv l+1), 80 dL/dlogits, 81/82 dL/d(FC7/FC6
  * pre-activation); 90/91/94 the uint8 window choices (argmax) of the pools
  * after conv1/conv2/conv5.  Copies min(bytes, tensor bytes) to dst (host or
- * device). */
+ * device).  10/11 and 70/71 hold data only for calls made with
+ * alexnet_debug_keep(h, 1): normalisation and pooling run as one fused
+ * kernel that otherwise keeps the normalised map and its gradient on chip. */
+/* Which kernel runs convolution `layer` (0..4) for a batch of `batch`
+ * images: pass 0 forward, 1 data gradient (layers 1..4), 2 weight gradient.
+ * *algo = 1: the shifted-box kernel (one input box per 64-channel chunk for
+ * all filter taps), 0: the im2col GEMM. */
+ALEXNET_API alexnet_status alexnet_conv_algo(alexnet_t* h, int batch, int layer, int pass,
+                                             int* algo);
+
+/* keep != 0: later forward and training calls also store the normalised
+ * maps after conv1/conv2 and their gradients (debug_copy 10/11, 70/71), at
+ * the cost of the extra writes; results are otherwise identical.  Default 0.
+ * The pages have no counterpart (a debugging aid). */
+ALEXNET_API alexnet_status alexnet_debug_keep(alexnet_t* h, int keep);
+
 ALEXNET_API alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst, size_t bytes,
                                   void* stream);
 

@@ -39,8 +39,13 @@ def _oracle_params(params, net):
     return p
 
 
-def _make(ax, **cfg):
+def _make(ax, keep=True, **cfg):
+    """A handle that also stores the normalised maps and their gradients
+    (which the fused normalisation + pooling kernels otherwise keep on chip),
+    so the tests can read them; test_keep_switch_changes_nothing checks that
+    storing them changes no result."""
     net = ax.AlexNet(**cfg)
+    net.debug_keep(keep)
     return net
 
 
@@ -370,6 +375,44 @@ def test_resume_is_bit_identical(ax):
     pc = torch.zeros(c.params_bytes() // 4, dtype=torch.float32)
     c.get_params(pc)
     np.testing.assert_array_equal(pa.numpy(), pc.numpy())
+
+
+def test_convolutions_use_the_box_kernel(ax):
+    """At the benchmark's batch every convolution pass of the network runs the
+    shifted-box kernel (one input box per channel chunk for all taps)."""
+    net = _make(ax, batch_max=128)
+    for l in range(5):
+        for p in range(3):
+            if p == 1 and l == 0:
+                continue
+            assert net.conv_algo(128, l, p) == 1, (l, p)
+            assert net.conv_algo(2, l, p) == 1, (l, p)
+    net.close()
+
+
+def test_keep_switch_changes_nothing(ax):
+    """Training steps and a forward with the intermediate maps stored and
+    without them give bit-identical parameters, logits and pool choices."""
+    import torch
+    B, N = 4, 2
+    xs = [synthetic.to_bf16(synthetic.images(70 + i, B))[0].cuda() for i in range(N)]
+    ys = [dev(synthetic.labels(80 + i, B)) for i in range(N)]
+    out = []
+    for keep in (False, True):
+        net = _make(ax, keep=keep, batch_max=B, seed=21)
+        for i in range(N):
+            net.train_step(xs[i], ys[i], B, 0.01)
+        p = torch.zeros(net.params_bytes() // 4, dtype=torch.float32)
+        net.get_params(p)
+        logits = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+        net.forward(xs[0], B, ax.INFERENCE, logits)
+        torch.cuda.synchronize()
+        out.append((p.numpy().copy(), logits.cpu().numpy(), _gpu_pool_choices(net, B)))
+        net.close()
+    np.testing.assert_array_equal(out[0][0], out[1][0])
+    np.testing.assert_array_equal(out[0][1], out[1][1])
+    for l in out[0][2]:
+        np.testing.assert_array_equal(out[0][2][l], out[1][2][l])
 
 
 def test_label_out_of_range_sets_status(ax):

@@ -119,6 +119,93 @@ def test_pool_backward(ax, relu_mask):
     assert rel_l2(host(dx), want) < 4e-3
 
 
+# ------------------------------------------------------------------ normalisation + pooling, fused
+FUSED_SHAPES = [((3, 55, 55, 96), 3), ((2, 27, 27, 256), 3), ((2, 13, 13, 64), 3),
+                ((2, 55, 55, 96), 2), ((1, 20, 17, 32), 3), ((1, 18, 18, 32), 3), ((1, 9, 9, 32), 2)]
+
+
+def _lrn_input(seed, shape):
+    r = _rng(seed)
+    a = np.maximum(r.standard_normal(shape) * 20.0, 0.0)
+    # image 0 has one channel vector at every pixel: every window is a tie
+    a[0] = a[0, :1, :1, :]
+    return bf16_round(a)
+
+
+@pytest.mark.parametrize("shape,z", FUSED_SHAPES)
+def test_lrn_pool_forward_fused(ax, shape, z):
+    """Bit-identical to the separate normalisation and pooling kernels; the
+    normalised map within the bf16 bound of the oracle's; the window choices
+    the oracle's first maxima of that map, bit-exact."""
+    import torch
+    B, H, W, C = shape
+    a = _lrn_input(sum(shape) + z, shape)
+    Ho, Wo = (H - z) // 2 + 1, (W - z) // 2 + 1
+    da_ = dev(a, "bf16")
+    lo = torch.empty_like(da_)
+    y = torch.empty((B, Ho, Wo, C), dtype=torch.bfloat16, device="cuda")
+    am = torch.empty((B, Ho, Wo, C), dtype=torch.uint8, device="cuda")
+    ax.op_lrn_pool_fwd(da_, B, H, W, C, z, 2.0, 1e-4, 0.75, lo, y, am)
+    lo_ref = torch.empty_like(da_)
+    ax.op_lrn_fwd(da_, B * H * W, C, 2.0, 1e-4, 0.75, lo_ref)
+    y_ref = torch.empty_like(y)
+    am_ref = torch.empty_like(am)
+    ax.op_pool_fwd(lo_ref, B, H, W, C, z, 2, y_ref, am_ref)
+    torch.cuda.synchronize()
+    assert torch.equal(lo.view(torch.int16), lo_ref.view(torch.int16))
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    assert torch.equal(am, am_ref)
+    glo = host(lo)
+    assert rel_l2(glo, oracle.lrn_fwd(a)) < 4e-3
+    wy, wam = oracle.maxpool_fwd(glo, z, 2)
+    np.testing.assert_array_equal(host(am), wam)
+    np.testing.assert_array_equal(host(y), wy)
+    assert np.all(host(am)[0] == 0)
+    # without the normalised map: same pooled output
+    y2 = torch.empty_like(y)
+    am2 = torch.empty_like(am)
+    ax.op_lrn_pool_fwd(da_, B, H, W, C, z, 2.0, 1e-4, 0.75, None, y2, am2)
+    torch.cuda.synchronize()
+    assert torch.equal(y2.view(torch.int16), y.view(torch.int16)) and torch.equal(am2, am)
+
+
+@pytest.mark.parametrize("shape,z", FUSED_SHAPES)
+def test_pool_lrn_backward_fused(ax, shape, z):
+    """da = ReLU'(a) * LRN-backward(a, pool-backward(dy)) against the oracle
+    on the GPU's own window choices; dl = the pool backward alone."""
+    import torch
+    B, H, W, C = shape
+    a = _lrn_input(sum(shape) + 7 * z, shape)
+    Ho, Wo = (H - z) // 2 + 1, (W - z) // 2 + 1
+    da_ = dev(a, "bf16")
+    y = torch.empty((B, Ho, Wo, C), dtype=torch.bfloat16, device="cuda")
+    am = torch.empty((B, Ho, Wo, C), dtype=torch.uint8, device="cuda")
+    ax.op_lrn_pool_fwd(da_, B, H, W, C, z, 2.0, 1e-4, 0.75, None, y, am)
+    g = bf16_round(_rng(sum(shape)).standard_normal((B, Ho, Wo, C)))
+    dl = torch.empty_like(da_)
+    dout = torch.empty_like(da_)
+    ax.op_pool_lrn_bwd(dev(g, "bf16"), am, da_, B, H, W, C, z, 2.0, 1e-4, 0.75, dl, dout)
+    gam = host(am)
+    want_dl = oracle.maxpool_bwd(g, gam, H, W, z, 2)
+    assert rel_l2(host(dl), want_dl) < 4e-3
+    want = oracle.lrn_bwd(a, want_dl) * (a > 0)
+    assert rel_l2(host(dout), want) < 4e-3
+    d2 = torch.empty_like(da_)
+    ax.op_pool_lrn_bwd(dev(g, "bf16"), am, da_, B, H, W, C, z, 2.0, 1e-4, 0.75, None, d2)
+    torch.cuda.synchronize()
+    assert torch.equal(d2.view(torch.int16), dout.view(torch.int16))
+
+
+def test_fused_pool_rejects_bad_shapes(ax):
+    import torch
+    t = torch.zeros(4 * 9 * 9 * 48, dtype=torch.bfloat16, device="cuda")
+    am = torch.zeros(4 * 4 * 4 * 48, dtype=torch.uint8, device="cuda")
+    with pytest.raises(Exception):
+        ax.op_lrn_pool_fwd(t, 4, 9, 9, 48, 3, 2.0, 1e-4, 0.75, None, t, am)  # C % 32
+    with pytest.raises(Exception):
+        ax.op_pool_lrn_bwd(t, am, t, 1, 9, 9, 32, 4, 2.0, 1e-4, 0.75, None, t)  # z = 4
+
+
 # ------------------------------------------------------------------ softmax + CE
 def test_softmax_cross_entropy(ax, ws):
     import torch
@@ -145,6 +232,9 @@ CONVS = [  # (name, H, Cin, Cout, K, pad, groups, B)
     ("conv4_ungrouped", 13, 384, 384, 3, 1, 1, 2),
     ("conv5", 13, 384, 256, 3, 1, 2, 3),
     ("conv5_ungrouped", 13, 384, 256, 3, 1, 1, 2),
+    ("ragged_5x5", 20, 64, 128, 5, 2, 1, 2),
+    ("one_by_one", 9, 32, 64, 1, 0, 1, 2),
+    ("wide_im2col_fallback", 258, 64, 64, 3, 1, 1, 1),
 ]
 
 
@@ -217,8 +307,10 @@ def test_conv_weight_gradient(ax, ws, name, H, Cin, Cout, K, pad, groups, B):
         results.append(got)
         err = rel_l2(got, want)
         assert err < TOL_F32_ACC, (splits, err)
-    # the fixed-order split-K sum differs from the unsplit one by fp32 rounding only
-    assert rel_l2(results[1], results[0]) < 1e-5
+    # the fixed-order split-K sum differs from the unsplit one by fp32 rounding
+    # only: about 2^-24 * sqrt(terms) relative, terms = B * Ho * Wo (66,564 for
+    # the widest case here)
+    assert rel_l2(results[1], results[0]) < 1e-4
 
 
 def test_conv1_weight_gradient(ax, ws):
