@@ -160,7 +160,8 @@ class AlexNet:
         self.h = h
 
     def close(self):
-        if getattr(self, "h", None):
+        # at interpreter exit the module globals may already be gone
+        if getattr(self, "h", None) and lib is not None:
             lib.alexnet_destroy(self.h)
             self.h = None
 

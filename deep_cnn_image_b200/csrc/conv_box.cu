@@ -6,9 +6,10 @@
 // pass"): a sum over the (kh, kw, cin) taps, here ordered chunk by chunk of
 // 64 input channels, tap by tap within a chunk.
 //
-// Both kernels are persistent (one 192-thread CTA per SM): warps 0-3 drain
-// tensor memory (epilogue), warp 4 issues TMA loads, warp 5 issues tcgen05
-// MMAs and owns the tensor memory.  Every mbarrier wait is bounded; on
+// Both kernels are persistent (one 320-thread CTA per SM): warps 0-7 drain
+// tensor memory (epilogue; warps w and w + 4 share TMEM lane quarter w and
+// split its 16-column chunks), warp 8 issues TMA loads, warp 9 issues
+// tcgen05 MMAs and owns the tensor memory.  Every mbarrier wait is bounded; on
 // expiry the kernel records a timeout in the status word and winds down.
 #include <cudaTypedefs.h>
 
@@ -22,7 +23,7 @@ namespace alx {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kSmemBudget = 227 * 1024;
 constexpr int kBarBytes = 1024;  // mbarriers, tmem slot, abort flag
 
@@ -49,8 +50,8 @@ __device__ __forceinline__ void zero_smem(uint8_t* p, int bytes) {
 template <int BN, int NSUB>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_box_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                 const __grid_constant__ BoxArgs a, int stA, int stB, int a_bytes) {
-  constexpr int B_BYTES = BN * 128;
+                 const __grid_constant__ BoxArgs a, int stA, int stB, int a_bytes, int tps) {
+  constexpr int B_BYTES = BN * 128;  // one tap's weight slab; a B stage holds tps of them
   constexpr int ACC_BUFS = (2 * NSUB * BN <= 512) ? 2 : 1;
   constexpr int TMEM_COLS = pow2_cols(ACC_BUFS * NSUB * BN);
   constexpr uint32_t IDESC = idesc_bf16(128, BN, 0, 0);
@@ -60,7 +61,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + stA * a_bytes;
-  uint8_t* barp = smem + stA * a_bytes + stB * B_BYTES;
+  const int b_stage = tps * B_BYTES;
+  uint8_t* barp = smem + stA * a_bytes + stB * b_stage;
   const uint32_t a_full = smem_u32(barp);
   const uint32_t a_empty = a_full + 8 * stA;
   const uint32_t b_full = a_empty + 8 * stA;
@@ -85,13 +87,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full + 8 * i, 1);
-      mbar_init(acc_empty + 8 * i, 128);
+      mbar_init(acc_empty + 8 * i, 256);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
   fence_proxy_async_smem();
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
@@ -104,12 +106,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int taps = a.K * a.K;
   const uint32_t box_bytes = static_cast<uint32_t>(a.Hb) * a.Wb * 128;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
       tma_prefetch_desc(&tmX);
       tma_prefetch_desc(&tmW);
-      uint32_t ia = 0, ib = 0;
+      RingPos ra, rb;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         int q = t;
@@ -120,32 +122,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = q % a.B;
         const int g = q / a.B;
         const int oh0 = ti * a.To_h;
-        for (int ch = 0; ch < a.cpt && ok; ++ch, ++ia) {
-          const int s = ia % stA;
-          if (!mbar_wait(a_empty + 8 * s, ((ia / stA) & 1) ^ 1, a.status, abort_flag)) {
+        for (int ch = 0; ch < a.cpt && ok; ++ch, ra.next(stA)) {
+          const int s = ra.slot;
+          if (!mbar_wait(a_empty + 8 * s, ra.phase ^ 1, a.status, abort_flag)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(a_full + 8 * s, box_bytes);
           tma_load_4d(sA + s * a_bytes, &tmX, g * a.cg_off + ch * 64, -a.pad, oh0 - a.pad, b,
                       a_full + 8 * s);
-          for (int tap = 0; tap < taps; ++tap, ++ib) {
-            const int sb = ib % stB;
-            if (!mbar_wait(b_empty + 8 * sb, ((ib / stB) & 1) ^ 1, a.status, abort_flag)) {
+          for (int tap0 = 0; tap0 < taps; tap0 += tps, rb.next(stB)) {
+            const int sb = rb.slot;
+            const int n = min(tps, taps - tap0);
+            if (!mbar_wait(b_empty + 8 * sb, rb.phase ^ 1, a.status, abort_flag)) {
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(b_full + 8 * sb, B_BYTES);
-            tma_load_2d(sB + sb * B_BYTES, &tmW, (tap * a.cpt + ch) * 64, g * a.Og + n_t * BN,
-                        b_full + 8 * sb);
+            mbar_arrive_expect_tx(b_full + 8 * sb, n * B_BYTES);
+            for (int j = 0; j < n; ++j)
+              tma_load_2d(sB + sb * b_stage + j * B_BYTES, &tmW, ((tap0 + j) * a.cpt + ch) * 64,
+                          g * a.Og + n_t * BN, b_full + 8 * sb);
           }
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA
+    // Descriptors are built once and advanced by adding 16-byte units to
+    // their start-address field: a single issuing thread cannot afford to
+    // rebuild two 64-bit descriptors per MMA.
     if (lane == 0) {
-      uint32_t ia = 0, ib = 0, tcount = 0;
+      const uint64_t adesc0 = smem_desc_sw128(sA, 16, 1024);
+      const uint64_t bdesc0 = smem_desc_sw128(sB, 16, 1024);
+      const uint32_t a_units = static_cast<uint32_t>(a_bytes) >> 4;
+      RingPos ra, rb;
+      uint32_t tcount = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tcount) {
         const int acc = ACC_BUFS == 2 ? (tcount & 1) : 0;
@@ -153,31 +164,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(acc_empty + 8 * acc, aph ^ 1, a.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t dbase = tmem_base + acc * NSUB * BN;
-        for (int ch = 0; ch < a.cpt && ok; ++ch, ++ia) {
-          const int s = ia % stA;
-          if (!mbar_wait(a_full + 8 * s, (ia / stA) & 1, a.status, abort_flag)) {
+        for (int ch = 0; ch < a.cpt && ok; ++ch, ra.next(stA)) {
+          const int s = ra.slot;
+          if (!mbar_wait(a_full + 8 * s, ra.phase, a.status, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t abox = sA + s * a_bytes;
-          for (int tap = 0; tap < taps; ++tap, ++ib) {
-            const int sb = ib % stB;
-            if (!mbar_wait(b_full + 8 * sb, (ib / stB) & 1, a.status, abort_flag)) {
+          const uint64_t abox = adesc0 + s * a_units;
+          int kh = 0, kw = 0;
+          for (int tap0 = 0; tap0 < taps; tap0 += tps, rb.next(stB)) {
+            const int sb = rb.slot;
+            const int n = min(tps, taps - tap0);
+            if (!mbar_wait(b_full + 8 * sb, rb.phase, a.status, abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const int kh = tap / a.K, kw = tap - (tap / a.K) * a.K;
-            const uint32_t shift = static_cast<uint32_t>(kh * a.Wb + kw) * 128;
-            const uint32_t bt = sB + sb * B_BYTES;
+            uint64_t bd = bdesc0 + sb * (b_stage >> 4);
+            for (int j = 0; j < n; ++j, bd += B_BYTES >> 4) {
+              const uint64_t ad = abox + static_cast<uint32_t>(kh * a.Wb + kw) * 8;  // 128-B rows
+              const uint32_t first = (ch == 0 && tap0 + j == 0) ? 1u : 0u;
 #pragma unroll
-            for (int sub = 0; sub < NSUB; ++sub) {
+              for (int sub = 0; sub < NSUB; ++sub) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const uint64_t ad = smem_desc_sw128(abox + sub * 128 * 128 + shift + k * 32, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(bt + k * 32, 16, 1024);
-                tc_mma_f16(dbase + sub * BN, ad, bd, IDESC, (ch | tap | k) != 0 ? 1u : 0u);
+                for (int k = 0; k < 4; ++k)
+                  tc_mma_f16(dbase + sub * BN, ad + sub * (128 * 128 / 16) + k * 2, bd + k * 2,
+                             IDESC, (k == 0 && first) ? 0u : 1u);
+              }
+              if (++kw == a.K) {
+                kw = 0;
+                ++kh;
               }
             }
             tc_commit(b_empty + 8 * sb);
@@ -189,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(acc_full + 8 * acc);
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ---------------------------------------------------------------- epilogue
     uint32_t tcount = 0;
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
@@ -206,18 +223,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t aph = ACC_BUFS == 2 ? ((tcount >> 1) & 1) : (tcount & 1);
       if (!mbar_wait(acc_full + 8 * acc, aph, a.status, abort_flag)) break;
       tc_fence_after();
+      const int quarter = warp & 3, half = warp >> 2;
 #pragma unroll 1
       for (int sub = 0; sub < NSUB; ++sub) {
-        const int m = sub * 128 + warp * 32 + lane;
+        const int m = sub * 128 + quarter * 32 + lane;
         const int r = m / a.Wb;
         const int col = m - r * a.Wb;
         const int oh = oh0 + r;
         const bool valid = r < a.To_h && oh < a.Ho && col < a.Wo;
         const long long row = (static_cast<long long>(b) * a.Ho + oh) * a.Wo + col;
-        const uint32_t tb = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                             acc * NSUB * BN + sub * BN;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
+        for (int c0 = 16 * half; c0 < BN; c0 += 32) {
           float v[16];
           tmem_ld16(tb + c0, v);
           if (!valid) continue;
@@ -262,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (*abort_flag) {
     for (int i = 0; i < 1000; ++i) __nanosleep(1000);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
@@ -308,12 +326,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(empty + 8 * s, 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 128);
+    mbar_init(acc_empty, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
   fence_proxy_async_smem();
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
@@ -328,11 +346,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t x_box = static_cast<uint32_t>(a.Hb) * a.Wb * 128;
   const uint32_t y_box = static_cast<uint32_t>(a.To_h) * a.Wb * 128;
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
       tma_prefetch_desc(&tmX);
       tma_prefetch_desc(&tmY);
-      uint32_t it = 0;
+      RingPos r;
       bool ok = true;
       for (int i = blockIdx.x; i < items && ok; i += gridDim.x) {
         int q = i / a.tsets;
@@ -344,11 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sp = q / a.groups;
         const int p0 = sp * a.tiles_per_split;
         const int p1 = min(ptiles, p0 + a.tiles_per_split);
-        for (int p = p0; p < p1; ++p, ++it) {
+        for (int p = p0; p < p1; ++p, r.next(stages)) {
           const int b = p / a.tiles_img;
           const int oh0 = (p - b * a.tiles_img) * a.To_h;
-          const int s = it % stages;
-          if (!mbar_wait(empty + 8 * s, ((it / stages) & 1) ^ 1, a.status, abort_flag)) {
+          const int s = r.slot;
+          if (!mbar_wait(empty + 8 * s, r.phase ^ 1, a.status, abort_flag)) {
             ok = false;
             break;
           }
@@ -362,9 +380,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
-      uint32_t it = 0, icount = 0;
+      // stage-relative descriptors plus the stage's start address: the
+      // descriptor's start field is additive (16-byte units)
+      const uint64_t sdesc0 = static_cast<uint64_t>((s0 & 0x3FFFFu) >> 4);
+      const uint64_t ydesc = smem_desc_sw128(static_cast<uint32_t>(x_bytes), y_block, 1024);
+      const int ksteps = a.rows_pad / 16;
+      RingPos r;
+      uint32_t icount = 0;
       bool ok = true;
       for (int i = blockIdx.x; i < items && ok; i += gridDim.x, ++icount) {
         const int ts = i % a.tsets;
@@ -378,25 +402,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int p1 = min(ptiles, p0 + a.tiles_per_split);
         if (!mbar_wait(acc_empty, (icount & 1) ^ 1, a.status, abort_flag)) break;
         tc_fence_after();
-        for (int p = p0; p < p1; ++p, ++it) {
-          const int s = it % stages;
-          if (!mbar_wait(full + 8 * s, (it / stages) & 1, a.status, abort_flag)) {
+        // per pair: start row and leading offset of its A operand (the two
+        // taps' shifts), relative to a stage's first byte
+        uint64_t pair_desc[NPAIR];
+#pragma unroll
+        for (int j = 0; j < NPAIR; ++j) {
+          const int ta = 2 * (q0 + (j < nq ? j : 0));
+          const int tb = ta + 1;
+          const int sa = (ta / a.K) * a.Wb + ta % a.K;
+          const int sb = tb < taps ? (tb / a.K) * a.Wb + tb % a.K : sa + 1;
+          pair_desc[j] = smem_desc_sw128(static_cast<uint32_t>(sa) * 128,
+                                         static_cast<uint32_t>(sb - sa) * 128, 1024);
+        }
+        for (int p = p0; p < p1; ++p, r.next(stages)) {
+          const int s = r.slot;
+          if (!mbar_wait(full + 8 * s, r.phase, a.status, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t st = s0 + s * stage_bytes;
-#pragma unroll 1
-          for (int j = 0; j < nq; ++j) {
-            const int ta = 2 * (q0 + j);
-            const int tb = ta + 1;
-            const int sa = (ta / a.K) * a.Wb + ta % a.K;
-            const int sb = tb < taps ? (tb / a.K) * a.Wb + tb % a.K : sa + 1;
-            const uint32_t lbo = static_cast<uint32_t>(sb - sa) * 128;
-            for (int k = 0; k < a.rows_pad / 16; ++k) {
-              const uint64_t ad = smem_desc_sw128(st + sa * 128 + k * 2048, lbo, 1024);
-              const uint64_t bd = smem_desc_sw128(st + x_bytes + k * 2048, y_block, 1024);
-              tc_mma_f16(tmem_base + j * BN, ad, bd, IDESC, (p > p0 || k > 0) ? 1u : 0u);
+          const uint64_t st = sdesc0 + s * (stage_bytes >> 4);
+#pragma unroll
+          for (int j = 0; j < NPAIR; ++j) {
+            if (j < nq) {
+              const uint64_t ad = st + pair_desc[j];
+              const uint64_t bd = st + ydesc;
+              for (int k = 0; k < ksteps; ++k)
+                tc_mma_f16(tmem_base + j * BN, ad + k * 128, bd + k * 128, IDESC,
+                           (p > p0 || k > 0) ? 1u : 0u);
             }
           }
           tc_commit(empty + 8 * s);
@@ -405,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(acc_full);
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     uint32_t icount = 0;
     for (int i = blockIdx.x; i < items; i += gridDim.x, ++icount) {
       const int ts = i % a.tsets;
@@ -420,7 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int sp = q / a.groups;
       if (!mbar_wait(acc_full, icount & 1, a.status, abort_flag)) break;
       tc_fence_after();
-      const int m = warp * 32 + lane;  // row of D: half m / 64 of the pair, channel m % 64
+      const int quarter = warp & 3, half = warp >> 2;
+      const int m = quarter * 32 + lane;  // row of D: half m / 64 of the pair, channel m % 64
       const int c = ch * 64 + (m & 63);
       float* base = a.part + sp * a.split_stride + g * a.group_stride;
 #pragma unroll 1
@@ -428,9 +462,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= nq) break;
         const int tap = 2 * (q0 + j) + (m >> 6);
         const bool valid = tap < taps;
-        const uint32_t tb = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + j * BN;
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + j * BN;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
+        for (int c0 = 16 * half; c0 < BN; c0 += 32) {
           float v[16];
           tmem_ld16(tb + c0, v);
           if (!valid) continue;
@@ -450,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (*abort_flag) {
     for (int i = 0; i < 1000; ++i) __nanosleep(1000);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
@@ -539,10 +573,13 @@ bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
   d->b_bytes = bn * 128;
   d->stages_a = 2;
   const int left = kSmemBudget - 1024 - kBarBytes - 2 * d->a_bytes;
-  d->stages_b = left / d->b_bytes;
+  // two taps per weight stage (half the barrier round trips of the single
+  // issuing thread) while at least three stages fit
+  d->tps = (left / (2 * d->b_bytes) >= 3 && cs.K * cs.K > 1) ? 2 : 1;
+  d->stages_b = left / (d->tps * d->b_bytes);
   if (d->stages_b > 8) d->stages_b = 8;
   if (d->stages_b < 2) return false;
-  d->smem = 1024 + kBarBytes + 2 * d->a_bytes + d->stages_b * d->b_bytes;
+  d->smem = 1024 + kBarBytes + 2 * d->a_bytes + d->stages_b * d->tps * d->b_bytes;
   const long long tiles = 1LL * a.n_tiles * a.tiles_img * a.B * a.groups;
   d->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   if (!dry) {
@@ -658,7 +695,8 @@ cudaError_t box_launch(const BoxDesc& d, cudaStream_t stream) {
   if (d.kind == 0) {
     void* params[] = {const_cast<CUtensorMap*>(&d.tmX), const_cast<CUtensorMap*>(&d.tmW),
                       const_cast<BoxArgs*>(&d.args), const_cast<int*>(&d.stages_a),
-                      const_cast<int*>(&d.stages_b), const_cast<int*>(&d.a_bytes)};
+                      const_cast<int*>(&d.stages_b), const_cast<int*>(&d.a_bytes),
+                      const_cast<int*>(&d.tps)};
     return cudaLaunchKernel(e->fn, dim3(d.grid), dim3(kThreads), params, d.smem, stream);
   }
   void* params[] = {const_cast<CUtensorMap*>(&d.tmX), const_cast<CUtensorMap*>(&d.tmW),

@@ -65,7 +65,8 @@ struct BoxDesc {
   BoxArgs args;
   int grid, smem;
   int stages_a, stages_b;  // weight gradient: stages_a only
-  int a_bytes, b_bytes;    // per-stage shared memory of each ring
+  int a_bytes, b_bytes;    // per-stage shared memory of each ring (forward: b_bytes per tap)
+  int tps;                 // forward: taps per weight stage
 };
 
 // Forward (or data gradient as a forward convolution of dY): same meaning as

@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
-      uint32_t it = 0;
+      RingPos r;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const TileCoord tc = decode_tile(args, t);
@@ -189,9 +189,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ih0 = rem / G.Wo - G.pad;
           iw0 = rem - (rem / G.Wo) * G.Wo - G.pad;
         }
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % stages;
-          const uint32_t ph = (it / stages) & 1;
+        for (int kb = kb0; kb < kb1; ++kb, r.next(stages)) {
+          const int s = r.slot;
+          const uint32_t ph = r.phase;
           if (!mbar_wait(bar_empty + 8 * s, ph ^ 1, args.status, abort_flag)) {
             ok = false;
             break;
@@ -250,7 +250,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
-      uint32_t it = 0, tcount = 0;
+      const uint64_t adesc0 = A_MN ? smem_desc_sw128(sA, MN_BLOCK_BYTES, 1024)
+                                   : smem_desc_sw128(sA, 16, 1024);
+      const uint64_t bdesc0 = B_MN ? smem_desc_sw128(sB, MN_BLOCK_BYTES, 1024)
+                                   : smem_desc_sw128(sB, 16, 1024);
+      RingPos r;
+      uint32_t tcount = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tcount) {
         const TileCoord tc = decode_tile(args, t);
@@ -261,24 +266,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(bar_acc_empty + 8 * acc, aph ^ 1, args.status, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * (TMEM_COLS / 2);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % stages;
-          const uint32_t ph = (it / stages) & 1;
+        for (int kb = kb0; kb < kb1; ++kb, r.next(stages)) {
+          const int s = r.slot;
+          const uint32_t ph = r.phase;
           if (!mbar_wait(bar_full + 8 * s, ph, args.status, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = sA + s * A_TILE_BYTES;
-          const uint32_t b0 = sB + s * B_TILE_BYTES;
+          // descriptors advance by adding 16-byte units to the start field
+          const uint64_t ad0 = adesc0 + s * (A_TILE_BYTES >> 4);
+          const uint64_t bd0 = bdesc0 + s * (B_TILE_BYTES >> 4);
+          const uint32_t first = kb == kb0 ? 1u : 0u;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = A_MN ? smem_desc_sw128(a0 + k * 2048, MN_BLOCK_BYTES, 1024)
-                                     : smem_desc_sw128(a0 + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, MN_BLOCK_BYTES, 1024)
-                                     : smem_desc_sw128(b0 + k * 32, 16, 1024);
-            tc_mma_f16(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-          }
+          for (int k = 0; k < BK / 16; ++k)
+            tc_mma_f16(d_tmem, ad0 + k * (A_MN ? 128 : 2), bd0 + k * (B_MN ? 128 : 2), idesc,
+                       (k == 0 && first) ? 0u : 1u);
           tc_commit(bar_empty + 8 * s);
         }
         if (!ok) break;
