@@ -47,14 +47,15 @@ __device__ __forceinline__ void zero_smem(uint8_t* p, int bytes) {
 // ---------------------------------------------------------------- forward
 // Tile t = ((g * B + b) * tiles_img + ti) * n_tiles + n_t: output rows
 // ti * To_h .. of image b, output channels n_t * BN .. of group g.
-template <int BN, int NSUB>
+template <int BN, int NSUB, int BMN>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_box_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ BoxArgs a, int stA, int stB, int a_bytes, int tps) {
   constexpr int B_BYTES = BN * 128;  // one tap's weight slab; a B stage holds tps of them
   constexpr int ACC_BUFS = (2 * NSUB * BN <= 512) ? 2 : 1;
   constexpr int TMEM_COLS = pow2_cols(ACC_BUFS * NSUB * BN);
-  constexpr uint32_t IDESC = idesc_bf16(128, BN, 0, 0);
+  constexpr uint32_t IDESC = idesc_bf16(128, BN, 0, BMN);
+  static_assert(!BMN || BN % 64 == 0, "MN-major weights come in 64-channel blocks");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -139,9 +140,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(b_full + 8 * sb, n * B_BYTES);
-            for (int j = 0; j < n; ++j)
-              tma_load_2d(sB + sb * b_stage + j * B_BYTES, &tmW, ((tap0 + j) * a.cpt + ch) * 64,
-                          g * a.Og + n_t * BN, b_full + 8 * sb);
+            for (int j = 0; j < n; ++j) {
+              const uint32_t dst = sB + sb * b_stage + j * B_BYTES;
+              if (BMN) {
+                // forward weight rows g * w_og + ch * 64 .. (64 dy channels),
+                // columns of the flipped tap, output channels n_t * BN ..
+                const int tapf = taps - 1 - (tap0 + j);
+#pragma unroll
+                for (int q = 0; q < BN / 64; ++q)
+                  tma_load_2d(dst + q * 8192, &tmW, tapf * a.w_p + n_t * BN + 64 * q,
+                              g * a.w_og + ch * 64, b_full + 8 * sb);
+              } else {
+                tma_load_2d(dst, &tmW, ((tap0 + j) * a.cpt + ch) * 64, g * a.Og + n_t * BN,
+                            b_full + 8 * sb);
+              }
+            }
           }
         }
       }
@@ -153,8 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rebuild two 64-bit descriptors per MMA.
     if (lane == 0) {
       const uint64_t adesc0 = smem_desc_sw128(sA, 16, 1024);
-      const uint64_t bdesc0 = smem_desc_sw128(sB, 16, 1024);
+      const uint64_t bdesc0 = BMN ? smem_desc_sw128(sB, 8192, 1024) : smem_desc_sw128(sB, 16, 1024);
+      const uint32_t a_lo0 = static_cast<uint32_t>(adesc0), a_hi = static_cast<uint32_t>(adesc0 >> 32);
+      const uint32_t b_lo0 = static_cast<uint32_t>(bdesc0), b_hi = static_cast<uint32_t>(bdesc0 >> 32);
       const uint32_t a_units = static_cast<uint32_t>(a_bytes) >> 4;
+      const uint32_t row_adv = static_cast<uint32_t>(a.Wb - a.K + 1) * 8;  // next kernel row
       RingPos ra, rb;
       uint32_t tcount = 0;
       bool ok = true;
@@ -171,8 +187,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t abox = adesc0 + s * a_units;
-          int kh = 0, kw = 0;
+          const uint32_t abox = a_lo0 + s * a_units;
+          uint32_t shift = 0;  // (kh * Wb + kw) rows, in 16-byte units
+          int kw = 0;
           for (int tap0 = 0; tap0 < taps; tap0 += tps, rb.next(stB)) {
             const int sb = rb.slot;
             const int n = min(tps, taps - tap0);
@@ -181,20 +198,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            uint64_t bd = bdesc0 + sb * (b_stage >> 4);
-            for (int j = 0; j < n; ++j, bd += B_BYTES >> 4) {
-              const uint64_t ad = abox + static_cast<uint32_t>(kh * a.Wb + kw) * 8;  // 128-B rows
-              const uint32_t first = (ch == 0 && tap0 + j == 0) ? 1u : 0u;
+            const uint32_t bst = b_lo0 + sb * (b_stage >> 4);
+            for (int j = 0; j < n; ++j) {
+              const uint32_t acc0 = (ch == 0 && tap0 + j == 0) ? 0u : 1u;
 #pragma unroll
-              for (int sub = 0; sub < NSUB; ++sub) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                  tc_mma_f16(dbase + sub * BN, ad + sub * (128 * 128 / 16) + k * 2, bd + k * 2,
-                             IDESC, (k == 0 && first) ? 0u : 1u);
-              }
+              for (int sub = 0; sub < NSUB; ++sub)
+                tc_mma_k4<2, BMN ? 128 : 2>(dbase + sub * BN, abox + shift + sub * (128 * 128 / 16),
+                                            a_hi, bst + j * (B_BYTES >> 4), b_hi, IDESC, acc0);
               if (++kw == a.K) {
                 kw = 0;
-                ++kh;
+                shift += row_adv;
+              } else {
+                shift += 8;
               }
             }
             tc_commit(b_empty + 8 * sb);
@@ -384,8 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // stage-relative descriptors plus the stage's start address: the
       // descriptor's start field is additive (16-byte units)
-      const uint64_t sdesc0 = static_cast<uint64_t>((s0 & 0x3FFFFu) >> 4);
+      const uint32_t sdesc0 = (s0 & 0x3FFFFu) >> 4;
       const uint64_t ydesc = smem_desc_sw128(static_cast<uint32_t>(x_bytes), y_block, 1024);
+      const uint32_t y_lo = static_cast<uint32_t>(ydesc), y_hi = static_cast<uint32_t>(ydesc >> 32);
       const int ksteps = a.rows_pad / 16;
       RingPos r;
       uint32_t icount = 0;
@@ -404,15 +420,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // per pair: start row and leading offset of its A operand (the two
         // taps' shifts), relative to a stage's first byte
-        uint64_t pair_desc[NPAIR];
+        uint32_t pair_lo[NPAIR];
+        uint32_t pair_hi = 0;
 #pragma unroll
         for (int j = 0; j < NPAIR; ++j) {
           const int ta = 2 * (q0 + (j < nq ? j : 0));
           const int tb = ta + 1;
           const int sa = (ta / a.K) * a.Wb + ta % a.K;
           const int sb = tb < taps ? (tb / a.K) * a.Wb + tb % a.K : sa + 1;
-          pair_desc[j] = smem_desc_sw128(static_cast<uint32_t>(sa) * 128,
-                                         static_cast<uint32_t>(sb - sa) * 128, 1024);
+          const uint64_t pd = smem_desc_sw128(static_cast<uint32_t>(sa) * 128,
+                                              static_cast<uint32_t>(sb - sa) * 128, 1024);
+          pair_lo[j] = static_cast<uint32_t>(pd);
+          pair_hi = static_cast<uint32_t>(pd >> 32);
         }
         for (int p = p0; p < p1; ++p, r.next(stages)) {
           const int s = r.slot;
@@ -421,15 +440,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t st = sdesc0 + s * (stage_bytes >> 4);
+          const uint32_t st = sdesc0 + s * (stage_bytes >> 4);
+          const uint32_t acc0 = p > p0 ? 1u : 0u;
 #pragma unroll
           for (int j = 0; j < NPAIR; ++j) {
             if (j < nq) {
-              const uint64_t ad = st + pair_desc[j];
-              const uint64_t bd = st + ydesc;
-              for (int k = 0; k < ksteps; ++k)
-                tc_mma_f16(tmem_base + j * BN, ad + k * 128, bd + k * 128, IDESC,
-                           (p > p0 || k > 0) ? 1u : 0u);
+              const uint32_t al = st + pair_lo[j];
+              const uint32_t bl = st + y_lo;
+              for (int k = 0; k < ksteps; k += 4)
+                tc_mma_k4<128, 128>(tmem_base + j * BN, al + k * 128, pair_hi, bl + k * 128, y_hi,
+                                    IDESC, k == 0 ? acc0 : 1u);
             }
           }
           tc_commit(empty + 8 * s);
@@ -496,9 +516,9 @@ struct Entry {
   void* fn;
   bool attr;
 };
-template <int BN, int NSUB>
+template <int BN, int NSUB, int BMN = 0>
 void* fwd_ptr() {
-  return reinterpret_cast<void*>(&conv_box_fwd<BN, NSUB>);
+  return reinterpret_cast<void*>(&conv_box_fwd<BN, NSUB, BMN>);
 }
 template <int BN, int NPAIR>
 void* wgrad_ptr() {
@@ -508,6 +528,8 @@ Entry g_entries[] = {
     {0, 48, 2, fwd_ptr<48, 2>(), false},    {0, 96, 2, fwd_ptr<96, 2>(), false},
     {0, 128, 2, fwd_ptr<128, 2>(), false},  {0, 192, 2, fwd_ptr<192, 2>(), false},
     {0, 256, 2, fwd_ptr<256, 2>(), false},  {0, 64, 2, fwd_ptr<64, 2>(), false},
+    {2, 64, 2, fwd_ptr<64, 2, 1>(), false},  {2, 128, 2, fwd_ptr<128, 2, 1>(), false},
+    {2, 192, 2, fwd_ptr<192, 2, 1>(), false}, {2, 256, 2, fwd_ptr<256, 2, 1>(), false},
     {1, 64, 8, wgrad_ptr<64, 8>(), false},  {1, 128, 4, wgrad_ptr<128, 4>(), false},
     {1, 192, 2, wgrad_ptr<192, 2>(), false}, {1, 256, 2, wgrad_ptr<256, 2>(), false},
 };
@@ -528,6 +550,10 @@ int fwd_bn(int og) {
 
 }  // namespace
 
+// Shared geometry of the forward-type launches (kind 0 and 2).
+static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, const float* bias,
+                           int relu, const void* mask, void* y, int num_sms, int* status);
+
 bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
                   const float* bias, int relu, const void* mask, void* y, int num_sms,
                   int* status, bool dry) {
@@ -535,6 +561,41 @@ bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
   if (cs.Cg % 8 || cs.Og % 8 || cs.C % 8 || cs.Ho() < 1 || cs.Wo() < 1) return false;
   const int bn = fwd_bn(cs.Og);
   if (!bn || !find_entry(0, bn, 2)) return false;
+  if (!box_fwd_common(d, cs, 0, bn, bias, relu, mask, y, num_sms, status)) return false;
+  if (!dry) {
+    const BoxArgs& a = d->args;
+    if (!make_tmap_bf16_4d(&d->tmX, x, cs.C, cs.W, cs.H, cs.B, 64, a.Wb, a.Hb)) return false;
+    const int Kd = cs.Kdim();
+    if (!make_tmap_bf16(&d->tmW, w, Kd, static_cast<uint64_t>(cs.groups) * cs.Og,
+                        static_cast<uint64_t>(Kd) * 2, 64, bn))
+      return false;
+  }
+  return true;
+}
+
+bool box_desc_dgrad(BoxDesc* d, const ConvShape& cs, const void* dy, const void* w_fwd,
+                    int p_fwd, const void* mask, void* dx, int num_sms, int* status, bool dry) {
+  memset(d, 0, sizeof(*d));
+  if (cs.Cg % 64 || cs.Og % 8 || cs.C % 8 || cs.Ho() < 1 || cs.Wo() < 1 || p_fwd < cs.Og)
+    return false;
+  const int bn = cs.Og <= 64 ? 64 : (cs.Og == 192 ? 192 : (cs.Og % 128 == 0 ? 128 : 256));
+  if (!find_entry(2, bn, 2)) return false;
+  if (!box_fwd_common(d, cs, 2, bn, nullptr, 0, mask, dx, num_sms, status)) return false;
+  d->args.w_og = cs.Cg;
+  d->args.w_p = p_fwd;
+  if (!dry) {
+    const BoxArgs& a = d->args;
+    if (!make_tmap_bf16_4d(&d->tmX, dy, cs.C, cs.W, cs.H, cs.B, 64, a.Wb, a.Hb)) return false;
+    const int Kd_fwd = cs.K * cs.K * p_fwd;
+    if (!make_tmap_bf16(&d->tmW, w_fwd, Kd_fwd, static_cast<uint64_t>(cs.groups) * cs.Cg,
+                        static_cast<uint64_t>(Kd_fwd) * 2, 64, 64))
+      return false;
+  }
+  return true;
+}
+
+static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, const float* bias,
+                           int relu, const void* mask, void* y, int num_sms, int* status) {
   BoxArgs& a = d->args;
   a.B = cs.B;
   a.Ho = cs.Ho();
@@ -566,7 +627,7 @@ bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
   a.mask = static_cast<const __nv_bfloat16*>(mask);
   a.ld_mask = a.ld_out;
   a.status = status;
-  d->kind = 0;
+  d->kind = kind;
   d->bn = bn;
   d->nsub = nsub;
   d->a_bytes = ((a.Hb * a.Wb * 128) + 1023) / 1024 * 1024;
@@ -582,13 +643,6 @@ bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
   d->smem = 1024 + kBarBytes + 2 * d->a_bytes + d->stages_b * d->tps * d->b_bytes;
   const long long tiles = 1LL * a.n_tiles * a.tiles_img * a.B * a.groups;
   d->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  if (!dry) {
-    if (!make_tmap_bf16_4d(&d->tmX, x, cs.C, cs.W, cs.H, cs.B, 64, a.Wb, a.Hb)) return false;
-    const int Kd = cs.Kdim();
-    if (!make_tmap_bf16(&d->tmW, w, Kd, static_cast<uint64_t>(cs.groups) * cs.Og,
-                        static_cast<uint64_t>(Kd) * 2, 64, bn))
-      return false;
-  }
   return true;
 }
 
@@ -607,7 +661,7 @@ bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* 
   // position tiles of at most 128 positions (8 K steps)
   a.To_h = 128 / a.Wb;
   if (a.To_h > a.Ho) a.To_h = a.Ho;
-  a.rows_pad = (a.To_h * a.Wb + 15) / 16 * 16;
+  a.rows_pad = (a.To_h * a.Wb + 63) / 64 * 64;  // whole groups of four 16-row K steps
   const int taps = cs.K * cs.K;
   // rows read: the largest second-half shift plus one (the dropped half of an
   // odd last pair) plus the K rows
@@ -692,7 +746,7 @@ cudaError_t box_launch(const BoxDesc& d, cudaStream_t stream) {
     e->attr = true;
   }
   count_launch();
-  if (d.kind == 0) {
+  if (d.kind == 0 || d.kind == 2) {
     void* params[] = {const_cast<CUtensorMap*>(&d.tmX), const_cast<CUtensorMap*>(&d.tmW),
                       const_cast<BoxArgs*>(&d.args), const_cast<int*>(&d.stages_a),
                       const_cast<int*>(&d.stages_b), const_cast<int*>(&d.a_bytes),

@@ -45,12 +45,15 @@ struct BoxArgs {
   const float* bias;
   const __nv_bfloat16* mask;
   long long ld_mask;
+  // data gradient from the forward weights (B operand MN-major): the
+  // forward kernel's output channels per group and padded channels per tap
+  int w_og, w_p;
   // weight gradient
   int npairs;           // ceil(K * K / 2) tap pairs
   int tsets;            // items the pairs are split over
   int splits;           // position splits
   int tiles_per_split;  // position tiles per split
-  int rows_pad;         // K rows (positions) per position tile, multiple of 16
+  int rows_pad;         // K rows (positions) per position tile, multiple of 64
   int P;                // padded channels per tap in the partial sums
   long long split_stride, group_stride;
   float* part;
@@ -58,7 +61,7 @@ struct BoxArgs {
 };
 
 struct BoxDesc {
-  int kind;  // 0: forward / data gradient, 1: weight gradient
+  int kind;  // 0: forward / data gradient, 1: weight gradient, 2: data gradient from the forward weights
   int bn;
   int nsub;  // forward: 128-row sub-tiles per tile; weight gradient: pairs per item
   CUtensorMap tmX, tmW;  // weight gradient: tmW maps dY
@@ -74,6 +77,16 @@ struct BoxDesc {
 bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
                   const float* bias, int relu, const void* mask, void* y, int num_sms,
                   int* status, bool dry = false);
+
+// Data gradient of a forward convolution, as the forward convolution of dy
+// (shape dg: the dgrad geometry, channels of dy in, input channels out) with
+// the kernel flipped, reading the forward weight operand w_fwd
+// ([groups * dg.Cg][K * K * p_fwd], p_fwd = padded input channels per tap of
+// the forward convolution) transposed, so no flipped copy is needed.
+// Requires dg.Cg % 64 == 0.  mask as in box_desc_fwd.
+bool box_desc_dgrad(BoxDesc* d, const ConvShape& dg, const void* dy, const void* w_fwd,
+                    int p_fwd, const void* mask, void* dx, int num_sms, int* status,
+                    bool dry = false);
 
 // Weight gradient into split partial sums, same layout as conv_desc_wgrad:
 // part[s][g][o][tap * P + c].  splits <= 0: automatic.  Returns the split

@@ -125,6 +125,15 @@ bool conv_plan_fwd(ConvPlan* p, const ConvShape& cs, const void* x, const void* 
   return conv_desc_fwd(&p->g, cs, x, w, bias, relu, mask, y, num_sms, status, dry);
 }
 
+bool conv_plan_dgrad(ConvPlan* p, const ConvShape& dg, const void* dy, const void* w_fwd,
+                     int p_fwd, const void* w_dg, const void* mask, void* dx, int num_sms,
+                     int* status, bool dry) {
+  p->box = box_desc_dgrad(&p->b, dg, dy, w_fwd, p_fwd, mask, dx, num_sms, status, dry);
+  if (p->box) return true;
+  if (!w_dg && !dry) return false;
+  return conv_desc_fwd(&p->g, dg, dy, w_dg, nullptr, 0, mask, dx, num_sms, status, dry);
+}
+
 bool conv_plan_wgrad(ConvPlan* p, const ConvShape& cs, const void* x, const void* dy,
                      float* part, int splits, int num_sms, int* status, bool dry) {
   p->box = box_desc_wgrad(&p->b, cs, x, dy, part, splits, num_sms, status, dry);

@@ -45,6 +45,12 @@ struct ConvPlan {
 bool conv_plan_fwd(ConvPlan* p, const ConvShape& cs, const void* x, const void* w,
                    const float* bias, int relu, const void* mask, void* y, int num_sms,
                    int* status, bool dry = false);
+// Data gradient: the box kernel reading the forward weights transposed
+// when the shape allows, else the im2col GEMM on the flipped copy w_dg
+// (which may then not be null).
+bool conv_plan_dgrad(ConvPlan* p, const ConvShape& dg, const void* dy, const void* w_fwd,
+                     int p_fwd, const void* w_dg, const void* mask, void* dx, int num_sms,
+                     int* status, bool dry = false);
 bool conv_plan_wgrad(ConvPlan* p, const ConvShape& cs, const void* x, const void* dy,
                      float* part, int splits, int num_sms, int* status, bool dry = false);
 cudaError_t conv_plan_launch(const ConvPlan& p, cudaStream_t s);

@@ -254,6 +254,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                    : smem_desc_sw128(sA, 16, 1024);
       const uint64_t bdesc0 = B_MN ? smem_desc_sw128(sB, MN_BLOCK_BYTES, 1024)
                                    : smem_desc_sw128(sB, 16, 1024);
+      const uint32_t a_lo0 = static_cast<uint32_t>(adesc0), a_hi = static_cast<uint32_t>(adesc0 >> 32);
+      const uint32_t b_lo0 = static_cast<uint32_t>(bdesc0), b_hi = static_cast<uint32_t>(bdesc0 >> 32);
       RingPos r;
       uint32_t tcount = 0;
       bool ok = true;
@@ -275,13 +277,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after();
           // descriptors advance by adding 16-byte units to the start field
-          const uint64_t ad0 = adesc0 + s * (A_TILE_BYTES >> 4);
-          const uint64_t bd0 = bdesc0 + s * (B_TILE_BYTES >> 4);
-          const uint32_t first = kb == kb0 ? 1u : 0u;
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            tc_mma_f16(d_tmem, ad0 + k * (A_MN ? 128 : 2), bd0 + k * (B_MN ? 128 : 2), idesc,
-                       (k == 0 && first) ? 0u : 1u);
+          tc_mma_k4<A_MN ? 128 : 2, B_MN ? 128 : 2>(
+              d_tmem, a_lo0 + s * (A_TILE_BYTES >> 4), a_hi, b_lo0 + s * (B_TILE_BYTES >> 4), b_hi,
+              idesc, kb == kb0 ? 0u : 1u);
           tc_commit(bar_empty + 8 * s);
         }
         if (!ok) break;

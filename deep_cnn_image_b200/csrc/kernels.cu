@@ -898,8 +898,17 @@ __global__ void k_sgd_conv(float* __restrict__ w, float* __restrict__ v,
        p += 1LL * gridDim.x * blockDim.x) {
     const ConvIdx ix = conv_index(m, p);
     const long long base = (1LL * ix.g * Og + ix.co) * Kg + ix.part_inner;
+    // the slices summed in order s = 0, 1, ...; loads issued four at a time
     float g = 0.f;
-    for (int s = 0; s < S; ++s) g += part[s * split_stride + base];
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {
+      float q[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) q[i] = part[(s + i) * split_stride + base];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) g += q[i];
+    }
+    for (; s < S; ++s) g += part[s * split_stride + base];
     float wv = w[p], vv = v[p];
     sgd_one(wv, vv, g, hp);
     w[p] = wv;

@@ -158,6 +158,9 @@ struct alexnet {
   // also store the normalised maps (lo) and their gradients (dl), which the
   // fused normalisation + pooling kernels otherwise keep on chip
   bool keep = false;
+  // the flipped weight copies (wd) are refreshed only while some data-gradient
+  // plan reads them (the box kernel reads the forward copies transposed)
+  bool need_wd = false;
   bool capturing = false;
   StepRec direct_rec;
   std::map<int, StepRec> graph_rec;
@@ -373,9 +376,10 @@ bool build_plan(alexnet* h, int B, Plan* P) {
     if (l > 0) {
       const bf16* mask = (!h->conv[l - 1].pool) ? h->a[l - 1] : nullptr;
       bf16* out = mask ? h->da[l - 1] : h->dp[l - 1];
-      if (!conv_plan_fwd(&P->cd[l], L.dgrad(B), h->da[l], h->wd[l], nullptr, 0, mask, out, ns,
-                         h->status, g_dry_tmaps))
+      if (!conv_plan_dgrad(&P->cd[l], L.dgrad(B), h->da[l], h->wf[l], L.Pch(), h->wd[l], mask,
+                           out, ns, h->status, g_dry_tmaps))
         return set_err(h, "conv data-gradient plan");
+      if (!P->cd[l].box) h->need_wd = true;
     }
     if (!conv_plan_wgrad(&P->cw[l], L.fwd(B), h->conv_input(l), h->da[l], h->scratch, 0, ns,
                          h->status, g_dry_tmaps))
@@ -710,8 +714,8 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     }
     ALX_TRY(run_gemm(h, P->cw[l], P->conv_flops[l], s), "conv wgrad launch");
     launch_sgd_conv(h->params + h->w_off[l], h->vel + h->w_off[l], h->scratch,
-                    P->cw[l].splits(), conv_map(h, l), h->wf[l], h->wd[l], gptr(h->w_off[l]),
-                    h->hp, s);
+                    P->cw[l].splits(), conv_map(h, l), h->wf[l], h->need_wd ? h->wd[l] : nullptr,
+                    gptr(h->w_off[l]), h->hp, s);
     const long long rows = 1LL * B * L.Ho * L.Ho;
     launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart, s);
     launch_sgd_bias(h->params + h->b_off[l], h->vel + h->b_off[l], h->cpart, colsum_chunks(rows),

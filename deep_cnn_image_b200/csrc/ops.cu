@@ -144,8 +144,8 @@ alexnet_status alexnet_op_conv_dgrad(const void* dy, int B, int H, int W, int Ci
   launch_f32_from_bf16(static_cast<const bf16*>(w), wf, n, s);
   launch_conv_shadows(wf, m, fwd, dg, s);
   ConvPlan d;
-  if (!conv_plan_fwd(&d, ConvShape{B, Ho, Wo, Cout, Og, Cg, groups, K, K - 1 - pad}, dy, dg,
-                     nullptr, 0, mask, dx, num_sms(), status))
+  if (!conv_plan_dgrad(&d, ConvShape{B, Ho, Wo, Cout, Og, Cg, groups, K, K - 1 - pad}, dy, fwd,
+                       m.P, dg, mask, dx, num_sms(), status))
     return ALEXNET_ERR_UNSUPPORTED;
   return done(conv_plan_launch(d, s));
 }
