@@ -9,13 +9,22 @@ torch.distributed.run; each rank trains its own replica on its own batch
 (no gradient exchange is built), so the scaling is weak and `value` is the
 images of all ranks divided by the slowest rank's device time.
 
-Timing: W untimed steps; then K steps, each bracketed by CUDA events on the
-library's stream, with a 256 MB buffer written between steps (outside the
-events) so no step starts with the previous step's data in the 126 MB L2;
-barrier + synchronize on both sides; max over ranks.  `e2e` times the same
-steps through the public call with every batch copied from pinned host
-memory and every loss copied back inside the timed span (the copy of batch
-i+1 overlaps step i on a second stream).
+Timing: W untimed steps; then K steps back to back between two CUDA events
+on the library's stream, barrier + synchronize on both sides; max over
+ranks.  A step's working set (about 1.2 GB of activations, gradients and
+weights) is far larger than the 126 MB L2, so no step finds the previous
+step's data there and no flush is needed.  The GEMM roofline comes from a
+separate pass with per-GEMM events (L2 flushed before each step).  `e2e`
+times the same steps through the public call with every batch copied from
+pinned host memory and every loss copied back inside the timed span (the
+copy of batch i+1 overlaps step i on a second stream).
+
+`--mode forward|augment|tencrop|fp32|train_variant` times the other
+workloads instead (not the headline): the batch-128 inference forward, the
+batch-512 training step fed by on-device augmentation of 256x256 uint8
+sources, batch-256 ten-crop inference, the fp32 ungrouped batch-1 forward,
+and the batch-128 training step of one of the pages' ablations
+(`--variant pool2|nolrn|nodropout|ungrouped`).
 
 `--impl reference` times the CPU oracle (the plain fp64 C implementation
 under oracle/) as it stands on the host cores: each step is a training step
@@ -329,6 +338,108 @@ def run_ours(args):
     return 0
 
 
+def run_mode(args):
+    """The non-headline workloads: forward (batch 128, inference),
+    augment (batch 512: augmentation + training step), tencrop (batch 256
+    source images, 10 crops each).  Device-timed, inputs resident."""
+    import numpy as np
+    import torch
+    from deep_cnn_image_b200 import alexnet as ax
+    from deep_cnn_image_b200 import synthetic
+
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    # the pages' ablations (throughput only): non-overlapping 2x2 pooling, no
+    # LRN, no dropout, ungrouped convolutions
+    variant = {"pool2": {"pool_size": 2}, "nolrn": {"lrn_on": 0}, "nodropout": {"dropout_on": 0},
+               "ungrouped": {"grouped": 0}, "none": {}}[args.variant]
+    if args.mode == "fp32":
+        # batch 1, fp32, ungrouped, inference: latency-bound, reads the fp32
+        # weights once per image
+        B = 1
+        net = ax.AlexNet(batch_max=1, seed=1, dtype=ax.FP32, grouped=0)
+        x = torch.from_numpy(synthetic.images(100, 1)).cuda()
+        logits = torch.empty((1, 1000), dtype=torch.float32, device="cuda")
+        probs = torch.empty_like(logits)
+        def step():
+            net.forward(x, 1, ax.INFERENCE, logits, probs)
+        images, metric = 1, "images/sec, AlexNet fp32 ungrouped inference forward, batch 1"
+        flops = 2.0 * 1135256096
+    elif args.mode == "train_variant":
+        B = 128
+        net = ax.AlexNet(batch_max=B, seed=1, **variant)
+        x = synthetic.to_bf16(synthetic.images(100, B))[0].cuda()
+        y = torch.from_numpy(synthetic.labels(200, B)).cuda()
+        loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+        def step():
+            net.train_step(x, y, B, 0.01, loss)
+        images = B
+        metric = "images/sec, AlexNet bf16 train step, batch 128, variant " + args.variant
+        flops = step_flops_per_image()
+    elif args.mode == "forward":
+        B = 128
+        net = ax.AlexNet(batch_max=B, seed=1)
+        x = synthetic.to_bf16(synthetic.images(100, B))[0].cuda()
+        logits = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+        probs = torch.empty_like(logits)
+        def step():
+            net.forward(x, B, ax.INFERENCE, logits, probs)
+        images, metric = B, "images/sec, AlexNet bf16 inference forward (logits + softmax), batch 128"
+        flops = 2.0 * FWD_MACS_PER_IMAGE
+    elif args.mode == "augment":
+        B = 512
+        net = ax.AlexNet(batch_max=B, seed=1)
+        src_np = synthetic.source_images(8, B)
+        src = torch.from_numpy(src_np).cuda()
+        mean = torch.from_numpy(synthetic.mean_image(src_np)).cuda()
+        vec, val = synthetic.pca(9)
+        vec, val = torch.from_numpy(vec).cuda(), torch.from_numpy(val).cuda()
+        x = torch.empty((B, 227, 227, 3), dtype=torch.bfloat16, device="cuda")
+        y = torch.from_numpy(synthetic.labels(200, B)).cuda()
+        loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+        def step():
+            net.augment(src, B, mean, vec, val, x)
+            net.train_step(x, y, B, 0.01, loss)
+        images = B
+        metric = "images/sec, AlexNet bf16 train step with on-device augmentation, batch 512"
+        flops = step_flops_per_image()
+    else:
+        B = 256
+        net = ax.AlexNet(batch_max=10 * B, seed=1)
+        src_np = synthetic.source_images(42, B)
+        src = torch.from_numpy(src_np).cuda()
+        mean = torch.from_numpy(synthetic.mean_image(src_np)).cuda()
+        probs = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+        top5 = torch.empty((B, 5), dtype=torch.int32, device="cuda")
+        def step():
+            net.tencrop(src, B, mean, probs, top5)
+        images = B
+        metric = "source images/sec, AlexNet bf16 ten-crop inference (10 forwards each), batch 256"
+        flops = 10 * 2.0 * FWD_MACS_PER_IMAGE
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert net.get_status() == ax.OK
+    peak = load_peaks()["bf16_tflops_sustained"]
+    value = images * args.steps / (ms / 1e3)
+    line = {"metric": metric, "value": value, "unit": "images/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.mode, "batch": B, "variant": args.variant},
+            "step_roofline": {"achieved": flops * value / 1e12, "peak": peak,
+                              "unit": "TFLOP/s", "frac": flops * value / 1e12 / peak}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -336,13 +447,19 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--batch", type=int, default=128)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-images", type=int, default=2)
+    ap.add_argument("--cpu-images", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["train", "forward", "augment", "tencrop", "fp32",
+                                       "train_variant"], default="train")
+    ap.add_argument("--variant", choices=["none", "pool2", "nolrn", "nodropout", "ungrouped"],
+                    default="none")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.mode != "train":
+        return run_mode(args)
     return run_ours(args)
 
 

@@ -693,9 +693,26 @@ bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* 
   const int ptiles = a.B * a.tiles_img;
   const long long base_items = 1LL * a.tsets * a.n_tiles * a.cpt * a.groups;
   if (splits <= 0) {
-    long long s = (2LL * num_sms + base_items - 1) / base_items;
-    if (s > ptiles / 4) s = ptiles / 4;
-    splits = s < 1 ? 1 : static_cast<int>(s);
+    // the fewest position splits that give every SM an item and fill whole
+    // waves (a mostly empty last wave costs a full item's time); fewer
+    // splits also mean fewer partial sums to write and reduce
+    const long long smax = ptiles / 4 > 0 ? ptiles / 4 : 1;
+    long long best = 1;
+    double best_eff = -1.0;
+    for (long long s = 1; s <= smax && s * base_items <= 4LL * num_sms; ++s) {
+      const long long items = s * base_items;
+      const long long waves = (items + num_sms - 1) / num_sms;
+      const double eff = static_cast<double>(items) / static_cast<double>(waves * num_sms);
+      if (items >= num_sms && eff >= 0.95) {
+        best = s;
+        break;
+      }
+      if (eff > best_eff + 1e-9) {
+        best_eff = eff;
+        best = s;
+      }
+    }
+    splits = static_cast<int>(best);
   }
   if (splits > ptiles) splits = ptiles;
   a.tiles_per_split = (ptiles + splits - 1) / splits;

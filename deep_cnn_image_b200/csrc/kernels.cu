@@ -50,25 +50,61 @@ __device__ __forceinline__ float2 ld_bf16x2(const bf16* p) {
 __global__ void k_write_hparams(HParams* hp, HParams v) { *hp = v; }
 
 // ------------------------------------------------------------------ s2d
-__global__ void k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs, int B) {
-  const uint32_t n = static_cast<uint32_t>(B) * 57 * 57 * 8;
-  for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
-    const int chunk = static_cast<int>(t % 8);
-    const uint32_t pix = t / 8;
-    const int j = static_cast<int>(pix % 57);
-    const int i = static_cast<int>((pix / 57) % 57);
-    const int b = static_cast<int>(pix / (57 * 57));
-    float f[8];
+// One block per (image, output row i): the four input rows 4i .. 4i+3 are
+// one contiguous span of x (4 x 227 x 3 bf16), staged in shared memory with
+// aligned 16-byte loads, then written as 57 pixels x 64 channels in 16-byte
+// vectors: channel (dy * 4 + dx) * 3 + c of pixel j = x[4i + dy][4j + dx][c],
+// channels 48..63, columns past 226 and rows past 226 zero.
+__global__ void __launch_bounds__(256) k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs,
+                                             int B) {
+  constexpr int kRow = 227 * 3;                   // elements per input row
+  constexpr int kSpan16 = (4 * kRow * 2 + 15) / 16 + 1;  // 16-byte chunks covering 4 rows
+  __shared__ uint4 stage[kSpan16];
+  const int i = blockIdx.x % 57;
+  const int b = blockIdx.x / 57;
+  const int rows = min(4, 227 - 4 * i);  // valid input rows of this output row
+  const size_t first = (static_cast<size_t>(b) * 227 + 4 * i) * kRow;  // element index
+  const size_t total_bytes = static_cast<size_t>(B) * 227 * kRow * 2;
+  const uintptr_t base = reinterpret_cast<uintptr_t>(x);
+  const uintptr_t lo = (base + first * 2) & ~static_cast<uintptr_t>(15);
+  const uintptr_t hi = base + (first + static_cast<size_t>(rows) * kRow) * 2;  // exclusive
+  const int n16 = static_cast<int>((hi - lo + 15) / 16);
+  for (int q = threadIdx.x; q < n16; q += blockDim.x) {
+    const uintptr_t addr = lo + 16 * static_cast<uintptr_t>(q);
+    if (addr + 16 <= base + total_bytes) {
+      stage[q] = *reinterpret_cast<const uint4*>(addr);
+    } else {  // the tensor's last, partial chunk: element by element
+      uint16_t t[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        t[e] = addr + 2 * e + 2 <= base + total_bytes
+                   ? *reinterpret_cast<const uint16_t*>(addr + 2 * e)
+                   : 0;
+      stage[q] = make_uint4(t[0] | (static_cast<uint32_t>(t[1]) << 16),
+                            t[2] | (static_cast<uint32_t>(t[3]) << 16),
+                            t[4] | (static_cast<uint32_t>(t[5]) << 16),
+                            t[6] | (static_cast<uint32_t>(t[7]) << 16));
+    }
+  }
+  __syncthreads();
+  const uint16_t* su = reinterpret_cast<const uint16_t*>(stage);
+  const int off = static_cast<int>((base + first * 2 - lo) / 2);  // element offset of row 4i
+  for (int u = threadIdx.x; u < 57 * 8; u += blockDim.x) {
+    const int j = u >> 3, chunk = u & 7;
+    uint16_t v[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int ch = chunk * 8 + q;
-      const int dy = ch / 12, dx = (ch / 3) % 4, c = ch % 3;
-      const int y = 4 * i + dy, xx = 4 * j + dx;
-      f[q] = (ch < 48 && y < 227 && xx < 227)
-                 ? __bfloat162float(x[((static_cast<long long>(b) * 227 + y) * 227 + xx) * 3 + c])
-                 : 0.f;
+      const int dy = ch / 12, r = ch - dy * 12;  // r = dx * 3 + c
+      v[q] = (ch < 48 && dy < rows && 4 * j + r / 3 < 227) ? su[off + dy * kRow + 12 * j + r] : 0;
     }
-    *reinterpret_cast<uint4*>(xs + static_cast<size_t>(pix) * 64 + chunk * 8) = pack8(f);
+    uint4 o;
+    o.x = v[0] | (static_cast<uint32_t>(v[1]) << 16);
+    o.y = v[2] | (static_cast<uint32_t>(v[3]) << 16);
+    o.z = v[4] | (static_cast<uint32_t>(v[5]) << 16);
+    o.w = v[6] | (static_cast<uint32_t>(v[7]) << 16);
+    *reinterpret_cast<uint4*>(xs + ((static_cast<size_t>(b) * 57 + i) * 57 + j) * 64 + chunk * 8) =
+        o;
   }
 }
 
@@ -500,7 +536,8 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
                                                       bf16* __restrict__ dl,
                                                       bf16* __restrict__ da, int npix,
                                                       int np, int H, int W, int C, int z,
-                                                      float k, float alpha, float beta) {
+                                                      float k, float alpha, float beta,
+                                                      float* __restrict__ bias_part) {
   // a_s[p][4 + c] and t_s[p][4 + c], four zeros at each end of a row; every
   // access is a 16-byte vector (a unit touches channels c0-4 .. c0+11)
   extern __shared__ float4 fsm4[];
@@ -511,82 +548,107 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
   const int CH = C >> 3;
   const int up = threadIdx.x / CH;
   const int uj = threadIdx.x - up * CH;
-  const int pix = blockIdx.x * np + up;
   const bool mine = up < np;
-  const bool live = mine && pix < npix;
-  float g[8], av[8];
+  // this thread's share of the bias gradient (sum of the stored da values of
+  // its channels over the pixels it handles)
+  float bsum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int blk = blockIdx.x; blk * np < npix; blk += gridDim.x) {
+    const int pix = blk * np + up;
+    const bool live = mine && pix < npix;
+    float g[8], av[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) g[i] = av[i] = 0.f;
-  if (live) {
-    const int q = pix / W;
-    const int iw = pix - q * W;
-    const int b = q / H;
-    const int ih = q - b * H;
-    unpack8(*reinterpret_cast<const uint4*>(a + static_cast<size_t>(pix) * C + uj * 8), av);
-    pool_grad8(dy, am, b, ih, iw, uj * 8, C, Ho, Wo, z, g);
+    for (int i = 0; i < 8; ++i) g[i] = av[i] = 0.f;
+    if (live) {
+      const int q = pix / W;
+      const int iw = pix - q * W;
+      const int b = q / H;
+      const int ih = q - b * H;
+      unpack8(*reinterpret_cast<const uint4*>(a + static_cast<size_t>(pix) * C + uj * 8), av);
+      pool_grad8(dy, am, b, ih, iw, uj * 8, C, Ho, Wo, z, g);
+    }
+    if (mine) {
+      float4* ar = a_s + up * ld4 + 1 + uj * 2;
+      ar[0] = make_float4(av[0], av[1], av[2], av[3]);
+      ar[1] = make_float4(av[4], av[5], av[6], av[7]);
+      if (uj == 0) ar[-1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (uj == CH - 1) ar[2] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    float first[8];
+    if (mine) {
+      const float4* ar = a_s + up * ld4 + uj * 2;  // channels c0-4 .. c0+11
+      float w[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 x = ar[q];
+        w[4 * q] = x.x;
+        w[4 * q + 1] = x.y;
+        w[4 * q + 2] = x.z;
+        w[4 * q + 3] = x.w;
+      }
+      float tv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float sum = 0.f;
+#pragma unroll
+        for (int q = 2; q <= 6; ++q) sum += w[i + q] * w[i + q];
+        const float sc = k + alpha * sum;
+        const float sb = __powf(sc, -beta);
+        first[i] = g[i] * sb;
+        tv[i] = g[i] * av[i] * __fdividef(sb, sc);
+      }
+      float4* tr = t_s + up * ld4 + 1 + uj * 2;
+      tr[0] = make_float4(tv[0], tv[1], tv[2], tv[3]);
+      tr[1] = make_float4(tv[4], tv[5], tv[6], tv[7]);
+      if (uj == 0) tr[-1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (uj == CH - 1) tr[2] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    if (live) {
+      const float4* tr = t_s + up * ld4 + uj * 2;  // channels c0-4 .. c0+11
+      float w[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 x = tr[q];
+        w[4 * q] = x.x;
+        w[4 * q + 1] = x.y;
+        w[4 * q + 2] = x.z;
+        w[4 * q + 3] = x.w;
+      }
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float cross = 0.f;
+#pragma unroll
+        for (int q = 2; q <= 6; ++q) cross += w[i + q];
+        const float aj = av[i];
+        const float d = first[i] - 2.f * alpha * beta * aj * cross;
+        o[i] = aj > 0.f ? d : 0.f;
+      }
+      const uint4 packed = pack8(o);
+      const size_t e = static_cast<size_t>(pix) * C + uj * 8;
+      *reinterpret_cast<uint4*>(da + e) = packed;
+      if (dl) *reinterpret_cast<uint4*>(dl + e) = pack8(g);
+      float r[8];
+      unpack8(packed, r);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) bsum[i] += r[i];
+    }
+    __syncthreads();  // the next group reuses a_s / t_s
   }
+  if (!bias_part) return;
+  // per-channel sum over the block's pixel lanes, in lane order
+  float* red = reinterpret_cast<float*>(fsm4);
   if (mine) {
-    float4* ar = a_s + up * ld4 + 1 + uj * 2;
-    ar[0] = make_float4(av[0], av[1], av[2], av[3]);
-    ar[1] = make_float4(av[4], av[5], av[6], av[7]);
-    if (uj == 0) ar[-1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (uj == CH - 1) ar[2] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[up * C + uj * 8 + i] = bsum[i];
   }
   __syncthreads();
-  float first[8];
-  if (mine) {
-    const float4* ar = a_s + up * ld4 + uj * 2;  // channels c0-4 .. c0+11
-    float w[16];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 x = ar[q];
-      w[4 * q] = x.x;
-      w[4 * q + 1] = x.y;
-      w[4 * q + 2] = x.z;
-      w[4 * q + 3] = x.w;
-    }
-    float tv[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float sum = 0.f;
-#pragma unroll
-      for (int q = 2; q <= 6; ++q) sum += w[i + q] * w[i + q];
-      const float sc = k + alpha * sum;
-      const float sb = __powf(sc, -beta);
-      first[i] = g[i] * sb;
-      tv[i] = g[i] * av[i] * __fdividef(sb, sc);
-    }
-    float4* tr = t_s + up * ld4 + 1 + uj * 2;
-    tr[0] = make_float4(tv[0], tv[1], tv[2], tv[3]);
-    tr[1] = make_float4(tv[4], tv[5], tv[6], tv[7]);
-    if (uj == 0) tr[-1] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (uj == CH - 1) tr[2] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float v = 0.f;
+    for (int q = 0; q < np; ++q) v += red[q * C + c];
+    bias_part[static_cast<size_t>(blockIdx.x) * C + c] = v;
   }
-  __syncthreads();
-  if (!live) return;
-  const float4* tr = t_s + up * ld4 + uj * 2;  // channels c0-4 .. c0+11
-  float w[16];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 x = tr[q];
-    w[4 * q] = x.x;
-    w[4 * q + 1] = x.y;
-    w[4 * q + 2] = x.z;
-    w[4 * q + 3] = x.w;
-  }
-  float o[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float cross = 0.f;
-#pragma unroll
-    for (int q = 2; q <= 6; ++q) cross += w[i + q];
-    const float aj = av[i];
-    const float d = first[i] - 2.f * alpha * beta * aj * cross;
-    o[i] = aj > 0.f ? d : 0.f;
-  }
-  const size_t e = static_cast<size_t>(pix) * C + uj * 8;
-  *reinterpret_cast<uint4*>(da + e) = pack8(o);
-  if (dl) *reinterpret_cast<uint4*>(dl + e) = pack8(g);
 }
 
 __global__ void k_pool_fwd_f32(const float* __restrict__ x, float* __restrict__ y, int B, int H,
@@ -849,11 +911,7 @@ __global__ void __launch_bounds__(256) k_colsum_partial(const bf16* __restrict__
 // ------------------------------------------------------------------ SGD
 // [S] 3.4 "Training Procedure Details", update rule; [W] listing TRAIN_STEP:
 // v <- momentum v - wd lr w - lr g ; w <- w + v, for every parameter.
-__device__ __forceinline__ void sgd_one(float& w, float& v, float g, const HParams& hp) {
-  const float vn = hp.momentum * v - hp.weight_decay * hp.lr * w - hp.lr * g;
-  v = vn;
-  w = w + vn;
-}
+// (sgd_one, the per-parameter update, is in kernels.h)
 
 struct ConvIdx {
   long long fwd, dg, part_inner;
@@ -1252,7 +1310,7 @@ void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s) {
 }
 
 void launch_s2d(const bf16* x, bf16* xs, int B, cudaStream_t s) {
-  k_s2d<<<grid_for(1LL * B * 57 * 57 * 8, 256), 256, 0, s>>>(x, xs, B);
+  k_s2d<<<B * 57, 256, 0, s>>>(x, xs, B);
   count_launch();
 }
 void launch_lrn_fwd(const bf16* a, bf16* b, long long P, int C, int, float k, float alpha,
@@ -1303,17 +1361,24 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
   count_launch();
   return true;
 }
+constexpr int kPoolLrnBlocks = 148 * 8;  // persistent blocks: eight per SM
+int pool_lrn_bwd_parts(long long npix, int C) {
+  const int np = 256 / (C / 8);
+  const long long groups = np > 0 ? (npix + np - 1) / np : 0;
+  return static_cast<int>(groups < kPoolLrnBlocks ? groups : kPoolLrnBlocks);
+}
 bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
                          int B, int H, int W, int C, int z, float k, float alpha, float beta,
-                         cudaStream_t s) {
+                         float* bias_part, cudaStream_t s) {
   if (C % kSlab || C > 2048 || (z != 2 && z != 3) || H < z || W < z) return false;
   const int np = 256 / (C / 8);  // whole pixels per block, one 8-channel unit per thread
   const long long npix = 1LL * B * H * W;
   if (npix * C >= (1LL << 31)) return false;  // 32-bit element offsets
   const size_t smem = static_cast<size_t>(np) * 2 * (C + 8) * sizeof(float);
   if (np < 1 || smem > 48 * 1024) return false;
-  k_pool_lrn_bwd<<<static_cast<unsigned>((npix + np - 1) / np), 256, smem, s>>>(
-      dy, am, a, dl, da, static_cast<int>(npix), np, H, W, C, z, k, alpha, beta);
+  // persistent blocks (at most kPoolLrnBlocks, one bias partial row each)
+  k_pool_lrn_bwd<<<pool_lrn_bwd_parts(npix, C), 256, smem, s>>>(
+      dy, am, a, dl, da, static_cast<int>(npix), np, H, W, C, z, k, alpha, beta, bias_part);
   count_launch();
   return true;
 }

@@ -24,6 +24,14 @@ struct HParams {
   uint32_t drop_thresh;  // keep iff Philox word >= drop_thresh
 };
 
+// [S] 3.4 "Training Procedure Details", update rule; [W] listing TRAIN_STEP:
+// v <- momentum v - wd lr w - lr g ; w <- w + v, for every parameter.
+__device__ __forceinline__ void sgd_one(float& w, float& v, float g, const HParams& hp) {
+  const float vn = hp.momentum * v - hp.weight_decay * hp.lr * w - hp.lr * g;
+  v = vn;
+  w = w + vn;
+}
+
 // Canonical conv weight [Cout][K][K][Cg] -> positions in the GEMM layouts.
 struct ConvMap {
   int Cout, K, Cg, groups;
@@ -66,9 +74,12 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
                          int C, int z, float k, float alpha, float beta, cudaStream_t s);
 // Fused stride-2 max-pool backward + normalisation backward + ReLU mask
 // (a > 0) into da; dl (the normalised map's gradient) written when non-null.
+// bias_part (nullable): per-block column sums of the stored da,
+// [pool_lrn_bwd_parts(B*H*W, C)][C] fp32, for the conv bias update.
 bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
                          int B, int H, int W, int C, int z, float k, float alpha, float beta,
-                         cudaStream_t s);
+                         float* bias_part, cudaStream_t s);
+int pool_lrn_bwd_parts(long long npix, int C);
 void launch_pool_fwd_f32(const float* x, float* y, int B, int H, int W, int C, int z, int st,
                          cudaStream_t s);
 

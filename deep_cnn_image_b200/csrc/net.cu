@@ -70,12 +70,25 @@ struct Plan {
   bool ok = false;
 };
 
+// K blocks per split of a split-K GEMM with `tiles` output tiles: the split
+// count that minimises waves x (K blocks per item + a fixed per-item cost of
+// writing its fp32 partial tile, about two K blocks of loads), preferring
+// fewer splits (fewer partials to reduce) on ties.
 int pick_kbps(long long tiles, int kblocks, int num_sms, int min_blocks) {
-  long long s = (2LL * num_sms + tiles - 1) / tiles;
-  const long long smax = kblocks / min_blocks > 0 ? kblocks / min_blocks : 1;
-  if (s > smax) s = smax;
-  if (s < 1) s = 1;
-  return static_cast<int>((kblocks + s - 1) / s);
+  const int smax = kblocks / min_blocks > 0 ? kblocks / min_blocks : 1;
+  int best_kbps = kblocks;
+  long long best_cost = -1;
+  for (int s = 1; s <= smax; ++s) {
+    const int kbps = (kblocks + s - 1) / s;
+    const long long items = tiles * ((kblocks + kbps - 1) / kbps);
+    const long long waves = (items + num_sms - 1) / num_sms;
+    const long long cost = waves * (kbps + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_kbps = kbps;
+    }
+  }
+  return best_kbps;
 }
 
 }  // namespace
@@ -296,7 +309,7 @@ bool desc_fc_fwd(GemmDesc* d, const FcL& F, const bf16* x, const bf16* w, float*
   a.groups = 1;
   const long long tiles = 1LL * ((B + 127) / 128) * ((F.Out + 127) / 128);
   a.kb_per_split = splits > 0 ? (a.Kblocks + splits - 1) / splits
-                              : pick_kbps(tiles, a.Kblocks, num_sms / 2, 4);
+                              : pick_kbps(tiles, a.Kblocks, num_sms, 4);
   a.epi = EPI_F32;
   a.out = part;
   a.ld_out = F.Out;
@@ -321,7 +334,7 @@ bool desc_fc_dgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* w, flo
   a.groups = 1;
   const long long tiles = 1LL * ((B + 127) / 128) * ((F.In + d->bn - 1) / d->bn);
   a.kb_per_split = splits > 0 ? (a.Kblocks + splits - 1) / splits
-                              : pick_kbps(tiles, a.Kblocks, num_sms / 2, 4);
+                              : pick_kbps(tiles, a.Kblocks, num_sms, 4);
   a.epi = EPI_F32;
   a.out = part;
   a.ld_out = F.In;
@@ -334,26 +347,31 @@ bool desc_fc_dgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* w, flo
   return gemm_finalize(d, num_sms);
 }
 
-// FC weight gradient dW[o][i] = sum_b dz[b, o] x[b, i] (fp32, to scratch).
+
+// FC weight gradient dW[o][i] = sum_b dz[b][o] x[b][i], computed as
+// D[i][o] (rows = input features): the epilogue's lanes are consecutive
+// input features, so each column o is written as 128 contiguous bytes of
+// the fp32 [out][in] gradient (to scratch, for k_sgd_dense).
 bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, float* out, int B,
                    int num_sms, int* status) {
   memset(d, 0, sizeof(*d));
   d->asrc = A_TMA_MN;
   d->bsrc = B_TMA_MN;
-  d->bn = F.In % 256 == 0 ? 256 : 128;
+  d->bn = F.Out % 256 == 0 ? 256 : 128;
   GemmArgs& a = d->args;
-  a.M = F.Out;
-  a.N = F.In;
+  a.M = F.In;
+  a.N = F.Out;
   a.Kblocks = (B + 63) / 64;
   a.groups = 1;
   a.kb_per_split = a.Kblocks;
-  a.epi = EPI_F32;
+  a.epi = EPI_F32_T;
   a.out = out;
   a.ld_out = F.In;
-  a.split_stride = 0;
+  a.split_stride = static_cast<long long>(F.In) * F.Out;
+  a.group_stride = 0;
   a.status = status;
-  if (!tmap(&d->tmA, dz, F.Out, B, static_cast<uint64_t>(F.Out) * 2, 64, 64)) return false;
-  if (!tmap(&d->tmB, x, F.In, B, static_cast<uint64_t>(F.In) * 2, 64, 64)) return false;
+  if (!tmap(&d->tmA, x, F.In, B, static_cast<uint64_t>(F.In) * 2, 64, 64)) return false;
+  if (!tmap(&d->tmB, dz, F.Out, B, static_cast<uint64_t>(F.Out) * 2, 64, 64)) return false;
   return gemm_finalize(d, num_sms);
 }
 
@@ -483,6 +501,9 @@ size_t carve(alexnet* h, void* base) {
     const ConvL& L = h->conv[l];
     const size_t e = static_cast<size_t>(colsum_chunks(1LL * B * L.Ho * L.Ho)) * L.Cout;
     if (e > cp) cp = e;
+    // bias partials of the fused pool + normalisation backward
+    const size_t f = static_cast<size_t>(pool_lrn_bwd_parts(1LL * B * L.Ho * L.Ho, L.Cout)) * L.Cout;
+    if (f > cp) cp = f;
   }
   h->cpart_floats = cp;
   h->cpart = c.take<float>(cp);
@@ -688,9 +709,21 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     launch_pool_bwd(h->dp5, h->am[4], h->p[4], h->da[4], B, L.Ho, L.Ho, L.Cout, cfg.pool_size, 2,
                     1, s);
   }
+  // Per conv layer, top down: bias update (its column sums come from the
+  // fused pool + normalisation backward where that ran, else from da),
+  // data gradient into the layer below (and that layer's pool/LRN/ReLU
+  // backward), weight gradient and update.
   bool fused_bwd[5] = {false, false, false, false, false};
+  int bias_parts[5] = {0, 0, 0, 0, 0};
   for (int l = 4; l >= 0; --l) {
     const ConvL& L = h->conv[l];
+    const long long rows = 1LL * B * L.Ho * L.Ho;
+    if (!fused_bwd[l]) {
+      launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart, s);
+      bias_parts[l] = colsum_chunks(rows);
+    }
+    launch_sgd_bias(h->params + h->b_off[l], h->vel + h->b_off[l], h->cpart, bias_parts[l],
+                    L.Cout, gptr(h->b_off[l]), h->hp, s);
     if (l > 0) {
       ALX_TRY(run_gemm(h, P->cd[l], P->conv_flops[l], s), "conv dgrad launch");
       const ConvL& Q = h->conv[l - 1];
@@ -698,12 +731,15 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
         // dp[l-1] = d(pooled map) -> through the pool (and LRN) to da[l-1]
         if (Q.lrn) {
           // pool + normalisation + ReLU backward in one pass when the shape
-          // allows it, else pool backward now and normalisation below
+          // allows it (with layer l-1's bias column sums), else pool
+          // backward now and normalisation below
           fused_bwd[l - 1] = launch_pool_lrn_bwd(
               h->dp[l - 1], h->am[l - 1], h->a[l - 1], h->keep ? h->dl[l - 1] : nullptr,
               h->da[l - 1], B, Q.Ho, Q.Ho, Q.Cout, cfg.pool_size, cfg.lrn_k, cfg.lrn_alpha,
-              cfg.lrn_beta, s);
-          if (!fused_bwd[l - 1])
+              cfg.lrn_beta, h->cpart, s);
+          if (fused_bwd[l - 1])
+            bias_parts[l - 1] = pool_lrn_bwd_parts(1LL * B * Q.Ho * Q.Ho, Q.Cout);
+          else
             launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->dl[l - 1], B, Q.Ho, Q.Ho,
                             Q.Cout, cfg.pool_size, 2, 0, s);
         } else {
@@ -716,10 +752,6 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     launch_sgd_conv(h->params + h->w_off[l], h->vel + h->w_off[l], h->scratch,
                     P->cw[l].splits(), conv_map(h, l), h->wf[l], h->need_wd ? h->wd[l] : nullptr,
                     gptr(h->w_off[l]), h->hp, s);
-    const long long rows = 1LL * B * L.Ho * L.Ho;
-    launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart, s);
-    launch_sgd_bias(h->params + h->b_off[l], h->vel + h->b_off[l], h->cpart, colsum_chunks(rows),
-                    L.Cout, gptr(h->b_off[l]), h->hp, s);
     if (l > 0) {
       const ConvL& Q = h->conv[l - 1];
       if (Q.pool && Q.lrn && !fused_bwd[l - 1])

@@ -365,7 +365,7 @@ alexnet_status alexnet_op_pool_lrn_bwd(const void* dy, const uint8_t* argmax, co
     return ALEXNET_ERR_INVALID_ARG;
   if (!launch_pool_lrn_bwd(static_cast<const bf16*>(dy), argmax, static_cast<const bf16*>(a),
                            static_cast<bf16*>(dl), static_cast<bf16*>(da), B, H, W, C, z, k, alpha,
-                           beta, static_cast<cudaStream_t>(stream)))
+                           beta, nullptr, static_cast<cudaStream_t>(stream)))
     return ALEXNET_ERR_UNSUPPORTED;
   return done(cudaGetLastError());
 }
