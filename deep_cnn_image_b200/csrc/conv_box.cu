@@ -312,7 +312,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     conv_box_wgrad(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                    const __grid_constant__ BoxArgs a, int stages, int x_bytes) {
   constexpr int NB = (BN + 63) / 64;  // 64-channel blocks of dY per stage
-  constexpr int TMEM_COLS = pow2_cols(NPAIR * BN);
+  // two accumulator sets: the epilogue of item i drains one while the MMAs
+  // of item i + 1 fill the other
+  constexpr int ACC_COLS = NPAIR * BN;
+  constexpr int TMEM_COLS = pow2_cols(2 * ACC_COLS);
+  static_assert(2 * ACC_COLS <= 512, "two accumulator sets must fit in tensor memory");
   constexpr uint32_t IDESC = idesc_bf16(128, BN, 1, 1);
 
   extern __shared__ uint8_t smem_raw[];
@@ -325,8 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t full = smem_u32(barp);
   const uint32_t empty = full + 8 * stages;
   const uint32_t acc_full = empty + 8 * stages;
-  const uint32_t acc_empty = acc_full + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barp + 8 * (2 * stages + 2));
+  const uint32_t acc_empty = acc_full + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barp + 8 * (2 * stages + 4));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -340,8 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(full + 8 * s, 1);
       mbar_init(empty + 8 * s, 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 256);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(acc_full + 8 * q, 1);
+      mbar_init(acc_empty + 8 * q, 256);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -416,8 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sp = q / a.groups;
         const int p0 = sp * a.tiles_per_split;
         const int p1 = min(ptiles, p0 + a.tiles_per_split);
-        if (!mbar_wait(acc_empty, (icount & 1) ^ 1, a.status, abort_flag)) break;
+        const int acc = icount & 1;
+        if (!mbar_wait(acc_empty + 8 * acc, ((icount >> 1) & 1) ^ 1, a.status, abort_flag)) break;
         tc_fence_after();
+        const uint32_t dacc = tmem_base + acc * ACC_COLS;
         // per pair: start row and leading offset of its A operand (the two
         // taps' shifts), relative to a stage's first byte
         uint32_t pair_lo[NPAIR];
@@ -448,14 +456,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t al = st + pair_lo[j];
               const uint32_t bl = st + y_lo;
               for (int k = 0; k < ksteps; k += 4)
-                tc_mma_k4<128, 128>(tmem_base + j * BN, al + k * 128, pair_hi, bl + k * 128, y_hi,
+                tc_mma_k4<128, 128>(dacc + j * BN, al + k * 128, pair_hi, bl + k * 128, y_hi,
                                     IDESC, k == 0 ? acc0 : 1u);
             }
           }
           tc_commit(empty + 8 * s);
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        tc_commit(acc_full + 8 * acc);
       }
     }
   } else if (warp < 8) {
@@ -471,7 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       q /= a.cpt;
       const int g = q % a.groups;
       const int sp = q / a.groups;
-      if (!mbar_wait(acc_full, icount & 1, a.status, abort_flag)) break;
+      const int acc = icount & 1;
+      if (!mbar_wait(acc_full + 8 * acc, (icount >> 1) & 1, a.status, abort_flag)) break;
       tc_fence_after();
       const int quarter = warp & 3, half = warp >> 2;
       const int m = quarter * 32 + lane;  // row of D: half m / 64 of the pair, channel m % 64
@@ -482,7 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= nq) break;
         const int tap = 2 * (q0 + j) + (m >> 6);
         const bool valid = tap < taps;
-        const uint32_t tb = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + j * BN;
+        const uint32_t tb =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS + j * BN;
 #pragma unroll 1
         for (int c0 = 16 * half; c0 < BN; c0 += 32) {
           float v[16];
@@ -496,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(acc_empty);
+      mbar_arrive(acc_empty + 8 * acc);
     }
   }
 
@@ -530,8 +540,8 @@ Entry g_entries[] = {
     {0, 256, 2, fwd_ptr<256, 2>(), false},  {0, 64, 2, fwd_ptr<64, 2>(), false},
     {2, 64, 2, fwd_ptr<64, 2, 1>(), false},  {2, 128, 2, fwd_ptr<128, 2, 1>(), false},
     {2, 192, 2, fwd_ptr<192, 2, 1>(), false}, {2, 256, 2, fwd_ptr<256, 2, 1>(), false},
-    {1, 64, 8, wgrad_ptr<64, 8>(), false},  {1, 128, 4, wgrad_ptr<128, 4>(), false},
-    {1, 192, 2, wgrad_ptr<192, 2>(), false}, {1, 256, 2, wgrad_ptr<256, 2>(), false},
+    {1, 64, 4, wgrad_ptr<64, 4>(), false},  {1, 128, 2, wgrad_ptr<128, 2>(), false},
+    {1, 192, 1, wgrad_ptr<192, 1>(), false}, {1, 256, 1, wgrad_ptr<256, 1>(), false},
 };
 
 Entry* find_entry(int kind, int bn, int nsub) {
@@ -686,7 +696,7 @@ bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* 
     bn = 128;
   else
     bn = 256;
-  const int npair = 512 / bn > 8 ? 8 : 512 / bn;
+  const int npair = 256 / bn;  // pairs per item: two accumulator sets of npair * bn columns
   if (!find_entry(1, bn, npair)) return false;
   a.tsets = (a.npairs + npair - 1) / npair;
   a.n_tiles = (cs.Og + bn - 1) / bn;

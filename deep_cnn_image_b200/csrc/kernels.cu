@@ -383,12 +383,15 @@ __global__ void k_pool_bwd(const bf16* __restrict__ dy, const uint8_t* __restric
 constexpr int kPoolTileRows = 4;
 constexpr int kSlab = 32;  // channels per block
 
-template <int Z>
+// WC != 0: the map is WC x WC (H == W == WC known at compile time, so the
+// index divisions are by constants).
+template <int Z, int WC>
 __global__ void __launch_bounds__(256) k_lrn_pool_fwd(const bf16* __restrict__ a,
                                                       bf16* __restrict__ lo,
                                                       bf16* __restrict__ y,
-                                                      uint8_t* __restrict__ am, int H, int W,
+                                                      uint8_t* __restrict__ am, int H_, int W_,
                                                       int C, float k, float alpha, float beta) {
+  const int H = WC ? WC : H_, W = WC ? WC : W_;
   extern __shared__ __align__(16) uint4 lds[];  // [rows][W][4 chunks]
   const int Ho = (H - Z) / 2 + 1, Wo = (W - Z) / 2 + 1;
   const int oh0 = blockIdx.x * kPoolTileRows;
@@ -530,14 +533,17 @@ __device__ __forceinline__ void pool_grad8(const bf16* __restrict__ dy,
 // channel window never leaves the block: a and the cross terms
 // t_i = g_i a_i s_i^(-beta-1) go through shared memory.  Arithmetic as
 // k_lrn_bwd.
+template <int ZC, int WC>
 __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ dy,
                                                       const uint8_t* __restrict__ am,
                                                       const bf16* __restrict__ a,
                                                       bf16* __restrict__ dl,
                                                       bf16* __restrict__ da, int npix,
-                                                      int np, int H, int W, int C, int z,
+                                                      int np, int H_, int W_, int C, int z_,
                                                       float k, float alpha, float beta,
                                                       float* __restrict__ bias_part) {
+  // ZC / WC != 0: window and (square) map size known at compile time
+  const int H = WC ? WC : H_, W = WC ? WC : W_, z = ZC ? ZC : z_;
   // a_s[p][4 + c] and t_s[p][4 + c], four zeros at each end of a row; every
   // access is a 16-byte vector (a unit touches channels c0-4 .. c0+11)
   extern __shared__ float4 fsm4[];
@@ -1354,10 +1360,14 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
   const size_t smem = static_cast<size_t>(rows) * W * kSlab * 2;
   if (smem > 48 * 1024) return false;
   const dim3 grid((Ho + kPoolTileRows - 1) / kPoolTileRows, B, C / kSlab);
-  if (z == 3)
-    k_lrn_pool_fwd<3><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+  if (z == 3 && H == 55 && W == 55)
+    k_lrn_pool_fwd<3, 55><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+  else if (z == 3 && H == 27 && W == 27)
+    k_lrn_pool_fwd<3, 27><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+  else if (z == 3)
+    k_lrn_pool_fwd<3, 0><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
   else
-    k_lrn_pool_fwd<2><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+    k_lrn_pool_fwd<2, 0><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
   count_launch();
   return true;
 }
@@ -1377,8 +1387,16 @@ bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16*
   const size_t smem = static_cast<size_t>(np) * 2 * (C + 8) * sizeof(float);
   if (np < 1 || smem > 48 * 1024) return false;
   // persistent blocks (at most kPoolLrnBlocks, one bias partial row each)
-  k_pool_lrn_bwd<<<pool_lrn_bwd_parts(npix, C), 256, smem, s>>>(
-      dy, am, a, dl, da, static_cast<int>(npix), np, H, W, C, z, k, alpha, beta, bias_part);
+  const int blocks = pool_lrn_bwd_parts(npix, C);
+  if (z == 3 && H == 55 && W == 55)
+    k_pool_lrn_bwd<3, 55><<<blocks, 256, smem, s>>>(dy, am, a, dl, da, static_cast<int>(npix), np,
+                                                    H, W, C, z, k, alpha, beta, bias_part);
+  else if (z == 3 && H == 27 && W == 27)
+    k_pool_lrn_bwd<3, 27><<<blocks, 256, smem, s>>>(dy, am, a, dl, da, static_cast<int>(npix), np,
+                                                    H, W, C, z, k, alpha, beta, bias_part);
+  else
+    k_pool_lrn_bwd<0, 0><<<blocks, 256, smem, s>>>(dy, am, a, dl, da, static_cast<int>(npix), np,
+                                                   H, W, C, z, k, alpha, beta, bias_part);
   count_launch();
   return true;
 }
