@@ -25,7 +25,8 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kSmemBudget = 227 * 1024;
-constexpr int kBarBytes = 1024;  // mbarriers, tmem slot, abort flag
+constexpr int kBarBytes = 3072;  // mbarriers, tmem slot, abort flag (first 512 B); staged bias
+constexpr int kMaxBias = (kBarBytes - 512) / 4;
 
 __host__ __device__ constexpr int pow2_cols(int n) {
   return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : (n <= 256 ? 256 : 512)));
@@ -106,6 +107,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total = a.n_tiles * a.tiles_img * a.B * a.groups;
   const int taps = a.K * a.K;
   const uint32_t box_bytes = static_cast<uint32_t>(a.Hb) * a.Wb * 128;
+  // the layer's bias, staged once (read by every epilogue chunk)
+  float* sbias = reinterpret_cast<float*>(barp + 512);
+  if (a.bias && a.epi == EPI_BF16) {
+    for (int i = threadIdx.x; i < a.groups * a.col_goff; i += blockDim.x) sbias[i] = a.bias[i];
+  }
+  __syncthreads();
 
   if (warp == 8) {
     // ---------------------------------------------------------------- TMA
@@ -249,40 +256,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long row = (static_cast<long long>(b) * a.Ho + oh) * a.Wo + col;
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                             acc * NSUB * BN + sub * BN;
-#pragma unroll 1
-        for (int c0 = 16 * half; c0 < BN; c0 += 32) {
-          float v[16];
-          tmem_ld16(tb + c0, v);
-          if (!valid) continue;
+        // 8 output channels n .. n + 7 from v[0..7]: bias + ReLU or the mask
+        auto emit8 = [&](const float* v, int n) {
+          if (n >= a.Og) return;
+          const long long cg = static_cast<long long>(g) * a.col_goff + n;
+          float f[8];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int n = n_t * BN + c0 + 8 * h;
-            if (n >= a.Og) continue;
-            const long long cg = static_cast<long long>(g) * a.col_goff + n;
-            float f[8];
+          for (int i = 0; i < 8; ++i) f[i] = v[i];
+          if (a.epi == EPI_BF16) {
+            if (a.bias) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = v[8 * h + i];
-            if (a.epi == EPI_BF16) {
-              if (a.bias) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] += a.bias[cg + i];
-              }
-              if (a.relu) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] = f[i] > 0.f ? f[i] : 0.f;
-              }
-            } else {
-              const uint4 mv = *reinterpret_cast<const uint4*>(a.mask + row * a.ld_mask + cg);
-              const __nv_bfloat16* mb = reinterpret_cast<const __nv_bfloat16*>(&mv);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) f[i] = __bfloat162float(mb[i]) > 0.f ? f[i] : 0.f;
+              for (int i = 0; i < 8; ++i) f[i] += sbias[cg + i];
             }
-            uint4 o;
-            o.x = pack2(f[0], f[1]);
-            o.y = pack2(f[2], f[3]);
-            o.z = pack2(f[4], f[5]);
-            o.w = pack2(f[6], f[7]);
-            *reinterpret_cast<uint4*>(out + row * a.ld_out + cg) = o;
+            if (a.relu) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) f[i] = f[i] > 0.f ? f[i] : 0.f;
+            }
+          } else {
+            const uint4 mv = *reinterpret_cast<const uint4*>(a.mask + row * a.ld_mask + cg);
+            const __nv_bfloat16* mb = reinterpret_cast<const __nv_bfloat16*>(&mv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = __bfloat162float(mb[i]) > 0.f ? f[i] : 0.f;
+          }
+          uint4 o;
+          o.x = pack2(f[0], f[1]);
+          o.y = pack2(f[2], f[3]);
+          o.z = pack2(f[4], f[5]);
+          o.w = pack2(f[6], f[7]);
+          *reinterpret_cast<uint4*>(out + row * a.ld_out + cg) = o;
+        };
+        // 32-column loads, alternating between the two warps of a quarter
+#pragma unroll 1
+        for (int c0 = 32 * half; c0 < BN; c0 += 64) {
+          if (c0 + 32 <= BN) {
+            float v[32];
+            tmem_ld32(tb + c0, v);
+            if (!valid) continue;
+#pragma unroll
+            for (int h = 0; h < 4; ++h) emit8(v + 8 * h, n_t * BN + c0 + 8 * h);
+          } else {
+            float v[16];
+            tmem_ld16(tb + c0, v);
+            if (!valid) continue;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) emit8(v + 8 * h, n_t * BN + c0 + 8 * h);
           }
         }
       }
@@ -569,6 +586,7 @@ bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
                   int* status, bool dry) {
   memset(d, 0, sizeof(*d));
   if (cs.Cg % 8 || cs.Og % 8 || cs.C % 8 || cs.Ho() < 1 || cs.Wo() < 1) return false;
+  if (bias && cs.groups * cs.Og > kMaxBias) return false;  // the bias is staged in shared memory
   const int bn = fwd_bn(cs.Og);
   if (!bn || !find_entry(0, bn, 2)) return false;
   if (!box_fwd_common(d, cs, 0, bn, bias, relu, mask, y, num_sms, status)) return false;
