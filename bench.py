@@ -309,7 +309,9 @@ def run_ours(args):
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "no flush: a step's ~1.2 GB working set exceeds the 126 MB L2"},
         "roofline": {
-            "kernel": "tcgen05 GEMM (all conv/FC forward, data- and weight-gradient launches)",
+            "kernel": "tcgen05 GEMM (conv forward, data- and weight-gradient, FC forward and data-"
+                      "gradient launches; the FC weight-gradient launches apply the SGD update in "
+                      "their epilogue, are HBM-bound and are not counted here)",
             "bound": "tensor", "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s",
             "frac": gemm_tflops / peak if gemm_tflops else None, "traffic": None,
             "peak_source": peaks["source"] + " bf16_tflops_sustained",

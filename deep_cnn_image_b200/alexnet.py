@@ -88,6 +88,7 @@ def _load():
         "alexnet_op_philox": (st, [vp, vp, i, vp, vp]),
         "alexnet_debug_copy": (st, [vp, i, vp, sz, vp]),
         "alexnet_debug_keep": (st, [vp, i]),
+        "alexnet_debug_fc_update": (st, [vp, i]),
         "alexnet_conv_algo": (st, [vp, i, i, i, POINTER(c_int)]),
         "alexnet_stats_enable": (st, [vp, i]),
         "alexnet_stats_read": (st, [vp, POINTER(Stats)]),
@@ -222,6 +223,11 @@ class AlexNet:
         """Also store the normalised maps and their gradients (debug_copy
         10/11, 70/71) in later calls."""
         return check(lib.alexnet_debug_keep(self.h, 1 if keep else 0))
+
+    def debug_fc_update(self, fused=True):
+        """FC weights updated by the weight-gradient GEMM's epilogue (True,
+        the default) or by a separate kernel (False); identical results."""
+        return check(lib.alexnet_debug_fc_update(self.h, 1 if fused else 0))
 
     def debug_copy(self, which, dst, stream=None):
         return check(lib.alexnet_debug_copy(self.h, which, _ptr(dst), dst.numel() * dst.element_size(),

@@ -274,9 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           } else {
             const uint4 mv = *reinterpret_cast<const uint4*>(a.mask + row * a.ld_mask + cg);
-            const __nv_bfloat16* mb = reinterpret_cast<const __nv_bfloat16*>(&mv);
+            float mf[8];
+            unpack8_bits(mv, mf);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = __bfloat162float(mb[i]) > 0.f ? f[i] : 0.f;
+            for (int i = 0; i < 8; ++i) f[i] = mf[i] > 0.f ? f[i] : 0.f;
           }
           uint4 o;
           o.x = pack2(f[0], f[1]);
@@ -557,7 +558,9 @@ Entry g_entries[] = {
     {0, 256, 2, fwd_ptr<256, 2>(), false},  {0, 64, 2, fwd_ptr<64, 2>(), false},
     {2, 64, 2, fwd_ptr<64, 2, 1>(), false},  {2, 128, 2, fwd_ptr<128, 2, 1>(), false},
     {2, 192, 2, fwd_ptr<192, 2, 1>(), false}, {2, 256, 2, fwd_ptr<256, 2, 1>(), false},
-    {1, 64, 4, wgrad_ptr<64, 4>(), false},  {1, 128, 2, wgrad_ptr<128, 2>(), false},
+    {2, 256, 1, fwd_ptr<256, 1, 1>(), false},
+    {1, 64, 4, wgrad_ptr<64, 4>(), false},  {1, 96, 2, wgrad_ptr<96, 2>(), false},
+    {1, 128, 2, wgrad_ptr<128, 2>(), false},
     {1, 192, 1, wgrad_ptr<192, 1>(), false}, {1, 256, 1, wgrad_ptr<256, 1>(), false},
 };
 
@@ -578,8 +581,9 @@ int fwd_bn(int og) {
 }  // namespace
 
 // Shared geometry of the forward-type launches (kind 0 and 2).
-static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, const float* bias,
-                           int relu, const void* mask, void* y, int num_sms, int* status);
+static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, int nsub,
+                           const float* bias, int relu, const void* mask, void* y, int num_sms,
+                           int* status);
 
 bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
                   const float* bias, int relu, const void* mask, void* y, int num_sms,
@@ -589,7 +593,7 @@ bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
   if (bias && cs.groups * cs.Og > kMaxBias) return false;  // the bias is staged in shared memory
   const int bn = fwd_bn(cs.Og);
   if (!bn || !find_entry(0, bn, 2)) return false;
-  if (!box_fwd_common(d, cs, 0, bn, bias, relu, mask, y, num_sms, status)) return false;
+  if (!box_fwd_common(d, cs, 0, bn, 2, bias, relu, mask, y, num_sms, status)) return false;
   if (!dry) {
     const BoxArgs& a = d->args;
     if (!make_tmap_bf16_4d(&d->tmX, x, cs.C, cs.W, cs.H, cs.B, 64, a.Wb, a.Hb)) return false;
@@ -607,8 +611,9 @@ bool box_desc_dgrad(BoxDesc* d, const ConvShape& cs, const void* dy, const void*
   if (cs.Cg % 64 || cs.Og % 8 || cs.C % 8 || cs.Ho() < 1 || cs.Wo() < 1 || p_fwd < cs.Og)
     return false;
   const int bn = cs.Og <= 64 ? 64 : (cs.Og == 192 ? 192 : (cs.Og % 128 == 0 ? 128 : 256));
-  if (!find_entry(2, bn, 2)) return false;
-  if (!box_fwd_common(d, cs, 2, bn, nullptr, 0, mask, dx, num_sms, status)) return false;
+  const int nsub = 2;
+  if (!find_entry(2, bn, nsub)) return false;
+  if (!box_fwd_common(d, cs, 2, bn, nsub, nullptr, 0, mask, dx, num_sms, status)) return false;
   d->args.w_og = cs.Cg;
   d->args.w_p = p_fwd;
   if (!dry) {
@@ -622,8 +627,9 @@ bool box_desc_dgrad(BoxDesc* d, const ConvShape& cs, const void* dy, const void*
   return true;
 }
 
-static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, const float* bias,
-                           int relu, const void* mask, void* y, int num_sms, int* status) {
+static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, int nsub,
+                           const float* bias, int relu, const void* mask, void* y, int num_sms,
+                           int* status) {
   BoxArgs& a = d->args;
   a.B = cs.B;
   a.Ho = cs.Ho();
@@ -632,7 +638,6 @@ static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, co
   a.pad = cs.pad;
   a.Wb = a.Wo + cs.K - 1;
   if (a.Wb > 256) return false;
-  const int nsub = 2;
   a.To_h = (nsub * 128) / a.Wb;
   if (a.To_h < 1) return false;
   if (a.To_h > a.Ho) a.To_h = a.Ho;
@@ -703,11 +708,14 @@ bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* 
   a.Og = cs.Og;
   a.npairs = (taps + 1) / 2;
   a.P = cs.P();
-  // output-channel tile (N, a multiple of 64: the dY operand is MN-major in
-  // 64-channel blocks) and pairs per item within the 512 tensor-memory columns
+  // output-channel tile N (the dY operand is MN-major in 64-channel blocks;
+  // N = 96 reads two blocks and multiplies 96 channels of them) and pairs per
+  // item within the 512 tensor-memory columns
   int bn;
   if (cs.Og <= 64)
     bn = 64;
+  else if (cs.Og == 96)
+    bn = 96;
   else if (cs.Og == 192)
     bn = 192;
   else if (cs.Og <= 128 || cs.Og % 128 == 0)
@@ -721,9 +729,9 @@ bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* 
   const int ptiles = a.B * a.tiles_img;
   const long long base_items = 1LL * a.tsets * a.n_tiles * a.cpt * a.groups;
   if (splits <= 0) {
-    // the fewest position splits that give every SM an item and fill whole
-    // waves (a mostly empty last wave costs a full item's time); fewer
-    // splits also mean fewer partial sums to write and reduce
+    // the fewest position splits that give (nearly) every SM an item and
+    // fill whole waves (a mostly empty last wave costs a full item's time);
+    // fewer splits also mean fewer partial sums to write and reduce
     const long long smax = ptiles / 4 > 0 ? ptiles / 4 : 1;
     long long best = 1;
     double best_eff = -1.0;
@@ -731,7 +739,7 @@ bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* 
       const long long items = s * base_items;
       const long long waves = (items + num_sms - 1) / num_sms;
       const double eff = static_cast<double>(items) / static_cast<double>(waves * num_sms);
-      if (items >= num_sms && eff >= 0.95) {
+      if (eff >= 0.95) {
         best = s;
         break;
       }

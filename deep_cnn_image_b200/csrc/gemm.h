@@ -24,6 +24,8 @@
 
 namespace alx {
 
+struct HParams;
+
 enum ASrc : int {
   A_TMA_K = 0,
   A_TMA_MN = 1,
@@ -36,6 +38,8 @@ enum Epi : int {
   EPI_BF16_MASK = 1,  // out_bf16[row, col] = acc if mask[row, col] > 0 else 0
   EPI_F32 = 2,        // out_f32[split][group][row, col] = acc
   EPI_F32_T = 3,      // out_f32[split][group][col, row] = acc
+  EPI_SGD_T = 4,      // acc[row, col] = dL/dw of the parameter at col * ld_out + row: the
+                      // update applied in place (one split, one group)
 };
 
 struct GatherDesc {           // im2col geometry of a stride-1 convolution
@@ -67,6 +71,13 @@ struct GemmArgs {
   const float* bias;       // nullable, indexed by col + g * col_goff
   const __nv_bfloat16* mask;
   long long ld_mask;
+  // EPI_SGD_T: fp32 parameters and momentum updated in place, their bf16
+  // copy refreshed, the raw gradient stored when sgd_grads is non-null
+  float* sgd_w;
+  float* sgd_v;
+  __nv_bfloat16* sgd_shadow;
+  float* sgd_grads;
+  const HParams* hp;
   int* status;
 };
 

@@ -86,9 +86,10 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, const TileCoor
         }
       } else {
         const uint4 mv = *reinterpret_cast<const uint4*>(a.mask + row * a.ld_mask + cg);
-        const __nv_bfloat16* mb = reinterpret_cast<const __nv_bfloat16*>(&mv);
+        float mf[8];
+        unpack8_bits(mv, mf);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = __bfloat162float(mb[i]) > 0.f ? f[i] : 0.f;
+        for (int i = 0; i < 8; ++i) f[i] = mf[i] > 0.f ? f[i] : 0.f;
       }
       uint4 o;
       o.x = pack_bf16x2(f[0], f[1]);
@@ -117,6 +118,43 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, const TileCoor
   }
 }
 
+// EPI_SGD_T, [S] 3.4 "Training Procedure Details" update rule (sgd_one).
+// A thread owns one row (input feature) of the tile and walks its columns
+// (output units) 16 at a time.  For a fixed column the 32 lanes of a warp
+// touch 32 consecutive parameters, so every access is one 128-byte line per
+// warp.  The loads of the next 16 columns are issued before the current
+// ones are updated, so 32 to 64 loads per thread stay in flight.
+__device__ __forceinline__ void sgd_load16(const GemmArgs& a, size_t base, int nc,
+                                           float (&wv)[16], float (&vv)[16]) {
+  const uint32_t ld = static_cast<uint32_t>(a.ld_out);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    wv[i] = 0.f;
+    vv[i] = 0.f;
+    if (i < nc) {
+      wv[i] = a.sgd_w[base + i * ld];
+      vv[i] = a.sgd_v[base + i * ld];
+    }
+  }
+}
+__device__ __forceinline__ void sgd_apply16(const GemmArgs& a, const HParams& hp, size_t base,
+                                            int nc, float (&wv)[16], float (&vv)[16],
+                                            uint32_t taddr) {
+  const uint32_t ld = static_cast<uint32_t>(a.ld_out);
+  float g[16];
+  tmem_ld16(taddr, g);  // every lane takes part (warp-wide load)
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (i < nc) {
+      sgd_one(wv[i], vv[i], g[i], hp);
+      a.sgd_w[base + i * ld] = wv[i];
+      a.sgd_v[base + i * ld] = vv[i];
+      a.sgd_shadow[base + i * ld] = __float2bfloat16_rn(wv[i]);
+      if (a.sgd_grads) a.sgd_grads[base + i * ld] = g[i];
+    }
+  }
+}
+
 template <int BN, int ASRC, int BSRC>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -125,6 +163,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr int TMEM_COLS = tmem_cols_for(BN);
   constexpr int A_MN = (ASRC == A_TMA_MN || ASRC == A_IM2COL_MN) ? 1 : 0;
   constexpr int B_MN = (BSRC == B_TMA_MN) ? 1 : 0;
+  // the in-place update epilogue exists in the FC weight-gradient kernels only
+  constexpr bool kSgd = ASRC == A_TMA_MN && BSRC == B_TMA_MN && BN % 64 == 0;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -292,6 +332,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;
     const int half = warp >> 2;
     const int row_in_tile = quarter * 32 + lane;
+    HParams hp{};
+    if (kSgd && args.epi == EPI_SGD_T) hp = *args.hp;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tcount) {
       const TileCoord tc = decode_tile(args, t);
       const int acc = tcount & 1;
@@ -301,11 +343,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row = tc.m_t * BM + row_in_tile;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * (TMEM_COLS / 2);
+      if (kSgd && args.epi == EPI_SGD_T) {
+        // each half of the warps takes a contiguous half of the columns
+        const bool live = row < args.M;
+        const size_t ld = static_cast<size_t>(args.ld_out);
+        auto base_of = [&](int c0) {
+          return static_cast<size_t>(tc.n_t * BN + c0) * ld + (live ? row : 0);
+        };
+        auto nc_of = [&](int c0) { return live ? min(16, args.N - (tc.n_t * BN + c0)) : 0; };
+        const int cb = half * (BN / 2), ce = cb + BN / 2;  // (BN / 2) % 32 == 0
+        float wa[16], va[16], wb[16], vb[16];
+        sgd_load16(args, base_of(cb), nc_of(cb), wa, va);
 #pragma unroll 1
-      for (int c0 = 16 * half; c0 < BN; c0 += 32) {
-        float v[16];
-        tmem_ld16(tbase + c0, v);
-        epilogue_store<BN>(args, tc, row, tc.n_t * BN + c0, v);
+        for (int c0 = cb; c0 < ce; c0 += 32) {
+          sgd_load16(args, base_of(c0 + 16), nc_of(c0 + 16), wb, vb);
+          sgd_apply16(args, hp, base_of(c0), nc_of(c0), wa, va, tbase + c0);
+          if (c0 + 32 < ce) sgd_load16(args, base_of(c0 + 32), nc_of(c0 + 32), wa, va);
+          sgd_apply16(args, hp, base_of(c0 + 16), nc_of(c0 + 16), wb, vb, tbase + c0 + 16);
+        }
+      } else {
+#pragma unroll 1
+        for (int c0 = 16 * half; c0 < BN; c0 += 32) {
+          float v[16];
+          tmem_ld16(tbase + c0, v);
+          epilogue_store<BN>(args, tc, row, tc.n_t * BN + c0, v);
+        }
       }
       tc_fence_before();
       mbar_arrive(bar_acc_empty + 8 * acc);
@@ -449,6 +511,10 @@ bool gemm_finalize(GemmDesc* d, int num_sms) {
   if (a.M <= 0 || a.N <= 0 || a.Kblocks <= 0 || a.groups <= 0) return false;
   if (a.N % 8) return false;
   if (d->bsrc == B_TMA_MN && d->bn % 64) return false;
+  if (a.epi == EPI_SGD_T &&
+      (d->asrc != A_TMA_MN || d->bsrc != B_TMA_MN || d->bn % 64 || a.groups != 1 ||
+       a.kb_per_split < a.Kblocks))
+    return false;
   a.m_tiles = (a.M + BM - 1) / BM;
   a.n_tiles = (a.N + d->bn - 1) / d->bn;
   if (a.kb_per_split <= 0 || a.kb_per_split > a.Kblocks) a.kb_per_split = a.Kblocks;

@@ -26,15 +26,7 @@ inline int grid_for(long long n, int block) {
   return static_cast<int>(g);
 }
 
-__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 t = __bfloat1622float2(h[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
-}
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) { unpack8_bits(u, f); }
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   uint4 u;
   __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
@@ -43,7 +35,34 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return u;
 }
 __device__ __forceinline__ float2 ld_bf16x2(const bf16* p) {
-  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(bf16_lo(u), bf16_hi(u));
+}
+
+// LRN powers of the scale s = k + alpha * sum a^2 (s >= k > 0): s^(-beta),
+// and s^(-beta-1) for the backward.  For beta = 3/4, the pages' value, both
+// come from two reciprocal square roots: q = s^(-1/2), r = q^(-1/2) = s^(1/4),
+// s^(-3/4) = q^2 r, s^(-7/4) = s^(-3/4) q^2.  Otherwise s^(-beta) is
+// exp2(-beta log2 s) and s^(-beta-1) = s^(-beta) / s.
+template <bool B34>
+__device__ __forceinline__ float lrn_pow(float sc, float beta) {
+  if (B34) {
+    const float q = rsqrt_approx(sc);
+    return q * q * rsqrt_approx(q);
+  }
+  return __powf(sc, -beta);
+}
+template <bool B34>
+__device__ __forceinline__ void lrn_pow2(float sc, float beta, float& sb, float& sb1) {
+  if (B34) {
+    const float q = rsqrt_approx(sc);
+    const float q2 = q * q;
+    sb = q2 * rsqrt_approx(q);
+    sb1 = sb * q2;
+  } else {
+    sb = __powf(sc, -beta);
+    sb1 = __fdividef(sb, sc);
+  }
 }
 
 // ------------------------------------------------------------------ hparams
@@ -114,6 +133,7 @@ __global__ void __launch_bounds__(256) k_s2d(const bf16* __restrict__ x, bf16* _
 // Each thread owns one 8-channel chunk; consecutive lanes own consecutive
 // chunks, so the channel halo comes from the neighbouring lanes (explicit
 // loads only at the warp's edges).
+template <bool B34>
 __global__ void k_lrn_fwd(const bf16* __restrict__ a, bf16* __restrict__ b, long long P, int C,
                           float k, float alpha, float beta) {
   const uint32_t chunks = static_cast<uint32_t>(C) >> 3;
@@ -162,7 +182,7 @@ __global__ void k_lrn_fwd(const bf16* __restrict__ a, bf16* __restrict__ b, long
 #pragma unroll
       for (int j = 0; j < 5; ++j) sum += v[i + j] * v[i + j];
       const float sc = k + alpha * sum;
-      o[i] = v[i + 2] * __powf(sc, -beta);
+      o[i] = v[i + 2] * lrn_pow<B34>(sc, beta);
     }
     *reinterpret_cast<uint4*>(b + static_cast<size_t>(p) * C + c0) = pack8(o);
   }
@@ -170,6 +190,7 @@ __global__ void k_lrn_fwd(const bf16* __restrict__ a, bf16* __restrict__ b, long
 
 // Backward: da_j = g_j s_j^-beta - 2 alpha beta a_j sum_{|i-j|<=2} g_i a_i s_i^(-beta-1),
 // then times relu'(a_j) (a is the ReLU output, so a_j > 0 <=> the unit was active).
+template <bool B34>
 __global__ void k_lrn_bwd(const bf16* __restrict__ a, const bf16* __restrict__ g,
                           bf16* __restrict__ da, long long P, int C, float k, float alpha,
                           float beta) {
@@ -247,9 +268,10 @@ __global__ void k_lrn_bwd(const bf16* __restrict__ a, const bf16* __restrict__ g
 #pragma unroll
       for (int j = 0; j < 5; ++j) sum += av[i + j] * av[i + j];
       const float sc = k + alpha * sum;
-      const float sb = __powf(sc, -beta);
+      float sb, sb1;
+      lrn_pow2<B34>(sc, beta, sb, sb1);
       sp[i] = sb;
-      tt[i] = gv[i] * av[i + 2] * (sb / sc);
+      tt[i] = gv[i] * av[i + 2] * sb1;
     }
     float o[8];
 #pragma unroll
@@ -385,7 +407,7 @@ constexpr int kSlab = 32;  // channels per block
 
 // WC != 0: the map is WC x WC (H == W == WC known at compile time, so the
 // index divisions are by constants).
-template <int Z, int WC>
+template <int Z, int WC, bool B34>
 __global__ void __launch_bounds__(256) k_lrn_pool_fwd(const bf16* __restrict__ a,
                                                       bf16* __restrict__ lo,
                                                       bf16* __restrict__ y,
@@ -434,7 +456,7 @@ __global__ void __launch_bounds__(256) k_lrn_pool_fwd(const bf16* __restrict__ a
 #pragma unroll
       for (int q = 0; q < 5; ++q) sum += v[i + q] * v[i + q];
       const float sc = k + alpha * sum;
-      o[i] = v[i + 2] * __powf(sc, -beta);
+      o[i] = v[i + 2] * lrn_pow<B34>(sc, beta);
     }
     const uint4 packed = pack8(o);
     lds[(r * W + x) * 4 + j] = packed;
@@ -514,14 +536,20 @@ __device__ __forceinline__ void pool_grad8(const bf16* __restrict__ dy,
     const int oh = oh_a + (q >> 1);
     const int ow = ow_a + (q & 1);
     const uint32_t rep = static_cast<uint32_t>((ih - 2 * oh) * z + (iw - 2 * ow)) * 0x01010101u;
-    const uint32_t m0 = __vcmpeq4(av[q].x, rep), m1 = __vcmpeq4(av[q].y, rep);
+    // bytes of x that differ from this pixel's offset get their top bit set
+    // (no carry crosses a byte: (b & 0x7f) + 0x7f <= 0xfe)
+    const uint32_t x0 = av[q].x ^ rep, x1 = av[q].y ^ rep;
+    const uint32_t n0 = ((x0 & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x0;
+    const uint32_t n1 = ((x1 & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x1;
+    // sign-replicating byte permutes widen each byte's flag to its channel's
+    // 16 bits; the pooled gradient is kept where the flag is clear
+    const uint4 m = make_uint4(prmt(n0, 0, 0x9988), prmt(n0, 0, 0xBBAA), prmt(n1, 0, 0x9988),
+                               prmt(n1, 0, 0xBBAA));
+    const uint4 kept = make_uint4(gv[q].x & ~m.x, gv[q].y & ~m.y, gv[q].z & ~m.z, gv[q].w & ~m.w);
     float f[8];
-    unpack8(gv[q], f);
+    unpack8_bits(kept, f);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t m = i < 4 ? m0 : m1;
-      if ((m >> (8 * (i & 3))) & 1u) g[i] += f[i];
-    }
+    for (int i = 0; i < 8; ++i) g[i] += f[i];
   }
 }
 
@@ -533,7 +561,7 @@ __device__ __forceinline__ void pool_grad8(const bf16* __restrict__ dy,
 // channel window never leaves the block: a and the cross terms
 // t_i = g_i a_i s_i^(-beta-1) go through shared memory.  Arithmetic as
 // k_lrn_bwd.
-template <int ZC, int WC>
+template <int ZC, int WC, bool B34>
 __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ dy,
                                                       const uint8_t* __restrict__ am,
                                                       const bf16* __restrict__ a,
@@ -599,9 +627,10 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
 #pragma unroll
         for (int q = 2; q <= 6; ++q) sum += w[i + q] * w[i + q];
         const float sc = k + alpha * sum;
-        const float sb = __powf(sc, -beta);
+        float sb, sb1;
+        lrn_pow2<B34>(sc, beta, sb, sb1);
         first[i] = g[i] * sb;
-        tv[i] = g[i] * av[i] * __fdividef(sb, sc);
+        tv[i] = g[i] * av[i] * sb1;
       }
       float4* tr = t_s + up * ld4 + 1 + uj * 2;
       tr[0] = make_float4(tv[0], tv[1], tv[2], tv[3]);
@@ -1023,24 +1052,42 @@ __global__ void k_sgd_dense(float* __restrict__ w, float* __restrict__ v,
   }
 }
 
-__global__ void k_sgd_bias(float* __restrict__ b, float* __restrict__ v,
-                           const float* __restrict__ partial, int chunks, int n, float* grads_out,
-                           const HParams* __restrict__ hpp) {
-  const HParams hp = *hpp;
-  const int lane = threadIdx.x & 31;
-  const int warps = gridDim.x * (blockDim.x >> 5);
-  for (int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < n; i += warps) {
-    float g = 0.f;
-    for (int c = lane; c < chunks; c += 32) g += partial[static_cast<size_t>(c) * n + i];
+// One block per 32 channels: thread (tx, ty) sums the partial rows
+// ty, ty + 32, ... of channel tx (four loads in flight), then row ty = 0
+// adds the 32 row-group sums in order and applies the update.
+__global__ void __launch_bounds__(1024) k_sgd_bias(float* __restrict__ b, float* __restrict__ v,
+                                                   const float* __restrict__ partial, int chunks,
+                                                   int n, float* grads_out,
+                                                   const HParams* __restrict__ hpp) {
+  __shared__ float red[32][33];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int i = blockIdx.x * 32 + tx;
+  float g = 0.f;
+  if (i < n) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* p = partial + i;
+    const size_t n32 = static_cast<size_t>(n) * 32;
+    int c = ty;
+    for (; c + 96 < chunks; c += 128) {
+      const float* q = p + static_cast<size_t>(c) * n;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) g += __shfl_xor_sync(0xffffffffu, g, o);
-    if (lane == 0) {
-      float wv = b[i], vv = v[i];
-      sgd_one(wv, vv, g, hp);
-      b[i] = wv;
-      v[i] = vv;
-      if (grads_out) grads_out[i] = g;
+      for (int u = 0; u < 4; ++u) acc[u] += q[u * n32];
     }
+    for (; c < chunks; c += 32) acc[0] += p[static_cast<size_t>(c) * n];
+    g = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  }
+  red[ty][tx] = g;
+  __syncthreads();
+  if (ty == 0 && i < n) {
+    float sum = 0.f;
+#pragma unroll 8
+    for (int q = 0; q < 32; ++q) sum += red[q][tx];
+    const HParams hp = *hpp;
+    float wv = b[i], vv = v[i];
+    sgd_one(wv, vv, sum, hp);
+    b[i] = wv;
+    v[i] = vv;
+    if (grads_out) grads_out[i] = sum;
   }
 }
 
@@ -1321,12 +1368,18 @@ void launch_s2d(const bf16* x, bf16* xs, int B, cudaStream_t s) {
 }
 void launch_lrn_fwd(const bf16* a, bf16* b, long long P, int C, int, float k, float alpha,
                     float beta, cudaStream_t s) {
-  k_lrn_fwd<<<grid_for(P * (C / 8), 256), 256, 0, s>>>(a, b, P, C, k, alpha, beta);
+  if (beta == 0.75f)
+    k_lrn_fwd<true><<<grid_for(P * (C / 8), 256), 256, 0, s>>>(a, b, P, C, k, alpha, beta);
+  else
+    k_lrn_fwd<false><<<grid_for(P * (C / 8), 256), 256, 0, s>>>(a, b, P, C, k, alpha, beta);
   count_launch();
 }
 void launch_lrn_bwd(const bf16* a, const bf16* g, bf16* da, long long P, int C, int, float k,
                     float alpha, float beta, cudaStream_t s) {
-  k_lrn_bwd<<<grid_for(P * (C / 8), 256), 256, 0, s>>>(a, g, da, P, C, k, alpha, beta);
+  if (beta == 0.75f)
+    k_lrn_bwd<true><<<grid_for(P * (C / 8), 256), 256, 0, s>>>(a, g, da, P, C, k, alpha, beta);
+  else
+    k_lrn_bwd<false><<<grid_for(P * (C / 8), 256), 256, 0, s>>>(a, g, da, P, C, k, alpha, beta);
   count_launch();
 }
 void launch_lrn_fwd_f32(const float* a, float* b, long long P, int C, int, float k, float alpha,
@@ -1360,19 +1413,24 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
   const size_t smem = static_cast<size_t>(rows) * W * kSlab * 2;
   if (smem > 48 * 1024) return false;
   const dim3 grid((Ho + kPoolTileRows - 1) / kPoolTileRows, B, C / kSlab);
+  auto go = [&](auto kern) { kern<<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta); };
+  const bool b34 = beta == 0.75f;
   if (z == 3 && H == 55 && W == 55)
-    k_lrn_pool_fwd<3, 55><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+    b34 ? go(k_lrn_pool_fwd<3, 55, true>) : go(k_lrn_pool_fwd<3, 55, false>);
   else if (z == 3 && H == 27 && W == 27)
-    k_lrn_pool_fwd<3, 27><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+    b34 ? go(k_lrn_pool_fwd<3, 27, true>) : go(k_lrn_pool_fwd<3, 27, false>);
   else if (z == 3)
-    k_lrn_pool_fwd<3, 0><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+    b34 ? go(k_lrn_pool_fwd<3, 0, true>) : go(k_lrn_pool_fwd<3, 0, false>);
   else
-    k_lrn_pool_fwd<2, 0><<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta);
+    b34 ? go(k_lrn_pool_fwd<2, 0, true>) : go(k_lrn_pool_fwd<2, 0, false>);
   count_launch();
   return true;
 }
 constexpr int kPoolLrnBlocks = 148 * 8;  // persistent blocks: eight per SM
-int pool_lrn_bwd_parts(long long npix, int C) {
+int pool_lrn_bwd_parts(int B, int H, int W, int C, int z) {
+  (void)z;
+  if (C <= 0 || C % 8) return 0;
+  const long long npix = 1LL * B * H * W;
   const int np = 256 / (C / 8);
   const long long groups = np > 0 ? (npix + np - 1) / np : 0;
   return static_cast<int>(groups < kPoolLrnBlocks ? groups : kPoolLrnBlocks);
@@ -1381,22 +1439,24 @@ bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16*
                          int B, int H, int W, int C, int z, float k, float alpha, float beta,
                          float* bias_part, cudaStream_t s) {
   if (C % kSlab || C > 2048 || (z != 2 && z != 3) || H < z || W < z) return false;
-  const int np = 256 / (C / 8);  // whole pixels per block, one 8-channel unit per thread
   const long long npix = 1LL * B * H * W;
   if (npix * C >= (1LL << 31)) return false;  // 32-bit element offsets
+  const bool b34 = beta == 0.75f;
+  const int blocks = pool_lrn_bwd_parts(B, H, W, C, z);
+  const int np = 256 / (C / 8);  // whole pixels per block, one 8-channel unit per thread
   const size_t smem = static_cast<size_t>(np) * 2 * (C + 8) * sizeof(float);
   if (np < 1 || smem > 48 * 1024) return false;
   // persistent blocks (at most kPoolLrnBlocks, one bias partial row each)
-  const int blocks = pool_lrn_bwd_parts(npix, C);
+  auto go = [&](auto kern) {
+    kern<<<blocks, 256, smem, s>>>(dy, am, a, dl, da, static_cast<int>(npix), np, H, W, C, z, k,
+                                   alpha, beta, bias_part);
+  };
   if (z == 3 && H == 55 && W == 55)
-    k_pool_lrn_bwd<3, 55><<<blocks, 256, smem, s>>>(dy, am, a, dl, da, static_cast<int>(npix), np,
-                                                    H, W, C, z, k, alpha, beta, bias_part);
+    b34 ? go(k_pool_lrn_bwd<3, 55, true>) : go(k_pool_lrn_bwd<3, 55, false>);
   else if (z == 3 && H == 27 && W == 27)
-    k_pool_lrn_bwd<3, 27><<<blocks, 256, smem, s>>>(dy, am, a, dl, da, static_cast<int>(npix), np,
-                                                    H, W, C, z, k, alpha, beta, bias_part);
+    b34 ? go(k_pool_lrn_bwd<3, 27, true>) : go(k_pool_lrn_bwd<3, 27, false>);
   else
-    k_pool_lrn_bwd<0, 0><<<blocks, 256, smem, s>>>(dy, am, a, dl, da, static_cast<int>(npix), np,
-                                                   H, W, C, z, k, alpha, beta, bias_part);
+    b34 ? go(k_pool_lrn_bwd<0, 0, true>) : go(k_pool_lrn_bwd<0, 0, false>);
   count_launch();
   return true;
 }
@@ -1459,8 +1519,8 @@ void launch_sgd_dense(float* w, float* v, const float* g, long long n, bf16* sha
 }
 void launch_sgd_bias(float* b, float* v, const float* partial, int chunks, int n, float* grads_out,
                      const HParams* hp, cudaStream_t s) {
-  k_sgd_bias<<<grid_for(static_cast<long long>(n) * 32, 256), 256, 0, s>>>(b, v, partial, chunks,
-                                                                           n, grads_out, hp);
+  if (n <= 0) return;
+  k_sgd_bias<<<(n + 31) / 32, dim3(32, 32), 0, s>>>(b, v, partial, chunks, n, grads_out, hp);
   count_launch();
 }
 void launch_conv_shadows(const float* w, const ConvMap& m, bf16* fwd, bf16* dg, cudaStream_t s) {

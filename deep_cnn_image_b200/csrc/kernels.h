@@ -75,11 +75,11 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
 // Fused stride-2 max-pool backward + normalisation backward + ReLU mask
 // (a > 0) into da; dl (the normalised map's gradient) written when non-null.
 // bias_part (nullable): per-block column sums of the stored da,
-// [pool_lrn_bwd_parts(B*H*W, C)][C] fp32, for the conv bias update.
+// [pool_lrn_bwd_parts(B, H, W, C, z)][C] fp32, for the conv bias update.
 bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
                          int B, int H, int W, int C, int z, float k, float alpha, float beta,
                          float* bias_part, cudaStream_t s);
-int pool_lrn_bwd_parts(long long npix, int C);
+int pool_lrn_bwd_parts(int B, int H, int W, int C, int z);
 void launch_pool_fwd_f32(const float* x, float* y, int B, int H, int W, int C, int z, int st,
                          cudaStream_t s);
 

@@ -66,6 +66,7 @@ struct FcL {
 struct Plan {
   ConvPlan cf[5], cd[5], cw[5];
   GemmDesc ff[3], fd[3], fw[3];
+  GemmDesc fws[3];  // FC weight gradient with the update in its epilogue
   double conv_flops[5], fc_flops[3];  // algorithmic FLOPs of one pass of each layer
   bool ok = false;
 };
@@ -171,6 +172,9 @@ struct alexnet {
   // also store the normalised maps (lo) and their gradients (dl), which the
   // fused normalisation + pooling kernels otherwise keep on chip
   bool keep = false;
+  // FC weights updated by the weight-gradient GEMM's epilogue (else by a
+  // separate update kernel reading an fp32 gradient)
+  bool fc_fused = true;
   // the flipped weight copies (wd) are refreshed only while some data-gradient
   // plan reads them (the box kernel reads the forward copies transposed)
   bool need_wd = false;
@@ -375,6 +379,23 @@ bool desc_fc_wgrad(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, flo
   return gemm_finalize(d, num_sms);
 }
 
+// The same product with [S] 3.4's update applied by the epilogue: w, v
+// ([Out][In] fp32) updated in place, the bf16 copy refreshed, the gradient
+// kept in grads when given.  No fp32 gradient reaches global memory.
+bool desc_fc_wgrad_sgd(GemmDesc* d, const FcL& F, const bf16* dz, const bf16* x, float* w,
+                       float* v, bf16* shadow, float* grads, const HParams* hp, int B,
+                       int num_sms, int* status) {
+  if (!desc_fc_wgrad(d, F, dz, x, nullptr, B, num_sms, status)) return false;
+  GemmArgs& a = d->args;
+  a.epi = EPI_SGD_T;
+  a.sgd_w = w;
+  a.sgd_v = v;
+  a.sgd_shadow = shadow;
+  a.sgd_grads = grads;
+  a.hp = hp;
+  return gemm_finalize(d, num_sms);
+}
+
 size_t desc_f32_need(const GemmDesc& d) {
   const GemmArgs& a = d.args;
   if (a.epi == EPI_F32_T) return static_cast<size_t>(a.splits) * a.split_stride;
@@ -417,6 +438,10 @@ bool build_plan(alexnet* h, int B, Plan* P) {
       return set_err(h, "fc data-gradient plan");
     if (!desc_fc_wgrad(&P->fw[f], h->fc[f], dz[f], fin[f], h->scratch, B, ns, h->status))
       return set_err(h, "fc weight-gradient plan");
+    float* gr = h->grads ? h->grads + h->w_off[5 + f] : nullptr;
+    if (!desc_fc_wgrad_sgd(&P->fws[f], h->fc[f], dz[f], fin[f], h->params + h->w_off[5 + f],
+                           h->vel + h->w_off[5 + f], h->wf[5 + f], gr, h->hp, B, ns, h->status))
+      return set_err(h, "fc weight-gradient + update plan");
   }
   if (h->scratch) {
     const GemmDesc* all[] = {&P->ff[0], &P->ff[1], &P->ff[2], &P->fd[0], &P->fd[1],
@@ -502,7 +527,8 @@ size_t carve(alexnet* h, void* base) {
     const size_t e = static_cast<size_t>(colsum_chunks(1LL * B * L.Ho * L.Ho)) * L.Cout;
     if (e > cp) cp = e;
     // bias partials of the fused pool + normalisation backward
-    const size_t f = static_cast<size_t>(pool_lrn_bwd_parts(1LL * B * L.Ho * L.Ho, L.Cout)) * L.Cout;
+    const size_t f =
+        static_cast<size_t>(pool_lrn_bwd_parts(B, L.Ho, L.Ho, L.Cout, cfg.pool_size)) * L.Cout;
     if (f > cp) cp = f;
   }
   h->cpart_floats = cp;
@@ -696,9 +722,15 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     const FcL& F = h->fc[f];
     ALX_TRY(run_gemm(h, P->fd[f], P->fc_flops[f], s), "fc dgrad launch");
     launch_dgrad_finalize(h->scratch, P->fd[f].args.splits, B, F.In, mask[f], dxo[f], s);
-    ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s), "fc wgrad launch");
-    launch_sgd_dense(h->params + h->w_off[5 + f], h->vel + h->w_off[5 + f], h->scratch,
-                     h->w_len[5 + f], h->wf[5 + f], gptr(h->w_off[5 + f]), h->hp, s);
+    if (h->fc_fused) {
+      // HBM-bound (the update moves 20 bytes per weight against 256 MMA
+      // FLOPs): launched outside the per-GEMM tensor-roofline records
+      ALX_TRY(launch_any(P->fws[f], s), "fc wgrad + update launch");
+    } else {
+      ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s), "fc wgrad launch");
+      launch_sgd_dense(h->params + h->w_off[5 + f], h->vel + h->w_off[5 + f], h->scratch,
+                       h->w_len[5 + f], h->wf[5 + f], gptr(h->w_off[5 + f]), h->hp, s);
+    }
     launch_colsum_partial(dz[f], B, F.Out, h->cpart, s);
     launch_sgd_bias(h->params + h->b_off[5 + f], h->vel + h->b_off[5 + f], h->cpart,
                     colsum_chunks(B), F.Out, gptr(h->b_off[5 + f]), h->hp, s);
@@ -738,7 +770,7 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
               h->da[l - 1], B, Q.Ho, Q.Ho, Q.Cout, cfg.pool_size, cfg.lrn_k, cfg.lrn_alpha,
               cfg.lrn_beta, h->cpart, s);
           if (fused_bwd[l - 1])
-            bias_parts[l - 1] = pool_lrn_bwd_parts(1LL * B * Q.Ho * Q.Ho, Q.Cout);
+            bias_parts[l - 1] = pool_lrn_bwd_parts(B, Q.Ho, Q.Ho, Q.Cout, cfg.pool_size);
           else
             launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->dl[l - 1], B, Q.Ho, Q.Ho,
                             Q.Cout, cfg.pool_size, 2, 0, s);
@@ -929,7 +961,7 @@ alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* la
   alexnet_status st = ALEXNET_OK;
   const int64_t l0 = launch_counter();
   if (h->use_graphs) {
-    const int key = 4 * B + (h->keep ? 2 : 0) + (h->stats_on ? 1 : 0);
+    const int key = 8 * B + (h->fc_fused ? 4 : 0) + (h->keep ? 2 : 0) + (h->stats_on ? 1 : 0);
     auto it = h->train_graphs.find(key);
     if (it == h->train_graphs.end()) {
       if (!h->cap_stream)
@@ -1140,6 +1172,12 @@ alexnet_status alexnet_conv_algo(alexnet_t* h, int batch, int layer, int pass, i
 alexnet_status alexnet_debug_keep(alexnet_t* h, int keep) {
   if (!h) return ALEXNET_ERR_INVALID_ARG;
   h->keep = keep != 0;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_debug_fc_update(alexnet_t* h, int fused) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  h->fc_fused = fused != 0;
   return ALEXNET_OK;
 }
 

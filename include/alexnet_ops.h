@@ -180,6 +180,14 @@ ALEXNET_API alexnet_status alexnet_conv_algo(alexnet_t* h, int batch, int layer,
  * The pages have no counterpart (a debugging aid). */
 ALEXNET_API alexnet_status alexnet_debug_keep(alexnet_t* h, int keep);
 
+/* fused != 0 (default): the FC weight-gradient GEMM applies the SGD update
+ * ([S] "ImageNet Classification with Deep Convolutional Neural Networks",
+ * 3.4 "Training Procedure Details") to the FC weights in its epilogue, so
+ * no fp32 weight gradient reaches memory.  0: the gradient goes to scratch
+ * and a separate kernel applies the same update.  Results are identical;
+ * the switch exists to compare the two. */
+ALEXNET_API alexnet_status alexnet_debug_fc_update(alexnet_t* h, int fused);
+
 ALEXNET_API alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst, size_t bytes,
                                   void* stream);
 

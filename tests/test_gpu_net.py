@@ -415,6 +415,31 @@ def test_keep_switch_changes_nothing(ax):
         np.testing.assert_array_equal(out[0][2][l], out[1][2][l])
 
 
+def test_fused_fc_update_changes_nothing(ax):
+    """The FC update applied in the weight-gradient epilogue and by the
+    separate kernel give bit-identical parameters, momenta and gradients."""
+    import torch
+    B, N = 4, 2
+    xs = [synthetic.to_bf16(synthetic.images(90 + i, B))[0].cuda() for i in range(N)]
+    ys = [dev(synthetic.labels(95 + i, B)) for i in range(N)]
+    out = []
+    for fused in (False, True):
+        net = _make(ax, batch_max=B, seed=23, keep_grads=1)
+        net.debug_fc_update(fused)
+        for i in range(N):
+            net.train_step(xs[i], ys[i], B, 0.01)
+        n = net.params_bytes() // 4
+        p = torch.zeros(n, dtype=torch.float32)
+        net.get_params(p)
+        g = torch.zeros(n, dtype=torch.float32)
+        net.get_grads(g)
+        torch.cuda.synchronize()
+        out.append((p.numpy().copy(), g.numpy().copy()))
+        net.close()
+    np.testing.assert_array_equal(out[0][0], out[1][0])
+    np.testing.assert_array_equal(out[0][1], out[1][1])
+
+
 def test_label_out_of_range_sets_status(ax):
     import torch
     B = 2
