@@ -610,8 +610,14 @@ bool box_desc_dgrad(BoxDesc* d, const ConvShape& cs, const void* dy, const void*
   memset(d, 0, sizeof(*d));
   if (cs.Cg % 64 || cs.Og % 8 || cs.C % 8 || cs.Ho() < 1 || cs.Wo() < 1 || p_fwd < cs.Og)
     return false;
-  const int bn = cs.Og <= 64 ? 64 : (cs.Og == 192 ? 192 : (cs.Og % 128 == 0 ? 128 : 256));
-  const int nsub = 2;
+  // 256 output channels: one 128-row sub-tile of N = 256 (half the MMA
+  // instructions of two N = 128 tiles, accumulators still double-buffered)
+  int bn = cs.Og <= 64 ? 64 : (cs.Og == 192 ? 192 : (cs.Og % 128 == 0 ? 128 : 256));
+  int nsub = 2;
+  if (cs.Og % 256 == 0 && cs.Wo() + cs.K - 1 <= 128) {
+    bn = 256;
+    nsub = 1;
+  }
   if (!find_entry(2, bn, nsub)) return false;
   if (!box_fwd_common(d, cs, 2, bn, nsub, nullptr, 0, mask, dx, num_sms, status)) return false;
   d->args.w_og = cs.Cg;
@@ -716,8 +722,8 @@ bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* 
     bn = 64;
   else if (cs.Og == 96)
     bn = 96;
-  else if (cs.Og == 192)
-    bn = 192;
+  else if (cs.Og == 192 || cs.Og == 384)
+    bn = 192;  // 384: two N = 192 tiles issue a third fewer MMAs than three of 128
   else if (cs.Og <= 128 || cs.Og % 128 == 0)
     bn = 128;
   else
