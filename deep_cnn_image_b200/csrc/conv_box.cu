@@ -558,7 +558,8 @@ Entry g_entries[] = {
     {0, 256, 2, fwd_ptr<256, 2>(), false},  {0, 64, 2, fwd_ptr<64, 2>(), false},
     {2, 64, 2, fwd_ptr<64, 2, 1>(), false},  {2, 128, 2, fwd_ptr<128, 2, 1>(), false},
     {2, 192, 2, fwd_ptr<192, 2, 1>(), false}, {2, 256, 2, fwd_ptr<256, 2, 1>(), false},
-    {2, 256, 1, fwd_ptr<256, 1, 1>(), false},
+    {2, 256, 1, fwd_ptr<256, 1, 1>(), false}, {2, 192, 1, fwd_ptr<192, 1, 1>(), false},
+    {0, 192, 1, fwd_ptr<192, 1>(), false},    {0, 256, 1, fwd_ptr<256, 1>(), false},
     {1, 64, 4, wgrad_ptr<64, 4>(), false},  {1, 96, 2, wgrad_ptr<96, 2>(), false},
     {1, 128, 2, wgrad_ptr<128, 2>(), false},
     {1, 192, 1, wgrad_ptr<192, 1>(), false}, {1, 256, 1, wgrad_ptr<256, 1>(), false},
@@ -568,6 +569,13 @@ Entry* find_entry(int kind, int bn, int nsub) {
   for (auto& e : g_entries)
     if (e.kind == kind && e.bn == bn && e.nsub == nsub) return &e;
   return nullptr;
+}
+
+// One 128-row sub-tile per tile when two would not leave room for a second
+// accumulator set in the 512 TMEM columns (N = 192, 256): the epilogue then
+// still overlaps the next tile's MMAs.  Needs a box row of at most 128.
+bool single_sub(int bn, const ConvShape& cs) {
+  return (bn == 192 || bn == 256) && cs.Wo() + cs.K - 1 <= 128;
 }
 
 int fwd_bn(int og) {
@@ -592,8 +600,9 @@ bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
   if (cs.Cg % 8 || cs.Og % 8 || cs.C % 8 || cs.Ho() < 1 || cs.Wo() < 1) return false;
   if (bias && cs.groups * cs.Og > kMaxBias) return false;  // the bias is staged in shared memory
   const int bn = fwd_bn(cs.Og);
-  if (!bn || !find_entry(0, bn, 2)) return false;
-  if (!box_fwd_common(d, cs, 0, bn, 2, bias, relu, mask, y, num_sms, status)) return false;
+  const int nsub = single_sub(bn, cs) ? 1 : 2;
+  if (!bn || !find_entry(0, bn, nsub)) return false;
+  if (!box_fwd_common(d, cs, 0, bn, nsub, bias, relu, mask, y, num_sms, status)) return false;
   if (!dry) {
     const BoxArgs& a = d->args;
     if (!make_tmap_bf16_4d(&d->tmX, x, cs.C, cs.W, cs.H, cs.B, 64, a.Wb, a.Hb)) return false;
@@ -613,11 +622,8 @@ bool box_desc_dgrad(BoxDesc* d, const ConvShape& cs, const void* dy, const void*
   // 256 output channels: one 128-row sub-tile of N = 256 (half the MMA
   // instructions of two N = 128 tiles, accumulators still double-buffered)
   int bn = cs.Og <= 64 ? 64 : (cs.Og == 192 ? 192 : (cs.Og % 128 == 0 ? 128 : 256));
-  int nsub = 2;
-  if (cs.Og % 256 == 0 && cs.Wo() + cs.K - 1 <= 128) {
-    bn = 256;
-    nsub = 1;
-  }
+  if (cs.Og % 256 == 0 && cs.Wo() + cs.K - 1 <= 128) bn = 256;
+  const int nsub = single_sub(bn, cs) ? 1 : 2;
   if (!find_entry(2, bn, nsub)) return false;
   if (!box_fwd_common(d, cs, 2, bn, nsub, nullptr, 0, mask, dx, num_sms, status)) return false;
   d->args.w_og = cs.Cg;
