@@ -434,7 +434,8 @@ def run_mode(args):
     value = images * args.steps / (ms / 1e3)
     line = {"metric": metric, "value": value, "unit": "images/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "higher_is_better": True, "dtype": "f32" if args.mode == "fp32" else "bf16",
+            "data": "synthetic",
             "config": {"workload": args.mode, "batch": B, "variant": args.variant},
             "step_roofline": {"achieved": flops * value / 1e12, "peak": peak,
                               "unit": "TFLOP/s", "frac": flops * value / 1e12 / peak}}

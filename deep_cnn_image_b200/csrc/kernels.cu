@@ -1052,11 +1052,14 @@ __global__ void k_sgd_dense(float* __restrict__ w, float* __restrict__ v,
   }
 }
 
-// One block per 32 channels: thread (tx, ty) sums the partial rows
-// ty, ty + 32, ... of channel tx (four loads in flight), then row ty = 0
-// adds the 32 row-group sums in order and applies the update.
+// One block per 32 channels: thread (tx, ty) sums the rows ty, ty + 32, ...
+// of channel tx (four loads in flight), then row ty = 0 adds the 32
+// row-group sums in order and applies the update.  The rows are fp32
+// partial column sums (T = float), or, for a short matrix, the bf16
+// gradient rows themselves (T = bf16: the column sum is the bias gradient).
+template <typename T>
 __global__ void __launch_bounds__(1024) k_sgd_bias(float* __restrict__ b, float* __restrict__ v,
-                                                   const float* __restrict__ partial, int chunks,
+                                                   const T* __restrict__ partial, int chunks,
                                                    int n, float* grads_out,
                                                    const HParams* __restrict__ hpp) {
   __shared__ float red[32][33];
@@ -1065,15 +1068,15 @@ __global__ void __launch_bounds__(1024) k_sgd_bias(float* __restrict__ b, float*
   float g = 0.f;
   if (i < n) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* p = partial + i;
+    const T* p = partial + i;
     const size_t n32 = static_cast<size_t>(n) * 32;
     int c = ty;
     for (; c + 96 < chunks; c += 128) {
-      const float* q = p + static_cast<size_t>(c) * n;
+      const T* q = p + static_cast<size_t>(c) * n;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] += q[u * n32];
+      for (int u = 0; u < 4; ++u) acc[u] += static_cast<float>(q[u * n32]);
     }
-    for (; c < chunks; c += 32) acc[0] += p[static_cast<size_t>(c) * n];
+    for (; c < chunks; c += 32) acc[0] += static_cast<float>(p[static_cast<size_t>(c) * n]);
     g = (acc[0] + acc[1]) + (acc[2] + acc[3]);
   }
   red[ty][tx] = g;
@@ -1326,6 +1329,129 @@ __global__ void k_conv_fwd_f32(const float* __restrict__ x, const float* __restr
   }
 }
 
+// Register-tiled fp32 direct convolution (+ bias + ReLU): a block computes
+// kTileP consecutive output pixels of one output row for up to 128 output
+// channels of one group (one channel per thread, kTileP accumulators).  The
+// input patch the tile reads (K rows x ((kTileP - 1) * stride + K) columns x
+// Cg channels, zero outside the map) is staged in shared memory; every
+// weight loaded from global memory then serves kTileP pixels.  VEC4: Cg % 4
+// == 0, the channel loop runs four channels at a time.
+constexpr int kTileP = 8;
+template <bool VEC4>
+__global__ void __launch_bounds__(128) k_conv_fwd_f32_tiled(
+    const float* __restrict__ x, const float* __restrict__ wt, const float* __restrict__ bias,
+    float* __restrict__ y, int H, int W, int Cin, int Cout, int K, int stride, int pad,
+    int groups, int Ho, int Wo) {
+  extern __shared__ float4 xs4[];
+  float* xs = reinterpret_cast<float*>(xs4);
+  const int Og = Cout / groups, Cg = Cin / groups;
+  const int g = blockIdx.z;
+  const int co = blockIdx.y * blockDim.x + threadIdx.x;
+  const int tiles_w = (Wo + kTileP - 1) / kTileP;
+  const int ow0 = (blockIdx.x % tiles_w) * kTileP;
+  const int oh = (blockIdx.x / tiles_w) % Ho;
+  const int b = blockIdx.x / (tiles_w * Ho);
+  const int PW = (kTileP - 1) * stride + K;  // patch columns
+  const int ih0 = oh * stride - pad, iw0 = ow0 * stride - pad;
+  const int n = K * PW * Cg;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int ci = i % Cg;
+    const int col = (i / Cg) % PW;
+    const int r = i / (Cg * PW);
+    const int ih = ih0 + r, iw = iw0 + col;
+    xs[i] = (ih >= 0 && ih < H && iw >= 0 && iw < W)
+                ? x[((static_cast<size_t>(b) * H + ih) * W + iw) * Cin + g * Cg + ci]
+                : 0.f;
+  }
+  __syncthreads();
+  if (co >= Og) return;
+  float acc[kTileP];
+#pragma unroll
+  for (int p = 0; p < kTileP; ++p) acc[p] = 0.f;
+  const float* wg = wt + static_cast<size_t>(g) * K * K * Cg * Og + co;
+  for (int kh = 0; kh < K; ++kh)
+    for (int kw = 0; kw < K; ++kw) {
+      const float* wp = wg + static_cast<size_t>(kh * K + kw) * Cg * Og;
+      const float* xr = xs + (kh * PW + kw) * Cg;
+      if (VEC4) {
+        for (int ci = 0; ci < Cg; ci += 4) {
+          const float w0 = wp[(ci + 0) * Og], w1 = wp[(ci + 1) * Og];
+          const float w2 = wp[(ci + 2) * Og], w3 = wp[(ci + 3) * Og];
+#pragma unroll
+          for (int p = 0; p < kTileP; ++p) {
+            const float4 v = *reinterpret_cast<const float4*>(xr + p * stride * Cg + ci);
+            acc[p] = fmaf(v.x, w0, acc[p]);
+            acc[p] = fmaf(v.y, w1, acc[p]);
+            acc[p] = fmaf(v.z, w2, acc[p]);
+            acc[p] = fmaf(v.w, w3, acc[p]);
+          }
+        }
+      } else {
+        for (int ci = 0; ci < Cg; ++ci) {
+          const float w0 = wp[ci * Og];
+#pragma unroll
+          for (int p = 0; p < kTileP; ++p) acc[p] = fmaf(xr[p * stride * Cg + ci], w0, acc[p]);
+        }
+      }
+    }
+  const float bv = bias[g * Og + co];
+#pragma unroll
+  for (int p = 0; p < kTileP; ++p) {
+    const int ow = ow0 + p;
+    if (ow < Wo) {
+      const float v = acc[p] + bv;
+      y[((static_cast<size_t>(b) * Ho + oh) * Wo + ow) * Cout + g * Og + co] = v > 0.f ? v : 0.f;
+    }
+  }
+}
+
+// fp32 FC row dot products with 16-byte loads, four in flight per lane
+// (In % 4 == 0, rows 16-byte aligned).
+__global__ void k_fc_fwd_f32_v4(const float* __restrict__ x, const float* __restrict__ w,
+                                const float* __restrict__ bias, float* __restrict__ y, int B,
+                                int In, int Out, int relu, float scale) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = 1LL * gridDim.x * (blockDim.x >> 5);
+  const int n4 = In >> 2;
+  for (long long job = blockIdx.x * 1LL * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       job < 1LL * B * Out; job += warps) {
+    const int b = static_cast<int>(job / Out), o = static_cast<int>(job % Out);
+    const float4* xr = reinterpret_cast<const float4*>(x + 1LL * b * In);
+    const float4* wr = reinterpret_cast<const float4*>(w + 1LL * o * In);
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int i = lane;
+    for (; i + 96 < n4; i += 128) {
+      float4 wv[4], xv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        wv[u] = wr[i + 32 * u];
+        xv[u] = xr[i + 32 * u];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        s0 = fmaf(xv[u].x, wv[u].x, s0);
+        s1 = fmaf(xv[u].y, wv[u].y, s1);
+        s2 = fmaf(xv[u].z, wv[u].z, s2);
+        s3 = fmaf(xv[u].w, wv[u].w, s3);
+      }
+    }
+    for (; i < n4; i += 32) {
+      const float4 wv = wr[i], xv = xr[i];
+      s0 = fmaf(xv.x, wv.x, s0);
+      s1 = fmaf(xv.y, wv.y, s1);
+      s2 = fmaf(xv.z, wv.z, s2);
+      s3 = fmaf(xv.w, wv.w, s3);
+    }
+    float s = (s0 + s1) + (s2 + s3);
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) {
+      float v = s + bias[o];
+      if (relu) v = v > 0.f ? v : 0.f;
+      y[job] = v * scale;
+    }
+  }
+}
+
 __global__ void k_fc_fwd_f32(const float* __restrict__ x, const float* __restrict__ w,
                              const float* __restrict__ bias, float* __restrict__ y, int B, int In,
                              int Out, int relu, float scale) {
@@ -1520,7 +1646,14 @@ void launch_sgd_dense(float* w, float* v, const float* g, long long n, bf16* sha
 void launch_sgd_bias(float* b, float* v, const float* partial, int chunks, int n, float* grads_out,
                      const HParams* hp, cudaStream_t s) {
   if (n <= 0) return;
-  k_sgd_bias<<<(n + 31) / 32, dim3(32, 32), 0, s>>>(b, v, partial, chunks, n, grads_out, hp);
+  k_sgd_bias<float><<<(n + 31) / 32, dim3(32, 32), 0, s>>>(b, v, partial, chunks, n, grads_out,
+                                                          hp);
+  count_launch();
+}
+void launch_sgd_bias_rows(float* b, float* v, const bf16* g, int rows, int n, float* grads_out,
+                          const HParams* hp, cudaStream_t s) {
+  if (n <= 0) return;
+  k_sgd_bias<bf16><<<(n + 31) / 32, dim3(32, 32), 0, s>>>(b, v, g, rows, n, grads_out, hp);
   count_launch();
 }
 void launch_conv_shadows(const float* w, const ConvMap& m, bf16* fwd, bf16* dg, cudaStream_t s) {
@@ -1571,17 +1704,35 @@ void launch_conv_wt_f32(const float* w, float* wt, int Cout, int K, int Cg, int 
 void launch_conv_fwd_f32(const float* x, const float* wt, const float* bias, float* y, int B,
                          int H, int W, int Cin, int Cout, int K, int stride, int pad, int groups,
                          int Ho, int Wo, cudaStream_t s) {
-  const int Og = Cout / groups;
-  long long pix = 1LL * B * Ho * Wo;
-  dim3 grid(static_cast<unsigned>(pix < 65535 * 4 ? pix : 65535 * 4), (Og + 127) / 128, groups);
-  k_conv_fwd_f32<<<grid, 128, 0, s>>>(x, wt, bias, y, B, H, W, Cin, Cout, K, stride, pad, groups,
-                                      Ho, Wo);
+  const int Og = Cout / groups, Cg = Cin / groups;
+  const long long tiles = 1LL * B * Ho * ((Wo + kTileP - 1) / kTileP);
+  const size_t smem = static_cast<size_t>(K) * ((kTileP - 1) * stride + K) * Cg * sizeof(float);
+  if (smem <= 48 * 1024 && tiles < (1LL << 31)) {
+    const dim3 grid(static_cast<unsigned>(tiles), (Og + 127) / 128, groups);
+    if (Cg % 4 == 0)
+      k_conv_fwd_f32_tiled<true><<<grid, 128, smem, s>>>(x, wt, bias, y, H, W, Cin, Cout, K,
+                                                         stride, pad, groups, Ho, Wo);
+    else
+      k_conv_fwd_f32_tiled<false><<<grid, 128, smem, s>>>(x, wt, bias, y, H, W, Cin, Cout, K,
+                                                          stride, pad, groups, Ho, Wo);
+  } else {
+    long long pix = 1LL * B * Ho * Wo;
+    dim3 grid(static_cast<unsigned>(pix < 65535 * 4 ? pix : 65535 * 4), (Og + 127) / 128, groups);
+    k_conv_fwd_f32<<<grid, 128, 0, s>>>(x, wt, bias, y, B, H, W, Cin, Cout, K, stride, pad,
+                                        groups, Ho, Wo);
+  }
   count_launch();
 }
 void launch_fc_fwd_f32(const float* x, const float* w, const float* bias, float* y, int B, int In,
                        int Out, int relu, float scale, cudaStream_t s) {
-  k_fc_fwd_f32<<<grid_for(1LL * B * Out * 32, 256), 256, 0, s>>>(x, w, bias, y, B, In, Out, relu,
-                                                                 scale);
+  const bool v4 = In % 4 == 0 && ((reinterpret_cast<uintptr_t>(x) |
+                                    reinterpret_cast<uintptr_t>(w)) & 15) == 0;
+  if (v4)
+    k_fc_fwd_f32_v4<<<grid_for(1LL * B * Out * 32, 256), 256, 0, s>>>(x, w, bias, y, B, In, Out,
+                                                                      relu, scale);
+  else
+    k_fc_fwd_f32<<<grid_for(1LL * B * Out * 32, 256), 256, 0, s>>>(x, w, bias, y, B, In, Out,
+                                                                   relu, scale);
   count_launch();
 }
 

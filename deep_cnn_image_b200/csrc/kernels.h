@@ -117,6 +117,10 @@ void launch_sgd_dense(float* w, float* v, const float* g, long long n, bf16* sha
                       float* grads_out, const HParams* hp, cudaStream_t s);
 void launch_sgd_bias(float* b, float* v, const float* partial, int chunks, int n,
                      float* grads_out, const HParams* hp, cudaStream_t s);
+// Bias update straight from a short bf16 gradient matrix g [rows][n]: the
+// bias gradient is its column sum (the FC layers, rows = batch).
+void launch_sgd_bias_rows(float* b, float* v, const bf16* g, int rows, int n, float* grads_out,
+                          const HParams* hp, cudaStream_t s);
 // Refresh bf16 operands from the fp32 masters (after init / set_params).
 void launch_conv_shadows(const float* w, const ConvMap& m, bf16* fwd, bf16* dg, cudaStream_t s);
 void launch_f32_to_bf16(const float* w, bf16* out, long long n, cudaStream_t s);

@@ -731,9 +731,8 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
       launch_sgd_dense(h->params + h->w_off[5 + f], h->vel + h->w_off[5 + f], h->scratch,
                        h->w_len[5 + f], h->wf[5 + f], gptr(h->w_off[5 + f]), h->hp, s);
     }
-    launch_colsum_partial(dz[f], B, F.Out, h->cpart, s);
-    launch_sgd_bias(h->params + h->b_off[5 + f], h->vel + h->b_off[5 + f], h->cpart,
-                    colsum_chunks(B), F.Out, gptr(h->b_off[5 + f]), h->hp, s);
+    launch_sgd_bias_rows(h->params + h->b_off[5 + f], h->vel + h->b_off[5 + f], dz[f], B, F.Out,
+                         gptr(h->b_off[5 + f]), h->hp, s);
   }
   // pool5 backward straight into conv5's pre-activation gradient
   {
