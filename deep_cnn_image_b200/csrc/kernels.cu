@@ -1329,16 +1329,19 @@ __global__ void k_conv_fwd_f32(const float* __restrict__ x, const float* __restr
   }
 }
 
-// Register-tiled fp32 direct convolution (+ bias + ReLU): a block computes
-// kTileP consecutive output pixels of one output row for up to 128 output
-// channels of one group (one channel per thread, kTileP accumulators).  The
+// Register-tiled fp32 direct convolution (+ bias + ReLU) for small batches.
+// A block computes kTileP consecutive output pixels of one output row for 32
+// output channels of one group (lane = channel, kTileP accumulators).  The
 // input patch the tile reads (K rows x ((kTileP - 1) * stride + K) columns x
-// Cg channels, zero outside the map) is staged in shared memory; every
-// weight loaded from global memory then serves kTileP pixels.  VEC4: Cg % 4
-// == 0, the channel loop runs four channels at a time.
+// Cg channels, zero outside the map) is staged in shared memory, so every
+// weight loaded from global memory serves kTileP pixels.  The block's
+// kConvWarps warps split the reduction (SPLIT_CI: each takes an equal share
+// of the input channels of every tap, Cg % (4 * kConvWarps) == 0; else a
+// share of the taps) and their sums are added in warp order.
 constexpr int kTileP = 8;
-template <bool VEC4>
-__global__ void __launch_bounds__(128) k_conv_fwd_f32_tiled(
+constexpr int kConvWarps = 8;
+template <bool SPLIT_CI>
+__global__ void __launch_bounds__(32 * kConvWarps) k_conv_fwd_f32_tiled(
     const float* __restrict__ x, const float* __restrict__ wt, const float* __restrict__ bias,
     float* __restrict__ y, int H, int W, int Cin, int Cout, int K, int stride, int pad,
     int groups, int Ho, int Wo) {
@@ -1346,7 +1349,8 @@ __global__ void __launch_bounds__(128) k_conv_fwd_f32_tiled(
   float* xs = reinterpret_cast<float*>(xs4);
   const int Og = Cout / groups, Cg = Cin / groups;
   const int g = blockIdx.z;
-  const int co = blockIdx.y * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31, wq = threadIdx.x >> 5;
+  const int co = blockIdx.y * 32 + lane;
   const int tiles_w = (Wo + kTileP - 1) / kTileP;
   const int ow0 = (blockIdx.x % tiles_w) * kTileP;
   const int oh = (blockIdx.x / tiles_w) % Ho;
@@ -1364,17 +1368,23 @@ __global__ void __launch_bounds__(128) k_conv_fwd_f32_tiled(
                 : 0.f;
   }
   __syncthreads();
-  if (co >= Og) return;
   float acc[kTileP];
 #pragma unroll
   for (int p = 0; p < kTileP; ++p) acc[p] = 0.f;
-  const float* wg = wt + static_cast<size_t>(g) * K * K * Cg * Og + co;
-  for (int kh = 0; kh < K; ++kh)
-    for (int kw = 0; kw < K; ++kw) {
-      const float* wp = wg + static_cast<size_t>(kh * K + kw) * Cg * Og;
+  if (co < Og) {
+    const float* wg = wt + static_cast<size_t>(g) * K * K * Cg * Og + co;
+    const int taps = K * K;
+    const int t0 = SPLIT_CI ? 0 : wq * taps / kConvWarps;
+    const int t1 = SPLIT_CI ? taps : (wq + 1) * taps / kConvWarps;
+    const int c0 = SPLIT_CI ? wq * (Cg / kConvWarps) : 0;
+    const int c1 = SPLIT_CI ? c0 + Cg / kConvWarps : Cg;
+    for (int t = t0; t < t1; ++t) {
+      const int kh = t / K, kw = t - kh * K;
+      const float* wp = wg + static_cast<size_t>(t) * Cg * Og;
       const float* xr = xs + (kh * PW + kw) * Cg;
-      if (VEC4) {
-        for (int ci = 0; ci < Cg; ci += 4) {
+      if (SPLIT_CI) {
+#pragma unroll 2
+        for (int ci = c0; ci < c1; ci += 4) {
           const float w0 = wp[(ci + 0) * Og], w1 = wp[(ci + 1) * Og];
           const float w2 = wp[(ci + 2) * Og], w3 = wp[(ci + 3) * Og];
 #pragma unroll
@@ -1387,21 +1397,30 @@ __global__ void __launch_bounds__(128) k_conv_fwd_f32_tiled(
           }
         }
       } else {
-        for (int ci = 0; ci < Cg; ++ci) {
+        for (int ci = c0; ci < c1; ++ci) {
           const float w0 = wp[ci * Og];
 #pragma unroll
           for (int p = 0; p < kTileP; ++p) acc[p] = fmaf(xr[p * stride * Cg + ci], w0, acc[p]);
         }
       }
     }
+  }
+  __syncthreads();  // the patch is no longer read: its space takes the warp sums
+  float* red = xs;  // [warp][pixel][lane]
+#pragma unroll
+  for (int p = 0; p < kTileP; ++p) red[(wq * kTileP + p) * 32 + lane] = acc[p];
+  __syncthreads();
+  if (wq != 0 || co >= Og) return;
   const float bv = bias[g * Og + co];
 #pragma unroll
   for (int p = 0; p < kTileP; ++p) {
     const int ow = ow0 + p;
-    if (ow < Wo) {
-      const float v = acc[p] + bv;
+    float v = 0.f;
+#pragma unroll
+    for (int q = 0; q < kConvWarps; ++q) v += red[(q * kTileP + p) * 32 + lane];
+    v += bv;
+    if (ow < Wo)
       y[((static_cast<size_t>(b) * Ho + oh) * Wo + ow) * Cout + g * Og + co] = v > 0.f ? v : 0.f;
-    }
   }
 }
 
@@ -1706,15 +1725,18 @@ void launch_conv_fwd_f32(const float* x, const float* wt, const float* bias, flo
                          int Ho, int Wo, cudaStream_t s) {
   const int Og = Cout / groups, Cg = Cin / groups;
   const long long tiles = 1LL * B * Ho * ((Wo + kTileP - 1) / kTileP);
-  const size_t smem = static_cast<size_t>(K) * ((kTileP - 1) * stride + K) * Cg * sizeof(float);
+  size_t smem = static_cast<size_t>(K) * ((kTileP - 1) * stride + K) * Cg * sizeof(float);
+  // the warp sums reuse the patch space
+  const size_t red = static_cast<size_t>(kConvWarps) * kTileP * 32 * sizeof(float);
+  if (smem < red) smem = red;
   if (smem <= 48 * 1024 && tiles < (1LL << 31)) {
-    const dim3 grid(static_cast<unsigned>(tiles), (Og + 127) / 128, groups);
-    if (Cg % 4 == 0)
-      k_conv_fwd_f32_tiled<true><<<grid, 128, smem, s>>>(x, wt, bias, y, H, W, Cin, Cout, K,
-                                                         stride, pad, groups, Ho, Wo);
+    const dim3 grid(static_cast<unsigned>(tiles), (Og + 31) / 32, groups);
+    if (Cg % (4 * kConvWarps) == 0)
+      k_conv_fwd_f32_tiled<true><<<grid, 32 * kConvWarps, smem, s>>>(
+          x, wt, bias, y, H, W, Cin, Cout, K, stride, pad, groups, Ho, Wo);
     else
-      k_conv_fwd_f32_tiled<false><<<grid, 128, smem, s>>>(x, wt, bias, y, H, W, Cin, Cout, K,
-                                                          stride, pad, groups, Ho, Wo);
+      k_conv_fwd_f32_tiled<false><<<grid, 32 * kConvWarps, smem, s>>>(
+          x, wt, bias, y, H, W, Cin, Cout, K, stride, pad, groups, Ho, Wo);
   } else {
     long long pix = 1LL * B * Ho * Wo;
     dim3 grid(static_cast<unsigned>(pix < 65535 * 4 ? pix : 65535 * 4), (Og + 127) / 128, groups);
