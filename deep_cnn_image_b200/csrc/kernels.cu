@@ -70,60 +70,43 @@ __global__ void k_write_hparams(HParams* hp, HParams v) { *hp = v; }
 
 // ------------------------------------------------------------------ s2d
 // One block per (image, output row i): the four input rows 4i .. 4i+3 are
-// one contiguous span of x (4 x 227 x 3 bf16), staged in shared memory with
-// aligned 16-byte loads, then written as 57 pixels x 64 channels in 16-byte
-// vectors: channel (dy * 4 + dx) * 3 + c of pixel j = x[4i + dy][4j + dx][c],
-// channels 48..63, columns past 226 and rows past 226 zero.
+// staged in shared memory, each at a stride of 688 elements (rows past 226
+// and columns past 226 zero).  Output pixel j holds channel
+// (dy * 4 + dx) * 3 + c = x[4i + dy][4j + dx][c]: its channels 0-23 are the
+// 12 elements at 12j of staged rows 0 and 1, channels 24-47 those of rows 2
+// and 3, channels 48-63 zero.  A thread writes one of these three parts of a
+// pixel: six 8-byte shared loads, then 16-byte stores.
 __global__ void __launch_bounds__(256) k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs,
                                              int B) {
-  constexpr int kRow = 227 * 3;                   // elements per input row
-  constexpr int kSpan16 = (4 * kRow * 2 + 15) / 16 + 1;  // 16-byte chunks covering 4 rows
-  __shared__ uint4 stage[kSpan16];
+  constexpr int kRow = 227 * 3;  // elements per input row
+  constexpr int kStride = 688;   // staged row stride: 8-byte aligned pixel groups
+  __shared__ __align__(16) uint16_t st[4 * kStride];
   const int i = blockIdx.x % 57;
   const int b = blockIdx.x / 57;
-  const int rows = min(4, 227 - 4 * i);  // valid input rows of this output row
-  const size_t first = (static_cast<size_t>(b) * 227 + 4 * i) * kRow;  // element index
-  const size_t total_bytes = static_cast<size_t>(B) * 227 * kRow * 2;
-  const uintptr_t base = reinterpret_cast<uintptr_t>(x);
-  const uintptr_t lo = (base + first * 2) & ~static_cast<uintptr_t>(15);
-  const uintptr_t hi = base + (first + static_cast<size_t>(rows) * kRow) * 2;  // exclusive
-  const int n16 = static_cast<int>((hi - lo + 15) / 16);
-  for (int q = threadIdx.x; q < n16; q += blockDim.x) {
-    const uintptr_t addr = lo + 16 * static_cast<uintptr_t>(q);
-    if (addr + 16 <= base + total_bytes) {
-      stage[q] = *reinterpret_cast<const uint4*>(addr);
-    } else {  // the tensor's last, partial chunk: element by element
-      uint16_t t[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        t[e] = addr + 2 * e + 2 <= base + total_bytes
-                   ? *reinterpret_cast<const uint16_t*>(addr + 2 * e)
-                   : 0;
-      stage[q] = make_uint4(t[0] | (static_cast<uint32_t>(t[1]) << 16),
-                            t[2] | (static_cast<uint32_t>(t[3]) << 16),
-                            t[4] | (static_cast<uint32_t>(t[5]) << 16),
-                            t[6] | (static_cast<uint32_t>(t[7]) << 16));
-    }
+  const int rows = min(4, 227 - 4 * i);
+  const uint16_t* src =
+      reinterpret_cast<const uint16_t*>(x) + (static_cast<size_t>(b) * 227 + 4 * i) * kRow;
+  for (int e = threadIdx.x; e < 4 * kStride; e += blockDim.x) {
+    const int dy = e / kStride, c = e - dy * kStride;
+    st[e] = (dy < rows && c < kRow) ? src[dy * kRow + c] : static_cast<uint16_t>(0);
   }
   __syncthreads();
-  const uint16_t* su = reinterpret_cast<const uint16_t*>(stage);
-  const int off = static_cast<int>((base + first * 2 - lo) / 2);  // element offset of row 4i
-  for (int u = threadIdx.x; u < 57 * 8; u += blockDim.x) {
-    const int j = u >> 3, chunk = u & 7;
-    uint16_t v[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int ch = chunk * 8 + q;
-      const int dy = ch / 12, r = ch - dy * 12;  // r = dx * 3 + c
-      v[q] = (ch < 48 && dy < rows && 4 * j + r / 3 < 227) ? su[off + dy * kRow + 12 * j + r] : 0;
+  uint4* out = reinterpret_cast<uint4*>(xs + (static_cast<size_t>(b) * 57 + i) * 57 * 64);
+  for (int u = threadIdx.x; u < 57 * 3; u += blockDim.x) {
+    const int j = u / 3, h = u - j * 3;
+    uint4* o = out + j * 8 + h * 3;  // 16-byte chunks: 0-2, 3-5, 6-7
+    if (h == 2) {
+      o[0] = make_uint4(0, 0, 0, 0);
+      o[1] = make_uint4(0, 0, 0, 0);
+      continue;
     }
-    uint4 o;
-    o.x = v[0] | (static_cast<uint32_t>(v[1]) << 16);
-    o.y = v[2] | (static_cast<uint32_t>(v[3]) << 16);
-    o.z = v[4] | (static_cast<uint32_t>(v[5]) << 16);
-    o.w = v[6] | (static_cast<uint32_t>(v[7]) << 16);
-    *reinterpret_cast<uint4*>(xs + ((static_cast<size_t>(b) * 57 + i) * 57 + j) * 64 + chunk * 8) =
-        o;
+    const uint2* r0 = reinterpret_cast<const uint2*>(st + (2 * h) * kStride + 12 * j);
+    const uint2* r1 = reinterpret_cast<const uint2*>(st + (2 * h + 1) * kStride + 12 * j);
+    const uint2 a0 = r0[0], a1 = r0[1], a2 = r0[2];
+    const uint2 b0 = r1[0], b1 = r1[1], b2 = r1[2];
+    o[0] = make_uint4(a0.x, a0.y, a1.x, a1.y);
+    o[1] = make_uint4(a2.x, a2.y, b0.x, b0.y);
+    o[2] = make_uint4(b1.x, b1.y, b2.x, b2.y);
   }
 }
 
@@ -347,12 +330,19 @@ __global__ void k_pool_fwd(const bf16* __restrict__ x, bf16* __restrict__ y,
   }
 }
 
-__global__ void k_pool_bwd(const bf16* __restrict__ dy, const uint8_t* __restrict__ am,
-                           const bf16* __restrict__ pooled, bf16* __restrict__ dx, int B, int H,
-                           int W, int C, int z, int st, int relu_mask) {
+// bias_part (nullable; needs 256 % (C / 8) == 0 and 256 threads): per-block
+// column sums of the stored dx, [gridDim.x][C] fp32.  A thread keeps the
+// same 8 channels on every grid-stride step, so it sums them in registers.
+__global__ void __launch_bounds__(256) k_pool_bwd(const bf16* __restrict__ dy,
+                                                  const uint8_t* __restrict__ am,
+                                                  const bf16* __restrict__ pooled,
+                                                  bf16* __restrict__ dx, int B, int H, int W,
+                                                  int C, int z, int st, int relu_mask,
+                                                  float* __restrict__ bias_part) {
   const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
   const uint32_t chunks = static_cast<uint32_t>(C) >> 3;
   const uint32_t n = static_cast<uint32_t>(B) * H * W * chunks;
+  float bsum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
     const uint32_t pix = t / chunks;
     const int c0 = static_cast<int>(t - pix * chunks) * 8;
@@ -388,7 +378,28 @@ __global__ void k_pool_bwd(const bf16* __restrict__ dy, const uint8_t* __restric
           if (ai == off && pv[i] > 0.f) acc[i] += g[i];
         }
       }
-    *reinterpret_cast<uint4*>(dx + static_cast<size_t>(pix) * C + c0) = pack8(acc);
+    const uint4 packed = pack8(acc);
+    *reinterpret_cast<uint4*>(dx + static_cast<size_t>(pix) * C + c0) = packed;
+    if (bias_part) {
+      float r[8];
+      unpack8(packed, r);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) bsum[i] += r[i];
+    }
+  }
+  if (!bias_part) return;
+  // threads with the same channels (tid mod chunks) summed in thread order
+  __shared__ float red[256 * 8];
+  const int ch = static_cast<int>(threadIdx.x % chunks);
+  const int grp = static_cast<int>(threadIdx.x / chunks);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[grp * C + ch * 8 + i] = bsum[i];
+  __syncthreads();
+  const int groups = static_cast<int>(blockDim.x / chunks);
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float v = 0.f;
+    for (int q = 0; q < groups; ++q) v += red[q * C + c];
+    bias_part[static_cast<size_t>(blockIdx.x) * C + c] = v;
   }
 }
 
@@ -729,7 +740,18 @@ __global__ void k_fc_finalize(const float* __restrict__ part, int S, int rows, i
     const long long e = q * 4;
     const int col = static_cast<int>(static_cast<uint32_t>(e) % static_cast<uint32_t>(cols));
     float4 acc = *reinterpret_cast<const float4*>(part + e);
-    for (int s = 1; s < S; ++s) {
+    // slices added in order s = 1, 2, ...; four loads in flight
+    int s = 1;
+    for (; s + 4 <= S; s += 4) {
+      float4 p[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) p[k] = *reinterpret_cast<const float4*>(part + (s + k) * plane + e);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc.x += p[k].x; acc.y += p[k].y; acc.z += p[k].z; acc.w += p[k].w;
+      }
+    }
+    for (; s < S; ++s) {
       const float4 p = *reinterpret_cast<const float4*>(part + s * plane + e);
       acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
     }
@@ -789,7 +811,22 @@ __global__ void k_dgrad_finalize(const float* __restrict__ part, int S, int rows
       v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
       v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
     }
-    for (int s = 1; s < S; ++s) {
+    // slices added in order s = 1, 2, ...; two slices (four loads) in flight
+    int s = 1;
+    for (; s + 2 <= S; s += 2) {
+      float4 a[2], b[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        a[k] = *reinterpret_cast<const float4*>(part + (s + k) * plane + e);
+        b[k] = *reinterpret_cast<const float4*>(part + (s + k) * plane + e + 4);
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        v[0] += a[k].x; v[1] += a[k].y; v[2] += a[k].z; v[3] += a[k].w;
+        v[4] += b[k].x; v[5] += b[k].y; v[6] += b[k].z; v[7] += b[k].w;
+      }
+    }
+    for (; s < S; ++s) {
       const float4 a = *reinterpret_cast<const float4*>(part + s * plane + e);
       const float4 b = *reinterpret_cast<const float4*>(part + s * plane + e + 4);
       v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
@@ -1542,11 +1579,21 @@ void launch_pool_fwd(const bf16* x, bf16* y, uint8_t* am, int B, int H, int W, i
     k_pool_fwd<2><<<grid, 256, 0, s>>>(x, y, am, B, H, W, C, st);
   count_launch();
 }
-void launch_pool_bwd(const bf16* dy, const uint8_t* am, const bf16* pooled, bf16* dx, int B,
-                     int H, int W, int C, int z, int st, int relu_mask, cudaStream_t s) {
-  k_pool_bwd<<<grid_for(1LL * B * H * W * (C / 8), 256), 256, 0, s>>>(dy, am, pooled, dx, B, H,
-                                                                     W, C, z, st, relu_mask);
+constexpr int kPoolBwdPartBlocks = 148 * 4;  // grid when the bias sums are produced
+int pool_bwd_parts(int B, int H, int W, int C) {
+  if (C < 8 || C % 8 || 256 % (C / 8)) return 0;
+  const int g = grid_for(1LL * B * H * W * (C / 8), 256);
+  return g < kPoolBwdPartBlocks ? g : kPoolBwdPartBlocks;
+}
+int launch_pool_bwd(const bf16* dy, const uint8_t* am, const bf16* pooled, bf16* dx, int B,
+                    int H, int W, int C, int z, int st, int relu_mask, cudaStream_t s,
+                    float* bias_part) {
+  const int parts = bias_part ? pool_bwd_parts(B, H, W, C) : 0;
+  const int grid = parts > 0 ? parts : grid_for(1LL * B * H * W * (C / 8), 256);
+  k_pool_bwd<<<grid, 256, 0, s>>>(dy, am, pooled, dx, B, H, W, C, z, st, relu_mask,
+                                  parts > 0 ? bias_part : nullptr);
   count_launch();
+  return parts;
 }
 bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, int H, int W,
                          int C, int z, float k, float alpha, float beta, cudaStream_t s) {

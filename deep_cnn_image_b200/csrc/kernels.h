@@ -65,8 +65,13 @@ void launch_pool_fwd(const bf16* x, bf16* y, uint8_t* am, int B, int H, int W, i
                      int st, cudaStream_t s);
 // dx[b,ih,iw,c] = sum over windows covering it whose argmax names it of dy;
 // relu_mask: also zero where the pooled value (= the selected input) is <= 0.
-void launch_pool_bwd(const bf16* dy, const uint8_t* am, const bf16* pooled, bf16* dx, int B,
-                     int H, int W, int C, int z, int st, int relu_mask, cudaStream_t s);
+// Returns the number of per-block bias partial rows written to bias_part
+// ([rows][C] fp32, column sums of the stored dx), 0 when bias_part is null
+// or the shape does not allow them (256 % (C / 8) != 0).
+int launch_pool_bwd(const bf16* dy, const uint8_t* am, const bf16* pooled, bf16* dx, int B,
+                    int H, int W, int C, int z, int st, int relu_mask, cudaStream_t s,
+                    float* bias_part = nullptr);
+int pool_bwd_parts(int B, int H, int W, int C);
 // Fused normalisation (n = 5) + stride-2 max-pool forward; lo (the
 // normalised map) is written only when non-null.  False if C % 32 != 0,
 // z not in {2, 3}, or the row tile does not fit in shared memory.

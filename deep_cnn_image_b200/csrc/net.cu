@@ -526,10 +526,13 @@ size_t carve(alexnet* h, void* base) {
     const ConvL& L = h->conv[l];
     const size_t e = static_cast<size_t>(colsum_chunks(1LL * B * L.Ho * L.Ho)) * L.Cout;
     if (e > cp) cp = e;
-    // bias partials of the fused pool + normalisation backward
+    // bias partials of the fused pool + normalisation backward, and of the
+    // pool backward
     const size_t f =
         static_cast<size_t>(pool_lrn_bwd_parts(B, L.Ho, L.Ho, L.Cout, cfg.pool_size)) * L.Cout;
     if (f > cp) cp = f;
+    const size_t pb = static_cast<size_t>(pool_bwd_parts(B, L.Ho, L.Ho, L.Cout)) * L.Cout;
+    if (pb > cp) cp = pb;
   }
   h->cpart_floats = cp;
   h->cpart = c.take<float>(cp);
@@ -734,18 +737,23 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     launch_sgd_bias_rows(h->params + h->b_off[5 + f], h->vel + h->b_off[5 + f], dz[f], B, F.Out,
                          gptr(h->b_off[5 + f]), h->hp, s);
   }
-  // pool5 backward straight into conv5's pre-activation gradient
-  {
-    const ConvL& L = h->conv[4];
-    launch_pool_bwd(h->dp5, h->am[4], h->p[4], h->da[4], B, L.Ho, L.Ho, L.Cout, cfg.pool_size, 2,
-                    1, s);
-  }
   // Per conv layer, top down: bias update (its column sums come from the
-  // fused pool + normalisation backward where that ran, else from da),
-  // data gradient into the layer below (and that layer's pool/LRN/ReLU
-  // backward), weight gradient and update.
+  // pool (+ normalisation) backward that produced da where it made them,
+  // else from da), data gradient into the layer below (and that layer's
+  // pool/LRN/ReLU backward), weight gradient and update.
   bool fused_bwd[5] = {false, false, false, false, false};
   int bias_parts[5] = {0, 0, 0, 0, 0};
+  // pool5 backward straight into conv5's pre-activation gradient, with
+  // conv5's bias column sums
+  {
+    const ConvL& L = h->conv[4];
+    const int parts = launch_pool_bwd(h->dp5, h->am[4], h->p[4], h->da[4], B, L.Ho, L.Ho, L.Cout,
+                                      cfg.pool_size, 2, 1, s, h->cpart);
+    if (parts > 0) {
+      fused_bwd[4] = true;
+      bias_parts[4] = parts;
+    }
+  }
   for (int l = 4; l >= 0; --l) {
     const ConvL& L = h->conv[l];
     const long long rows = 1LL * B * L.Ho * L.Ho;
