@@ -86,6 +86,7 @@ def _load():
         "alexnet_op_dropout_mask": (st, [c_uint64, c_uint32, c_uint32, c_float, i, i, vp, vp, sz,
                                          vp]),
         "alexnet_op_philox": (st, [vp, vp, i, vp, vp]),
+        "alexnet_op_wait_probe": (st, [vp, c_int64, vp]),
         "alexnet_debug_copy": (st, [vp, i, vp, sz, vp]),
         "alexnet_debug_keep": (st, [vp, i]),
         "alexnet_debug_fc_update": (st, [vp, i]),
@@ -318,6 +319,12 @@ def op_pool_lrn_bwd(dy, argmax, a, B, H, W, C, z, k, alpha, beta, dl, da, stream
 def op_softmax_ce(logits, labels, B, N, probs, dlogits, loss, ws, stream=None):
     return _op("alexnet_op_softmax_ce", _ptr(logits), _ptr(labels), B, N, _ptr(probs),
                _ptr(dlogits), _ptr(loss), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def op_wait_probe(status, limit_cycles, stream=None):
+    """A bounded device wait that nothing completes: sets the TIMEOUT bit of
+    the int32 device tensor `status` after limit_cycles clocks."""
+    return _op("alexnet_op_wait_probe", _ptr(status), limit_cycles, _stream(stream))
 
 
 def op_dropout_mask(seed, layer, step, p, rows, cols, keep, ws, stream=None):

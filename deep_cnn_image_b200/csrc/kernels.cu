@@ -1531,6 +1531,21 @@ __global__ void k_fc_fwd_f32(const float* __restrict__ x, const float* __restric
 
 }  // namespace
 
+// The bounded wait of the pipelined kernels, made to run out: one thread
+// waits on an mbarrier that nothing arrives at, with a limit of `limit`
+// clocks; on expiry the wait records TIMEOUT in *status and returns, and so
+// does the kernel.
+__global__ void k_wait_probe(int* status, long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  mbar_wait_limit(b, 0, status, &abort_flag, limit);
+}
+
 // ================================================================== launchers
 namespace {
 std::atomic<int64_t> g_launches{0};
@@ -1539,6 +1554,10 @@ int64_t launch_counter() { return g_launches.load(); }
 void count_launch() { g_launches.fetch_add(1); }
 void count_launch_n(int64_t n) { g_launches.fetch_add(n); }
 
+void launch_wait_probe(int* status, long long limit_cycles, cudaStream_t s) {
+  k_wait_probe<<<1, 32, 0, s>>>(status, limit_cycles);
+  count_launch();
+}
 void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s) {
   k_write_hparams<<<1, 1, 0, s>>>(hp, v);
   count_launch();

@@ -45,6 +45,10 @@ int64_t launch_counter();
 void count_launch();
 void count_launch_n(int64_t n);
 
+// A bounded device wait that nothing completes, limited to limit_cycles
+// clocks: it must set the TIMEOUT bit in *status and return (failure
+// detection without a fault).
+void launch_wait_probe(int* status, long long limit_cycles, cudaStream_t s);
 void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s);
 
 // x [B,227,227,3] (bf16) -> xs [B,57,57,64]: xs[b,i,j,(dy*4+dx)*3+c] = x[b,4i+dy,4j+dx,c]

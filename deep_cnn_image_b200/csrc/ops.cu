@@ -370,6 +370,12 @@ alexnet_status alexnet_op_pool_lrn_bwd(const void* dy, const uint8_t* argmax, co
   return done(cudaGetLastError());
 }
 
+alexnet_status alexnet_op_wait_probe(int* status, long long limit_cycles, void* stream) {
+  if (!status || limit_cycles < 1 || limit_cycles > 4000000000LL) return ALEXNET_ERR_INVALID_ARG;
+  launch_wait_probe(status, limit_cycles, static_cast<cudaStream_t>(stream));
+  return done(cudaGetLastError());
+}
+
 alexnet_status alexnet_op_softmax_ce(const float* logits, const int32_t* labels, int B, int N,
                                      float* probs, void* dlogits, float* loss, void* ws,
                                      size_t ws_bytes, void* stream) {

@@ -80,21 +80,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 // Bounded wait for the phase with the given parity.  `abort_flag` (shared)
 // lets every role of a CTA give up once one of them has timed out.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status,
-                                          volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, int* status,
+                                                volatile int* abort_flag, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+      if (clock64() - t0 > limit) {
         atomicOr(status, STATUS_TIMEOUT);
         *abort_flag = 1;
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status,
+                                          volatile int* abort_flag) {
+  return mbar_wait_limit(bar, parity, status, abort_flag, WAIT_LIMIT_CYCLES);
 }
 
 // Position in a ring of n pipeline stages: slot and the parity of the

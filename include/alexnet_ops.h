@@ -180,6 +180,16 @@ ALEXNET_API alexnet_status alexnet_conv_algo(alexnet_t* h, int batch, int layer,
  * The pages have no counterpart (a debugging aid). */
 ALEXNET_API alexnet_status alexnet_debug_keep(alexnet_t* h, int keep);
 
+/* Failure detection without a fault: one device thread waits on an
+ * mbarrier that nothing completes, through the same bounded wait the
+ * pipelined kernels use, limited to limit_cycles SM clocks (1 ..
+ * 4,000,000,000).  When the limit runs out the wait ORs the TIMEOUT bit (1)
+ * into *status (a caller-owned device int) and the kernel returns; the
+ * context stays usable.  The pages have no counterpart (a reliability
+ * check).  INVALID_ARG for a null status or a limit out of range. */
+ALEXNET_API alexnet_status alexnet_op_wait_probe(int* status, long long limit_cycles,
+                                                 void* stream);
+
 /* fused != 0 (default): the FC weight-gradient GEMM applies the SGD update
  * ([S] "ImageNet Classification with Deep Convolutional Neural Networks",
  * 3.4 "Training Procedure Details") to the FC weights in its epilogue, so

@@ -208,6 +208,26 @@ def test_fused_pool_rejects_bad_shapes(ax):
         ax.op_pool_lrn_bwd(t, am, t, 1, 9, 9, 32, 4, 2.0, 1e-4, 0.75, None, t)  # z = 4
 
 
+# ------------------------------------------------------------------ failure detection
+def test_bounded_wait_runs_out_and_reports_timeout(ax, ws):
+    """A device wait that nothing completes (the pipelined kernels' bounded
+    mbarrier wait, limited to about a millisecond) returns with the TIMEOUT
+    bit set instead of hanging, and the context stays usable."""
+    import torch
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ax.op_wait_probe(status, 2_000_000)
+    torch.cuda.synchronize()
+    assert int(status.item()) & 1 == 1
+    # the next launch on the same context still works
+    z = torch.zeros((2, 1000), dtype=torch.float32, device="cuda")
+    probs = torch.empty_like(z)
+    ax.op_softmax_ce(z, None, 2, 1000, probs, None, None, ws)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(host(probs), np.full((2, 1000), 1e-3), rtol=1e-6)
+    with pytest.raises(Exception):
+        ax.op_wait_probe(status, 0)
+
+
 # ------------------------------------------------------------------ softmax + CE
 def test_softmax_cross_entropy(ax, ws):
     import torch
