@@ -19,11 +19,12 @@ times the same steps through the public call with every batch copied from
 pinned host memory and every loss copied back inside the timed span (the
 copy of batch i+1 overlaps step i on a second stream).
 
-`--mode forward|augment|tencrop|fp32|train_variant` times the other
-workloads instead (not the headline): the batch-128 inference forward, the
-batch-512 training step fed by on-device augmentation of 256x256 uint8
-sources, batch-256 ten-crop inference, the fp32 ungrouped batch-1 forward,
-and the batch-128 training step of one of the pages' ablations
+`--mode forward|augment|tencrop|fp32|ensemble|train_variant` times the
+other workloads instead (not the headline): the batch-128 inference
+forward, the batch-512 training step fed by on-device augmentation of
+256x256 uint8 sources, batch-256 ten-crop inference, the fp32 ungrouped
+batch-1 forward, a five-network batch-128 ensemble, and the batch-128
+training step of one of the pages' ablations
 (`--variant pool2|nolrn|nodropout|ungrouped`).
 
 `--impl reference` times the CPU oracle (the plain fp64 C implementation
@@ -392,6 +393,21 @@ def run_mode(args):
         images = B
         metric = "images/sec, AlexNet bf16 train step, batch 128, variant " + args.variant
         flops = step_flops_per_image()
+    elif args.mode == "ensemble":
+        # five networks averaged ([S] ILSVRC-2012 results): every image goes
+        # through five inference forwards, then the mean softmax and top 5
+        B, M = 128, 5
+        nets = [ax.AlexNet(batch_max=B, seed=1 + m) for m in range(M)]
+        net = nets[0]
+        x = synthetic.to_bf16(synthetic.images(100, B))[0].cuda()
+        probs = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+        top5 = torch.empty((B, 5), dtype=torch.int32, device="cuda")
+        ws = torch.empty(ax.ensemble_workspace_bytes(M, B), dtype=torch.uint8, device="cuda")
+        def step():
+            ax.ensemble_forward(nets, x, B, probs, top5, ws)
+        images = B
+        metric = "images/sec, AlexNet bf16 five-network ensemble inference, batch 128"
+        flops = M * 2.0 * FWD_MACS_PER_IMAGE
     elif args.mode == "forward":
         B = 128
         net = ax.AlexNet(batch_max=B, seed=1)
@@ -466,7 +482,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-images", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", choices=["train", "forward", "augment", "tencrop", "fp32",
+    ap.add_argument("--mode", choices=["train", "forward", "augment", "tencrop", "fp32", "ensemble",
                                        "train_variant"], default="train")
     ap.add_argument("--variant", choices=["none", "pool2", "nolrn", "nodropout", "ungrouped"],
                     default="none")

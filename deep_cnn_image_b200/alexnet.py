@@ -58,6 +58,8 @@ def _load():
         "alexnet_train_step": (st, [vp, vp, vp, i, c_float, vp, vp]),
         "alexnet_augment": (st, [vp, vp, i, vp, vp, vp, vp, vp]),
         "alexnet_tencrop": (st, [vp, vp, i, vp, vp, vp, vp]),
+        "alexnet_ensemble_workspace_bytes": (sz, [i, i]),
+        "alexnet_ensemble_forward": (st, [vp, i, vp, i, vp, vp, vp, sz, vp]),
         "alexnet_params_bytes": (sz, [vp]),
         "alexnet_get_params": (st, [vp, vp, sz, vp]),
         "alexnet_set_params": (st, [vp, vp, sz, vp]),
@@ -319,6 +321,18 @@ def op_pool_lrn_bwd(dy, argmax, a, B, H, W, C, z, k, alpha, beta, dl, da, stream
 def op_softmax_ce(logits, labels, B, N, probs, dlogits, loss, ws, stream=None):
     return _op("alexnet_op_softmax_ce", _ptr(logits), _ptr(labels), B, N, _ptr(probs),
                _ptr(dlogits), _ptr(loss), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def ensemble_workspace_bytes(n_models, B):
+    return lib.alexnet_ensemble_workspace_bytes(n_models, B)
+
+
+def ensemble_forward(nets, x, B, probs_avg, top5, ws, stream=None):
+    """Mean of the softmax outputs of several networks on one batch (and its
+    top 5); ws: a device byte tensor of ensemble_workspace_bytes(len(nets), B)."""
+    arr = (c_void_p * len(nets))(*[n.h for n in nets])
+    return _op("alexnet_ensemble_forward", arr, len(nets), _ptr(x), B, _ptr(probs_avg),
+               _ptr(top5), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
 
 
 def op_wait_probe(status, limit_cycles, stream=None):

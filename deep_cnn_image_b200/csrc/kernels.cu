@@ -1268,16 +1268,22 @@ __global__ void k_tencrop_inputs(const uint8_t* __restrict__ src, int B,
 
 // Average of the ten softmax outputs, then top-5 by descending probability,
 // ties to the lower class index.
-__global__ void k_tencrop_reduce(const float* __restrict__ probs10, int B, int N,
-                                 float* __restrict__ avg, int32_t* __restrict__ top5) {
+// Mean of n probability rows per image, then its top 5 (descending, ties
+// to the lower class).  Row m of image b starts at probs + m * stride_m +
+// b * stride_b; the n rows are added in order m = 0, 1, ... and divided by n.
+// Ten-crop: the 10 crops of an image are consecutive rows; ensemble: model
+// m's rows form the m-th [B][N] block.
+__global__ void k_avg_top5(const float* __restrict__ probs, int n, long long stride_m,
+                           long long stride_b, int N, float* __restrict__ avg,
+                           int32_t* __restrict__ top5) {
   extern __shared__ float sp[];
   __shared__ float bv[32];
   __shared__ int bi[32];
   const int b = blockIdx.x;
   for (int j = threadIdx.x; j < N; j += blockDim.x) {
     float s = 0.f;
-    for (int p = 0; p < 10; ++p) s += probs10[(1LL * b * 10 + p) * N + j];
-    s = s / 10.f;
+    for (int p = 0; p < n; ++p) s += probs[p * stride_m + b * stride_b + j];
+    s = s / static_cast<float>(n);
     sp[j] = s;
     avg[1LL * b * N + j] = s;
   }
@@ -1777,7 +1783,12 @@ void launch_tencrop_inputs(const uint8_t* src, int B, const float* mean, bf16* o
 }
 void launch_tencrop_reduce(const float* probs10, int B, int N, float* probs_avg, int32_t* top5,
                            cudaStream_t s) {
-  k_tencrop_reduce<<<B, 256, N * sizeof(float), s>>>(probs10, B, N, probs_avg, top5);
+  k_avg_top5<<<B, 256, N * sizeof(float), s>>>(probs10, 10, N, 10LL * N, N, probs_avg, top5);
+  count_launch();
+}
+void launch_ensemble_reduce(const float* probs, int n, int B, int N, float* probs_avg,
+                            int32_t* top5, cudaStream_t s) {
+  k_avg_top5<<<B, 256, N * sizeof(float), s>>>(probs, n, 1LL * B * N, N, N, probs_avg, top5);
   count_launch();
 }
 void launch_conv_wt_f32(const float* w, float* wt, int Cout, int K, int Cg, int groups,

@@ -148,6 +148,10 @@ void launch_tencrop_inputs(const uint8_t* src, int B, const float* mean, bf16* o
 // Average of the ten softmaxes per image and top-5 (descending, ties -> lower index).
 void launch_tencrop_reduce(const float* probs10, int B, int N, float* probs_avg, int32_t* top5,
                            cudaStream_t s);
+// Ensemble: probs holds n models' [B][N] probabilities one after another;
+// probs_avg = their mean per image (models added in order), top5 its top 5.
+void launch_ensemble_reduce(const float* probs, int n, int B, int N, float* probs_avg,
+                            int32_t* top5, cudaStream_t s);
 
 // fp32 SIMT forward path.
 void launch_conv_wt_f32(const float* w, float* wt, int Cout, int K, int Cg, int groups,

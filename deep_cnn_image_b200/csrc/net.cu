@@ -1068,6 +1068,33 @@ alexnet_status alexnet_tencrop(alexnet_t* h, const uint8_t* src, int B, const fl
   return cuda_status(h, cudaGetLastError(), "tencrop");
 }
 
+size_t alexnet_ensemble_workspace_bytes(int n_models, int B) {
+  if (n_models < 1 || B < 1) return 0;
+  return (static_cast<size_t>(n_models) + 1) * B * kClasses * sizeof(float);
+}
+
+alexnet_status alexnet_ensemble_forward(alexnet_t* const* nets, int n_models, const void* x,
+                                        int B, float* probs_avg, int32_t* top5, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  if (!nets || n_models < 1 || !x || B < 1 || !probs_avg || !top5 || !ws ||
+      ws_bytes < alexnet_ensemble_workspace_bytes(n_models, B))
+    return ALEXNET_ERR_INVALID_ARG;
+  for (int m = 0; m < n_models; ++m)
+    if (!nets[m] || nets[m]->cfg.dtype != nets[0]->cfg.dtype || B > nets[m]->cfg.batch_max)
+      return ALEXNET_ERR_INVALID_ARG;
+  float* logits = static_cast<float*>(ws);
+  float* probs = logits + static_cast<size_t>(B) * kClasses;
+  for (int m = 0; m < n_models; ++m) {
+    const alexnet_status st =
+        alexnet_forward(nets[m], x, B, ALEXNET_INFERENCE, logits,
+                        probs + static_cast<size_t>(m) * B * kClasses, stream);
+    if (st != ALEXNET_OK) return st;
+  }
+  launch_ensemble_reduce(probs, n_models, B, kClasses, probs_avg, top5,
+                         static_cast<cudaStream_t>(stream));
+  return cudaGetLastError() == cudaSuccess ? ALEXNET_OK : ALEXNET_ERR_CUDA;
+}
+
 size_t alexnet_params_bytes(const alexnet_t* h) {
   return h ? 8 * h->n_params + 8 : 0;
 }

@@ -158,6 +158,24 @@ ALEXNET_API alexnet_status alexnet_augment(alexnet_t* h, const uint8_t* src, int
 ALEXNET_API alexnet_status alexnet_tencrop(alexnet_t* h, const uint8_t* src, int B, const float* mean,
                                float* probs_avg, int32_t* top5, void* stream);
 
+/* Ensemble of networks ([S] "ILSVRC-2012: Single CNN, Ensemble, and
+ * Pre-Training Variants": the predictions of several CNNs averaged as the
+ * mean of their softmax outputs): each of the n_models handles runs the
+ * inference forward on the same batch x, and probs_avg is the mean of their
+ * softmax outputs (added in handle order, divided by n_models), top5 its
+ * five most probable classes (descending, ties to the lower index).
+ *   nets: host array of n_models handles of one dtype, each with
+ *   batch_max >= B; x: device [B,227,227,3] in that dtype; probs_avg:
+ *   device fp32 [B,1000]; top5: device int32 [B,5]; ws: caller-owned
+ *   device scratch of alexnet_ensemble_workspace_bytes(n_models, B) bytes.
+ * INVALID_ARG on null pointers, mixed dtypes, B above a handle's batch_max
+ * or a scratch too small; otherwise the first failing forward's status. */
+ALEXNET_API size_t alexnet_ensemble_workspace_bytes(int n_models, int B);
+ALEXNET_API alexnet_status alexnet_ensemble_forward(alexnet_t* const* nets, int n_models,
+                                                    const void* x, int B, float* probs_avg,
+                                                    int32_t* top5, void* ws, size_t ws_bytes,
+                                                    void* stream);
+
 /* Size of the parameter blob: n fp32 parameters, n fp32 momentum values,
  * then the uint64 step counter (8n + 8 bytes).  Parameter order: conv1.W
  * conv1.b conv2.W conv2.b ... conv5.b fc6.W fc6.b fc7.W fc7.b fc8.W fc8.b;

@@ -440,6 +440,49 @@ def test_fused_fc_update_changes_nothing(ax):
     np.testing.assert_array_equal(out[0][1], out[1][1])
 
 
+def test_ensemble_matches_oracle(ax):
+    """Three networks on one batch: the mean of their softmax outputs and its
+    top 5 against the oracle's forwards of the same parameters."""
+    import torch
+    B, M = 2, 3
+    nets, ops = [], []
+    onet = oracle.alexnet()
+    lay = oracle.param_layout(onet)
+    for m in range(M):
+        net = _make(ax, batch_max=4)
+        n = ax.param_count(net.cfg)
+        params = synthetic.params(61 + m)
+        # a shared class signal so that the ranking is well separated
+        bo = lay[7][2]
+        params[bo:bo + 1000] = np.linspace(0, 3, 1000, dtype=np.float32)[::-1]
+        net.set_params(_blob(params, n))
+        nets.append(net)
+        ops.append(_oracle_params(params, onet))
+    xt, xr = synthetic.to_bf16(synthetic.images(64, B))
+    probs = torch.empty((B, 1000), dtype=torch.float32, device="cuda")
+    top5 = torch.empty((B, 5), dtype=torch.int32, device="cuda")
+    ws = torch.empty(ax.ensemble_workspace_bytes(M, B), dtype=torch.uint8, device="cuda")
+    ax.ensemble_forward(nets, xt.cuda(), B, probs, top5, ws)
+    torch.cuda.synchronize()
+    want = sum(oracle.forward(onet, op, xr, mode=1)[1] for op in ops) / M
+    gp = host(probs)
+    assert rel_l2(gp, want) < TOL_BF16
+    np.testing.assert_allclose(gp.sum(1), 1.0, rtol=1e-5)
+    np.testing.assert_array_equal(host(top5), oracle.topk(gp, 5))
+    # a single network: the ensemble is that network's softmax
+    one = torch.empty_like(probs)
+    ax.ensemble_forward(nets[:1], xt.cuda(), B, one, top5, ws)
+    logits = torch.empty_like(probs)
+    p1 = torch.empty_like(probs)
+    nets[0].forward(xt.cuda(), B, ax.INFERENCE, logits, p1)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(one), host(p1))
+    with pytest.raises(Exception):
+        ax.ensemble_forward(nets, xt.cuda(), B, probs, top5, ws[:16])
+    for net in nets:
+        net.close()
+
+
 def test_label_out_of_range_sets_status(ax):
     import torch
     B = 2
