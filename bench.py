@@ -19,13 +19,13 @@ times the same steps through the public call with every batch copied from
 pinned host memory and every loss copied back inside the timed span (the
 copy of batch i+1 overlaps step i on a second stream).
 
-`--mode forward|augment|tencrop|fp32|ensemble|train_variant` times the
+`--mode forward|augment|tencrop|fp32|ensemble|knn|train_variant` times the
 other workloads instead (not the headline): the batch-128 inference
 forward, the batch-512 training step fed by on-device augmentation of
 256x256 uint8 sources, batch-256 ten-crop inference, the fp32 ungrouped
-batch-1 forward, a five-network batch-128 ensemble, and the batch-128
-training step of one of the pages' ablations
-(`--variant pool2|nolrn|nodropout|ungrouped`).
+batch-1 forward, a five-network batch-128 ensemble, 128 nearest-neighbour
+queries against a million 4096-d features, and the batch-128 training step
+of one of the pages' ablations (`--variant pool2|nolrn|nodropout|ungrouped`).
 
 `--impl reference` times the CPU oracle (the plain fp64 C implementation
 under oracle/) as it stands on the host cores: each step is a training step
@@ -408,6 +408,29 @@ def run_mode(args):
         images = B
         metric = "images/sec, AlexNet bf16 five-network ensemble inference, batch 128"
         flops = M * 2.0 * FWD_MACS_PER_IMAGE
+    elif args.mode == "knn":
+        # Euclidean retrieval over 4096-d feature vectors ([S] "Qualitative
+        # Evaluation"): 128 queries against a base of one million synthetic
+        # ReLU-like bf16 features (a stand-in for last-hidden-layer
+        # activations of a million images); the base is read once per call
+        Q, N, D, K = 128, 1_000_000, 4096, 10
+        B = Q
+        g = torch.Generator(device="cuda").manual_seed(7)
+        base = torch.randn((N, D), device="cuda", dtype=torch.bfloat16, generator=g).relu_()
+        qs = torch.randn((Q, D), device="cuda", dtype=torch.bfloat16, generator=g).relu_()
+        dist = torch.empty((Q, K), dtype=torch.float32, device="cuda")
+        idx = torch.empty((Q, K), dtype=torch.int32, device="cuda")
+        ws = torch.empty(ax.knn_workspace_bytes(Q, N), dtype=torch.uint8, device="cuda")
+        # a fixed base: its squared norms computed once, outside the timing
+        bnorm = torch.empty(N, dtype=torch.float32, device="cuda")
+        ax.knn_sqnorms(base, bnorm)
+        net = None
+        def step():
+            ax.knn(qs, base, K, dist, idx, ws, base_sqnorm=bnorm)
+        images = Q
+        metric = "queries/sec, Euclidean 10-NN of 4096-d bf16 features in a base of 1,000,000"
+        flops = 2.0 * N * D
+        hbm_bytes = 2.0 * N * D
     elif args.mode == "forward":
         B = 128
         net = ax.AlexNet(batch_max=B, seed=1)
@@ -459,7 +482,8 @@ def run_mode(args):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
-    assert net.get_status() == ax.OK
+    if net is not None:
+        assert net.get_status() == ax.OK
     peak = load_peaks()["bf16_tflops_sustained"]
     value = images * args.steps / (ms / 1e3)
     line = {"metric": metric, "value": value, "unit": "images/s", "n_gpus": 1,
@@ -469,6 +493,15 @@ def run_mode(args):
             "config": {"workload": args.mode, "batch": B, "variant": args.variant},
             "step_roofline": {"achieved": flops * value / 1e12, "peak": peak,
                               "unit": "TFLOP/s", "frac": flops * value / 1e12 / peak}}
+    if args.mode == "knn":
+        # the base is streamed once per call: HBM-bound
+        gbs = hbm_bytes * args.steps / (ms / 1e3) / 1e9
+        hbm = load_peaks()["hbm_gbs"]
+        line["unit"] = "queries/s"
+        line["config"].update({"base_rows": N, "dims": D, "k": K})
+        line["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                            "frac": gbs / hbm, "traffic": None,
+                            "kernel": "base rows read by the dot-product GEMM (N x D bf16)"}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -482,8 +515,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-images", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", choices=["train", "forward", "augment", "tencrop", "fp32", "ensemble",
-                                       "train_variant"], default="train")
+    ap.add_argument("--mode", choices=["train", "forward", "augment", "tencrop", "fp32",
+                                       "ensemble", "knn", "train_variant"], default="train")
     ap.add_argument("--variant", choices=["none", "pool2", "nolrn", "nodropout", "ungrouped"],
                     default="none")
     args = ap.parse_args()

@@ -59,6 +59,9 @@ def _load():
         "alexnet_augment": (st, [vp, vp, i, vp, vp, vp, vp, vp]),
         "alexnet_tencrop": (st, [vp, vp, i, vp, vp, vp, vp]),
         "alexnet_ensemble_workspace_bytes": (sz, [i, i]),
+        "alexnet_knn_workspace_bytes": (sz, [i, i]),
+        "alexnet_knn": (st, [vp, i, vp, i, i, i, vp, vp, vp, vp, sz, vp]),
+        "alexnet_knn_sqnorms": (st, [vp, i, i, vp, vp]),
         "alexnet_ensemble_forward": (st, [vp, i, vp, i, vp, vp, vp, sz, vp]),
         "alexnet_params_bytes": (sz, [vp]),
         "alexnet_get_params": (st, [vp, vp, sz, vp]),
@@ -333,6 +336,25 @@ def ensemble_forward(nets, x, B, probs_avg, top5, ws, stream=None):
     arr = (c_void_p * len(nets))(*[n.h for n in nets])
     return _op("alexnet_ensemble_forward", arr, len(nets), _ptr(x), B, _ptr(probs_avg),
                _ptr(top5), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+
+
+def knn_workspace_bytes(Q, N):
+    return lib.alexnet_knn_workspace_bytes(Q, N)
+
+
+def knn(queries, base, k, dist, idx, ws, base_sqnorm=None, stream=None):
+    """k nearest base rows (squared Euclidean distance) of every query row;
+    queries [Q, D] and base [N, D] bf16 on the device; base_sqnorm: the base
+    rows' squared norms (knn_sqnorms), computed per call when None."""
+    Q, D = queries.shape
+    N = base.shape[0]
+    return _op("alexnet_knn", _ptr(queries), Q, _ptr(base), N, D, k, _ptr(base_sqnorm),
+               _ptr(dist), _ptr(idx), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+
+
+def knn_sqnorms(x, out, stream=None):
+    rows, D = x.shape
+    return _op("alexnet_knn_sqnorms", _ptr(x), rows, D, _ptr(out), _stream(stream))
 
 
 def op_wait_probe(status, limit_cycles, stream=None):

@@ -170,6 +170,32 @@ ALEXNET_API alexnet_status alexnet_tencrop(alexnet_t* h, const uint8_t* src, int
  *   device scratch of alexnet_ensemble_workspace_bytes(n_models, B) bytes.
  * INVALID_ARG on null pointers, mixed dtypes, B above a handle's batch_max
  * or a scratch too small; otherwise the first failing forward's status. */
+/* Nearest neighbours of feature vectors ([S] "Qualitative Evaluation",
+ * Figure 4 right: retrieval by the Euclidean distance between 4096-d
+ * last-hidden-layer activations).  For each of Q query rows, the k base rows
+ * of smallest squared distance ||q||^2 + ||x||^2 - 2 q.x (the dot products
+ * on the tensor cores, fp32 accumulation; negative rounding clamped to 0),
+ * ascending, ties to the lower base index.
+ *   queries: device bf16 [Q, D]; base: device bf16 [N, D] (both 16-byte
+ *   aligned); base_sqnorm: nullable device fp32 [N], the base rows' squared
+ *   norms (alexnet_knn_sqnorms); dist: device fp32 [Q, k]; idx: device
+ *   int32 [Q, k]; ws: caller-owned device scratch of
+ *   alexnet_knn_workspace_bytes(Q, N) bytes (holds the Q x N dot products).
+ * INVALID_ARG on null pointers, k outside 1..min(32, N), N or D not a
+ * multiple of 8, or a scratch too small; UNSUPPORTED if the tensor maps
+ * cannot be built (a base pointer not 16-byte aligned). */
+ALEXNET_API size_t alexnet_knn_workspace_bytes(int Q, int N);
+ALEXNET_API alexnet_status alexnet_knn(const void* queries, int Q, const void* base, int N, int D,
+                                       int k, const float* base_sqnorm, float* dist,
+                                       int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+/* Squared norms of the rows of a device bf16 [rows, D] matrix into a device
+ * fp32 [rows] array, the base_sqnorm alexnet_knn accepts (a fixed base needs
+ * them once; with base_sqnorm null alexnet_knn computes them every call).
+ * INVALID_ARG on null pointers, D not a positive multiple of 8 or x not
+ * 16-byte aligned. */
+ALEXNET_API alexnet_status alexnet_knn_sqnorms(const void* x, int rows, int D, float* out,
+                                               void* stream);
+
 ALEXNET_API size_t alexnet_ensemble_workspace_bytes(int n_models, int B);
 ALEXNET_API alexnet_status alexnet_ensemble_forward(alexnet_t* const* nets, int n_models,
                                                     const void* x, int B, float* probs_avg,

@@ -341,6 +341,26 @@ def topk(probs, k=5):
     return idx
 
 
+def knn(queries, base, k):
+    """[S] "Qualitative Evaluation" (Figure 4, right): retrieval by the
+    Euclidean distance between feature vectors.  For every query row the k
+    base rows of smallest squared distance sum_d (q_d - x_d)^2, in fp64 and
+    written out directly (no norm expansion); ties go to the lower base
+    index.  Returns (squared distances [Q, k], indices [Q, k])."""
+    q = np.asarray(queries, dtype=np.float64)
+    x = np.asarray(base, dtype=np.float64)
+    Q, N = q.shape[0], x.shape[0]
+    dist = np.zeros((Q, k))
+    idx = np.zeros((Q, k), np.int64)
+    for i in range(Q):
+        diff = x - q[i]
+        d = np.einsum("nd,nd->n", diff, diff)
+        order = np.lexsort((np.arange(N), d))[:k]  # by distance, then index
+        dist[i] = d[order]
+        idx[i] = order
+    return dist, idx
+
+
 # --------------------------------------------------------------------------
 # Whole network
 # --------------------------------------------------------------------------

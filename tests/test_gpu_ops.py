@@ -208,6 +208,61 @@ def test_fused_pool_rejects_bad_shapes(ax):
         ax.op_pool_lrn_bwd(t, am, t, 1, 9, 9, 32, 4, 2.0, 1e-4, 0.75, None, t)  # z = 4
 
 
+# ------------------------------------------------------------------ nearest neighbours
+@pytest.mark.parametrize("Q,N,D,k", [(8, 1000, 4096, 10), (3, 136, 64, 1), (130, 520, 128, 32)])
+def test_knn_matches_oracle(ax, Q, N, D, k):
+    """Squared distances within the fp32 bound of the oracle's direct fp64
+    sums; neighbour indices equal wherever the oracle's ranking is separated
+    by more than that bound; a planted duplicate of query 0 is its nearest."""
+    import torch
+    r = _rng(Q * 7 + N)
+    base = bf16_round(np.maximum(r.standard_normal((N, D)), 0.0))  # ReLU-like features
+    q = bf16_round(np.maximum(r.standard_normal((Q, D)), 0.0))
+    base[N // 3] = q[0]
+    dist = torch.empty((Q, k), dtype=torch.float32, device="cuda")
+    idx = torch.empty((Q, k), dtype=torch.int32, device="cuda")
+    ws = torch.empty(ax.knn_workspace_bytes(Q, N), dtype=torch.uint8, device="cuda")
+    ax.knn(dev(q, "bf16"), dev(base, "bf16"), k, dist, idx, ws)
+    torch.cuda.synchronize()
+    wd, wi = oracle.knn(q, base, k)
+    gd, gi = host(dist), host(idx)
+    # fp32 accumulation of D products of size ~1 and the norm expansion
+    tol = 1e-5 * (np.sum(q * q, axis=1).max() + np.sum(base * base, axis=1).max())
+    assert np.abs(gd - wd).max() <= tol
+    assert gi[0, 0] == N // 3 and gd[0, 0] <= tol
+    # with the base norms precomputed: identical results
+    bn = torch.empty(N, dtype=torch.float32, device="cuda")
+    ax.knn_sqnorms(dev(base, "bf16"), bn)
+    d2 = torch.empty_like(dist)
+    i2 = torch.empty_like(idx)
+    ax.knn(dev(q, "bf16"), dev(base, "bf16"), k, d2, i2, ws, base_sqnorm=bn)
+    torch.cuda.synchronize()
+    assert torch.equal(d2, dist) and torch.equal(i2, idx)
+    np.testing.assert_allclose(host(bn), np.sum(base * base, axis=1), rtol=1e-5)
+    full, _ = oracle.knn(q, base, min(N, k + 1))
+    for i in range(Q):
+        for j in range(k):
+            gap_lo = full[i, j] - full[i, j - 1] if j > 0 else np.inf
+            gap_hi = full[i, j + 1] - full[i, j] if j + 1 < full.shape[1] else np.inf
+            if min(gap_lo, gap_hi) > 2 * tol:
+                assert gi[i, j] == wi[i, j], (i, j)
+
+
+def test_knn_rejects_bad_arguments(ax):
+    import torch
+    q = torch.zeros((2, 64), dtype=torch.bfloat16, device="cuda")
+    base = torch.zeros((16, 64), dtype=torch.bfloat16, device="cuda")
+    dist = torch.empty((2, 40), dtype=torch.float32, device="cuda")
+    idx = torch.empty((2, 40), dtype=torch.int32, device="cuda")
+    ws = torch.empty(ax.knn_workspace_bytes(2, 16), dtype=torch.uint8, device="cuda")
+    with pytest.raises(Exception):
+        ax.knn(q, base, 33, dist, idx, ws)  # k above 32
+    with pytest.raises(Exception):
+        ax.knn(q, base, 17, dist, idx, ws)  # k above N
+    with pytest.raises(Exception):
+        ax.knn(q, base[:12], 4, dist, idx, ws)  # N not a multiple of 8
+
+
 # ------------------------------------------------------------------ failure detection
 def test_bounded_wait_runs_out_and_reports_timeout(ax, ws):
     """A device wait that nothing completes (the pipelined kernels' bounded

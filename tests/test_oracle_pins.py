@@ -491,3 +491,17 @@ def test_topk_against_numpy_sort():
     p = r.random((5, 1000))
     idx = oracle.topk(p, 5)
     np.testing.assert_array_equal(idx, np.argsort(-p, axis=1, kind="stable")[:, :5])
+
+
+def test_knn_hand_example():
+    """[S] "Qualitative Evaluation": Euclidean retrieval.  Worked by hand:
+    query (0, 0) against base points (3, 4) -> 25, (1, 1) -> 2, (0, 0) -> 0,
+    (1, 1) again -> 2 (tie: lower index first), (-2, 0) -> 4; query (3, 3)
+    against the same points -> 1, 8, 18, 8, 34."""
+    base = np.array([[3, 4], [1, 1], [0, 0], [1, 1], [-2, 0]], dtype=np.float64)
+    q = np.array([[0, 0], [3, 3]], dtype=np.float64)
+    d, i = oracle.knn(q, base, 4)
+    np.testing.assert_array_equal(i[0], [2, 1, 3, 4])
+    np.testing.assert_array_equal(d[0], [0, 2, 2, 4])
+    np.testing.assert_array_equal(i[1], [0, 1, 3, 2])
+    np.testing.assert_array_equal(d[1], [1, 8, 8, 18])
