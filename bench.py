@@ -178,7 +178,9 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "global_batch": 1, "images_per_step": 1},
+        # our arm's workload; each timed step is a bounded sample of it
+        "config": {"workload": WORKLOAD, "global_batch": 128, "batch_per_gpu": 128,
+                   "parallelism": "single", "sampled_images_per_step": 1},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
