@@ -726,7 +726,7 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     ALX_TRY(run_gemm(h, P->fd[f], P->fc_flops[f], s), "fc dgrad launch");
     launch_dgrad_finalize(h->scratch, P->fd[f].args.splits, B, F.In, mask[f], dxo[f], s);
     if (h->fc_fused) {
-      // HBM-bound (the update moves 20 bytes per weight against 256 MMA
+      // HBM-bound (the update moves 18 bytes per weight against 256 MMA
       // FLOPs): launched outside the per-GEMM tensor-roofline records
       ALX_TRY(launch_any(P->fws[f], s), "fc wgrad + update launch");
     } else {
