@@ -121,6 +121,8 @@ def lib():
             "oracle_forward": (None, [netp, dp, dp, c_int, c_int, c_uint64, c_uint32, dp, dp]),
             "oracle_forward_probe": (None, [netp, dp, dp, c_int, c_int, c_uint64, c_uint32, c_int,
                                             dp]),
+            "oracle_forward_trace": (None, [netp, dp, dp, c_int, c_int, c_uint64, c_uint32, c_int,
+                                            ip, POINTER(dp)]),
             "oracle_train_step": (c_double, [netp, dp, dp, dp, i32p, c_int, c_double, c_double,
                                              c_double, c_uint64, c_uint32, dp, dp]),
             "oracle_loss": (c_double, [netp, dp, dp, i32p, c_int, c_uint64, c_uint32]),
@@ -436,6 +438,34 @@ def forward_probe(net, params, x, which, mode=1, seed=0, step=0):
     lib().oracle_forward_probe(ctypes.byref(net), pp, xp, B, mode, seed, step, which,
                                _p(out, c_double))
     return out
+
+
+# forward_trace codes beyond forward_probe's: pre-activations (before the ReLU)
+TRACE_PRE, TRACE_FC_PRE = 100, 105
+
+
+def trace_size(net, which):
+    """Elements per image of the map forward_trace returns for `which`."""
+    if which < 100:
+        return probe_size(net, which)
+    if which in (105, 106):
+        return net.fc_n[which - 105]
+    return map_sizes(net)[which - 100][1] ** 2 * net.conv_c[which - 100]
+
+
+def forward_trace(net, params, x, which, mode=1, seed=0, step=0):
+    """Several maps of ONE forward pass (codes of forward_probe, plus the
+    pre-activations TRACE_PRE + l and TRACE_FC_PRE + f), as {code: flat array}."""
+    params, pp = _d(params)
+    x, xp = _d(x)
+    B = x.shape[0]
+    which = [int(w) for w in which]
+    outs = [np.zeros(B * trace_size(net, w)) for w in which]
+    arr = (POINTER(c_double) * len(which))(*[_p(o, c_double) for o in outs])
+    wv = (c_int * len(which))(*which)
+    lib().oracle_forward_trace(ctypes.byref(net), pp, xp, B, mode, seed, step, len(which), wv,
+                               arr)
+    return dict(zip(which, outs))
 
 
 def train_step(net, params, velocity, x, labels, lr=0.01, momentum=0.9, wd=5e-4, seed=0,

@@ -611,6 +611,8 @@ typedef struct {
   uint8_t* keep[2];
   double* logits;
   const uint8_t* relu_given[7];  /* optional ReLU decisions: conv1..5, FC6, FC7 */
+  int keep_pre;                  /* store the pre-activations below */
+  double* pre[7];                /* conv1..5, FC6, FC7 before the ReLU (keep_pre only) */
 } fwd_cache;
 
 static double* dalloc(int64_t n) { return (double*)calloc((size_t)(n > 0 ? n : 1), sizeof(double)); }
@@ -628,6 +630,7 @@ static void cache_free(fwd_cache* c) {
     free(c->fc_out[f]);
     free(c->keep[f]);
   }
+  for (int i = 0; i < 7; ++i) free(c->pre[i]);
   free(c->logits);
 }
 
@@ -639,6 +642,7 @@ static void net_forward_given(const oracle_net* net, const double* params, const
 
 static void net_forward(const oracle_net* net, const double* params, const double* x, int B,
                         int mode, uint64_t seed, uint32_t step, fwd_cache* c) {
+  c->keep_pre = 0;
   net_forward_given(net, params, x, B, mode, seed, step, NULL, NULL, c);
 }
 
@@ -669,7 +673,9 @@ static void net_forward_given(const oracle_net* net, const double* params, const
                               int B, int mode, uint64_t seed, uint32_t step,
                               const uint8_t* const* am_in, const uint8_t* const* relu_in,
                               fwd_cache* c) {
+  const int keep_pre = c->keep_pre;
   memset(c, 0, sizeof(*c));
+  c->keep_pre = keep_pre;
   for (int i = 0; i < 7; ++i) c->relu_given[i] = relu_in ? relu_in[i] : NULL;
   net_shapes(net, &c->s);
   const oracle_shapes* s = &c->s;
@@ -683,6 +689,10 @@ static void net_forward_given(const oracle_net* net, const double* params, const
     oracle_conv_fwd(in, B, H, H, C, params + s->w_off[l], params + s->b_off[l], Co,
                     net->conv_k[l], net->conv_s[l], net->conv_p[l], net->conv_g[l],
                     c->relu_out[l]);
+    if (c->keep_pre) {
+      c->pre[l] = dalloc(n);
+      memcpy(c->pre[l], c->relu_out[l], sizeof(double) * (size_t)n);
+    }
     relu_decided(c->relu_out[l], n, c->relu_given[l]);
     const double* cur = c->relu_out[l];
     if (net->lrn_after[l]) {
@@ -723,6 +733,10 @@ static void net_forward_given(const oracle_net* net, const double* params, const
     double* z = dalloc((int64_t)B * Out);
     oracle_fc_fwd(c->fc_in[f], B, In, params + s->w_off[5 + f], params + s->b_off[5 + f], Out, z);
     if (f < 2) {
+      if (c->keep_pre) {
+        c->pre[5 + f] = dalloc((int64_t)B * Out);
+        memcpy(c->pre[5 + f], z, sizeof(double) * (size_t)B * Out);
+      }
       relu_decided(z, (int64_t)B * Out, c->relu_given[5 + f]);
       c->fc_relu[f] = z;
       double* d = dalloc((int64_t)B * Out);
@@ -759,31 +773,65 @@ ORACLE_API void oracle_forward(const oracle_net* net, const double* params, cons
  *   0..4  relu output of conv l      10..14 LRN output of conv l
  *   20..24 pooled map after conv l   30, 31 FC6/FC7 output after dropout
  *   40 logits */
+/* Copy map `which` (codes of oracle_forward_probe) out of a forward cache. */
+static void oracle_forward_probe_from(const oracle_net* net, const fwd_cache* c, int B, int which,
+                                      double* out) {
+  const oracle_shapes* s = &c->s;
+  const double* src = NULL;
+  int64_t n = 0;
+  if (which >= 0 && which < 5) {
+    src = c->relu_out[which];
+    n = (int64_t)B * s->conv_out[which] * s->conv_out[which] * net->conv_c[which];
+  } else if (which >= 10 && which < 15) {
+    src = c->lrn_out[which - 10];
+    n = (int64_t)B * s->conv_out[which - 10] * s->conv_out[which - 10] * net->conv_c[which - 10];
+  } else if (which >= 20 && which < 25) {
+    src = c->pool_out[which - 20];
+    n = (int64_t)B * s->pool_out[which - 20] * s->pool_out[which - 20] * net->conv_c[which - 20];
+  } else if (which == 30 || which == 31) {
+    src = c->fc_out[which - 30];
+    n = (int64_t)B * net->fc_n[which - 30];
+  } else if (which == 40) {
+    src = c->logits;
+    n = (int64_t)B * net->fc_n[2];
+  }
+  if (src) memcpy(out, src, sizeof(double) * (size_t)n);
+}
+
 ORACLE_API void oracle_forward_probe(const oracle_net* net, const double* params,
                                      const double* x, int B, int mode, uint64_t seed,
                                      uint32_t step, int which, double* out) {
   fwd_cache c;
   net_forward(net, params, x, B, mode, seed, step, &c);
+  oracle_forward_probe_from(net, &c, B, which, out);
+  cache_free(&c);
+}
+
+/* Several intermediate maps of one forward pass, each copied to its own
+ * output (which[i] -> out[i]):
+ *   0..4, 10..14, 20..24, 30, 31, 40  as oracle_forward_probe;
+ *   100+l  pre-activation of conv l (before the ReLU); 105, 106 FC6, FC7.
+ * One pass instead of one per map: at the benchmark's batch a forward of
+ * this oracle takes tens of seconds. */
+ORACLE_API void oracle_forward_trace(const oracle_net* net, const double* params, const double* x,
+                                     int B, int mode, uint64_t seed, uint32_t step, int n,
+                                     const int* which, double* const* out) {
+  fwd_cache c;
+  c.keep_pre = 1;
+  net_forward_given(net, params, x, B, mode, seed, step, NULL, NULL, &c);
   const oracle_shapes* s = &c.s;
-  const double* src = NULL;
-  int64_t n = 0;
-  if (which >= 0 && which < 5) {
-    src = c.relu_out[which];
-    n = (int64_t)B * s->conv_out[which] * s->conv_out[which] * net->conv_c[which];
-  } else if (which >= 10 && which < 15) {
-    src = c.lrn_out[which - 10];
-    n = (int64_t)B * s->conv_out[which - 10] * s->conv_out[which - 10] * net->conv_c[which - 10];
-  } else if (which >= 20 && which < 25) {
-    src = c.pool_out[which - 20];
-    n = (int64_t)B * s->pool_out[which - 20] * s->pool_out[which - 20] * net->conv_c[which - 20];
-  } else if (which == 30 || which == 31) {
-    src = c.fc_out[which - 30];
-    n = (int64_t)B * net->fc_n[which - 30];
-  } else if (which == 40) {
-    src = c.logits;
-    n = (int64_t)B * net->fc_n[2];
+  for (int i = 0; i < n; ++i) {
+    const int w = which[i];
+    if (w < 100) {
+      oracle_forward_probe_from(net, &c, B, w, out[i]);
+    } else if (w >= 100 && w < 105) {
+      const int l = w - 100;
+      memcpy(out[i], c.pre[l],
+             sizeof(double) * (size_t)B * s->conv_out[l] * s->conv_out[l] * net->conv_c[l]);
+    } else if (w == 105 || w == 106) {
+      memcpy(out[i], c.pre[w - 100], sizeof(double) * (size_t)B * net->fc_n[w - 105]);
+    }
   }
-  if (src) memcpy(out, src, sizeof(double) * (size_t)n);
   cache_free(&c);
 }
 
@@ -852,6 +900,7 @@ static double train_step_probe(const oracle_net* net, double* params, double* ve
                                double* grads, double* logits, int probe, double* probe_out,
                                const uint8_t* const* am_in, const uint8_t* const* relu_in) {
   fwd_cache c;
+  c.keep_pre = 0;
   net_forward_given(net, params, x, B, 0, seed, step, am_in, relu_in, &c);
   const oracle_shapes* s = &c.s;
   const int N = net->fc_n[2];
