@@ -14,9 +14,21 @@
 // stand-in, not a device address), so the device address is looked up with
 // cudaGetSymbolAddress once per device, with that device current, the first
 // time the entry point runs on it.  That first call should therefore come
-// before any stream capture.  All calls share the one array: two calls whose
-// work overlaps on the GPU (different streams, or different host threads)
-// race on it and must be ordered by the caller.
+// before any stream capture.  The cached address belongs to the device's
+// context at that time: after cudaDeviceReset (or any other teardown of the
+// primary context) it is stale, so the cache is keyed by the context and
+// looked up again when the context changes.  All calls share the one array:
+// two calls whose work overlaps on the GPU (different streams, or different
+// host threads) race on it and must be ordered by the caller.
+//
+// The array's first 256 bytes hold the status word of the pipelined GEMM's
+// bounded waits.  The call clears it, launches, and reads it back before it
+// returns, so a wait that ran out is reported as ALEXNET_ERR_TIMEOUT instead
+// of a silently wrong gradient; the call therefore returns only once its
+// result is in dw.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cstring>
 #include <mutex>
 
@@ -38,17 +50,38 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
+
+// The calling thread's current context (null if none yet), through the
+// driver entry point the runtime hands out (the library links no libcuda).
+CUcontext current_ctx() {
+  static PFN_cuCtxGetCurrent_v4000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+  }();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
 
 // Device address of the scratch array on the current device (set-up on the
-// first call per device).
+// first call per device, and again whenever the device's context is a
+// different one than at the last look-up).
 void* noalloc_scratch() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  const CUcontext ctx = current_ctx();
+  if (!g_noalloc_ptr[dev] || !ctx || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
+    // (initialises the device's primary context if nothing has yet)
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = current_ctx();
   }
   return g_noalloc_ptr[dev];
 }
@@ -116,5 +149,12 @@ extern "C" alexnet_status alexnet_op_conv_wgrad_noalloc(const void* x, int B, in
   const int grid = static_cast<int>((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
   k_wgrad_sum<<<grid, 256, 0, s>>>(part, d.args.splits, Cout, K, cs.Cg, cs.P(), groups, dw);
   count_launch();
-  return cudaGetLastError() == cudaSuccess ? ALEXNET_OK : ALEXNET_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return ALEXNET_ERR_CUDA;
+  // the GEMM's status word: a bounded wait that ran out leaves dw invalid
+  int st = 0;
+  if (cudaMemcpyAsync(&st, status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ALEXNET_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ALEXNET_ERR_CUDA;
+  if (st & STATUS_TIMEOUT) return ALEXNET_ERR_TIMEOUT;
+  return ALEXNET_OK;
 }

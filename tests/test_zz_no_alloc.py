@@ -37,7 +37,11 @@ def test_noalloc_weight_gradient_matches_scratch_version(order):
     ws = workspace(512)
     shapes = [(13, 384, 256, 3, 1, 2, 4, 0, 11),   # conv5 shape
               (27, 96, 256, 5, 2, 2, 2, 0, 12),    # conv2 shape
-              (13, 384, 256, 3, 1, 2, 4, 3, 13)]   # conv5 again, new data, 3 splits
+              (13, 384, 256, 3, 1, 2, 4, 3, 13),   # conv5 again, new data, 3 splits
+              # conv2 shape asking for 16 K-slices: 23 K blocks, but only 10
+              # slices of partial sums fit in the array, so the call lowers
+              # the count and the summing kernel sees the lowered one
+              (27, 96, 256, 5, 2, 2, 2, 16, 14)]
     if order:
         shapes = shapes[::-1]
     for (H, Cin, Cout, K, pad, groups, B, splits, seed) in shapes:
@@ -52,6 +56,29 @@ def test_noalloc_weight_gradient_matches_scratch_version(order):
         st = _call_noalloc(ax.lib, xt, B, H, Cin, dyt, Cout, K, pad, groups, splits, got)
         assert st == ax.OK
         assert rel_l2(host(got), host(want)) < TOL_F32_ACC
+
+
+def test_noalloc_weight_gradient_matches_oracle():
+    """The allocation-free call runs the im2col GEMM, which the scratch-taking
+    call may not: one small grouped shape against the oracle's fp64 weight
+    gradient, within the fp32-accumulation bound of the other weight-gradient
+    tests (two calls, so the second one finds the first one's leftovers)."""
+    import torch
+    import oracle
+    from deep_cnn_image_b200 import alexnet as ax
+    H, Cin, Cout, K, pad, groups, B = 13, 128, 64, 3, 1, 2, 3
+    for seed in (21, 22):
+        r = np.random.default_rng(seed)
+        x = bf16_round(np.maximum(r.standard_normal((B, H, H, Cin)), 0.0))
+        dy = bf16_round(r.standard_normal((B, H, H, Cout)))
+        got = torch.full((Cout, K, K, Cin // groups), float("nan"), dtype=torch.float32,
+                         device="cuda")
+        st = _call_noalloc(ax.lib, dev(x, "bf16"), B, H, Cin, dev(dy, "bf16"), Cout, K, pad,
+                           groups, 0, got)
+        assert st == ax.OK
+        _, want, _ = oracle.conv_bwd(x, np.zeros((Cout, K, K, Cin // groups)), dy, 1, pad, groups,
+                                     need_dx=False)
+        assert rel_l2(host(got), want) < TOL_F32_ACC
 
 
 def test_noalloc_rejects_sizes_beyond_the_array():
