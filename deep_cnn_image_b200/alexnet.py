@@ -63,6 +63,11 @@ def _load():
         "alexnet_knn": (st, [vp, i, vp, i, i, i, vp, vp, vp, vp, sz, vp]),
         "alexnet_knn_sqnorms": (st, [vp, i, i, vp, vp]),
         "alexnet_ensemble_forward": (st, [vp, i, vp, i, vp, vp, vp, sz, vp]),
+        "alexnet_train_grads": (st, [vp, vp, vp, i, c_int64, vp, vp]),
+        "alexnet_stream_wait_fc_grads": (st, [vp, vp]),
+        "alexnet_sgd_range": (st, [vp, c_int64, c_int64, vp, c_float, c_float, vp]),
+        "alexnet_params_updated": (st, [vp, vp]),
+        "alexnet_device_buffer": (st, [vp, i, POINTER(vp), POINTER(c_int64)]),
         "alexnet_params_bytes": (sz, [vp]),
         "alexnet_get_params": (st, [vp, vp, sz, vp]),
         "alexnet_set_params": (st, [vp, vp, sz, vp]),
@@ -95,6 +100,7 @@ def _load():
         "alexnet_debug_copy": (st, [vp, i, vp, sz, vp]),
         "alexnet_debug_keep": (st, [vp, i]),
         "alexnet_debug_fc_update": (st, [vp, i]),
+        "alexnet_debug_canaries": (st, [vp, POINTER(c_int64)]),
         "alexnet_conv_algo": (st, [vp, i, i, i, POINTER(c_int)]),
         "alexnet_stats_enable": (st, [vp, i]),
         "alexnet_stats_read": (st, [vp, POINTER(Stats)]),
@@ -192,6 +198,31 @@ class AlexNet:
         return check(lib.alexnet_tencrop(self.h, _ptr(src), B, _ptr(mean), _ptr(probs_avg),
                                          _ptr(top5), _stream(stream)), self.h)
 
+    # -- data-parallel step (see alexnet.h) ------------------------------
+    def train_grads(self, x, labels, B, image_offset, loss=None, stream=None):
+        return check(lib.alexnet_train_grads(self.h, _ptr(x), _ptr(labels), B, image_offset,
+                                             _ptr(loss), _stream(stream)), self.h)
+
+    def stream_wait_fc_grads(self, stream):
+        return check(lib.alexnet_stream_wait_fc_grads(self.h, _stream(stream)), self.h)
+
+    def sgd_range(self, offset, count, gsum, grad_scale, lr, stream=None):
+        return check(lib.alexnet_sgd_range(self.h, offset, count, _ptr(gsum), grad_scale, lr,
+                                           _stream(stream)), self.h)
+
+    def params_updated(self, stream=None):
+        return check(lib.alexnet_params_updated(self.h, _stream(stream)), self.h)
+
+    def device_buffer(self, which):
+        """The handle's fp32 parameters (0), momentum (1) or gradients (2) as
+        a torch view of the workspace (blob order)."""
+        import torch
+        p = c_void_p()
+        n = c_int64()
+        check(lib.alexnet_device_buffer(self.h, which, byref(p), byref(n)), self.h)
+        off = p.value - self.workspace.data_ptr()
+        return self.workspace[off:off + 4 * n.value].view(torch.float32)
+
     def params_bytes(self):
         return lib.alexnet_params_bytes(self.h)
 
@@ -234,6 +265,13 @@ class AlexNet:
         """FC weights updated by the weight-gradient GEMM's epilogue (True,
         the default) or by a separate kernel (False); identical results."""
         return check(lib.alexnet_debug_fc_update(self.h, 1 if fused else 0))
+
+    def debug_canaries(self):
+        """Bytes changed in the guard regions after the workspace's buffers
+        (0 unless some kernel wrote past the end of a buffer); synchronises."""
+        v = c_int64(-1)
+        check(lib.alexnet_debug_canaries(self.h, byref(v)), self.h)
+        return v.value
 
     def debug_copy(self, which, dst, stream=None):
         return check(lib.alexnet_debug_copy(self.h, which, _ptr(dst), dst.numel() * dst.element_size(),

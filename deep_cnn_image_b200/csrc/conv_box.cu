@@ -206,12 +206,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t bst = b_lo0 + sb * (b_stage >> 4);
+            // a last chunk of 48 real channels (conv1's space-to-depth input,
+            // conv2's 48 channels per group) skips the K step of zeros
+            const bool k3 = !BMN && ch == a.cpt - 1 && a.k16_last == 3;
             for (int j = 0; j < n; ++j) {
               const uint32_t acc0 = (ch == 0 && tap0 + j == 0) ? 0u : 1u;
 #pragma unroll
-              for (int sub = 0; sub < NSUB; ++sub)
-                tc_mma_k4<2, BMN ? 128 : 2>(dbase + sub * BN, abox + shift + sub * (128 * 128 / 16),
-                                            a_hi, bst + j * (B_BYTES >> 4), b_hi, IDESC, acc0);
+              for (int sub = 0; sub < NSUB; ++sub) {
+                if (k3)
+                  tc_mma_k3<2, 2>(dbase + sub * BN, abox + shift + sub * (128 * 128 / 16), a_hi,
+                                  bst + j * (B_BYTES >> 4), b_hi, IDESC, acc0);
+                else
+                  tc_mma_k4<2, BMN ? 128 : 2>(dbase + sub * BN,
+                                              abox + shift + sub * (128 * 128 / 16), a_hi,
+                                              bst + j * (B_BYTES >> 4), b_hi, IDESC, acc0);
+              }
               if (++kw == a.K) {
                 kw = 0;
                 shift += row_adv;
@@ -664,6 +673,12 @@ static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, in
   if (a.Hb > 256) return false;
   a.tiles_img = (a.Ho + a.To_h - 1) / a.To_h;
   a.cpt = cs.P() / 64;
+  {
+    // K steps of 16 channels of the last chunk that can hold real channels;
+    // only 3 (48 channels) is used to skip work, other counts run all 4
+    const int real = cs.Cg - 64 * (a.cpt - 1);
+    a.k16_last = (real + 15) / 16 == 3 ? 3 : 4;
+  }
   a.cg_off = cs.Cg;
   a.groups = cs.groups;
   a.Og = cs.Og;

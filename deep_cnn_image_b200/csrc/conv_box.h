@@ -33,6 +33,7 @@ struct BoxArgs {
   int Hb;          // input rows per box
   int tiles_img;   // ceil(Ho / To_h)
   int cpt;         // 64-channel chunks per tap
+  int k16_last;    // 16-channel K steps of the last chunk that hold real channels (forward)
   int cg_off;      // input channel offset of group g: g * cg_off
   int groups;
   int Og;          // output channels per group

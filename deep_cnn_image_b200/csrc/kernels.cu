@@ -514,177 +514,179 @@ __global__ void __launch_bounds__(256) k_lrn_pool_fwd(const bf16* __restrict__ a
   }
 }
 
-// Gradient arriving at input pixel (ih, iw), channels c .. c+7, through the
-// stride-2 max-pool: the sum, in ascending window order, of the pooled
-// gradients of the windows whose recorded choice is this pixel.  A pixel
-// lies in at most two windows per axis, (i >> 1) - 1 and i >> 1; all four
-// candidates are loaded at once.
-__device__ __forceinline__ void pool_grad8(const bf16* __restrict__ dy,
-                                           const uint8_t* __restrict__ am, int b, int ih, int iw,
-                                           int c, int C, int Ho, int Wo, int z, float (&g)[8]) {
-  uint4 gv[4];
-  uint2 av[4];
-  const int oh_a = (ih >> 1) - 1, ow_a = (iw >> 1) - 1;
-  const uint32_t base = static_cast<uint32_t>((b * Ho + oh_a) * Wo + ow_a) * C + c;
+// The channels of one pooled-gradient vector (8 bf16 in dyv) whose recorded
+// window offset (one byte each in amv) equals `off`, added to g in fp32.
+// The offset test works on all eight bytes at once: xor with the offset
+// replicated into every byte, a carry-free per-byte non-zero test
+// ((b & 0x7f) + 0x7f <= 0xfe, so no carry crosses a byte), then
+// sign-replicating byte permutes widen each byte's flag to its channel's 16
+// bits; the gradient is kept where the flag is clear.
+__device__ __forceinline__ void add_routed8(const uint4& dyv, const uint2& amv, uint32_t off,
+                                            float (&g)[8]) {
+  const uint32_t rep = off * 0x01010101u;
+  const uint32_t x0 = amv.x ^ rep, x1 = amv.y ^ rep;
+  const uint32_t n0 = ((x0 & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x0;
+  const uint32_t n1 = ((x1 & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x1;
+  const uint4 kept = make_uint4(dyv.x & ~prmt(n0, 0, 0x9988), dyv.y & ~prmt(n0, 0, 0xBBAA),
+                                dyv.z & ~prmt(n1, 0, 0x9988), dyv.w & ~prmt(n1, 0, 0xBBAA));
+  float f[8];
+  unpack8_bits(kept, f);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int oh = oh_a + (q >> 1);
-    const int ow = ow_a + (q & 1);
-    const bool ok =
-        oh >= 0 && oh < Ho && ow >= 0 && ow < Wo && ih - 2 * oh < z && iw - 2 * ow < z;
-    gv[q] = make_uint4(0, 0, 0, 0);
-    av[q] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);  // no window offset is 255
-    if (ok) {
-      const uint32_t o = base + static_cast<uint32_t>(((q >> 1) * Wo + (q & 1)) * C);
-      gv[q] = *reinterpret_cast<const uint4*>(dy + o);
-      av[q] = *reinterpret_cast<const uint2*>(am + o);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) g[i] = 0.f;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int oh = oh_a + (q >> 1);
-    const int ow = ow_a + (q & 1);
-    const uint32_t rep = static_cast<uint32_t>((ih - 2 * oh) * z + (iw - 2 * ow)) * 0x01010101u;
-    // bytes of x that differ from this pixel's offset get their top bit set
-    // (no carry crosses a byte: (b & 0x7f) + 0x7f <= 0xfe)
-    const uint32_t x0 = av[q].x ^ rep, x1 = av[q].y ^ rep;
-    const uint32_t n0 = ((x0 & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x0;
-    const uint32_t n1 = ((x1 & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x1;
-    // sign-replicating byte permutes widen each byte's flag to its channel's
-    // 16 bits; the pooled gradient is kept where the flag is clear
-    const uint4 m = make_uint4(prmt(n0, 0, 0x9988), prmt(n0, 0, 0xBBAA), prmt(n1, 0, 0x9988),
-                               prmt(n1, 0, 0xBBAA));
-    const uint4 kept = make_uint4(gv[q].x & ~m.x, gv[q].y & ~m.y, gv[q].z & ~m.z, gv[q].w & ~m.w);
-    float f[8];
-    unpack8_bits(kept, f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) g[i] += f[i];
-  }
+  for (int i = 0; i < 8; ++i) g[i] += f[i];
 }
 
 // Backward of normalisation + pooling, fused: the pooled gradient is routed
 // to the chosen pixels and pushed through the normalisation (and the ReLU
 // below it, by the stored conv output a > 0) in one pass; `dl` (the
-// normalised map's gradient) is written only when given.  A block owns
-// `np` whole pixels (all C channels, one 8-channel unit per thread), so the
-// channel window never leaves the block: a and the cross terms
-// t_i = g_i a_i s_i^(-beta-1) go through shared memory.  Arithmetic as
-// k_lrn_bwd.
+// normalised map's gradient) is written only when given.
+//
+// A thread owns a 2 x 2 quad of pixels (rows 2qi, 2qi + 1, columns 2qj,
+// 2qj + 1) and one 8-channel unit.  With stride 2 the windows that can
+// route gradient into the quad are (qi - 1 + wr, qj - 1 + wc), wr, wc in
+// {0, 1} (only (qi, qj) for z = 2), and the pixel at (h, d) of the quad sits
+// at offset (h + 2 - 2 wr, d + 2 - 2 wc) of window (wr, wc): the four windows
+// are loaded once for four pixels, and which pixel may take which window is
+// known at compile time.  Gradients are summed in ascending (row-major)
+// window order.  The normalisation's channel window reaches two channels
+// into the neighbouring units; those edge values (a, then the cross terms
+// t_i = g_i a_i s_i^(-beta-1)) go through shared memory, one quad row at a
+// time.  Arithmetic of the normalisation as k_lrn_bwd.  Per block the
+// column sums of the stored da (the layer's bias gradient) are written to
+// bias_part[blockIdx.x][C] (nullable).
 template <int ZC, int WC, bool B34>
 __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ dy,
                                                       const uint8_t* __restrict__ am,
                                                       const bf16* __restrict__ a,
                                                       bf16* __restrict__ dl,
-                                                      bf16* __restrict__ da, int npix,
-                                                      int np, int H_, int W_, int C, int z_,
+                                                      bf16* __restrict__ da, int nquads,
+                                                      int nq, int H_, int W_, int C, int z_,
                                                       float k, float alpha, float beta,
                                                       float* __restrict__ bias_part) {
   // ZC / WC != 0: window and (square) map size known at compile time
   const int H = WC ? WC : H_, W = WC ? WC : W_, z = ZC ? ZC : z_;
-  // a_s[p][4 + c] and t_s[p][4 + c], four zeros at each end of a row; every
-  // access is a 16-byte vector (a unit touches channels c0-4 .. c0+11)
-  extern __shared__ float4 fsm4[];
-  const int ld4 = (C + 8) >> 2;  // row length in float4
-  float4* a_s = fsm4;
-  float4* t_s = fsm4 + np * ld4;
   const int Ho = (H - z) / 2 + 1, Wo = (W - z) / 2 + 1;
+  const int QH = (H + 1) >> 1, QW = (W + 1) >> 1;
   const int CH = C >> 3;
   const int up = threadIdx.x / CH;
   const int uj = threadIdx.x - up * CH;
-  const bool mine = up < np;
-  // this thread's share of the bias gradient (sum of the stored da values of
-  // its channels over the pixels it handles)
+  const bool mine = up < nq;
+  const int tid = threadIdx.x;
+  // edge values of every thread's unit (channels 0, 1, 6, 7), per quad
+  // column: normalisation inputs (ea) and cross terms (et)
+  __shared__ float4 ea[2][256], et[2][256];
+  __shared__ float red[256 * 8];
+  const float c2ab = 2.f * alpha * beta;
   float bsum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int blk = blockIdx.x; blk * np < npix; blk += gridDim.x) {
-    const int pix = blk * np + up;
-    const bool live = mine && pix < npix;
-    float g[8], av[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) g[i] = av[i] = 0.f;
+  for (int blk = blockIdx.x; blk * nq < nquads; blk += gridDim.x) {
+    const int q = blk * nq + up;
+    const bool live = mine && q < nquads;
+    int b = 0, qi = 0, qj = 0;
     if (live) {
-      const int q = pix / W;
-      const int iw = pix - q * W;
-      const int b = q / H;
-      const int ih = q - b * H;
-      unpack8(*reinterpret_cast<const uint4*>(a + static_cast<size_t>(pix) * C + uj * 8), av);
-      pool_grad8(dy, am, b, ih, iw, uj * 8, C, Ho, Wo, z, g);
+      qj = q % QW;
+      const int r = q / QW;
+      qi = r % QH;
+      b = r / QH;
     }
-    if (mine) {
-      float4* ar = a_s + up * ld4 + 1 + uj * 2;
-      ar[0] = make_float4(av[0], av[1], av[2], av[3]);
-      ar[1] = make_float4(av[4], av[5], av[6], av[7]);
-      if (uj == 0) ar[-1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (uj == CH - 1) ar[2] = make_float4(0.f, 0.f, 0.f, 0.f);
+    uint4 wdy[4];
+    uint2 wam[4];
+    bool wok[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int oh = qi - 1 + (w >> 1), ow = qj - 1 + (w & 1);
+      wok[w] = live && oh >= 0 && oh < Ho && ow >= 0 && ow < Wo && (z == 3 || w == 3);
+      wdy[w] = make_uint4(0, 0, 0, 0);
+      wam[w] = make_uint2(0, 0);
+      if (wok[w]) {
+        const uint32_t o = static_cast<uint32_t>((b * Ho + oh) * Wo + ow) * C + uj * 8;
+        wdy[w] = *reinterpret_cast<const uint4*>(dy + o);
+        wam[w] = *reinterpret_cast<const uint2*>(am + o);
+      }
     }
-    __syncthreads();
-    float first[8];
-    if (mine) {
-      const float4* ar = a_s + up * ld4 + uj * 2;  // channels c0-4 .. c0+11
-      float w[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 x = ar[q];
-        w[4 * q] = x.x;
-        w[4 * q + 1] = x.y;
-        w[4 * q + 2] = x.z;
-        w[4 * q + 3] = x.w;
+    for (int h = 0; h < 2; ++h) {
+      const int ih = 2 * qi + h;
+      float g[2][8], av[2][8];
+      bool pv[2];
+#pragma unroll
+      for (int d = 0; d < 2; ++d) {
+        const int iw = 2 * qj + d;
+        pv[d] = live && ih < H && iw < W;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g[d][i] = av[d][i] = 0.f;
+        if (pv[d]) {
+          unpack8(*reinterpret_cast<const uint4*>(
+                      a + static_cast<uint32_t>((b * H + ih) * W + iw) * C + uj * 8),
+                  av[d]);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int rr = h + 2 - 2 * (w >> 1), rc = d + 2 - 2 * (w & 1);
+            if (wok[w] && rr < z && rc < z)
+              add_routed8(wdy[w], wam[w], static_cast<uint32_t>(rr * z + rc), g[d]);
+          }
+        }
+        ea[d][tid] = make_float4(av[d][0], av[d][1], av[d][6], av[d][7]);
       }
-      float tv[8];
+      __syncthreads();
+      float first[2][8], tv[2][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float sum = 0.f;
+      for (int d = 0; d < 2; ++d) {
+        const float4 L = mine && uj > 0 ? ea[d][tid - 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 R = mine && uj < CH - 1 ? ea[d][tid + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+        float w12[12];
+        w12[0] = L.z;
+        w12[1] = L.w;
 #pragma unroll
-        for (int q = 2; q <= 6; ++q) sum += w[i + q] * w[i + q];
-        const float sc = k + alpha * sum;
-        float sb, sb1;
-        lrn_pow2<B34>(sc, beta, sb, sb1);
-        first[i] = g[i] * sb;
-        tv[i] = g[i] * av[i] * sb1;
+        for (int i = 0; i < 8; ++i) w12[2 + i] = av[d][i];
+        w12[10] = R.x;
+        w12[11] = R.y;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < 5; ++j) sum += w12[i + j] * w12[i + j];
+          const float sc = k + alpha * sum;
+          float sb, sb1;
+          lrn_pow2<B34>(sc, beta, sb, sb1);
+          first[d][i] = g[d][i] * sb;
+          tv[d][i] = g[d][i] * av[d][i] * sb1;
+        }
+        et[d][tid] = make_float4(tv[d][0], tv[d][1], tv[d][6], tv[d][7]);
       }
-      float4* tr = t_s + up * ld4 + 1 + uj * 2;
-      tr[0] = make_float4(tv[0], tv[1], tv[2], tv[3]);
-      tr[1] = make_float4(tv[4], tv[5], tv[6], tv[7]);
-      if (uj == 0) tr[-1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (uj == CH - 1) tr[2] = make_float4(0.f, 0.f, 0.f, 0.f);
+      __syncthreads();
+#pragma unroll
+      for (int d = 0; d < 2; ++d) {
+        const float4 L = mine && uj > 0 ? et[d][tid - 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 R = mine && uj < CH - 1 ? et[d][tid + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (!pv[d]) continue;
+        float w12[12];
+        w12[0] = L.z;
+        w12[1] = L.w;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w12[2 + i] = tv[d][i];
+        w12[10] = R.x;
+        w12[11] = R.y;
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float cross = 0.f;
+#pragma unroll
+          for (int j = 0; j < 5; ++j) cross += w12[i + j];
+          const float aj = av[d][i];
+          o[i] = aj > 0.f ? first[d][i] - c2ab * aj * cross : 0.f;
+        }
+        const uint4 packed = pack8(o);
+        const uint32_t e = static_cast<uint32_t>((b * H + ih) * W + 2 * qj + d) * C + uj * 8;
+        *reinterpret_cast<uint4*>(da + e) = packed;
+        if (dl) *reinterpret_cast<uint4*>(dl + e) = pack8(g[d]);
+        float r[8];
+        unpack8(packed, r);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bsum[i] += r[i];
+      }
     }
-    __syncthreads();
-    if (live) {
-      const float4* tr = t_s + up * ld4 + uj * 2;  // channels c0-4 .. c0+11
-      float w[16];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 x = tr[q];
-        w[4 * q] = x.x;
-        w[4 * q + 1] = x.y;
-        w[4 * q + 2] = x.z;
-        w[4 * q + 3] = x.w;
-      }
-      float o[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float cross = 0.f;
-#pragma unroll
-        for (int q = 2; q <= 6; ++q) cross += w[i + q];
-        const float aj = av[i];
-        const float d = first[i] - 2.f * alpha * beta * aj * cross;
-        o[i] = aj > 0.f ? d : 0.f;
-      }
-      const uint4 packed = pack8(o);
-      const size_t e = static_cast<size_t>(pix) * C + uj * 8;
-      *reinterpret_cast<uint4*>(da + e) = packed;
-      if (dl) *reinterpret_cast<uint4*>(dl + e) = pack8(g);
-      float r[8];
-      unpack8(packed, r);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) bsum[i] += r[i];
-    }
-    __syncthreads();  // the next group reuses a_s / t_s
   }
   if (!bias_part) return;
-  // per-channel sum over the block's pixel lanes, in lane order
-  float* red = reinterpret_cast<float*>(fsm4);
+  // per-channel sum over the block's quad slots, in slot order
   if (mine) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) red[up * C + uj * 8 + i] = bsum[i];
@@ -692,7 +694,7 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
   __syncthreads();
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
     float v = 0.f;
-    for (int q = 0; q < np; ++q) v += red[q * C + c];
+    for (int q = 0; q < nq; ++q) v += red[q * C + c];
     bias_part[static_cast<size_t>(blockIdx.x) * C + c] = v;
   }
 }
@@ -765,7 +767,7 @@ __global__ void k_fc_finalize(const float* __restrict__ part, int S, int rows, i
       for (int i = 0; i < 4; ++i) v[i] = v[i] > 0.f ? v[i] : 0.f;
     }
     if (dropout_mode == 1) {
-      const U4 w = dropout_words(hp, q, layer);
+      const U4 w = dropout_words(hp, q + static_cast<long long>(hp.row_offset) * (cols / 4), layer);
 #pragma unroll
       for (int i = 0; i < 4; ++i) v[i] = u4_word(w, i) >= hp.drop_thresh ? v[i] : 0.f;
     } else if (dropout_mode == 2) {
@@ -791,7 +793,7 @@ __global__ void k_dropout_mask(const HParams* __restrict__ hpp, int layer, int r
   const long long n4 = 1LL * rows * cols / 4;
   for (long long q = blockIdx.x * 1LL * blockDim.x + threadIdx.x; q < n4;
        q += 1LL * gridDim.x * blockDim.x) {
-    const U4 w = dropout_words(hp, q, layer);
+    const U4 w = dropout_words(hp, q + static_cast<long long>(hp.row_offset) * (cols / 4), layer);
 #pragma unroll
     for (int i = 0; i < 4; ++i) keep[q * 4 + i] = u4_word(w, i) >= hp.drop_thresh ? 1 : 0;
   }
@@ -1039,13 +1041,15 @@ __global__ void k_sgd_conv(float* __restrict__ w, float* __restrict__ v,
       for (int i = 0; i < 4; ++i) g += q[i];
     }
     for (; s < S; ++s) g += part[s * split_stride + base];
-    float wv = w[p], vv = v[p];
-    sgd_one(wv, vv, g, hp);
-    w[p] = wv;
-    v[p] = vv;
-    const bf16 hb = __float2bfloat16_rn(wv);
-    fwd[ix.fwd] = hb;
-    if (dg) dg[ix.dg] = hb;
+    if (hp.update) {
+      float wv = w[p], vv = v[p];
+      sgd_one(wv, vv, g, hp);
+      w[p] = wv;
+      v[p] = vv;
+      const bf16 hb = __float2bfloat16_rn(wv);
+      fwd[ix.fwd] = hb;
+      if (dg) dg[ix.dg] = hb;
+    }
     if (grads_out) grads_out[p] = g;
   }
 }
@@ -1068,9 +1072,11 @@ __global__ void k_sgd_dense(float* __restrict__ w, float* __restrict__ v,
   const long long n4 = n / 4;
   for (long long q = blockIdx.x * 1LL * blockDim.x + threadIdx.x; q < n4;
        q += 1LL * gridDim.x * blockDim.x) {
+    const float4 gv = reinterpret_cast<const float4*>(g)[q];
+    if (grads_out) reinterpret_cast<float4*>(grads_out)[q] = gv;
+    if (!hp.update) continue;
     float4 wv = reinterpret_cast<float4*>(w)[q];
     float4 vv = reinterpret_cast<float4*>(v)[q];
-    const float4 gv = reinterpret_cast<const float4*>(g)[q];
     sgd_one(wv.x, vv.x, gv.x, hp);
     sgd_one(wv.y, vv.y, gv.y, hp);
     sgd_one(wv.z, vv.z, gv.z, hp);
@@ -1085,7 +1091,6 @@ __global__ void k_sgd_dense(float* __restrict__ w, float* __restrict__ v,
       u.y = *reinterpret_cast<uint32_t*>(&h1);
       reinterpret_cast<uint2*>(shadow)[q] = u;
     }
-    if (grads_out) reinterpret_cast<float4*>(grads_out)[q] = gv;
   }
 }
 
@@ -1123,11 +1128,28 @@ __global__ void __launch_bounds__(1024) k_sgd_bias(float* __restrict__ b, float*
 #pragma unroll 8
     for (int q = 0; q < 32; ++q) sum += red[q][tx];
     const HParams hp = *hpp;
-    float wv = b[i], vv = v[i];
-    sgd_one(wv, vv, sum, hp);
-    b[i] = wv;
-    v[i] = vv;
+    if (hp.update) {
+      float wv = b[i], vv = v[i];
+      sgd_one(wv, vv, sum, hp);
+      b[i] = wv;
+      v[i] = vv;
+    }
     if (grads_out) grads_out[i] = sum;
+  }
+}
+
+// [S] 3.4 "Training Procedure Details", update rule, on a range of the
+// parameter blob with a gradient that arrives scaled: g = scale * gsum (the
+// sum of the ranks' gradients of their own batch means, scale = 1 / ranks).
+__global__ void k_sgd_range(float* __restrict__ w, float* __restrict__ v,
+                            const float* __restrict__ gsum, long long n, float scale, float lr,
+                            float momentum, float wd) {
+  for (long long p = blockIdx.x * 1LL * blockDim.x + threadIdx.x; p < n;
+       p += 1LL * gridDim.x * blockDim.x) {
+    const float g = scale * gsum[p];
+    const float vn = momentum * v[p] - wd * lr * w[p] - lr * g;
+    v[p] = vn;
+    w[p] += vn;
   }
 }
 
@@ -1644,12 +1666,14 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
   return true;
 }
 constexpr int kPoolLrnBlocks = 148 * 8;  // persistent blocks: eight per SM
+// quads of 2 x 2 pixels per block (one 8-channel unit per thread)
+inline int pool_lrn_quads_per_block(int C) { return 256 / (C / 8); }
 int pool_lrn_bwd_parts(int B, int H, int W, int C, int z) {
   (void)z;
-  if (C <= 0 || C % 8) return 0;
-  const long long npix = 1LL * B * H * W;
-  const int np = 256 / (C / 8);
-  const long long groups = np > 0 ? (npix + np - 1) / np : 0;
+  if (C <= 0 || C % 8 || C > 2048) return 0;
+  const long long nquads = 1LL * B * ((H + 1) / 2) * ((W + 1) / 2);
+  const int nq = pool_lrn_quads_per_block(C);
+  const long long groups = nq > 0 ? (nquads + nq - 1) / nq : 0;
   return static_cast<int>(groups < kPoolLrnBlocks ? groups : kPoolLrnBlocks);
 }
 bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
@@ -1660,13 +1684,13 @@ bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16*
   if (npix * C >= (1LL << 31)) return false;  // 32-bit element offsets
   const bool b34 = beta == 0.75f;
   const int blocks = pool_lrn_bwd_parts(B, H, W, C, z);
-  const int np = 256 / (C / 8);  // whole pixels per block, one 8-channel unit per thread
-  const size_t smem = static_cast<size_t>(np) * 2 * (C + 8) * sizeof(float);
-  if (np < 1 || smem > 48 * 1024) return false;
+  const int nq = pool_lrn_quads_per_block(C);
+  if (nq < 1 || blocks < 1) return false;
+  const int nquads = static_cast<int>(1LL * B * ((H + 1) / 2) * ((W + 1) / 2));
   // persistent blocks (at most kPoolLrnBlocks, one bias partial row each)
   auto go = [&](auto kern) {
-    kern<<<blocks, 256, smem, s>>>(dy, am, a, dl, da, static_cast<int>(npix), np, H, W, C, z, k,
-                                   alpha, beta, bias_part);
+    kern<<<blocks, 256, 0, s>>>(dy, am, a, dl, da, nquads, nq, H, W, C, z, k, alpha, beta,
+                                bias_part);
   };
   if (z == 3 && H == 55 && W == 55)
     b34 ? go(k_pool_lrn_bwd<3, 55, true>) : go(k_pool_lrn_bwd<3, 55, false>);
@@ -1750,6 +1774,11 @@ void launch_sgd_bias_rows(float* b, float* v, const bf16* g, int rows, int n, fl
 void launch_conv_shadows(const float* w, const ConvMap& m, bf16* fwd, bf16* dg, cudaStream_t s) {
   const long long n = 1LL * m.Cout * m.K * m.K * m.Cg;
   k_conv_shadows<<<grid_for(n, 256), 256, 0, s>>>(w, m, fwd, dg);
+  count_launch();
+}
+void launch_sgd_range(float* w, float* v, const float* gsum, long long n, float scale, float lr,
+                      float momentum, float wd, cudaStream_t s) {
+  k_sgd_range<<<grid_for(n, 256), 256, 0, s>>>(w, v, gsum, n, scale, lr, momentum, wd);
   count_launch();
 }
 void launch_f32_to_bf16(const float* w, bf16* out, long long n, cudaStream_t s) {

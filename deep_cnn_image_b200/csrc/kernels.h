@@ -22,6 +22,8 @@ struct HParams {
   uint32_t step;
   uint32_t seed_lo, seed_hi;
   uint32_t drop_thresh;  // keep iff Philox word >= drop_thresh
+  uint32_t update;       // 1: apply the update; 0: only write the gradients out
+  uint32_t row_offset;   // index of the batch's first image in the whole minibatch (dropout draws)
 };
 
 // [S] 3.4 "Training Procedure Details", update rule; [W] listing TRAIN_STEP:
@@ -50,6 +52,8 @@ void count_launch_n(int64_t n);
 // detection without a fault).
 void launch_wait_probe(int* status, long long limit_cycles, cudaStream_t s);
 void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s);
+void launch_sgd_range(float* w, float* v, const float* gsum, long long n, float scale, float lr,
+                      float momentum, float wd, cudaStream_t s);
 
 // x [B,227,227,3] (bf16) -> xs [B,57,57,64]: xs[b,i,j,(dy*4+dx)*3+c] = x[b,4i+dy,4j+dx,c]
 // (zero beyond row/column 226, and channels 48..63 zero).

@@ -5,9 +5,12 @@
 // Euclidean distance between their 4096-dimensional last-hidden-layer
 // activations.  For Q query rows q and N base rows x (D features each):
 //   d(i, j) = ||q_i||^2 + ||x_j||^2 - 2 q_i . x_j
-// The dot products are one tcgen05 GEMM (queries as A, base as B, fp32
-// out); the squared norms come from a row kernel; a selection kernel keeps
-// each query's k smallest distances (ties to the lower base index).
+// The dot products are a tcgen05 GEMM (queries as A, base rows as B) whose
+// epilogue turns each product into a distance and keeps, per query, the k
+// smallest seen so far in registers: the Q x N distances never reach memory.
+// Each CTA leaves two candidate lists per query (one per epilogue column
+// half); a merge kernel picks the k smallest of them (ties to the lower base
+// index).  The squared norms come from a row kernel.
 #include <cuda_bf16.h>
 
 #include <cfloat>
@@ -17,6 +20,7 @@
 #include "alexnet.h"
 #include "gemm.h"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace alx {
 namespace {
@@ -54,23 +58,236 @@ __device__ __forceinline__ bool before(float a, int ia, float b, int ib) {
   return a < b || (a == b && ia < ib);
 }
 
-// One block per query: every thread keeps its k best candidates of a
-// strided share of the base (a sorted list, insertion from the tail), then k
-// rounds of a block-wide minimum over the threads' list heads pick the
-// result in order.  Lists live in registers (all indices compile-time);
-// KMAX >= k is their capacity, THREADS the block size (fewer threads for the
-// longest lists, which need the most registers).
-template <int KMAX, int THREADS>
-__global__ void __launch_bounds__(THREADS) k_knn_select(const float* __restrict__ dots, int N,
-                                                    const float* __restrict__ qn,
-                                                    const float* __restrict__ xn, int k,
-                                                    float* __restrict__ dist,
-                                                    int32_t* __restrict__ idx) {
-  __shared__ float wv[32];
-  __shared__ int wi[32], wt[32];
+// ---------------------------------------------------------------- fused GEMM + selection
+// One persistent 320-thread CTA per SM: warps 0-7 epilogue, warp 8 TMA
+// producer, warp 9 MMA issuer and TMEM owner (the layout of the library's
+// other tensor-core kernels).  Tile t covers base rows t * 256 .. t * 256 +
+// 255 against the (at most 128) queries of this launch; K walks the D
+// features in blocks of 64.  Two accumulators of 256 fp32 columns in tensor
+// memory let the epilogue of tile i overlap the MMAs of tile i + 1.
+constexpr int kKnnBN = 256;
+constexpr int kKnnThreads = 320;
+constexpr int kKnnA = 128 * 64 * 2;      // queries: 128 rows x 64 features
+constexpr int kKnnB = kKnnBN * 64 * 2;   // base: 256 rows x 64 features
+
+// Insert (d, j) into the ascending list (bd, bi) of length k (k <= KMAX) if
+// it ranks before the current k-th; (td, ti) caches the k-th entry.
+template <int KMAX>
+__device__ __forceinline__ void topk_insert(float (&bd)[KMAX], int (&bi)[KMAX], float& td,
+                                            int& ti, int k, float d, int j) {
+  if (!before(d, j, td, ti)) return;
+  // from the tail: an entry after which (d, j) ranks moves down one place;
+  // the first entry before which it does not rank is where it goes
+#pragma unroll
+  for (int t = KMAX - 1; t > 0; --t) {
+    if (t < k) {
+      const bool shift = before(d, j, bd[t - 1], bi[t - 1]);
+      const bool here = before(d, j, bd[t], bi[t]);
+      bd[t] = shift ? bd[t - 1] : (here ? d : bd[t]);
+      bi[t] = shift ? bi[t - 1] : (here ? j : bi[t]);
+    }
+  }
+  if (before(d, j, bd[0], bi[0])) {
+    bd[0] = d;
+    bi[0] = j;
+  }
+#pragma unroll
+  for (int t = 0; t < KMAX; ++t)
+    if (t == k - 1) {
+      td = bd[t];
+      ti = bi[t];
+    }
+}
+
+struct KnnArgs {
+  int Q, N, Kblocks, k, tiles;
+  const float* qn;   // [Q] query squared norms (this launch's queries)
+  const float* xn;   // [N] base squared norms
+  float* cd;         // candidates [gridDim.x * 2][128][k] distances
+  int* ci;           // and base indices
+  int* status;
+};
+
+template <int KMAX>
+__global__ void __launch_bounds__(kKnnThreads, 1)
+    k_knn_gemm_select(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmX, const __grid_constant__ KnnArgs a,
+                      int stages) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + stages * kKnnA;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * (kKnnA + kKnnB));
+  const uint32_t full = smem_u32(bars);
+  const uint32_t empty = full + 8 * stages;
+  const uint32_t acc_full = full + 16 * stages;
+  const uint32_t acc_empty = acc_full + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * stages + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full + 8 * s, 1);
+      mbar_init(empty + 8 * s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full + 8 * i, 1);
+      mbar_init(acc_empty + 8 * i, 256);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmX);
+      RingPos r;
+      bool ok = true;
+      for (int t = blockIdx.x; t < a.tiles && ok; t += gridDim.x) {
+        for (int kb = 0; kb < a.Kblocks; ++kb, r.next(stages)) {
+          if (!mbar_wait(empty + 8 * r.slot, r.phase ^ 1, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full + 8 * r.slot;
+          mbar_arrive_expect_tx(fb, kKnnA + kKnnB);
+          tma_load_2d(sA + r.slot * kKnnA, &tmQ, kb * 64, 0, fb);
+          tma_load_2d(sB + r.slot * kKnnB, &tmX, kb * 64, t * kKnnBN, fb);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, kKnnBN, 0, 0);
+      const uint64_t ad = smem_desc_sw128(sA, 16, 1024), bd = smem_desc_sw128(sB, 16, 1024);
+      const uint32_t a_lo = static_cast<uint32_t>(ad), a_hi = static_cast<uint32_t>(ad >> 32);
+      const uint32_t b_lo = static_cast<uint32_t>(bd), b_hi = static_cast<uint32_t>(bd >> 32);
+      RingPos r;
+      uint32_t tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < a.tiles && ok; t += gridDim.x, ++tcount) {
+        const int acc = tcount & 1;
+        if (!mbar_wait(acc_empty + 8 * acc, ((tcount >> 1) & 1) ^ 1, a.status, abort_flag))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * kKnnBN;
+        for (int kb = 0; kb < a.Kblocks; ++kb, r.next(stages)) {
+          if (!mbar_wait(full + 8 * r.slot, r.phase, a.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          tc_mma_k4<2, 2>(d, a_lo + r.slot * (kKnnA >> 4), a_hi, b_lo + r.slot * (kKnnB >> 4),
+                          b_hi, idesc, kb == 0 ? 0u : 1u);
+          tc_commit(empty + 8 * r.slot);
+        }
+        if (!ok) break;
+        tc_commit(acc_full + 8 * acc);
+      }
+    }
+  } else {
+    // epilogue: thread = one query (TMEM lane), half of each tile's columns
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const bool live = row < a.Q;
+    const float nq = live ? a.qn[row] : 0.f;
+    float bd[KMAX];
+    int bi[KMAX];
+#pragma unroll
+    for (int t = 0; t < KMAX; ++t) {
+      bd[t] = FLT_MAX;
+      bi[t] = 0x7fffffff;
+    }
+    float td = FLT_MAX;
+    int ti = 0x7fffffff;
+    // candidates of a chunk that beat the current k-th go through shared
+    // memory (lane-contiguous per warp), so the rare insertions index them
+    // dynamically instead of unrolling an insertion per column
+    float* sd = reinterpret_cast<float*>(smem + stages * (kKnnA + kKnnB) + 1024) + warp * 32 * 32;
+    uint32_t tcount = 0;
+    for (int t = blockIdx.x; t < a.tiles; t += gridDim.x, ++tcount) {
+      const int acc = tcount & 1;
+      if (!mbar_wait(acc_full + 8 * acc, (tcount >> 1) & 1, a.status, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * kKnnBN;
+#pragma unroll 1
+      for (int c0 = 32 * half; c0 < kKnnBN; c0 += 64) {
+        float v[32];
+        tmem_ld32(tb + c0, v);
+        const int j0 = t * kKnnBN + c0;
+        if (!live) continue;
+        float dd[32];
+        uint32_t m = 0;
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const int j = j0 + 4 * q4;
+          // N % 8 == 0: a group of four is wholly inside or outside the base
+          const float4 n4 = j < a.N ? __ldg(reinterpret_cast<const float4*>(a.xn + j))
+                                    : make_float4(FLT_MAX, FLT_MAX, FLT_MAX, FLT_MAX);
+          const float nn[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float d = j < a.N ? fmaxf(nq + nn[e] - 2.f * v[4 * q4 + e], 0.f) : FLT_MAX;
+            dd[4 * q4 + e] = d;
+            m |= (before(d, j + e, td, ti) ? 1u : 0u) << (4 * q4 + e);
+          }
+        }
+        if (m) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sd[e * 32 + lane] = dd[e];
+          while (m) {
+            const int e = __ffs(m) - 1;
+            m &= m - 1;
+            topk_insert<KMAX>(bd, bi, td, ti, a.k, sd[e * 32 + lane], j0 + e);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty + 8 * acc);
+    }
+    const size_t list = (static_cast<size_t>(blockIdx.x) * 2 + half) * 128 + row;
+#pragma unroll
+    for (int t = 0; t < KMAX; ++t)
+      if (t < a.k) {
+        a.cd[list * a.k + t] = bd[t];
+        a.ci[list * a.k + t] = bi[t];
+      }
+  }
+  __syncthreads();
+  if (*abort_flag) {
+    for (int i = 0; i < 1000; ++i) __nanosleep(1000);
+  }
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// One block per query: the k smallest of its `lists` candidate lists (each
+// of k entries, ascending) -- a thread walks a strided share of the lists
+// keeping its own k best, then k rounds of a block-wide minimum over the
+// threads' list heads.
+template <int KMAX>
+__global__ void __launch_bounds__(256) k_knn_merge(const float* __restrict__ cd,
+                                                   const int* __restrict__ ci, int lists, int k,
+                                                   int q0, float* __restrict__ dist,
+                                                   int32_t* __restrict__ idx) {
+  __shared__ float wv[8];
+  __shared__ int wi[8], wt[8];
   __shared__ int winner;
-  const int q = blockIdx.x;
-  const float nq = qn[q];
+  const int q = blockIdx.x;  // query within this launch's block of 128
   float bd[KMAX];
   int bi[KMAX];
 #pragma unroll
@@ -78,40 +295,15 @@ __global__ void __launch_bounds__(THREADS) k_knn_select(const float* __restrict_
     bd[t] = FLT_MAX;
     bi[t] = 0x7fffffff;
   }
-  // four consecutive candidates per step (N % 4 == 0, rows 16-byte aligned)
-  const float4* row4 = reinterpret_cast<const float4*>(dots + static_cast<size_t>(q) * N);
-  const float4* xn4 = reinterpret_cast<const float4*>(xn);
-  for (int j4 = threadIdx.x; j4 < (N >> 2); j4 += blockDim.x) {
-    const float4 g4 = row4[j4], n4 = xn4[j4];
-  #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float gv = e == 0 ? g4.x : e == 1 ? g4.y : e == 2 ? g4.z : g4.w;
-      const float nv = e == 0 ? n4.x : e == 1 ? n4.y : e == 2 ? n4.z : n4.w;
-      const int j = 4 * j4 + e;
-      const float d = fmaxf(nq + nv - 2.f * gv, 0.f);
-      float last = FLT_MAX;
-      int last_i = 0x7fffffff;
-  #pragma unroll
-      for (int t = 0; t < KMAX; ++t)
-        if (t == k - 1) {
-          last = bd[t];
-          last_i = bi[t];
-        }
-      if (!before(d, j, last, last_i)) continue;
-      bool placed = false;
-  #pragma unroll
-      for (int t = KMAX - 1; t >= 0; --t) {
-        if (t < k && !placed) {
-          if (t > 0 && before(d, j, bd[t - 1 > 0 ? t - 1 : 0], bi[t - 1 > 0 ? t - 1 : 0])) {
-            bd[t] = bd[t - 1 > 0 ? t - 1 : 0];
-            bi[t] = bi[t - 1 > 0 ? t - 1 : 0];
-          } else {
-            bd[t] = d;
-            bi[t] = j;
-            placed = true;
-          }
-        }
-      }
+  float td = FLT_MAX;
+  int ti = 0x7fffffff;
+  for (int L = threadIdx.x; L < lists; L += blockDim.x) {
+    const size_t base = (static_cast<size_t>(L) * 128 + q) * k;
+    for (int t = 0; t < k; ++t) {
+      const float d = cd[base + t];
+      const int j = ci[base + t];
+      if (!before(d, j, td, ti)) break;  // the list is ascending
+      topk_insert<KMAX>(bd, bi, td, ti, k, d, j);
     }
   }
   int head = 0;
@@ -151,8 +343,8 @@ __global__ void __launch_bounds__(THREADS) k_knn_select(const float* __restrict_
           bix = wi[u];
           bt = wt[u];
         }
-      dist[static_cast<size_t>(q) * k + r] = b;
-      idx[static_cast<size_t>(q) * k + r] = bix;
+      dist[static_cast<size_t>(q0 + q) * k + r] = b;
+      idx[static_cast<size_t>(q0 + q) * k + r] = bix;
       winner = bt;
     }
     __syncthreads();
@@ -179,12 +371,29 @@ using namespace alx;
 
 extern "C" {
 
+namespace {
+constexpr int kKnnMaxGrid = 160;  // candidate lists are sized for this many CTAs
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+size_t knn_cand_bytes() {
+  return align256(static_cast<size_t>(kKnnMaxGrid) * 2 * 128 * kKnnMaxK * sizeof(float));
+}
+
+bool knn_prepared = false;
+cudaError_t knn_prepare(int smem) {
+  if (knn_prepared) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(&k_knn_gemm_select<kKnnMaxK>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  knn_prepared = e == cudaSuccess;
+  return e;
+}
+}  // namespace
+
 size_t alexnet_knn_workspace_bytes(int Q, int N) {
   if (Q < 1 || N < 1) return 0;
-  const size_t a = (static_cast<size_t>(Q) * N * sizeof(float) + 255) & ~static_cast<size_t>(255);
-  const size_t b = (static_cast<size_t>(Q) * sizeof(float) + 255) & ~static_cast<size_t>(255);
-  const size_t c = (static_cast<size_t>(N) * sizeof(float) + 255) & ~static_cast<size_t>(255);
-  return a + b + c + 256 + 256;  // + the GEMM's status word, + alignment
+  return align256(static_cast<size_t>(Q) * sizeof(float)) +
+         align256(static_cast<size_t>(N) * sizeof(float)) + 2 * knn_cand_bytes() + 256 + 256;
 }
 
 alexnet_status alexnet_knn_sqnorms(const void* x, int rows, int D, float* out, void* stream) {
@@ -208,36 +417,24 @@ alexnet_status alexnet_knn(const void* queries, int Q, const void* base, int N, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* p = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(ws) + 255) &
                                     ~static_cast<uintptr_t>(255));
-  float* dots = reinterpret_cast<float*>(p);
-  p += (static_cast<size_t>(Q) * N * sizeof(float) + 255) & ~static_cast<size_t>(255);
   float* qn = reinterpret_cast<float*>(p);
-  p += (static_cast<size_t>(Q) * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  p += align256(static_cast<size_t>(Q) * sizeof(float));
   float* xn = reinterpret_cast<float*>(p);
-  p += (static_cast<size_t>(N) * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  p += align256(static_cast<size_t>(N) * sizeof(float));
+  float* cd = reinterpret_cast<float*>(p);
+  p += knn_cand_bytes();
+  int* ci = reinterpret_cast<int*>(p);
+  p += knn_cand_bytes();
   int* status = reinterpret_cast<int*>(p);  // a bounded wait that runs out sets a bit here
-  // dots[i][j] = q_i . x_j: queries K-major as A, base K-major as B
-  GemmDesc d;
-  memset(&d, 0, sizeof(d));
-  d.asrc = A_TMA_K;
-  d.bsrc = B_TMA_K;
-  d.bn = 128;
-  GemmArgs& a = d.args;
-  a.M = Q;
-  a.N = N;
-  a.Kblocks = (D + 63) / 64;
-  a.kb_per_split = a.Kblocks;
-  a.groups = 1;
-  a.epi = EPI_F32;
-  a.out = dots;
-  a.ld_out = N;
-  a.split_stride = static_cast<long long>(Q) * N;
-  a.status = status;
   const auto* qb = static_cast<const __nv_bfloat16*>(queries);
   const auto* xb = static_cast<const __nv_bfloat16*>(base);
-  if (!make_tmap_bf16(&d.tmA, qb, D, Q, static_cast<uint64_t>(D) * 2, 64, 128) ||
-      !make_tmap_bf16(&d.tmB, xb, D, N, static_cast<uint64_t>(D) * 2, 64, 128) ||
-      !gemm_finalize(&d, knn_sms()))
+  CUtensorMap tmX;
+  if (!make_tmap_bf16(&tmX, xb, D, N, static_cast<uint64_t>(D) * 2, 64, kKnnBN))
     return ALEXNET_ERR_UNSUPPORTED;
+  const int stages = 3;
+  // stages, barriers (1 KB) and the epilogue's candidate buffer (32 KB)
+  const int smem = 1024 + stages * (kKnnA + kKnnB) + 1024 + 8 * 32 * 32 * 4;
+  if (knn_prepare(smem) != cudaSuccess) return ALEXNET_ERR_CUDA;
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return ALEXNET_ERR_CUDA;
   k_row_sqnorm<<<(Q + 7) / 8, 256, 0, s>>>(qb, Q, D, qn);
   count_launch();
@@ -249,14 +446,32 @@ alexnet_status alexnet_knn(const void* queries, int Q, const void* base, int N, 
                                                                                        xn);
     count_launch();
   }
-  if (gemm_launch(d, s) != cudaSuccess) return ALEXNET_ERR_CUDA;
-  if (k <= 8)
-    k_knn_select<8, 512><<<Q, 512, 0, s>>>(dots, N, qn, xn, k, dist, idx);
-  else if (k <= 16)
-    k_knn_select<16, 512><<<Q, 512, 0, s>>>(dots, N, qn, xn, k, dist, idx);
-  else
-    k_knn_select<32, 256><<<Q, 256, 0, s>>>(dots, N, qn, xn, k, dist, idx);
-  count_launch();
+  KnnArgs a;
+  a.N = N;
+  a.Kblocks = (D + 63) / 64;
+  a.k = k;
+  a.tiles = (N + kKnnBN - 1) / kKnnBN;
+  a.xn = xn;
+  a.cd = cd;
+  a.ci = ci;
+  a.status = status;
+  int grid = a.tiles < knn_sms() ? a.tiles : knn_sms();
+  if (grid > kKnnMaxGrid) grid = kKnnMaxGrid;
+  // queries in blocks of 128 (one MMA tile of rows)
+  for (int q0 = 0; q0 < Q; q0 += 128) {
+    const int Qb = Q - q0 < 128 ? Q - q0 : 128;
+    CUtensorMap tmQ;
+    if (!make_tmap_bf16(&tmQ, qb + static_cast<size_t>(q0) * D, D, Qb,
+                        static_cast<uint64_t>(D) * 2, 64, 128))
+      return ALEXNET_ERR_UNSUPPORTED;
+    a.Q = Qb;
+    a.qn = qn + q0;
+    // one list capacity for every k <= 32: insertions are rare, and the
+    // 32-entry lists stay in registers
+    k_knn_gemm_select<kKnnMaxK><<<grid, kKnnThreads, smem, s>>>(tmQ, tmX, a, stages);
+    k_knn_merge<kKnnMaxK><<<Qb, 256, 0, s>>>(cd, ci, 2 * grid, k, q0, dist, idx);
+    count_launch_n(2);
+  }
   return cudaGetLastError() == cudaSuccess ? ALEXNET_OK : ALEXNET_ERR_CUDA;
 }
 

@@ -26,16 +26,27 @@ namespace {
 
 constexpr int kClasses = 1000;
 
+// Guard region after every workspace buffer: filled with kCanaryByte at
+// create and compared by alexnet_debug_canaries, so that a kernel writing
+// past the end of any buffer is caught.
+constexpr size_t kCanaryBytes = 256;
+constexpr unsigned char kCanaryByte = 0xA5;
+
 // Bump allocator over the caller's workspace (base == nullptr: size only).
+// Every buffer starts on a 256-byte boundary and is followed by a guard.
 struct Carver {
   char* base;
   size_t off = 0;
-  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  std::vector<size_t>* guards;  // offsets of the guard regions (nullable)
+  explicit Carver(void* b, std::vector<size_t>* g = nullptr)
+      : base(static_cast<char*>(b)), guards(g) {}
   template <typename T>
   T* take(size_t n) {
     off = (off + 255) & ~static_cast<size_t>(255);
     T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
     off += n * sizeof(T);
+    if (guards) guards->push_back(off);
+    off += kCanaryBytes;
     return p;
   }
 };
@@ -67,6 +78,8 @@ struct Plan {
   ConvPlan cf[5], cd[5], cw[5];
   GemmDesc ff[3], fd[3], fw[3];
   GemmDesc fws[3];  // FC weight gradient with the update in its epilogue
+  GemmDesc fwg[3];  // FC weight gradient straight into the handle's gradient buffer
+  bool has_fwg = false;
   double conv_flops[5], fc_flops[3];  // algorithmic FLOPs of one pass of each layer
   bool ok = false;
 };
@@ -99,6 +112,7 @@ struct alexnet {
   int num_sms = 148;
   char* ws = nullptr;
   size_t ws_bytes = 0;
+  std::vector<size_t> guards;  // workspace offsets of the guard regions
   std::string err;
   cudaStream_t last_stream = nullptr;
   uint64_t step = 0;
@@ -178,6 +192,12 @@ struct alexnet {
   // the flipped weight copies (wd) are refreshed only while some data-gradient
   // plan reads them (the box kernel reads the forward copies transposed)
   bool need_wd = false;
+  // data-parallel gradient step (alexnet_train_grads): no update, every
+  // parameter gradient written to `grads`, dropout rows offset by the first
+  // image's index in the whole minibatch; fc_event marks the FC gradients
+  bool grads_only = false;
+  uint32_t row_offset = 0;
+  cudaEvent_t fc_event = nullptr;
   bool capturing = false;
   StepRec direct_rec;
   std::map<int, StepRec> graph_rec;
@@ -442,6 +462,11 @@ bool build_plan(alexnet* h, int B, Plan* P) {
     if (!desc_fc_wgrad_sgd(&P->fws[f], h->fc[f], dz[f], fin[f], h->params + h->w_off[5 + f],
                            h->vel + h->w_off[5 + f], h->wf[5 + f], gr, h->hp, B, ns, h->status))
       return set_err(h, "fc weight-gradient + update plan");
+    // one K-slice (the batch fits one split), so the product lands in place
+    P->has_fwg = gr != nullptr;
+    if (gr && (!desc_fc_wgrad(&P->fwg[f], h->fc[f], dz[f], fin[f], gr, B, ns, h->status) ||
+               P->fwg[f].args.splits != 1))
+      P->has_fwg = false;
   }
   if (h->scratch) {
     const GemmDesc* all[] = {&P->ff[0], &P->ff[1], &P->ff[2], &P->fd[0], &P->fd[1],
@@ -458,7 +483,8 @@ bool build_plan(alexnet* h, int B, Plan* P) {
 
 // Carve every buffer of the handle out of the workspace (or size it).
 size_t carve(alexnet* h, void* base) {
-  Carver c(base);
+  if (base) h->guards.clear();
+  Carver c(base, base ? &h->guards : nullptr);
   const alexnet_config& cfg = h->cfg;
   const int B = cfg.batch_max;
   const size_t n = h->n_params;
@@ -570,6 +596,8 @@ void write_hp(alexnet* h, float lr, cudaStream_t s) {
   h->hp_host.seed_hi = static_cast<uint32_t>(h->cfg.seed >> 32);
   const double t = static_cast<double>(h->cfg.dropout_p) * 4294967296.0 + 0.5;
   h->hp_host.drop_thresh = t >= 4294967295.0 ? 0xFFFFFFFFu : static_cast<uint32_t>(t);
+  h->hp_host.update = h->grads_only ? 0u : 1u;
+  h->hp_host.row_offset = h->grads_only ? h->row_offset : 0u;
   launch_write_hparams(h->hp, h->hp_host, s);
 }
 
@@ -706,8 +734,10 @@ alexnet_status forward_f32(alexnet* h, const float* x, int B, float* logits, cud
   return cuda_status(h, cudaGetLastError(), "forward fp32");
 }
 
-alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int B, float* loss,
-                          cudaStream_t s, Plan* P) {
+// Forward, loss and the FC layers' backward (with their update, unless the
+// handle runs a gradient-only step).
+alexnet_status train_fc_part(alexnet* h, const bf16* x, const int32_t* labels, int B, float* loss,
+                             cudaStream_t s, Plan* P) {
   const alexnet_config& cfg = h->cfg;
   alexnet_status st = forward_bf16(h, x, B, cfg.dropout_on ? 1 : 0, h->logits, s, P);
   // (x == nullptr: the caller converted the input already)
@@ -725,7 +755,9 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     const FcL& F = h->fc[f];
     ALX_TRY(run_gemm(h, P->fd[f], P->fc_flops[f], s), "fc dgrad launch");
     launch_dgrad_finalize(h->scratch, P->fd[f].args.splits, B, F.In, mask[f], dxo[f], s);
-    if (h->fc_fused) {
+    if (h->grads_only) {
+      ALX_TRY(run_gemm(h, P->fwg[f], P->fc_flops[f], s), "fc wgrad launch");
+    } else if (h->fc_fused) {
       // HBM-bound (the update moves 18 bytes per weight against 256 MMA
       // FLOPs): launched outside the per-GEMM tensor-roofline records
       ALX_TRY(launch_any(P->fws[f], s), "fc wgrad + update launch");
@@ -737,6 +769,14 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     launch_sgd_bias_rows(h->params + h->b_off[5 + f], h->vel + h->b_off[5 + f], dz[f], B, F.Out,
                          gptr(h->b_off[5 + f]), h->hp, s);
   }
+  return cuda_status(h, cudaGetLastError(), "train step (FC part)");
+}
+
+// The convolutions' backward and update (or gradients only), top down.
+alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
+  const alexnet_config& cfg = h->cfg;
+  float* gr = h->grads;
+  auto gptr = [&](size_t off) { return gr ? gr + off : nullptr; };
   // Per conv layer, top down: bias update (its column sums come from the
   // pool (+ normalisation) backward that produced da where it made them,
   // else from da), data gradient into the layer below (and that layer's
@@ -799,6 +839,59 @@ alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int 
     }
   }
   return cuda_status(h, cudaGetLastError(), "train step");
+}
+
+alexnet_status train_bf16(alexnet* h, const bf16* x, const int32_t* labels, int B, float* loss,
+                          cudaStream_t s, Plan* P) {
+  alexnet_status st = train_fc_part(h, x, labels, B, loss, s, P);
+  if (st != ALEXNET_OK) return st;
+  return train_conv_part(h, B, s, P);
+}
+
+// Runs body(stream) for graph `key`: captured into a CUDA graph the first
+// time, replayed afterwards (direct launches when graphs are off).
+template <typename F>
+alexnet_status replay(alexnet* h, int key, cudaStream_t s, F&& body) {
+  if (!h->use_graphs) {
+    h->direct_rec.reset();
+    h->rec = h->stats_on ? &h->direct_rec : nullptr;
+    const alexnet_status st = body(s);
+    h->rec = nullptr;
+    if (h->stats_on) h->last_rec = &h->direct_rec;
+    return st;
+  }
+  auto it = h->train_graphs.find(key);
+  if (it == h->train_graphs.end()) {
+    if (!h->cap_stream)
+      ALX_TRY(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking), "capture stream");
+    ALX_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal),
+            "begin capture");
+    const int64_t c0 = launch_counter();
+    h->rec = h->stats_on ? &h->graph_rec[key] : nullptr;
+    h->capturing = true;
+    const alexnet_status st = body(h->cap_stream);
+    h->capturing = false;
+    h->rec = nullptr;
+    // captured kernels are counted when a replay runs them, not now
+    h->graph_kernels[key] = launch_counter() - c0;
+    count_launch_n(-(launch_counter() - c0));
+    cudaGraph_t g = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(h->cap_stream, &g);
+    if (st != ALEXNET_OK) {
+      if (g) cudaGraphDestroy(g);
+      return st;
+    }
+    ALX_TRY(ce, "end capture");
+    cudaGraphExec_t ex = nullptr;
+    const cudaError_t ie = cudaGraphInstantiate(&ex, g, 0);
+    cudaGraphDestroy(g);
+    ALX_TRY(ie, "graph instantiate");
+    it = h->train_graphs.emplace(key, ex).first;
+  }
+  ALX_TRY(cudaGraphLaunch(it->second, s), "graph launch");
+  count_launch_n(h->graph_kernels[key]);
+  if (h->stats_on) h->last_rec = &h->graph_rec[key];
+  return ALEXNET_OK;
 }
 
 }  // namespace
@@ -888,6 +981,8 @@ alexnet_status alexnet_create(const alexnet_config* cfg, void* workspace, size_t
   }
   launch_fill(h->vel, h->n_params, 0.f, s);
   cudaError_t e = cudaMemsetAsync(h->status, 0, sizeof(int), s);
+  for (size_t i = 0; i < h->guards.size() && e == cudaSuccess; ++i)
+    e = cudaMemsetAsync(h->ws + h->guards[i], kCanaryByte, kCanaryBytes, s);
   for (int l = 0; l < 5 && e == cudaSuccess && h->cfg.dtype == ALEXNET_BF16; ++l)
     e = cudaMemsetAsync(h->wf[l], 0, sizeof(bf16) * h->conv[l].Cout * h->conv[l].Kdim(), s);
   refresh_shadows(h, s);
@@ -965,48 +1060,11 @@ alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* la
   launch_s2d(static_cast<const bf16*>(x), h->xs, B, s);
   ALX_TRY(cudaMemcpyAsync(h->labels_buf, labels, sizeof(int32_t) * B, cudaMemcpyDeviceToDevice, s),
           "train_step labels");
-  alexnet_status st = ALEXNET_OK;
   const int64_t l0 = launch_counter();
-  if (h->use_graphs) {
-    const int key = 8 * B + (h->fc_fused ? 4 : 0) + (h->keep ? 2 : 0) + (h->stats_on ? 1 : 0);
-    auto it = h->train_graphs.find(key);
-    if (it == h->train_graphs.end()) {
-      if (!h->cap_stream)
-        ALX_TRY(cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking), "capture stream");
-      ALX_TRY(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal),
-              "begin capture");
-      const int64_t c0 = launch_counter();
-      h->rec = h->stats_on ? &h->graph_rec[key] : nullptr;
-      h->capturing = true;
-      st = train_bf16(h, nullptr, h->labels_buf, B, nullptr, h->cap_stream, P);
-      h->capturing = false;
-      h->rec = nullptr;
-      // captured kernels are counted when a replay runs them, not now
-      h->graph_kernels[key] = launch_counter() - c0;
-      count_launch_n(-(launch_counter() - c0));
-      cudaGraph_t g = nullptr;
-      const cudaError_t ce = cudaStreamEndCapture(h->cap_stream, &g);
-      if (st != ALEXNET_OK) {
-        if (g) cudaGraphDestroy(g);
-        return st;
-      }
-      ALX_TRY(ce, "end capture");
-      cudaGraphExec_t ex = nullptr;
-      const cudaError_t ie = cudaGraphInstantiate(&ex, g, 0);
-      cudaGraphDestroy(g);
-      ALX_TRY(ie, "graph instantiate");
-      it = h->train_graphs.emplace(key, ex).first;
-    }
-    ALX_TRY(cudaGraphLaunch(it->second, s), "graph launch");
-    count_launch_n(h->graph_kernels[key]);
-    if (h->stats_on) h->last_rec = &h->graph_rec[key];
-  } else {
-    h->direct_rec.reset();
-    h->rec = h->stats_on ? &h->direct_rec : nullptr;
-    st = train_bf16(h, nullptr, h->labels_buf, B, nullptr, s, P);
-    h->rec = nullptr;
-    if (h->stats_on) h->last_rec = &h->direct_rec;
-  }
+  const int key = 32 * B + (h->fc_fused ? 4 : 0) + (h->keep ? 2 : 0) + (h->stats_on ? 1 : 0);
+  const alexnet_status st = replay(h, key, s, [&](cudaStream_t cs) {
+    return train_bf16(h, nullptr, h->labels_buf, B, nullptr, cs, P);
+  });
   if (h->stats_on) {
     h->last_launches = launch_counter() - l0;
     h->stats_stream = s;
@@ -1017,6 +1075,98 @@ alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* la
             "train_step loss");
   h->step += 1;
   return cuda_status(h, cudaGetLastError(), "train step");
+}
+
+alexnet_status alexnet_train_grads(alexnet_t* h, const void* x, const int32_t* labels, int B,
+                                   int64_t image_offset, float* loss, void* stream) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  if (!x || !labels || B < 1 || B > h->cfg.batch_max || image_offset < 0 ||
+      image_offset > 0x7FFFFFFF - B) {
+    h->err = "train_grads: invalid argument";
+    return ALEXNET_ERR_INVALID_ARG;
+  }
+  if (h->cfg.dtype != ALEXNET_BF16 || !h->grads) {
+    h->err = "train_grads: needs a bf16 handle created with keep_grads";
+    return ALEXNET_ERR_UNSUPPORTED;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  Plan* P = get_plan(h, B);
+  if (!P) return ALEXNET_ERR_CUDA;
+  if (!P->has_fwg) {
+    h->err = "train_grads: the FC weight gradients do not fit one K-slice at this batch";
+    return ALEXNET_ERR_UNSUPPORTED;
+  }
+  if (!h->fc_event)
+    ALX_TRY(cudaEventCreateWithFlags(&h->fc_event, cudaEventDisableTiming), "fc event");
+  h->grads_only = true;
+  h->row_offset = static_cast<uint32_t>(image_offset);
+  write_hp(h, 0.f, s);
+  launch_s2d(static_cast<const bf16*>(x), h->xs, B, s);
+  alexnet_status st = ALEXNET_OK;
+  cudaError_t e = cudaMemcpyAsync(h->labels_buf, labels, sizeof(int32_t) * B,
+                                  cudaMemcpyDeviceToDevice, s);
+  const bool stats = h->stats_on;
+  h->stats_on = false;
+  // two graphs: forward + FC backward, then the convolutions' backward, with
+  // the FC-gradients event recorded between them
+  const int base = 32 * B + (h->keep ? 2 : 0) + 16;
+  if (e == cudaSuccess)
+    st = replay(h, base, s, [&](cudaStream_t cs) {
+      return train_fc_part(h, nullptr, h->labels_buf, B, nullptr, cs, P);
+    });
+  if (e == cudaSuccess && st == ALEXNET_OK) e = cudaEventRecord(h->fc_event, s);
+  if (e == cudaSuccess && st == ALEXNET_OK)
+    st = replay(h, base + 8, s, [&](cudaStream_t cs) { return train_conv_part(h, B, cs, P); });
+  h->stats_on = stats;
+  h->grads_only = false;
+  h->row_offset = 0;
+  if (e != cudaSuccess) return cuda_status(h, e, "train_grads");
+  if (st != ALEXNET_OK) return st;
+  if (loss)
+    ALX_TRY(cudaMemcpyAsync(loss, h->loss_dev, sizeof(float), cudaMemcpyDeviceToDevice, s),
+            "train_grads loss");
+  return cuda_status(h, cudaGetLastError(), "train_grads");
+}
+
+alexnet_status alexnet_stream_wait_fc_grads(alexnet_t* h, void* stream) {
+  if (!h || !h->fc_event) return ALEXNET_ERR_INVALID_ARG;
+  return cuda_status(h, cudaStreamWaitEvent(static_cast<cudaStream_t>(stream), h->fc_event, 0),
+                     "stream_wait_fc_grads");
+}
+
+alexnet_status alexnet_sgd_range(alexnet_t* h, int64_t offset, int64_t count, const float* g,
+                                 float grad_scale, float lr, void* stream) {
+  if (!h || !g || offset < 0 || count < 0 ||
+      offset + count > static_cast<int64_t>(h->n_params) || !(lr >= 0.f) ||
+      h->cfg.dtype != ALEXNET_BF16)
+    return ALEXNET_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  if (count == 0) return ALEXNET_OK;
+  launch_sgd_range(h->params + offset, h->vel + offset, g, count, grad_scale, lr,
+                   h->cfg.momentum, h->cfg.weight_decay, s);
+  return cuda_status(h, cudaGetLastError(), "sgd_range");
+}
+
+alexnet_status alexnet_params_updated(alexnet_t* h, void* stream) {
+  if (!h || h->cfg.dtype != ALEXNET_BF16) return ALEXNET_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  refresh_shadows(h, s);
+  h->step += 1;
+  return cuda_status(h, cudaGetLastError(), "params_updated");
+}
+
+alexnet_status alexnet_device_buffer(alexnet_t* h, int which, void** ptr, int64_t* count) {
+  if (!h || !ptr || !count) return ALEXNET_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  *count = 0;
+  float* p = which == 0 ? h->params : (which == 1 ? h->vel : (which == 2 ? h->grads : nullptr));
+  if (!p) return ALEXNET_ERR_INVALID_ARG;
+  *ptr = p;
+  *count = static_cast<int64_t>(h->n_params);
+  return ALEXNET_OK;
 }
 
 alexnet_status alexnet_augment(alexnet_t* h, const uint8_t* src, int B, const float* mean,
@@ -1178,6 +1328,7 @@ alexnet_status alexnet_destroy(alexnet_t* h) {
     for (auto& kv : h->graph_rec)
       for (cudaEvent_t e : kv.second.ev) cudaEventDestroy(e);
     for (auto& kv : h->train_graphs) cudaGraphExecDestroy(kv.second);
+    if (h->fc_event) cudaEventDestroy(h->fc_event);
     if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   }
   delete h;
@@ -1231,6 +1382,22 @@ alexnet_status alexnet_stats_read(alexnet_t* h, alexnet_stats* out) {
   out->gemm_launches = R.gemm_launches;
   out->gemm_flops = R.gemm_flops;
   out->gemm_ms = ms;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_debug_canaries(alexnet_t* h, int64_t* bad_bytes) {
+  if (!h || !bad_bytes) return ALEXNET_ERR_INVALID_ARG;
+  *bad_bytes = 0;
+  cudaError_t e = cudaStreamSynchronize(h->last_stream);
+  if (e != cudaSuccess) return cuda_status(h, e, "debug_canaries");
+  std::vector<unsigned char> buf(kCanaryBytes);
+  int64_t bad = 0;
+  for (size_t g : h->guards) {
+    e = cudaMemcpy(buf.data(), h->ws + g, kCanaryBytes, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(h, e, "debug_canaries");
+    for (unsigned char b : buf) bad += b != kCanaryByte;
+  }
+  *bad_bytes = bad;
   return ALEXNET_OK;
 }
 

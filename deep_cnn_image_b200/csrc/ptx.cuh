@@ -229,6 +229,38 @@ __device__ __forceinline__ void tc_mma_k4(uint32_t d_tmem, uint32_t a_lo, uint32
       : "memory");
 }
 
+// The first three MMAs of tc_mma_k4: for a 64-element K block whose last 16
+// elements are known zeros (48 real channels in a 64-channel chunk).
+template <int AS, int BS>
+__device__ __forceinline__ void tc_mma_k3(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                          uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                          uint32_t acc0) {
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p0, p1;\n\t"
+      ".reg .b32 al, bl;\n\t"
+      ".reg .b64 da, db;\n\t"
+      "setp.ne.b32 p0, %6, 0;\n\t"
+      "setp.eq.b32 p1, %6, %6;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p0;\n\t"
+      "add.u32 al, %1, %7;\n\t"
+      "add.u32 bl, %3, %8;\n\t"
+      "mov.b64 da, {al, %2};\n\t"
+      "mov.b64 db, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p1;\n\t"
+      "add.u32 al, %1, %9;\n\t"
+      "add.u32 bl, %3, %10;\n\t"
+      "mov.b64 da, {al, %2};\n\t"
+      "mov.b64 db, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p1;\n\t"
+      "}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc0), "n"(AS), "n"(BS),
+      "n"(2 * AS), "n"(2 * BS)
+      : "memory");
+}
+
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile(

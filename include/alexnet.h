@@ -158,18 +158,6 @@ ALEXNET_API alexnet_status alexnet_augment(alexnet_t* h, const uint8_t* src, int
 ALEXNET_API alexnet_status alexnet_tencrop(alexnet_t* h, const uint8_t* src, int B, const float* mean,
                                float* probs_avg, int32_t* top5, void* stream);
 
-/* Ensemble of networks ([S] "ILSVRC-2012: Single CNN, Ensemble, and
- * Pre-Training Variants": the predictions of several CNNs averaged as the
- * mean of their softmax outputs): each of the n_models handles runs the
- * inference forward on the same batch x, and probs_avg is the mean of their
- * softmax outputs (added in handle order, divided by n_models), top5 its
- * five most probable classes (descending, ties to the lower index).
- *   nets: host array of n_models handles of one dtype, each with
- *   batch_max >= B; x: device [B,227,227,3] in that dtype; probs_avg:
- *   device fp32 [B,1000]; top5: device int32 [B,5]; ws: caller-owned
- *   device scratch of alexnet_ensemble_workspace_bytes(n_models, B) bytes.
- * INVALID_ARG on null pointers, mixed dtypes, B above a handle's batch_max
- * or a scratch too small; otherwise the first failing forward's status. */
 /* Nearest neighbours of feature vectors ([S] "Qualitative Evaluation",
  * Figure 4 right: retrieval by the Euclidean distance between 4096-d
  * last-hidden-layer activations).  For each of Q query rows, the k base rows
@@ -180,7 +168,9 @@ ALEXNET_API alexnet_status alexnet_tencrop(alexnet_t* h, const uint8_t* src, int
  *   aligned); base_sqnorm: nullable device fp32 [N], the base rows' squared
  *   norms (alexnet_knn_sqnorms); dist: device fp32 [Q, k]; idx: device
  *   int32 [Q, k]; ws: caller-owned device scratch of
- *   alexnet_knn_workspace_bytes(Q, N) bytes (holds the Q x N dot products).
+ *   alexnet_knn_workspace_bytes(Q, N) bytes (squared norms and per-block
+ *   candidate lists, about 10 MB: the Q x N distances are never stored --
+ *   the dot-product kernel keeps each query's k best in registers).
  * INVALID_ARG on null pointers, k outside 1..min(32, N), N or D not a
  * multiple of 8, or a scratch too small; UNSUPPORTED if the tensor maps
  * cannot be built (a base pointer not 16-byte aligned). */
@@ -196,11 +186,78 @@ ALEXNET_API alexnet_status alexnet_knn(const void* queries, int Q, const void* b
 ALEXNET_API alexnet_status alexnet_knn_sqnorms(const void* x, int rows, int D, float* out,
                                                void* stream);
 
+/* Ensemble of networks ([S] "ILSVRC-2012: Single CNN, Ensemble, and
+ * Pre-Training Variants": the predictions of several CNNs averaged as the
+ * mean of their softmax outputs): each of the n_models handles runs the
+ * inference forward on the same batch x, and probs_avg is the mean of their
+ * softmax outputs (added in handle order, divided by n_models), top5 its
+ * five most probable classes (descending, ties to the lower index).
+ *   nets: host array of n_models handles of one dtype, each with
+ *   batch_max >= B; x: device [B,227,227,3] in that dtype; probs_avg:
+ *   device fp32 [B,1000]; top5: device int32 [B,5]; ws: caller-owned
+ *   device scratch of alexnet_ensemble_workspace_bytes(n_models, B) bytes.
+ * INVALID_ARG on null pointers, mixed dtypes, B above a handle's batch_max
+ * or a scratch too small; otherwise the first failing forward's status. */
 ALEXNET_API size_t alexnet_ensemble_workspace_bytes(int n_models, int B);
 ALEXNET_API alexnet_status alexnet_ensemble_forward(alexnet_t* const* nets, int n_models,
                                                     const void* x, int B, float* probs_avg,
                                                     int32_t* top5, void* ws, size_t ws_bytes,
                                                     void* stream);
+
+/* Data-parallel training.  The pages train one network split across two
+ * GPUs by its channels ([S] 3.4 "Training on Multiple GPUs"); here each
+ * GPU holds the whole network and the minibatch is split: each rank computes
+ * the gradient of its own images' mean loss, the ranks average the
+ * gradients (a reduce-scatter, issued by the caller with its collective
+ * library), each rank applies the update of [S] 3.4 "Training Procedure
+ * Details" to its own slice of the parameters, and the ranks gather the
+ * updated parameters (an all-gather).  The sequence per step:
+ *   alexnet_train_grads -> (reduce-scatter of the gradients) ->
+ *   alexnet_sgd_range on the rank's slice -> (all-gather of the fp32
+ *   parameters into alexnet_device_buffer(h, 0)) -> alexnet_params_updated.
+ * The momentum is kept per slice: outside its own slice a rank's momentum
+ * values are not updated. */
+
+/* Forward and backward of B images without an update: dL/dparams of the
+ * mean loss over these B images into the handle's gradient buffer
+ * (alexnet_device_buffer(h, 2); blob order).  image_offset: the index of
+ * the first of these images in the whole minibatch; the dropout masks of
+ * [S] 3.4 "Dropout" are drawn for those rows of the whole batch, so the
+ * ranks together draw exactly the masks one handle would draw for the whole
+ * batch.  loss (nullable): device fp32 scalar, the mean over these B images.
+ * The FC layers' gradients (the blob from fc6.W on) are complete before the
+ * convolutions' backward starts: alexnet_stream_wait_fc_grads lets another
+ * stream start reducing them then.  Does not advance the step counter.
+ * UNSUPPORTED unless the handle is bf16 and was created with keep_grads. */
+ALEXNET_API alexnet_status alexnet_train_grads(alexnet_t* h, const void* x, const int32_t* labels,
+                                               int B, int64_t image_offset, float* loss,
+                                               void* stream);
+
+/* Makes `stream` wait until the FC gradients of the last alexnet_train_grads
+ * are complete (call it after that call; INVALID_ARG before any). */
+ALEXNET_API alexnet_status alexnet_stream_wait_fc_grads(alexnet_t* h, void* stream);
+
+/* The update on the parameters [offset, offset + count) of the blob:
+ * v <- momentum v - weight_decay lr w - lr (grad_scale gsum); w <- w + v,
+ * gsum: device fp32 [count] (the sum of the ranks' gradients of this slice;
+ * grad_scale = 1 / ranks gives their mean).  The bf16 operand copies are not
+ * refreshed (alexnet_params_updated does that).  INVALID_ARG for a range
+ * outside the blob, a null gsum or lr < 0. */
+ALEXNET_API alexnet_status alexnet_sgd_range(alexnet_t* h, int64_t offset, int64_t count,
+                                             const float* gsum, float grad_scale, float lr,
+                                             void* stream);
+
+/* After the fp32 parameters have been replaced in place (all-gathered into
+ * alexnet_device_buffer(h, 0)): rebuild the bf16 operand copies the kernels
+ * read and advance the step counter. */
+ALEXNET_API alexnet_status alexnet_params_updated(alexnet_t* h, void* stream);
+
+/* Device address and element count of one of the handle's fp32 arrays in
+ * blob order: which = 0 parameters, 1 momentum, 2 gradients (keep_grads
+ * handles).  The arrays live in the caller's workspace.  INVALID_ARG for an
+ * unknown or absent array. */
+ALEXNET_API alexnet_status alexnet_device_buffer(alexnet_t* h, int which, void** ptr,
+                                                 int64_t* count);
 
 /* Size of the parameter blob: n fp32 parameters, n fp32 momentum values,
  * then the uint64 step counter (8n + 8 bytes).  Parameter order: conv1.W

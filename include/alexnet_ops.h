@@ -65,12 +65,17 @@ ALEXNET_API alexnet_status alexnet_op_conv_wgrad(const void* x, int B, int H, in
  * in a 16 MiB array in this library's own device memory, which every GPU
  * that loads the library holds until the process exits.  Its device address
  * is looked up (cudaGetSymbolAddress) on the first call on each device, so
- * that first call should come before any stream capture.  All calls share
- * the array: calls whose work overlaps on the GPU race and must be ordered
- * by the caller.  Returns ALEXNET_ERR_UNSUPPORTED when even one K-slice of
- * partial sums (Cout * K * K * Cin/groups floats) exceeds the array; splits
- * is reduced to what the array holds.  The pages have no counterpart: this
- * is an integration convenience, not part of the method. */
+ * that first call should come before any stream capture; the look-up is
+ * repeated when the device's context has changed (after cudaDeviceReset).
+ * All calls share the array: calls whose work overlaps on the GPU race and
+ * must be ordered by the caller.  Returns ALEXNET_ERR_UNSUPPORTED when even
+ * one K-slice of partial sums (Cout * K * K * roundup(Cin/groups, 64)
+ * floats: the channels of a tap are padded to a multiple of 64) exceeds the
+ * array; splits is reduced to what the array holds.  The call waits for its
+ * own work before it returns (it reads back the kernel's status word): on
+ * ALEXNET_OK dw holds the result; ALEXNET_ERR_TIMEOUT means a bounded wait
+ * inside the kernel ran out and dw is not valid.  The pages have no
+ * counterpart: this is an integration convenience, not part of the method. */
 ALEXNET_API alexnet_status alexnet_op_conv_wgrad_noalloc(const void* x, int B, int H, int W,
                                                          int Cin, const void* dy, int Cout, int K,
                                                          int pad, int groups, int splits,
@@ -156,17 +161,6 @@ ALEXNET_API alexnet_status alexnet_op_dropout_mask(uint64_t seed, uint32_t layer
 ALEXNET_API alexnet_status alexnet_op_philox(const uint32_t* ctr, const uint32_t* key, int n, uint32_t* out,
                                  void* stream);
 
-/* One internal tensor of the handle's last forward (debug / parity):
- * which = 0..4 conv l+1 output after ReLU, 10/11 LRN1/LRN2 output,
- * 20/21/24 pool1/pool2/pool5 output, 30/31 FC6/FC7 output after dropout,
- * 40 logits (fp32); gradients of the last training step (bf16):
- * 50+l dL/d(pre-activation of conv l+1), 60+l dL/d(pooled map after conv
- * l+1), 70+l dL/d(LRN output of conv l+1), 80 dL/dlogits, 81/82 dL/d(FC7/FC6
- * pre-activation); 90/91/94 the uint8 window choices (argmax) of the pools
- * after conv1/conv2/conv5.  Copies min(bytes, tensor bytes) to dst (host or
- * device).  10/11 and 70/71 hold data only for calls made with
- * alexnet_debug_keep(h, 1): normalisation and pooling run as one fused
- * kernel that otherwise keeps the normalised map and its gradient on chip. */
 /* Which kernel runs convolution `layer` (0..4) for a batch of `batch`
  * images: pass 0 forward, 1 data gradient (layers 1..4), 2 weight gradient.
  * *algo = 1: the shifted-box kernel (one input box per 64-channel chunk for
@@ -198,6 +192,26 @@ ALEXNET_API alexnet_status alexnet_op_wait_probe(int* status, long long limit_cy
  * the switch exists to compare the two. */
 ALEXNET_API alexnet_status alexnet_debug_fc_update(alexnet_t* h, int fused);
 
+/* Bounds evidence without a sanitiser: every buffer the handle carves out of
+ * its workspace is followed by a 256-byte guard region, filled with the byte
+ * 0xA5 by alexnet_create.  This call synchronises the handle's last stream
+ * and stores in *bad_bytes how many guard bytes no longer hold 0xA5: 0
+ * unless some kernel wrote past the end of a workspace buffer.  INVALID_ARG
+ * for a null handle or pointer.  The pages have no counterpart (a debugging
+ * aid). */
+ALEXNET_API alexnet_status alexnet_debug_canaries(alexnet_t* h, int64_t* bad_bytes);
+
+/* One internal tensor of the handle's last forward (debug / parity):
+ * which = 0..4 conv l+1 output after ReLU, 10/11 LRN1/LRN2 output,
+ * 20/21/24 pool1/pool2/pool5 output, 30/31 FC6/FC7 output after dropout,
+ * 40 logits (fp32); gradients of the last training step (bf16):
+ * 50+l dL/d(pre-activation of conv l+1), 60+l dL/d(pooled map after conv
+ * l+1), 70+l dL/d(LRN output of conv l+1), 80 dL/dlogits, 81/82 dL/d(FC7/FC6
+ * pre-activation); 90/91/94 the uint8 window choices (argmax) of the pools
+ * after conv1/conv2/conv5.  Copies min(bytes, tensor bytes) to dst (host or
+ * device).  10/11 and 70/71 hold data only for calls made with
+ * alexnet_debug_keep(h, 1): normalisation and pooling run as one fused
+ * kernel that otherwise keeps the normalised map and its gradient on chip. */
 ALEXNET_API alexnet_status alexnet_debug_copy(alexnet_t* h, int which, void* dst, size_t bytes,
                                   void* stream);
 

@@ -125,6 +125,11 @@ def lib():
                                             ip, POINTER(dp)]),
             "oracle_train_step": (c_double, [netp, dp, dp, dp, i32p, c_int, c_double, c_double,
                                              c_double, c_uint64, c_uint32, dp, dp]),
+            "oracle_train_step_rows": (c_double, [netp, dp, dp, dp, i32p, c_int, c_double,
+                                                  c_double, c_double, c_uint64, c_uint32, c_int,
+                                                  dp, dp]),
+            "oracle_dropout_mask_rows": (None, [c_uint64, c_uint32, c_uint32, c_int, c_int, c_int,
+                                                c_double, u8p]),
             "oracle_loss": (c_double, [netp, dp, dp, i32p, c_int, c_uint64, c_uint32]),
             "oracle_train_probe": (None, [netp, dp, dp, i32p, c_int, c_uint64, c_uint32, c_int,
                                           dp, u8p, u8p, u8p, POINTER(u8p)]),
@@ -167,10 +172,11 @@ def philox4x32_10(ctr, key):
     return [int(v) for v in o]
 
 
-def dropout_mask(seed, layer, step, B, out, p=0.5):
-    """[S] 3.4 "Dropout": keep mask (uint8 0/1) of FC layer 6 or 7."""
+def dropout_mask(seed, layer, step, B, out, p=0.5, row0=0):
+    """[S] 3.4 "Dropout": keep mask (uint8 0/1) of FC layer 6 or 7; row0: the
+    first image's index in the whole minibatch."""
     m = np.zeros((B, out), np.uint8)
-    lib().oracle_dropout_mask(seed, layer, step, B, out, p, _p(m, c_uint8))
+    lib().oracle_dropout_mask_rows(seed, layer, step, row0, B, out, p, _p(m, c_uint8))
     return m
 
 
@@ -466,6 +472,25 @@ def forward_trace(net, params, x, which, mode=1, seed=0, step=0):
     lib().oracle_forward_trace(ctypes.byref(net), pp, xp, B, mode, seed, step, len(which), wv,
                                arr)
     return dict(zip(which, outs))
+
+
+def train_step_rows(net, params, velocity, x, labels, row0, lr=0.01, momentum=0.9, wd=5e-4,
+                    seed=0, step=0):
+    """The step of images row0 .. row0 + B - 1 of a minibatch (their rows of
+    the dropout masks; the loss averaged over these B).  Returns (loss,
+    new_params, new_velocity, grads, logits)."""
+    params = np.array(params, dtype=np.float64, copy=True)
+    velocity = np.array(velocity, dtype=np.float64, copy=True)
+    x, xp = _d(x)
+    labels = np.ascontiguousarray(labels, dtype=np.int32)
+    B = x.shape[0]
+    grads = np.zeros_like(params)
+    logits = np.zeros((B, net.fc_n[2]))
+    loss = lib().oracle_train_step_rows(ctypes.byref(net), _p(params, c_double),
+                                        _p(velocity, c_double), xp, _p(labels, ctypes.c_int32),
+                                        B, lr, momentum, wd, seed, step, row0,
+                                        _p(grads, c_double), _p(logits, c_double))
+    return loss, params, velocity, grads, logits
 
 
 def train_step(net, params, velocity, x, labels, lr=0.01, momentum=0.9, wd=5e-4, seed=0,

@@ -434,17 +434,25 @@ ORACLE_API void oracle_fc_bwd(const double* x, int B, int In, const double* w, i
 /* e = b*Out + j of FC layer `layer` (6 or 7) at training step `step` is      */
 /* word (e & 3) of Philox4x32-10(counter = (e >> 2, layer, step, 0),          */
 /* key = (seed low 32, seed high 32)); the element is kept iff that word is   */
-/* >= round(p * 2^32) (for p = 0.5: iff its top bit is set).                  */
+/* >= round(p * 2^32) (for p = 0.5: iff its top bit is set).  b is the       */
+/* image's index in the whole minibatch: a part of a batch that starts at    */
+/* image row0 draws the rows row0, row0 + 1, ... of the whole batch's mask.   */
 /* ------------------------------------------------------------------------ */
-ORACLE_API void oracle_dropout_mask(uint64_t seed, uint32_t layer, uint32_t step, int B, int Out,
-                                    double p, uint8_t* keep) {
+ORACLE_API void oracle_dropout_mask_rows(uint64_t seed, uint32_t layer, uint32_t step, int row0,
+                                         int B, int Out, double p, uint8_t* keep) {
   const double t = floor(p * 4294967296.0 + 0.5);
   const uint64_t thresh = (uint64_t)t;
-  for (int64_t e = 0; e < (int64_t)B * Out; ++e) {
+  for (int64_t i = 0; i < (int64_t)B * Out; ++i) {
+    const int64_t e = (int64_t)row0 * Out + i;
     uint32_t r[4];
     philox_seeded(seed, (uint32_t)(e >> 2), layer, step, 0u, r);
-    keep[e] = (uint64_t)r[e & 3] >= thresh ? 1 : 0;
+    keep[i] = (uint64_t)r[e & 3] >= thresh ? 1 : 0;
   }
+}
+
+ORACLE_API void oracle_dropout_mask(uint64_t seed, uint32_t layer, uint32_t step, int B, int Out,
+                                    double p, uint8_t* keep) {
+  oracle_dropout_mask_rows(seed, layer, step, 0, B, Out, p, keep);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -612,6 +620,7 @@ typedef struct {
   double* logits;
   const uint8_t* relu_given[7];  /* optional ReLU decisions: conv1..5, FC6, FC7 */
   int keep_pre;                  /* store the pre-activations below */
+  int row0;                      /* index of the first image in the whole minibatch (dropout) */
   double* pre[7];                /* conv1..5, FC6, FC7 before the ReLU (keep_pre only) */
 } fwd_cache;
 
@@ -643,6 +652,7 @@ static void net_forward_given(const oracle_net* net, const double* params, const
 static void net_forward(const oracle_net* net, const double* params, const double* x, int B,
                         int mode, uint64_t seed, uint32_t step, fwd_cache* c) {
   c->keep_pre = 0;
+  c->row0 = 0;
   net_forward_given(net, params, x, B, mode, seed, step, NULL, NULL, c);
 }
 
@@ -673,9 +683,10 @@ static void net_forward_given(const oracle_net* net, const double* params, const
                               int B, int mode, uint64_t seed, uint32_t step,
                               const uint8_t* const* am_in, const uint8_t* const* relu_in,
                               fwd_cache* c) {
-  const int keep_pre = c->keep_pre;
+  const int keep_pre = c->keep_pre, row0 = c->row0;
   memset(c, 0, sizeof(*c));
   c->keep_pre = keep_pre;
+  c->row0 = row0;
   for (int i = 0; i < 7; ++i) c->relu_given[i] = relu_in ? relu_in[i] : NULL;
   net_shapes(net, &c->s);
   const oracle_shapes* s = &c->s;
@@ -742,7 +753,8 @@ static void net_forward_given(const oracle_net* net, const double* params, const
       double* d = dalloc((int64_t)B * Out);
       c->keep[f] = (uint8_t*)calloc((size_t)B * Out, 1);
       if (net->dropout_on && mode == 0) {
-        oracle_dropout_mask(seed, (uint32_t)(6 + f), step, B, Out, net->dropout_p, c->keep[f]);
+        oracle_dropout_mask_rows(seed, (uint32_t)(6 + f), step, c->row0, B, Out, net->dropout_p,
+                                 c->keep[f]);
         for (int64_t e = 0; e < (int64_t)B * Out; ++e) d[e] = c->keep[f][e] ? z[e] : 0.0;
       } else if (net->dropout_on) {
         for (int64_t e = 0; e < (int64_t)B * Out; ++e) d[e] = z[e] * (1.0 - net->dropout_p);
@@ -818,6 +830,7 @@ ORACLE_API void oracle_forward_trace(const oracle_net* net, const double* params
                                      const int* which, double* const* out) {
   fwd_cache c;
   c.keep_pre = 1;
+  c.row0 = 0;
   net_forward_given(net, params, x, B, mode, seed, step, NULL, NULL, &c);
   const oracle_shapes* s = &c.s;
   for (int i = 0; i < n; ++i) {
@@ -845,14 +858,15 @@ static double train_step_probe(const oracle_net* net, double* params, double* ve
                                const double* x, const int32_t* labels, int B, double lr,
                                double momentum, double wd, uint64_t seed, uint32_t step,
                                double* grads, double* logits, int probe, double* probe_out,
-                               const uint8_t* const* am_in, const uint8_t* const* relu_in);
+                               const uint8_t* const* am_in, const uint8_t* const* relu_in,
+                               int row0);
 
 ORACLE_API double oracle_train_step(const oracle_net* net, double* params, double* velocity,
                                     const double* x, const int32_t* labels, int B, double lr,
                                     double momentum, double wd, uint64_t seed, uint32_t step,
                                     double* grads, double* logits) {
   return train_step_probe(net, params, velocity, x, labels, B, lr, momentum, wd, seed, step,
-                          grads, logits, -1, NULL, NULL, NULL);
+                          grads, logits, -1, NULL, NULL, NULL, 0);
 }
 
 /* The same step with the max-pool window choices given (am1, am2, am5 for the
@@ -866,7 +880,19 @@ ORACLE_API double oracle_train_step_given(const oracle_net* net, double* params,
                                           const uint8_t* am5, const uint8_t* const* relu7) {
   const uint8_t* am_in[5] = {am1, am2, NULL, NULL, am5};
   return train_step_probe(net, params, velocity, x, labels, B, lr, momentum, wd, seed, step,
-                          grads, logits, -1, NULL, am_in, relu7);
+                          grads, logits, -1, NULL, am_in, relu7, 0);
+}
+
+/* The step of a part of a minibatch: B images that are images row0 ..
+ * row0 + B - 1 of the whole batch (their dropout draws are those rows of the
+ * whole batch's masks), the loss averaged over these B images.  With
+ * row0 = 0 and the whole batch this is oracle_train_step. */
+ORACLE_API double oracle_train_step_rows(const oracle_net* net, double* params, double* velocity,
+                                         const double* x, const int32_t* labels, int B,
+                                         double lr, double momentum, double wd, uint64_t seed,
+                                         uint32_t step, int row0, double* grads, double* logits) {
+  return train_step_probe(net, params, velocity, x, labels, B, lr, momentum, wd, seed, step,
+                          grads, logits, -1, NULL, NULL, NULL, row0);
 }
 
 /* Intermediate gradients of a training step (no update is kept):
@@ -885,7 +911,7 @@ ORACLE_API void oracle_train_probe(const oracle_net* net, const double* params, 
   double* v = dalloc(s.n_params);
   memcpy(p, params, sizeof(double) * (size_t)s.n_params);
   train_step_probe(net, p, v, x, labels, B, 0.0, 0.0, 0.0, seed, step, NULL, NULL, which, out,
-                   am_in, relu7);
+                   am_in, relu7, 0);
   free(p);
   free(v);
 }
@@ -898,9 +924,11 @@ static double train_step_probe(const oracle_net* net, double* params, double* ve
                                const double* x, const int32_t* labels, int B, double lr,
                                double momentum, double wd, uint64_t seed, uint32_t step,
                                double* grads, double* logits, int probe, double* probe_out,
-                               const uint8_t* const* am_in, const uint8_t* const* relu_in) {
+                               const uint8_t* const* am_in, const uint8_t* const* relu_in,
+                               int row0) {
   fwd_cache c;
   c.keep_pre = 0;
+  c.row0 = row0;
   net_forward_given(net, params, x, B, 0, seed, step, am_in, relu_in, &c);
   const oracle_shapes* s = &c.s;
   const int N = net->fc_n[2];

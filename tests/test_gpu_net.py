@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 from deep_cnn_image_b200 import synthetic
+from tests import _decisions as D
 from tests._gpu import TOL_BF16, TOL_FP32, bf16_round, dev, host, rel_l2
 
 pytestmark = pytest.mark.gpu
@@ -49,15 +50,38 @@ def _make(ax, keep=True, **cfg):
     return net
 
 
-POOLS = ((0, oracle.PROBE_LRN + 0, 55, 96), (1, oracle.PROBE_LRN + 1, 27, 256),
-         (4, oracle.PROBE_RELU + 4, 13, 256))
+def _gpu_maps(net, onet, B):
+    """The GPU's maps of its last training-mode forward, by debug code: conv
+    outputs after the ReLU (0..4), normalised maps (10 + l, where the network
+    normalises; the handle must store them: debug_keep), pooled maps
+    (20 + l), FC6/FC7 outputs after dropout (30, 31) and the window choices
+    (90 + l)."""
+    import torch
+    ms = oracle.map_sizes(onet)
+    want = {}
+    for l in range(5):
+        side, pside, C = ms[l][1], ms[l][2], onet.conv_c[l]
+        want[l] = (B * side * side * C, torch.bfloat16)
+        if onet.pool_after[l]:
+            if onet.lrn_after[l]:
+                want[10 + l] = (B * side * side * C, torch.bfloat16)
+            want[20 + l] = (B * pside * pside * C, torch.bfloat16)
+            want[90 + l] = (B * pside * pside * C, torch.uint8)
+    for f in range(2):
+        want[30 + f] = (B * onet.fc_n[f], torch.bfloat16)
+    out = {}
+    for code, (n, dt) in want.items():
+        t = torch.empty(n, dtype=dt, device="cuda")
+        net.debug_copy(code, t)
+        out[code] = host(t) if dt == torch.bfloat16 else t.cpu().numpy()
+    return out
 
 
 def _gpu_pool_choices(net, B):
     """The GPU's own max-pool window choices of its last forward."""
     import torch
     out = {}
-    for l, _, side, C in POOLS:
+    for l, side, C in ((0, 55, 96), (1, 27, 256), (4, 13, 256)):
         P = (side - 3) // 2 + 1
         t = torch.empty(B * P * P * C, dtype=torch.uint8, device="cuda")
         net.debug_copy(90 + l, t)
@@ -66,62 +90,16 @@ def _gpu_pool_choices(net, B):
     return out
 
 
-CONV_MAPS = ((0, 55, 96), (1, 27, 256), (2, 13, 384), (3, 13, 384), (4, 13, 256))
-
-
-def _gpu_relu_decisions(net, B):
-    """The GPU's ReLU sign decisions of its last forward: unit active iff its
-    stored output is positive (conv1..conv5, then FC6, FC7 after dropout)."""
-    import torch
-    out = {}
-    for l, side, C in CONV_MAPS:
-        t = torch.empty(B * side * side * C, dtype=torch.bfloat16, device="cuda")
-        net.debug_copy(l, t)
-        out[l] = (host(t) > 0).astype(np.uint8)
-    for f in range(2):
-        t = torch.empty(B * 4096, dtype=torch.bfloat16, device="cuda")
-        net.debug_copy(30 + f, t)
-        out[5 + f] = (host(t) > 0).astype(np.uint8)
-    return out
-
-
-def _check_relu_valid(onet, op, xr, relu, seed, step):
-    """Where the GPU's sign decision differs from the oracle's, the unit sits
-    at the ReLU's kink: the active side's value is within 5% of the layer's
-    RMS activation.  Returns the fraction of units decided differently."""
-    flips = []
+def _report(tag, rates):
+    """Decision-disagreement rates, printed (pytest -s shows them) and bounded:
+    local mismatches happen only within fp32 rounding of zero; end-to-end the
+    GPU and the oracle may decide differently only where the oracle's own
+    value is within rounding of the boundary, a small share of the units."""
+    print("%s decisions: %s" % (tag, {k: v for k, v in rates.items()}))
     for l in range(7):
-        which = oracle.PROBE_RELU + l if l < 5 else oracle.PROBE_FC + (l - 5)
-        a = oracle.forward_probe(onet, op, xr, which, mode=0, seed=seed, step=step)
-        mine = (a > 0)
-        theirs = relu[l].ravel().astype(bool)
-        diff = mine != theirs
-        rms = np.sqrt(np.mean(a * a))
-        # oracle active but GPU not: the oracle's value is small
-        assert np.all(a[diff & mine] <= 0.05 * rms), l
-        flips.append(float(diff.mean()))
-    return flips
-
-
-def _check_choices_valid(net, onet, op, xr, choices, seed, step):
-    """The GPU's window choices are exactly the first maxima of the GPU's own
-    pooled-from map (bit-exact on identical inputs), and that map matches the
-    oracle's within the bf16 bound; returns the fraction of windows where the
-    choice is also the oracle's fp64 argmax."""
-    import torch
-    B = xr.shape[0]
-    same = []
-    for l, which, side, C in POOLS:
-        t = torch.empty(B * side * side * C, dtype=torch.bfloat16, device="cuda")
-        net.debug_copy(which, t)
-        gmap = host(t).reshape(B, side, side, C)
-        _, gam = oracle.maxpool_fwd(gmap)
-        np.testing.assert_array_equal(gam, choices[l])
-        m = oracle.forward_probe(onet, op, xr, which, mode=0, seed=seed, step=step)
-        m = m.reshape(B, side, side, C)
-        assert rel_l2(gmap, m) < TOL_BF16, l
-        same.append(float((oracle.maxpool_fwd(m)[1] == choices[l]).mean()))
-    return same
+        local, e2e = rates[l]
+        assert local <= 1e-3, (tag, l, rates[l])
+        assert e2e <= 0.05, (tag, l, rates[l])
 
 
 def test_init_distribution(ax):
@@ -186,14 +164,16 @@ def test_fp32_path_matches_oracle(ax):
     assert rel_l2(host(probs), wp) < TOL_FP32
 
 
-def _train_compare(ax, B, seed, grouped=True, lr=0.01):
+def _train_compare(ax, B, seed, grouped=True, lr=0.01, variant=None):
     """One GPU training step and the oracle's step on the same inputs.  The
     max-pool window choices and the ReLU sign decisions are decisions taken on
-    rounded values: the oracle takes the GPU's own, after checking that each
-    pool choice is the first maximum of the GPU's own map and that every
-    differing sign decision sits at the ReLU's kink."""
+    rounded values: the oracle takes the GPU's own, after tests/_decisions.py
+    has checked every one of them against the rounding bound of the layer's
+    own inputs and against the oracle's own forward.  variant: the pages'
+    ablations as (handle options, oracle network options)."""
     import torch
-    net = _make(ax, batch_max=B, keep_grads=1, grouped=int(grouped), seed=seed)
+    hopts, oopts = variant or ({}, {})
+    net = _make(ax, batch_max=B, keep_grads=1, grouped=int(grouped), seed=seed, **hopts)
     n = ax.param_count(net.cfg)
     params = synthetic.params(seed + 1, grouped=grouped)
     step = 5
@@ -208,15 +188,14 @@ def _train_compare(ax, B, seed, grouped=True, lr=0.01):
     net.get_grads(grads)
     blob = torch.zeros(net.params_bytes() // 4, dtype=torch.float32)
     net.get_params(blob)
-    onet = oracle.alexnet(grouped=grouped)
+    onet = oracle.alexnet(grouped=grouped, **oopts)
     op = _oracle_params(params, onet)
-    choices = _gpu_pool_choices(net, B)
-    _check_choices_valid(net, onet, op, xr, choices, net.cfg.seed, step)
-    relu = _gpu_relu_decisions(net, B)
-    _check_relu_valid(onet, op, xr, relu, net.cfg.seed, step)
-    wloss, _, _, wg, _ = oracle.train_step(onet, op, np.zeros(n), xr, y, lr=lr,
-                                           seed=net.cfg.seed, step=step, given_argmax=choices,
-                                           given_relu=relu)
+    g = _gpu_maps(net, onet, B)
+    choices, relu, rates = D.validate(onet, op, xr, g, net.cfg.seed, step)
+    _report("B=%d %s" % (B, oopts), rates)
+    wloss, wp, wv, wg, _ = oracle.train_step(onet, op, np.zeros(n), xr, y, lr=lr,
+                                             seed=net.cfg.seed, step=step, given_argmax=choices,
+                                             given_relu=relu)
     net.choices = choices
     net.relu = relu
     return net, host(loss)[0], grads.numpy(), blob.numpy(), wloss, wg, params, n, xr, y
@@ -325,29 +304,78 @@ def test_full_batch_forward_sampled(ax):
     assert rel_l2(got[idx], wl) < TOL_BF16
 
 
-def test_full_batch_train_step_properties(ax):
-    """Batch 128: the loss at the pages' initialisation is finite, every
-    gradient is finite, and two identical handles give bit-identical results
-    (the step is deterministic: fixed-order split-K sums, no atomics)."""
+def _block_errors(g, wg, onet):
+    names = ["conv1", "conv2", "conv3", "conv4", "conv5", "fc6", "fc7", "fc8"]
+    errs = {}
+    for l, (wo, wl, bo, bl) in enumerate(oracle.param_layout(onet)):
+        errs[names[l] + ".W"] = rel_l2(g[wo:wo + wl], wg[wo:wo + wl])
+        errs[names[l] + ".b"] = rel_l2(g[bo:bo + bl], wg[bo:bo + bl])
+    return errs
+
+
+def test_full_batch_train_step_matches_oracle(ax):
+    """The benchmark's configuration: one bf16 grouped training step at batch
+    128 with the FC update applied in the weight-gradient epilogue (the
+    default), against the oracle's step on the same inputs ([W] training-step
+    listing; [S] 3.4 "Training Procedure Details": batch 128, the update rule).
+    Every GPU decision is validated first (tests/_decisions.py).  Then a
+    second identical handle must give bit-identical results (fixed-order
+    split-K sums, no atomics), and a handle applying the FC update with the
+    separate kernel bit-identical parameters and gradients."""
     import torch
-    B = 128
-    outs = []
-    for _ in range(2):
-        net = _make(ax, batch_max=B, keep_grads=1, seed=5)
-        x = synthetic.images(6, B)
-        y = synthetic.labels(7, B)
-        xt, _ = synthetic.to_bf16(x)
-        loss = torch.zeros(1, dtype=torch.float32, device="cuda")
-        net.train_step(xt.cuda(), dev(y), B, 0.01, loss)
-        assert net.get_status() == ax.OK
-        g = torch.zeros(ax.param_count(net.cfg), dtype=torch.float32)
-        net.get_grads(g)
-        outs.append((host(loss)[0], g.numpy().copy()))
-        net.close()
-    assert np.isfinite(outs[0][0]) and 0.0 < outs[0][0] < 20.0
-    assert np.all(np.isfinite(outs[0][1]))
-    assert outs[0][0] == outs[1][0]
-    np.testing.assert_array_equal(outs[0][1], outs[1][1])
+    B, seed = 128, 500
+    net, loss, g, blob, wloss, wg, params, n, xr, y = _train_compare(ax, B, seed)
+    print("B=128 loss GPU %.6f oracle %.6f" % (loss, wloss))
+    assert abs(loss - wloss) / wloss < 1e-2
+    errs = _block_errors(g, wg, oracle.alexnet())
+    print("B=128 gradient rel-L2 per block: %s" % errs)
+    bad = {k: v for k, v in errs.items() if not v < TOL_BF16}
+    assert not bad, (bad, errs)
+    w_new, v_new = oracle.sgd(params.astype(np.float64), np.zeros(n), wg, 0.01)
+    assert rel_l2(blob[n:2 * n], v_new) < TOL_BF16
+    assert rel_l2(blob[:n], w_new) < 1e-4
+    assert blob[2 * n:].view(np.uint64)[0] == 6
+    net.close()
+    xt = synthetic.to_bf16(synthetic.images(seed + 2, B))[0].cuda()
+    yt = dev(synthetic.labels(seed + 3, B))
+    for fused in (True, False):
+        other = _make(ax, batch_max=B, keep_grads=1, seed=seed)
+        other.debug_fc_update(fused)
+        other.set_params(_blob(params, n, 5))
+        lo = torch.zeros(1, dtype=torch.float32, device="cuda")
+        other.train_step(xt, yt, B, 0.01, lo)
+        assert other.get_status() == ax.OK
+        g2 = torch.zeros(n, dtype=torch.float32)
+        other.get_grads(g2)
+        b2 = torch.zeros(other.params_bytes() // 4, dtype=torch.float32)
+        other.get_params(b2)
+        assert host(lo)[0] == loss
+        np.testing.assert_array_equal(g2.numpy(), g)
+        np.testing.assert_array_equal(b2.numpy(), blob)
+        other.close()
+
+
+@pytest.mark.parametrize("name,hopts,oopts", [
+    ("nolrn", {"lrn_on": 0}, {"lrn": False}),
+    ("nodropout", {"dropout_on": 0}, {"dropout": False}),
+    ("pool2", {"pool_size": 2}, {"pool_z": 2}),
+    ("ungrouped", {}, {}),
+])
+def test_ablation_train_step_matches_oracle(ax, name, hopts, oopts):
+    """The pages' ablations as network options ([S] 3.4 "Local Response
+    Normalization" (its removal), "Overlapping Pooling" (z = 2, non-overlapping),
+    "Dropout" (off), and the full connectivity of one-GPU training): one
+    training step each against the oracle's network with the same option."""
+    grouped = name != "ungrouped"
+    net, loss, g, blob, wloss, wg, params, n, xr, y = _train_compare(
+        ax, 3, 700 + len(name), grouped=grouped, variant=(hopts, oopts))
+    assert abs(loss - wloss) / wloss < 1e-2
+    errs = _block_errors(g, wg, oracle.alexnet(grouped=grouped, **oopts))
+    bad = {k: v for k, v in errs.items() if not v < TOL_BF16}
+    assert not bad, (name, bad, errs)
+    w_new, v_new = oracle.sgd(params.astype(np.float64), np.zeros(n), wg, 0.01)
+    assert rel_l2(blob[:n], w_new) < 1e-4
+    net.close()
 
 
 def test_resume_is_bit_identical(ax):
