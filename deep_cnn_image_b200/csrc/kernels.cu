@@ -65,6 +65,74 @@ __device__ __forceinline__ void lrn_pow2(float sc, float beta, float& sb, float&
   }
 }
 
+// Channel pairs (2m, 2m + 1) as float2, so that Blackwell's paired fp32
+// instructions (__fadd2_rn, __fmul2_rn, __ffma2_rn) do two channels at once.
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+__device__ __forceinline__ void unpack4x2(const uint4& u, float2 (&p)[4]) {
+  p[0] = bf2_to_f2(u.x);
+  p[1] = bf2_to_f2(u.y);
+  p[2] = bf2_to_f2(u.z);
+  p[3] = bf2_to_f2(u.w);
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float2 v) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Sums over the five-channel window i - 2 .. i + 2 of the eight channels of
+// a unit, from channel pairs P[0] = (c - 2, c - 1), P[1..4] = the unit's
+// pairs, P[5] = (c + 8, c + 9).  With T_q = P[q].x + P[q].y, the window of
+// channel 2m is T_{m} + T_{m+1} + P[m+2].x and that of 2m + 1 is
+// P[m].y + T_{m+1} + T_{m+2} (pair indices of P).
+__device__ __forceinline__ void window5(const float2 (&P)[6], float2 (&out)[4]) {
+  float T[6];
+#pragma unroll
+  for (int q = 0; q < 6; ++q) T[q] = P[q].x + P[q].y;
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+    out[m] = __fadd2_rn(__fadd2_rn(make_float2(T[m], P[m].y), make_float2(T[m + 1], T[m + 1])),
+                        make_float2(P[m + 2].x, T[m + 2]));
+}
+
+// s^-beta and s^-beta-1 of a pair of normalisation scales (see lrn_pow2).
+template <bool B34>
+__device__ __forceinline__ void lrn_pow2x2(float2 sc, float beta, float2& sb, float2& sb1) {
+  if (B34) {
+    const float2 q = make_float2(rsqrt_approx(sc.x), rsqrt_approx(sc.y));
+    const float2 q2 = __fmul2_rn(q, q);
+    sb = __fmul2_rn(q2, make_float2(rsqrt_approx(q.x), rsqrt_approx(q.y)));
+    sb1 = __fmul2_rn(sb, q2);
+  } else {
+    sb = make_float2(__powf(sc.x, -beta), __powf(sc.y, -beta));
+    sb1 = make_float2(__fdividef(sb.x, sc.x), __fdividef(sb.y, sc.y));
+  }
+}
+
+// Normalised values of a unit's eight channels ([S] 3.4 "Local Response
+// Normalization": b_i = a_i (k + alpha sum_{|j - i| <= 2} a_j^2)^-beta), from
+// channel pairs P[0] = (c - 2, c - 1), P[1..4] = the unit, P[5] =
+// (c + 8, c + 9) (zeros outside the layer), packed to bf16.  Shared by the
+// single normalisation kernel and the fused normalisation + pooling one, so
+// the two give bit-identical maps.
+template <bool B34>
+__device__ __forceinline__ uint4 lrn8(const float2 (&P)[6], float2 k2, float2 alpha2, float beta) {
+  float2 sq[6], S[4];
+#pragma unroll
+  for (int q = 0; q < 6; ++q) sq[q] = __fmul2_rn(P[q], P[q]);
+  window5(sq, S);
+  uint4 out;
+  uint32_t* w = &out.x;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    float2 sb, sb1;
+    lrn_pow2x2<B34>(__ffma2_rn(alpha2, S[m], k2), beta, sb, sb1);
+    w[m] = f2_to_bf2(__fmul2_rn(P[1 + m], sb));
+  }
+  return out;
+}
+
 // ------------------------------------------------------------------ hparams
 __global__ void k_write_hparams(HParams* hp, HParams v) { *hp = v; }
 
@@ -131,43 +199,17 @@ __global__ void k_lrn_fwd(const bf16* __restrict__ a, bf16* __restrict__ b, long
     const bf16* ap = a + static_cast<size_t>(p) * C;
     float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (active) unpack8(*reinterpret_cast<const uint4*>(ap + c0), f);
-    float v[12];
+    float2 P[6];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[2 + i] = f[i];
+    for (int m = 0; m < 4; ++m) P[1 + m] = make_float2(f[2 * m], f[2 * m + 1]);
     const float up6 = __shfl_up_sync(0xffffffffu, f[6], 1), up7 = __shfl_up_sync(0xffffffffu, f[7], 1);
     const float dn0 = __shfl_down_sync(0xffffffffu, f[0], 1), dn1 = __shfl_down_sync(0xffffffffu, f[1], 1);
-    v[0] = v[1] = v[10] = v[11] = 0.f;
-    if (active && c0 > 0) {
-      if (lane > 0) {
-        v[0] = up6;
-        v[1] = up7;
-      } else {
-        const float2 lo = ld_bf16x2(ap + c0 - 2);
-        v[0] = lo.x;
-        v[1] = lo.y;
-      }
-    }
-    if (active && c0 + 8 < C) {
-      if (lane < 31) {
-        v[10] = dn0;
-        v[11] = dn1;
-      } else {
-        const float2 hi = ld_bf16x2(ap + c0 + 8);
-        v[10] = hi.x;
-        v[11] = hi.y;
-      }
-    }
+    P[0] = P[5] = make_float2(0.f, 0.f);
+    if (active && c0 > 0) P[0] = lane > 0 ? make_float2(up6, up7) : ld_bf16x2(ap + c0 - 2);
+    if (active && c0 + 8 < C) P[5] = lane < 31 ? make_float2(dn0, dn1) : ld_bf16x2(ap + c0 + 8);
     if (!active) continue;
-    float o[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float sum = 0.f;
-#pragma unroll
-      for (int j = 0; j < 5; ++j) sum += v[i + j] * v[i + j];
-      const float sc = k + alpha * sum;
-      o[i] = v[i + 2] * lrn_pow<B34>(sc, beta);
-    }
-    *reinterpret_cast<uint4*>(b + static_cast<size_t>(p) * C + c0) = pack8(o);
+    *reinterpret_cast<uint4*>(b + static_cast<size_t>(p) * C + c0) =
+        lrn8<B34>(P, make_float2(k, k), make_float2(alpha, alpha), beta);
   }
 }
 
@@ -444,32 +486,14 @@ __global__ void __launch_bounds__(256) k_lrn_pool_fwd(const bf16* __restrict__ a
     const int r = (u >> 2) / W;
     const int c0 = cs + j * 8;
     const bf16* ap = a + ((static_cast<size_t>(b) * H + r0 + r) * W + x) * C + c0;
-    float v[12];
     float f[8];
     unpack8(*reinterpret_cast<const uint4*>(ap), f);
+    float2 P[6];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[2 + i] = f[i];
-    v[0] = v[1] = v[10] = v[11] = 0.f;
-    if (c0 > 0) {
-      const float2 l2 = ld_bf16x2(ap - 2);
-      v[0] = l2.x;
-      v[1] = l2.y;
-    }
-    if (c0 + 8 < C) {
-      const float2 h2 = ld_bf16x2(ap + 8);
-      v[10] = h2.x;
-      v[11] = h2.y;
-    }
-    float o[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float sum = 0.f;
-#pragma unroll
-      for (int q = 0; q < 5; ++q) sum += v[i + q] * v[i + q];
-      const float sc = k + alpha * sum;
-      o[i] = v[i + 2] * lrn_pow<B34>(sc, beta);
-    }
-    const uint4 packed = pack8(o);
+    for (int m = 0; m < 4; ++m) P[1 + m] = make_float2(f[2 * m], f[2 * m + 1]);
+    P[0] = c0 > 0 ? ld_bf16x2(ap - 2) : make_float2(0.f, 0.f);
+    P[5] = c0 + 8 < C ? ld_bf16x2(ap + 8) : make_float2(0.f, 0.f);
+    const uint4 packed = lrn8<B34>(P, make_float2(k, k), make_float2(alpha, alpha), beta);
     lds[(r * W + x) * 4 + j] = packed;
     if (lo && r0 + r < own1)
       *reinterpret_cast<uint4*>(lo + ((static_cast<size_t>(b) * H + r0 + r) * W + x) * C + c0) =
@@ -522,17 +546,17 @@ __global__ void __launch_bounds__(256) k_lrn_pool_fwd(const bf16* __restrict__ a
 // sign-replicating byte permutes widen each byte's flag to its channel's 16
 // bits; the gradient is kept where the flag is clear.
 __device__ __forceinline__ void add_routed8(const uint4& dyv, const uint2& amv, uint32_t off,
-                                            float (&g)[8]) {
+                                            float2 (&g)[4]) {
   const uint32_t rep = off * 0x01010101u;
   const uint32_t x0 = amv.x ^ rep, x1 = amv.y ^ rep;
   const uint32_t n0 = ((x0 & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x0;
   const uint32_t n1 = ((x1 & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x1;
   const uint4 kept = make_uint4(dyv.x & ~prmt(n0, 0, 0x9988), dyv.y & ~prmt(n0, 0, 0xBBAA),
                                 dyv.z & ~prmt(n1, 0, 0x9988), dyv.w & ~prmt(n1, 0, 0xBBAA));
-  float f[8];
-  unpack8_bits(kept, f);
+  float2 f[4];
+  unpack4x2(kept, f);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) g[i] += f[i];
+  for (int m = 0; m < 4; ++m) g[m] = __fadd2_rn(g[m], f[m]);
 }
 
 // Backward of normalisation + pooling, fused: the pooled gradient is routed
@@ -550,9 +574,9 @@ __device__ __forceinline__ void add_routed8(const uint4& dyv, const uint2& amv, 
 // window order.  The normalisation's channel window reaches two channels
 // into the neighbouring units; those edge values (a, then the cross terms
 // t_i = g_i a_i s_i^(-beta-1)) go through shared memory, one quad row at a
-// time.  Arithmetic of the normalisation as k_lrn_bwd.  Per block the
-// column sums of the stored da (the layer's bias gradient) are written to
-// bias_part[blockIdx.x][C] (nullable).
+// time.  The arithmetic works on channel pairs with paired fp32
+// instructions.  Per block the column sums of the stored da (the layer's
+// bias gradient) are written to bias_part[blockIdx.x][C] (nullable).
 template <int ZC, int WC, bool B34>
 __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ dy,
                                                       const uint8_t* __restrict__ am,
@@ -571,12 +595,15 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
   const int uj = threadIdx.x - up * CH;
   const bool mine = up < nq;
   const int tid = threadIdx.x;
-  // edge values of every thread's unit (channels 0, 1, 6, 7), per quad
+  // edge pairs of every thread's unit (channels 0, 1 and 6, 7), per quad
   // column: normalisation inputs (ea) and cross terms (et)
   __shared__ float4 ea[2][256], et[2][256];
   __shared__ float red[256 * 8];
-  const float c2ab = 2.f * alpha * beta;
-  float bsum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const float2 k2 = make_float2(k, k), alpha2 = make_float2(alpha, alpha);
+  const float2 mc2ab = make_float2(-2.f * alpha * beta, -2.f * alpha * beta);
+  float2 bsum[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) bsum[m] = make_float2(0.f, 0.f);
   for (int blk = blockIdx.x; blk * nq < nquads; blk += gridDim.x) {
     const int q = blk * nq + up;
     const bool live = mine && q < nquads;
@@ -605,18 +632,18 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int ih = 2 * qi + h;
-      float g[2][8], av[2][8];
+      float2 g[2][4], av[2][4];
       bool pv[2];
 #pragma unroll
       for (int d = 0; d < 2; ++d) {
         const int iw = 2 * qj + d;
         pv[d] = live && ih < H && iw < W;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) g[d][i] = av[d][i] = 0.f;
+        for (int m = 0; m < 4; ++m) g[d][m] = av[d][m] = make_float2(0.f, 0.f);
         if (pv[d]) {
-          unpack8(*reinterpret_cast<const uint4*>(
-                      a + static_cast<uint32_t>((b * H + ih) * W + iw) * C + uj * 8),
-                  av[d]);
+          unpack4x2(*reinterpret_cast<const uint4*>(
+                        a + static_cast<uint32_t>((b * H + ih) * W + iw) * C + uj * 8),
+                    av[d]);
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             const int rr = h + 2 - 2 * (w >> 1), rc = d + 2 - 2 * (w & 1);
@@ -624,33 +651,28 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
               add_routed8(wdy[w], wam[w], static_cast<uint32_t>(rr * z + rc), g[d]);
           }
         }
-        ea[d][tid] = make_float4(av[d][0], av[d][1], av[d][6], av[d][7]);
+        ea[d][tid] = make_float4(av[d][0].x, av[d][0].y, av[d][3].x, av[d][3].y);
       }
       __syncthreads();
-      float first[2][8], tv[2][8];
+      float2 first[2][4], tv[2][4];
 #pragma unroll
       for (int d = 0; d < 2; ++d) {
         const float4 L = mine && uj > 0 ? ea[d][tid - 1] : make_float4(0.f, 0.f, 0.f, 0.f);
         const float4 R = mine && uj < CH - 1 ? ea[d][tid + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
-        float w12[12];
-        w12[0] = L.z;
-        w12[1] = L.w;
+        float2 sq[6], S[4];
+        sq[0] = __fmul2_rn(make_float2(L.z, L.w), make_float2(L.z, L.w));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w12[2 + i] = av[d][i];
-        w12[10] = R.x;
-        w12[11] = R.y;
+        for (int m = 0; m < 4; ++m) sq[1 + m] = __fmul2_rn(av[d][m], av[d][m]);
+        sq[5] = __fmul2_rn(make_float2(R.x, R.y), make_float2(R.x, R.y));
+        window5(sq, S);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float sum = 0.f;
-#pragma unroll
-          for (int j = 0; j < 5; ++j) sum += w12[i + j] * w12[i + j];
-          const float sc = k + alpha * sum;
-          float sb, sb1;
-          lrn_pow2<B34>(sc, beta, sb, sb1);
-          first[d][i] = g[d][i] * sb;
-          tv[d][i] = g[d][i] * av[d][i] * sb1;
+        for (int m = 0; m < 4; ++m) {
+          float2 sb, sb1;
+          lrn_pow2x2<B34>(__ffma2_rn(alpha2, S[m], k2), beta, sb, sb1);
+          first[d][m] = __fmul2_rn(g[d][m], sb);
+          tv[d][m] = __fmul2_rn(__fmul2_rn(g[d][m], av[d][m]), sb1);
         }
-        et[d][tid] = make_float4(tv[d][0], tv[d][1], tv[d][6], tv[d][7]);
+        et[d][tid] = make_float4(tv[d][0].x, tv[d][0].y, tv[d][3].x, tv[d][3].y);
       }
       __syncthreads();
 #pragma unroll
@@ -658,30 +680,34 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
         const float4 L = mine && uj > 0 ? et[d][tid - 1] : make_float4(0.f, 0.f, 0.f, 0.f);
         const float4 R = mine && uj < CH - 1 ? et[d][tid + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
         if (!pv[d]) continue;
-        float w12[12];
-        w12[0] = L.z;
-        w12[1] = L.w;
+        float2 tp[6], cross[4];
+        tp[0] = make_float2(L.z, L.w);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w12[2 + i] = tv[d][i];
-        w12[10] = R.x;
-        w12[11] = R.y;
-        float o[8];
+        for (int m = 0; m < 4; ++m) tp[1 + m] = tv[d][m];
+        tp[5] = make_float2(R.x, R.y);
+        window5(tp, cross);
+        uint4 packed;
+        uint32_t* pw = &packed.x;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float cross = 0.f;
-#pragma unroll
-          for (int j = 0; j < 5; ++j) cross += w12[i + j];
-          const float aj = av[d][i];
-          o[i] = aj > 0.f ? first[d][i] - c2ab * aj * cross : 0.f;
+        for (int m = 0; m < 4; ++m) {
+          const float2 dd = __ffma2_rn(mc2ab, __fmul2_rn(av[d][m], cross[m]), first[d][m]);
+          pw[m] = f2_to_bf2(make_float2(av[d][m].x > 0.f ? dd.x : 0.f,
+                                        av[d][m].y > 0.f ? dd.y : 0.f));
         }
-        const uint4 packed = pack8(o);
         const uint32_t e = static_cast<uint32_t>((b * H + ih) * W + 2 * qj + d) * C + uj * 8;
         *reinterpret_cast<uint4*>(da + e) = packed;
-        if (dl) *reinterpret_cast<uint4*>(dl + e) = pack8(g[d]);
-        float r[8];
-        unpack8(packed, r);
+        if (dl) {
+          uint4 gp;
+          gp.x = f2_to_bf2(g[d][0]);
+          gp.y = f2_to_bf2(g[d][1]);
+          gp.z = f2_to_bf2(g[d][2]);
+          gp.w = f2_to_bf2(g[d][3]);
+          *reinterpret_cast<uint4*>(dl + e) = gp;
+        }
+        float2 r[4];
+        unpack4x2(packed, r);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) bsum[i] += r[i];
+        for (int m = 0; m < 4; ++m) bsum[m] = __fadd2_rn(bsum[m], r[m]);
       }
     }
   }
@@ -689,7 +715,10 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
   // per-channel sum over the block's quad slots, in slot order
   if (mine) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) red[up * C + uj * 8 + i] = bsum[i];
+    for (int m = 0; m < 4; ++m) {
+      red[up * C + uj * 8 + 2 * m] = bsum[m].x;
+      red[up * C + uj * 8 + 2 * m + 1] = bsum[m].y;
+    }
   }
   __syncthreads();
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
