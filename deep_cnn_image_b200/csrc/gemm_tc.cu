@@ -35,6 +35,11 @@ constexpr int BK = 64;
 constexpr int NUM_THREADS = 320;
 constexpr int A_TILE_BYTES = BM * BK * 2;
 constexpr int MN_BLOCK_BYTES = 64 * 128;  // 64 K-rows x 64 MN elements (bf16)
+// EPI_SGD_T: per epilogue warp, SGD_NBUF chunks of 16 columns x 32 rows of
+// the fp32 weights and momenta staged in shared memory by cp.async
+constexpr int SGD_NBUF = 3;
+constexpr int SGD_CHUNK_FLOATS = 16 * 32;
+constexpr int SGD_STAGE_BYTES = 8 * SGD_NBUF * 2 * SGD_CHUNK_FLOATS * 4;  // 96 KB
 
 __host__ __device__ constexpr int tmem_cols_for(int bn) {
   return 2 * bn <= 32 ? 32 : (2 * bn <= 64 ? 64 : (2 * bn <= 128 ? 128 : (2 * bn <= 256 ? 256 : 512)));
@@ -118,42 +123,10 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, const TileCoor
   }
 }
 
-// EPI_SGD_T, [S] 3.4 "Training Procedure Details" update rule (sgd_one).
-// A thread owns one row (input feature) of the tile and walks its columns
-// (output units) 16 at a time.  For a fixed column the 32 lanes of a warp
-// touch 32 consecutive parameters, so every access is one 128-byte line per
-// warp.  The loads of the next 16 columns are issued before the current
-// ones are updated, so 32 to 64 loads per thread stay in flight.
-__device__ __forceinline__ void sgd_load16(const GemmArgs& a, size_t base, int nc,
-                                           float (&wv)[16], float (&vv)[16]) {
-  const uint32_t ld = static_cast<uint32_t>(a.ld_out);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    wv[i] = 0.f;
-    vv[i] = 0.f;
-    if (i < nc) {
-      wv[i] = a.sgd_w[base + i * ld];
-      vv[i] = a.sgd_v[base + i * ld];
-    }
-  }
-}
-__device__ __forceinline__ void sgd_apply16(const GemmArgs& a, const HParams& hp, size_t base,
-                                            int nc, float (&wv)[16], float (&vv)[16],
-                                            uint32_t taddr) {
-  const uint32_t ld = static_cast<uint32_t>(a.ld_out);
-  float g[16];
-  tmem_ld16(taddr, g);  // every lane takes part (warp-wide load)
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if (i < nc) {
-      sgd_one(wv[i], vv[i], g[i], hp);
-      a.sgd_w[base + i * ld] = wv[i];
-      a.sgd_v[base + i * ld] = vv[i];
-      a.sgd_shadow[base + i * ld] = __float2bfloat16_rn(wv[i]);
-      if (a.sgd_grads) a.sgd_grads[base + i * ld] = g[i];
-    }
-  }
-}
+// EPI_SGD_T: [S] 3.4 "Training Procedure Details" update rule (sgd_one)
+// applied in the epilogue to the parameters whose gradients the tile holds
+// (rows = input features, columns = output units of an [Out][In] matrix);
+// see the epilogue below for the staging of w and v.
 
 template <int BN, int ASRC, int BSRC>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -178,6 +151,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t bar_acc_empty = bar_acc_full + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * stages + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // EPI_SGD_T staging, after the barriers (whose region is under 256 bytes)
+  uint8_t* sgd_stage = smem + stages * (A_TILE_BYTES + B_TILE_BYTES) + 256;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -344,22 +319,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * (TMEM_COLS / 2);
       if (kSgd && args.epi == EPI_SGD_T) {
-        // each half of the warps takes a contiguous half of the columns
-        const bool live = row < args.M;
+        // each half of the warps takes a contiguous half of the columns, in
+        // chunks of 16; a chunk's w and v (16 lines of 128 bytes each: the 32
+        // rows of this warp) arrive in shared memory by cp.async SGD_NBUF - 1
+        // chunks ahead, so many lines are in flight without holding registers
+        const int cb = half * (BN / 2);
+        constexpr int nchunks = BN / 2 / 16;
+        const int row_base = tc.m_t * BM + quarter * 32;
         const size_t ld = static_cast<size_t>(args.ld_out);
-        auto base_of = [&](int c0) {
-          return static_cast<size_t>(tc.n_t * BN + c0) * ld + (live ? row : 0);
+        float* sw = reinterpret_cast<float*>(sgd_stage) + warp * (SGD_NBUF * 2 * SGD_CHUNK_FLOATS);
+        auto issue = [&](int c) {
+          const int buf = c % SGD_NBUF;
+          float* dw = sw + buf * 2 * SGD_CHUNK_FLOATS;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int pidx = lane + 32 * t;
+            const int col = pidx >> 3, part = pidx & 7;
+            const int o = tc.n_t * BN + cb + 16 * c + col;
+            if (o < args.N && row_base < args.M) {  // M % 32 == 0: all 32 rows exist
+              const size_t src = static_cast<size_t>(o) * ld + row_base + part * 4;
+              cp_async16(smem_u32(dw + col * 32 + part * 4), args.sgd_w + src);
+              cp_async16(smem_u32(dw + SGD_CHUNK_FLOATS + col * 32 + part * 4), args.sgd_v + src);
+            }
+          }
+          cp_async_commit();
         };
-        auto nc_of = [&](int c0) { return live ? min(16, args.N - (tc.n_t * BN + c0)) : 0; };
-        const int cb = half * (BN / 2), ce = cb + BN / 2;  // (BN / 2) % 32 == 0
-        float wa[16], va[16], wb[16], vb[16];
-        sgd_load16(args, base_of(cb), nc_of(cb), wa, va);
+        const bool live = row < args.M;
 #pragma unroll 1
-        for (int c0 = cb; c0 < ce; c0 += 32) {
-          sgd_load16(args, base_of(c0 + 16), nc_of(c0 + 16), wb, vb);
-          sgd_apply16(args, hp, base_of(c0), nc_of(c0), wa, va, tbase + c0);
-          if (c0 + 32 < ce) sgd_load16(args, base_of(c0 + 32), nc_of(c0 + 32), wa, va);
-          sgd_apply16(args, hp, base_of(c0 + 16), nc_of(c0 + 16), wb, vb, tbase + c0 + 16);
+        for (int c = 0; c < nchunks; ++c) {
+          if (c == 0) {
+#pragma unroll
+            for (int q = 0; q < SGD_NBUF - 1; ++q) {
+              if (q < nchunks) issue(q);
+              else cp_async_commit();
+            }
+          }
+          if (c + SGD_NBUF - 1 < nchunks) issue(c + SGD_NBUF - 1);
+          else cp_async_commit();
+          cp_async_wait<SGD_NBUF - 1>();
+          __syncwarp();
+          const float* srcw = sw + (c % SGD_NBUF) * 2 * SGD_CHUNK_FLOATS;
+          float g[16];
+          tmem_ld16(tbase + cb + 16 * c, g);  // every lane takes part (warp-wide load)
+          const int o0 = tc.n_t * BN + cb + 16 * c;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (live && o0 + i < args.N) {
+              float wv = srcw[i * 32 + lane], vv = srcw[SGD_CHUNK_FLOATS + i * 32 + lane];
+              sgd_one(wv, vv, g[i], hp);
+              const size_t e = static_cast<size_t>(o0 + i) * ld + row;
+              args.sgd_w[e] = wv;
+              args.sgd_v[e] = vv;
+              args.sgd_shadow[e] = __float2bfloat16_rn(wv);
+              if (args.sgd_grads) args.sgd_grads[e] = g[i];
+            }
+          }
+          __syncwarp();  // the buffer is refilled next
         }
       } else {
 #pragma unroll 1
@@ -520,12 +535,17 @@ bool gemm_finalize(GemmDesc* d, int num_sms) {
   if (a.kb_per_split <= 0 || a.kb_per_split > a.Kblocks) a.kb_per_split = a.Kblocks;
   a.splits = (a.Kblocks + a.kb_per_split - 1) / a.kb_per_split;
   const int stage_bytes = A_TILE_BYTES + d->bn * BK * 2;
-  const int budget = 227 * 1024 - 1024 - 256;
+  // the in-place update stages its fp32 weights and momenta (rows in
+  // 16-byte pieces: M % 32 == 0 keeps every piece inside the matrix)
+  const bool sgd = a.epi == EPI_SGD_T;
+  if (sgd && a.M % 32) return false;
+  const int extra = sgd ? SGD_STAGE_BYTES : 0;
+  const int budget = 227 * 1024 - 1024 - 256 - extra;
   int stages = budget / stage_bytes;
   if (stages > 8) stages = 8;
-  if (stages < 3) return false;
+  if (stages < (sgd ? 2 : 3)) return false;
   d->stages = stages;
-  d->smem = stages * stage_bytes + 1024 + 256;
+  d->smem = stages * stage_bytes + 1024 + 256 + extra;
   const long long tiles = 1LL * a.m_tiles * a.n_tiles * a.splits * a.groups;
   d->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   return true;

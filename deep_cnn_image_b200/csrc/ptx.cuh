@@ -160,6 +160,21 @@ __device__ __forceinline__ void tma_load_im2col_4d(uint32_t dst, const void* tma
       : "memory");
 }
 
+// ---------------------------------------------------------------- cp.async
+// 16-byte asynchronous copy global -> shared (L2 only), and its groups:
+// a thread's copies complete in commit order; wait_group<n> returns once at
+// most n of this thread's groups are still in flight.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -259,6 +274,25 @@ __device__ __forceinline__ void tc_mma_k3(uint32_t d_tmem, uint32_t a_lo, uint32
       "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc0), "n"(AS), "n"(BS),
       "n"(2 * AS), "n"(2 * BS)
       : "memory");
+}
+
+// Eight (KS = 4) or six (KS = 3) MMAs: K steps k = 0 .. KS-1 into two
+// accumulators d0 / d1 (A operands a0 / a1, one shared B), alternating
+// between them, so that consecutive MMAs never accumulate into the same
+// tensor memory.  acc0 = 0 overwrites both accumulators with the first
+// products.
+template <int AS, int BS, int KS>
+__device__ __forceinline__ void tc_mma_x2(uint32_t d0, uint32_t d1, uint32_t a0_lo, uint32_t a1_lo,
+                                          uint32_t a_hi, uint32_t b_lo, uint32_t b_hi,
+                                          uint32_t idesc, uint32_t acc0) {
+#pragma unroll
+  for (int k = 0; k < KS; ++k) {
+    const uint64_t a0 = (static_cast<uint64_t>(a_hi) << 32) | (a0_lo + k * AS);
+    const uint64_t a1 = (static_cast<uint64_t>(a_hi) << 32) | (a1_lo + k * AS);
+    const uint64_t b = (static_cast<uint64_t>(b_hi) << 32) | (b_lo + k * BS);
+    tc_mma_f16(d0, a0, b, idesc, k == 0 ? acc0 : 1u);
+    tc_mma_f16(d1, a1, b, idesc, k == 0 ? acc0 : 1u);
+  }
 }
 
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
