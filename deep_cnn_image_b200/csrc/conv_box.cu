@@ -27,6 +27,10 @@ constexpr int kThreads = 320;
 constexpr int kSmemBudget = 227 * 1024;
 constexpr int kBarBytes = 3072;  // mbarriers, tmem slot, abort flag (first 512 B); staged bias
 constexpr int kMaxBias = (kBarBytes - 512) / 4;
+// swapped tiles: per epilogue warp, a staging area for one 32-position chunk
+// of 32 bf16 channels, after the barrier block
+constexpr int kStageWarp = 32 * 32 * 2;
+constexpr int kStageBytes = 8 * kStageWarp;
 
 __host__ __device__ constexpr int pow2_cols(int n) {
   return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : (n <= 256 ? 256 : 512)));
@@ -48,15 +52,24 @@ __device__ __forceinline__ void zero_smem(uint8_t* p, int bytes) {
 // ---------------------------------------------------------------- forward
 // Tile t = ((g * B + b) * tiles_img + ti) * n_tiles + n_t: output rows
 // ti * To_h .. of image b, output channels n_t * BN .. of group g.
-template <int BN, int NSUB, int BMN>
+// SW = 1 swaps the roles: M = the BN (128, or 64 for a data gradient read
+// from the forward weights) output channels (the weight slab is the A
+// operand), N = the tile's box positions, a.sw_n <= 256 (the shifted box is
+// the B operand), so one MMA does BN x sw_n x 16 instead of two
+// 128 x BN x 16 ones; the accumulator holds channels in its lanes and
+// positions in its columns.  With M = 64, accumulator row r sits in lane
+// 32 * (r / 16) + r % 16.
+template <int BN, int NSUB, int BMN, int SW = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_box_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ BoxArgs a, int stA, int stB, int a_bytes, int tps) {
   constexpr int B_BYTES = BN * 128;  // one tap's weight slab; a B stage holds tps of them
-  constexpr int ACC_BUFS = (2 * NSUB * BN <= 512) ? 2 : 1;
-  constexpr int TMEM_COLS = pow2_cols(ACC_BUFS * NSUB * BN);
-  constexpr uint32_t IDESC = idesc_bf16(128, BN, 0, BMN);
+  constexpr int ACC_COLS = SW ? 128 * NSUB : NSUB * BN;
+  constexpr int ACC_BUFS = (2 * ACC_COLS <= 512) ? 2 : 1;
+  constexpr int TMEM_COLS = pow2_cols(ACC_BUFS * ACC_COLS);
   static_assert(!BMN || BN % 64 == 0, "MN-major weights come in 64-channel blocks");
+  static_assert(!SW || (NSUB == 2 && (BN == 128 || (BN == 64 && BMN))),
+                "swapped tiles: 128 (or 64 MN-major) channels x up to 256 positions");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -172,6 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // their start-address field: a single issuing thread cannot afford to
     // rebuild two 64-bit descriptors per MMA.
     if (lane == 0) {
+      const uint32_t IDESC = SW ? idesc_bf16(BN, a.sw_n, BMN, 0) : idesc_bf16(128, BN, 0, BMN);
       const uint64_t adesc0 = smem_desc_sw128(sA, 16, 1024);
       const uint64_t bdesc0 = BMN ? smem_desc_sw128(sB, 8192, 1024) : smem_desc_sw128(sB, 16, 1024);
       const uint32_t a_lo0 = static_cast<uint32_t>(adesc0), a_hi = static_cast<uint32_t>(adesc0 >> 32);
@@ -186,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t aph = ACC_BUFS == 2 ? ((tcount >> 1) & 1) : (tcount & 1);
         if (!mbar_wait(acc_empty + 8 * acc, aph ^ 1, a.status, abort_flag)) break;
         tc_fence_after();
-        const uint32_t dbase = tmem_base + acc * NSUB * BN;
+        const uint32_t dbase = tmem_base + acc * ACC_COLS;
         for (int ch = 0; ch < a.cpt && ok; ++ch, ra.next(stA)) {
           const int s = ra.slot;
           if (!mbar_wait(a_full + 8 * s, ra.phase, a.status, abort_flag)) {
@@ -211,15 +225,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool k3 = !BMN && ch == a.cpt - 1 && a.k16_last == 3;
             for (int j = 0; j < n; ++j) {
               const uint32_t acc0 = (ch == 0 && tap0 + j == 0) ? 0u : 1u;
-#pragma unroll
-              for (int sub = 0; sub < NSUB; ++sub) {
+              const uint32_t bj = bst + j * (B_BYTES >> 4);
+              if (SW) {
+                // A = the tap's weight slab (K-major, or MN-major for the data
+                // gradient), B = the box at the tap's shift
                 if (k3)
-                  tc_mma_k3<2, 2>(dbase + sub * BN, abox + shift + sub * (128 * 128 / 16), a_hi,
-                                  bst + j * (B_BYTES >> 4), b_hi, IDESC, acc0);
+                  tc_mma_k3<2, 2>(dbase, bj, b_hi, abox + shift, a_hi, IDESC, acc0);
                 else
-                  tc_mma_k4<2, BMN ? 128 : 2>(dbase + sub * BN,
-                                              abox + shift + sub * (128 * 128 / 16), a_hi,
-                                              bst + j * (B_BYTES >> 4), b_hi, IDESC, acc0);
+                  tc_mma_k4<BMN ? 128 : 2, 2>(dbase, bj, b_hi, abox + shift, a_hi, IDESC, acc0);
+              } else if (NSUB == 2) {
+                // the two sub-tiles' accumulators alternate MMA by MMA: a
+                // 128-row MMA that accumulates into the tensor memory the
+                // previous one wrote waits for it, about 106 clocks for
+                // N <= 192 (measured), longer than the MMA itself
+                const uint32_t a0 = abox + shift, a1 = a0 + (128 * 128 / 16);
+                if (k3)
+                  tc_mma_x2<2, 2, 3>(dbase, dbase + BN, a0, a1, a_hi, bj, b_hi, IDESC, acc0);
+                else
+                  tc_mma_x2<2, BMN ? 128 : 2, 4>(dbase, dbase + BN, a0, a1, a_hi, bj, b_hi, IDESC,
+                                                 acc0);
+              } else {
+                if (k3)
+                  tc_mma_k3<2, 2>(dbase, abox + shift, a_hi, bj, b_hi, IDESC, acc0);
+                else
+                  tc_mma_k4<2, BMN ? 128 : 2>(dbase, abox + shift, a_hi, bj, b_hi, IDESC, acc0);
               }
               if (++kw == a.K) {
                 kw = 0;
@@ -255,6 +284,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(acc_full + 8 * acc, aph, a.status, abort_flag)) break;
       tc_fence_after();
       const int quarter = warp & 3, half = warp >> 2;
+      if constexpr (SW) {
+        // lane = output channel, columns = positions: this warp's CW = 32
+        // (M = 64: 16) channels at the 128 positions of its half, 32
+        // positions per chunk.  A chunk goes through the warp's staging
+        // area transposed (position-major rows of CW bf16 channels), so the
+        // global stores are 16-byte vectors of eight channels.
+        constexpr int CW = BN == 64 ? 16 : 32;
+        constexpr int PIECES = CW / 8;  // 16-byte pieces per position
+        const int nw = n_t * BN + quarter * CW;  // the warp's first channel
+        const int n = nw + lane;
+        const bool cvalid = lane < CW && n < a.Og;
+        const float bv = (a.bias && cvalid) ? sbias[static_cast<long long>(g) * a.col_goff + n] : 0.f;
+        uint8_t* stg = barp + kBarBytes + warp * kStageWarp;
+        const long long cg0 = static_cast<long long>(g) * a.col_goff + nw;
+        const uint32_t tb =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
+#pragma unroll 1
+        for (int c0 = 128 * half; c0 < 128 * half + 128 && c0 < a.sw_n; c0 += 32) {
+          float v[32];
+          tmem_ld32(tb + c0, v);
+          if (lane < CW) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              float f = v[e] + bv;
+              if (a.relu) f = f > 0.f ? f : 0.f;
+              reinterpret_cast<__nv_bfloat16*>(stg)[e * CW + lane] = __float2bfloat16_rn(f);
+            }
+          }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < PIECES; ++i) {
+            const int j = lane + 32 * i;
+            const int e = j / PIECES, part = j % PIECES;
+            const int c = c0 + e;
+            const int r = c / a.Wb;
+            const int col = c - r * a.Wb;
+            const int oh = oh0 + r;
+            if (r < a.To_h && oh < a.Ho && col < a.Wo && nw + part * 8 < a.Og) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + e * (CW * 2) + part * 16);
+              *reinterpret_cast<uint4*>(
+                  out + ((static_cast<long long>(b) * a.Ho + oh) * a.Wo + col) * a.ld_out + cg0 +
+                  part * 8) = val;
+            }
+          }
+          __syncwarp();
+        }
+      } else {
 #pragma unroll 1
       for (int sub = 0; sub < NSUB; ++sub) {
         const int m = sub * 128 + quarter * 32 + lane;
@@ -274,8 +350,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 8; ++i) f[i] = v[i];
           if (a.epi == EPI_BF16) {
             if (a.bias) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) f[i] += sbias[cg + i];
+              // cg is a multiple of 8 and the staged bias 16-byte aligned
+              const float4 b0 = *reinterpret_cast<const float4*>(sbias + cg);
+              const float4 b1 = *reinterpret_cast<const float4*>(sbias + cg + 4);
+              f[0] += b0.x;
+              f[1] += b0.y;
+              f[2] += b0.z;
+              f[3] += b0.w;
+              f[4] += b1.x;
+              f[5] += b1.y;
+              f[6] += b1.z;
+              f[7] += b1.w;
             }
             if (a.relu) {
 #pragma unroll
@@ -295,10 +380,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           o.w = pack2(f[6], f[7]);
           *reinterpret_cast<uint4*>(out + row * a.ld_out + cg) = o;
         };
-        // 32-column loads, alternating between the two warps of a quarter
+        // 32-column loads alternating between the two warps of a quarter, or,
+        // where that would leave one warp twice the columns of the other and
+        // halves split into 16-column loads (BN = 96), each warp half of the
+        // columns (32 then 16)
+        constexpr bool kAlt = BN % 64 == 0 || (BN / 2) % 16 != 0;
+        const int cbeg = kAlt ? 32 * half : half * (BN / 2);
+        const int cend = kAlt ? BN : (half + 1) * (BN / 2);
+        const int cstep = kAlt ? 64 : 32;
 #pragma unroll 1
-        for (int c0 = 32 * half; c0 < BN; c0 += 64) {
-          if (c0 + 32 <= BN) {
+        for (int c0 = cbeg; c0 < cend; c0 += cstep) {
+          if (c0 + 32 <= cend) {
             float v[32];
             tmem_ld32(tb + c0, v);
             if (!valid) continue;
@@ -312,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int h = 0; h < 2; ++h) emit8(v + 8 * h, n_t * BN + c0 + 8 * h);
           }
         }
+      }
       }
       tc_fence_before();
       mbar_arrive(acc_empty + 8 * acc);
@@ -477,14 +570,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t st = sdesc0 + s * (stage_bytes >> 4);
           const uint32_t acc0 = p > p0 ? 1u : 0u;
+          const uint32_t bl = st + y_lo;
+          if (NPAIR == 2 && nq == 2) {
+            // two tap pairs, two accumulators: alternate them MMA by MMA
+            const uint32_t al0 = st + pair_lo[0], al1 = st + pair_lo[NPAIR - 1];
+            for (int k = 0; k < ksteps; k += 4)
+              tc_mma_x2<128, 128, 4>(dacc, dacc + BN, al0 + k * 128, al1 + k * 128, pair_hi,
+                                     bl + k * 128, y_hi, IDESC, k == 0 ? acc0 : 1u);
+          } else {
 #pragma unroll
-          for (int j = 0; j < NPAIR; ++j) {
-            if (j < nq) {
-              const uint32_t al = st + pair_lo[j];
-              const uint32_t bl = st + y_lo;
-              for (int k = 0; k < ksteps; k += 4)
-                tc_mma_k4<128, 128>(dacc + j * BN, al + k * 128, pair_hi, bl + k * 128, y_hi,
-                                    IDESC, k == 0 ? acc0 : 1u);
+            for (int j = 0; j < NPAIR; ++j) {
+              if (j < nq) {
+                const uint32_t al = st + pair_lo[j];
+                for (int k = 0; k < ksteps; k += 4)
+                  tc_mma_k4<128, 128>(dacc + j * BN, al + k * 128, pair_hi, bl + k * 128, y_hi,
+                                      IDESC, k == 0 ? acc0 : 1u);
+              }
             }
           }
           tc_commit(empty + 8 * s);
@@ -553,9 +654,9 @@ struct Entry {
   void* fn;
   bool attr;
 };
-template <int BN, int NSUB, int BMN = 0>
+template <int BN, int NSUB, int BMN = 0, int SW = 0>
 void* fwd_ptr() {
-  return reinterpret_cast<void*>(&conv_box_fwd<BN, NSUB, BMN>);
+  return reinterpret_cast<void*>(&conv_box_fwd<BN, NSUB, BMN, SW>);
 }
 template <int BN, int NPAIR>
 void* wgrad_ptr() {
@@ -569,6 +670,8 @@ Entry g_entries[] = {
     {2, 192, 2, fwd_ptr<192, 2, 1>(), false}, {2, 256, 2, fwd_ptr<256, 2, 1>(), false},
     {2, 256, 1, fwd_ptr<256, 1, 1>(), false}, {2, 192, 1, fwd_ptr<192, 1, 1>(), false},
     {0, 192, 1, fwd_ptr<192, 1>(), false},    {0, 256, 1, fwd_ptr<256, 1>(), false},
+    {3, 128, 2, fwd_ptr<128, 2, 0, 1>(), false}, {4, 64, 2, fwd_ptr<64, 2, 1, 1>(), false},
+    {4, 128, 2, fwd_ptr<128, 2, 1, 1>(), false},
     {1, 64, 4, wgrad_ptr<64, 4>(), false},  {1, 96, 2, wgrad_ptr<96, 2>(), false},
     {1, 128, 2, wgrad_ptr<128, 2>(), false},
     {1, 192, 1, wgrad_ptr<192, 1>(), false}, {1, 256, 1, wgrad_ptr<256, 1>(), false},
@@ -613,10 +716,22 @@ bool box_desc_fwd(BoxDesc* d, const ConvShape& cs, const void* x, const void* w,
   memset(d, 0, sizeof(*d));
   if (cs.Cg % 8 || cs.Og % 8 || cs.C % 8 || cs.Ho() < 1 || cs.Wo() < 1) return false;
   if (bias && cs.groups * cs.Og > kMaxBias) return false;  // the bias is staged in shared memory
-  const int bn = fwd_bn(cs.Og);
-  const int nsub = single_sub(bn, cs) ? 1 : 2;
+  int bn = fwd_bn(cs.Og);
+  int nsub = single_sub(bn, cs) ? 1 : 2;
   if (!bn || !find_entry(0, bn, nsub)) return false;
-  if (!box_fwd_common(d, cs, 0, bn, nsub, bias, relu, mask, y, num_sms, status)) return false;
+  // a multiple of 128 output channels per group whose usual tile would be a
+  // single 128 x 192 or 128 x 256 sub-tile (maps at most 128 - K + 1 wide,
+  // conv3): the swapped tile, one 128-channel x (up to) 256-position MMA
+  // per K step.  Where the usual tile has two sub-tiles, their alternating
+  // accumulators issue as fast as the swapped MMA (measured, conv2 and
+  // conv5) and the usual epilogue is cheaper, so it stays.
+  int kind = 0;
+  if (!mask && nsub == 1 && cs.Og % 128 == 0) {
+    kind = 3;
+    bn = 128;
+    nsub = 2;
+  }
+  if (!box_fwd_common(d, cs, kind, bn, nsub, bias, relu, mask, y, num_sms, status)) return false;
   if (!dry) {
     const BoxArgs& a = d->args;
     if (!make_tmap_bf16_4d(&d->tmX, x, cs.C, cs.W, cs.H, cs.B, 64, a.Wb, a.Hb)) return false;
@@ -637,9 +752,20 @@ bool box_desc_dgrad(BoxDesc* d, const ConvShape& cs, const void* dy, const void*
   // instructions of two N = 128 tiles, accumulators still double-buffered)
   int bn = cs.Og <= 64 ? 64 : (cs.Og == 192 ? 192 : (cs.Og % 128 == 0 ? 128 : 256));
   if (cs.Og % 256 == 0 && cs.Wo() + cs.K - 1 <= 128) bn = 256;
-  const int nsub = single_sub(bn, cs) ? 1 : 2;
+  int nsub = single_sub(bn, cs) ? 1 : 2;
   if (!find_entry(2, bn, nsub)) return false;
-  if (!box_fwd_common(d, cs, 2, bn, nsub, nullptr, 0, mask, dx, num_sms, status)) return false;
+  // no mask and at most 64 input channels per group (conv2's 48) or a
+  // multiple of 128: the swapped tile, one 64- or 128-channel x (up to)
+  // 256-position MMA per K step (the MN-major weight slab as A) instead of
+  // 128-position ones that need two MMAs, or leave most of the tensor pipe
+  // idle with N = 64
+  int kind = 2;
+  if (!mask && (cs.Og <= 64 || cs.Og % 128 == 0)) {
+    kind = 4;
+    bn = cs.Og <= 64 ? 64 : 128;
+    nsub = 2;
+  }
+  if (!box_fwd_common(d, cs, kind, bn, nsub, nullptr, 0, mask, dx, num_sms, status)) return false;
   d->args.w_og = cs.Cg;
   d->args.w_p = p_fwd;
   if (!dry) {
@@ -672,6 +798,10 @@ static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, in
   a.Hb = (rows + a.Wb - 1) / a.Wb;
   if (a.Hb > 256) return false;
   a.tiles_img = (a.Ho + a.To_h - 1) / a.To_h;
+  // swapped tiles multiply only the tile's positions, rounded up to 16 (N of
+  // an M = 64 or 128 MMA): 208 of the 256 for a whole 13 x 15 box
+  a.sw_n = (a.To_h * a.Wb + 15) / 16 * 16;
+  if (a.sw_n > 256) a.sw_n = 256;
   a.cpt = cs.P() / 64;
   {
     // K steps of 16 channels of the last chunk that can hold real channels;
@@ -698,14 +828,15 @@ static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, in
   d->a_bytes = ((a.Hb * a.Wb * 128) + 1023) / 1024 * 1024;
   d->b_bytes = bn * 128;
   d->stages_a = 2;
-  const int left = kSmemBudget - 1024 - kBarBytes - 2 * d->a_bytes;
+  const int stg = (kind == 3 || kind == 4) ? kStageBytes : 0;
+  const int left = kSmemBudget - 1024 - kBarBytes - stg - 2 * d->a_bytes;
   // two taps per weight stage (half the barrier round trips of the single
   // issuing thread) while at least three stages fit
   d->tps = (left / (2 * d->b_bytes) >= 3 && cs.K * cs.K > 1) ? 2 : 1;
   d->stages_b = left / (d->tps * d->b_bytes);
   if (d->stages_b > 8) d->stages_b = 8;
   if (d->stages_b < 2) return false;
-  d->smem = 1024 + kBarBytes + 2 * d->a_bytes + d->stages_b * d->tps * d->b_bytes;
+  d->smem = 1024 + kBarBytes + stg + 2 * d->a_bytes + d->stages_b * d->tps * d->b_bytes;
   const long long tiles = 1LL * a.n_tiles * a.tiles_img * a.B * a.groups;
   d->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   return true;
@@ -831,7 +962,7 @@ cudaError_t box_launch(const BoxDesc& d, cudaStream_t stream) {
     e->attr = true;
   }
   count_launch();
-  if (d.kind == 0 || d.kind == 2) {
+  if (d.kind != 1) {
     void* params[] = {const_cast<CUtensorMap*>(&d.tmX), const_cast<CUtensorMap*>(&d.tmW),
                       const_cast<BoxArgs*>(&d.args), const_cast<int*>(&d.stages_a),
                       const_cast<int*>(&d.stages_b), const_cast<int*>(&d.a_bytes),

@@ -38,6 +38,7 @@ struct BoxArgs {
   int groups;
   int Og;          // output channels per group
   int n_tiles;     // BN-wide tiles over Og
+  int sw_n;        // swapped tiles: MMA N = the tile's positions rounded up to 16 (<= 256)
   // forward epilogue (as GemmArgs)
   int epi, relu;
   void* out;
@@ -62,7 +63,10 @@ struct BoxArgs {
 };
 
 struct BoxDesc {
-  int kind;  // 0: forward / data gradient, 1: weight gradient, 2: data gradient from the forward weights
+  // 0: forward / data gradient, 1: weight gradient, 2: data gradient from the
+  // forward weights, 3: forward with swapped operands (M = 128 output channels,
+  // N = the tile's positions), 4: kind 2 swapped (M = 64 or 128 input channels)
+  int kind;
   int bn;
   int nsub;  // forward: 128-row sub-tiles per tile; weight gradient: pairs per item
   CUtensorMap tmX, tmW;  // weight gradient: tmW maps dY

@@ -137,39 +137,89 @@ __device__ __forceinline__ uint4 lrn8(const float2 (&P)[6], float2 k2, float2 al
 __global__ void k_write_hparams(HParams* hp, HParams v) { *hp = v; }
 
 // ------------------------------------------------------------------ s2d
-// One block per (image, output row i): the four input rows 4i .. 4i+3 are
-// staged in shared memory, each at a stride of 688 elements (rows past 226
-// and columns past 226 zero).  Output pixel j holds channel
-// (dy * 4 + dx) * 3 + c = x[4i + dy][4j + dx][c]: its channels 0-23 are the
-// 12 elements at 12j of staged rows 0 and 1, channels 24-47 those of rows 2
-// and 3, channels 48-63 zero.  A thread writes one of these three parts of a
-// pixel: six 8-byte shared loads, then 16-byte stores.
+// One block per (image, pair of output rows i0, i0 + 1): the eight input
+// rows 4 i0 .. 4 i0 + 7 are staged in shared memory, each at a stride of 688
+// elements (rows past 226 and columns past 226 zero).  Output pixel j of row
+// i holds channel (dy * 4 + dx) * 3 + c = x[4i + dy][4j + dx][c]: its
+// channels 0-23 are the 12 elements at 12j of staged rows 4(i - i0) and
+// 4(i - i0) + 1, channels 24-47 those of the next two rows, channels 48-63
+// zero.  A thread writes one of these three parts of a pixel: six 8-byte
+// shared loads, then 16-byte stores.
+constexpr int kS2dRows = 2;  // output rows per block
 __global__ void __launch_bounds__(256) k_s2d(const bf16* __restrict__ x, bf16* __restrict__ xs,
                                              int B) {
   constexpr int kRow = 227 * 3;  // elements per input row
   constexpr int kStride = 688;   // staged row stride: 8-byte aligned pixel groups
-  __shared__ __align__(16) uint16_t st[4 * kStride];
-  const int i = blockIdx.x % 57;
-  const int b = blockIdx.x / 57;
-  const int rows = min(4, 227 - 4 * i);
-  const uint16_t* src =
-      reinterpret_cast<const uint16_t*>(x) + (static_cast<size_t>(b) * 227 + 4 * i) * kRow;
-  for (int e = threadIdx.x; e < 4 * kStride; e += blockDim.x) {
-    const int dy = e / kStride, c = e - dy * kStride;
-    st[e] = (dy < rows && c < kRow) ? src[dy * kRow + c] : static_cast<uint16_t>(0);
+  constexpr int kIn = 4 * kS2dRows;
+  constexpr int kWords = (kIn * kRow + 7) / 8 + 1;  // 16-byte words a block's rows can touch
+  constexpr int kPer = (kWords + 255) / 256;
+  __shared__ __align__(16) uint16_t st[kIn * kStride];
+  const int tiles = (57 + kS2dRows - 1) / kS2dRows;
+  const int i0 = (blockIdx.x % tiles) * kS2dRows;
+  const int b = blockIdx.x / tiles;
+  const int rows = min(kIn, 227 - 4 * i0);
+  // the block's input rows are one contiguous run of rows * kRow elements;
+  // it is read in 16-byte words aligned to x (x is 16-byte aligned), all of
+  // a thread's words in flight at once, each word's in-range elements then
+  // scattered to their staged row and column
+  const long long base = (static_cast<long long>(b) * 227 + 4 * i0) * kRow;
+  const int len = rows * kRow;
+  const long long total = static_cast<long long>(B) * 227 * kRow;
+  const long long w0 = base >> 3;
+  const int lead = static_cast<int>(base - w0 * 8);  // elements of word 0 before the run
+  // zero what no input element lands on: columns 681-687 of every staged
+  // row, and the rows past the image
+  for (int e = threadIdx.x; e < kIn * 8; e += blockDim.x) {
+    const int r = e >> 3, c = kRow + (e & 7);
+    if (c < kStride) st[r * kStride + c] = 0;
+  }
+  for (int e = threadIdx.x; e < (kIn - rows) * kStride; e += blockDim.x) st[rows * kStride + e] = 0;
+  uint4 u[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const long long w = w0 + threadIdx.x + k * 256;
+    u[k] = make_uint4(0, 0, 0, 0);
+    if (w * 8 >= base + len) continue;
+    if (w * 8 + 8 <= total) {
+      u[k] = reinterpret_cast<const uint4*>(x)[w];
+    } else {  // the tensor's last, partial word
+      const uint16_t* xv = reinterpret_cast<const uint16_t*>(x);
+      uint32_t h[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) h[q] = w * 8 + q < total ? xv[w * 8 + q] : 0u;
+      u[k] = make_uint4(h[0] | h[1] << 16, h[2] | h[3] << 16, h[4] | h[5] << 16, h[6] | h[7] << 16);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int r0 = (threadIdx.x + k * 256) * 8 - lead;  // run index of the word's first element
+    const uint32_t wv[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int g = r0 + q;
+      if (g >= 0 && g < len) {
+        const int dy = g / kRow;
+        st[dy * kStride + (g - dy * kRow)] =
+            static_cast<uint16_t>(q & 1 ? wv[q >> 1] >> 16 : wv[q >> 1] & 0xFFFFu);
+      }
+    }
   }
   __syncthreads();
-  uint4* out = reinterpret_cast<uint4*>(xs + (static_cast<size_t>(b) * 57 + i) * 57 * 64);
-  for (int u = threadIdx.x; u < 57 * 3; u += blockDim.x) {
-    const int j = u / 3, h = u - j * 3;
-    uint4* o = out + j * 8 + h * 3;  // 16-byte chunks: 0-2, 3-5, 6-7
+  const int nout = min(kS2dRows, 57 - i0);
+  for (int t = threadIdx.x; t < nout * 57 * 3; t += blockDim.x) {
+    const int ii = t / (57 * 3);
+    const int u3 = t - ii * (57 * 3);
+    const int j = u3 / 3, h = u3 - j * 3;
+    uint4* o = reinterpret_cast<uint4*>(xs + ((static_cast<size_t>(b) * 57 + i0 + ii) * 57 + j) * 64) +
+               h * 3;  // 16-byte chunks: 0-2, 3-5, 6-7
     if (h == 2) {
       o[0] = make_uint4(0, 0, 0, 0);
       o[1] = make_uint4(0, 0, 0, 0);
       continue;
     }
-    const uint2* r0 = reinterpret_cast<const uint2*>(st + (2 * h) * kStride + 12 * j);
-    const uint2* r1 = reinterpret_cast<const uint2*>(st + (2 * h + 1) * kStride + 12 * j);
+    const uint16_t* sr = st + (4 * ii + 2 * h) * kStride + 12 * j;
+    const uint2* r0 = reinterpret_cast<const uint2*>(sr);
+    const uint2* r1 = reinterpret_cast<const uint2*>(sr + kStride);
     const uint2 a0 = r0[0], a1 = r0[1], a2 = r0[2];
     const uint2 b0 = r1[0], b1 = r1[1], b2 = r1[2];
     o[0] = make_uint4(a0.x, a0.y, a1.x, a1.y);
@@ -480,24 +530,47 @@ __global__ void __launch_bounds__(256) k_lrn_pool_fwd(const bf16* __restrict__ a
   // rows whose normalised values this block writes to `lo` (each row once)
   const int own1 = oh1 == Ho ? H : 2 * oh1;
   const int units1 = (r1 - r0) * W * 4;
-  for (int u = threadIdx.x; u < units1; u += blockDim.x) {
-    const int j = u & 3;
-    const int x = (u >> 2) % W;
-    const int r = (u >> 2) / W;
-    const int c0 = cs + j * 8;
-    const bf16* ap = a + ((static_cast<size_t>(b) * H + r0 + r) * W + x) * C + c0;
-    float f[8];
-    unpack8(*reinterpret_cast<const uint4*>(ap), f);
-    float2 P[6];
+  // four units per thread per pass, their loads issued before any is used
+  constexpr int U = 4;
+  for (int u0 = threadIdx.x; u0 < units1; u0 += U * blockDim.x) {
+    uint4 v[U];
+    uint32_t hl[U], hr[U];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) P[1 + m] = make_float2(f[2 * m], f[2 * m + 1]);
-    P[0] = c0 > 0 ? ld_bf16x2(ap - 2) : make_float2(0.f, 0.f);
-    P[5] = c0 + 8 < C ? ld_bf16x2(ap + 8) : make_float2(0.f, 0.f);
-    const uint4 packed = lrn8<B34>(P, make_float2(k, k), make_float2(alpha, alpha), beta);
-    lds[(r * W + x) * 4 + j] = packed;
-    if (lo && r0 + r < own1)
-      *reinterpret_cast<uint4*>(lo + ((static_cast<size_t>(b) * H + r0 + r) * W + x) * C + c0) =
-          packed;
+    for (int q = 0; q < U; ++q) {
+      const int u = u0 + q * blockDim.x;
+      v[q] = make_uint4(0, 0, 0, 0);
+      hl[q] = hr[q] = 0;
+      if (u < units1) {
+        const int j = u & 3;
+        const int x = (u >> 2) % W;
+        const int r = (u >> 2) / W;
+        const int c0 = cs + j * 8;
+        const bf16* ap = a + ((static_cast<size_t>(b) * H + r0 + r) * W + x) * C + c0;
+        v[q] = *reinterpret_cast<const uint4*>(ap);
+        if (c0 > 0) hl[q] = *reinterpret_cast<const uint32_t*>(ap - 2);
+        if (c0 + 8 < C) hr[q] = *reinterpret_cast<const uint32_t*>(ap + 8);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < U; ++q) {
+      const int u = u0 + q * blockDim.x;
+      if (u >= units1) break;
+      const int j = u & 3;
+      const int x = (u >> 2) % W;
+      const int r = (u >> 2) / W;
+      const int c0 = cs + j * 8;
+      float2 P[6], mid[4];
+      unpack4x2(v[q], mid);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) P[1 + m] = mid[m];
+      P[0] = bf2_to_f2(hl[q]);
+      P[5] = bf2_to_f2(hr[q]);
+      const uint4 packed = lrn8<B34>(P, make_float2(k, k), make_float2(alpha, alpha), beta);
+      lds[(r * W + x) * 4 + j] = packed;
+      if (lo && r0 + r < own1)
+        *reinterpret_cast<uint4*>(lo + ((static_cast<size_t>(b) * H + r0 + r) * W + x) * C + c0) =
+            packed;
+    }
   }
   __syncthreads();
   const int units2 = (oh1 - oh0) * Wo * 4;
@@ -728,6 +801,402 @@ __global__ void __launch_bounds__(256) k_pool_lrn_bwd(const bf16* __restrict__ d
   }
 }
 
+// The same backward with each quad's CH = C / 8 channel units in
+// consecutive lanes of one warp (32 / CH quads per warp; C <= 256): the
+// normalisation's channel halo moves between neighbouring lanes by shuffles,
+// so the loop needs no block-wide barrier and a warp never waits for
+// another.  Lanes past the last whole quad of a warp stay idle.  Same
+// arithmetic, window order and bias partial layout as k_pool_lrn_bwd.
+template <int ZC, int WC, bool B34>
+__global__ void __launch_bounds__(256, 3) k_pool_lrn_bwd_w(const bf16* __restrict__ dy,
+                                                        const uint8_t* __restrict__ am,
+                                                        const bf16* __restrict__ a,
+                                                        bf16* __restrict__ dl,
+                                                        bf16* __restrict__ da, int nquads,
+                                                        int H_, int W_, int C, int z_, float k,
+                                                        float alpha, float beta,
+                                                        float* __restrict__ bias_part) {
+  const int H = WC ? WC : H_, W = WC ? WC : W_, z = ZC ? ZC : z_;
+  const int Ho = (H - z) / 2 + 1, Wo = (W - z) / 2 + 1;
+  const int QH = (H + 1) >> 1, QW = (W + 1) >> 1;
+  const int CH = C >> 3;
+  const int qpw = 32 / CH;  // quads per warp
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int qslot = lane / CH, uj = lane - qslot * CH;
+  const bool mine = qslot < qpw;
+  const int wpb = blockDim.x >> 5;
+  __shared__ float red[8 * 32 * 8];  // [warp][lane][8 channels]
+  const float2 k2 = make_float2(k, k), alpha2 = make_float2(alpha, alpha);
+  const float2 mc2ab = make_float2(-2.f * alpha * beta, -2.f * alpha * beta);
+  float2 bsum[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) bsum[m] = make_float2(0.f, 0.f);
+  const int gwarp = blockIdx.x * wpb + warp, nwarps = gridDim.x * wpb;
+  for (int q0 = gwarp * qpw; q0 < nquads; q0 += nwarps * qpw) {
+    const int q = q0 + qslot;
+    const bool live = mine && q < nquads;
+    int b = 0, qi = 0, qj = 0;
+    if (live) {
+      qj = q % QW;
+      const int r = q / QW;
+      qi = r % QH;
+      b = r / QH;
+    }
+    uint4 wdy[4];
+    uint2 wam[4];
+    bool wok[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int oh = qi - 1 + (w >> 1), ow = qj - 1 + (w & 1);
+      wok[w] = live && oh >= 0 && oh < Ho && ow >= 0 && ow < Wo && (z == 3 || w == 3);
+      wdy[w] = make_uint4(0, 0, 0, 0);
+      wam[w] = make_uint2(0, 0);
+      if (wok[w]) {
+        const uint32_t o = static_cast<uint32_t>((b * Ho + oh) * Wo + ow) * C + uj * 8;
+        wdy[w] = *reinterpret_cast<const uint4*>(dy + o);
+        wam[w] = *reinterpret_cast<const uint2*>(am + o);
+      }
+    }
+#pragma unroll
+    for (int px = 0; px < 4; ++px) {
+      const int h = px >> 1, d = px & 1;
+      const int ih = 2 * qi + h, iw = 2 * qj + d;
+      const bool pv = live && ih < H && iw < W;
+      float2 g[4], av[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) g[m] = av[m] = make_float2(0.f, 0.f);
+      if (pv) {
+        unpack4x2(*reinterpret_cast<const uint4*>(
+                      a + static_cast<uint32_t>((b * H + ih) * W + iw) * C + uj * 8),
+                  av);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int rr = h + 2 - 2 * (w >> 1), rc = d + 2 - 2 * (w & 1);
+          if (wok[w] && rr < z && rc < z)
+            add_routed8(wdy[w], wam[w], static_cast<uint32_t>(rr * z + rc), g);
+        }
+      }
+      // channel halo from the neighbouring lanes of the same quad
+      float2 Lh = make_float2(__shfl_up_sync(0xffffffffu, av[3].x, 1),
+                              __shfl_up_sync(0xffffffffu, av[3].y, 1));
+      float2 Rh = make_float2(__shfl_down_sync(0xffffffffu, av[0].x, 1),
+                              __shfl_down_sync(0xffffffffu, av[0].y, 1));
+      if (uj == 0) Lh = make_float2(0.f, 0.f);
+      if (uj == CH - 1) Rh = make_float2(0.f, 0.f);
+      float2 sq[6], S[4], first[4], tv[4];
+      sq[0] = __fmul2_rn(Lh, Lh);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) sq[1 + m] = __fmul2_rn(av[m], av[m]);
+      sq[5] = __fmul2_rn(Rh, Rh);
+      window5(sq, S);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float2 sb, sb1;
+        lrn_pow2x2<B34>(__ffma2_rn(alpha2, S[m], k2), beta, sb, sb1);
+        first[m] = __fmul2_rn(g[m], sb);
+        tv[m] = __fmul2_rn(__fmul2_rn(g[m], av[m]), sb1);
+      }
+      float2 TL = make_float2(__shfl_up_sync(0xffffffffu, tv[3].x, 1),
+                              __shfl_up_sync(0xffffffffu, tv[3].y, 1));
+      float2 TR = make_float2(__shfl_down_sync(0xffffffffu, tv[0].x, 1),
+                              __shfl_down_sync(0xffffffffu, tv[0].y, 1));
+      if (uj == 0) TL = make_float2(0.f, 0.f);
+      if (uj == CH - 1) TR = make_float2(0.f, 0.f);
+      if (!pv) continue;
+      float2 tp[6], cross[4];
+      tp[0] = TL;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) tp[1 + m] = tv[m];
+      tp[5] = TR;
+      window5(tp, cross);
+      uint4 packed;
+      uint32_t* pw = &packed.x;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float2 dd = __ffma2_rn(mc2ab, __fmul2_rn(av[m], cross[m]), first[m]);
+        pw[m] = f2_to_bf2(make_float2(av[m].x > 0.f ? dd.x : 0.f, av[m].y > 0.f ? dd.y : 0.f));
+      }
+      const uint32_t e = static_cast<uint32_t>((b * H + ih) * W + iw) * C + uj * 8;
+      *reinterpret_cast<uint4*>(da + e) = packed;
+      if (dl) {
+        uint4 gp;
+        gp.x = f2_to_bf2(g[0]);
+        gp.y = f2_to_bf2(g[1]);
+        gp.z = f2_to_bf2(g[2]);
+        gp.w = f2_to_bf2(g[3]);
+        *reinterpret_cast<uint4*>(dl + e) = gp;
+      }
+      float2 r[4];
+      unpack4x2(packed, r);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) bsum[m] = __fadd2_rn(bsum[m], r[m]);
+    }
+  }
+  if (!bias_part) return;
+  // per-channel sums over the block's (warp, quad slot) pairs, in that order
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    red[(warp * 32 + lane) * 8 + 2 * m] = bsum[m].x;
+    red[(warp * 32 + lane) * 8 + 2 * m + 1] = bsum[m].y;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    const int u = c >> 3, i = c & 7;
+    float v = 0.f;
+    for (int w = 0; w < wpb; ++w)
+      for (int qs = 0; qs < qpw; ++qs) v += red[(w * 32 + qs * CH + u) * 8 + i];
+    bias_part[static_cast<size_t>(blockIdx.x) * C + c] = v;
+  }
+}
+
+// The same backward with each work item's rows staged in shared memory by
+// bulk asynchronous copies, so that the loads of the next items are in
+// flight while one is computed.  Item (b, qi) = quad row qi of image b: the
+// input rows 2 qi, 2 qi + 1 of a (contiguous in NHWC) and the pooled rows
+// qi - 1, qi of dy and of the window choices (the only windows that cover
+// the quad row).  Thread (qj, uj) = quad column qj, channel unit uj (eight
+// channels), blockDim = QW * CH rounded up to a warp (at most 448, two
+// blocks per SM); the channel halo of the normalisation sums is read from
+// the staged row itself, that of the cross term goes through shared memory
+// (two barriers per input row).  Every bulk copy lands in a stage no thread
+// reads any more (a block barrier precedes the issue); every wait is
+// bounded.  Per block, the column sums of the stored da go to
+// bias_part[blockIdx.x][C] in a fixed order.
+struct PlbGeom {
+  int rowA, rowO;              // elements per input / pooled row
+  int off_dy, off_am, stage;   // byte offsets within a stage, stage bytes
+};
+__host__ __device__ inline int round128(int v) { return (v + 127) & ~127; }
+__host__ __device__ inline PlbGeom plb_geom(int W, int Wo, int C) {
+  PlbGeom g;
+  g.rowA = W * C;
+  g.rowO = Wo * C;
+  g.off_dy = round128(2 * g.rowA * 2);
+  g.off_am = g.off_dy + round128(2 * g.rowO * 2);
+  g.stage = g.off_am + round128(2 * g.rowO);
+  return g;
+}
+
+template <int ZC, int WC, bool B34>
+__global__ void __launch_bounds__(448, 2) k_pool_lrn_bwd_s(
+    const bf16* __restrict__ dy, const uint8_t* __restrict__ am, const bf16* __restrict__ a,
+    bf16* __restrict__ dl, bf16* __restrict__ da, int B, int H_, int W_, int C, int z_, float k,
+    float alpha, float beta, int nst, float* __restrict__ bias_part, int* status) {
+  const int H = WC ? WC : H_, W = WC ? WC : W_, z = ZC ? ZC : z_;
+  const int Ho = (H - z) / 2 + 1, Wo = (W - z) / 2 + 1;
+  const int QH = (H + 1) >> 1;
+  const int QW = (W + 1) >> 1;
+  const int CH = C >> 3;
+  const PlbGeom G = plb_geom(W, Wo, C);
+  extern __shared__ __align__(128) uint8_t plb_smem[];
+  const int nt = blockDim.x;
+  float4* tvs = reinterpret_cast<float4*>(plb_smem + nst * G.stage);  // [pixel][thread]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tvs + 2 * nt);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + nst);
+  const uint32_t bar0 = smem_u32(bars);
+  const int tid = threadIdx.x;
+  const int qj = tid / CH, uj = tid - qj * CH;
+  const bool mine = qj < QW;
+  const int items = B * QH;
+  const float2 k2 = make_float2(k, k), alpha2 = make_float2(alpha, alpha);
+  const float2 mc2ab = make_float2(-2.f * alpha * beta, -2.f * alpha * beta);
+
+  // the pooled rows an item needs: qi - 1 (z = 3 only) .. qi, inside the map
+  auto out_rows = [&](int qi, int& olo) {
+    olo = z == 3 ? max(qi - 1, 0) : qi;
+    const int ohi = min(qi, Ho - 1);
+    return ohi >= olo ? ohi - olo + 1 : 0;
+  };
+  auto issue = [&](int item, int st) {
+    const int b = item / QH, qi = item - b * QH;
+    const int nra = min(2, H - 2 * qi);
+    int olo;
+    const int nro = out_rows(qi, olo);
+    const uint32_t bar = bar0 + 8 * st;
+    const uint32_t dst = smem_u32(plb_smem + st * G.stage);
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nra * G.rowA * 2 + nro * G.rowO * 3));
+    bulk_load(dst, a + (static_cast<size_t>(b) * H + 2 * qi) * G.rowA,
+              static_cast<uint32_t>(nra * G.rowA * 2), bar);
+    if (nro) {
+      const size_t o = (static_cast<size_t>(b) * Ho + olo) * G.rowO;
+      bulk_load(dst + G.off_dy, dy + o, static_cast<uint32_t>(nro * G.rowO * 2), bar);
+      bulk_load(dst + G.off_am, am + o, static_cast<uint32_t>(nro * G.rowO), bar);
+    }
+  };
+
+  if (tid == 0) {
+    for (int st = 0; st < nst; ++st) mbar_init(bar0 + 8 * st, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int st = 0; st < nst; ++st) {
+      const int item = blockIdx.x + st * gridDim.x;
+      if (item < items) issue(item, st);
+    }
+  }
+
+  float2 bsum[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) bsum[m] = make_float2(0.f, 0.f);
+  int n = 0;
+  bool aborted = false;
+  for (int item = blockIdx.x; item < items; item += gridDim.x, ++n) {
+    const int st = n % nst;
+    // (a thread whose wait gave up computes on whatever the stage holds,
+    // in bounds, and leaves with the others at the first barrier)
+    mbar_wait_limit(bar0 + 8 * st, static_cast<uint32_t>((n / nst) & 1), status, abort_flag,
+                     WAIT_LIMIT_CYCLES);
+    const int b = item / QH, qi = item - b * QH;
+    int olo;
+    out_rows(qi, olo);
+    const uint8_t* sbase = plb_smem + st * G.stage;
+    const bf16* SA = reinterpret_cast<const bf16*>(sbase);
+    const bf16* SD = reinterpret_cast<const bf16*>(sbase + G.off_dy);
+    const uint8_t* SM = sbase + G.off_am;
+    uint4 wdy[4];
+    uint2 wam[4];
+    bool wok[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int oh = qi - 1 + (w >> 1), ow = qj - 1 + (w & 1);
+      wok[w] = mine && oh >= 0 && oh < Ho && ow >= 0 && ow < Wo && (z == 3 || w == 3);
+      wdy[w] = make_uint4(0, 0, 0, 0);
+      wam[w] = make_uint2(0, 0);
+      if (wok[w]) {
+        const int o = (oh - olo) * G.rowO + ow * C + uj * 8;
+        wdy[w] = *reinterpret_cast<const uint4*>(SD + o);
+        wam[w] = *reinterpret_cast<const uint2*>(SM + o);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int ih = 2 * qi + h;
+      float2 first[2][4], tv[2][4];
+      bool pv[2];
+#pragma unroll
+      for (int d = 0; d < 2; ++d) {
+        const int iw = 2 * qj + d;
+        pv[d] = mine && ih < H && iw < W;
+        float2 g[4], P[6];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) g[m] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 6; ++q) P[q] = make_float2(0.f, 0.f);
+        if (pv[d]) {
+          const int o = h * G.rowA + iw * C + uj * 8;
+          float2 av[4];
+          unpack4x2(*reinterpret_cast<const uint4*>(SA + o), av);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) P[1 + m] = av[m];
+          if (uj > 0) P[0] = bf2_to_f2(*reinterpret_cast<const uint32_t*>(SA + o - 2));
+          if (uj < CH - 1) P[5] = bf2_to_f2(*reinterpret_cast<const uint32_t*>(SA + o + 8));
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int rr = h + 2 - 2 * (w >> 1), rc = d + 2 - 2 * (w & 1);
+            if (wok[w] && rr < z && rc < z)
+              add_routed8(wdy[w], wam[w], static_cast<uint32_t>(rr * z + rc), g);
+          }
+          if (dl) {
+            uint4 gp;
+            gp.x = f2_to_bf2(g[0]);
+            gp.y = f2_to_bf2(g[1]);
+            gp.z = f2_to_bf2(g[2]);
+            gp.w = f2_to_bf2(g[3]);
+            *reinterpret_cast<uint4*>(
+                dl + static_cast<uint32_t>((b * H + ih) * W + iw) * C + uj * 8) = gp;
+          }
+        }
+        float2 sq[6], S[4];
+#pragma unroll
+        for (int q = 0; q < 6; ++q) sq[q] = __fmul2_rn(P[q], P[q]);
+        window5(sq, S);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          float2 sb, sb1;
+          lrn_pow2x2<B34>(__ffma2_rn(alpha2, S[m], k2), beta, sb, sb1);
+          first[d][m] = __fmul2_rn(g[m], sb);
+          tv[d][m] = __fmul2_rn(__fmul2_rn(g[m], P[1 + m]), sb1);
+        }
+        tvs[d * nt + tid] = make_float4(tv[d][0].x, tv[d][0].y, tv[d][3].x, tv[d][3].y);
+      }
+      __syncthreads();
+      if (*abort_flag) break;
+#pragma unroll
+      for (int d = 0; d < 2; ++d) {
+        if (!pv[d]) continue;
+        const int iw = 2 * qj + d;
+        const float4 L = uj > 0 ? tvs[d * nt + tid - 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 R = uj < CH - 1 ? tvs[d * nt + tid + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+        float2 tp[6], cross[4], av[4];
+        unpack4x2(*reinterpret_cast<const uint4*>(SA + h * G.rowA + iw * C + uj * 8), av);
+        tp[0] = make_float2(L.z, L.w);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) tp[1 + m] = tv[d][m];
+        tp[5] = make_float2(R.x, R.y);
+        window5(tp, cross);
+        uint4 packed;
+        uint32_t* pw = &packed.x;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float2 dd = __ffma2_rn(mc2ab, __fmul2_rn(av[m], cross[m]), first[d][m]);
+          pw[m] = f2_to_bf2(make_float2(av[m].x > 0.f ? dd.x : 0.f, av[m].y > 0.f ? dd.y : 0.f));
+        }
+        *reinterpret_cast<uint4*>(da + static_cast<uint32_t>((b * H + ih) * W + iw) * C +
+                                  uj * 8) = packed;
+        float2 r[4];
+        unpack4x2(packed, r);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) bsum[m] = __fadd2_rn(bsum[m], r[m]);
+      }
+      // the cross-term slots are free again; after the second row, stage st too
+      __syncthreads();
+    }
+    if (*abort_flag) {
+      aborted = true;
+      break;
+    }
+    if (tid == 0) {
+      const int next = item + nst * gridDim.x;
+      if (next < items) {
+        fence_proxy_async_smem();
+        issue(next, st);
+      }
+    }
+  }
+  if (aborted) {
+    // copies still in flight land before the block exits (bounded wait)
+    if (tid == 0) {
+      for (int j = 0; j < nst; ++j) {
+        const int nn = n + j;
+        if (blockIdx.x + nn * gridDim.x >= items) break;
+        const uint32_t bar = bar0 + 8 * (nn % nst);
+        const uint32_t par = static_cast<uint32_t>((nn / nst) & 1);
+        for (int i = 0; i < (1 << 20) && !mbar_try_wait(bar, par); ++i) __nanosleep(64);
+      }
+    }
+    return;
+  }
+  if (!bias_part) return;
+  // per-channel sums over the block's quad columns, in column order (the
+  // stages are idle: every issued copy has been consumed)
+  float* red = reinterpret_cast<float*>(plb_smem);
+  if (mine) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      red[qj * C + uj * 8 + 2 * m] = bsum[m].x;
+      red[qj * C + uj * 8 + 2 * m + 1] = bsum[m].y;
+    }
+  }
+  __syncthreads();
+  for (int c = tid; c < C; c += nt) {
+    float v = 0.f;
+    for (int q = 0; q < QW; ++q) v += red[q * C + c];
+    bias_part[static_cast<size_t>(blockIdx.x) * C + c] = v;
+  }
+}
+
 __global__ void k_pool_fwd_f32(const float* __restrict__ x, float* __restrict__ y, int B, int H,
                                int W, int C, int z, int st) {
   const int Ho = (H - z) / st + 1, Wo = (W - z) / st + 1;
@@ -944,7 +1413,7 @@ __global__ void k_loss_mean(const float* __restrict__ rows, int B, float* out1, 
 }
 
 // ------------------------------------------------------------------ bias gradients
-constexpr int kColsumRows = 128;  // minimum rows per chunk
+constexpr int kColsumRows = 32;  // minimum rows per chunk (more chunks: more loads in flight)
 constexpr int kColsumMaxChunks = 512;
 
 // Rows per chunk: at least kColsumRows, a multiple of it, and no more than
@@ -1083,6 +1552,65 @@ __global__ void k_sgd_conv(float* __restrict__ w, float* __restrict__ v,
   }
 }
 
+// k_sgd_conv for four consecutive parameters per thread (same kernel tap,
+// four consecutive input channels: Cg % 4 == 0, not the space-to-depth
+// form, no flipped copy), so that every partial-sum, weight and momentum
+// access is a 16-byte vector and four splits' loads are in flight at once.
+// Same summation order (slices s = 0, 1, ...) and update as k_sgd_conv.
+__global__ void k_sgd_conv4(float* __restrict__ w, float* __restrict__ v,
+                            const float* __restrict__ part, int S, ConvMap m, bf16* fwd,
+                            float* grads_out, const HParams* __restrict__ hpp) {
+  const HParams hp = *hpp;
+  const long long n4 = 1LL * m.Cout * m.K * m.K * m.Cg / 4;
+  const int Og = m.Cout / m.groups;
+  const long long Kg = 1LL * m.K * m.K * m.P;
+  const long long split4 = 1LL * m.groups * Og * Kg / 4;  // split stride in float4
+  const float4* part4 = reinterpret_cast<const float4*>(part);
+  for (long long q = blockIdx.x * 1LL * blockDim.x + threadIdx.x; q < n4;
+       q += 1LL * gridDim.x * blockDim.x) {
+    const ConvIdx ix = conv_index(m, 4 * q);
+    const long long base4 = ((1LL * ix.g * Og + ix.co) * Kg + ix.part_inner) / 4;
+    float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {
+      float4 t[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) t[i] = part4[(s + i) * split4 + base4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        g.x += t[i].x;
+        g.y += t[i].y;
+        g.z += t[i].z;
+        g.w += t[i].w;
+      }
+    }
+    for (; s < S; ++s) {
+      const float4 t = part4[s * split4 + base4];
+      g.x += t.x;
+      g.y += t.y;
+      g.z += t.z;
+      g.w += t.w;
+    }
+    if (hp.update) {
+      float4 wv = reinterpret_cast<float4*>(w)[q];
+      float4 vv = reinterpret_cast<float4*>(v)[q];
+      sgd_one(wv.x, vv.x, g.x, hp);
+      sgd_one(wv.y, vv.y, g.y, hp);
+      sgd_one(wv.z, vv.z, g.z, hp);
+      sgd_one(wv.w, vv.w, g.w, hp);
+      reinterpret_cast<float4*>(w)[q] = wv;
+      reinterpret_cast<float4*>(v)[q] = vv;
+      uint2 u;
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(wv.x, wv.y);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(wv.z, wv.w);
+      u.x = *reinterpret_cast<uint32_t*>(&h0);
+      u.y = *reinterpret_cast<uint32_t*>(&h1);
+      *reinterpret_cast<uint2*>(fwd + ix.fwd) = u;
+    }
+    if (grads_out) reinterpret_cast<float4*>(grads_out)[q] = g;
+  }
+}
+
 __global__ void k_conv_shadows(const float* __restrict__ w, ConvMap m, bf16* fwd, bf16* dg) {
   const long long n = 1LL * m.Cout * m.K * m.K * m.Cg;
   for (long long p = blockIdx.x * 1LL * blockDim.x + threadIdx.x; p < n;
@@ -1129,13 +1657,12 @@ __global__ void k_sgd_dense(float* __restrict__ w, float* __restrict__ v,
 // partial column sums (T = float), or, for a short matrix, the bf16
 // gradient rows themselves (T = bf16: the column sum is the bias gradient).
 template <typename T>
-__global__ void __launch_bounds__(1024) k_sgd_bias(float* __restrict__ b, float* __restrict__ v,
-                                                   const T* __restrict__ partial, int chunks,
-                                                   int n, float* grads_out,
-                                                   const HParams* __restrict__ hpp) {
-  __shared__ float red[32][33];
+__device__ __forceinline__ void bias_block(float* __restrict__ b, float* __restrict__ v,
+                                           const T* __restrict__ partial, int chunks, int n,
+                                           float* grads_out, const HParams* __restrict__ hpp,
+                                           int blk, float (&red)[32][33]) {
   const int tx = threadIdx.x, ty = threadIdx.y;
-  const int i = blockIdx.x * 32 + tx;
+  const int i = blk * 32 + tx;
   float g = 0.f;
   if (i < n) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1165,6 +1692,27 @@ __global__ void __launch_bounds__(1024) k_sgd_bias(float* __restrict__ b, float*
     }
     if (grads_out) grads_out[i] = sum;
   }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(1024) k_sgd_bias(float* __restrict__ b, float* __restrict__ v,
+                                                   const T* __restrict__ partial, int chunks,
+                                                   int n, float* grads_out,
+                                                   const HParams* __restrict__ hpp) {
+  __shared__ float red[32][33];
+  bias_block<T>(b, v, partial, chunks, n, grads_out, hpp, blockIdx.x, red);
+}
+
+// Several layers' bias updates in one launch: block k belongs to the last
+// job whose first block is <= k.
+__global__ void __launch_bounds__(1024) k_sgd_bias_jobs(BiasJobs jobs,
+                                                        const HParams* __restrict__ hpp) {
+  __shared__ float red[32][33];
+  int k = 0;
+  while (k + 1 < jobs.count && static_cast<int>(blockIdx.x) >= jobs.j[k + 1].block0) ++k;
+  const BiasJob& J = jobs.j[k];
+  bias_block<float>(J.b, J.v, J.partial, J.chunks, J.n, J.grads_out, hpp,
+                    static_cast<int>(blockIdx.x) - J.block0, red);
 }
 
 // [S] 3.4 "Training Procedure Details", update rule, on a range of the
@@ -1621,7 +2169,7 @@ void launch_write_hparams(HParams* hp, HParams v, cudaStream_t s) {
 }
 
 void launch_s2d(const bf16* x, bf16* xs, int B, cudaStream_t s) {
-  k_s2d<<<B * 57, 256, 0, s>>>(x, xs, B);
+  k_s2d<<<B * ((57 + kS2dRows - 1) / kS2dRows), 256, 0, s>>>(x, xs, B);
   count_launch();
 }
 void launch_lrn_fwd(const bf16* a, bf16* b, long long P, int C, int, float k, float alpha,
@@ -1694,29 +2242,122 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
   count_launch();
   return true;
 }
+__device__ int g_aux_status;
+int* aux_status_word() {
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_aux_status) == cudaSuccess ? static_cast<int*>(p) : nullptr;
+}
 constexpr int kPoolLrnBlocks = 148 * 8;  // persistent blocks: eight per SM
 // quads of 2 x 2 pixels per block (one 8-channel unit per thread)
 inline int pool_lrn_quads_per_block(int C) { return 256 / (C / 8); }
-int pool_lrn_bwd_parts(int B, int H, int W, int C, int z) {
-  (void)z;
+// quads per block of the warp-segment kernel (8 warps of 32 / (C / 8) quads)
+inline int pool_lrn_quads_per_block_w(int C) { return 8 * (32 / (C / 8)); }
+inline bool pool_lrn_use_warp_kernel(int C) { return C >= 8 && C <= 256; }
+// Launch shape of the staged kernel: stages per block, threads, dynamic
+// shared memory and blocks (persistent, over the SMs).  False if the shape
+// does not suit it (bulk copies need 16-byte rows; at most 448 threads).
+struct PlbCfg {
+  int nst, threads, smem, blocks;
+};
+bool pool_lrn_staged_cfg(int B, int H, int W, int C, int z, PlbCfg* c) {
+  if (C <= 0 || C % 8 || (z != 2 && z != 3) || H < z || W < z) return false;
+  const int Wo = (W - z) / 2 + 1;
+  if ((W * C * 2) % 16 || (Wo * C) % 16) return false;
+  const int QW = (W + 1) / 2, QH = (H + 1) / 2;
+  const int threads = (QW * (C / 8) + 31) / 32 * 32;
+  if (threads > 448) return false;
+  const PlbGeom G = plb_geom(W, Wo, C);
+  constexpr int kBudget = 227 * 1024, kSmPerSm = 228 * 1024;
+  // registers per thread as allocated (the kernel is built for two blocks of
+  // 448 threads per SM: at most 72)
+  constexpr int kRegs = 72;
+  // the most items in flight per SM (stages x resident blocks); ties go to
+  // fewer stages and more blocks
+  int best = 0;
+  for (int nst = 2; nst <= 4; ++nst) {
+    const int smem = nst * G.stage + 2 * threads * 16 + 8 * nst + 16;
+    if (smem > kBudget) break;
+    int bps = kSmPerSm / (smem + 1024);
+    bps = std::min(bps, 2048 / threads);
+    bps = std::min(bps, 65536 / (kRegs * threads));
+    if (bps < 1) break;
+    if (nst * bps > best) {
+      best = nst * bps;
+      c->nst = nst;
+      c->smem = smem;
+      c->blocks = bps;
+    }
+  }
+  if (!best) return false;
+  // the bias column sums reuse the first stage: QW x C floats
+  if (QW * C * 4 > c->nst * G.stage) return false;
+  c->threads = threads;
+  const long long items = 1LL * B * QH;
+  const long long grid = std::min<long long>(items, 148LL * c->blocks);
+  c->blocks = static_cast<int>(grid);
+  return true;
+}
+// Rows of bias partial sums the block-per-row kernels write.
+static int pool_lrn_bwd_parts_unstaged(int B, int H, int W, int C) {
   if (C <= 0 || C % 8 || C > 2048) return 0;
   const long long nquads = 1LL * B * ((H + 1) / 2) * ((W + 1) / 2);
-  const int nq = pool_lrn_quads_per_block(C);
+  const int nq = pool_lrn_use_warp_kernel(C) ? pool_lrn_quads_per_block_w(C)
+                                             : pool_lrn_quads_per_block(C);
   const long long groups = nq > 0 ? (nquads + nq - 1) / nq : 0;
   return static_cast<int>(groups < kPoolLrnBlocks ? groups : kPoolLrnBlocks);
 }
-bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
-                         int B, int H, int W, int C, int z, float k, float alpha, float beta,
-                         float* bias_part, cudaStream_t s) {
-  if (C % kSlab || C > 2048 || (z != 2 && z != 3) || H < z || W < z) return false;
+int pool_lrn_bwd_parts(int B, int H, int W, int C, int z) {
+  PlbCfg pc;
+  const int staged = pool_lrn_staged_cfg(B, H, W, C, z, &pc) ? pc.blocks : 0;
+  return std::max(staged, pool_lrn_bwd_parts_unstaged(B, H, W, C));
+}
+int launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
+                        int B, int H, int W, int C, int z, float k, float alpha, float beta,
+                        float* bias_part, int* status, cudaStream_t s) {
+  if (C % kSlab || C > 2048 || (z != 2 && z != 3) || H < z || W < z) return 0;
   const long long npix = 1LL * B * H * W;
-  if (npix * C >= (1LL << 31)) return false;  // 32-bit element offsets
+  if (npix * C >= (1LL << 31)) return 0;  // 32-bit element offsets
   const bool b34 = beta == 0.75f;
-  const int blocks = pool_lrn_bwd_parts(B, H, W, C, z);
+  const int blocks = pool_lrn_bwd_parts_unstaged(B, H, W, C);
   const int nq = pool_lrn_quads_per_block(C);
-  if (nq < 1 || blocks < 1) return false;
+  if (nq < 1 || blocks < 1) return 0;
   const int nquads = static_cast<int>(1LL * B * ((H + 1) / 2) * ((W + 1) / 2));
+  const uintptr_t vec = reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(a) |
+                        reinterpret_cast<uintptr_t>(da) | reinterpret_cast<uintptr_t>(dl);
+  if ((vec & 15) || (reinterpret_cast<uintptr_t>(am) & 7)) return 0;  // vector accesses
+  PlbCfg pc;
+  if (!(reinterpret_cast<uintptr_t>(am) & 15) && pool_lrn_staged_cfg(B, H, W, C, z, &pc)) {
+    int* st = status ? status : aux_status_word();
+    if (!st) return 0;
+    auto gs = [&](auto kern) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pc.smem);
+      kern<<<pc.blocks, pc.threads, pc.smem, s>>>(dy, am, a, dl, da, B, H, W, C, z, k, alpha,
+                                                  beta, pc.nst, bias_part, st);
+    };
+    if (z == 3 && H == 55 && W == 55)
+      b34 ? gs(k_pool_lrn_bwd_s<3, 55, true>) : gs(k_pool_lrn_bwd_s<3, 55, false>);
+    else if (z == 3 && H == 27 && W == 27)
+      b34 ? gs(k_pool_lrn_bwd_s<3, 27, true>) : gs(k_pool_lrn_bwd_s<3, 27, false>);
+    else
+      b34 ? gs(k_pool_lrn_bwd_s<0, 0, true>) : gs(k_pool_lrn_bwd_s<0, 0, false>);
+    count_launch();
+    return pc.blocks;
+  }
   // persistent blocks (at most kPoolLrnBlocks, one bias partial row each)
+  if (pool_lrn_use_warp_kernel(C)) {
+    auto gw = [&](auto kern) {
+      kern<<<blocks, 256, 0, s>>>(dy, am, a, dl, da, nquads, H, W, C, z, k, alpha, beta,
+                                  bias_part);
+    };
+    if (z == 3 && H == 55 && W == 55)
+      b34 ? gw(k_pool_lrn_bwd_w<3, 55, true>) : gw(k_pool_lrn_bwd_w<3, 55, false>);
+    else if (z == 3 && H == 27 && W == 27)
+      b34 ? gw(k_pool_lrn_bwd_w<3, 27, true>) : gw(k_pool_lrn_bwd_w<3, 27, false>);
+    else
+      b34 ? gw(k_pool_lrn_bwd_w<0, 0, true>) : gw(k_pool_lrn_bwd_w<0, 0, false>);
+    count_launch();
+    return blocks;
+  }
   auto go = [&](auto kern) {
     kern<<<blocks, 256, 0, s>>>(dy, am, a, dl, da, nquads, nq, H, W, C, z, k, alpha, beta,
                                 bias_part);
@@ -1728,7 +2369,7 @@ bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16*
   else
     b34 ? go(k_pool_lrn_bwd<0, 0, true>) : go(k_pool_lrn_bwd<0, 0, false>);
   count_launch();
-  return true;
+  return blocks;
 }
 void launch_pool_fwd_f32(const float* x, float* y, int B, int H, int W, int C, int z, int st,
                          cudaStream_t s) {
@@ -1779,7 +2420,14 @@ void launch_colsum_partial(const bf16* m, long long rows, int cols, float* parti
 void launch_sgd_conv(float* w, float* v, const float* part, int S, const ConvMap& m, bf16* fwd,
                      bf16* dg, float* grads_out, const HParams* hp, cudaStream_t s) {
   const long long n = 1LL * m.Cout * m.K * m.K * m.Cg;
-  k_sgd_conv<<<grid_for(n, 256), 256, 0, s>>>(w, v, part, S, m, fwd, dg, grads_out, hp);
+  if (!m.s2d && !dg && m.Cg % 4 == 0 &&
+      ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(v) |
+        reinterpret_cast<uintptr_t>(part) | reinterpret_cast<uintptr_t>(grads_out)) & 15) == 0 &&
+      (reinterpret_cast<uintptr_t>(fwd) & 7) == 0) {
+    k_sgd_conv4<<<grid_for(n / 4, 256), 256, 0, s>>>(w, v, part, S, m, fwd, grads_out, hp);
+  } else {
+    k_sgd_conv<<<grid_for(n, 256), 256, 0, s>>>(w, v, part, S, m, fwd, dg, grads_out, hp);
+  }
   count_launch();
 }
 void launch_sgd_dense(float* w, float* v, const float* g, long long n, bf16* shadow,
@@ -1792,6 +2440,16 @@ void launch_sgd_bias(float* b, float* v, const float* partial, int chunks, int n
   if (n <= 0) return;
   k_sgd_bias<float><<<(n + 31) / 32, dim3(32, 32), 0, s>>>(b, v, partial, chunks, n, grads_out,
                                                           hp);
+  count_launch();
+}
+void launch_sgd_bias_jobs(BiasJobs jobs, const HParams* hp, cudaStream_t s) {
+  int blocks = 0;
+  for (int k = 0; k < jobs.count; ++k) {
+    jobs.j[k].block0 = blocks;
+    blocks += (jobs.j[k].n + 31) / 32;
+  }
+  if (blocks <= 0) return;
+  k_sgd_bias_jobs<<<blocks, dim3(32, 32), 0, s>>>(jobs, hp);
   count_launch();
 }
 void launch_sgd_bias_rows(float* b, float* v, const bf16* g, int rows, int n, float* grads_out,

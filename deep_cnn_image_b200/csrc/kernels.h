@@ -87,11 +87,17 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
                          int C, int z, float k, float alpha, float beta, cudaStream_t s);
 // Fused stride-2 max-pool backward + normalisation backward + ReLU mask
 // (a > 0) into da; dl (the normalised map's gradient) written when non-null.
-// bias_part (nullable): per-block column sums of the stored da,
-// [pool_lrn_bwd_parts(B, H, W, C, z)][C] fp32, for the conv bias update.
-bool launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
-                         int B, int H, int W, int C, int z, float k, float alpha, float beta,
-                         float* bias_part, cudaStream_t s);
+// bias_part (nullable): per-block column sums of the stored da, one row of C
+// fp32 per block, at most pool_lrn_bwd_parts(B, H, W, C, z) rows, for the
+// conv bias update.  status: the word a bounded wait that runs out sets
+// (STATUS_TIMEOUT); null: aux_status_word().  Returns the number of bias
+// partial rows (blocks), 0 if the shape or the pointers are not supported.
+int launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
+                        int B, int H, int W, int C, int z, float k, float alpha, float beta,
+                        float* bias_part, int* status, cudaStream_t s);
+// A device status word for single-op calls that have no workspace to hold
+// one (never cleared by the library; nullptr if it cannot be looked up).
+int* aux_status_word();
 int pool_lrn_bwd_parts(int B, int H, int W, int C, int z);
 void launch_pool_fwd_f32(const float* x, float* y, int B, int H, int W, int C, int z, int st,
                          cudaStream_t s);
@@ -130,6 +136,21 @@ void launch_sgd_dense(float* w, float* v, const float* g, long long n, bf16* sha
                       float* grads_out, const HParams* hp, cudaStream_t s);
 void launch_sgd_bias(float* b, float* v, const float* partial, int chunks, int n,
                      float* grads_out, const HParams* hp, cudaStream_t s);
+// Several bias updates from fp32 partial column sums in one launch (the
+// conv layers' at the end of the backward pass); block0 is filled in.
+struct BiasJob {
+  float* b;
+  float* v;
+  const float* partial;
+  int chunks, n;
+  float* grads_out;
+  int block0;
+};
+struct BiasJobs {
+  BiasJob j[5];
+  int count;
+};
+void launch_sgd_bias_jobs(BiasJobs jobs, const HParams* hp, cudaStream_t s);
 // Bias update straight from a short bf16 gradient matrix g [rows][n]: the
 // bias gradient is its column sum (the FC layers, rows = batch).
 void launch_sgd_bias_rows(float* b, float* v, const bf16* g, int rows, int n, float* grads_out,

@@ -153,6 +153,7 @@ struct alexnet {
   size_t scratch_floats = 0;
   float* cpart = nullptr;
   size_t cpart_floats = 0;
+  size_t cpart_off[5] = {0, 0, 0, 0, 0};  // per conv layer, floats
   // fp32 path
   float* fa = nullptr;
   float* fb = nullptr;
@@ -546,19 +547,19 @@ size_t carve(alexnet* h, void* base) {
   h->dlogits = c.take<bf16>(static_cast<size_t>(B) * kClasses);
   h->d7 = c.take<bf16>(static_cast<size_t>(B) * 4096);
   h->d6 = c.take<bf16>(static_cast<size_t>(B) * 4096);
-  // column-sum partials for bias gradients: max over layers of chunks x cols
-  size_t cp = static_cast<size_t>(colsum_chunks(B)) * 4096;
+  // column-sum partials for the conv bias gradients, one region per layer
+  // (all five updates run in one launch at the end of the backward pass):
+  // the most rows any producer writes (column sums of da, the fused pool +
+  // normalisation backward, the pool backward) x cols
+  size_t cp = 0;
   for (int l = 0; l < 5; ++l) {
     const ConvL& L = h->conv[l];
-    const size_t e = static_cast<size_t>(colsum_chunks(1LL * B * L.Ho * L.Ho)) * L.Cout;
-    if (e > cp) cp = e;
-    // bias partials of the fused pool + normalisation backward, and of the
-    // pool backward
-    const size_t f =
-        static_cast<size_t>(pool_lrn_bwd_parts(B, L.Ho, L.Ho, L.Cout, cfg.pool_size)) * L.Cout;
-    if (f > cp) cp = f;
-    const size_t pb = static_cast<size_t>(pool_bwd_parts(B, L.Ho, L.Ho, L.Cout)) * L.Cout;
-    if (pb > cp) cp = pb;
+    size_t rows = static_cast<size_t>(colsum_chunks(1LL * B * L.Ho * L.Ho));
+    rows = std::max(rows, static_cast<size_t>(
+                              pool_lrn_bwd_parts(B, L.Ho, L.Ho, L.Cout, cfg.pool_size)));
+    rows = std::max(rows, static_cast<size_t>(pool_bwd_parts(B, L.Ho, L.Ho, L.Cout)));
+    h->cpart_off[l] = cp;
+    cp += (rows * L.Cout + 63) / 64 * 64;
   }
   h->cpart_floats = cp;
   h->cpart = c.take<float>(cp);
@@ -788,7 +789,7 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
   {
     const ConvL& L = h->conv[4];
     const int parts = launch_pool_bwd(h->dp5, h->am[4], h->p[4], h->da[4], B, L.Ho, L.Ho, L.Cout,
-                                      cfg.pool_size, 2, 1, s, h->cpart);
+                                      cfg.pool_size, 2, 1, s, h->cpart + h->cpart_off[4]);
     if (parts > 0) {
       fused_bwd[4] = true;
       bias_parts[4] = parts;
@@ -798,11 +799,9 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
     const ConvL& L = h->conv[l];
     const long long rows = 1LL * B * L.Ho * L.Ho;
     if (!fused_bwd[l]) {
-      launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart, s);
+      launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart + h->cpart_off[l], s);
       bias_parts[l] = colsum_chunks(rows);
     }
-    launch_sgd_bias(h->params + h->b_off[l], h->vel + h->b_off[l], h->cpart, bias_parts[l],
-                    L.Cout, gptr(h->b_off[l]), h->hp, s);
     if (l > 0) {
       ALX_TRY(run_gemm(h, P->cd[l], P->conv_flops[l], s), "conv dgrad launch");
       const ConvL& Q = h->conv[l - 1];
@@ -812,12 +811,13 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
           // pool + normalisation + ReLU backward in one pass when the shape
           // allows it (with layer l-1's bias column sums), else pool
           // backward now and normalisation below
-          fused_bwd[l - 1] = launch_pool_lrn_bwd(
+          const int rows = launch_pool_lrn_bwd(
               h->dp[l - 1], h->am[l - 1], h->a[l - 1], h->keep ? h->dl[l - 1] : nullptr,
               h->da[l - 1], B, Q.Ho, Q.Ho, Q.Cout, cfg.pool_size, cfg.lrn_k, cfg.lrn_alpha,
-              cfg.lrn_beta, h->cpart, s);
-          if (fused_bwd[l - 1])
-            bias_parts[l - 1] = pool_lrn_bwd_parts(B, Q.Ho, Q.Ho, Q.Cout, cfg.pool_size);
+              cfg.lrn_beta, h->cpart + h->cpart_off[l - 1], h->status, s);
+          fused_bwd[l - 1] = rows > 0;
+          if (rows > 0)
+            bias_parts[l - 1] = rows;
           else
             launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->dl[l - 1], B, Q.Ho, Q.Ho,
                             Q.Cout, cfg.pool_size, 2, 0, s);
@@ -838,6 +838,19 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
                        cfg.lrn_n, cfg.lrn_k, cfg.lrn_alpha, cfg.lrn_beta, s);
     }
   }
+  // the five conv bias updates, from their column-sum partials
+  BiasJobs jobs{};
+  jobs.count = 5;
+  for (int l = 0; l < 5; ++l) {
+    BiasJob& J = jobs.j[l];
+    J.b = h->params + h->b_off[l];
+    J.v = h->vel + h->b_off[l];
+    J.partial = h->cpart + h->cpart_off[l];
+    J.chunks = bias_parts[l];
+    J.n = h->conv[l].Cout;
+    J.grads_out = gptr(h->b_off[l]);
+  }
+  launch_sgd_bias_jobs(jobs, h->hp, s);
   return cuda_status(h, cudaGetLastError(), "train step");
 }
 
@@ -1001,8 +1014,9 @@ alexnet_status alexnet_forward(alexnet_t* h, const void* x, int B, alexnet_mode 
                                float* logits, float* probs, void* stream) {
   if (!h) return ALEXNET_ERR_INVALID_ARG;
   if (!x || !logits || B < 1 || B > h->cfg.batch_max ||
-      (mode != ALEXNET_TRAIN && mode != ALEXNET_INFERENCE)) {
-    h->err = "forward: invalid argument";
+      (mode != ALEXNET_TRAIN && mode != ALEXNET_INFERENCE) ||
+      (reinterpret_cast<uintptr_t>(x) & 15)) {
+    h->err = "forward: invalid argument (x must be a 16-byte aligned device pointer)";
     return ALEXNET_ERR_INVALID_ARG;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -1041,8 +1055,9 @@ alexnet_status alexnet_forward(alexnet_t* h, const void* x, int B, alexnet_mode 
 alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* labels, int B,
                                   float lr, float* loss, void* stream) {
   if (!h) return ALEXNET_ERR_INVALID_ARG;
-  if (!x || !labels || B < 1 || B > h->cfg.batch_max || !(lr >= 0.f)) {
-    h->err = "train_step: invalid argument";
+  if (!x || !labels || B < 1 || B > h->cfg.batch_max || !(lr >= 0.f) ||
+      (reinterpret_cast<uintptr_t>(x) & 15)) {
+    h->err = "train_step: invalid argument (x must be a 16-byte aligned device pointer)";
     return ALEXNET_ERR_INVALID_ARG;
   }
   if (h->cfg.dtype != ALEXNET_BF16) {
@@ -1081,7 +1096,7 @@ alexnet_status alexnet_train_grads(alexnet_t* h, const void* x, const int32_t* l
                                    int64_t image_offset, float* loss, void* stream) {
   if (!h) return ALEXNET_ERR_INVALID_ARG;
   if (!x || !labels || B < 1 || B > h->cfg.batch_max || image_offset < 0 ||
-      image_offset > 0x7FFFFFFF - B) {
+      image_offset > 0x7FFFFFFF - B || (reinterpret_cast<uintptr_t>(x) & 15)) {
     h->err = "train_grads: invalid argument";
     return ALEXNET_ERR_INVALID_ARG;
   }

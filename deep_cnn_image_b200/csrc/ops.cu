@@ -99,7 +99,8 @@ alexnet_status alexnet_op_conv_fwd(const void* x, int B, int H, int W, int Cin, 
 
 alexnet_status alexnet_op_conv1_fwd(const void* x, int B, const void* w, const float* bias,
                                     void* y, void* ws, size_t ws_bytes, void* stream) {
-  if (!x || !w || !y || B < 1) return ALEXNET_ERR_INVALID_ARG;
+  if (!x || !w || !y || B < 1 || (reinterpret_cast<uintptr_t>(x) & 15))
+    return ALEXNET_ERR_INVALID_ARG;
   Scratch sc(ws, ws_bytes);
   int* status = sc.take<int>(1);
   bf16* xs = sc.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 64);
@@ -175,7 +176,8 @@ alexnet_status alexnet_op_conv_wgrad(const void* x, int B, int H, int W, int Cin
 
 alexnet_status alexnet_op_conv1_wgrad(const void* x, int B, const void* dy, int splits, float* dw,
                                       void* ws, size_t ws_bytes, void* stream) {
-  if (!x || !dy || !dw || B < 1) return ALEXNET_ERR_INVALID_ARG;
+  if (!x || !dy || !dw || B < 1 || (reinterpret_cast<uintptr_t>(x) & 15))
+    return ALEXNET_ERR_INVALID_ARG;
   Scratch sc(ws, ws_bytes);
   int* status = sc.take<int>(1);
   bf16* xs = sc.take<bf16>(static_cast<size_t>(B) * 57 * 57 * 64);
@@ -365,7 +367,7 @@ alexnet_status alexnet_op_pool_lrn_bwd(const void* dy, const uint8_t* argmax, co
     return ALEXNET_ERR_INVALID_ARG;
   if (!launch_pool_lrn_bwd(static_cast<const bf16*>(dy), argmax, static_cast<const bf16*>(a),
                            static_cast<bf16*>(dl), static_cast<bf16*>(da), B, H, W, C, z, k, alpha,
-                           beta, nullptr, static_cast<cudaStream_t>(stream)))
+                           beta, nullptr, nullptr, static_cast<cudaStream_t>(stream)))
     return ALEXNET_ERR_UNSUPPORTED;
   return done(cudaGetLastError());
 }

@@ -145,6 +145,18 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int 
       : "memory");
 }
 
+// Untiled bulk copy of `bytes` contiguous bytes from global to shared memory
+// (no multicast), completion signalled on `bar` as transaction bytes.  Both
+// addresses 16-byte aligned, bytes a nonzero multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // im2col load of a 4-D NHWC tensor: pixelsPerColumn consecutive output
 // positions starting at (w, h, n) (top-left input corner of the filter window,
 // may be negative), each fetching the map's channelsPerPixel channels from

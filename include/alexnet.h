@@ -113,7 +113,8 @@ ALEXNET_API alexnet_status alexnet_create(const alexnet_config* cfg, void* works
                               void* stream, alexnet_t** out);
 
 /* Forward pass of B images (1 <= B <= batch_max).
- *   x:      device, [B,227,227,3] NHWC, bf16 (BF16 handle) or fp32 (FP32).
+ *   x:      device, [B,227,227,3] NHWC, bf16 (BF16 handle) or fp32 (FP32),
+ *           16-byte aligned.
  *   mode:   ALEXNET_TRAIN draws the dropout masks of the current step
  *           (Philox(seed, step, index)); ALEXNET_INFERENCE keeps every unit
  *           and scales FC6/FC7 outputs by 1 - p ([S] 3.4 "Dropout").
@@ -126,7 +127,8 @@ ALEXNET_API alexnet_status alexnet_forward(alexnet_t* h, const void* x, int B, a
  * step's dropout masks, mean cross-entropy against labels, backward through
  * all eight layers, then the SGD update of every parameter with learning
  * rate lr; the step counter then advances by one.
- *   x:      device bf16 [B,227,227,3];  labels: device int32 [B] in [0,1000)
+ *   x:      device bf16 [B,227,227,3], 16-byte aligned;  labels: device int32
+ *           [B] in [0,1000)
  *           (an out-of-range label sets ALEXNET_ERR_LABEL_RANGE in the
  *           status word and contributes no loss or gradient);
  *   loss:   device fp32 scalar, nullable: the mean loss of this batch at the

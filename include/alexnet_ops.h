@@ -34,7 +34,8 @@ ALEXNET_API alexnet_status alexnet_op_conv_fwd(const void* x, int B, int H, int 
 
 /* conv1 of the network: 11x11, stride 4, no padding, on a [B,227,227,3]
  * input (computed as a 3x3 stride-1 convolution of its 4x4 space-to-depth
- * form).  w bf16 [96][11][11][3]; y bf16 [B,55,55,96] = relu(conv + bias). */
+ * form).  x 16-byte aligned; w bf16 [96][11][11][3]; y bf16 [B,55,55,96] =
+ * relu(conv + bias). */
 ALEXNET_API alexnet_status alexnet_op_conv1_fwd(const void* x, int B, const void* w, const float* bias,
                                     void* y, void* ws, size_t ws_bytes, void* stream);
 
@@ -81,7 +82,8 @@ ALEXNET_API alexnet_status alexnet_op_conv_wgrad_noalloc(const void* x, int B, i
                                                          int pad, int groups, int splits,
                                                          float* dw, void* stream);
 
-/* conv1 weight gradient on a [B,227,227,3] input: dw fp32 [96][11][11][3]. */
+/* conv1 weight gradient on a [B,227,227,3] input (16-byte aligned): dw fp32
+ * [96][11][11][3]. */
 ALEXNET_API alexnet_status alexnet_op_conv1_wgrad(const void* x, int B, const void* dy, int splits,
                                       float* dw, void* ws, size_t ws_bytes, void* stream);
 

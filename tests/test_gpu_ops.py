@@ -388,10 +388,23 @@ def test_conv_weight_gradient(ax, ws, name, H, Cin, Cout, K, pad, groups, B):
         results.append(got)
         err = rel_l2(got, want)
         assert err < TOL_F32_ACC, (splits, err)
-    # the fixed-order split-K sum differs from the unsplit one by fp32 rounding
-    # only: about 2^-24 * sqrt(terms) relative, terms = B * Ho * Wo (66,564 for
-    # the widest case here)
-    assert rel_l2(results[1], results[0]) < 1e-4
+    # Both results sum the same exact bf16 products in fp32 on the tensor core:
+    # T = terms / 16 + S accumulation steps (16 products each, terms =
+    # B * Ho * Wo positions; S <= 16 split partial sums), each rounding the running sum by at most one
+    # fp32 unit (2^-23) in either direction; the rounding mode of the tensor
+    # core's accumulation is not documented, so the errors may all lean one
+    # way and add up linearly: at most T * 2^-23 of the running sums, which
+    # for these zero-mean inputs stay within about twice the final one (in
+    # L2).  Measured: 1e-7 .. 1e-6 for the box kernels (short chains), 7e-5
+    # for the 66,564-position im2col case, against bounds of 7e-6 .. 1e-3.
+    terms = B * H * H
+    bound = 2.0 * (np.ceil(terms / 16.0) + 16) * 2.0**-23
+    split_err = rel_l2(results[1], results[0])
+    print("conv wgrad %s: oracle rel-L2 %.3g, split 3 vs 1 rel-L2 %.3g (bound %.3g)" %
+          (name, rel_l2(results[0], want), split_err, bound))
+    for got in results:
+        assert rel_l2(got, want) < bound
+    assert split_err < 2.0 * bound
 
 
 def test_conv1_weight_gradient(ax, ws):
