@@ -519,10 +519,13 @@ __global__ void __launch_bounds__(256) k_lrn_pool_fwd(const bf16* __restrict__ a
   const int H = WC ? WC : H_, W = WC ? WC : W_;
   extern __shared__ __align__(16) uint4 lds[];  // [rows][W][4 chunks]
   const int Ho = (H - Z) / 2 + 1, Wo = (W - Z) / 2 + 1;
-  const int oh0 = blockIdx.x * kPoolTileRows;
+  // the channel slab varies fastest across the grid, so the blocks that
+  // read a pixel's neighbouring slabs (the normalisation's channel halo
+  // reaches into them) run together and share those lines in L2
+  const int oh0 = blockIdx.y * kPoolTileRows;
   const int oh1 = min(Ho, oh0 + kPoolTileRows);
-  const int b = blockIdx.y;
-  const int cs = blockIdx.z * kSlab;
+  const int b = blockIdx.z;
+  const int cs = blockIdx.x * kSlab;
   const int r0 = 2 * oh0;
   // rows this block normalises: those its windows read; the last tile also
   // takes the rows below the last window so that `lo` is complete
@@ -2228,7 +2231,7 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
   const int rows = 2 * kPoolTileRows + 2;
   const size_t smem = static_cast<size_t>(rows) * W * kSlab * 2;
   if (smem > 48 * 1024) return false;
-  const dim3 grid((Ho + kPoolTileRows - 1) / kPoolTileRows, B, C / kSlab);
+  const dim3 grid(C / kSlab, (Ho + kPoolTileRows - 1) / kPoolTileRows, B);
   auto go = [&](auto kern) { kern<<<grid, 256, smem, s>>>(a, lo, y, am, H, W, C, k, alpha, beta); };
   const bool b34 = beta == 0.75f;
   if (z == 3 && H == 55 && W == 55)
