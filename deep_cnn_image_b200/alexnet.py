@@ -100,6 +100,7 @@ def _load():
         "alexnet_debug_copy": (st, [vp, i, vp, sz, vp]),
         "alexnet_debug_keep": (st, [vp, i]),
         "alexnet_debug_fc_update": (st, [vp, i]),
+        "alexnet_debug_overlap": (st, [vp, i]),
         "alexnet_debug_canaries": (st, [vp, POINTER(c_int64)]),
         "alexnet_conv_algo": (st, [vp, i, i, i, POINTER(c_int)]),
         "alexnet_stats_enable": (st, [vp, i]),
@@ -260,6 +261,10 @@ class AlexNet:
         """Also store the normalised maps and their gradients (debug_copy
         10/11, 70/71) in later calls."""
         return check(lib.alexnet_debug_keep(self.h, 1 if keep else 0))
+
+    def debug_overlap(self, on=True):
+        """Weight gradients on a second stream beside the data gradients (default on)."""
+        return check(lib.alexnet_debug_overlap(self.h, 1 if on else 0))
 
     def debug_fc_update(self, fused=True):
         """FC weights updated by the weight-gradient GEMM's epilogue (True,

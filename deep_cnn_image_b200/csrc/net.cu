@@ -199,6 +199,12 @@ struct alexnet {
   bool grads_only = false;
   uint32_t row_offset = 0;
   cudaEvent_t fc_event = nullptr;
+  // conv weight gradients and updates run on a second stream beside the
+  // data-gradient chain (fork when dY is complete, the update after the
+  // data gradient that reads the layer's old weights, join at the end)
+  bool overlap_wgrad = true;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_dy[5] = {}, ev_dg[5] = {}, ev_join = nullptr;
   bool capturing = false;
   StepRec direct_rec;
   std::map<int, StepRec> graph_rec;
@@ -784,6 +790,19 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
   // pool/LRN/ReLU backward), weight gradient and update.
   bool fused_bwd[5] = {false, false, false, false, false};
   int bias_parts[5] = {0, 0, 0, 0, 0};
+  cudaStream_t side = nullptr;
+  // (not while per-GEMM timing is on: each GEMM is then timed alone)
+  if (h->overlap_wgrad && !h->stats_on) {
+    if (!h->side) {
+      ALX_TRY(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking), "side stream");
+      for (int l = 0; l < 5; ++l) {
+        ALX_TRY(cudaEventCreateWithFlags(&h->ev_dy[l], cudaEventDisableTiming), "event");
+        ALX_TRY(cudaEventCreateWithFlags(&h->ev_dg[l], cudaEventDisableTiming), "event");
+      }
+      ALX_TRY(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming), "event");
+    }
+    side = h->side;
+  }
   // pool5 backward straight into conv5's pre-activation gradient, with
   // conv5's bias column sums
   {
@@ -802,8 +821,16 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
       launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart + h->cpart_off[l], s);
       bias_parts[l] = colsum_chunks(rows);
     }
+    // dY of layer l is complete: its weight gradient may start beside
+    cudaStream_t ws = s;
+    if (side) {
+      ALX_TRY(cudaEventRecord(h->ev_dy[l], s), "fork");
+      ALX_TRY(cudaStreamWaitEvent(side, h->ev_dy[l], 0), "fork");
+      ws = side;
+    }
     if (l > 0) {
       ALX_TRY(run_gemm(h, P->cd[l], P->conv_flops[l], s), "conv dgrad launch");
+      if (side) ALX_TRY(cudaEventRecord(h->ev_dg[l], s), "data gradient done");
       const ConvL& Q = h->conv[l - 1];
       if (Q.pool) {
         // dp[l-1] = d(pooled map) -> through the pool (and LRN) to da[l-1]
@@ -827,16 +854,24 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
         }
       }
     }
-    ALX_TRY(run_gemm(h, P->cw[l], P->conv_flops[l], s), "conv wgrad launch");
-    launch_sgd_conv(h->params + h->w_off[l], h->vel + h->w_off[l], h->scratch,
-                    P->cw[l].splits(), conv_map(h, l), h->wf[l], h->need_wd ? h->wd[l] : nullptr,
-                    gptr(h->w_off[l]), h->hp, s);
     if (l > 0) {
       const ConvL& Q = h->conv[l - 1];
       if (Q.pool && Q.lrn && !fused_bwd[l - 1])
         launch_lrn_bwd(h->a[l - 1], h->dl[l - 1], h->da[l - 1], 1LL * B * Q.Ho * Q.Ho, Q.Cout,
                        cfg.lrn_n, cfg.lrn_k, cfg.lrn_alpha, cfg.lrn_beta, s);
     }
+    // weight gradient (split partials in scratch, one layer at a time on
+    // the side stream) and update; the update rewrites the bf16 weights the
+    // data gradient above reads, so it waits for it
+    ALX_TRY(run_gemm(h, P->cw[l], P->conv_flops[l], ws), "conv wgrad launch");
+    if (side && l > 0) ALX_TRY(cudaStreamWaitEvent(side, h->ev_dg[l], 0), "update after dgrad");
+    launch_sgd_conv(h->params + h->w_off[l], h->vel + h->w_off[l], h->scratch,
+                    P->cw[l].splits(), conv_map(h, l), h->wf[l], h->need_wd ? h->wd[l] : nullptr,
+                    gptr(h->w_off[l]), h->hp, ws);
+  }
+  if (side) {
+    ALX_TRY(cudaEventRecord(h->ev_join, side), "join");
+    ALX_TRY(cudaStreamWaitEvent(s, h->ev_join, 0), "join");
   }
   // the five conv bias updates, from their column-sum partials
   BiasJobs jobs{};
@@ -1076,7 +1111,8 @@ alexnet_status alexnet_train_step(alexnet_t* h, const void* x, const int32_t* la
   ALX_TRY(cudaMemcpyAsync(h->labels_buf, labels, sizeof(int32_t) * B, cudaMemcpyDeviceToDevice, s),
           "train_step labels");
   const int64_t l0 = launch_counter();
-  const int key = 32 * B + (h->fc_fused ? 4 : 0) + (h->keep ? 2 : 0) + (h->stats_on ? 1 : 0);
+  const int key = 64 * B + (h->overlap_wgrad ? 32 : 0) + (h->fc_fused ? 4 : 0) +
+                  (h->keep ? 2 : 0) + (h->stats_on ? 1 : 0);
   const alexnet_status st = replay(h, key, s, [&](cudaStream_t cs) {
     return train_bf16(h, nullptr, h->labels_buf, B, nullptr, cs, P);
   });
@@ -1125,7 +1161,7 @@ alexnet_status alexnet_train_grads(alexnet_t* h, const void* x, const int32_t* l
   h->stats_on = false;
   // two graphs: forward + FC backward, then the convolutions' backward, with
   // the FC-gradients event recorded between them
-  const int base = 32 * B + (h->keep ? 2 : 0) + 16;
+  const int base = 64 * B + (h->overlap_wgrad ? 32 : 0) + (h->keep ? 2 : 0) + 16;
   if (e == cudaSuccess)
     st = replay(h, base, s, [&](cudaStream_t cs) {
       return train_fc_part(h, nullptr, h->labels_buf, B, nullptr, cs, P);
@@ -1345,6 +1381,12 @@ alexnet_status alexnet_destroy(alexnet_t* h) {
     for (auto& kv : h->train_graphs) cudaGraphExecDestroy(kv.second);
     if (h->fc_event) cudaEventDestroy(h->fc_event);
     if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+    if (h->side) cudaStreamDestroy(h->side);
+    for (int l = 0; l < 5; ++l) {
+      if (h->ev_dy[l]) cudaEventDestroy(h->ev_dy[l]);
+      if (h->ev_dg[l]) cudaEventDestroy(h->ev_dg[l]);
+    }
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
   }
   delete h;
   return ALEXNET_OK;
@@ -1378,6 +1420,12 @@ alexnet_status alexnet_debug_keep(alexnet_t* h, int keep) {
 alexnet_status alexnet_debug_fc_update(alexnet_t* h, int fused) {
   if (!h) return ALEXNET_ERR_INVALID_ARG;
   h->fc_fused = fused != 0;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_debug_overlap(alexnet_t* h, int on) {
+  if (!h) return ALEXNET_ERR_INVALID_ARG;
+  h->overlap_wgrad = on != 0;
   return ALEXNET_OK;
 }
 

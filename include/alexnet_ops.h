@@ -194,6 +194,16 @@ ALEXNET_API alexnet_status alexnet_op_wait_probe(int* status, long long limit_cy
  * the switch exists to compare the two. */
 ALEXNET_API alexnet_status alexnet_debug_fc_update(alexnet_t* h, int fused);
 
+/* on != 0 (default): in a training step each conv layer's weight gradient and
+ * update run on a second stream of the handle beside the data-gradient chain
+ * (forked once the layer's output gradient is complete; the update waits
+ * for the data gradient that reads the layer's old bf16 weights; joined
+ * before the step ends), so the two fill each other's idle SMs.  0: one
+ * stream.  Results are bit-identical; the switch exists to compare the two.
+ * While stats_enable is on the step runs on one stream either way, so that
+ * every GEMM is timed alone. */
+ALEXNET_API alexnet_status alexnet_debug_overlap(alexnet_t* h, int on);
+
 /* Bounds evidence without a sanitiser: every buffer the handle carves out of
  * its workspace is followed by a 256-byte guard region, filled with the byte
  * 0xA5 by alexnet_create.  This call synchronises the handle's last stream

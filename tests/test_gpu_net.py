@@ -321,7 +321,8 @@ def test_full_batch_train_step_matches_oracle(ax):
     Every GPU decision is validated first (tests/_decisions.py).  Then a
     second identical handle must give bit-identical results (fixed-order
     split-K sums, no atomics), and a handle applying the FC update with the
-    separate kernel bit-identical parameters and gradients."""
+    separate kernel, or running the conv weight gradients on the same stream
+    as the data gradients, bit-identical parameters and gradients."""
     import torch
     B, seed = 128, 500
     net, loss, g, blob, wloss, wg, params, n, xr, y = _train_compare(ax, B, seed)
@@ -338,9 +339,10 @@ def test_full_batch_train_step_matches_oracle(ax):
     net.close()
     xt = synthetic.to_bf16(synthetic.images(seed + 2, B))[0].cuda()
     yt = dev(synthetic.labels(seed + 3, B))
-    for fused in (True, False):
+    for fused, overlap in ((True, True), (False, True), (True, False)):
         other = _make(ax, batch_max=B, keep_grads=1, seed=seed)
         other.debug_fc_update(fused)
+        other.debug_overlap(overlap)
         other.set_params(_blob(params, n, 5))
         lo = torch.zeros(1, dtype=torch.float32, device="cuda")
         other.train_step(xt, yt, B, 0.01, lo)
