@@ -205,6 +205,9 @@ struct alexnet {
   bool overlap_wgrad = true;
   cudaStream_t side = nullptr;
   cudaEvent_t ev_dy[5] = {}, ev_dg[5] = {}, ev_join = nullptr;
+  cudaEvent_t ev_fdz[3] = {}, ev_fdg[3] = {}, ev_fjoin = nullptr;  // the FC layers'
+
+
   bool capturing = false;
   StepRec direct_rec;
   std::map<int, StepRec> graph_rec;
@@ -743,6 +746,33 @@ alexnet_status forward_f32(alexnet* h, const float* x, int B, float* logits, cud
 
 // Forward, loss and the FC layers' backward (with their update, unless the
 // handle runs a gradient-only step).
+// The second stream for the weight gradients and updates (created with its
+// events on first use); nullptr when the overlap is off, or while per-GEMM
+// timing is on (each GEMM is then timed alone).
+cudaError_t side_stream(alexnet* h, cudaStream_t* out) {
+  *out = nullptr;
+  if (!h->overlap_wgrad || h->stats_on) return cudaSuccess;
+  if (!h->side) {
+    cudaError_t e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
+    auto ev = [&](cudaEvent_t* x) {
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(x, cudaEventDisableTiming);
+    };
+    for (int l = 0; l < 5; ++l) {
+      ev(&h->ev_dy[l]);
+      ev(&h->ev_dg[l]);
+    }
+    for (int f = 0; f < 3; ++f) {
+      ev(&h->ev_fdz[f]);
+      ev(&h->ev_fdg[f]);
+    }
+    ev(&h->ev_join);
+    ev(&h->ev_fjoin);
+    if (e != cudaSuccess) return e;
+  }
+  *out = h->side;
+  return cudaSuccess;
+}
+
 alexnet_status train_fc_part(alexnet* h, const bf16* x, const int32_t* labels, int B, float* loss,
                              cudaStream_t s, Plan* P) {
   const alexnet_config& cfg = h->cfg;
@@ -754,27 +784,49 @@ alexnet_status train_fc_part(alexnet* h, const bf16* x, const int32_t* labels, i
   launch_loss_mean(h->loss_rows, B, h->loss_dev, loss, s);
   float* gr = h->grads;
   auto gptr = [&](size_t off) { return gr ? gr + off : nullptr; };
-  // FC8, FC7, FC6: data gradient (old weights), then weight gradient + SGD
+  // FC8, FC7, FC6: data gradient (old weights), then weight gradient + SGD.
+  // With the update in the weight-gradient epilogue (or gradients only) the
+  // weight gradient, update and bias update go to the second stream once dz
+  // is complete, the update after the data gradient that reads the layer's
+  // old weights (the separate-kernel update shares the split-K scratch with
+  // the data gradients and stays on one stream).
   const bf16* dz[3] = {h->d6, h->d7, h->dlogits};
   bf16* dxo[3] = {h->dp5, h->d6, h->d7};
   const bf16* mask[3] = {nullptr, h->f6, h->f7};
+  cudaStream_t side = nullptr;
+  if (h->fc_fused || h->grads_only) ALX_TRY(side_stream(h, &side), "side stream");
   for (int f = 2; f >= 0; --f) {
     const FcL& F = h->fc[f];
+    cudaStream_t ws = s;
+    if (side) {
+      ALX_TRY(cudaEventRecord(h->ev_fdz[f], s), "fork");
+      ALX_TRY(cudaStreamWaitEvent(side, h->ev_fdz[f], 0), "fork");
+      ws = side;
+    }
     ALX_TRY(run_gemm(h, P->fd[f], P->fc_flops[f], s), "fc dgrad launch");
+    if (side) ALX_TRY(cudaEventRecord(h->ev_fdg[f], s), "data gradient done");
     launch_dgrad_finalize(h->scratch, P->fd[f].args.splits, B, F.In, mask[f], dxo[f], s);
     if (h->grads_only) {
-      ALX_TRY(run_gemm(h, P->fwg[f], P->fc_flops[f], s), "fc wgrad launch");
+      ALX_TRY(run_gemm(h, P->fwg[f], P->fc_flops[f], ws), "fc wgrad launch");
     } else if (h->fc_fused) {
       // HBM-bound (the update moves 18 bytes per weight against 256 MMA
       // FLOPs): launched outside the per-GEMM tensor-roofline records
-      ALX_TRY(launch_any(P->fws[f], s), "fc wgrad + update launch");
+      if (side) ALX_TRY(cudaStreamWaitEvent(side, h->ev_fdg[f], 0), "update after dgrad");
+      ALX_TRY(launch_any(P->fws[f], ws), "fc wgrad + update launch");
     } else {
       ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s), "fc wgrad launch");
       launch_sgd_dense(h->params + h->w_off[5 + f], h->vel + h->w_off[5 + f], h->scratch,
                        h->w_len[5 + f], h->wf[5 + f], gptr(h->w_off[5 + f]), h->hp, s);
     }
     launch_sgd_bias_rows(h->params + h->b_off[5 + f], h->vel + h->b_off[5 + f], dz[f], B, F.Out,
-                         gptr(h->b_off[5 + f]), h->hp, s);
+                         gptr(h->b_off[5 + f]), h->hp, ws);
+  }
+  // gradients only: the FC gradients are complete when this part ends (the
+  // caller's event marks them); in a training step the side stream carries
+  // on into the convolutions' part and is joined at its end
+  if (side && h->grads_only) {
+    ALX_TRY(cudaEventRecord(h->ev_fjoin, side), "join");
+    ALX_TRY(cudaStreamWaitEvent(s, h->ev_fjoin, 0), "join");
   }
   return cuda_status(h, cudaGetLastError(), "train step (FC part)");
 }
@@ -791,18 +843,7 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
   bool fused_bwd[5] = {false, false, false, false, false};
   int bias_parts[5] = {0, 0, 0, 0, 0};
   cudaStream_t side = nullptr;
-  // (not while per-GEMM timing is on: each GEMM is then timed alone)
-  if (h->overlap_wgrad && !h->stats_on) {
-    if (!h->side) {
-      ALX_TRY(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking), "side stream");
-      for (int l = 0; l < 5; ++l) {
-        ALX_TRY(cudaEventCreateWithFlags(&h->ev_dy[l], cudaEventDisableTiming), "event");
-        ALX_TRY(cudaEventCreateWithFlags(&h->ev_dg[l], cudaEventDisableTiming), "event");
-      }
-      ALX_TRY(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming), "event");
-    }
-    side = h->side;
-  }
+  ALX_TRY(side_stream(h, &side), "side stream");
   // pool5 backward straight into conv5's pre-activation gradient, with
   // conv5's bias column sums
   {
@@ -1386,7 +1427,12 @@ alexnet_status alexnet_destroy(alexnet_t* h) {
       if (h->ev_dy[l]) cudaEventDestroy(h->ev_dy[l]);
       if (h->ev_dg[l]) cudaEventDestroy(h->ev_dg[l]);
     }
+    for (int f = 0; f < 3; ++f) {
+      if (h->ev_fdz[f]) cudaEventDestroy(h->ev_fdz[f]);
+      if (h->ev_fdg[f]) cudaEventDestroy(h->ev_fdg[f]);
+    }
     if (h->ev_join) cudaEventDestroy(h->ev_join);
+    if (h->ev_fjoin) cudaEventDestroy(h->ev_fjoin);
   }
   delete h;
   return ALEXNET_OK;
