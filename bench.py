@@ -47,6 +47,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "images/sec, AlexNet bf16 train step, batch 128, 1×B200; % of bf16 tensor roofline"
+# DRAM bytes (read + written) per batch-128 step of the GEMM class's 20
+# launches, summed from the per-launch ncu counters recorded in
+# profiles/train_step_counters_b128.md (None once those kernels change)
+GEMM_CLASS_TRAFFIC_BYTES = 816_401_920
 UNIT = "images/s"
 WORKLOAD = "AlexNet (grouped conv2/4/5) bf16 training step: forward + backward + SGD-momentum, " \
            "227x227x3 NHWC inputs ~N(0,1), labels U[0,1000)"
@@ -348,7 +352,9 @@ def run_ours(args):
                       "gradient launches; the FC weight-gradient launches apply the SGD update in "
                       "their epilogue, are HBM-bound and are not counted here)",
             "bound": "tensor", "achieved": gemm_tflops, "peak": peak, "unit": "TFLOP/s",
-            "frac": gemm_tflops / peak if gemm_tflops else None, "traffic": None,
+            "frac": gemm_tflops / peak if gemm_tflops else None,
+            "traffic": GEMM_CLASS_TRAFFIC_BYTES if B == 128 and world == 1 else None,
+            "traffic_unit": "bytes per step (DRAM read + write of the class's launches, ncu)",
             "peak_source": peaks["source"] + " bf16_tflops (burst)",
             "gemm_launches_per_step": stats["gemm_launches"] / stat_steps,
             "gemm_ms_per_step": stats["gemm_ms"] / stat_steps,
