@@ -226,11 +226,11 @@ def run_ours(args):
         from deep_cnn_image_b200.dp import DataParallelStep
         dp_step = DataParallelStep(net)
 
-        def train(xb, yb):
-            dp_step.step(xb, yb, B, 0.01, loss)
+        def train(xb, yb, lo=loss):
+            dp_step.step(xb, yb, B, 0.01, lo)
     else:
-        def train(xb, yb):
-            net.train_step(xb, yb, B, 0.01, loss)
+        def train(xb, yb, lo=loss):
+            net.train_step(xb, yb, B, 0.01, lo)
 
     def barrier():
         torch.cuda.synchronize()
@@ -285,13 +285,17 @@ def run_ours(args):
     # ---- end to end through the public call, host buffers: every step's
     # batch is copied from pinned host memory and its loss read back inside
     # the timed span; the copy of batch i+1 (its own stream, into the other
-    # of two device buffers) overlaps step i.  The step's activations
-    # (about 1 GB) exceed the L2, so no flush is needed between steps.
+    # of two device buffers) overlaps step i, and so does the read-back of
+    # step i's loss (from one of two device loss slots, on the copy stream,
+    # so that the compute stream does not wait for it).  The step's
+    # activations (about 1 GB) exceed the L2, so no flush is needed between
+    # steps.
     x_pin = x_host.pin_memory()
     y_pin = torch.from_numpy(y_np).pin_memory()
     loss_pin = torch.zeros(args.steps, dtype=torch.float32).pin_memory()
     xs = [x, torch.empty_like(x)]
     ys = [y, torch.empty_like(y)]
+    losses = [torch.zeros(1, dtype=torch.float32, device="cuda") for _ in range(2)]
     copy_stream = torch.cuda.Stream()
     copied = [torch.cuda.Event(), torch.cuda.Event()]
     consumed = [torch.cuda.Event(), torch.cuda.Event()]
@@ -316,9 +320,15 @@ def run_ours(args):
         if i + 1 < args.steps:
             stage(i + 1)
         stream.wait_event(copied[buf])
-        train(xs[buf], ys[buf])
+        train(xs[buf], ys[buf], losses[buf])
         consumed[buf].record(stream)
-        loss_pin[i:i + 1].copy_(loss, non_blocking=True)
+        # step i's loss, read back on the copy stream: queued before the copy
+        # that refills this buffer pair, which step i + 2 (the next writer of
+        # the slot) waits for
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(consumed[buf])
+            loss_pin[i:i + 1].copy_(losses[buf], non_blocking=True)
+    stream.wait_stream(copy_stream)
     e_end.record(stream)
     barrier()
     ms_e2e = e_start.elapsed_time(e_end)
