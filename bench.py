@@ -529,6 +529,24 @@ def run_mode(args):
             "config": {"workload": args.mode, "batch": B, "variant": args.variant},
             "step_roofline": {"achieved": flops * value / 1e12, "peak": peak,
                               "unit": "TFLOP/s", "frac": flops * value / 1e12 / peak}}
+    if args.mode == "augment":
+        # the augmentation kernel alone (HBM-bound): per image the 256x256x3
+        # u8 source read once and the 227x227x3 bf16 crop written once (the
+        # mean image is shared by the batch)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        reps = 50
+        a0.record(stream)
+        for _ in range(reps):
+            net.augment(src, B, mean, vec, val, x)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        aug_ms = a0.elapsed_time(a1) / reps
+        aug_bytes = B * (256 * 256 * 3 + 227 * 227 * 3 * 2)
+        hbm = load_peaks()["hbm_gbs"]
+        gbs = aug_bytes / (aug_ms / 1e3) / 1e9
+        line["augment_kernel"] = {"ms": aug_ms, "bytes": aug_bytes, "achieved": gbs, "peak": hbm,
+                                  "unit": "GB/s", "frac": gbs / hbm}
     if args.mode == "knn":
         # the base is streamed once per call: HBM-bound
         gbs = hbm_bytes * args.steps / (ms / 1e3) / 1e9
