@@ -1810,33 +1810,41 @@ __device__ __forceinline__ AugDraw aug_draw(const HParams& hp, uint32_t img, con
   return d;
 }
 
+// One block per (image, run of kAugRows output rows): the image's draw
+// (Philox + Box-Muller, one thread) is taken once per run, not once per row,
+// and the run's rows are written element by element (bf16, coalesced).
+constexpr int kAugRows = 8;
 __global__ void k_augment(const uint8_t* __restrict__ src, int B, const float* __restrict__ mean,
                           const float* __restrict__ pca_vec, const float* __restrict__ pca_val,
                           const HParams* __restrict__ hpp, bf16* __restrict__ out) {
   const HParams hp = *hpp;
   __shared__ AugDraw d;
   __shared__ float pv[9], pl[3];
-  // one block per (image, output row)
-  for (long long job = blockIdx.x; job < 1LL * B * 227; job += gridDim.x) {
-    const int b = static_cast<int>(job / 227);
-    const int y = static_cast<int>(job % 227);
-    __syncthreads();
-    if (threadIdx.x < 9) pv[threadIdx.x] = pca_vec[threadIdx.x];
-    if (threadIdx.x < 3) pl[threadIdx.x] = pca_val[threadIdx.x];
-    __syncthreads();
+  if (threadIdx.x < 9) pv[threadIdx.x] = pca_vec[threadIdx.x];
+  if (threadIdx.x < 3) pl[threadIdx.x] = pca_val[threadIdx.x];
+  constexpr int kRuns = (227 + kAugRows - 1) / kAugRows;
+  for (long long job = blockIdx.x; job < 1LL * B * kRuns; job += gridDim.x) {
+    const int b = static_cast<int>(job / kRuns);
+    const int y0 = static_cast<int>(job % kRuns) * kAugRows;
+    const int rows = min(kAugRows, 227 - y0);
+    __syncthreads();  // pv / pl written; the previous run's d no longer read
     if (threadIdx.x == 0) d = aug_draw(hp, static_cast<uint32_t>(b), pv, pl);
     __syncthreads();
-    bf16* orow = out + (1LL * b * 227 + y) * 227 * 3;
-    for (int e = threadIdx.x; e < 227 * 3; e += blockDim.x) {
-      const int x = e / 3, c = e - x * 3;
+    const uint8_t* simg = src + 1LL * b * 256 * 256 * 3;
+    bf16* orun = out + (1LL * b * 227 + y0) * 227 * 3;
+    for (int e = threadIdx.x; e < rows * 227 * 3; e += blockDim.x) {
+      const int r = e / (227 * 3);
+      const int q = e - r * (227 * 3);
+      const int x = q / 3, c = q - x * 3;
+      const int y = y0 + r;
       float v = 0.f;
       if (y < 224 && x < 224) {
         const int sy = d.oy + y;
         const int sx = d.flip ? d.ox + 223 - x : d.ox + x;
-        const long long si = (1LL * sy * 256 + sx) * 3 + c;
-        v = static_cast<float>(src[1LL * b * 256 * 256 * 3 + si]) - mean[si] + d.add[c];
+        const int si = (sy * 256 + sx) * 3 + c;
+        v = static_cast<float>(simg[si]) - mean[si] + d.add[c];
       }
-      orow[e] = __float2bfloat16_rn(v);
+      orun[e] = __float2bfloat16_rn(v);
     }
   }
 }
@@ -2491,8 +2499,8 @@ void launch_fill(float* w, long long n, float value, cudaStream_t s) {
 }
 void launch_augment(const uint8_t* src, int B, const float* mean, const float* pca_vec,
                     const float* pca_val, const HParams* hp, bf16* out, cudaStream_t s) {
-  k_augment<<<grid_for(1LL * B * 227 * 256, 256), 256, 0, s>>>(src, B, mean, pca_vec, pca_val,
-                                                                hp, out);
+  k_augment<<<grid_for(1LL * B * ((227 + kAugRows - 1) / kAugRows) * 256, 256), 256, 0, s>>>(
+      src, B, mean, pca_vec, pca_val, hp, out);
   count_launch();
 }
 void launch_tencrop_inputs(const uint8_t* src, int B, const float* mean, bf16* out,
