@@ -266,6 +266,10 @@ def run_ours(args):
     # replayed step graph around every GEMM launch (a separate pass, L2
     # flushed before each step)
     stats = {"launches": 0, "gemm_launches": 0, "gemm_flops": 0.0, "gemm_ms": 0.0}
+    # the class split by kind: convolutions (tensor-bound) and the FC forward
+    # and data-gradient products (HBM-bound at batch 128: every weight is
+    # read once per launch for 2 x 128 FLOPs)
+    by_kind = {0: [0.0, 0.0], 1: [0.0, 0.0]}
     stat_steps = min(args.steps, 20)
     net.stats_enable(True)
     for _ in range(2):
@@ -277,6 +281,10 @@ def run_ours(args):
         st = net.stats_read()  # this step's GEMM times (synchronises the stream)
         for k in stats:
             stats[k] += st[k]
+        for kind, fl, t in net.stats_launches():
+            if kind in by_kind:
+                by_kind[kind][0] += fl
+                by_kind[kind][1] += t
     net.stats_enable(False)
     for _ in range(2):  # the step graph without timing nodes
         net.train_step(x, y, B, 0.01, loss)
@@ -369,6 +377,20 @@ def run_ours(args):
             "gemm_launches_per_step": stats["gemm_launches"] / stat_steps,
             "gemm_ms_per_step": stats["gemm_ms"] / stat_steps,
             "gemm_timing": f"{stat_steps} separate steps with per-GEMM events, L2 flushed before each",
+        },
+        "roofline_by_kind": {
+            "conv": {"bound": "tensor",
+                     "achieved": by_kind[0][0] / (by_kind[0][1] / 1e3) / 1e12 if by_kind[0][1] else None,
+                     "peak": peak, "unit": "TFLOP/s",
+                     "frac": by_kind[0][0] / (by_kind[0][1] / 1e3) / 1e12 / peak if by_kind[0][1] else None,
+                     "ms_per_step": by_kind[0][1] / stat_steps},
+            "fc": {"bound": "hbm",
+                   # bf16 weights read once per launch: FLOPs / batch bytes
+                   "achieved": by_kind[1][0] / B / (by_kind[1][1] / 1e3) / 1e9 if by_kind[1][1] else None,
+                   "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                   "frac": by_kind[1][0] / B / (by_kind[1][1] / 1e3) / 1e9 / peaks["hbm_gbs"]
+                   if by_kind[1][1] else None,
+                   "ms_per_step": by_kind[1][1] / stat_steps},
         },
         "step_roofline": {"achieved": step_tflops, "peak": peak, "unit": "TFLOP/s",
                           "frac": step_tflops / peak,

@@ -105,6 +105,8 @@ def _load():
         "alexnet_conv_algo": (st, [vp, i, i, i, POINTER(c_int)]),
         "alexnet_stats_enable": (st, [vp, i]),
         "alexnet_stats_read": (st, [vp, POINTER(Stats)]),
+        "alexnet_stats_launch": (st, [vp, i, POINTER(c_int), POINTER(ctypes.c_double),
+                                      POINTER(ctypes.c_double)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -249,6 +251,18 @@ class AlexNet:
         check(lib.alexnet_stats_read(self.h, ctypes.byref(st_)), self.h)
         return {"launches": st_.launches, "gemm_launches": st_.gemm_launches,
                 "gemm_flops": st_.gemm_flops, "gemm_ms": st_.gemm_ms}
+
+    def stats_launches(self):
+        """(kind, flops, ms) of every GEMM launch stats_read reports: kind 0
+        a convolution, 1 an FC forward or data gradient, 2 an FC weight
+        gradient written to memory."""
+        out = []
+        k, f, m = c_int(), ctypes.c_double(), ctypes.c_double()
+        for idx in range(self.stats_read()["gemm_launches"]):
+            check(lib.alexnet_stats_launch(self.h, idx, ctypes.byref(k), ctypes.byref(f),
+                                           ctypes.byref(m)), self.h)
+            out.append((k.value, f.value, m.value))
+        return out
 
     def conv_algo(self, batch, layer, pass_):
         """1 if convolution `layer` runs the shifted-box kernel for this batch

@@ -177,10 +177,14 @@ struct alexnet {
     size_t used = 0;
     int64_t gemm_launches = 0;
     double gemm_flops = 0.0;
+    std::vector<double> flops;  // per GEMM launch, in launch order
+    std::vector<int> kind;      // 0: convolution, 1: FC forward / data gradient, 2: FC weight gradient
     void reset() {
       used = 0;
       gemm_launches = 0;
       gemm_flops = 0.0;
+      flops.clear();
+      kind.clear();
     }
   };
   bool stats_on = false;
@@ -649,7 +653,7 @@ cudaError_t launch_any(const GemmDesc& d, cudaStream_t s) { return gemm_launch(d
 cudaError_t launch_any(const ConvPlan& d, cudaStream_t s) { return conv_plan_launch(d, s); }
 
 template <typename D>
-cudaError_t run_gemm(alexnet* h, const D& d, double flops, cudaStream_t s) {
+cudaError_t run_gemm(alexnet* h, const D& d, double flops, cudaStream_t s, int kind = 0) {
   if (!h->stats_on || !h->rec) return launch_any(d, s);
   alexnet::StepRec& R = *h->rec;
   while (R.used + 2 > R.ev.size()) {
@@ -667,6 +671,8 @@ cudaError_t run_gemm(alexnet* h, const D& d, double flops, cudaStream_t s) {
   cudaEventRecordWithFlags(e1, s, flags);
   R.gemm_launches += 1;
   R.gemm_flops += flops;
+  R.flops.push_back(flops);
+  R.kind.push_back(kind);
   return r;
 }
 
@@ -693,7 +699,7 @@ alexnet_status forward_bf16(alexnet* h, const bf16* x, int B, int dropout_mode, 
   }
   bf16* fout[2] = {h->f6, h->f7};
   for (int f = 0; f < 3; ++f) {
-    ALX_TRY(run_gemm(h, P->ff[f], P->fc_flops[f], s), "fc forward launch");
+    ALX_TRY(run_gemm(h, P->ff[f], P->fc_flops[f], s, 1), "fc forward launch");
     const float* bias = h->params + h->b_off[5 + f];
     if (f < 2)
       launch_fc_finalize(h->scratch, P->ff[f].args.splits, B, h->fc[f].Out, bias, 1, dropout_mode,
@@ -803,18 +809,18 @@ alexnet_status train_fc_part(alexnet* h, const bf16* x, const int32_t* labels, i
       ALX_TRY(cudaStreamWaitEvent(side, h->ev_fdz[f], 0), "fork");
       ws = side;
     }
-    ALX_TRY(run_gemm(h, P->fd[f], P->fc_flops[f], s), "fc dgrad launch");
+    ALX_TRY(run_gemm(h, P->fd[f], P->fc_flops[f], s, 1), "fc dgrad launch");
     if (side) ALX_TRY(cudaEventRecord(h->ev_fdg[f], s), "data gradient done");
     launch_dgrad_finalize(h->scratch, P->fd[f].args.splits, B, F.In, mask[f], dxo[f], s);
     if (h->grads_only) {
-      ALX_TRY(run_gemm(h, P->fwg[f], P->fc_flops[f], ws), "fc wgrad launch");
+      ALX_TRY(run_gemm(h, P->fwg[f], P->fc_flops[f], ws, 2), "fc wgrad launch");
     } else if (h->fc_fused) {
       // HBM-bound (the update moves 18 bytes per weight against 256 MMA
       // FLOPs): launched outside the per-GEMM tensor-roofline records
       if (side) ALX_TRY(cudaStreamWaitEvent(side, h->ev_fdg[f], 0), "update after dgrad");
       ALX_TRY(launch_any(P->fws[f], ws), "fc wgrad + update launch");
     } else {
-      ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s), "fc wgrad launch");
+      ALX_TRY(run_gemm(h, P->fw[f], P->fc_flops[f], s, 2), "fc wgrad launch");
       launch_sgd_dense(h->params + h->w_off[5 + f], h->vel + h->w_off[5 + f], h->scratch,
                        h->w_len[5 + f], h->wf[5 + f], gptr(h->w_off[5 + f]), h->hp, s);
     }
@@ -1491,6 +1497,20 @@ alexnet_status alexnet_stats_read(alexnet_t* h, alexnet_stats* out) {
   out->gemm_launches = R.gemm_launches;
   out->gemm_flops = R.gemm_flops;
   out->gemm_ms = ms;
+  return ALEXNET_OK;
+}
+
+alexnet_status alexnet_stats_launch(alexnet_t* h, int i, int* kind, double* flops, double* ms) {
+  if (!h || !kind || !flops || !ms || i < 0) return ALEXNET_ERR_INVALID_ARG;
+  if (!h->last_rec || static_cast<size_t>(i) >= h->last_rec->flops.size())
+    return ALEXNET_ERR_INVALID_ARG;
+  ALX_TRY(cudaStreamSynchronize(h->stats_stream), "stats_launch");
+  const alexnet::StepRec& R = *h->last_rec;
+  float t = 0.f;
+  ALX_TRY(cudaEventElapsedTime(&t, R.ev[2 * i], R.ev[2 * i + 1]), "stats_launch");
+  *kind = R.kind[i];
+  *flops = R.flops[i];
+  *ms = t;
   return ALEXNET_OK;
 }
 

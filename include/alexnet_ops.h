@@ -247,6 +247,15 @@ typedef struct {
 ALEXNET_API alexnet_status alexnet_stats_enable(alexnet_t* h, int enable);
 ALEXNET_API alexnet_status alexnet_stats_read(alexnet_t* h, alexnet_stats* out);
 
+/* The i-th GEMM launch (launch order, 0 <= i < gemm_launches) of the call
+ * alexnet_stats_read reports: *kind 0 = a convolution (forward, data or
+ * weight gradient), 1 = an FC forward or data gradient, 2 = an FC weight
+ * gradient written to memory; *flops its algorithmic FLOPs; *ms its device
+ * time.  Synchronises that call's stream; ALEXNET_ERR_INVALID_ARG past the
+ * last launch. */
+ALEXNET_API alexnet_status alexnet_stats_launch(alexnet_t* h, int i, int* kind, double* flops,
+                                               double* ms);
+
 #ifdef __cplusplus
 }
 #endif
