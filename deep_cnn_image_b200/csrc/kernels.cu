@@ -980,7 +980,10 @@ __host__ __device__ inline PlbGeom plb_geom(int W, int Wo, int C) {
   return g;
 }
 
-template <int ZC, int WC, bool B34>
+// LRN = false: the same staged pool backward without a normalisation
+// between the conv output and the pool (pool5, and the pages' no-LRN
+// ablation): da = ReLU'(a) * (the routed pooled gradient).
+template <int ZC, int WC, bool B34, bool LRN = true>
 __global__ void __launch_bounds__(448, 2) k_pool_lrn_bwd_s(
     const bf16* __restrict__ dy, const uint8_t* __restrict__ am, const bf16* __restrict__ a,
     bf16* __restrict__ dl, bf16* __restrict__ da, int B, int H_, int W_, int C, int z_, float k,
@@ -1089,12 +1092,14 @@ __global__ void __launch_bounds__(448, 2) k_pool_lrn_bwd_s(
         for (int q = 0; q < 6; ++q) P[q] = make_float2(0.f, 0.f);
         if (pv[d]) {
           const int o = h * G.rowA + iw * C + uj * 8;
-          float2 av[4];
-          unpack4x2(*reinterpret_cast<const uint4*>(SA + o), av);
+          if constexpr (LRN) {
+            float2 av[4];
+            unpack4x2(*reinterpret_cast<const uint4*>(SA + o), av);
 #pragma unroll
-          for (int m = 0; m < 4; ++m) P[1 + m] = av[m];
-          if (uj > 0) P[0] = bf2_to_f2(*reinterpret_cast<const uint32_t*>(SA + o - 2));
-          if (uj < CH - 1) P[5] = bf2_to_f2(*reinterpret_cast<const uint32_t*>(SA + o + 8));
+            for (int m = 0; m < 4; ++m) P[1 + m] = av[m];
+            if (uj > 0) P[0] = bf2_to_f2(*reinterpret_cast<const uint32_t*>(SA + o - 2));
+            if (uj < CH - 1) P[5] = bf2_to_f2(*reinterpret_cast<const uint32_t*>(SA + o + 8));
+          }
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             const int rr = h + 2 - 2 * (w >> 1), rc = d + 2 - 2 * (w & 1);
@@ -1111,18 +1116,26 @@ __global__ void __launch_bounds__(448, 2) k_pool_lrn_bwd_s(
                 dl + static_cast<uint32_t>((b * H + ih) * W + iw) * C + uj * 8) = gp;
           }
         }
-        float2 sq[6], S[4];
+        if constexpr (LRN) {
+          float2 sq[6], S[4];
 #pragma unroll
-        for (int q = 0; q < 6; ++q) sq[q] = __fmul2_rn(P[q], P[q]);
-        window5(sq, S);
+          for (int q = 0; q < 6; ++q) sq[q] = __fmul2_rn(P[q], P[q]);
+          window5(sq, S);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          float2 sb, sb1;
-          lrn_pow2x2<B34>(__ffma2_rn(alpha2, S[m], k2), beta, sb, sb1);
-          first[d][m] = __fmul2_rn(g[m], sb);
-          tv[d][m] = __fmul2_rn(__fmul2_rn(g[m], P[1 + m]), sb1);
+          for (int m = 0; m < 4; ++m) {
+            float2 sb, sb1;
+            lrn_pow2x2<B34>(__ffma2_rn(alpha2, S[m], k2), beta, sb, sb1);
+            first[d][m] = __fmul2_rn(g[m], sb);
+            tv[d][m] = __fmul2_rn(__fmul2_rn(g[m], P[1 + m]), sb1);
+          }
+          tvs[d * nt + tid] = make_float4(tv[d][0].x, tv[d][0].y, tv[d][3].x, tv[d][3].y);
+        } else {
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            first[d][m] = g[m];
+            tv[d][m] = make_float2(0.f, 0.f);
+          }
         }
-        tvs[d * nt + tid] = make_float4(tv[d][0].x, tv[d][0].y, tv[d][3].x, tv[d][3].y);
       }
       __syncthreads();
       if (*abort_flag) break;
@@ -1130,20 +1143,25 @@ __global__ void __launch_bounds__(448, 2) k_pool_lrn_bwd_s(
       for (int d = 0; d < 2; ++d) {
         if (!pv[d]) continue;
         const int iw = 2 * qj + d;
-        const float4 L = uj > 0 ? tvs[d * nt + tid - 1] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 R = uj < CH - 1 ? tvs[d * nt + tid + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
-        float2 tp[6], cross[4], av[4];
+        float2 av[4], cross[4];
         unpack4x2(*reinterpret_cast<const uint4*>(SA + h * G.rowA + iw * C + uj * 8), av);
-        tp[0] = make_float2(L.z, L.w);
+        if constexpr (LRN) {
+          const float4 L = uj > 0 ? tvs[d * nt + tid - 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 R =
+              uj < CH - 1 ? tvs[d * nt + tid + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+          float2 tp[6];
+          tp[0] = make_float2(L.z, L.w);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) tp[1 + m] = tv[d][m];
-        tp[5] = make_float2(R.x, R.y);
-        window5(tp, cross);
+          for (int m = 0; m < 4; ++m) tp[1 + m] = tv[d][m];
+          tp[5] = make_float2(R.x, R.y);
+          window5(tp, cross);
+        }
         uint4 packed;
         uint32_t* pw = &packed.x;
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          const float2 dd = __ffma2_rn(mc2ab, __fmul2_rn(av[m], cross[m]), first[d][m]);
+          const float2 dd =
+              LRN ? __ffma2_rn(mc2ab, __fmul2_rn(av[m], cross[m]), first[d][m]) : first[d][m];
           pw[m] = f2_to_bf2(make_float2(av[m].x > 0.f ? dd.x : 0.f, av[m].y > 0.f ? dd.y : 0.f));
         }
         *reinterpret_cast<uint4*>(da + static_cast<uint32_t>((b * H + ih) * W + iw) * C +
@@ -2214,7 +2232,7 @@ void launch_pool_fwd(const bf16* x, bf16* y, uint8_t* am, int B, int H, int W, i
     k_pool_fwd<2><<<grid, 256, 0, s>>>(x, y, am, B, H, W, C, st);
   count_launch();
 }
-constexpr int kPoolBwdPartBlocks = 148 * 4;  // grid when the bias sums are produced
+constexpr int kPoolBwdPartBlocks = 148 * 8;  // grid when the bias sums are produced
 int pool_bwd_parts(int B, int H, int W, int C) {
   if (C < 8 || C % 8 || 256 % (C / 8)) return 0;
   const int g = grid_for(1LL * B * H * W * (C / 8), 256);
@@ -2381,6 +2399,26 @@ int launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* 
     b34 ? go(k_pool_lrn_bwd<0, 0, true>) : go(k_pool_lrn_bwd<0, 0, false>);
   count_launch();
   return blocks;
+}
+int launch_pool_relu_bwd_staged(const bf16* dy, const uint8_t* am, const bf16* a, bf16* da,
+                                int B, int H, int W, int C, int z, float* bias_part, int* status,
+                                cudaStream_t s) {
+  if (C % kSlab || C > 2048 || (z != 2 && z != 3) || H < z || W < z) return 0;
+  if (1LL * B * H * W * C >= (1LL << 31)) return 0;  // 32-bit element offsets
+  const uintptr_t vec = reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(a) |
+                        reinterpret_cast<uintptr_t>(da) | reinterpret_cast<uintptr_t>(am);
+  PlbCfg pc;
+  if ((vec & 15) || !pool_lrn_staged_cfg(B, H, W, C, z, &pc)) return 0;
+  int* st = status ? status : aux_status_word();
+  if (!st) return 0;
+  auto gs = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pc.smem);
+    kern<<<pc.blocks, pc.threads, pc.smem, s>>>(dy, am, a, nullptr, da, B, H, W, C, z, 0.f, 0.f,
+                                                0.f, pc.nst, bias_part, st);
+  };
+  gs(k_pool_lrn_bwd_s<0, 0, false, false>);
+  count_launch();
+  return pc.blocks;
 }
 void launch_pool_fwd_f32(const float* x, float* y, int B, int H, int W, int C, int z, int st,
                          cudaStream_t s) {

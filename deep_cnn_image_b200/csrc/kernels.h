@@ -95,6 +95,13 @@ bool launch_lrn_pool_fwd(const bf16* a, bf16* lo, bf16* y, uint8_t* am, int B, i
 int launch_pool_lrn_bwd(const bf16* dy, const uint8_t* am, const bf16* a, bf16* dl, bf16* da,
                         int B, int H, int W, int C, int z, float k, float alpha, float beta,
                         float* bias_part, int* status, cudaStream_t s);
+// The staged pool backward without a normalisation: da = ReLU'(a) * (dy
+// routed to the window choices of the stride-2 pool over a); bias column
+// sums as launch_pool_lrn_bwd.  Returns the bias partial rows, 0 if the
+// shape or the pointers do not suit it (the caller then uses launch_pool_bwd).
+int launch_pool_relu_bwd_staged(const bf16* dy, const uint8_t* am, const bf16* a, bf16* da,
+                                int B, int H, int W, int C, int z, float* bias_part, int* status,
+                                cudaStream_t s);
 // A device status word for single-op calls that have no workspace to hold
 // one (never cleared by the library; nullptr if it cannot be looked up).
 int* aux_status_word();

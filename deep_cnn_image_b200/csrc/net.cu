@@ -854,8 +854,12 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
   // conv5's bias column sums
   {
     const ConvL& L = h->conv[4];
-    const int parts = launch_pool_bwd(h->dp5, h->am[4], h->p[4], h->da[4], B, L.Ho, L.Ho, L.Cout,
-                                      cfg.pool_size, 2, 1, s, h->cpart + h->cpart_off[4]);
+    float* part = h->cpart + h->cpart_off[4];
+    int parts = launch_pool_relu_bwd_staged(h->dp5, h->am[4], h->a[4], h->da[4], B, L.Ho, L.Ho,
+                                            L.Cout, cfg.pool_size, part, h->status, s);
+    if (parts == 0)
+      parts = launch_pool_bwd(h->dp5, h->am[4], h->p[4], h->da[4], B, L.Ho, L.Ho, L.Cout,
+                              cfg.pool_size, 2, 1, s, part);
     if (parts > 0) {
       fused_bwd[4] = true;
       bias_parts[4] = parts;
@@ -896,8 +900,17 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
             launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->dl[l - 1], B, Q.Ho, Q.Ho,
                             Q.Cout, cfg.pool_size, 2, 0, s);
         } else {
-          launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->da[l - 1], B, Q.Ho, Q.Ho,
-                          Q.Cout, cfg.pool_size, 2, 1, s);
+          // pool + ReLU backward (the no-normalisation variant), with layer
+          // l-1's bias column sums where the staged kernel takes the shape
+          float* part = h->cpart + h->cpart_off[l - 1];
+          int rows = launch_pool_relu_bwd_staged(h->dp[l - 1], h->am[l - 1], h->a[l - 1],
+                                                 h->da[l - 1], B, Q.Ho, Q.Ho, Q.Cout,
+                                                 cfg.pool_size, part, h->status, s);
+          if (rows == 0)
+            rows = launch_pool_bwd(h->dp[l - 1], h->am[l - 1], h->p[l - 1], h->da[l - 1], B,
+                                   Q.Ho, Q.Ho, Q.Cout, cfg.pool_size, 2, 1, s, part);
+          fused_bwd[l - 1] = rows > 0;
+          if (rows > 0) bias_parts[l - 1] = rows;
         }
       }
     }
