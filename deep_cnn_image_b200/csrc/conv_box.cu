@@ -793,15 +793,17 @@ static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, in
   a.To_h = (nsub * 128) / a.Wb;
   if (a.To_h < 1) return false;
   if (a.To_h > a.Ho) a.To_h = a.Ho;
-  // rows the MMAs read: the last sub-tile's 128 rows at the largest shift
-  const int rows = nsub * 128 + (cs.K - 1) * (a.Wb + 1);
-  a.Hb = (rows + a.Wb - 1) / a.Wb;
-  if (a.Hb > 256) return false;
   a.tiles_img = (a.Ho + a.To_h - 1) / a.To_h;
   // swapped tiles multiply only the tile's positions, rounded up to 16 (N of
   // an M = 64 or 128 MMA): 208 of the 256 for a whole 13 x 15 box
   a.sw_n = (a.To_h * a.Wb + 15) / 16 * 16;
   if (a.sw_n > 256) a.sw_n = 256;
+  // rows the MMAs read: the last sub-tile's 128 rows (a swapped tile's sw_n
+  // rows) at the largest shift
+  const bool swapped = kind == 3 || kind == 4;
+  const int rows = (swapped ? a.sw_n : nsub * 128) + (cs.K - 1) * (a.Wb + 1);
+  a.Hb = (rows + a.Wb - 1) / a.Wb;
+  if (a.Hb > 256) return false;
   a.cpt = cs.P() / 64;
   {
     // K steps of 16 channels of the last chunk that can hold real channels;
@@ -828,11 +830,19 @@ static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, in
   d->a_bytes = ((a.Hb * a.Wb * 128) + 1023) / 1024 * 1024;
   d->b_bytes = bn * 128;
   d->stages_a = 2;
-  const int stg = (kind == 3 || kind == 4) ? kStageBytes : 0;
+  const int stg = swapped ? kStageBytes : 0;
   const int left = kSmemBudget - 1024 - kBarBytes - stg - 2 * d->a_bytes;
-  // two taps per weight stage (half the barrier round trips of the single
-  // issuing thread) while at least three stages fit
-  d->tps = (left / (2 * d->b_bytes) >= 3 && cs.K * cs.K > 1) ? 2 : 1;
+  // As few weight stages per input chunk as two stages in flight allow: each
+  // stage costs the MMA warp a fixed ~400 clocks of hand-over beside its
+  // MMAs (measured on B200: conv3's forward loop 83k / 65k / 57k clocks at
+  // one / two / three taps per stage), more than a deeper ring gains.  The
+  // taps are spread evenly over the stages (9 taps: 3 + 3 + 3, not 4 + 4 + 1).
+  const int taps = cs.K * cs.K;
+  int tmax = left / (2 * d->b_bytes);
+  if (tmax < 1) return false;
+  if (tmax > taps) tmax = taps;
+  const int nst = (taps + tmax - 1) / tmax;
+  d->tps = (taps + nst - 1) / nst;
   d->stages_b = left / (d->tps * d->b_bytes);
   if (d->stages_b > 8) d->stages_b = 8;
   if (d->stages_b < 2) return false;
