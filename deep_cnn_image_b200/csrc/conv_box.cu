@@ -58,8 +58,10 @@ __device__ __forceinline__ void zero_smem(uint8_t* p, int bytes) {
 // the B operand), so one MMA does BN x sw_n x 16 instead of two
 // 128 x BN x 16 ones; the accumulator holds channels in its lanes and
 // positions in its columns.  With M = 64, accumulator row r sits in lane
-// 32 * (r / 16) + r % 16.
-template <int BN, int NSUB, int BMN, int SW = 0>
+// 32 * (r / 16) + r % 16.  KT = 10 * K + taps per weight stage selects a copy
+// whose tap loop is unrolled for that kernel size and stage width (0: both
+// at run time).
+template <int BN, int NSUB, int BMN, int SW = 0, int KT = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_box_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ BoxArgs a, int stA, int stB, int a_bytes, int tps) {
@@ -192,6 +194,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t b_lo0 = static_cast<uint32_t>(bdesc0), b_hi = static_cast<uint32_t>(bdesc0 >> 32);
       const uint32_t a_units = static_cast<uint32_t>(a_bytes) >> 4;
       const uint32_t row_adv = static_cast<uint32_t>(a.Wb - a.K + 1) * 8;  // next kernel row
+      // unrolled taps: the box offset of each kernel row, 16-byte units
+      constexpr int KR = KT ? KT / 10 : 1;
+      uint32_t rowoff[KR];
+#pragma unroll
+      for (int kh = 0; kh < KR; ++kh) rowoff[kh] = static_cast<uint32_t>(kh * a.Wb) * 8;
       RingPos ra, rb;
       uint32_t tcount = 0;
       bool ok = true;
@@ -209,55 +216,82 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t abox = a_lo0 + s * a_units;
-          uint32_t shift = 0;  // (kh * Wb + kw) rows, in 16-byte units
-          int kw = 0;
-          for (int tap0 = 0; tap0 < taps; tap0 += tps, rb.next(stB)) {
-            const int sb = rb.slot;
-            const int n = min(tps, taps - tap0);
-            if (!mbar_wait(b_full + 8 * sb, rb.phase, a.status, abort_flag)) {
-              ok = false;
-              break;
+          // a last chunk of 48 real channels (conv1's space-to-depth input,
+          // conv2's 48 channels per group) skips the K step of zeros
+          const bool k3 = !BMN && ch == a.cpt - 1 && a.k16_last == 3;
+          // the MMAs of one tap: A / B at the tap's box shift and weight slab
+          auto issue = [&](uint32_t shift, uint32_t bj, uint32_t acc0) {
+            if (SW) {
+              // A = the tap's weight slab (K-major, or MN-major for the data
+              // gradient), B = the box at the tap's shift
+              if (k3)
+                tc_mma_k3<2, 2>(dbase, bj, b_hi, abox + shift, a_hi, IDESC, acc0);
+              else
+                tc_mma_k4<BMN ? 128 : 2, 2>(dbase, bj, b_hi, abox + shift, a_hi, IDESC, acc0);
+            } else if (NSUB == 2) {
+              // the two sub-tiles' accumulators alternate MMA by MMA
+              const uint32_t a0 = abox + shift, a1 = a0 + (128 * 128 / 16);
+              if (k3)
+                tc_mma_x2<2, 2, 3>(dbase, dbase + BN, a0, a1, a_hi, bj, b_hi, IDESC, acc0);
+              else
+                tc_mma_x2<2, BMN ? 128 : 2, 4>(dbase, dbase + BN, a0, a1, a_hi, bj, b_hi, IDESC,
+                                               acc0);
+            } else {
+              if (k3)
+                tc_mma_k3<2, 2>(dbase, abox + shift, a_hi, bj, b_hi, IDESC, acc0);
+              else
+                tc_mma_k4<2, BMN ? 128 : 2>(dbase, abox + shift, a_hi, bj, b_hi, IDESC, acc0);
             }
-            tc_fence_after();
-            const uint32_t bst = b_lo0 + sb * (b_stage >> 4);
-            // a last chunk of 48 real channels (conv1's space-to-depth input,
-            // conv2's 48 channels per group) skips the K step of zeros
-            const bool k3 = !BMN && ch == a.cpt - 1 && a.k16_last == 3;
-            for (int j = 0; j < n; ++j) {
-              const uint32_t acc0 = (ch == 0 && tap0 + j == 0) ? 0u : 1u;
-              const uint32_t bj = bst + j * (B_BYTES >> 4);
-              if (SW) {
-                // A = the tap's weight slab (K-major, or MN-major for the data
-                // gradient), B = the box at the tap's shift
-                if (k3)
-                  tc_mma_k3<2, 2>(dbase, bj, b_hi, abox + shift, a_hi, IDESC, acc0);
-                else
-                  tc_mma_k4<BMN ? 128 : 2, 2>(dbase, bj, b_hi, abox + shift, a_hi, IDESC, acc0);
-              } else if (NSUB == 2) {
-                // the two sub-tiles' accumulators alternate MMA by MMA: a
-                // 128-row MMA that accumulates into the tensor memory the
-                // previous one wrote waits for it, about 106 clocks for
-                // N <= 192 (measured), longer than the MMA itself
-                const uint32_t a0 = abox + shift, a1 = a0 + (128 * 128 / 16);
-                if (k3)
-                  tc_mma_x2<2, 2, 3>(dbase, dbase + BN, a0, a1, a_hi, bj, b_hi, IDESC, acc0);
-                else
-                  tc_mma_x2<2, BMN ? 128 : 2, 4>(dbase, dbase + BN, a0, a1, a_hi, bj, b_hi, IDESC,
-                                                 acc0);
-              } else {
-                if (k3)
-                  tc_mma_k3<2, 2>(dbase, abox + shift, a_hi, bj, b_hi, IDESC, acc0);
-                else
-                  tc_mma_k4<2, BMN ? 128 : 2>(dbase, abox + shift, a_hi, bj, b_hi, IDESC, acc0);
+          };
+          if constexpr (KT == 0) {
+            uint32_t shift = 0;  // (kh * Wb + kw) rows, in 16-byte units
+            int kw = 0;
+            for (int tap0 = 0; tap0 < taps; tap0 += tps, rb.next(stB)) {
+              const int sb = rb.slot;
+              const int n = min(tps, taps - tap0);
+              if (!mbar_wait(b_full + 8 * sb, rb.phase, a.status, abort_flag)) {
+                ok = false;
+                break;
               }
-              if (++kw == a.K) {
-                kw = 0;
-                shift += row_adv;
-              } else {
-                shift += 8;
+              tc_fence_after();
+              const uint32_t bst = b_lo0 + sb * (b_stage >> 4);
+              for (int j = 0; j < n; ++j) {
+                issue(shift, bst + j * (B_BYTES >> 4), (ch == 0 && tap0 + j == 0) ? 0u : 1u);
+                if (++kw == a.K) {
+                  kw = 0;
+                  shift += row_adv;
+                } else {
+                  shift += 8;
+                }
               }
+              tc_commit(b_empty + 8 * sb);
             }
-            tc_commit(b_empty + 8 * sb);
+          } else {
+            // K x K taps in stages of TP, unrolled: every tap's shift and
+            // slab offset is a constant plus its kernel row's offset, so the
+            // issuing thread spends its time on MMAs rather than on loop
+            // bookkeeping (each instruction of that single thread is on the
+            // critical path between two stages' MMAs)
+            constexpr int KK = KT / 10, TP = KT % 10, NT = KK * KK;
+#pragma unroll
+            for (int st = 0; st < (NT + TP - 1) / TP; ++st) {
+              const int sb = rb.slot;
+              if (!mbar_wait(b_full + 8 * sb, rb.phase, a.status, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t bst = b_lo0 + sb * (b_stage >> 4);
+#pragma unroll
+              for (int j = 0; j < TP; ++j) {
+                const int tap = st * TP + j;
+                if (tap < NT)
+                  issue(rowoff[tap / KK] + (tap % KK) * 8, bst + j * (B_BYTES >> 4),
+                        (tap == 0 && ch == 0) ? 0u : 1u);
+              }
+              tc_commit(b_empty + 8 * sb);
+              rb.next(stB);
+            }
           }
           if (!ok) break;
           tc_commit(a_empty + 8 * s);
@@ -653,10 +687,11 @@ struct Entry {
   int kind, bn, nsub;
   void* fn;
   bool attr;
+  int kt = 0;  // forward kinds: 10 * K + taps per stage of an unrolled copy, 0 = generic
 };
-template <int BN, int NSUB, int BMN = 0, int SW = 0>
+template <int BN, int NSUB, int BMN = 0, int SW = 0, int KT = 0>
 void* fwd_ptr() {
-  return reinterpret_cast<void*>(&conv_box_fwd<BN, NSUB, BMN, SW>);
+  return reinterpret_cast<void*>(&conv_box_fwd<BN, NSUB, BMN, SW, KT>);
 }
 template <int BN, int NPAIR>
 void* wgrad_ptr() {
@@ -675,11 +710,20 @@ Entry g_entries[] = {
     {1, 64, 4, wgrad_ptr<64, 4>(), false},  {1, 96, 2, wgrad_ptr<96, 2>(), false},
     {1, 128, 2, wgrad_ptr<128, 2>(), false},
     {1, 192, 1, wgrad_ptr<192, 1>(), false}, {1, 256, 1, wgrad_ptr<256, 1>(), false},
+    // unrolled copies for the network's 3 x 3 layers (conv3-5, in stages of
+    // three taps) with one accumulator per tile.  The two-sub-tile tiles
+    // (conv1, conv2, conv5's forward) stay generic: unrolled, their
+    // alternating MMA pairs measured slower on B200 (conv2 forward 75 ->
+    // 95 us, conv5 33 -> 35 us), where these gain 5-10%.
+    {3, 128, 2, fwd_ptr<128, 2, 0, 1, 33>(), false, 33},
+    {4, 128, 2, fwd_ptr<128, 2, 1, 1, 33>(), false, 33},
+    {0, 192, 1, fwd_ptr<192, 1, 0, 0, 33>(), false, 33},
+    {2, 192, 1, fwd_ptr<192, 1, 1, 0, 33>(), false, 33},
 };
 
-Entry* find_entry(int kind, int bn, int nsub) {
+Entry* find_entry(int kind, int bn, int nsub, int kt = 0) {
   for (auto& e : g_entries)
-    if (e.kind == kind && e.bn == bn && e.nsub == nsub) return &e;
+    if (e.kind == kind && e.bn == bn && e.nsub == nsub && e.kt == kt) return &e;
   return nullptr;
 }
 
@@ -963,7 +1007,10 @@ cudaError_t box_prepare() {
 }
 
 cudaError_t box_launch(const BoxDesc& d, cudaStream_t stream) {
-  Entry* e = find_entry(d.kind, d.bn, d.nsub);
+  Entry* e = nullptr;
+  if (d.kind != 1 && d.tps >= 1 && d.tps <= 9 && (d.args.K == 3 || d.args.K == 5))
+    e = find_entry(d.kind, d.bn, d.nsub, 10 * d.args.K + d.tps);
+  if (!e) e = find_entry(d.kind, d.bn, d.nsub);
   if (!e) return cudaErrorInvalidValue;
   if (!e->attr) {
     cudaError_t r =
