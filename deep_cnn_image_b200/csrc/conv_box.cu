@@ -6,10 +6,14 @@
 // pass"): a sum over the (kh, kw, cin) taps, here ordered chunk by chunk of
 // 64 input channels, tap by tap within a chunk.
 //
-// Both kernels are persistent (one 320-thread CTA per SM): warps 0-7 drain
+// Both kernels are persistent (one 352-thread CTA per SM): warps 0-7 drain
 // tensor memory (epilogue; warps w and w + 4 share TMEM lane quarter w and
 // split its 16-column chunks), warp 8 issues TMA loads, warp 9 issues
-// tcgen05 MMAs and owns the tensor memory.  Every mbarrier wait is bounded; on
+// tcgen05 MMAs and owns the tensor memory.  Where a tile has two independent
+// accumulators (two position sub-tiles, two tap pairs), warp 10 issues the
+// second one's MMAs: the per-stage hand-over of each issuing thread (about
+// 400 clocks of waits, fences, commits and loop control, measured on B200)
+// then runs in parallel instead of adding up in one thread.  Every mbarrier wait is bounded; on
 // expiry the kernel records a timeout in the status word and winds down.
 #include <cudaTypedefs.h>
 
@@ -23,7 +27,7 @@ namespace alx {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kSmemBudget = 227 * 1024;
 constexpr int kBarBytes = 3072;  // mbarriers, tmem slot, abort flag (first 512 B); staged bias
 constexpr int kMaxBias = (kBarBytes - 512) / 4;
@@ -92,18 +96,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // MMA warps: two where the tile's two sub-tile accumulators are separate
+  constexpr int NMW = (NSUB == 2 && !SW) ? 2 : 1;
   zero_smem(smem, stA * a_bytes);
   if (threadIdx.x == 0) {
     for (int s = 0; s < stA; ++s) {
       mbar_init(a_full + 8 * s, 1);
-      mbar_init(a_empty + 8 * s, 1);
+      mbar_init(a_empty + 8 * s, NMW);
     }
     for (int s = 0; s < stB; ++s) {
       mbar_init(b_full + 8 * s, 1);
-      mbar_init(b_empty + 8 * s, 1);
+      mbar_init(b_empty + 8 * s, NMW);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(acc_full + 8 * i, 1);
+      mbar_init(acc_full + 8 * i, NMW);
       mbar_init(acc_empty + 8 * i, 256);
     }
     *abort_flag = 0;
@@ -181,12 +187,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 9 || warp == 10) {
     // ---------------------------------------------------------------- MMA
     // Descriptors are built once and advanced by adding 16-byte units to
     // their start-address field: a single issuing thread cannot afford to
-    // rebuild two 64-bit descriptors per MMA.
-    if (lane == 0) {
+    // rebuild two 64-bit descriptors per MMA.  With two MMA warps, warp
+    // 9 + mw issues sub-tile mw's MMAs.
+    const int mw = warp - 9;
+    if (lane == 0 && mw < NMW) {
       const uint32_t IDESC = SW ? idesc_bf16(BN, a.sw_n, BMN, 0) : idesc_bf16(128, BN, 0, BMN);
       const uint64_t adesc0 = smem_desc_sw128(sA, 16, 1024);
       const uint64_t bdesc0 = BMN ? smem_desc_sw128(sB, 8192, 1024) : smem_desc_sw128(sB, 16, 1024);
@@ -229,13 +237,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               else
                 tc_mma_k4<BMN ? 128 : 2, 2>(dbase, bj, b_hi, abox + shift, a_hi, IDESC, acc0);
             } else if (NSUB == 2) {
-              // the two sub-tiles' accumulators alternate MMA by MMA
-              const uint32_t a0 = abox + shift, a1 = a0 + (128 * 128 / 16);
+              // this warp's sub-tile: rows 128 mw .. of the box, its own
+              // accumulator
+              const uint32_t am = abox + shift + mw * (128 * 128 / 16);
               if (k3)
-                tc_mma_x2<2, 2, 3>(dbase, dbase + BN, a0, a1, a_hi, bj, b_hi, IDESC, acc0);
+                tc_mma_k3<2, 2>(dbase + mw * BN, am, a_hi, bj, b_hi, IDESC, acc0);
               else
-                tc_mma_x2<2, BMN ? 128 : 2, 4>(dbase, dbase + BN, a0, a1, a_hi, bj, b_hi, IDESC,
-                                               acc0);
+                tc_mma_k4<2, BMN ? 128 : 2>(dbase + mw * BN, am, a_hi, bj, b_hi, IDESC, acc0);
             } else {
               if (k3)
                 tc_mma_k3<2, 2>(dbase, abox + shift, a_hi, bj, b_hi, IDESC, acc0);
@@ -472,6 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int TMEM_COLS = pow2_cols(2 * ACC_COLS);
   static_assert(2 * ACC_COLS <= 512, "two accumulator sets must fit in tensor memory");
   constexpr uint32_t IDESC = idesc_bf16(128, BN, 1, 1);
+  // MMA warps: with two tap pairs per item, warp 9 + j issues pair j
+  constexpr int NMW = NPAIR == 2 ? 2 : 1;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -496,10 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(full + 8 * s, 1);
-      mbar_init(empty + 8 * s, 1);
+      mbar_init(empty + 8 * s, NMW);
     }
     for (int q = 0; q < 2; ++q) {
-      mbar_init(acc_full + 8 * q, 1);
+      mbar_init(acc_full + 8 * q, NMW);
       mbar_init(acc_empty + 8 * q, 256);
     }
     *abort_flag = 0;
@@ -555,8 +565,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 9) {
-    if (lane == 0) {
+  } else if (warp == 9 || warp == 10) {
+    const int mw = warp - 9;
+    if (lane == 0 && mw < NMW) {
       // stage-relative descriptors plus the stage's start address: the
       // descriptor's start field is additive (16-byte units)
       const uint32_t sdesc0 = (s0 & 0x3FFFFu) >> 4;
@@ -605,12 +616,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st = sdesc0 + s * (stage_bytes >> 4);
           const uint32_t acc0 = p > p0 ? 1u : 0u;
           const uint32_t bl = st + y_lo;
-          if (NPAIR == 2 && nq == 2) {
-            // two tap pairs, two accumulators: alternate them MMA by MMA
-            const uint32_t al0 = st + pair_lo[0], al1 = st + pair_lo[NPAIR - 1];
-            for (int k = 0; k < ksteps; k += 4)
-              tc_mma_x2<128, 128, 4>(dacc, dacc + BN, al0 + k * 128, al1 + k * 128, pair_hi,
-                                     bl + k * 128, y_hi, IDESC, k == 0 ? acc0 : 1u);
+          if (NMW == 2) {
+            // this warp's tap pair (none if the item has one pair only)
+            if (mw < nq) {
+              const uint32_t al = st + (mw ? pair_lo[NPAIR - 1] : pair_lo[0]);
+              for (int k = 0; k < ksteps; k += 4)
+                tc_mma_k4<128, 128>(dacc + mw * BN, al + k * 128, pair_hi, bl + k * 128, y_hi,
+                                    IDESC, k == 0 ? acc0 : 1u);
+            }
           } else {
 #pragma unroll
             for (int j = 0; j < NPAIR; ++j) {
