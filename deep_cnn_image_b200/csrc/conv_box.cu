@@ -946,8 +946,8 @@ bool box_desc_wgrad(BoxDesc* d, const ConvShape& cs, const void* x, const void* 
     bn = 64;
   else if (cs.Og == 96)
     bn = 96;
-  else if (cs.Og == 192 || cs.Og == 384)
-    bn = 192;  // 384: two N = 192 tiles issue a third fewer MMAs than three of 128
+  else if (cs.Og == 192)
+    bn = 96;  // two tap pairs per item, one MMA warp each
   else if (cs.Og <= 128 || cs.Og % 128 == 0)
     bn = 128;
   else
