@@ -868,16 +868,17 @@ alexnet_status train_conv_part(alexnet* h, int B, cudaStream_t s, Plan* P) {
   for (int l = 4; l >= 0; --l) {
     const ConvL& L = h->conv[l];
     const long long rows = 1LL * B * L.Ho * L.Ho;
-    if (!fused_bwd[l]) {
-      launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart + h->cpart_off[l], s);
-      bias_parts[l] = colsum_chunks(rows);
-    }
-    // dY of layer l is complete: its weight gradient may start beside
+    // dY of layer l is complete: its weight gradient (and, where no pool
+    // backward made them, its bias column sums) may start beside
     cudaStream_t ws = s;
     if (side) {
       ALX_TRY(cudaEventRecord(h->ev_dy[l], s), "fork");
       ALX_TRY(cudaStreamWaitEvent(side, h->ev_dy[l], 0), "fork");
       ws = side;
+    }
+    if (!fused_bwd[l]) {
+      launch_colsum_partial(h->da[l], rows, L.Cout, h->cpart + h->cpart_off[l], ws);
+      bias_parts[l] = colsum_chunks(rows);
     }
     if (l > 0) {
       ALX_TRY(run_gemm(h, P->cd[l], P->conv_flops[l], s), "conv dgrad launch");
