@@ -62,7 +62,13 @@ __device__ __forceinline__ void zero_smem(uint8_t* p, int bytes) {
 // the B operand), so one MMA does BN x sw_n x 16 instead of two
 // 128 x BN x 16 ones; the accumulator holds channels in its lanes and
 // positions in its columns.  With M = 64, accumulator row r sits in lane
-// 32 * (r / 16) + r % 16.  KT = 10 * K + taps per weight stage selects a copy
+// 32 * (r / 16) + r % 16.  SW = 2 (data gradient, at most 64 input
+// channels): M = 128 holds two taps of a kernel row, (kh, 2p) in rows 0-63
+// and (kh, 2p + 1) in rows 64-127 (the MN-major weight slabs one after the
+// other, the odd last tap beside a zero slab), both multiplied by the box at
+// the first tap's shift; the second tap's partial sum for position c then
+// sits in column c + 1, and the epilogue adds the two halves.  That halves
+// the MMAs an M = 64 tile needs for the same channels.  KT = 10 * K + taps per weight stage selects a copy
 // whose tap loop is unrolled for that kernel size and stage width (0: both
 // at run time).
 template <int BN, int NSUB, int BMN, int SW = 0, int KT = 0>
@@ -76,13 +82,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   static_assert(!BMN || BN % 64 == 0, "MN-major weights come in 64-channel blocks");
   static_assert(!SW || (NSUB == 2 && (BN == 128 || (BN == 64 && BMN))),
                 "swapped tiles: 128 (or 64 MN-major) channels x up to 256 positions");
+  static_assert(SW != 2 || (BN == 64 && BMN && KT == 0),
+                "tap pairs: 64-channel MN-major slabs, generic tap loop");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + stA * a_bytes;
-  const int b_stage = tps * B_BYTES;
+  // a tap-pair tile's stage is one kernel row, padded to an even number of
+  // slabs: the last odd tap pairs with a slab of zeros that no load writes
+  const int b_stage = (SW == 2 ? ((a.K + 1) & ~1) : tps) * B_BYTES;
   uint8_t* barp = smem + stA * a_bytes + stB * b_stage;
   const uint32_t a_full = smem_u32(barp);
   const uint32_t a_empty = a_full + 8 * stA;
@@ -98,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // MMA warps: two where the tile's two sub-tile accumulators are separate
   constexpr int NMW = (NSUB == 2 && !SW) ? 2 : 1;
-  zero_smem(smem, stA * a_bytes);
+  zero_smem(smem, stA * a_bytes + (SW == 2 ? stB * b_stage : 0));
   if (threadIdx.x == 0) {
     for (int s = 0; s < stA; ++s) {
       mbar_init(a_full + 8 * s, 1);
@@ -195,7 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 9 + mw issues sub-tile mw's MMAs.
     const int mw = warp - 9;
     if (lane == 0 && mw < NMW) {
-      const uint32_t IDESC = SW ? idesc_bf16(BN, a.sw_n, BMN, 0) : idesc_bf16(128, BN, 0, BMN);
+      const uint32_t IDESC = SW == 2 ? idesc_bf16(128, a.sw_n, 1, 0)
+                             : (SW ? idesc_bf16(BN, a.sw_n, BMN, 0) : idesc_bf16(128, BN, 0, BMN));
       const uint64_t adesc0 = smem_desc_sw128(sA, 16, 1024);
       const uint64_t bdesc0 = BMN ? smem_desc_sw128(sB, 8192, 1024) : smem_desc_sw128(sB, 16, 1024);
       const uint32_t a_lo0 = static_cast<uint32_t>(adesc0), a_hi = static_cast<uint32_t>(adesc0 >> 32);
@@ -263,13 +274,25 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               tc_fence_after();
               const uint32_t bst = b_lo0 + sb * (b_stage >> 4);
-              for (int j = 0; j < n; ++j) {
-                issue(shift, bst + j * (B_BYTES >> 4), (ch == 0 && tap0 + j == 0) ? 0u : 1u);
-                if (++kw == a.K) {
-                  kw = 0;
-                  shift += row_adv;
-                } else {
-                  shift += 8;
+              if constexpr (SW == 2) {
+                // one kernel row per stage (tap0 = kh * K): pair p = taps
+                // (kh, 2p) and (kh, 2p + 1) as the two 64-row halves of
+                // M (the descriptor's leading offset is one slab), both
+                // against the box at the first tap's shift
+                const uint32_t srow = static_cast<uint32_t>((tap0 / a.K) * a.Wb) * 8;
+                for (int p = 0; 2 * p < a.K; ++p)
+                  tc_mma_k4<128, 2>(dbase, bst + 2 * p * (B_BYTES >> 4), b_hi,
+                                    abox + srow + 16 * p, a_hi, IDESC,
+                                    (ch == 0 && tap0 == 0 && p == 0) ? 0u : 1u);
+              } else {
+                for (int j = 0; j < n; ++j) {
+                  issue(shift, bst + j * (B_BYTES >> 4), (ch == 0 && tap0 + j == 0) ? 0u : 1u);
+                  if (++kw == a.K) {
+                    kw = 0;
+                    shift += row_adv;
+                  } else {
+                    shift += 8;
+                  }
                 }
               }
               tc_commit(b_empty + 8 * sb);
@@ -323,10 +346,77 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int oh0 = ti * a.To_h;
       const int acc = ACC_BUFS == 2 ? (tcount & 1) : 0;
       const uint32_t aph = ACC_BUFS == 2 ? ((tcount >> 1) & 1) : (tcount & 1);
-      if (!mbar_wait(acc_full + 8 * acc, aph, a.status, abort_flag)) break;
+      // (a tap-pair tile's warps meet at named barriers, so every warp runs
+      // every tile even after a timeout; it only stops storing)
+      const bool got = mbar_wait(acc_full + 8 * acc, aph, a.status, abort_flag);
+      if (!got && SW != 2) break;
       tc_fence_after();
       const int quarter = warp & 3, half = warp >> 2;
-      if constexpr (SW) {
+      if constexpr (SW == 2) {
+        // TMEM lanes 0-63 hold taps (kh, 2p) summed over p: input channel
+        // = lane, column = position.  Lanes 64-127 hold taps (kh, 2p + 1),
+        // read at the first tap's shift, so their column c belongs to
+        // position c - 1: dx[c] = low[c] + high[c + 1].  A high warp
+        // (quarter 2, 3) hands columns c0 + 1 .. c0 + 16 to the low warp
+        // of the same half (quarter 0, 1) through its staging area; the
+        // low warp adds, transposes through its own and stores 16-byte
+        // vectors of eight channels.
+        const bool high = quarter >= 2;
+        const uint32_t pair_bar = 1u + static_cast<uint32_t>(quarter & 1) + 2u * half;
+        float* U = reinterpret_cast<float*>(barp + kBarBytes + (warp | 2) * kStageWarp);
+        uint8_t* stg = barp + kBarBytes + warp * kStageWarp;
+        const int nw = (quarter & 1) * 32;  // the pair's first channel
+        const long long cg0 = static_cast<long long>(g) * a.col_goff + nw;
+        const uint32_t tb =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * ACC_COLS;
+#pragma unroll 1
+        for (int c0 = 128 * half; c0 < 128 * half + 128 && c0 < a.sw_n; c0 += 16) {
+          if (high) {
+            float v[32];
+            if (c0 + 32 <= ACC_COLS) {
+              tmem_ld32(tb + c0, v);
+            } else {
+              float w16[16];
+              tmem_ld16(tb + c0, w16);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = w16[e];
+#pragma unroll
+              for (int e = 16; e < 32; ++e) v[e] = 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) U[e * 32 + lane] = v[e + 1];
+            named_bar_sync(pair_bar, 64);  // handed over
+            named_bar_sync(pair_bar, 64);  // taken
+          } else {
+            float v[16];
+            tmem_ld16(tb + c0, v);
+            named_bar_sync(pair_bar, 64);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] += U[e * 32 + lane];
+            named_bar_sync(pair_bar, 64);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              reinterpret_cast<__nv_bfloat16*>(stg)[e * 32 + lane] = __float2bfloat16_rn(v[e]);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int j = lane + 32 * i;
+              const int e = j >> 2, part = j & 3;
+              const int c = c0 + e;
+              const int r = c / a.Wb;
+              const int col = c - r * a.Wb;
+              const int oh = oh0 + r;
+              if (got && r < a.To_h && oh < a.Ho && col < a.Wo && nw + part * 8 < a.Og) {
+                const uint4 val = *reinterpret_cast<const uint4*>(stg + e * 64 + part * 16);
+                *reinterpret_cast<uint4*>(
+                    out + ((static_cast<long long>(b) * a.Ho + oh) * a.Wo + col) * a.ld_out +
+                    cg0 + part * 8) = val;
+              }
+            }
+            __syncwarp();
+          }
+        }
+      } else if constexpr (SW) {
         // lane = output channel, columns = positions: this warp's CW = 32
         // (M = 64: 16) channels at the 128 positions of its half, 32
         // positions per chunk.  A chunk goes through the warp's staging
@@ -719,7 +809,7 @@ Entry g_entries[] = {
     {2, 256, 1, fwd_ptr<256, 1, 1>(), false}, {2, 192, 1, fwd_ptr<192, 1, 1>(), false},
     {0, 192, 1, fwd_ptr<192, 1>(), false},    {0, 256, 1, fwd_ptr<256, 1>(), false},
     {3, 128, 2, fwd_ptr<128, 2, 0, 1>(), false}, {4, 64, 2, fwd_ptr<64, 2, 1, 1>(), false},
-    {4, 128, 2, fwd_ptr<128, 2, 1, 1>(), false},
+    {4, 128, 2, fwd_ptr<128, 2, 1, 1>(), false}, {5, 64, 2, fwd_ptr<64, 2, 1, 2>(), false},
     {1, 64, 4, wgrad_ptr<64, 4>(), false},  {1, 96, 2, wgrad_ptr<96, 2>(), false},
     {1, 128, 2, wgrad_ptr<128, 2>(), false},
     {1, 192, 1, wgrad_ptr<192, 1>(), false}, {1, 256, 1, wgrad_ptr<256, 1>(), false},
@@ -822,7 +912,15 @@ bool box_desc_dgrad(BoxDesc* d, const ConvShape& cs, const void* dy, const void*
     bn = cs.Og <= 64 ? 64 : 128;
     nsub = 2;
   }
-  if (!box_fwd_common(d, cs, kind, bn, nsub, nullptr, 0, mask, dx, num_sms, status)) return false;
+  // at most 64 channels and a kernel of two taps or more: the tap-pair tile
+  // (two taps of a kernel row on M = 128 instead of one tap on M = 64, which
+  // costs the tensor pipe as much), where its stages fit
+  bool done = false;
+  if (kind == 4 && bn == 64 && cs.K >= 2)
+    done = box_fwd_common(d, cs, 5, 64, 2, nullptr, 0, mask, dx, num_sms, status);
+  if (!done &&
+      !box_fwd_common(d, cs, kind, bn, nsub, nullptr, 0, mask, dx, num_sms, status))
+    return false;
   d->args.w_og = cs.Cg;
   d->args.w_p = p_fwd;
   if (!dry) {
@@ -857,7 +955,7 @@ static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, in
   if (a.sw_n > 256) a.sw_n = 256;
   // rows the MMAs read: the last sub-tile's 128 rows (a swapped tile's sw_n
   // rows) at the largest shift
-  const bool swapped = kind == 3 || kind == 4;
+  const bool swapped = kind == 3 || kind == 4 || kind == 5;
   const int rows = (swapped ? a.sw_n : nsub * 128) + (cs.K - 1) * (a.Wb + 1);
   a.Hb = (rows + a.Wb - 1) / a.Wb;
   if (a.Hb > 256) return false;
@@ -895,15 +993,24 @@ static bool box_fwd_common(BoxDesc* d, const ConvShape& cs, int kind, int bn, in
   // one / two / three taps per stage), more than a deeper ring gains.  The
   // taps are spread evenly over the stages (9 taps: 3 + 3 + 3, not 4 + 4 + 1).
   const int taps = cs.K * cs.K;
-  int tmax = left / (2 * d->b_bytes);
-  if (tmax < 1) return false;
-  if (tmax > taps) tmax = taps;
-  const int nst = (taps + tmax - 1) / tmax;
-  d->tps = (taps + nst - 1) / nst;
-  d->stages_b = left / (d->tps * d->b_bytes);
+  // slabs per weight stage: the taps, or for a tap-pair tile one kernel row
+  // padded to an even count (the pad slab stays zero)
+  int slabs;
+  if (kind == 5) {
+    d->tps = cs.K;
+    slabs = (cs.K + 1) & ~1;
+  } else {
+    int tmax = left / (2 * d->b_bytes);
+    if (tmax < 1) return false;
+    if (tmax > taps) tmax = taps;
+    const int nst = (taps + tmax - 1) / tmax;
+    d->tps = (taps + nst - 1) / nst;
+    slabs = d->tps;
+  }
+  d->stages_b = left / (slabs * d->b_bytes);
   if (d->stages_b > 8) d->stages_b = 8;
   if (d->stages_b < 2) return false;
-  d->smem = 1024 + kBarBytes + stg + 2 * d->a_bytes + d->stages_b * d->tps * d->b_bytes;
+  d->smem = 1024 + kBarBytes + stg + 2 * d->a_bytes + d->stages_b * slabs * d->b_bytes;
   const long long tiles = 1LL * a.n_tiles * a.tiles_img * a.B * a.groups;
   d->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   return true;

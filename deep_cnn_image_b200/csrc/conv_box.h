@@ -65,7 +65,9 @@ struct BoxArgs {
 struct BoxDesc {
   // 0: forward / data gradient, 1: weight gradient, 2: data gradient from the
   // forward weights, 3: forward with swapped operands (M = 128 output channels,
-  // N = the tile's positions), 4: kind 2 swapped (M = 64 or 128 input channels)
+  // N = the tile's positions), 4: kind 2 swapped (M = 64 or 128 input channels),
+  // 5: kind 4 with two taps of a kernel row on M = 128 (64 input channels at
+  // most; a weight stage is one kernel row of 64-channel slabs)
   int kind;
   int bn;
   int nsub;  // forward: 128-row sub-tiles per tile; weight gradient: pairs per item

@@ -101,6 +101,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* st
   return mbar_wait_limit(bar, parity, status, abort_flag, WAIT_LIMIT_CYCLES);
 }
 
+// Named barrier `id` (1-15; 0 is __syncthreads) for `count` threads, a
+// multiple of 32: every warp that takes part reaches it the same number of
+// times.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Position in a ring of n pipeline stages: slot and the parity of the
 // slot's current phase, advanced without division.
 struct RingPos {
