@@ -50,7 +50,7 @@ METRIC = "images/sec, AlexNet bf16 train step, batch 128, 1×B200; % of bf16 ten
 # DRAM bytes (read + written) per batch-128 step of the GEMM class's 20
 # launches, summed from the per-launch ncu counters recorded in
 # profiles/train_step_counters_b128.md (None once those kernels change)
-GEMM_CLASS_TRAFFIC_BYTES = 810241536
+GEMM_CLASS_TRAFFIC_BYTES = 813034496
 UNIT = "images/s"
 WORKLOAD = "AlexNet (grouped conv2/4/5) bf16 training step: forward + backward + SGD-momentum, " \
            "227x227x3 NHWC inputs ~N(0,1), labels U[0,1000)"
