@@ -68,9 +68,9 @@ __device__ __forceinline__ void zero_smem(uint8_t* p, int bytes) {
 // other, the odd last tap beside a zero slab), both multiplied by the box at
 // the first tap's shift; the second tap's partial sum for position c then
 // sits in column c + 1, and the epilogue adds the two halves.  That halves
-// the MMAs an M = 64 tile needs for the same channels.  KT = 10 * K + taps per weight stage selects a copy
-// whose tap loop is unrolled for that kernel size and stage width (0: both
-// at run time).
+// the MMAs an M = 64 tile needs for the same channels.  KT = 10 * K + taps
+// per weight stage selects a copy whose tap loop is unrolled for that kernel
+// size and stage width (0: both at run time).
 template <int BN, int NSUB, int BMN, int SW = 0, int KT = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     conv_box_fwd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
