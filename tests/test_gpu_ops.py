@@ -310,6 +310,9 @@ CONVS = [  # (name, H, Cin, Cout, K, pad, groups, B)
     ("conv5", 13, 384, 256, 3, 1, 2, 3),
     ("conv5_ungrouped", 13, 384, 256, 3, 1, 1, 2),
     ("ragged_5x5", 20, 64, 128, 5, 2, 1, 2),
+    # 64 input channels per group and a 3 x 3 kernel: the data gradient's
+    # tap pairs with an odd last tap beside the zero slab in every row
+    ("pair_3x3", 15, 128, 128, 3, 1, 2, 2),
     ("one_by_one", 9, 32, 64, 1, 0, 1, 2),
     ("wide_im2col_fallback", 258, 64, 64, 3, 1, 1, 1),
 ]
